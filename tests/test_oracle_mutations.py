@@ -1,0 +1,118 @@
+"""Plant plausible mistakes in the oracle (CPU only) and check that the pins
+catch each one. A pin set that lets a mutation through would not pin much.
+"""
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as O
+import tests.test_oracle_pins as P
+
+PIN_TESTS = [
+    (P.test_e2m1_matches_generic_minifloat, {}),
+    (P.test_e8m0_scale_bias_and_nan, {}),
+    (P.test_mxfp4_nibble_order_and_group_axis, {}),
+    (P.test_router_bias_and_orientation, {}),
+    (P.test_all_ones_expert_closed_form, {}),
+    (P.test_gate_up_not_swapped_and_silu_sign, {}),
+    (P.test_down_projection_orientation, {}),
+    (P.test_weighted_combine_two_experts, {}),
+    (P.test_selected_softmax_properties, {}),
+    (P.test_routing_tables_match_stable_sort, {}),
+    (P.test_k_equals_E_is_dense_mixture, {}),
+]
+
+
+def _orig(name):
+    return getattr(O, name)
+
+
+def _mut_drop_bias(x, W_r, b_r):
+    return _orig_router(x, W_r, np.zeros_like(np.asarray(b_r, dtype=np.float64)))
+
+
+def _mut_softmax_all(s, idx):
+    full = np.exp(s - s.max(1, keepdims=True))
+    full /= full.sum(1, keepdims=True)
+    return np.take_along_axis(full, idx.astype(np.int64), 1)
+
+
+def _mut_swap_gate_up(xe, Wgu, I):
+    g = xe @ Wgu[:I].T
+    u = xe @ Wgu[I:].T
+    return g * O.silu(u)
+
+
+def _mut_nibble_order(codes, scales):
+    codes = np.asarray(codes, dtype=np.uint8)
+    sw = ((codes & 0x0F) << 4) | (codes >> 4)
+    return _orig_decode(sw.astype(np.uint8), scales)
+
+
+def _mut_scale_bias(scale):
+    return _orig_e8m0(np.asarray(scale).astype(np.int64) - 1)
+
+
+def _mut_silu_sign(z):
+    z = np.asarray(z, dtype=np.float64)
+    return z / (1.0 + np.exp(z))
+
+
+def _mut_down_transposed(h, Wd):
+    return h @ Wd.reshape(Wd.shape[1], Wd.shape[0]).T if Wd.shape[0] != Wd.shape[1] else h @ Wd
+
+
+def _mut_topk_high_index_ties(s, k):
+    s = np.asarray(s, dtype=np.float64)
+    T, E = s.shape
+    out = np.empty((T, k), dtype=np.int32)
+    for t in range(T):
+        order = np.lexsort((-np.arange(E), -s[t]))
+        out[t] = order[:k]
+    return out
+
+
+def _mut_unstable_tables(idx, E):
+    c, o, perm, inv = _orig_tables(idx, E)
+    perm = perm.copy()
+    for e in range(E):  # reverse the order inside each expert segment
+        perm[o[e]:o[e + 1]] = perm[o[e]:o[e + 1]][::-1]
+    inv = np.empty_like(perm)
+    inv[perm] = np.arange(perm.size, dtype=perm.dtype)
+    return c, o, perm, inv
+
+
+_orig_router = O.router_logits
+_orig_decode = O.mxfp4_decode
+_orig_e8m0 = O.e8m0_value
+_orig_tables = O.routing_tables
+
+MUTATIONS = {
+    "drop router bias": ("router_logits", _mut_drop_bias),
+    "softmax over all experts": ("selected_softmax", _mut_softmax_all),
+    "swap gate and up": ("expert_hidden", _mut_swap_gate_up),
+    "high nibble first": ("mxfp4_decode", _mut_nibble_order),
+    "scale bias off by one": ("e8m0_value", _mut_scale_bias),
+    "silu sign flipped": ("silu", _mut_silu_sign),
+    "down projection transposed": ("expert_out", _mut_down_transposed),
+    "ties to the higher index": ("topk_select", _mut_topk_high_index_ties),
+    "unstable grouping": ("routing_tables", _mut_unstable_tables),
+}
+
+
+@pytest.mark.parametrize("name", list(MUTATIONS))
+def test_pins_catch_mutation(name, monkeypatch, golden_dir):
+    attr, fn = MUTATIONS[name]
+    monkeypatch.setattr(O, attr, fn)
+    failures = 0
+    for test, kw in PIN_TESTS:
+        try:
+            test(**kw)
+        except Exception:
+            failures += 1
+    # the topk tie rule is pinned by the brute-force test
+    if name == "ties to the higher index":
+        try:
+            P.test_topk_brute_force(8, 2)
+        except Exception:
+            failures += 1
+    assert failures > 0, f"no pin caught the mutation '{name}'"
