@@ -1,0 +1,213 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) sparse-MoE layer forward pass.
+ *
+ * The layer is the gpt-oss-style Mixture-of-Experts feed-forward block:
+ *
+ *   s_e   = W_r[e] . x_t + b_r[e]                          (router logits)
+ *   S_t   = the k largest s_e (ties: lower expert index first)
+ *   p_j   = exp(s_j) / sum_{l in S_t} exp(s_l)             (softmax over S_t)
+ *   E_e(x)= W_down[e] (silu(W_gate[e] x) * (W_up[e] x))    (SwiGLU expert)
+ *   out_t = sum_{j in S_t} p_j E_j(x_t)
+ *
+ * Sources: "llm-surgery-dark-arts-gpt-oss-40b-64a8-init", section 2, "Proof"
+ * (the forward pass, the router logits and the softmax over the selected set);
+ * field guide "gpt-oss 20B", "03 Sparse Mixture of Experts" (score all experts,
+ * keep the top k, normalise those scores, weighted sum of SwiGLU experts);
+ * "gpt-oss-20b and gpt-oss-120b", "Four-bit expert weights" (MXFP4 experts,
+ * 4.25 bits per parameter); "shrink/gpt_oss-mic", "Preserved properties"
+ * (hidden_act silu).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named *_dev are CUDA device pointers; *_host are host pointers.
+ *   Every device pointer must be 16-byte aligned. Inputs are read-only.
+ * - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *   stream). All device work is enqueued on it; no entry point synchronises
+ *   the stream except moe_forward_hostio and moe_sync_status, which say so.
+ * - The library allocates no device memory. The caller owns every buffer,
+ *   including the workspace, whose size moe_workspace_size() returns.
+ *   Concurrent calls must not share a workspace.
+ * - Errors are returned as moe_status; nothing is thrown or printed.
+ *   Arguments are checked before anything is launched; on an argument error
+ *   no work is enqueued. Device-side timeouts (a bounded wait in a kernel
+ *   that gave up) are recorded in a status word inside the workspace and
+ *   reported by moe_sync_status() or by the next call on that workspace.
+ *
+ * Data layout (row-major, C order)
+ * --------------------------------
+ *   x           [T][d]        bf16 (raw 16-bit patterns)
+ *   W_r         [E][d]        float32
+ *   b_r         [E]           float32
+ *   Wgu_codes   [E][2I][d/2]  uint8  MXFP4 E2M1 codes; rows 0..I-1 are the
+ *                                    gate projection, rows I..2I-1 the up
+ *                                    projection; byte b of a row holds
+ *                                    element 2b in its low nibble and
+ *                                    element 2b+1 in its high nibble
+ *   Wgu_scales  [E][2I][d/32] uint8  E8M0 scale 2^(S-127) of each group of
+ *                                    32 consecutive elements along d
+ *   Wd_codes    [E][d][I/2]   uint8  down projection codes (contraction on I)
+ *   Wd_scales   [E][d][I/32]  uint8
+ *   out         [T][d]        bf16
+ *   topk_idx    [T][k]        int32  experts of token t, logit descending,
+ *                                    then expert index ascending
+ *   topk_w      [T][k]        float32 selected-set softmax weights
+ *
+ * Supported range: 1 <= E <= 256, 1 <= k <= min(E, 32), T >= 0,
+ * d and I multiples of 32 with 32 <= d, I <= 16384. Decoded weight
+ * magnitudes must be below 2^128 (E8M0 bytes up to 252), the range bf16
+ * represents; within it every decoded weight is exact.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1,   /* null pointer, misaligned pointer, bad shape  */
+  MOE_ERR_UNSUPPORTED = 2,   /* shape outside the supported range            */
+  MOE_ERR_WORKSPACE = 3,     /* workspace missing or smaller than required   */
+  MOE_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed            */
+  MOE_ERR_TIMEOUT = 5,       /* a kernel's bounded wait expired              */
+  MOE_ERR_NO_DEVICE = 6      /* no sm_100 device is current                  */
+} moe_status;
+
+/* Human-readable name of a status code (static storage, never NULL). */
+MOE_API const char* moe_status_string(moe_status s);
+
+/* Library version as major*10000 + minor*100 + patch. */
+MOE_API int moe_version(void);
+
+/*
+ * Bytes of device workspace moe_forward needs for this shape (0 for invalid
+ * shapes). The workspace holds the router's logits and top-k, the routing
+ * tables, the permuted activations, the SwiGLU hidden rows H [T*k][I] bf16 and
+ * the weighted per-slot expert outputs [T*k][d] bf16.
+ */
+MOE_API size_t moe_workspace_size(int E, int k, int T, int d, int I);
+
+/*
+ * Forward pass of the MoE layer (the whole path: router, top-k, selected-set
+ * softmax, permutation, gate/up grouped GEMM with SwiGLU, down grouped GEMM
+ * with the weighted un-permute, and the per-token sum).
+ * "llm-surgery-dark-arts-gpt-oss-40b-64a8-init", section 2, "Proof".
+ *
+ * Writes out_dev [T][d] bf16 completely. Asynchronous on `stream`.
+ */
+MOE_API moe_status moe_forward(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
+                       const uint8_t* Wgu_codes_dev, const uint8_t* Wgu_scales_dev,
+                       const uint8_t* Wd_codes_dev, const uint8_t* Wd_scales_dev,
+                       int E, int k, int T, int d, int I, void* out_dev,
+                       void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/*
+ * Same as moe_forward, instrumented: records a CUDA event on `stream` before
+ * every kernel the pass launches and one after the last, waits for the last
+ * event, and writes to stage_ms_host[0..9] (host memory, 10 floats) the
+ * device time in milliseconds of each launch, in order -- router logits,
+ * top-k/softmax, expert histogram, scan, scatter, activation gather, gate/up
+ * GEMM + SwiGLU, down GEMM + weighted un-permute, per-token sum -- and in
+ * stage_ms_host[9] the span from the first launch to the end of the last.
+ * Blocks the calling thread until the pass has finished.
+ */
+MOE_API moe_status moe_forward_timed(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
+                                     const uint8_t* Wgu_codes_dev, const uint8_t* Wgu_scales_dev,
+                                     const uint8_t* Wd_codes_dev, const uint8_t* Wd_scales_dev,
+                                     int E, int k, int T, int d, int I, void* out_dev,
+                                     void* workspace_dev, size_t workspace_bytes, void* stream,
+                                     float* stage_ms_host);
+
+/*
+ * Same as moe_forward with the activations in host memory: copies x_host
+ * (T*d*2 bytes; pinned memory gives asynchronous copies) to the workspace,
+ * runs the forward pass and copies the result to out_host, then synchronises
+ * `stream`. Expert and router weights stay on the device (the layer's
+ * resident parameters). moe_workspace_size_hostio() gives the workspace size.
+ */
+MOE_API size_t moe_workspace_size_hostio(int E, int k, int T, int d, int I);
+MOE_API moe_status moe_forward_hostio(const void* x_host, const float* W_r_dev, const float* b_r_dev,
+                              const uint8_t* Wgu_codes_dev, const uint8_t* Wgu_scales_dev,
+                              const uint8_t* Wd_codes_dev, const uint8_t* Wd_scales_dev,
+                              int E, int k, int T, int d, int I, void* out_host,
+                              void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/*
+ * Router and permutation only (the first two steps of the path): router
+ * logits in fp32, top-k with the lower-index tie rule, selected-set softmax
+ * ("Proof", s_i and p_i), then the stable grouping of the T*k (token, slot)
+ * pairs by expert.
+ *
+ *   topk_idx_dev [T][k] int32, topk_w_dev [T][k] float32
+ *   counts_dev   [E]    int32  pairs routed to each expert
+ *   offsets_dev  [E+1]  int32  exclusive prefix sum of counts
+ *   perm_dev     [T*k]  int32  pair ids (t*k + j) grouped by expert, in
+ *                              ascending pair id inside each expert
+ * Any of counts/offsets/perm may be NULL to skip the permutation outputs
+ * (all three NULL, or none). workspace size: moe_route_workspace_size().
+ */
+MOE_API size_t moe_route_workspace_size(int E, int k, int T, int d);
+MOE_API moe_status moe_route(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
+                     int E, int k, int T, int d,
+                     int32_t* topk_idx_dev, float* topk_w_dev,
+                     int32_t* counts_dev, int32_t* offsets_dev, int32_t* perm_dev,
+                     void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/*
+ * Where moe_forward keeps its intermediates inside the workspace (byte
+ * offsets from the workspace base), so that a caller can read them after a
+ * call for inspection: logits [T][E] f32, topk_idx [T][k] i32, topk_w [T][k]
+ * f32, counts [E] i32, offsets [E+1] i32, perm [T*k] i32 (pair id at each
+ * permuted row), xp [T*k][d] bf16 (permuted activations), h [T*k][I] bf16
+ * (SwiGLU hidden rows in permuted order), yw [T*k][d] bf16 (p-weighted expert
+ * outputs in pair order t*k+j). Returns MOE_ERR_INVALID_ARG for bad shapes.
+ */
+typedef struct {
+  size_t logits, topk_idx, topk_w, counts, offsets, perm, xp, h, yw, status, total;
+} moe_ws_layout;
+MOE_API moe_status moe_workspace_layout(int E, int k, int T, int d, int I, moe_ws_layout* layout);
+
+/*
+ * Decode MXFP4 rows to bf16 on the device with the same decoder the grouped
+ * GEMMs use ("Four-bit expert weights"). codes_dev [rows][K/2], scales_dev
+ * [rows][K/32] -> out_dev [rows][K] bf16. K must be a multiple of 32.
+ */
+MOE_API moe_status moe_mxfp4_to_bf16(const uint8_t* codes_dev, const uint8_t* scales_dev,
+                             int rows, int K, void* out_dev, void* stream);
+
+/*
+ * Synchronise `stream`, then read and clear the device status word in the
+ * workspace. Returns MOE_OK, or MOE_ERR_TIMEOUT when a kernel gave up a wait.
+ */
+MOE_API moe_status moe_sync_status(void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/*
+ * Failure-detection self-test: enqueues one kernel whose only thread waits,
+ * with the same bounded wait the GEMM roles use, on an mbarrier that nothing
+ * completes. After about two seconds the wait gives up and stores
+ * MOE_ERR_TIMEOUT in the status word at the start of workspace_dev (16 bytes
+ * suffice), which moe_sync_status() then returns. Nothing hangs or faults.
+ */
+MOE_API moe_status moe_selftest_wait_timeout(void* workspace_dev, void* stream);
+
+/*
+ * Number of kernel launches one moe_forward call enqueues for this shape
+ * (0 for T = 0). Used to count device work per step.
+ */
+MOE_API int moe_forward_launch_count(int E, int k, int T, int d, int I);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

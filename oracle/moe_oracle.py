@@ -75,6 +75,12 @@ def e8m0_value(scale: np.ndarray) -> np.ndarray:
     return np.where(s == 255, np.nan, v)
 
 
+def _byte_table() -> np.ndarray:
+    """[256, 2] values of the two E2M1 codes in each byte (low nibble first)."""
+    b = np.arange(256, dtype=np.uint8)
+    return np.stack([e2m1_value(b & 0x0F), e2m1_value(b >> 4)], axis=1)
+
+
 def mxfp4_decode(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     """Decode packed MXFP4 rows to float64.
 
@@ -83,15 +89,13 @@ def mxfp4_decode(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
     Returns [..., K] float64: e2m1(code) * 2^(S-127), exact.
     """
     codes = np.asarray(codes, dtype=np.uint8)
-    lo = codes & 0x0F
-    hi = codes >> 4
-    nib = np.stack([lo, hi], axis=-1).reshape(*codes.shape[:-1], codes.shape[-1] * 2)
-    vals = e2m1_value(nib)
-    K = vals.shape[-1]
+    scales = np.asarray(scales, dtype=np.uint8)
+    K = codes.shape[-1] * 2
     if scales.shape[-1] * 32 != K:
         raise ValueError("scales must hold one byte per 32 elements")
-    sv = np.repeat(e8m0_value(scales), 32, axis=-1)
-    return vals * sv
+    vals = _byte_table()[codes].reshape(*codes.shape[:-1], K // 32, 32)
+    out = vals * e8m0_value(scales)[..., None]
+    return out.reshape(*codes.shape[:-1], K)
 
 
 def mxfp4_bits_per_param(group: int = 32, element_bits: int = 4,

@@ -1,0 +1,447 @@
+// moe_abi.cu -- the extern "C" boundary: argument checks, workspace layout,
+// and the launch sequence of the MoE forward pass on the caller's stream.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "../../include/moe_b200.h"
+#include "moe_internal.h"
+
+namespace {
+
+constexpr int kVersion = 100;  // 0.1.0
+constexpr int kMaxDevices = 64;
+
+size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+struct Layout {
+  moe_ws_layout pub;
+  size_t mprefix, chunk_hist, chunk_base, x_in, out_buf;
+};
+
+bool shape_ok(int E, int k, int T, int d) {
+  if (E < 1 || E > 256) return false;
+  if (k < 1 || k > E || k > 32) return false;
+  if (T < 0) return false;
+  if (d < 32 || d > 16384 || d % 32) return false;
+  if (static_cast<int64_t>(T) * k >= (static_cast<int64_t>(1) << 31)) return false;
+  return true;
+}
+
+bool full_shape_ok(int E, int k, int T, int d, int I) {
+  return shape_ok(E, k, T, d) && I >= 32 && I <= 16384 && I % 32 == 0;
+}
+
+void make_layout(int E, int k, int T, int d, int I, bool hostio, Layout* L) {
+  const size_t P = static_cast<size_t>(T) * k;
+  const size_t NB = static_cast<size_t>(moe::perm_chunks(T));
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + (bytes ? bytes : 1));
+    return o;
+  };
+  memset(L, 0, sizeof(*L));
+  L->pub.status = take(16);
+  L->pub.logits = take(static_cast<size_t>(T) * E * 4);
+  L->pub.topk_idx = take(P * 4);
+  L->pub.topk_w = take(P * 4);
+  L->pub.counts = take(static_cast<size_t>(E) * 4);
+  L->pub.offsets = take(static_cast<size_t>(E + 1) * 4);
+  L->mprefix = take(static_cast<size_t>(E + 1) * 4);
+  L->chunk_hist = take(NB * E * 4);
+  L->chunk_base = take(NB * E * 4);
+  L->pub.perm = take(P * 4);
+  L->pub.xp = take(P * d * 2);
+  L->pub.h = take(P * static_cast<size_t>(I) * 2);
+  L->pub.yw = take(P * d * 2);
+  if (hostio) {
+    L->x_in = take(static_cast<size_t>(T) * d * 2);
+    L->out_buf = take(static_cast<size_t>(T) * d * 2);
+  }
+  L->pub.total = off;
+}
+
+void make_route_layout(int E, int k, int T, int d, Layout* L) {
+  const size_t NB = static_cast<size_t>(moe::perm_chunks(T));
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align256(off + (bytes ? bytes : 1));
+    return o;
+  };
+  (void)k;
+  (void)d;
+  memset(L, 0, sizeof(*L));
+  L->pub.status = take(16);
+  L->pub.logits = take(static_cast<size_t>(T) * E * 4);
+  L->mprefix = take(static_cast<size_t>(E + 1) * 4);
+  L->chunk_hist = take(NB * E * 4);
+  L->chunk_base = take(NB * E * 4);
+  L->pub.offsets = take(static_cast<size_t>(E + 1) * 4);  // used when the caller passes none
+  L->pub.total = off;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Device capability and SM count, cached per device.
+moe_status device_info(int* num_sms) {
+  static int sms[kMaxDevices] = {0};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
+    cudaGetLastError();
+    return MOE_ERR_NO_DEVICE;
+  }
+  if (dev < kMaxDevices && sms[dev] > 0) {
+    *num_sms = sms[dev];
+    return MOE_OK;
+  }
+  int major = 0, minor = 0, n = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_NO_DEVICE;
+  }
+  if (major != 10 || minor != 0) return MOE_ERR_NO_DEVICE;  // built for sm_100a only
+  if (dev < kMaxDevices) sms[dev] = n;
+  *num_sms = n;
+  return MOE_OK;
+}
+
+#define MOE_CUDA(call)                        \
+  do {                                        \
+    if ((call) != cudaSuccess) {              \
+      cudaGetLastError();                     \
+      return MOE_ERR_CUDA;                    \
+    }                                         \
+  } while (0)
+
+template <class T>
+T* at(void* base, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(base) + off);
+}
+
+moe_status check_forward_args(const void* x, const float* W_r, const float* b_r,
+                              const uint8_t* gc, const uint8_t* gs, const uint8_t* dc,
+                              const uint8_t* ds, int E, int k, int T, int d, int I,
+                              const void* out, const void* ws) {
+  if (!x || !W_r || !b_r || !gc || !gs || !dc || !ds || !out || !ws) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || k < 1 || T < 0 || d < 1 || I < 1) return MOE_ERR_INVALID_ARG;
+  if (!full_shape_ok(E, k, T, d, I)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(W_r) || !aligned16(b_r) || !aligned16(gc) || !aligned16(gs) ||
+      !aligned16(dc) || !aligned16(ds) || !aligned16(out) || !aligned16(ws))
+    return MOE_ERR_INVALID_ARG;
+  return MOE_OK;
+}
+
+// Optional per-launch event recording (moe_forward_timed): ev[i] is recorded
+// before launch i, ev[kStages] after the last one.
+constexpr int kStages = 9;
+
+struct StageEvents {
+  cudaEvent_t ev[kStages + 1];
+  cudaStream_t st;
+  void mark(int i) const {
+    if (ev[0]) cudaEventRecord(ev[i], st);
+  }
+};
+
+moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, const uint8_t* gc,
+                       const uint8_t* gs, const uint8_t* dc, const uint8_t* ds, int E, int k,
+                       int T, int d, int I, uint16_t* out, void* ws, const Layout& L,
+                       cudaStream_t st, int num_sms, const StageEvents* tev = nullptr) {
+  StageEvents none;
+  memset(&none, 0, sizeof(none));
+  const StageEvents& E_ = tev ? *tev : none;
+  const int P = T * k;
+  const int NB = moe::perm_chunks(T);
+  int* status = at<int>(ws, L.pub.status);
+  float* logits = at<float>(ws, L.pub.logits);
+  int32_t* topk_idx = at<int32_t>(ws, L.pub.topk_idx);
+  float* topk_w = at<float>(ws, L.pub.topk_w);
+  int32_t* counts = at<int32_t>(ws, L.pub.counts);
+  int32_t* offsets = at<int32_t>(ws, L.pub.offsets);
+  int32_t* mprefix = at<int32_t>(ws, L.mprefix);
+  int32_t* chunk_hist = at<int32_t>(ws, L.chunk_hist);
+  int32_t* chunk_base = at<int32_t>(ws, L.chunk_base);
+  int32_t* perm = at<int32_t>(ws, L.pub.perm);
+  uint16_t* xp = at<uint16_t>(ws, L.pub.xp);
+  uint16_t* h = at<uint16_t>(ws, L.pub.h);
+  uint16_t* yw = at<uint16_t>(ws, L.pub.yw);
+
+  E_.mark(0);
+  MOE_CUDA(moe::launch_router_logits(x, W_r, b_r, logits, T, E, d, status, st));
+  E_.mark(1);
+  MOE_CUDA(moe::launch_topk_softmax(logits, T, E, k, topk_idx, topk_w, st));
+  E_.mark(2);
+  MOE_CUDA(moe::launch_perm_hist(topk_idx, T, k, E, chunk_hist, st));
+  E_.mark(3);
+  MOE_CUDA(moe::launch_perm_scan(chunk_hist, NB, E, counts, offsets, chunk_base, mprefix, st));
+  E_.mark(4);
+  MOE_CUDA(moe::launch_perm_scatter(topk_idx, T, k, E, chunk_base, perm, nullptr, st));
+  E_.mark(5);
+  MOE_CUDA(moe::launch_gather_rows(x, perm, P, k, d, xp, st));
+  E_.mark(6);
+
+  moe::GroupedGemmProblem g1;
+  g1.A = xp;
+  g1.codes = gc;
+  g1.scales = gs;
+  g1.offsets = offsets;
+  g1.mprefix = mprefix;
+  g1.P = P;
+  g1.E = E;
+  g1.K = d;
+  g1.Nrows = 2 * I;
+  g1.out = h;
+  g1.perm = nullptr;
+  g1.topk_w = nullptr;
+  g1.n_out = I;
+  g1.status = status;
+  MOE_CUDA(moe::launch_gemm_gateup_swiglu(g1, num_sms, st));
+  E_.mark(7);
+
+  moe::GroupedGemmProblem g2 = g1;
+  g2.A = h;
+  g2.codes = dc;
+  g2.scales = ds;
+  g2.K = I;
+  g2.Nrows = d;
+  g2.out = yw;
+  g2.perm = perm;
+  g2.topk_w = topk_w;
+  g2.n_out = d;
+  MOE_CUDA(moe::launch_gemm_down_combine(g2, num_sms, st));
+  E_.mark(8);
+  MOE_CUDA(moe::launch_combine(yw, T, k, d, out, st));
+  E_.mark(9);
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* moe_status_string(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT";
+    case MOE_ERR_NO_DEVICE: return "MOE_ERR_NO_DEVICE";
+  }
+  return "MOE_ERR_UNKNOWN";
+}
+
+int moe_version(void) { return kVersion; }
+
+size_t moe_workspace_size(int E, int k, int T, int d, int I) {
+  if (!full_shape_ok(E, k, T, d, I)) return 0;
+  Layout L;
+  make_layout(E, k, T, d, I, false, &L);
+  return L.pub.total;
+}
+
+size_t moe_workspace_size_hostio(int E, int k, int T, int d, int I) {
+  if (!full_shape_ok(E, k, T, d, I)) return 0;
+  Layout L;
+  make_layout(E, k, T, d, I, true, &L);
+  return L.pub.total;
+}
+
+moe_status moe_workspace_layout(int E, int k, int T, int d, int I, moe_ws_layout* layout) {
+  if (!layout || !full_shape_ok(E, k, T, d, I)) return MOE_ERR_INVALID_ARG;
+  Layout L;
+  make_layout(E, k, T, d, I, false, &L);
+  *layout = L.pub;
+  return MOE_OK;
+}
+
+int moe_forward_launch_count(int E, int k, int T, int d, int I) {
+  if (!full_shape_ok(E, k, T, d, I) || T == 0) return 0;
+  return 9;
+}
+
+moe_status moe_forward(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
+                       const uint8_t* Wgu_codes_dev, const uint8_t* Wgu_scales_dev,
+                       const uint8_t* Wd_codes_dev, const uint8_t* Wd_scales_dev, int E, int k,
+                       int T, int d, int I, void* out_dev, void* workspace_dev,
+                       size_t workspace_bytes, void* stream) {
+  moe_status s = check_forward_args(x_dev, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev,
+                                    Wd_codes_dev, Wd_scales_dev, E, k, T, d, I, out_dev,
+                                    workspace_dev);
+  if (s != MOE_OK) return s;
+  Layout L;
+  make_layout(E, k, T, d, I, false, &L);
+  if (workspace_bytes < L.pub.total) return MOE_ERR_WORKSPACE;
+  if (T == 0) return MOE_OK;
+  int num_sms = 0;
+  if ((s = device_info(&num_sms)) != MOE_OK) return s;
+  return run_forward(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, Wgu_codes_dev,
+                     Wgu_scales_dev, Wd_codes_dev, Wd_scales_dev, E, k, T, d, I,
+                     static_cast<uint16_t*>(out_dev), workspace_dev, L,
+                     static_cast<cudaStream_t>(stream), num_sms);
+}
+
+moe_status moe_forward_hostio(const void* x_host, const float* W_r_dev, const float* b_r_dev,
+                              const uint8_t* Wgu_codes_dev, const uint8_t* Wgu_scales_dev,
+                              const uint8_t* Wd_codes_dev, const uint8_t* Wd_scales_dev, int E,
+                              int k, int T, int d, int I, void* out_host, void* workspace_dev,
+                              size_t workspace_bytes, void* stream) {
+  moe_status s = check_forward_args(x_host, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev,
+                                    Wd_codes_dev, Wd_scales_dev, E, k, T, d, I, out_host,
+                                    workspace_dev);
+  if (s != MOE_OK) return s;
+  Layout L;
+  make_layout(E, k, T, d, I, true, &L);
+  if (workspace_bytes < L.pub.total) return MOE_ERR_WORKSPACE;
+  if (T == 0) return MOE_OK;
+  int num_sms = 0;
+  if ((s = device_info(&num_sms)) != MOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t bytes = static_cast<size_t>(T) * d * 2;
+  uint16_t* x_in = at<uint16_t>(workspace_dev, L.x_in);
+  uint16_t* out_buf = at<uint16_t>(workspace_dev, L.out_buf);
+  MOE_CUDA(cudaMemcpyAsync(x_in, x_host, bytes, cudaMemcpyHostToDevice, st));
+  s = run_forward(x_in, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev, Wd_codes_dev,
+                  Wd_scales_dev, E, k, T, d, I, out_buf, workspace_dev, L, st, num_sms);
+  if (s != MOE_OK) return s;
+  MOE_CUDA(cudaMemcpyAsync(out_host, out_buf, bytes, cudaMemcpyDeviceToHost, st));
+  MOE_CUDA(cudaStreamSynchronize(st));
+  int dev_status = 0;
+  MOE_CUDA(cudaMemcpy(&dev_status, at<int>(workspace_dev, L.pub.status), sizeof(int),
+                      cudaMemcpyDeviceToHost));
+  return dev_status ? static_cast<moe_status>(dev_status) : MOE_OK;
+}
+
+moe_status moe_forward_timed(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
+                             const uint8_t* Wgu_codes_dev, const uint8_t* Wgu_scales_dev,
+                             const uint8_t* Wd_codes_dev, const uint8_t* Wd_scales_dev, int E,
+                             int k, int T, int d, int I, void* out_dev, void* workspace_dev,
+                             size_t workspace_bytes, void* stream, float* stage_ms_host) {
+  if (!stage_ms_host) return MOE_ERR_INVALID_ARG;
+  moe_status s = check_forward_args(x_dev, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev,
+                                    Wd_codes_dev, Wd_scales_dev, E, k, T, d, I, out_dev,
+                                    workspace_dev);
+  if (s != MOE_OK) return s;
+  Layout L;
+  make_layout(E, k, T, d, I, false, &L);
+  if (workspace_bytes < L.pub.total) return MOE_ERR_WORKSPACE;
+  for (int i = 0; i <= kStages; ++i) stage_ms_host[i] = 0.f;
+  if (T == 0) return MOE_OK;
+  int num_sms = 0;
+  if ((s = device_info(&num_sms)) != MOE_OK) return s;
+  StageEvents tev;
+  tev.st = static_cast<cudaStream_t>(stream);
+  for (int i = 0; i <= kStages; ++i) tev.ev[i] = nullptr;
+  for (int i = 0; i <= kStages; ++i) {
+    if (cudaEventCreate(&tev.ev[i]) != cudaSuccess) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(tev.ev[j]);
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+  }
+  s = run_forward(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, Wgu_codes_dev,
+                  Wgu_scales_dev, Wd_codes_dev, Wd_scales_dev, E, k, T, d, I,
+                  static_cast<uint16_t*>(out_dev), workspace_dev, L, tev.st, num_sms, &tev);
+  if (s == MOE_OK && cudaEventSynchronize(tev.ev[kStages]) == cudaSuccess) {
+    for (int i = 0; i < kStages; ++i) cudaEventElapsedTime(&stage_ms_host[i], tev.ev[i], tev.ev[i + 1]);
+    cudaEventElapsedTime(&stage_ms_host[kStages], tev.ev[0], tev.ev[kStages]);
+  } else if (s == MOE_OK) {
+    s = MOE_ERR_CUDA;
+  }
+  for (int i = 0; i <= kStages; ++i) cudaEventDestroy(tev.ev[i]);
+  cudaGetLastError();
+  return s;
+}
+
+size_t moe_route_workspace_size(int E, int k, int T, int d) {
+  if (!shape_ok(E, k, T, d)) return 0;
+  Layout L;
+  make_route_layout(E, k, T, d, &L);
+  return L.pub.total;
+}
+
+moe_status moe_route(const void* x_dev, const float* W_r_dev, const float* b_r_dev, int E, int k,
+                     int T, int d, int32_t* topk_idx_dev, float* topk_w_dev, int32_t* counts_dev,
+                     int32_t* offsets_dev, int32_t* perm_dev, void* workspace_dev,
+                     size_t workspace_bytes, void* stream) {
+  if (!x_dev || !W_r_dev || !b_r_dev || !topk_idx_dev || !topk_w_dev || !workspace_dev)
+    return MOE_ERR_INVALID_ARG;
+  const int nperm = (counts_dev != nullptr) + (offsets_dev != nullptr) + (perm_dev != nullptr);
+  if (nperm != 0 && nperm != 3) return MOE_ERR_INVALID_ARG;
+  if (E < 1 || k < 1 || T < 0 || d < 1) return MOE_ERR_INVALID_ARG;
+  if (!shape_ok(E, k, T, d)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x_dev) || !aligned16(W_r_dev) || !aligned16(b_r_dev) ||
+      !aligned16(workspace_dev))
+    return MOE_ERR_INVALID_ARG;
+  Layout L;
+  make_route_layout(E, k, T, d, &L);
+  if (workspace_bytes < L.pub.total) return MOE_ERR_WORKSPACE;
+  if (T == 0) return MOE_OK;
+  int num_sms = 0;
+  moe_status s = device_info(&num_sms);
+  if (s != MOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int NB = moe::perm_chunks(T);
+  float* logits = at<float>(workspace_dev, L.pub.logits);
+  int* status = at<int>(workspace_dev, L.pub.status);
+  MOE_CUDA(moe::launch_router_logits(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, logits,
+                                     T, E, d, status, st));
+  MOE_CUDA(moe::launch_topk_softmax(logits, T, E, k, topk_idx_dev, topk_w_dev, st));
+  if (nperm == 3) {
+    int32_t* chunk_hist = at<int32_t>(workspace_dev, L.chunk_hist);
+    int32_t* chunk_base = at<int32_t>(workspace_dev, L.chunk_base);
+    int32_t* mprefix = at<int32_t>(workspace_dev, L.mprefix);
+    MOE_CUDA(moe::launch_perm_hist(topk_idx_dev, T, k, E, chunk_hist, st));
+    MOE_CUDA(moe::launch_perm_scan(chunk_hist, NB, E, counts_dev, offsets_dev, chunk_base,
+                                   mprefix, st));
+    MOE_CUDA(moe::launch_perm_scatter(topk_idx_dev, T, k, E, chunk_base, perm_dev, nullptr, st));
+  }
+  return MOE_OK;
+}
+
+moe_status moe_mxfp4_to_bf16(const uint8_t* codes_dev, const uint8_t* scales_dev, int rows, int K,
+                             void* out_dev, void* stream) {
+  if (!codes_dev || !scales_dev || !out_dev || rows < 0 || K < 32 || K % 32)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(codes_dev) || !aligned16(out_dev)) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  int num_sms = 0;
+  moe_status s = device_info(&num_sms);
+  if (s != MOE_OK) return s;
+  MOE_CUDA(moe::launch_mxfp4_to_bf16(codes_dev, scales_dev, rows, K,
+                                     static_cast<uint16_t*>(out_dev),
+                                     static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_sync_status(void* workspace_dev, size_t workspace_bytes, void* stream) {
+  if (!workspace_dev || workspace_bytes < 16) return MOE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int v = 0;
+  MOE_CUDA(cudaStreamSynchronize(st));
+  MOE_CUDA(cudaMemcpy(&v, workspace_dev, sizeof(int), cudaMemcpyDeviceToHost));
+  MOE_CUDA(cudaMemsetAsync(workspace_dev, 0, sizeof(int), st));
+  MOE_CUDA(cudaStreamSynchronize(st));
+  return v ? static_cast<moe_status>(v) : MOE_OK;
+}
+
+// Runs one bounded wait that nothing completes; on return the status word at
+// the start of `workspace_dev` holds MOE_ERR_TIMEOUT. Exercises the
+// failure-detection path of the kernels without hanging the device.
+moe_status moe_selftest_wait_timeout(void* workspace_dev, void* stream) {
+  if (!workspace_dev || !aligned16(workspace_dev)) return MOE_ERR_INVALID_ARG;
+  int num_sms = 0;
+  moe_status s = device_info(&num_sms);
+  if (s != MOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  MOE_CUDA(cudaMemsetAsync(workspace_dev, 0, sizeof(int), st));
+  MOE_CUDA(moe::launch_wait_timeout_selftest(static_cast<int*>(workspace_dev), st));
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,66 @@
+// moe_internal.h -- launchers shared between the C-ABI layer and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace moe {
+
+// Token chunk of the permutation kernels (tokens per block).
+constexpr int kPermChunk = 256;
+// Rows of one M tile of the grouped GEMMs.
+constexpr int kTileM = 128;
+
+inline int perm_chunks(int T) { return (T + kPermChunk - 1) / kPermChunk; }
+
+// K1: router logits s[t][e] = W_r[e] . x[t] + b_r[e] in fp32.
+cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, const float* b_r,
+                                 float* logits, int T, int E, int d, int* status_to_clear,
+                                 cudaStream_t st);
+// K1: top-k (lower index wins ties) and the selected-set softmax.
+cudaError_t launch_topk_softmax(const float* logits, int T, int E, int k, int32_t* topk_idx,
+                                float* topk_w, cudaStream_t st);
+// K2: per-chunk expert histograms.
+cudaError_t launch_perm_hist(const int32_t* topk_idx, int T, int k, int E, int32_t* chunk_hist,
+                             cudaStream_t st);
+// K2: counts, offsets, per-chunk bases and the M-tile prefix of each expert.
+cudaError_t launch_perm_scan(const int32_t* chunk_hist, int nchunks, int E, int32_t* counts,
+                             int32_t* offsets, int32_t* chunk_base, int32_t* mtile_prefix,
+                             cudaStream_t st);
+// K2: stable scatter of pair ids into expert-contiguous order.
+cudaError_t launch_perm_scatter(const int32_t* topk_idx, int T, int k, int E,
+                                const int32_t* chunk_base, int32_t* perm, int32_t* inv,
+                                cudaStream_t st);
+// K2: gather activation rows into permuted order.
+cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* perm, int P, int k, int d,
+                               uint16_t* xp, cudaStream_t st);
+// Per-token sum of the k weighted expert rows, rounded to bf16.
+cudaError_t launch_combine(const uint16_t* yw, int T, int k, int d, uint16_t* out,
+                           cudaStream_t st);
+// MXFP4 rows -> bf16 rows (same decoder as the GEMMs).
+cudaError_t launch_mxfp4_to_bf16(const uint8_t* codes, const uint8_t* scales, int rows, int K,
+                                 uint16_t* out, cudaStream_t st);
+
+// K3/K4: expert-grouped MXFP4 GEMMs on tcgen05.
+struct GroupedGemmProblem {
+  const uint16_t* A;        // [P][K] bf16 rows in permuted order
+  const uint8_t* codes;     // [E][Nrows][K/2]
+  const uint8_t* scales;    // [E][Nrows][K/32]
+  const int32_t* offsets;   // [E+1]
+  const int32_t* mprefix;   // [E+1] prefix of M tiles per expert
+  int P, E, K, Nrows;
+  uint16_t* out;            // H [P][I] (SwiGLU) or Yw [T*k][d] (down)
+  const int32_t* perm;      // down: pair id of each permuted row
+  const float* topk_w;      // down: weight of each pair
+  int n_out;                // output columns (I for SwiGLU, d for down)
+  int* status;
+};
+cudaError_t launch_gemm_gateup_swiglu(const GroupedGemmProblem& p, int num_sms, cudaStream_t st);
+cudaError_t launch_gemm_down_combine(const GroupedGemmProblem& p, int num_sms, cudaStream_t st);
+
+// Debug/self-test: one bounded wait on an mbarrier that nothing completes.
+cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t st);
+
+}  // namespace moe

@@ -1,0 +1,408 @@
+// moe_routing.cu -- router (logits, top-k, selected-set softmax), the stable
+// expert permutation, the activation gather and the per-token combine.
+//
+// Router: "llm-surgery-dark-arts-gpt-oss-40b-64a8-init", section 2, "Proof":
+// s_i = W_r[i] . h + b_r[i]; p_i = exp(s_i) / sum over the selected set.
+// Field guide "gpt-oss 20B", "03 Sparse Mixture of Experts": score all
+// experts, keep the top k, normalise only those.
+#include <cuda_bf16.h>
+#include <float.h>
+#include <stdint.h>
+
+#include "moe_internal.h"
+#include "moe_ptx.cuh"
+
+namespace moe {
+namespace {
+
+// ------------------------------------------------------------ K1 logits ----
+// Block tile: 32 tokens x 64 experts, contraction in chunks of 32; each of the
+// 128 threads owns 4 tokens x 4 experts. Every logit is one fp32 accumulator
+// updated by fma in increasing contraction index, then the bias is added:
+// identical router rows therefore give bit-identical logits.
+constexpr int RT_T = 32, RT_E = 64, RT_K = 32;
+
+__global__ void __launch_bounds__(128) router_logits_kernel(const uint16_t* __restrict__ x,
+                                                            const float* __restrict__ W_r,
+                                                            const float* __restrict__ b_r,
+                                                            float* __restrict__ logits, int T,
+                                                            int E, int d, int* status) {
+  __shared__ __align__(16) float xs[RT_K][RT_T + 4];
+  __shared__ __align__(16) float ws[RT_K][RT_E + 4];
+  const int tid = threadIdx.x;
+  if (status && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *status = 0;
+  const int t0 = blockIdx.x * RT_T, e0 = blockIdx.y * RT_E;
+  const int ty = tid >> 4, tx = tid & 15;
+  float acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+
+  for (int k0 = 0; k0 < d; k0 += RT_K) {
+    {  // activations: 32 tokens x 32 bf16, 16 bytes per thread
+      const int tt = tid >> 2, kk = (tid & 3) * 8, t = t0 + tt;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (t < T) v = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d + k0 + kk));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        xs[kk + 2 * i][tt] = __uint_as_float(w[i] << 16);
+        xs[kk + 2 * i + 1][tt] = __uint_as_float(w[i] & 0xFFFF0000u);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {  // router rows: 64 experts x 32 fp32
+      const int idx = tid + r * 128, ee = idx >> 3, kk = (idx & 7) * 4, e = e0 + ee;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e < E) v = __ldg(reinterpret_cast<const float4*>(W_r + (size_t)e * d + k0 + kk));
+      ws[kk + 0][ee] = v.x;
+      ws[kk + 1][ee] = v.y;
+      ws[kk + 2][ee] = v.z;
+      ws[kk + 3][ee] = v.w;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int kk = 0; kk < RT_K; ++kk) {
+      const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
+      const float4 b = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
+      const float av[4] = {a.x, a.y, a.z, a.w};
+      const float bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = t0 + ty * 4 + i;
+    if (t >= T) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + tx * 4 + j;
+      if (e < E) logits[(size_t)t * E + e] = acc[i][j] + b_r[e];
+    }
+  }
+}
+
+// ------------------------------------------------------ K1 top-k/softmax ----
+// One warp per token. Lane l holds the logits of experts l, l+32, ...; k rounds
+// of a warp arg-max on (logit descending, index ascending). Lane j keeps the
+// j-th winner; the softmax runs over the k winners only.
+__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits,
+                                                           int T, int E, int k,
+                                                           int32_t* __restrict__ topk_idx,
+                                                           float* __restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;
+  const float* s = logits + (size_t)t * E;
+  float v[8];
+  uint32_t taken = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = lane + 32 * j;
+    v[j] = (e < E) ? s[e] : -FLT_MAX;
+    if (e >= E) taken |= 1u << j;
+  }
+  int my_idx = 0;
+  float my_val = 0.f, top = 0.f;
+  for (int r = 0; r < k; ++r) {
+    float bv = 0.f;
+    int bi = 0x7FFFFFFF;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (taken & (1u << j)) continue;
+      const int e = lane + 32 * j;
+      if (bi == 0x7FFFFFFF || v[j] > bv || (v[j] == bv && e < bi)) {
+        bv = v[j];
+        bi = e;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
+      const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
+      const bool better = (bi == 0x7FFFFFFF) ||
+                          (oi != 0x7FFFFFFF && (ov > bv || (ov == bv && oi < bi)));
+      if (better) {
+        bv = ov;
+        bi = oi;
+      }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (r == 0) top = bv;
+    if (lane == r) {
+      my_idx = bi;
+      my_val = bv;
+    }
+  }
+  const float ex = (lane < k) ? expf(my_val - top) : 0.f;
+  float sum = ex;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
+  if (lane < k) {
+    topk_idx[(size_t)t * k + lane] = my_idx;
+    topk_w[(size_t)t * k + lane] = ex / sum;
+  }
+}
+
+// --------------------------------------------------------- K2 histogram ----
+__global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t* __restrict__ topk_idx,
+                                                        int T, int k, int E,
+                                                        int32_t* __restrict__ chunk_hist) {
+  __shared__ int h[256];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
+  __syncthreads();
+  const int64_t q0 = (int64_t)blockIdx.x * kPermChunk * k;
+  const int64_t q1 = (int64_t)min(T, (blockIdx.x + 1) * kPermChunk) * k;
+  for (int64_t q = q0 + threadIdx.x; q < q1; q += blockDim.x) atomicAdd(&h[topk_idx[q]], 1);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_hist[(size_t)blockIdx.x * E + e] = h[e];
+}
+
+// ------------------------------------------------------------- K2 scan ----
+// One block. Thread e walks the chunks of expert e; then a block-wide scan of
+// the expert counts gives the offsets and the M-tile prefix.
+__global__ void __launch_bounds__(256) perm_scan_kernel(const int32_t* __restrict__ chunk_hist,
+                                                        int nchunks, int E,
+                                                        int32_t* __restrict__ counts,
+                                                        int32_t* __restrict__ offsets,
+                                                        int32_t* __restrict__ chunk_base,
+                                                        int32_t* __restrict__ mtile_prefix) {
+  __shared__ int s_cnt[256], s_mt[256];
+  const int e = threadIdx.x;
+  int run = 0;
+  if (e < E) {
+    for (int b = 0; b < nchunks; ++b) {
+      const int c = chunk_hist[(size_t)b * E + e];
+      chunk_base[(size_t)b * E + e] = run;
+      run += c;
+    }
+  }
+  s_cnt[e] = (e < E) ? run : 0;
+  s_mt[e] = (e < E) ? (run + kTileM - 1) / kTileM : 0;
+  __syncthreads();
+  if (e == 0) {  // E <= 256: a serial scan is cheap and plainly ordered
+    int a = 0, m = 0;
+    for (int i = 0; i < E; ++i) {
+      const int c = s_cnt[i], mt = s_mt[i];
+      s_cnt[i] = a;
+      s_mt[i] = m;
+      a += c;
+      m += mt;
+    }
+    offsets[E] = a;
+    mtile_prefix[E] = m;
+  }
+  __syncthreads();
+  if (e < E) {
+    offsets[e] = s_cnt[e];
+    mtile_prefix[e] = s_mt[e];
+    if (counts) counts[e] = run;
+    for (int b = 0; b < nchunks; ++b) chunk_base[(size_t)b * E + e] += s_cnt[e];
+  }
+}
+
+// ---------------------------------------------------------- K2 scatter ----
+// Block b owns the pairs of token chunk b; warp w the w-th eighth of them, in
+// pair order. Pass 1 counts per (warp, expert); the per-warp bases follow
+// from the chunk base; pass 2 ranks pairs inside each 32-pair round with
+// match_any, so that the order inside an expert is ascending pair id.
+__global__ void __launch_bounds__(256) perm_scatter_kernel(const int32_t* __restrict__ topk_idx,
+                                                           int T, int k, int E,
+                                                           const int32_t* __restrict__ chunk_base,
+                                                           int32_t* __restrict__ perm,
+                                                           int32_t* __restrict__ inv) {
+  __shared__ int wbase[8][256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < 8 * 256; i += blockDim.x) (&wbase[0][0])[i] = 0;
+  __syncthreads();
+  const int64_t qc0 = (int64_t)blockIdx.x * kPermChunk * k;
+  const int64_t qc1 = (int64_t)min(T, (blockIdx.x + 1) * kPermChunk) * k;
+  const int64_t seg = (int64_t)(kPermChunk / 8) * k;
+  const int64_t q0 = qc0 + warp * seg;
+  const int64_t q1 = min(qc1, q0 + seg);
+  for (int64_t q = q0 + lane; q < q1; q += 32) atomicAdd(&wbase[warp][topk_idx[q]], 1);
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = chunk_base[(size_t)blockIdx.x * E + e];
+    for (int w = 0; w < 8; ++w) {
+      const int c = wbase[w][e];
+      wbase[w][e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int64_t qb = q0; qb < q1; qb += 32) {
+    const int64_t q = qb + lane;
+    const bool valid = q < q1;
+    const int e = valid ? topk_idx[q] : -1 - lane;
+    const uint32_t m = __match_any_sync(0xFFFFFFFFu, e);
+    const int rank = __popc(m & lt);
+    int pos = 0;
+    if (valid) pos = wbase[warp][e] + rank;
+    __syncwarp();
+    if (valid && lane == __ffs(m) - 1) wbase[warp][e] += __popc(m);
+    __syncwarp();
+    if (valid) {
+      perm[pos] = (int32_t)q;
+      if (inv) inv[q] = pos;
+    }
+  }
+}
+
+// ----------------------------------------------------------- K2 gather ----
+__global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x,
+                                                          const int32_t* __restrict__ perm, int P,
+                                                          int k, int d,
+                                                          uint16_t* __restrict__ xp) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  const int vec = d / 8;  // 16-byte vectors per row
+  for (int r = warp; r < P; r += nwarps) {
+    const int t = perm[r] / k;
+    const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
+    uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * d);
+    for (int c = lane; c < vec; c += 32) dst[c] = __ldg(src + c);
+  }
+}
+
+// ------------------------------------------------------------- combine ----
+// out[t] = sum_j yw[t*k + j], j ascending, fp32, rounded once to bf16.
+__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ yw, int T,
+                                                      int k, int d, uint16_t* __restrict__ out) {
+  const int vec = d / 8;
+  const int64_t n = (int64_t)T * vec;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t t = i / vec;
+    const int c = (int)(i % vec);
+    float acc[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) acc[u] = 0.f;
+    for (int j = 0; j < k; ++j) {
+      const uint4 v = __ldg(reinterpret_cast<const uint4*>(yw + ((size_t)t * k + j) * d) + c);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc[2 * u] += __uint_as_float(w[u] << 16);
+        acc[2 * u + 1] += __uint_as_float(w[u] & 0xFFFF0000u);
+      }
+    }
+    uint32_t o[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const __nv_bfloat162 h = __floats2bfloat162_rn(acc[2 * u], acc[2 * u + 1]);
+      o[u] = *reinterpret_cast<const uint32_t*>(&h);
+    }
+    reinterpret_cast<uint4*>(out + (size_t)t * d)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// ------------------------------------------------------- MXFP4 decode ----
+__global__ void __launch_bounds__(256) mxfp4_to_bf16_kernel(const uint8_t* __restrict__ codes,
+                                                            const uint8_t* __restrict__ scales,
+                                                            int rows, int K,
+                                                            uint16_t* __restrict__ out) {
+  const int groups = K / 32;
+  const int64_t n = (int64_t)rows * groups;
+  for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n;
+       g += (int64_t)gridDim.x * blockDim.x) {
+    const uint4 q = __ldg(reinterpret_cast<const uint4*>(codes) + g);
+    uint4 o[4];
+    mxfp4x32_to_bf16(q, scales[g], o);
+    uint4* dst = reinterpret_cast<uint4*>(out) + g * 4;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) dst[i] = o[i];
+  }
+}
+
+// --------------------------------------------------- timeout self-test ----
+// A bounded wait on a barrier whose phase never completes; the wait gives up
+// after kWaitLimitNs and records MOE_ERR_TIMEOUT in *status.
+__global__ void wait_timeout_selftest_kernel(int* status) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(smem_u32(&bar), 0, &abort_flag, status);
+}
+
+int grid_for(int64_t n, int per_block, int cap) {
+  int64_t b = (n + per_block - 1) / per_block;
+  if (b < 1) b = 1;
+  if (b > cap) b = cap;
+  return (int)b;
+}
+
+}  // namespace
+
+cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, const float* b_r,
+                                 float* logits, int T, int E, int d, int* status,
+                                 cudaStream_t st) {
+  dim3 grid((T + RT_T - 1) / RT_T, (E + RT_E - 1) / RT_E);
+  router_logits_kernel<<<grid, 128, 0, st>>>(x, W_r, b_r, logits, T, E, d, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_topk_softmax(const float* logits, int T, int E, int k, int32_t* topk_idx,
+                                float* topk_w, cudaStream_t st) {
+  topk_softmax_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, topk_idx, topk_w);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_perm_hist(const int32_t* topk_idx, int T, int k, int E, int32_t* chunk_hist,
+                             cudaStream_t st) {
+  perm_hist_kernel<<<perm_chunks(T), 256, 0, st>>>(topk_idx, T, k, E, chunk_hist);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_perm_scan(const int32_t* chunk_hist, int nchunks, int E, int32_t* counts,
+                             int32_t* offsets, int32_t* chunk_base, int32_t* mtile_prefix,
+                             cudaStream_t st) {
+  perm_scan_kernel<<<1, 256, 0, st>>>(chunk_hist, nchunks, E, counts, offsets, chunk_base,
+                                      mtile_prefix);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_perm_scatter(const int32_t* topk_idx, int T, int k, int E,
+                                const int32_t* chunk_base, int32_t* perm, int32_t* inv,
+                                cudaStream_t st) {
+  perm_scatter_kernel<<<perm_chunks(T), 256, 0, st>>>(topk_idx, T, k, E, chunk_base, perm, inv);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* perm, int P, int k, int d,
+                               uint16_t* xp, cudaStream_t st) {
+  gather_rows_kernel<<<grid_for(P, 8, 148 * 16), 256, 0, st>>>(x, perm, P, k, d, xp);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const uint16_t* yw, int T, int k, int d, uint16_t* out,
+                           cudaStream_t st) {
+  const int64_t n = (int64_t)T * (d / 8);
+  combine_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(yw, T, k, d, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mxfp4_to_bf16(const uint8_t* codes, const uint8_t* scales, int rows, int K,
+                                 uint16_t* out, cudaStream_t st) {
+  const int64_t n = (int64_t)rows * (K / 32);
+  mxfp4_to_bf16_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(codes, scales, rows, K, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t st) {
+  wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(status);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,88 @@
+"""The C-ABI library loads and exports every function include/moe_b200.h
+declares; host-side checks (sizes, argument validation) behave without a GPU.
+No compute call is made here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from sparse_moe_layer_05_b200 import binding as B
+from sparse_moe_layer_05_b200 import build as BUILD
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    BUILD.build()
+    return B.load()
+
+
+def declared_functions():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names |= set(re.findall(r"^MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src, re.M))
+    return sorted(names)
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 13
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(B.EXPORTS)
+
+
+def test_status_strings_and_version(lib):
+    assert lib.moe_status_string(0) == b"MOE_OK"
+    assert lib.moe_status_string(5) == b"MOE_ERR_TIMEOUT"
+    assert lib.moe_version() == 100
+
+
+def test_workspace_sizes():
+    assert B.moe_workspace_size(32, 4, 8192, 2880, 2880) > 8192 * 4 * 2880 * 2 * 3
+    assert B.moe_workspace_size(4, 2, 0, 64, 128) > 0
+    assert B.moe_workspace_size(0, 1, 8, 64, 64) == 0        # E < 1
+    assert B.moe_workspace_size(4, 5, 8, 64, 64) == 0        # k > E
+    assert B.moe_workspace_size(300, 4, 8, 64, 64) == 0      # E > 256
+    assert B.moe_workspace_size(64, 33, 8, 64, 64) == 0      # k > 32
+    assert B.moe_workspace_size(4, 2, 8, 48, 64) == 0        # d % 32
+    assert B.moe_workspace_size(4, 2, 8, 64, 40) == 0        # I % 32
+    assert B.moe_workspace_size_hostio(4, 2, 8, 64, 64) > B.moe_workspace_size(4, 2, 8, 64, 64)
+    L = B.moe_workspace_layout(32, 4, 100, 2880, 2880)
+    offs = sorted((v, k) for k, v in L.items() if k != "total")
+    assert all(v % 256 == 0 for v, _ in offs)
+    assert L["status"] == 0 and L["total"] >= L["yw"] + 400 * 2880 * 2
+    assert B.moe_forward_launch_count(32, 4, 100, 2880, 2880) == 9
+    assert B.moe_forward_launch_count(32, 4, 0, 2880, 2880) == 0
+
+
+def test_argument_errors_before_any_launch(lib):
+    vp = ctypes.c_void_p
+    good = 0x10000  # 16-byte aligned fake address; never dereferenced on error paths
+    args = [good] * 7 + [4, 2, 8, 64, 128, good, good, 1 << 30, None]
+    f = lib.moe_forward
+    a = list(args)
+    a[0] = None
+    assert f(*a) == 1                                   # null x
+    a = list(args)
+    a[3] = good + 4
+    assert f(*a) == 1                                   # misaligned codes
+    a = list(args)
+    a[10] = 48
+    assert f(*a) == 2                                   # d not a multiple of 32
+    a = list(args)
+    a[8] = 5
+    assert f(*a) == 2                                   # k > E
+    a = list(args)
+    a[14] = 16
+    assert f(*a) == 3                                   # workspace too small
+    a = list(args)
+    a[9] = 0
+    assert f(*a) == 0                                   # T = 0: nothing to do
+    r = lib.moe_route
+    assert r(good, good, good, 4, 2, 8, 64, good, good, good, None, None, good, 1 << 20, None) == 1
+    assert lib.moe_mxfp4_to_bf16(good, good, 4, 40, good, None) == 1
