@@ -1,0 +1,376 @@
+"""Benchmark of the MoE layer forward pass (B200, sm_100a).
+
+One step = one full forward pass of the layer (router, top-k, selected-set
+softmax, permutation, gate/up GEMM + SwiGLU, down GEMM + weighted un-permute,
+per-token sum) over one batch of synthetic tokens already resident in HBM.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload 20b]
+                    [--impl ours|reference]
+
+N > 1 is launched with torch.distributed.run (one rank per GPU); every rank
+runs its own batch through its own copy of the layer (weak scaling, no
+collective on the data path) and rank 0 prints one JSON line. The reference
+arm (--impl reference) times the CPU oracle on the host cores.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from sparse_moe_layer_05_b200 import workloads as W  # noqa: E402
+
+METRIC = "MoE-layer tokens/s"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DOMINANT_STAGE = "gemm_gateup_swiglu"
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+KERNEL_SOURCES = ["moe_grouped_gemm.cu", "moe_ptx.cuh"]
+
+
+# ------------------------------------------------------------ host logic ----
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def rank_token_order(T: int, rank: int) -> np.ndarray:
+    """Rows of the workload batch that rank `rank` processes (a seeded
+    permutation, so each rank has a batch of its own; rank 0 is the identity)."""
+    if rank == 0:
+        return np.arange(T)
+    return np.random.Generator(np.random.PCG64(1000 + rank)).permutation(T)
+
+
+def reduce_max(value: float, world: int) -> float:
+    """Maximum of `value` over all ranks (timing plumbing, not data path)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([value], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int) -> None:
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "sparse_moe_layer_05_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    with open(TRAFFIC_FILE) as f:
+        d = json.load(f)
+    ent = d.get(workload)
+    if not ent or ent.get("source_hash") != kernel_source_hash():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+def layer_flops(d, I, E, k, T) -> float:
+    return 6.0 * d * I * T * k + 2.0 * d * E * T
+
+
+def workload_config(inp, name: str) -> dict:
+    return {
+        "workload": f"{name} MoE layer forward: d={inp.d} I={inp.I} E={inp.E} k={inp.k} T={inp.T}",
+        "d": inp.d, "I": inp.I, "E": inp.E, "k": inp.k, "tokens_per_gpu": inp.T,
+        "weights": "MXFP4 (E2M1 codes, one E8M0 scale per 32 elements)",
+        "l2": "flushed between timed steps (256 MiB write, outside the step events)",
+        "parallelism": "token-parallel replicas (no collective on the data path)",
+    }
+
+
+# --------------------------------------------------------------- clocks ----
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int, path: str | None = None):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.path = path
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        self.lines = []
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                out, _ = self.proc.communicate(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+                out, _ = self.proc.communicate()
+            self.lines = [ln for ln in out.splitlines() if ln.strip()]
+            if self.path:
+                with open(self.path, "w") as f:
+                    f.write("\n".join(self.lines) + "\n")
+
+    def summary(self) -> dict:
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in getattr(self, "lines", []):
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- CPU legs ----
+
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return len(os.sched_getaffinity(0))
+
+
+def oracle_tokens_per_s(inp, tokens: np.ndarray):
+    from oracle import moe_oracle as O
+    t0 = time.perf_counter()
+    O.moe_forward(inp.x, inp.W_r, inp.b_r, inp.Wgu_codes, inp.Wgu_scales, inp.Wd_codes,
+                  inp.Wd_scales, k=inp.k, tokens=tokens)
+    dt = time.perf_counter() - t0
+    return len(tokens) / dt, dt
+
+
+def run_reference(args, inp, name):
+    """The reference arm: the CPU oracle, as it stands, on bounded samples."""
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return None
+    per_step = args.ref_tokens
+    times = []
+    for s in range(args.warmup + args.steps):
+        toks = (np.arange(per_step) + s * per_step) % inp.T
+        _, dt = oracle_tokens_per_s(inp, toks)
+        if s >= args.warmup:
+            times.append(dt)
+    total = sum(times)
+    value = per_step * len(times) / total
+    cores = blas_threads()
+    sample = (f"{per_step} tokens per step of the {inp.T}-token batch (the oracle decodes every "
+              f"expert those tokens select, then runs fp64 numpy matmuls)")
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "impl": "reference",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * total / len(times), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(inp, name),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+# ------------------------------------------------------------- GPU leg ----
+
+def run_ours(args, inp, name):
+    import torch
+    from sparse_moe_layer_05_b200 import binding as B
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    T = inp.T
+    order = rank_token_order(T, rank)
+    x_host = torch.from_numpy(np.ascontiguousarray(inp.x[order])).pin_memory()
+    x = x_host.to(dev)
+    layer = B.MoELayer(inp, device=dev, hostio=True)
+    out = torch.empty((T, inp.d), dtype=torch.uint16, device=dev)
+    out_host = torch.empty((T, inp.d), dtype=torch.uint16).pin_memory()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        layer.forward_timed(x, out)
+    torch.cuda.synchronize()
+    status = B.moe_sync_status(layer.workspace)
+    if status != 0:
+        raise RuntimeError(f"device status {B.STATUS.get(status, status)} after warm-up")
+
+    clocks_path = os.path.join(ROOT, "gpurun_out", "bench_clocks.csv") if os.path.isdir(
+        os.path.join(ROOT, "gpurun_out")) else None
+    stage_ms = []
+    barrier(world)
+    torch.cuda.synchronize()
+    with ClockSampler(local, clocks_path) as clk:
+        for _ in range(args.steps):
+            flush.zero_()
+            stage_ms.append(layer.forward_timed(x, out))
+        torch.cuda.synchronize()
+    barrier(world)
+    status = B.moe_sync_status(layer.workspace)
+    if status != 0:
+        raise RuntimeError(f"device status {B.STATUS.get(status, status)} in the timed region")
+    step_s = sum(s[9] for s in stage_ms) / 1e3
+    step_s_max = reduce_max(step_s, world)
+    tokens_all = T * args.steps * world
+    value = tokens_all / step_s_max
+    ms_per_step = 1e3 * step_s_max / args.steps
+
+    # dominant kernel: live CUDA-event durations of the gate/up GEMM launches
+    dom = B.STAGES.index(DOMINANT_STAGE)
+    dom_ms = sum(s[dom] for s in stage_ms) / len(stage_ms)
+    dom_flops = 4.0 * inp.d * inp.I * T * inp.k
+    peaks, kind = load_peaks()
+    peak = float(peaks["bf16_tflops"])
+    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+    stage_avg = {n: sum(s[i] for s in stage_ms) / len(stage_ms) for i, n in enumerate(B.STAGES)}
+
+    # end to end through the C ABI with host buffers: H2D + forward + D2H
+    e2e_s = 0.0
+    barrier(world)
+    torch.cuda.synchronize()
+    for _ in range(args.steps):
+        flush.zero_()
+        ev0 = torch.cuda.Event(enable_timing=True)
+        ev1 = torch.cuda.Event(enable_timing=True)
+        ev0.record(stream)
+        layer.forward_hostio(x_host, out_host)
+        ev1.record(stream)
+        ev1.synchronize()
+        e2e_s += ev0.elapsed_time(ev1) / 1e3
+    barrier(world)
+    e2e_s_max = reduce_max(e2e_s, world)
+    e2e_value = tokens_all / e2e_s_max
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(inp, name),
+        "layer_tflops": layer_flops(inp.d, inp.I, inp.E, inp.k, T) * args.steps * world
+        / step_s_max / 1e12,
+        "roofline": {
+            "bound": "tensor", "kernel": DOMINANT_STAGE, "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_source": f"bf16_tflops ({kind}, burst)",
+            "traffic": recorded_traffic(name),
+            "algorithmic_flops_per_launch": dom_flops,
+            "avg_launch_ms": dom_ms,
+        },
+        "stage_ms": stage_avg,
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(T * inp.d * 2),
+                "d2h_bytes_per_step": int(T * inp.d * 2)},
+        "gpu_launches": B.moe_forward_launch_count(inp.E, inp.k, T, inp.d, inp.I) * args.steps,
+        "clocks": clk.summary(),
+    }
+    return line
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="20b", choices=list(W.SHAPES))
+    ap.add_argument("--T", type=int, default=None, help="tokens per GPU (default: prefill T)")
+    ap.add_argument("--ref-tokens", type=int, default=2, help="oracle tokens per reference step")
+    ap.add_argument("--cpu-sample", type=int, default=256,
+                    help="tokens of the batch the oracle runs for cpu_baseline (0 = skip)")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be at least 3")
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        if world == 1 and args.gpus > 1:
+            ap.error("--gpus N > 1 must be launched with torch.distributed.run")
+    name = args.workload
+    inp = W.make_inputs(name, T=args.T)
+
+    if world > 1:
+        import torch.distributed as dist
+        backend = "gloo" if args.impl == "reference" else "nccl"
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=300))
+
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, inp, name)
+        else:
+            line = run_ours(args, inp, name)
+            if line is not None and rank == 0 and world == 1 and args.cpu_sample > 0:
+                n = min(args.cpu_sample, inp.T)
+                v, dt = oracle_tokens_per_s(inp, np.arange(n))
+                line["cpu_baseline"] = {
+                    "value": v, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                    "sample": f"first {n} tokens of the {inp.T}-token batch, {dt:.1f} s of "
+                              f"fp64 oracle work on the host"}
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -93,7 +93,7 @@ MOE_API int moe_version(void);
  * Bytes of device workspace moe_forward needs for this shape (0 for invalid
  * shapes). The workspace holds the router's logits and top-k, the routing
  * tables, the permuted activations, the SwiGLU hidden rows H [T*k][I] bf16 and
- * the weighted per-slot expert outputs [T*k][d] bf16.
+ * the weighted per-slot expert outputs [T*k][d] fp32.
  */
 MOE_API size_t moe_workspace_size(int E, int k, int T, int d, int I);
 
@@ -169,7 +169,7 @@ MOE_API moe_status moe_route(const void* x_dev, const float* W_r_dev, const floa
  * call for inspection: logits [T][E] f32, topk_idx [T][k] i32, topk_w [T][k]
  * f32, counts [E] i32, offsets [E+1] i32, perm [T*k] i32 (pair id at each
  * permuted row), xp [T*k][d] bf16 (permuted activations), h [T*k][I] bf16
- * (SwiGLU hidden rows in permuted order), yw [T*k][d] bf16 (p-weighted expert
+ * (SwiGLU hidden rows in permuted order), yw [T*k][d] fp32 (p-weighted expert
  * outputs in pair order t*k+j). Returns MOE_ERR_INVALID_ARG for bad shapes.
  */
 typedef struct {

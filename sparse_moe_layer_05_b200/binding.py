@@ -263,7 +263,7 @@ class MoELayer:
             "topk_w": (torch.float32, (T, self.k)), "counts": (torch.int32, (self.E,)),
             "offsets": (torch.int32, (self.E + 1,)), "perm": (torch.int32, (P,)),
             "xp": (torch.uint16, (P, self.d)), "h": (torch.uint16, (P, self.I)),
-            "yw": (torch.uint16, (P, self.d)),
+            "yw": (torch.float32, (P, self.d)),
         }[name]
         dt, shape = spec
         n = 1

@@ -54,7 +54,7 @@ void make_layout(int E, int k, int T, int d, int I, bool hostio, Layout* L) {
   L->pub.perm = take(P * 4);
   L->pub.xp = take(P * d * 2);
   L->pub.h = take(P * static_cast<size_t>(I) * 2);
-  L->pub.yw = take(P * d * 2);
+  L->pub.yw = take(P * d * 4);
   if (hostio) {
     L->x_in = take(static_cast<size_t>(T) * d * 2);
     L->out_buf = take(static_cast<size_t>(T) * d * 2);
@@ -168,7 +168,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   int32_t* perm = at<int32_t>(ws, L.pub.perm);
   uint16_t* xp = at<uint16_t>(ws, L.pub.xp);
   uint16_t* h = at<uint16_t>(ws, L.pub.h);
-  uint16_t* yw = at<uint16_t>(ws, L.pub.yw);
+  float* yw = at<float>(ws, L.pub.yw);
 
   E_.mark(0);
   MOE_CUDA(moe::launch_router_logits(x, W_r, b_r, logits, T, E, d, status, st));
@@ -195,6 +195,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   g1.K = d;
   g1.Nrows = 2 * I;
   g1.out = h;
+  g1.out_f32 = nullptr;
   g1.perm = nullptr;
   g1.topk_w = nullptr;
   g1.n_out = I;
@@ -208,7 +209,8 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   g2.scales = ds;
   g2.K = I;
   g2.Nrows = d;
-  g2.out = yw;
+  g2.out = nullptr;
+  g2.out_f32 = yw;
   g2.perm = perm;
   g2.topk_w = topk_w;
   g2.n_out = d;

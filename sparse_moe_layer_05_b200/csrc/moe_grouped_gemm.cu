@@ -69,6 +69,7 @@ struct Args {
   int half_off;     // row offset of the second box relative to the first
   int n_out;
   uint16_t* out;
+  float* out_f32;
   const int32_t* perm;
   const float* topk_w;
   int* status;
@@ -266,6 +267,8 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           }
         }
       } else {
+        // weighted un-permute: fp32 row p * y of pair perm[row], stored at
+        // yw[pair] so that the per-token sum reads k contiguous rows
         const int col0 = ti.nt * BN;
         int pair = 0;
         float w = 0.f;
@@ -273,25 +276,26 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           pair = args.perm[grow];
           w = args.topk_w[pair];
         }
-        uint16_t* orow = args.out + static_cast<int64_t>(pair) * args.n_out;
+        float* orow = args.out_f32 + static_cast<int64_t>(pair) * args.n_out;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 16) {
           uint32_t y[16];
           tmem_ld16(taddr + c, y);
           tmem_ld_wait();
-          uint32_t o[8];
+          float v[16];
 #pragma unroll
-          for (int i = 0; i < 8; ++i)
-            o[i] = pack_bf16x2(w * __uint_as_float(y[2 * i]), w * __uint_as_float(y[2 * i + 1]));
+          for (int i = 0; i < 16; ++i) v[i] = w * __uint_as_float(y[i]);
           const int col = col0 + c;
           if (valid) {
             if (col + 16 <= args.n_out) {
-              uint4* dst = reinterpret_cast<uint4*>(orow + col);
-              dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
-              dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
+              float4* dst = reinterpret_cast<float4*>(orow + col);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
             } else {
-              for (int i = 0; i < 16 && col + i < args.n_out; ++i)
-                orow[col + i] = static_cast<uint16_t>(o[i >> 1] >> (16 * (i & 1)));
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                if (col + i < args.n_out) orow[col + i] = v[i];
             }
           }
         }
@@ -428,6 +432,7 @@ cudaError_t launch_impl(const GroupedGemmProblem& p, int num_sms, cudaStream_t s
   a.Nrows = p.Nrows;
   a.n_out = p.n_out;
   a.out = p.out;
+  a.out_f32 = p.out_f32;
   a.perm = p.perm;
   a.topk_w = p.topk_w;
   a.status = p.status;

@@ -37,7 +37,7 @@ cudaError_t launch_perm_scatter(const int32_t* topk_idx, int T, int k, int E,
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* perm, int P, int k, int d,
                                uint16_t* xp, cudaStream_t st);
 // Per-token sum of the k weighted expert rows, rounded to bf16.
-cudaError_t launch_combine(const uint16_t* yw, int T, int k, int d, uint16_t* out,
+cudaError_t launch_combine(const float* yw, int T, int k, int d, uint16_t* out,
                            cudaStream_t st);
 // MXFP4 rows -> bf16 rows (same decoder as the GEMMs).
 cudaError_t launch_mxfp4_to_bf16(const uint8_t* codes, const uint8_t* scales, int rows, int K,
@@ -51,7 +51,8 @@ struct GroupedGemmProblem {
   const int32_t* offsets;   // [E+1]
   const int32_t* mprefix;   // [E+1] prefix of M tiles per expert
   int P, E, K, Nrows;
-  uint16_t* out;            // H [P][I] (SwiGLU) or Yw [T*k][d] (down)
+  uint16_t* out;            // SwiGLU: H [P][I] bf16
+  float* out_f32;           // down: Yw [T*k][d] fp32, row t*k+j = p_j * y
   const int32_t* perm;      // down: pair id of each permuted row
   const float* topk_w;      // down: weight of each pair
   int n_out;                // output columns (I for SwiGLU, d for down)

@@ -273,8 +273,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
 
 // ------------------------------------------------------------- combine ----
 // out[t] = sum_j yw[t*k + j], j ascending, fp32, rounded once to bf16.
-__global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict__ yw, int T,
-                                                      int k, int d, uint16_t* __restrict__ out) {
+__global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ yw, int T, int k,
+                                                      int d, uint16_t* __restrict__ out) {
   const int vec = d / 8;
   const int64_t n = (int64_t)T * vec;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
@@ -285,13 +285,10 @@ __global__ void __launch_bounds__(256) combine_kernel(const uint16_t* __restrict
 #pragma unroll
     for (int u = 0; u < 8; ++u) acc[u] = 0.f;
     for (int j = 0; j < k; ++j) {
-      const uint4 v = __ldg(reinterpret_cast<const uint4*>(yw + ((size_t)t * k + j) * d) + c);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        acc[2 * u] += __uint_as_float(w[u] << 16);
-        acc[2 * u + 1] += __uint_as_float(w[u] & 0xFFFF0000u);
-      }
+      const float4* src = reinterpret_cast<const float4*>(yw + ((size_t)t * k + j) * d) + 2 * c;
+      const float4 a = __ldg(src), b = __ldg(src + 1);
+      acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
+      acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
     }
     uint32_t o[4];
 #pragma unroll
@@ -386,7 +383,7 @@ cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* perm, int P, in
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const uint16_t* yw, int T, int k, int d, uint16_t* out,
+cudaError_t launch_combine(const float* yw, int T, int k, int d, uint16_t* out,
                            cudaStream_t st) {
   const int64_t n = (int64_t)T * (d / 8);
   combine_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(yw, T, k, d, out);

@@ -4,7 +4,8 @@ import numpy as np
 
 from oracle import moe_oracle as O
 
-TOL_REL_RMS = 2e-2       # max |err| <= 2e-2 * RMS(oracle out)
+TOL_REL_RMS = 2e-2       # |err| <= 2e-2 * RMS(oracle out) ...
+BF16_REL = 2.0 ** -8     # ... + the bf16 output's own rounding, 2^-8 |oracle value|
 NEAR_TIE = 1e-5          # k-th vs (k+1)-th oracle logit gap exempt from index parity
 
 
@@ -37,10 +38,19 @@ def rel_rms_err(got, want):
 
 
 def assert_out_close(got_u16, want, tol=TOL_REL_RMS, what="out"):
+    """Element-wise |got - want| <= tol * RMS(want) + 2^-8 |want|.
+
+    The second term is the rounding of the bf16 output format itself: the
+    exact result rounded to bf16 is off by up to 2^-8 |want|, which for
+    heavy-tailed outputs exceeds 2e-2 * RMS on its own."""
     got = bf16_to_f64(got_u16)
     assert np.all(np.isfinite(got)), f"{what}: non-finite values"
     r, rms, err = rel_rms_err(got, want)
-    assert r <= tol, f"{what}: max|err| {err:.3e} = {r:.3e} x RMS {rms:.3e} > {tol}"
+    bound = tol * rms + BF16_REL * np.abs(want)
+    excess = np.abs(got - want) / bound
+    assert np.all(excess <= 1.0), (
+        f"{what}: worst element uses {excess.max():.3f} of the bound "
+        f"(max|err| {err:.3e} = {r:.3e} x RMS {rms:.3e})")
     return r
 
 

@@ -148,8 +148,11 @@ def test_forward_matches_oracle(case):
         for e, (toks, h) in hidden.items():
             rows = H[o[e]:o[e + 1]]
             assert np.array_equal(perm[o[e]:o[e + 1]] // k, toks)
-            rr, rms, err = G.rel_rms_err(rows, h)
-            assert rr < 1e-2, (e, rr)
+            # H is stored in bf16: each element within one bf16 ulp of the
+            # fp64 value, plus a small allowance for fp32 accumulation
+            rms = np.sqrt(np.mean(h ** 2))
+            bound = 2.0 ** -8 * np.abs(h) + 1e-3 * rms
+            assert np.all(np.abs(rows - h) <= bound), (e, np.max(np.abs(rows - h) / (bound)))
 
 
 def test_forward_deterministic_and_hostio_equal():
