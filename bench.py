@@ -123,57 +123,89 @@ def workload_config(inp, name: str) -> dict:
 # --------------------------------------------------------------- clocks ----
 
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples the SM clock and the active clock-event (throttle) reasons of
+    one GPU every few milliseconds while the timed region runs. Read-only NVML
+    queries; nothing about the GPU is changed."""
 
-    def __init__(self, gpu_index: int, path: str | None = None):
-        self.gpu_index = gpu_index
-        self.proc = None
-        self.path = path
+    REASONS = {  # NVML clocks-event reason bits
+        "sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40,
+    }
+
+    def __init__(self, gpu_index: int, path: str | None = None, period_s: float = 0.005):
+        self.gpu_index, self.path, self.period = gpu_index, path, period_s
+        self.samples = []
+        self._stop = None
+        self._thread = None
+        self.sm_max = None
+
+    def _sample(self, nv, h):
+        sm = nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)
+        try:
+            rs = nv.nvmlDeviceGetCurrentClocksEventReasons(h)
+        except Exception:
+            rs = nv.nvmlDeviceGetCurrentClocksThrottleReasons(h)
+        try:
+            pw = nv.nvmlDeviceGetPowerUsage(h) / 1000.0
+        except Exception:
+            pw = None
+        self.samples.append((time.perf_counter(), sm, rs, pw))
 
     def __enter__(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
-                 "-lms", "200", "-i", str(self.gpu_index)],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-        except OSError:
-            self.proc = None
+            import pynvml as nv
+            nv.nvmlInit()
+            h = self._handle(nv)
+            self.sm_max = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+            self._sample(nv, h)  # one sample before the region starts
+        except Exception:
+            return self
+        self._stop = threading.Event()
+
+        def loop():
+            while not self._stop.is_set():
+                try:
+                    self._sample(nv, h)
+                except Exception:
+                    break
+                self._stop.wait(self.period)
+
+        self._thread = threading.Thread(target=loop, daemon=True)
+        self._thread.start()
         return self
 
+    def _handle(self, nv):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if self.gpu_index < len(ids):
+            tok = ids[self.gpu_index]
+            if tok.isdigit():
+                return nv.nvmlDeviceGetHandleByIndex(int(tok))
+            return nv.nvmlDeviceGetHandleByUUID(tok)
+        return nv.nvmlDeviceGetHandleByIndex(self.gpu_index)
+
     def __exit__(self, *a):
-        self.lines = []
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                out, _ = self.proc.communicate(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-                out, _ = self.proc.communicate()
-            self.lines = [ln for ln in out.splitlines() if ln.strip()]
-            if self.path:
-                with open(self.path, "w") as f:
-                    f.write("\n".join(self.lines) + "\n")
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join(timeout=2)
+        if self.path and self.samples:
+            with open(self.path, "w") as f:
+                f.write("t_s,sm_mhz,reasons_mask,power_w\n")
+                t0 = self.samples[0][0]
+                for t, sm, rs, pw in self.samples:
+                    f.write(f"{t - t0:.4f},{sm},{rs:#x},{pw}\n")
 
     def summary(self) -> dict:
-        sm, mx, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in getattr(self, "lines", []):
-            f = [x.strip() for x in ln.split(",")]
-            if len(f) < 9:
-                continue
-            try:
-                sm.append(float(f[1]))
-                mx.append(float(f[2]))
-            except ValueError:
-                continue
-            for n, v in zip(names, f[5:9]):
-                if v.lower() == "active":
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.sm_max, "reasons": [], "samples": 0}
+        reasons = set()
+        for _, _, rs, _ in self.samples:
+            for n, bit in self.REASONS.items():
+                if rs & bit:
                     reasons.add(n)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx),
+        sm = [x[1] for x in self.samples]
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": self.sm_max,
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
@@ -269,7 +301,7 @@ def run_ours(args, inp, name):
     status = B.moe_sync_status(layer.workspace)
     if status != 0:
         raise RuntimeError(f"device status {B.STATUS.get(status, status)} in the timed region")
-    step_s = sum(s[9] for s in stage_ms) / 1e3
+    step_s = sum(s[-1] for s in stage_ms) / 1e3
     step_s_max = reduce_max(step_s, world)
     tokens_all = T * args.steps * world
     value = tokens_all / step_s_max

@@ -114,11 +114,12 @@ MOE_API moe_status moe_forward(const void* x_dev, const float* W_r_dev, const fl
 /*
  * Same as moe_forward, instrumented: records a CUDA event on `stream` before
  * every kernel the pass launches and one after the last, waits for the last
- * event, and writes to stage_ms_host[0..9] (host memory, 10 floats) the
+ * event, and writes to stage_ms_host[0..11] (host memory, 12 floats) the
  * device time in milliseconds of each launch, in order -- router logits,
- * top-k/softmax, expert histogram, scan, scatter, activation gather, gate/up
- * GEMM + SwiGLU, down GEMM + weighted un-permute, per-token sum -- and in
- * stage_ms_host[9] the span from the first launch to the end of the last.
+ * top-k/softmax, expert histogram, scan, scatter, activation gather, the two
+ * scale transposes (gate/up, down), gate/up GEMM + SwiGLU, down GEMM +
+ * weighted un-permute, per-token sum -- and in stage_ms_host[11] the span
+ * from the first launch to the end of the last.
  * Blocks the calling thread until the pass has finished.
  */
 MOE_API moe_status moe_forward_timed(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
@@ -170,7 +171,9 @@ MOE_API moe_status moe_route(const void* x_dev, const float* W_r_dev, const floa
  * f32, counts [E] i32, offsets [E+1] i32, perm [T*k] i32 (pair id at each
  * permuted row), xp [T*k][d] bf16 (permuted activations), h [T*k][I] bf16
  * (SwiGLU hidden rows in permuted order), yw [T*k][d] fp32 (p-weighted expert
- * outputs in pair order t*k+j). Returns MOE_ERR_INVALID_ARG for bad shapes.
+ * outputs in pair order t*k+j). Rows of xp and h keep each run of 8
+ * consecutive elements in the order 0,4,1,5,2,6,3,7 (the operand order of the
+ * grouped GEMMs). Returns MOE_ERR_INVALID_ARG for bad shapes.
  */
 typedef struct {
   size_t logits, topk_idx, topk_w, counts, offsets, perm, xp, h, yw, status, total;

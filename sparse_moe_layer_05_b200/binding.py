@@ -32,7 +32,8 @@ EXPORTS = [
 ]
 
 STAGES = ["router_logits", "topk_softmax", "perm_hist", "perm_scan", "perm_scatter",
-          "gather_rows", "gemm_gateup_swiglu", "gemm_down_combine", "combine"]
+          "gather_rows", "transpose_scales_gu", "transpose_scales_d", "gemm_gateup_swiglu",
+          "gemm_down_combine", "combine"]
 
 
 class MoEError(RuntimeError):
@@ -157,10 +158,11 @@ def moe_forward(x, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, E, k, T
 
 def moe_forward_timed(x, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, E, k, T, d, I,
                       out, workspace, stream=None) -> list:
-    """Forward pass with per-launch CUDA-event timing; returns 10 floats (ms):
-    one per launch in the order of STAGES, then the whole span. Blocks."""
+    """Forward pass with per-launch CUDA-event timing; returns len(STAGES)+1
+    floats (ms): one per launch in the order of STAGES, then the whole span.
+    Blocks."""
     _require_cuda(x, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, out, workspace)
-    ms = (ctypes.c_float * 10)()
+    ms = (ctypes.c_float * (len(STAGES) + 1))()
     _check("moe_forward_timed", load().moe_forward_timed(
         _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(Wgu_codes), _ptr(Wgu_scales), _ptr(Wd_codes),
         _ptr(Wd_scales), E, k, T, d, I, _ptr(out), _ptr(workspace), workspace.numel(),

@@ -16,7 +16,7 @@ size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 struct Layout {
   moe_ws_layout pub;
-  size_t mprefix, chunk_hist, chunk_base, x_in, out_buf;
+  size_t mprefix, chunk_hist, chunk_base, x_in, out_buf, gu_scales_t, d_scales_t;
 };
 
 bool shape_ok(int E, int k, int T, int d) {
@@ -55,6 +55,8 @@ void make_layout(int E, int k, int T, int d, int I, bool hostio, Layout* L) {
   L->pub.xp = take(P * d * 2);
   L->pub.h = take(P * static_cast<size_t>(I) * 2);
   L->pub.yw = take(P * d * 4);
+  L->gu_scales_t = take(static_cast<size_t>(E) * 2 * I * (d / 32));
+  L->d_scales_t = take(static_cast<size_t>(E) * d * (I / 32));
   if (hostio) {
     L->x_in = take(static_cast<size_t>(T) * d * 2);
     L->out_buf = take(static_cast<size_t>(T) * d * 2);
@@ -137,7 +139,7 @@ moe_status check_forward_args(const void* x, const float* W_r, const float* b_r,
 
 // Optional per-launch event recording (moe_forward_timed): ev[i] is recorded
 // before launch i, ev[kStages] after the last one.
-constexpr int kStages = 9;
+constexpr int kStages = 11;
 
 struct StageEvents {
   cudaEvent_t ev[kStages + 1];
@@ -169,6 +171,8 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   uint16_t* xp = at<uint16_t>(ws, L.pub.xp);
   uint16_t* h = at<uint16_t>(ws, L.pub.h);
   float* yw = at<float>(ws, L.pub.yw);
+  uint8_t* gst = at<uint8_t>(ws, L.gu_scales_t);
+  uint8_t* dst_ = at<uint8_t>(ws, L.d_scales_t);
 
   E_.mark(0);
   MOE_CUDA(moe::launch_router_logits(x, W_r, b_r, logits, T, E, d, status, st));
@@ -183,11 +187,15 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   E_.mark(5);
   MOE_CUDA(moe::launch_gather_rows(x, perm, P, k, d, xp, st));
   E_.mark(6);
+  MOE_CUDA(moe::launch_transpose_scales(gs, E, 2 * I, d / 32, gst, st));
+  E_.mark(7);
+  MOE_CUDA(moe::launch_transpose_scales(ds, E, d, I / 32, dst_, st));
+  E_.mark(8);
 
   moe::GroupedGemmProblem g1;
   g1.A = xp;
   g1.codes = gc;
-  g1.scales = gs;
+  g1.scales_t = gst;
   g1.offsets = offsets;
   g1.mprefix = mprefix;
   g1.P = P;
@@ -201,12 +209,12 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   g1.n_out = I;
   g1.status = status;
   MOE_CUDA(moe::launch_gemm_gateup_swiglu(g1, num_sms, st));
-  E_.mark(7);
+  E_.mark(9);
 
   moe::GroupedGemmProblem g2 = g1;
   g2.A = h;
   g2.codes = dc;
-  g2.scales = ds;
+  g2.scales_t = dst_;
   g2.K = I;
   g2.Nrows = d;
   g2.out = nullptr;
@@ -215,9 +223,9 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   g2.topk_w = topk_w;
   g2.n_out = d;
   MOE_CUDA(moe::launch_gemm_down_combine(g2, num_sms, st));
-  E_.mark(8);
+  E_.mark(10);
   MOE_CUDA(moe::launch_combine(yw, T, k, d, out, st));
-  E_.mark(9);
+  E_.mark(11);
   return MOE_OK;
 }
 
@@ -264,7 +272,7 @@ moe_status moe_workspace_layout(int E, int k, int T, int d, int I, moe_ws_layout
 
 int moe_forward_launch_count(int E, int k, int T, int d, int I) {
   if (!full_shape_ok(E, k, T, d, I) || T == 0) return 0;
-  return 9;
+  return 11;
 }
 
 moe_status moe_forward(const void* x_dev, const float* W_r_dev, const float* b_r_dev,

@@ -11,15 +11,24 @@
 //
 // One persistent CTA per SM walks the tiles (expert, n tile, m tile) that the
 // device-side routing tables define; no host synchronisation is needed.
-// Warp roles inside a CTA (512 threads):
-//   warp 0      TMA producer: activation tile (bf16, 128B swizzle) and the two
-//               MXFP4 code boxes of the weight tile
-//   warp 1      TMEM allocator and UMMA issuer (one elected thread)
+// A tile is 256 activation rows x 128 weight rows: the 128 x 64 decoded
+// weight block of a k-block feeds two M = 128 UMMAs (rows 0-127 and 128-255),
+// so each decoded weight serves 256 rows. When an expert's last tile has at
+// most 128 rows the second UMMA (and its activation load) is skipped.
+//
+// Warp roles (512 threads):
+//   warp 0      TMA producer: activation tiles (bf16, 128B swizzle), MXFP4 code
+//               boxes and the k-block's E8M0 scales of the weight tile
+//   warp 1      TMEM allocator and UMMA issuer (one thread)
 //   warps 4-7   epilogue: TMEM -> registers -> SwiGLU / weighted store
-//   warps 8-15  decoders: MXFP4 codes -> bf16 weight tile in the 128B
-//               swizzled K-major layout the UMMA descriptor expects
-// Accumulators: two 128 x 240 fp32 buffers in TMEM (512 columns allocated),
-// so the epilogue of one tile overlaps the main loop of the next.
+//   warps 8-15  decoders: two threads per weight row, each turns 32 codes and
+//               their scale into bf16 in the 128B-swizzled K-major layout
+// Accumulators: per tile two 128 x 128 fp32 blocks (256 TMEM columns),
+// double-buffered (512 columns) so the epilogue of one tile overlaps the main
+// loop of the next.
+//
+// Both operands keep every 8-element chunk of a row in kPerm8 order (see
+// moe_ptx.cuh); the H rows this kernel writes follow the same order.
 #include <cuda_bf16.h>
 #include <stdint.h>
 
@@ -29,22 +38,29 @@
 namespace moe {
 namespace {
 
-constexpr int BM = kTileM;        // rows per tile
-constexpr int BK = 64;            // contraction elements per k-block (128 B of bf16)
-constexpr int NH = 120;           // weight rows per TMA box (one half of the tile)
-constexpr int BN = 2 * NH;        // UMMA N
-constexpr int SA = 4;             // activation stages
-constexpr int SB = 3;             // decoded weight stages
-constexpr int SC = 4;             // code stages
-constexpr int A_BYTES = BM * BK * 2;   // 16384
-constexpr int B_BYTES = BN * BK * 2;   // 30720
-constexpr int C_BYTES = BN * BK / 2;   // 7680
+constexpr int BM = kTileM;            // 256 rows per tile (two UMMA halves)
+constexpr int BMH = 128;              // rows per UMMA
+constexpr int BK = 64;                // contraction elements per k-block (128 B of bf16)
+constexpr int NH = 64;                // weight rows per TMA box (half of the tile)
+constexpr int BN = 2 * NH;            // 128 = UMMA N
+constexpr int SA = 4;                 // activation stages
+constexpr int SB = 4;                 // decoded weight stages
+constexpr int SC = 6;                 // code stages
+constexpr int A_HALF = BMH * BK * 2;  // 16384
+constexpr int A_BYTES = 2 * A_HALF;   // 32768
+constexpr int B_BYTES = BN * BK * 2;  // 16384
+constexpr int C_CODES = BN * BK / 2;  // 4096 bytes of codes per stage
+constexpr int S_BOX = NH * 2;         // scales of one box: 64 rows x 2 groups
+constexpr int S_OFF0 = C_CODES;       // 4096
+constexpr int S_OFF1 = C_CODES + 128; // 4224
+constexpr int C_TX = C_CODES + 2 * S_BOX;
+constexpr int C_BYTES = 4352;         // stage stride (128-byte aligned)
 constexpr int NUM_THREADS = 512;
 constexpr int EPI_WARP0 = 4;
 constexpr int DEQ_WARP0 = 8;
 constexpr int DEQ_THREADS = 256;
 constexpr int TMEM_COLS = 512;
-constexpr int ACC_COLS = 256;     // column distance between the two accumulators
+constexpr int ACC_COLS = 256;         // column distance between the two tile buffers
 constexpr int MAX_E = 256;
 
 constexpr int OFF_A = 0;
@@ -56,11 +72,12 @@ constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
 constexpr int OFF_TAB = OFF_MISC + 16;
 constexpr int SMEM_BYTES = OFF_TAB + 2 * (MAX_E + 1) * 4;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;   // slack for 1024-byte alignment
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+static_assert(OFF_C % 1024 == 0 && C_BYTES % 128 == 0, "stage alignment");
 
 enum Epi { EPI_SWIGLU = 0, EPI_DOWN = 1 };
 
 struct Args {
-  const uint8_t* scales;
   const int32_t* offsets;
   const int32_t* mprefix;
   int E, K, Nrows;
@@ -98,7 +115,7 @@ __device__ __forceinline__ void decode_tile(int tile, int n_tiles, int E, const 
   ti.rows = min(BM, cnt - ti.mt * BM);
 }
 
-__device__ __forceinline__ float silu_f(float g) { return g / (1.0f + __expf(-g)); }
+__device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -108,15 +125,15 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
 template <int EPI>
 __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_mxfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
-                              const __grid_constant__ CUtensorMap tmB, const Args args) {
+                              const __grid_constant__ CUtensorMap tmB,
+                              const __grid_constant__ CUtensorMap tmS, const Args args) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + OFF_BAR);
-  const uint32_t bar0 = smem_u32(bars);
+  const uint32_t bar0 = sbase + OFF_BAR;
   auto bar_fullA = [&](int s) { return bar0 + 8u * s; };
   auto bar_emptyA = [&](int s) { return bar0 + 8u * (SA + s); };
   auto bar_fullB = [&](int s) { return bar0 + 8u * (2 * SA + s); };
@@ -156,6 +173,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmS);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(misc), TMEM_COLS);
@@ -168,7 +186,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int total = s_mp[E] * args.n_tiles;
   const int KB = (args.K + BK - 1) / BK;
-  const int KG = args.K / 32;  // scale groups per row
+  if (warp == 2 || warp == 3) return;  // no role; the final barrier counts the others
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer --
@@ -178,18 +196,24 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         TileInfo ti;
         decode_tile(tile, args.n_tiles, E, s_off, s_mp, ti);
+        const bool two = ti.rows > BMH;
         const int rA = ti.nt * args.row_step;
         const int rB = rA + args.half_off;
         for (int kb = 0; kb < KB; ++kb) {
           if (!(ok = mbar_wait(bar_emptyA(sa), pa ^ 1, abort_flag, args.status))) break;
-          mbar_expect_tx(bar_fullA(sa), A_BYTES);
-          tma_load_2d(sbase + OFF_A + sa * A_BYTES, &tmA, kb * BK, ti.row0, bar_fullA(sa));
+          const uint32_t adst = sbase + OFF_A + sa * A_BYTES;
+          mbar_expect_tx(bar_fullA(sa), two ? A_BYTES : A_HALF);
+          tma_load_2d(adst, &tmA, kb * BK, ti.row0, bar_fullA(sa));
+          if (two) tma_load_2d(adst + A_HALF, &tmA, kb * BK, ti.row0 + BMH, bar_fullA(sa));
           if (++sa == SA) { sa = 0; pa ^= 1; }
           if (!(ok = mbar_wait(bar_emptyC(sc), pc ^ 1, abort_flag, args.status))) break;
-          mbar_expect_tx(bar_fullC(sc), C_BYTES);
           const uint32_t cdst = sbase + OFF_C + sc * C_BYTES;
+          mbar_expect_tx(bar_fullC(sc), C_TX);
           tma_load_3d(cdst, &tmB, kb * (BK / 2), rA, ti.e, bar_fullC(sc));
           tma_load_3d(cdst + NH * (BK / 2), &tmB, kb * (BK / 2), rB, ti.e, bar_fullC(sc));
+          // scales [E][K/32][Nrows]: groups 2kb, 2kb+1 of each box's 64 rows
+          tma_load_3d(cdst + S_OFF0, &tmS, rA, 2 * kb, ti.e, bar_fullC(sc));
+          tma_load_3d(cdst + S_OFF1, &tmS, rB, 2 * kb, ti.e, bar_fullC(sc));
           if (++sc == SC) { sc = 0; pc ^= 1; }
         }
       }
@@ -197,15 +221,18 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp == 1) {
     // -------------------------------------------------------- UMMA issuer --
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(BM, BN);
+      const uint32_t idesc = idesc_bf16_f32(BMH, BN);
       int sa = 0, pa = 0, sb = 0, pb = 0, it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+        TileInfo ti;
+        decode_tile(tile, args.n_tiles, E, s_off, s_mp, ti);
+        const bool two = ti.rows > BMH;
         const int ab = it & 1;
         const uint32_t ap = (it >> 1) & 1;
         if (!(ok = mbar_wait(bar_accEmpty(ab), ap ^ 1, abort_flag, args.status))) break;
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + ab * ACC_COLS;
+        const uint32_t d0 = tmem_base + ab * ACC_COLS;
         for (int kb = 0; kb < KB; ++kb) {
           if (!(ok = mbar_wait(bar_fullA(sa), pa, abort_flag, args.status))) break;
           if (!(ok = mbar_wait(bar_fullB(sb), pb, abort_flag, args.status))) break;
@@ -214,8 +241,11 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           const uint32_t b_addr = sbase + OFF_B + sb * B_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk) {
-            umma_bf16(d_tmem, sdesc_k_sw128(a_addr + kk * 32), sdesc_k_sw128(b_addr + kk * 32),
-                      idesc, (kb | kk) != 0);
+            const uint64_t bdesc = sdesc_k_sw128(b_addr + kk * 32);
+            const uint32_t acc = (kb | kk) != 0;
+            umma_bf16(d0, sdesc_k_sw128(a_addr + kk * 32), bdesc, idesc, acc);
+            if (two)
+              umma_bf16(d0 + BN, sdesc_k_sw128(a_addr + A_HALF + kk * 32), bdesc, idesc, acc);
           }
           umma_commit(bar_emptyA(sa));
           umma_commit(bar_emptyB(sb));
@@ -228,7 +258,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   } else if (warp >= EPI_WARP0 && warp < EPI_WARP0 + 4) {
     // ----------------------------------------------------------- epilogue --
     const int quad = warp & 3;
-    const int r = quad * 32 + lane;
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       TileInfo ti;
@@ -237,65 +266,57 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
       const uint32_t ap = (it >> 1) & 1;
       if (!mbar_wait(bar_accFull(ab), ap, abort_flag, args.status)) break;
       tc_fence_after();
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + ab * ACC_COLS;
-      const bool valid = r < ti.rows;
-      const int64_t grow = ti.row0 + r;
-      if (EPI == EPI_SWIGLU) {
-        const int col0 = ti.nt * NH;
-        uint16_t* orow = args.out + grow * args.n_out;
+      const int halves = ti.rows > BMH ? 2 : 1;
+      for (int hh = 0; hh < halves; ++hh) {
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) +
+                               ab * ACC_COLS + hh * BN;
+        const int r = hh * BMH + quad * 32 + lane;
+        const bool valid = r < ti.rows;
+        const int64_t grow = ti.row0 + r;
+        if (EPI == EPI_SWIGLU) {
+          // columns 0..63 gate, 64..127 up; H stored in kPerm8 chunk order
+          const int col0 = ti.nt * NH;
+          uint16_t* orow = args.out + grow * args.n_out;
 #pragma unroll 1
-        for (int c = 0; c < NH; c += 8) {
-          uint32_t g[8], u[8];
-          tmem_ld8(taddr + c, g);
-          tmem_ld8(taddr + NH + c, u);
-          tmem_ld_wait();
-          uint32_t o[4];
+          for (int c = 0; c < NH; c += 8) {
+            uint32_t g[8], u[8];
+            tmem_ld8(taddr + c, g);
+            tmem_ld8(taddr + NH + c, u);
+            tmem_ld_wait();
+            float h[8];
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const float g0 = __uint_as_float(g[2 * i]), g1 = __uint_as_float(g[2 * i + 1]);
-            const float u0 = __uint_as_float(u[2 * i]), u1 = __uint_as_float(u[2 * i + 1]);
-            o[i] = pack_bf16x2(silu_f(g0) * u0, silu_f(g1) * u1);
-          }
-          const int col = col0 + c;
-          if (valid) {
-            if (col + 8 <= args.n_out) {
-              *reinterpret_cast<uint4*>(orow + col) = make_uint4(o[0], o[1], o[2], o[3]);
-            } else {
-              for (int i = 0; i < 8 && col + i < args.n_out; ++i)
-                orow[col + i] = static_cast<uint16_t>(o[i >> 1] >> (16 * (i & 1)));
+            for (int i = 0; i < 8; ++i)
+              h[i] = silu_f(__uint_as_float(g[i])) * __uint_as_float(u[i]);
+            const int col = col0 + c;
+            if (valid && col < args.n_out) {
+              *reinterpret_cast<uint4*>(orow + col) =
+                  make_uint4(pack_bf16x2(h[0], h[4]), pack_bf16x2(h[1], h[5]),
+                             pack_bf16x2(h[2], h[6]), pack_bf16x2(h[3], h[7]));
             }
           }
-        }
-      } else {
-        // weighted un-permute: fp32 row p * y of pair perm[row], stored at
-        // yw[pair] so that the per-token sum reads k contiguous rows
-        const int col0 = ti.nt * BN;
-        int pair = 0;
-        float w = 0.f;
-        if (valid) {
-          pair = args.perm[grow];
-          w = args.topk_w[pair];
-        }
-        float* orow = args.out_f32 + static_cast<int64_t>(pair) * args.n_out;
-#pragma unroll 1
-        for (int c = 0; c < BN; c += 16) {
-          uint32_t y[16];
-          tmem_ld16(taddr + c, y);
-          tmem_ld_wait();
-          float v[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) v[i] = w * __uint_as_float(y[i]);
-          const int col = col0 + c;
+        } else {
+          // weighted un-permute: fp32 row p * y of pair perm[row] at yw[pair]
+          const int col0 = ti.nt * BN;
+          int pair = 0;
+          float w = 0.f;
           if (valid) {
-            if (col + 16 <= args.n_out) {
+            pair = args.perm[grow];
+            w = args.topk_w[pair];
+          }
+          float* orow = args.out_f32 + static_cast<int64_t>(pair) * args.n_out;
+#pragma unroll 1
+          for (int c = 0; c < BN; c += 16) {
+            uint32_t y[16];
+            tmem_ld16(taddr + c, y);
+            tmem_ld_wait();
+            const int col = col0 + c;
+            if (valid && col < args.n_out) {
               float4* dst = reinterpret_cast<float4*>(orow + col);
 #pragma unroll
               for (int i = 0; i < 4; ++i)
-                dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            } else {
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                if (col + i < args.n_out) orow[col + i] = v[i];
+                dst[i] = make_float4(w * __uint_as_float(y[4 * i]), w * __uint_as_float(y[4 * i + 1]),
+                                     w * __uint_as_float(y[4 * i + 2]),
+                                     w * __uint_as_float(y[4 * i + 3]));
             }
           }
         }
@@ -305,47 +326,28 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     }
   } else if (warp >= DEQ_WARP0) {
     // ----------------------------------------------------------- decoders --
-    const int n = threadIdx.x - DEQ_WARP0 * 32;   // weight row inside the tile
-    const bool active = n < BN;
+    const int t = threadIdx.x - DEQ_WARP0 * 32;
+    const int n = t >> 1;             // weight row inside the tile (0..127)
+    const int g = t & 1;              // scale group inside the k-block
+    const int soff = (n < NH ? S_OFF0 : S_OFF1) + g * NH + (n & (NH - 1));
+    const int sw = n & 7;
     int sc = 0, pc = 0, sb = 0, pb = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-      TileInfo ti;
-      decode_tile(tile, args.n_tiles, E, s_off, s_mp, ti);
-      const int rA = ti.nt * args.row_step;
-      const int wrow = (n < NH) ? rA + n : rA + args.half_off + (n - NH);
-      const bool row_ok = active && wrow < args.Nrows;
-      const uint8_t* srow =
-          args.scales + (static_cast<int64_t>(ti.e) * args.Nrows + (row_ok ? wrow : 0)) * KG;
-      const int sw = n & 7;
       for (int kb = 0; kb < KB; ++kb) {
-        uint32_t s0 = 0, s1 = 0;
-        if (row_ok) {
-          const int g0 = 2 * kb;
-          s0 = srow[g0];
-          if (g0 + 1 < KG) s1 = srow[g0 + 1];
-        }
         if (!(ok = mbar_wait(bar_fullC(sc), pc, abort_flag, args.status))) break;
-        uint4 q0 = make_uint4(0, 0, 0, 0), q1 = q0;
-        if (active) {
-          const uint4* src = reinterpret_cast<const uint4*>(smem + OFF_C + sc * C_BYTES + n * 32);
-          q0 = src[0];
-          q1 = src[1];
-        }
+        const uint8_t* stage = smem + OFF_C + sc * C_BYTES;
+        const uint4 q = *reinterpret_cast<const uint4*>(stage + n * 32 + g * 16);
+        const uint32_t s = stage[soff];
         mbar_arrive(bar_emptyC(sc));
         if (++sc == SC) { sc = 0; pc ^= 1; }
+        uint4 o[4];
+        mxfp4x32_to_bf16(q, s, o);
         if (!(ok = mbar_wait(bar_emptyB(sb), pb ^ 1, abort_flag, args.status))) break;
-        if (active) {
-          uint8_t* brow = smem + OFF_B + sb * B_BYTES + n * 128;
-          uint4 o[4];
-          mxfp4x32_to_bf16(q0, s0, o);
+        uint8_t* brow = smem + OFF_B + sb * B_BYTES + n * 128;
 #pragma unroll
-          for (int c = 0; c < 4; ++c) *reinterpret_cast<uint4*>(brow + ((c ^ sw) << 4)) = o[c];
-          mxfp4x32_to_bf16(q1, s1, o);
-#pragma unroll
-          for (int c = 0; c < 4; ++c)
-            *reinterpret_cast<uint4*>(brow + (((c + 4) ^ sw) << 4)) = o[c];
-        }
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(brow + (((4 * g + c) ^ sw) << 4)) = o[c];
         fence_proxy_async_smem();
         mbar_arrive(bar_fullB(sb));
         if (++sb == SB) { sb = 0; pb ^= 1; }
@@ -381,32 +383,46 @@ EncodeTiledFn get_encode_fn() {
   return fn;
 }
 
-// [rows][K] bf16, box 64 x 128, 128-byte swizzle.
-bool make_act_map(CUtensorMap* m, const void* base, int rows, int K) {
+bool encode(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base,
+            const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+            CUtensorMapSwizzle sw) {
   EncodeTiledFn enc = get_encode_fn();
   if (!enc) return false;
-  cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
-  cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
-  cuuint32_t box[2] = {BK, BM};
-  cuuint32_t es[2] = {1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, dt, rank, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// [E][Nrows][K/2] uint8 codes, box 32 bytes x NH rows x 1 expert.
+// Activations [rows][K] bf16, box 64 x 128, 128-byte swizzle.
+bool make_act_map(CUtensorMap* m, const void* base, int rows, int K) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {BK, BMH};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
+                CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Codes [E][Nrows][K/2] uint8, box 32 bytes x 64 rows x 1 expert.
 bool make_code_map(CUtensorMap* m, const void* base, int E, int Nrows, int K) {
-  EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
-  cuuint64_t dims[3] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(Nrows),
-                        static_cast<cuuint64_t>(E)};
-  cuuint64_t strides[2] = {static_cast<cuuint64_t>(K / 2),
-                           static_cast<cuuint64_t>(K / 2) * static_cast<cuuint64_t>(Nrows)};
-  cuuint32_t box[3] = {BK / 2, NH, 1};
-  cuuint32_t es[3] = {1, 1, 1};
-  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box, es,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(Nrows),
+                              static_cast<cuuint64_t>(E)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K / 2),
+                                 static_cast<cuuint64_t>(K / 2) * static_cast<cuuint64_t>(Nrows)};
+  const cuuint32_t box[3] = {BK / 2, NH, 1};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
+                CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// Transposed scales [E][K/32][Nrows] uint8, box 64 rows x 2 groups x 1 expert.
+bool make_scale_map(CUtensorMap* m, const void* base, int E, int Nrows, int K) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(Nrows), static_cast<cuuint64_t>(K / 32),
+                              static_cast<cuuint64_t>(E)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(Nrows),
+                                 static_cast<cuuint64_t>(Nrows) * static_cast<cuuint64_t>(K / 32)};
+  const cuuint32_t box[3] = {NH, 2, 1};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
+                CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
 template <int EPI>
@@ -420,11 +436,11 @@ cudaError_t launch_impl(const GroupedGemmProblem& p, int num_sms, cudaStream_t s
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  CUtensorMap tmA, tmB;
+  CUtensorMap tmA, tmB, tmS;
   if (!make_act_map(&tmA, p.A, p.P, p.K)) return cudaErrorInvalidValue;
   if (!make_code_map(&tmB, p.codes, p.E, p.Nrows, p.K)) return cudaErrorInvalidValue;
+  if (!make_scale_map(&tmS, p.scales_t, p.E, p.Nrows, p.K)) return cudaErrorInvalidValue;
   Args a;
-  a.scales = p.scales;
   a.offsets = p.offsets;
   a.mprefix = p.mprefix;
   a.E = p.E;
@@ -449,7 +465,7 @@ cudaError_t launch_impl(const GroupedGemmProblem& p, int num_sms, cudaStream_t s
   const int64_t mt_bound = (static_cast<int64_t>(p.P) + BM - 1) / BM + p.E;
   const int64_t tiles_bound = mt_bound * a.n_tiles;
   const int grid = static_cast<int>(tiles_bound < num_sms ? tiles_bound : num_sms);
-  grouped_mxfp4_gemm_kernel<EPI><<<grid, NUM_THREADS, SMEM_ALLOC, st>>>(tmA, tmB, a);
+  grouped_mxfp4_gemm_kernel<EPI><<<grid, NUM_THREADS, SMEM_ALLOC, st>>>(tmA, tmB, tmS, a);
   return cudaGetLastError();
 }
 

@@ -11,7 +11,7 @@ namespace moe {
 // Token chunk of the permutation kernels (tokens per block).
 constexpr int kPermChunk = 256;
 // Rows of one M tile of the grouped GEMMs.
-constexpr int kTileM = 128;
+constexpr int kTileM = 256;
 
 inline int perm_chunks(int T) { return (T + kPermChunk - 1) / kPermChunk; }
 
@@ -39,6 +39,9 @@ cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* perm, int P, in
 // Per-token sum of the k weighted expert rows, rounded to bf16.
 cudaError_t launch_combine(const float* yw, int T, int k, int d, uint16_t* out,
                            cudaStream_t st);
+// E8M0 scales [E][N][G] -> [E][G][N] (the GEMMs load them with TMA per k-block).
+cudaError_t launch_transpose_scales(const uint8_t* in, int E, int N, int G, uint8_t* out,
+                                    cudaStream_t st);
 // MXFP4 rows -> bf16 rows (same decoder as the GEMMs).
 cudaError_t launch_mxfp4_to_bf16(const uint8_t* codes, const uint8_t* scales, int rows, int K,
                                  uint16_t* out, cudaStream_t st);
@@ -47,7 +50,7 @@ cudaError_t launch_mxfp4_to_bf16(const uint8_t* codes, const uint8_t* scales, in
 struct GroupedGemmProblem {
   const uint16_t* A;        // [P][K] bf16 rows in permuted order
   const uint8_t* codes;     // [E][Nrows][K/2]
-  const uint8_t* scales;    // [E][Nrows][K/32]
+  const uint8_t* scales_t;  // [E][K/32][Nrows] (transposed E8M0 scales)
   const int32_t* offsets;   // [E+1]
   const int32_t* mprefix;   // [E+1] prefix of M tiles per expert
   int P, E, K, Nrows;

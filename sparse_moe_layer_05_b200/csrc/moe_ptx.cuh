@@ -197,15 +197,35 @@ __device__ __forceinline__ uint32_t bf16x2_mul(uint32_t a, uint32_t b) {
   return d;
 }
 
+// Order of the elements inside every 8-element chunk of a GEMM operand row:
+// position p holds element kPerm8[p]. Both operands of the grouped GEMMs (the
+// activation rows and the decoded weight rows) use it, so each dot product is
+// unchanged; it lets the decoder emit bf16 pairs (j, j+4) straight from the
+// packed nibbles.
+//   kPerm8 = {0, 4, 1, 5, 2, 6, 3, 7}
+
+// 8 bf16 in natural order (4 words) -> chunk order.
+__device__ __forceinline__ uint4 chunk8_to_perm(uint4 v) {
+  return make_uint4(__byte_perm(v.x, v.z, 0x5410), __byte_perm(v.x, v.z, 0x7632),
+                    __byte_perm(v.y, v.w, 0x5410), __byte_perm(v.y, v.w, 0x7632));
+}
+
+// 8 bf16 in chunk order -> natural order.
+__device__ __forceinline__ uint4 chunk8_from_perm(uint4 v) {
+  return make_uint4(__byte_perm(v.x, v.y, 0x5410), __byte_perm(v.z, v.w, 0x5410),
+                    __byte_perm(v.x, v.y, 0x7632), __byte_perm(v.z, v.w, 0x7632));
+}
+
 // Decode 32 E2M1 codes (16 bytes; byte b holds element 2b in its low nibble)
-// sharing the E8M0 scale byte S into 32 bf16 values, written as four 16-byte
-// chunks of 8 consecutive elements.
+// sharing the E8M0 scale byte S into 32 bf16 values: four 16-byte chunks of
+// 8 elements, each chunk in kPerm8 order.
 //
 // An E2M1 code s|e1 e0|m placed in bf16 bits as s<<15 | (e1 e0 m)<<6 is the
 // bf16 number whose value is exactly 2^-126 times the E2M1 value, for the
 // normal codes and the subnormal alike. Multiplying by 2^(S-1) then yields
 // e2m1 * 2^(S-127) exactly (one product for S <= 128, two for larger S,
-// NaN for S = 255).
+// NaN for S = 255). Nibbles j and j+4 of a code word sit 16 bits apart, so
+// one shift and mask place both in their bf16 halves.
 __device__ __forceinline__ void mxfp4x32_to_bf16(uint4 q, uint32_t S, uint4 (&out)[4]) {
   uint32_t m1, m2 = 0;
   bool two = false;
@@ -224,19 +244,24 @@ __device__ __forceinline__ void mxfp4x32_to_bf16(uint4 q, uint32_t S, uint4 (&ou
   uint32_t r[16];
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
-    const uint32_t ev = w[i] & 0x0F0F0F0Fu;         // elements 8i+0, +2, +4, +6
-    const uint32_t od = (w[i] >> 4) & 0x0F0F0F0Fu;  // elements 8i+1, +3, +5, +7
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint32_t sel = (uint32_t)j | ((uint32_t)j << 4) | ((uint32_t)(4 + j) << 8) |
-                           ((uint32_t)(4 + j) << 12);
-      const uint32_t t = __byte_perm(ev, od, sel) & 0x000F000Fu;
-      // (c & 7) << 6 | (c & 8) << 12 in each 16-bit half
-      const uint32_t b = (t << 6) + (t & 0x00080008u) * 4032u;
-      uint32_t v = bf16x2_mul(b, m1);
-      if (two) v = bf16x2_mul(v, m2);
-      r[i * 4 + j] = v;
+    const uint32_t x = w[i];
+    // word j holds (element j, element j+4) of this 8-code word
+    const uint32_t b0 = ((x << 6) & 0x01C001C0u) | ((x << 12) & 0x80008000u);
+    const uint32_t b1 = ((x << 2) & 0x01C001C0u) | ((x << 8) & 0x80008000u);
+    const uint32_t b2 = ((x >> 2) & 0x01C001C0u) | ((x << 4) & 0x80008000u);
+    const uint32_t b3 = ((x >> 6) & 0x01C001C0u) | (x & 0x80008000u);
+    uint32_t v0 = bf16x2_mul(b0, m1), v1 = bf16x2_mul(b1, m1);
+    uint32_t v2 = bf16x2_mul(b2, m1), v3 = bf16x2_mul(b3, m1);
+    if (two) {
+      v0 = bf16x2_mul(v0, m2);
+      v1 = bf16x2_mul(v1, m2);
+      v2 = bf16x2_mul(v2, m2);
+      v3 = bf16x2_mul(v3, m2);
     }
+    r[4 * i + 0] = v0;
+    r[4 * i + 1] = v1;
+    r[4 * i + 2] = v2;
+    r[4 * i + 3] = v3;
   }
   out[0] = make_uint4(r[0], r[1], r[2], r[3]);
   out[1] = make_uint4(r[4], r[5], r[6], r[7]);

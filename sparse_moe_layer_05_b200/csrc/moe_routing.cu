@@ -256,6 +256,8 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(const int32_t* __rest
 }
 
 // ----------------------------------------------------------- K2 gather ----
+// xp[r] = x[perm[r] / k], each 8-element chunk stored in kPerm8 order (the
+// operand order of the grouped GEMMs).
 __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __restrict__ x,
                                                           const int32_t* __restrict__ perm, int P,
                                                           int k, int d,
@@ -267,7 +269,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
     const int t = perm[r] / k;
     const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * d);
     uint4* dst = reinterpret_cast<uint4*>(xp + (size_t)r * d);
-    for (int c = lane; c < vec; c += 32) dst[c] = __ldg(src + c);
+    for (int c = lane; c < vec; c += 32) dst[c] = chunk8_to_perm(__ldg(src + c));
   }
 }
 
@@ -314,7 +316,29 @@ __global__ void __launch_bounds__(256) mxfp4_to_bf16_kernel(const uint8_t* __res
     mxfp4x32_to_bf16(q, scales[g], o);
     uint4* dst = reinterpret_cast<uint4*>(out) + g * 4;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) dst[i] = o[i];
+    for (int i = 0; i < 4; ++i) dst[i] = chunk8_from_perm(o[i]);
+  }
+}
+
+// -------------------------------------------------- scale transpose ----
+// [E][N][G] -> [E][G][N], through a 32 x 32 shared tile.
+__global__ void __launch_bounds__(256) transpose_scales_kernel(const uint8_t* __restrict__ in,
+                                                               int N, int G,
+                                                               uint8_t* __restrict__ out) {
+  __shared__ uint8_t tile[32][33];
+  const int e = blockIdx.z;
+  const int n0 = blockIdx.x * 32, g0 = blockIdx.y * 32;
+  const uint8_t* src = in + (size_t)e * N * G;
+  uint8_t* dst = out + (size_t)e * N * G;
+  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
+  for (int r = ty; r < 32; r += 8) {
+    const int n = n0 + r, g = g0 + tx;
+    if (n < N && g < G) tile[r][tx] = src[(size_t)n * G + g];
+  }
+  __syncthreads();
+  for (int r = ty; r < 32; r += 8) {
+    const int g = g0 + r, n = n0 + tx;
+    if (n < N && g < G) dst[(size_t)g * N + n] = tile[tx][r];
   }
 }
 
@@ -387,6 +411,13 @@ cudaError_t launch_combine(const float* yw, int T, int k, int d, uint16_t* out,
                            cudaStream_t st) {
   const int64_t n = (int64_t)T * (d / 8);
   combine_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(yw, T, k, d, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_transpose_scales(const uint8_t* in, int E, int N, int G, uint8_t* out,
+                                    cudaStream_t st) {
+  dim3 grid((N + 31) / 32, (G + 31) / 32, E);
+  transpose_scales_kernel<<<grid, 256, 0, st>>>(in, N, G, out);
   return cudaGetLastError();
 }
 

@@ -31,6 +31,20 @@ def bf16_to_f64(u16):
     return O.bf16_to_f64(u16)
 
 
+# Inside every 8-element chunk the GEMM operand rows (xp, h) store element
+# CHUNK_ORDER[p] at position p.
+CHUNK_ORDER = np.array([0, 4, 1, 5, 2, 6, 3, 7])
+
+
+def unpermute_chunks(a):
+    """Natural column order of a [rows, n] array stored in chunk order."""
+    a = np.asarray(a)
+    n = a.shape[-1]
+    out = np.empty_like(a)
+    out.reshape(*a.shape[:-1], n // 8, 8)[..., CHUNK_ORDER] = a.reshape(*a.shape[:-1], n // 8, 8)
+    return out
+
+
 def rel_rms_err(got, want):
     rms = float(np.sqrt(np.mean(want ** 2)))
     err = float(np.max(np.abs(got - want))) if want.size else 0.0

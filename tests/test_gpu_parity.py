@@ -144,7 +144,9 @@ def test_forward_matches_oracle(case):
     c, o, p, _ = O.routing_tables(idx, E)
     assert np.array_equal(perm, p)
     if np.array_equal(idx, r.idx):
-        H = O.bf16_to_f64(layer.intermediate("h", T).cpu().numpy())
+        H = O.bf16_to_f64(G.unpermute_chunks(layer.intermediate("h", T).cpu().numpy()))
+        xp = G.unpermute_chunks(layer.intermediate("xp", T).cpu().numpy())
+        assert np.array_equal(xp, inp.x[perm // k])
         for e, (toks, h) in hidden.items():
             rows = H[o[e]:o[e + 1]]
             assert np.array_equal(perm[o[e]:o[e + 1]] // k, toks)
