@@ -90,6 +90,17 @@ MOE_API const char* moe_status_string(moe_status s);
 MOE_API int moe_version(void);
 
 /*
+ * Tile policy of the grouped GEMMs, process-wide: 0 (default) automatic --
+ * currently single-CTA tiles (256 x 128, the second 128-row half skipped for
+ * short expert tails), the faster on every measured shape; 1 forces
+ * single-CTA tiles; 2 forces CTA-pair tiles (a 2-CTA cluster computes
+ * 256 x 240 tiles with tcgen05 cta_group::2). Both compute the same function.
+ * Not thread-safe against concurrent forward calls. MOE_ERR_INVALID_ARG for
+ * other values.
+ */
+MOE_API moe_status moe_set_tile_policy(int policy);
+
+/*
  * Bytes of device workspace moe_forward needs for this shape (0 for invalid
  * shapes). The workspace holds the router's logits and top-k, the routing
  * tables, the permuted activations, the SwiGLU hidden rows H [T*k][I] bf16 and

@@ -29,6 +29,7 @@ EXPORTS = [
     "moe_workspace_size_hostio", "moe_forward_hostio", "moe_route_workspace_size",
     "moe_route", "moe_workspace_layout", "moe_mxfp4_to_bf16", "moe_sync_status",
     "moe_selftest_wait_timeout", "moe_forward_launch_count", "moe_forward_timed",
+    "moe_set_tile_policy",
 ]
 
 STAGES = ["router_logits", "topk_softmax", "perm_hist", "perm_scan", "perm_scatter",
@@ -88,6 +89,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_sync_status.argtypes = [vp, sz, vp]
     lib.moe_selftest_wait_timeout.restype = i32
     lib.moe_selftest_wait_timeout.argtypes = [vp, vp]
+    lib.moe_set_tile_policy.restype = i32
+    lib.moe_set_tile_policy.argtypes = [i32]
     lib.moe_forward_launch_count.restype = i32
     lib.moe_forward_launch_count.argtypes = [i32] * 5
     _lib = lib
@@ -194,6 +197,14 @@ def moe_mxfp4_to_bf16(codes, scales, rows: int, K: int, out, stream=None) -> Non
     _require_cuda(codes, scales, out)
     _check("moe_mxfp4_to_bf16", load().moe_mxfp4_to_bf16(
         _ptr(codes), _ptr(scales), rows, K, _ptr(out), _stream(stream)))
+
+
+TILE_AUTO, TILE_SINGLE, TILE_PAIR = 0, 1, 2
+
+
+def moe_set_tile_policy(policy: int) -> None:
+    """0 = by shape, 1 = single-CTA tiles, 2 = CTA-pair tiles (process-wide)."""
+    _check("moe_set_tile_policy", load().moe_set_tile_policy(policy))
 
 
 def moe_sync_status(workspace, stream=None) -> int:

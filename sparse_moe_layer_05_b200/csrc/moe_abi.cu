@@ -12,6 +12,18 @@ namespace {
 constexpr int kVersion = 100;  // 0.1.0
 constexpr int kMaxDevices = 64;
 
+// Grouped-GEMM tile policy: 0 = choose by shape, 1 = single-CTA tiles,
+// 2 = CTA-pair tiles.
+int g_tile_policy = 0;
+
+bool use_pair_tiles(int P, int E) {
+  (void)P;
+  (void)E;
+  // By shape the single-CTA tiles are faster on every measured workload so far,
+  // so the automatic choice is single-CTA; CTA-pair tiles are opt-in.
+  return g_tile_policy == 2;
+}
+
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 struct Layout {
@@ -208,6 +220,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   g1.topk_w = nullptr;
   g1.n_out = I;
   g1.status = status;
+  g1.use_pair = use_pair_tiles(P, E);
   MOE_CUDA(moe::launch_gemm_gateup_swiglu(g1, num_sms, st));
   E_.mark(9);
 
@@ -247,6 +260,12 @@ const char* moe_status_string(moe_status s) {
 }
 
 int moe_version(void) { return kVersion; }
+
+moe_status moe_set_tile_policy(int policy) {
+  if (policy < 0 || policy > 2) return MOE_ERR_INVALID_ARG;
+  g_tile_policy = policy;
+  return MOE_OK;
+}
 
 size_t moe_workspace_size(int E, int k, int T, int d, int I) {
   if (!full_shape_ok(E, k, T, d, I)) return 0;

@@ -17,8 +17,9 @@
 // most 128 rows the second UMMA (and its activation load) is skipped.
 //
 // Warp roles (512 threads):
-//   warp 0      TMA producer: activation tiles (bf16, 128B swizzle), MXFP4 code
-//               boxes and the k-block's E8M0 scales of the weight tile
+//   warp 0      TMA producer of the activation tiles (bf16, 128B swizzle)
+//   warp 2      TMA producer of the MXFP4 code boxes and the k-block's E8M0
+//               scales (a ring of its own, so codes run ahead of activations)
 //   warp 1      TMEM allocator and UMMA issuer (one thread)
 //   warps 4-7   epilogue: TMEM -> registers -> SwiGLU / weighted store
 //   warps 8-15  decoders: two threads per weight row, each turns 32 codes and
@@ -186,19 +187,17 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 
   const int total = s_mp[E] * args.n_tiles;
   const int KB = (args.K + BK - 1) / BK;
-  if (warp == 2 || warp == 3) return;  // no role; the final barrier counts the others
+  if (warp == 3) return;  // no role; the final barrier counts the others
 
   if (warp == 0) {
-    // ---------------------------------------------------------- producer --
+    // ------------------------------------------- producer: activations --
     if (lane == 0) {
-      int sa = 0, pa = 0, sc = 0, pc = 0;
+      int sa = 0, pa = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         TileInfo ti;
         decode_tile(tile, args.n_tiles, E, s_off, s_mp, ti);
         const bool two = ti.rows > BMH;
-        const int rA = ti.nt * args.row_step;
-        const int rB = rA + args.half_off;
         for (int kb = 0; kb < KB; ++kb) {
           if (!(ok = mbar_wait(bar_emptyA(sa), pa ^ 1, abort_flag, args.status))) break;
           const uint32_t adst = sbase + OFF_A + sa * A_BYTES;
@@ -206,6 +205,21 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           tma_load_2d(adst, &tmA, kb * BK, ti.row0, bar_fullA(sa));
           if (two) tma_load_2d(adst + A_HALF, &tmA, kb * BK, ti.row0 + BMH, bar_fullA(sa));
           if (++sa == SA) { sa = 0; pa ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // -------------------------------------- producer: codes and scales --
+    // Runs ahead of the activation ring as far as the code ring allows.
+    if (lane == 0) {
+      int sc = 0, pc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        TileInfo ti;
+        decode_tile(tile, args.n_tiles, E, s_off, s_mp, ti);
+        const int rA = ti.nt * args.row_step;
+        const int rB = rA + args.half_off;
+        for (int kb = 0; kb < KB; ++kb) {
           if (!(ok = mbar_wait(bar_emptyC(sc), pc ^ 1, abort_flag, args.status))) break;
           const uint32_t cdst = sbase + OFF_C + sc * C_BYTES;
           mbar_expect_tx(bar_fullC(sc), C_TX);
@@ -280,9 +294,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll 1
           for (int c = 0; c < NH; c += 8) {
             uint32_t g[8], u[8];
-            tmem_ld8(taddr + c, g);
-            tmem_ld8(taddr + NH + c, u);
-            tmem_ld_wait();
+            tmem_ld8x2_sync(taddr + c, taddr + NH + c, g, u);
             float h[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
@@ -307,8 +319,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll 1
           for (int c = 0; c < BN; c += 16) {
             uint32_t y[16];
-            tmem_ld16(taddr + c, y);
-            tmem_ld_wait();
+            tmem_ld16_sync(taddr + c, y);
             const int col = col0 + c;
             if (valid && col < args.n_out) {
               float4* dst = reinterpret_cast<float4*>(orow + col);
@@ -339,6 +350,9 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint8_t* stage = smem + OFF_C + sc * C_BYTES;
         const uint4 q = *reinterpret_cast<const uint4*>(stage + n * 32 + g * 16);
         const uint32_t s = stage[soff];
+        // the next TMA write into this stage (async proxy) must not overtake
+        // these generic-proxy reads
+        fence_proxy_async_smem();
         mbar_arrive(bar_emptyC(sc));
         if (++sc == SC) { sc = 0; pc ^= 1; }
         uint4 o[4];
@@ -360,6 +374,353 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
+// ================================================================= pair ====
+// CTA-pair variant for experts with many rows: a cluster of 2 CTAs (one per
+// SM) computes a 256 x 240 tile with tcgen05 cta_group::2 UMMAs (M = 256,
+// N = 240). CTA r holds activation rows r*128..r*128+127 and decodes weight
+// rows r*120..r*120+119 of the tile (the gate rows on CTA 0 and the matching
+// up rows on CTA 1 for the gate/up GEMM), so each SM decodes 120 rows per
+// k-block for 128 x 240 MACs and reads half as much B per MAC as a 1-SM tile.
+// All loads and decodes stay local to each CTA (warp 0 loads activations,
+// warp 2 codes and scales, warps 8-15 decode). The even CTA issues the UMMAs;
+// in the odd CTA warp 3 forwards "stage ready" per k-block and the first
+// epilogue thread forwards "accumulator released" per tile to the even CTA,
+// each with one remote mbarrier arrive.
+namespace pair {
+
+constexpr int BMH = 128;              // activation rows per CTA
+constexpr int BK = 64;
+constexpr int NH = 120;               // weight rows per CTA
+constexpr int BN = 2 * NH;            // 240 = UMMA N
+constexpr int SA = 5, SB = 5, SC = 8;
+constexpr int A_BYTES = BMH * BK * 2;       // 16384
+constexpr int B_BYTES = NH * BK * 2;        // 15360
+constexpr int C_CODES = NH * BK / 2;        // 3840
+constexpr int S_ROWS = 144;                 // 16-aligned window holding 120 rows
+constexpr int S_OFF = 3840;                 // scale box offset in a code stage
+constexpr int C_TX = C_CODES + 2 * S_ROWS;  // 4128
+constexpr int C_BYTES = 4224;
+constexpr int NUM_THREADS = 512;
+constexpr int DEQ_THREADS = 256;
+constexpr int TMEM_COLS = 512;
+constexpr int ACC_COLS = 256;
+
+constexpr int OFF_A = 0;
+constexpr int OFF_B = OFF_A + SA * A_BYTES;
+constexpr int OFF_C = OFF_B + SB * B_BYTES;
+constexpr int OFF_BAR = OFF_C + SC * C_BYTES;
+// fullA, emptyA, fullB, emptyB, peerFull (SB), fullC, emptyC, accFull,
+// accEmpty, peerAccEmpty
+constexpr int NUM_BARS = 2 * SA + 3 * SB + 2 * SC + 6;
+constexpr int OFF_MISC = (OFF_BAR + NUM_BARS * 8 + 15) & ~15;
+constexpr int OFF_TAB = OFF_MISC + 16;
+constexpr int SMEM_BYTES = OFF_TAB + 2 * (MAX_E + 1) * 4;
+constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+static_assert(OFF_B % 1024 == 0 && OFF_C % 1024 == 0 && B_BYTES % 1024 == 0, "alignment");
+
+}  // namespace pair
+
+template <int EPI>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::NUM_THREADS, 1)
+    grouped_mxfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                                   const __grid_constant__ CUtensorMap tmB,
+                                   const __grid_constant__ CUtensorMap tmS, const Args args) {
+  // local copies shadow the single-CTA kernel's constants of the same names
+  constexpr int BMH = pair::BMH;
+  constexpr int BK = pair::BK;
+  constexpr int NH = pair::NH;
+  constexpr int BN = pair::BN;
+  constexpr int SA = pair::SA;
+  constexpr int SB = pair::SB;
+  constexpr int SC = pair::SC;
+  constexpr int A_BYTES = pair::A_BYTES;
+  constexpr int B_BYTES = pair::B_BYTES;
+  constexpr int C_CODES = pair::C_CODES;
+  constexpr int S_ROWS = pair::S_ROWS;
+  constexpr int S_OFF = pair::S_OFF;
+  constexpr int C_TX = pair::C_TX;
+  constexpr int C_BYTES = pair::C_BYTES;
+  constexpr int NUM_THREADS = pair::NUM_THREADS;
+  constexpr int DEQ_THREADS = pair::DEQ_THREADS;
+  constexpr int TMEM_COLS = pair::TMEM_COLS;
+  constexpr int ACC_COLS = pair::ACC_COLS;
+  constexpr int OFF_A = pair::OFF_A;
+  constexpr int OFF_B = pair::OFF_B;
+  constexpr int OFF_C = pair::OFF_C;
+  constexpr int OFF_BAR = pair::OFF_BAR;
+  constexpr int OFF_MISC = pair::OFF_MISC;
+  constexpr int OFF_TAB = pair::OFF_TAB;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair_id = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  const uint32_t bar0 = sbase + OFF_BAR;
+  auto bar_fullA = [&](int s) { return bar0 + 8u * s; };
+  auto bar_emptyA = [&](int s) { return bar0 + 8u * (SA + s); };
+  auto bar_fullB = [&](int s) { return bar0 + 8u * (2 * SA + s); };
+  auto bar_emptyB = [&](int s) { return bar0 + 8u * (2 * SA + SB + s); };
+  auto bar_peerFull = [&](int s) { return bar0 + 8u * (2 * SA + 2 * SB + s); };
+  auto bar_fullC = [&](int s) { return bar0 + 8u * (2 * SA + 3 * SB + s); };
+  auto bar_emptyC = [&](int s) { return bar0 + 8u * (2 * SA + 3 * SB + SC + s); };
+  auto bar_accFull = [&](int s) { return bar0 + 8u * (2 * SA + 3 * SB + 2 * SC + s); };
+  auto bar_accEmpty = [&](int s) { return bar0 + 8u * (2 * SA + 3 * SB + 2 * SC + 2 + s); };
+  auto bar_peerAcc = [&](int s) { return bar0 + 8u * (2 * SA + 3 * SB + 2 * SC + 4 + s); };
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  int* s_off = reinterpret_cast<int*>(smem + OFF_TAB);
+  int* s_mp = s_off + (MAX_E + 1);
+
+  const int E = args.E;
+  for (int i = threadIdx.x; i <= E; i += NUM_THREADS) {
+    s_off[i] = args.offsets[i];
+    s_mp[i] = args.mprefix[i];
+  }
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < SA; ++s) {
+      mbar_init(bar_fullA(s), 1);
+      mbar_init(bar_emptyA(s), 1);
+    }
+    for (int s = 0; s < SB; ++s) {
+      mbar_init(bar_fullB(s), DEQ_THREADS);
+      mbar_init(bar_emptyB(s), 1);
+      mbar_init(bar_peerFull(s), 1);
+    }
+    for (int s = 0; s < SC; ++s) {
+      mbar_init(bar_fullC(s), 1);
+      mbar_init(bar_emptyC(s), DEQ_THREADS);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_accFull(s), 1);
+      mbar_init(bar_accEmpty(s), 4 * 32);
+      mbar_init(bar_peerAcc(s), 1);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmS);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(misc), TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = misc[0];
+
+  const int total = s_mp[E] * args.n_tiles;
+  const int KB = (args.K + BK - 1) / BK;
+
+  if (warp == 0) {
+    // ------------------------------------------- producer: activations --
+    if (lane == 0) {
+      int sa = 0, pa = 0;
+      bool ok = true;
+      for (int tile = pair_id; tile < total && ok; tile += npairs) {
+        TileInfo ti;
+        decode_tile(tile, args.n_tiles, E, s_off, s_mp, ti);
+        const int rAct = ti.row0 + static_cast<int>(rank) * BMH;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!(ok = mbar_wait_cluster(bar_emptyA(sa), pa ^ 1, abort_flag, args.status))) break;
+          mbar_expect_tx(bar_fullA(sa), A_BYTES);
+          tma_load_2d(sbase + OFF_A + sa * A_BYTES, &tmA, kb * BK, rAct, bar_fullA(sa));
+          if (++sa == SA) { sa = 0; pa ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // -------------------------------------- producer: codes and scales --
+    if (lane == 0) {
+      int sc = 0, pc = 0;
+      bool ok = true;
+      for (int tile = pair_id; tile < total && ok; tile += npairs) {
+        TileInfo ti;
+        decode_tile(tile, args.n_tiles, E, s_off, s_mp, ti);
+        const int rW = ti.nt * args.row_step + static_cast<int>(rank) * args.half_off;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!(ok = mbar_wait(bar_emptyC(sc), pc ^ 1, abort_flag, args.status))) break;
+          const uint32_t cdst = sbase + OFF_C + sc * C_BYTES;
+          mbar_expect_tx(bar_fullC(sc), C_TX);
+          tma_load_3d(cdst, &tmB, kb * (BK / 2), rW, ti.e, bar_fullC(sc));
+          tma_load_3d(cdst + S_OFF, &tmS, rW & ~15, 2 * kb, ti.e, bar_fullC(sc));
+          if (++sc == SC) { sc = 0; pc ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------- UMMA issuer (even CTA) --
+    if (rank == 0 && lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(2 * BMH, BN);
+      int sa = 0, pa = 0, sb = 0, pb = 0, it = 0;
+      bool ok = true;
+      for (int tile = pair_id; tile < total && ok; tile += npairs, ++it) {
+        const int ab = it & 1;
+        const uint32_t ap = (it >> 1) & 1;
+        if (!(ok = mbar_wait(bar_accEmpty(ab), ap ^ 1, abort_flag, args.status))) break;
+        if (!(ok = mbar_wait_cluster(bar_peerAcc(ab), ap ^ 1, abort_flag, args.status))) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + ab * ACC_COLS;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!(ok = mbar_wait(bar_fullA(sa), pa, abort_flag, args.status))) break;
+          if (!(ok = mbar_wait(bar_fullB(sb), pb, abort_flag, args.status))) break;
+          if (!(ok = mbar_wait_cluster(bar_peerFull(sb), pb, abort_flag, args.status))) break;
+          tc_fence_after();
+          const uint32_t a_addr = sbase + OFF_A + sa * A_BYTES;
+          const uint32_t b_addr = sbase + OFF_B + sb * B_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16_pair(d, sdesc_k_sw128(a_addr + kk * 32), sdesc_k_sw128(b_addr + kk * 32),
+                           idesc, (kb | kk) != 0);
+          umma_commit_pair(bar_emptyA(sa));
+          umma_commit_pair(bar_emptyB(sb));
+          if (++sa == SA) { sa = 0; pa ^= 1; }
+          if (++sb == SB) { sb = 0; pb ^= 1; }
+        }
+        if (ok) umma_commit_pair(bar_accFull(ab));
+      }
+    }
+  } else if (warp == 3) {
+    // ------------------------------------ stage relay (odd CTA) --
+    if (rank == 1 && lane == 0) {
+      int sa = 0, pa = 0, sb = 0, pb = 0;
+      bool ok = true;
+      for (int tile = pair_id; tile < total && ok; tile += npairs) {
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!(ok = mbar_wait(bar_fullA(sa), pa, abort_flag, args.status))) break;
+          if (!(ok = mbar_wait(bar_fullB(sb), pb, abort_flag, args.status))) break;
+          mbar_arrive_remote(mapa_shared(bar_peerFull(sb), 0));
+          if (++sa == SA) { sa = 0; pa ^= 1; }
+          if (++sb == SB) { sb = 0; pb ^= 1; }
+        }
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ----------------------------------------------------------- epilogue --
+    const int quad = warp & 3;
+    int it = 0;
+    for (int tile = pair_id; tile < total; tile += npairs, ++it) {
+      TileInfo ti;
+      decode_tile(tile, args.n_tiles, E, s_off, s_mp, ti);
+      const int ab = it & 1;
+      const uint32_t ap = (it >> 1) & 1;
+      if (!mbar_wait_cluster(bar_accFull(ab), ap, abort_flag, args.status)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + ab * ACC_COLS;
+      const int r = static_cast<int>(rank) * BMH + quad * 32 + lane;
+      const bool valid = r < ti.rows;
+      const int64_t grow = ti.row0 + r;
+      if (EPI == EPI_SWIGLU) {
+        // columns 0..119 gate (even CTA's rows), 120..239 up (odd CTA's rows)
+        const int col0 = ti.nt * NH;
+        uint16_t* orow = args.out + grow * args.n_out;
+#pragma unroll 1
+        for (int c = 0; c < NH; c += 8) {
+          uint32_t g[8], u[8];
+          tmem_ld8x2_sync(taddr + c, taddr + NH + c, g, u);
+          float h[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            h[i] = silu_f(__uint_as_float(g[i])) * __uint_as_float(u[i]);
+          const int col = col0 + c;
+          if (valid && col < args.n_out) {
+            *reinterpret_cast<uint4*>(orow + col) =
+                make_uint4(pack_bf16x2(h[0], h[4]), pack_bf16x2(h[1], h[5]),
+                           pack_bf16x2(h[2], h[6]), pack_bf16x2(h[3], h[7]));
+          }
+        }
+      } else {
+        const int col0 = ti.nt * BN;
+        int pr = 0;
+        float w = 0.f;
+        if (valid) {
+          pr = args.perm[grow];
+          w = args.topk_w[pr];
+        }
+        float* orow = args.out_f32 + static_cast<int64_t>(pr) * args.n_out;
+#pragma unroll 1
+        for (int c = 0; c < BN; c += 16) {
+          uint32_t y[16];
+          tmem_ld16_sync(taddr + c, y);
+          const int col = col0 + c;
+          if (valid && col < args.n_out) {
+            float4* dst = reinterpret_cast<float4*>(orow + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_float4(w * __uint_as_float(y[4 * i]), w * __uint_as_float(y[4 * i + 1]),
+                                   w * __uint_as_float(y[4 * i + 2]),
+                                   w * __uint_as_float(y[4 * i + 3]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_accEmpty(ab));
+      if (rank == 1 && threadIdx.x == 4 * 32) {
+        // accumulator relay: once all 128 epilogue threads of this CTA have
+        // released the buffer, tell the even CTA's UMMA issuer
+        if (!mbar_wait(bar_accEmpty(ab), ap, abort_flag, args.status)) break;
+        mbar_arrive_remote(mapa_shared(bar_peerAcc(ab), 0));
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- decoders --
+    const int t = threadIdx.x - 8 * 32;
+    const int n = t >> 1;             // weight row of this CTA (0..119 active)
+    const int g = t & 1;
+    const bool active = n < NH;
+    const int sw = n & 7;
+    int sc = 0, pc = 0, sb = 0, pb = 0;
+    bool ok = true;
+    for (int tile = pair_id; tile < total && ok; tile += npairs) {
+      TileInfo ti;
+      decode_tile(tile, args.n_tiles, E, s_off, s_mp, ti);
+      const int rW = ti.nt * args.row_step + static_cast<int>(rank) * args.half_off;
+      const int soff = S_OFF + g * S_ROWS + (rW & 15) + (active ? n : 0);
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!(ok = mbar_wait(bar_fullC(sc), pc, abort_flag, args.status))) break;
+        const uint8_t* stage = smem + OFF_C + sc * C_BYTES;
+        uint4 q = make_uint4(0, 0, 0, 0);
+        uint32_t sv = 0;
+        if (active) {
+          q = *reinterpret_cast<const uint4*>(stage + n * 32 + g * 16);
+          sv = stage[soff];
+        }
+        // the next TMA write into this stage (async proxy) must not overtake
+        // these generic-proxy reads
+        fence_proxy_async_smem();
+        mbar_arrive(bar_emptyC(sc));
+        if (++sc == SC) { sc = 0; pc ^= 1; }
+        uint4 o[4];
+        mxfp4x32_to_bf16(q, sv, o);
+        if (!(ok = mbar_wait_cluster(bar_emptyB(sb), pb ^ 1, abort_flag, args.status))) break;
+        if (active) {
+          uint8_t* brow = smem + OFF_B + sb * B_BYTES + n * 128;
+#pragma unroll
+          for (int c = 0; c < 4; ++c)
+            *reinterpret_cast<uint4*>(brow + (((4 * g + c) ^ sw) << 4)) = o[c];
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(bar_fullB(sb));
+        if (++sb == SB) { sb = 0; pb ^= 1; }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, TMEM_COLS);
   }
 }
 
@@ -414,15 +775,74 @@ bool make_code_map(CUtensorMap* m, const void* base, int E, int Nrows, int K) {
                 CU_TENSOR_MAP_SWIZZLE_NONE);
 }
 
-// Transposed scales [E][K/32][Nrows] uint8, box 64 rows x 2 groups x 1 expert.
-bool make_scale_map(CUtensorMap* m, const void* base, int E, int Nrows, int K) {
+// Transposed scales [E][K/32][Nrows] uint8, box `rows` x 2 groups x 1 expert.
+bool make_scale_map(CUtensorMap* m, const void* base, int E, int Nrows, int K, int rows) {
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(Nrows), static_cast<cuuint64_t>(K / 32),
                               static_cast<cuuint64_t>(E)};
   const cuuint64_t strides[2] = {static_cast<cuuint64_t>(Nrows),
                                  static_cast<cuuint64_t>(Nrows) * static_cast<cuuint64_t>(K / 32)};
-  const cuuint32_t box[3] = {NH, 2, 1};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(rows), 2, 1};
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
                 CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// Codes [E][Nrows][K/2] uint8, box 32 bytes x `rows` rows x 1 expert.
+bool make_code_map_rows(CUtensorMap* m, const void* base, int E, int Nrows, int K, int rows) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K / 2), static_cast<cuuint64_t>(Nrows),
+                              static_cast<cuuint64_t>(E)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K / 2),
+                                 static_cast<cuuint64_t>(K / 2) * static_cast<cuuint64_t>(Nrows)};
+  const cuuint32_t box[3] = {BK / 2, static_cast<cuuint32_t>(rows), 1};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
+                CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+template <int EPI>
+cudaError_t launch_pair_impl(const GroupedGemmProblem& p, int num_sms, cudaStream_t st) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_mxfp4_gemm_pair_kernel<EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         pair::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  CUtensorMap tmA, tmB, tmS;
+  if (!make_act_map(&tmA, p.A, p.P, p.K)) return cudaErrorInvalidValue;
+  if (!make_code_map_rows(&tmB, p.codes, p.E, p.Nrows, p.K, pair::NH)) return cudaErrorInvalidValue;
+  if (!make_scale_map(&tmS, p.scales_t, p.E, p.Nrows, p.K, pair::S_ROWS))
+    return cudaErrorInvalidValue;
+  Args a;
+  a.offsets = p.offsets;
+  a.mprefix = p.mprefix;
+  a.E = p.E;
+  a.K = p.K;
+  a.Nrows = p.Nrows;
+  a.n_out = p.n_out;
+  a.out = p.out;
+  a.out_f32 = p.out_f32;
+  a.perm = p.perm;
+  a.topk_w = p.topk_w;
+  a.status = p.status;
+  if (EPI == EPI_SWIGLU) {
+    a.n_tiles = (p.n_out + pair::NH - 1) / pair::NH;
+    a.row_step = pair::NH;
+    a.half_off = p.n_out;   // the odd CTA decodes the up rows
+  } else {
+    a.n_tiles = (p.n_out + pair::BN - 1) / pair::BN;
+    a.row_step = pair::BN;
+    a.half_off = pair::NH;
+  }
+  const int64_t mt_bound = (static_cast<int64_t>(p.P) + BM - 1) / BM + p.E;
+  const int64_t tiles_bound = mt_bound * a.n_tiles;
+  int64_t pairs = num_sms / 2;
+  if (tiles_bound < pairs) pairs = tiles_bound;
+  const int grid = static_cast<int>(2 * pairs);
+  grouped_mxfp4_gemm_pair_kernel<EPI><<<grid, pair::NUM_THREADS, pair::SMEM_ALLOC, st>>>(tmA, tmB,
+                                                                                      tmS, a);
+  return cudaGetLastError();
 }
 
 template <int EPI>
@@ -439,7 +859,7 @@ cudaError_t launch_impl(const GroupedGemmProblem& p, int num_sms, cudaStream_t s
   CUtensorMap tmA, tmB, tmS;
   if (!make_act_map(&tmA, p.A, p.P, p.K)) return cudaErrorInvalidValue;
   if (!make_code_map(&tmB, p.codes, p.E, p.Nrows, p.K)) return cudaErrorInvalidValue;
-  if (!make_scale_map(&tmS, p.scales_t, p.E, p.Nrows, p.K)) return cudaErrorInvalidValue;
+  if (!make_scale_map(&tmS, p.scales_t, p.E, p.Nrows, p.K, NH)) return cudaErrorInvalidValue;
   Args a;
   a.offsets = p.offsets;
   a.mprefix = p.mprefix;
@@ -472,10 +892,12 @@ cudaError_t launch_impl(const GroupedGemmProblem& p, int num_sms, cudaStream_t s
 }  // namespace
 
 cudaError_t launch_gemm_gateup_swiglu(const GroupedGemmProblem& p, int num_sms, cudaStream_t st) {
+  if (p.use_pair) return launch_pair_impl<EPI_SWIGLU>(p, num_sms, st);
   return launch_impl<EPI_SWIGLU>(p, num_sms, st);
 }
 
 cudaError_t launch_gemm_down_combine(const GroupedGemmProblem& p, int num_sms, cudaStream_t st) {
+  if (p.use_pair) return launch_pair_impl<EPI_DOWN>(p, num_sms, st);
   return launch_impl<EPI_DOWN>(p, num_sms, st);
 }
 

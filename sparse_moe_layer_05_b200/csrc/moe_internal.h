@@ -60,6 +60,7 @@ struct GroupedGemmProblem {
   const float* topk_w;      // down: weight of each pair
   int n_out;                // output columns (I for SwiGLU, d for down)
   int* status;
+  bool use_pair;            // CTA-pair (2-SM) tiles instead of single-CTA tiles
 };
 cudaError_t launch_gemm_gateup_swiglu(const GroupedGemmProblem& p, int num_sms, cudaStream_t st);
 cudaError_t launch_gemm_down_combine(const GroupedGemmProblem& p, int num_sms, cudaStream_t st);

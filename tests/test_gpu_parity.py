@@ -157,6 +157,38 @@ def test_forward_matches_oracle(case):
             assert np.all(np.abs(rows - h) <= bound), (e, np.max(np.abs(rows - h) / (bound)))
 
 
+PAIR_CASES = [
+    # name, d, I, E, k, T, seed -- experts with hundreds of rows, ragged tails
+    ("pair_ragged", 352, 224, 4, 2, 1500, 31),
+    ("pair_wide", 2880, 2880, 8, 2, 1100, 32),
+    ("pair_short_tail", 128, 256, 6, 3, 700, 33),
+]
+
+
+@pytest.mark.parametrize("policy", [1, 2], ids=["single", "pair"])
+@pytest.mark.parametrize("case", PAIR_CASES, ids=[c[0] for c in PAIR_CASES])
+def test_forward_both_tile_policies(case, policy):
+    from sparse_moe_layer_05_b200 import binding as B
+    name, d, I, E, k, T, seed = case
+    inp = W.make_custom(d, I, E, k, T, seed=seed)
+    B.moe_set_tile_policy(policy)
+    try:
+        out, layer = G.run_forward(inp)
+        assert B.moe_sync_status(layer.workspace) == 0
+    finally:
+        B.moe_set_tile_policy(0)
+    want, r, hidden = O.moe_forward(inp.x, inp.W_r, inp.b_r, inp.Wgu_codes, inp.Wgu_scales,
+                                    inp.Wd_codes, inp.Wd_scales, k=k, return_hidden=True)
+    G.assert_out_close(out, want)
+    idx = layer.intermediate("topk_idx", T).cpu().numpy()
+    if np.array_equal(idx, r.idx):
+        c, o, p, _ = O.routing_tables(idx, E)
+        H = O.bf16_to_f64(G.unpermute_chunks(layer.intermediate("h", T).cpu().numpy()))
+        for e, (toks, h) in hidden.items():
+            rms = np.sqrt(np.mean(h ** 2))
+            assert np.all(np.abs(H[o[e]:o[e + 1]] - h) <= 2.0 ** -8 * np.abs(h) + 1e-3 * rms), e
+
+
 def test_forward_deterministic_and_hostio_equal():
     from sparse_moe_layer_05_b200.binding import MoELayer
     inp = W.make_custom(352, 224, 8, 2, 600, seed=12)
