@@ -176,6 +176,31 @@ MOE_API moe_status moe_route(const void* x_dev, const float* W_r_dev, const floa
                      void* workspace_dev, size_t workspace_bytes, void* stream);
 
 /*
+ * moe_route without a workspace, for callers that cannot allocate device
+ * memory: code that is handed only its inputs, outputs and a stream (plugin
+ * hooks of inference runtimes, serving threads that must not call cudaMalloc,
+ * which can synchronise the device and can fail under memory pressure). The
+ * pages have no counterpart to this entry point; it is a deployment aid.
+ *
+ * Same arguments, outputs and results as moe_route (all five outputs are
+ * required here), minus the workspace. The scratch it needs (router logits
+ * and small routing tables) lives in one device array owned by the library:
+ * about 4.1 MiB that every GPU which loads the library holds until the
+ * process exits. Limit: T * E <= 1,048,576 (e.g. T = 8192 tokens at E = 128,
+ * or T = 4096 at E = 248); larger calls return MOE_ERR_UNSUPPORTED and
+ * launch nothing. The first call on a device looks up the array's device
+ * address (cudaGetSymbolAddress, with that device current); make that first
+ * call before any stream capture. All calls on a device share the array and
+ * it keeps the last call's contents (each call rewrites what it reads), so
+ * calls whose device work overlaps -- concurrent streams, or several host
+ * threads -- race on it; serialise them.
+ */
+MOE_API moe_status moe_route_noalloc(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
+                                     int E, int k, int T, int d, int32_t* topk_idx_dev,
+                                     float* topk_w_dev, int32_t* counts_dev,
+                                     int32_t* offsets_dev, int32_t* perm_dev, void* stream);
+
+/*
  * Where moe_forward keeps its intermediates inside the workspace (byte
  * offsets from the workspace base), so that a caller can read them after a
  * call for inspection: logits [T][E] f32, topk_idx [T][k] i32, topk_w [T][k]

@@ -29,7 +29,7 @@ EXPORTS = [
     "moe_workspace_size_hostio", "moe_forward_hostio", "moe_route_workspace_size",
     "moe_route", "moe_workspace_layout", "moe_mxfp4_to_bf16", "moe_sync_status",
     "moe_selftest_wait_timeout", "moe_forward_launch_count", "moe_forward_timed",
-    "moe_set_tile_policy",
+    "moe_set_tile_policy", "moe_route_noalloc",
 ]
 
 STAGES = ["router_logits", "topk_softmax", "perm_hist", "perm_scan", "perm_scatter",
@@ -81,6 +81,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_forward_timed.argtypes = fwd + [ctypes.POINTER(ctypes.c_float)]
     lib.moe_route.restype = i32
     lib.moe_route.argtypes = [vp, fp, fp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.moe_route_noalloc.restype = i32
+    lib.moe_route_noalloc.argtypes = [vp, fp, fp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]
     lib.moe_workspace_layout.restype = i32
     lib.moe_workspace_layout.argtypes = [i32] * 5 + [ctypes.POINTER(WsLayout)]
     lib.moe_mxfp4_to_bf16.restype = i32
@@ -191,6 +193,16 @@ def moe_route(x, W_r, b_r, E, k, T, d, topk_idx, topk_w, counts=None, offsets=No
     _check("moe_route", load().moe_route(
         _ptr(x), _ptr(W_r), _ptr(b_r), E, k, T, d, _ptr(topk_idx), _ptr(topk_w), _ptr(counts),
         _ptr(offsets), _ptr(perm), _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def moe_route_noalloc(x, W_r, b_r, E, k, T, d, topk_idx, topk_w, counts, offsets, perm,
+                      stream=None) -> None:
+    """moe_route with the library's own fixed device scratch (no workspace):
+    for callers that cannot allocate; T * E <= 1,048,576."""
+    _require_cuda(x, W_r, b_r, topk_idx, topk_w, counts, offsets, perm)
+    _check("moe_route_noalloc", load().moe_route_noalloc(
+        _ptr(x), _ptr(W_r), _ptr(b_r), E, k, T, d, _ptr(topk_idx), _ptr(topk_w), _ptr(counts),
+        _ptr(offsets), _ptr(perm), _stream(stream)))
 
 
 def moe_mxfp4_to_bf16(codes, scales, rows: int, K: int, out, stream=None) -> None:

@@ -1,0 +1,125 @@
+// moe_noalloc.cu -- moe_route_noalloc: the router + permutation entry point
+// for callers that cannot allocate device memory.
+//
+// Some callers of this library are handed only their inputs, their outputs
+// and a stream: plugin hooks of inference runtimes, or code on a serving
+// thread that must not call the device allocator (cudaMalloc can synchronise
+// the device and can fail under memory pressure, and such callers have no
+// workspace to offer). This file gives them one entry point whose scratch
+// memory lives in a fixed-size array in device global memory that the
+// library owns; it calls no allocator.
+//
+// The array is a file-scope __device__ variable: every GPU that loads this
+// library holds it, kNoAllocScratchBytes of device memory, until the process
+// exits. Host code cannot use the array's name as a device address, so the
+// first call on each device looks the address up once with
+// cudaGetSymbolAddress (with that device current) and caches it.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/moe_b200.h"
+#include "moe_internal.h"
+
+namespace {
+
+// Largest T * E accepted: the fp32 router logits take 4 bytes per
+// (token, expert); the rest of the scratch is small tables.
+constexpr size_t kNoAllocMaxTE = size_t(1) << 20;
+constexpr size_t kNoAllocScratchBytes = kNoAllocMaxTE * 4 + (size_t(64) << 10);
+constexpr int kMaxDevices = 64;
+
+__device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBytes];
+
+void* g_scratch_addr[kMaxDevices] = {nullptr};
+
+size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
+
+struct ScratchLayout {
+  size_t status, logits, mprefix, chunk_hist, chunk_base, total;
+};
+
+ScratchLayout scratch_layout(int E, int T) {
+  const size_t nb = static_cast<size_t>(moe::perm_chunks(T));
+  ScratchLayout L;
+  size_t off = 0;
+  L.status = off;
+  off = round256(off + 16);
+  L.mprefix = off;
+  off = round256(off + static_cast<size_t>(E + 1) * 4);
+  L.chunk_hist = off;
+  off = round256(off + nb * E * 4);
+  L.chunk_base = off;
+  off = round256(off + nb * E * 4);
+  L.logits = off;
+  off = round256(off + static_cast<size_t>(T) * E * 4);
+  L.total = off;
+  return L;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+// Device address of the scratch array on the current device (looked up once
+// per device).
+moe_status scratch_base(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return MOE_ERR_NO_DEVICE;
+  }
+  if (!g_scratch_addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+moe_status moe_route_noalloc(const void* x_dev, const float* W_r_dev, const float* b_r_dev, int E,
+                             int k, int T, int d, int32_t* topk_idx_dev, float* topk_w_dev,
+                             int32_t* counts_dev, int32_t* offsets_dev, int32_t* perm_dev,
+                             void* stream) {
+  if (!x_dev || !W_r_dev || !b_r_dev || !topk_idx_dev || !topk_w_dev || !counts_dev ||
+      !offsets_dev || !perm_dev)
+    return MOE_ERR_INVALID_ARG;
+  if (E < 1 || E > 256 || k < 1 || k > E || k > 32 || T < 0 || d < 32 || d > 16384 || d % 32)
+    return MOE_ERR_UNSUPPORTED;
+  if (static_cast<size_t>(T) * static_cast<size_t>(E) > kNoAllocMaxTE) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(x_dev) || !aligned16(W_r_dev) || !aligned16(b_r_dev)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  const ScratchLayout L = scratch_layout(E, T);
+  if (L.total > kNoAllocScratchBytes) return MOE_ERR_UNSUPPORTED;
+  void* base = nullptr;
+  moe_status s = scratch_base(&base);
+  if (s != MOE_OK) return s;
+  unsigned char* sb = static_cast<unsigned char*>(base);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* status = reinterpret_cast<int*>(sb + L.status);
+  float* logits = reinterpret_cast<float*>(sb + L.logits);
+  int32_t* mprefix = reinterpret_cast<int32_t*>(sb + L.mprefix);
+  int32_t* chunk_hist = reinterpret_cast<int32_t*>(sb + L.chunk_hist);
+  int32_t* chunk_base = reinterpret_cast<int32_t*>(sb + L.chunk_base);
+  // Every buffer below is fully written before it is read; the status word
+  // is cleared by the first kernel.
+  if (moe::launch_router_logits(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, logits, T,
+                                E, d, status, st) != cudaSuccess ||
+      moe::launch_topk_softmax(logits, T, E, k, topk_idx_dev, topk_w_dev, st) != cudaSuccess ||
+      moe::launch_perm_hist(topk_idx_dev, T, k, E, chunk_hist, st) != cudaSuccess ||
+      moe::launch_perm_scan(chunk_hist, moe::perm_chunks(T), E, counts_dev, offsets_dev,
+                            chunk_base, mprefix, st) != cudaSuccess ||
+      moe::launch_perm_scatter(topk_idx_dev, T, k, E, chunk_base, perm_dev, nullptr, st) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+}  // extern "C"
