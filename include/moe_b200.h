@@ -90,13 +90,13 @@ MOE_API const char* moe_status_string(moe_status s);
 MOE_API int moe_version(void);
 
 /*
- * Tile policy of the grouped GEMMs, process-wide: 0 (default) automatic --
- * currently single-CTA tiles (256 x 128, the second 128-row half skipped for
- * short expert tails), the faster on every measured shape; 1 forces
- * single-CTA tiles; 2 forces CTA-pair tiles (a 2-CTA cluster computes
- * 256 x 240 tiles with tcgen05 cta_group::2). Both compute the same function.
- * Not thread-safe against concurrent forward calls. MOE_ERR_INVALID_ARG for
- * other values.
+ * Tile policy of the grouped GEMMs, process-wide: 0 (default) picks by shape
+ * -- CTA-pair tiles (a 2-CTA cluster computes 256 x 240 tiles with tcgen05
+ * cta_group::2) when the experts average at least 192 routed rows, else
+ * single-CTA tiles (256 x 128, the second 128-row half skipped for short
+ * expert tails); 1 forces single-CTA tiles; 2 forces CTA-pair tiles. Both
+ * compute the same function. Not thread-safe against concurrent forward
+ * calls. MOE_ERR_INVALID_ARG for other values.
  */
 MOE_API moe_status moe_set_tile_policy(int policy);
 

@@ -350,11 +350,6 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
         const uint8_t* stage = smem + OFF_C + sc * C_BYTES;
         const uint4 q = *reinterpret_cast<const uint4*>(stage + n * 32 + g * 16);
         const uint32_t s = stage[soff];
-        // the next TMA write into this stage (async proxy) must not overtake
-        // these generic-proxy reads
-        fence_proxy_async_smem();
-        mbar_arrive(bar_emptyC(sc));
-        if (++sc == SC) { sc = 0; pc ^= 1; }
         uint4 o[4];
         mxfp4x32_to_bf16(q, s, o);
         if (!(ok = mbar_wait(bar_emptyB(sb), pb ^ 1, abort_flag, args.status))) break;
@@ -362,7 +357,13 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 4; ++c)
           *reinterpret_cast<uint4*>(brow + (((4 * g + c) ^ sw) << 4)) = o[c];
+        // One proxy fence orders this thread's generic-proxy accesses before
+        // the async proxy's next ones: the code-stage reads above (the next
+        // TMA write into that stage must not overtake them) and the
+        // decoded-weight writes (the UMMA must see them).
         fence_proxy_async_smem();
+        mbar_arrive(bar_emptyC(sc));
+        if (++sc == SC) { sc = 0; pc ^= 1; }
         mbar_arrive(bar_fullB(sb));
         if (++sb == SB) { sb = 0; pb ^= 1; }
       }
@@ -598,7 +599,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::NUM_THREADS, 1
         for (int kb = 0; kb < KB; ++kb) {
           if (!(ok = mbar_wait(bar_fullA(sa), pa, abort_flag, args.status))) break;
           if (!(ok = mbar_wait(bar_fullB(sb), pb, abort_flag, args.status))) break;
-          mbar_arrive_remote(mapa_shared(bar_peerFull(sb), 0));
+          // relaxed: a release at cluster scope per k-block cost about as much
+          // as the k-block itself; the stage was already observed complete
+          mbar_arrive_remote_relaxed(mapa_shared(bar_peerFull(sb), 0));
           if (++sa == SA) { sa = 0; pa ^= 1; }
           if (++sb == SB) { sb = 0; pb ^= 1; }
         }
@@ -694,11 +697,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::NUM_THREADS, 1
           q = *reinterpret_cast<const uint4*>(stage + n * 32 + g * 16);
           sv = stage[soff];
         }
-        // the next TMA write into this stage (async proxy) must not overtake
-        // these generic-proxy reads
-        fence_proxy_async_smem();
-        mbar_arrive(bar_emptyC(sc));
-        if (++sc == SC) { sc = 0; pc ^= 1; }
         uint4 o[4];
         mxfp4x32_to_bf16(q, sv, o);
         if (!(ok = mbar_wait_cluster(bar_emptyB(sb), pb ^ 1, abort_flag, args.status))) break;
@@ -708,7 +706,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::NUM_THREADS, 1
           for (int c = 0; c < 4; ++c)
             *reinterpret_cast<uint4*>(brow + (((4 * g + c) ^ sw) << 4)) = o[c];
         }
+        // one proxy fence for the code-stage reads and the decoded-weight
+        // writes (see the single-CTA kernel)
         fence_proxy_async_smem();
+        mbar_arrive(bar_emptyC(sc));
+        if (++sc == SC) { sc = 0; pc ^= 1; }
         mbar_arrive(bar_fullB(sb));
         if (++sb == SB) { sb = 0; pb ^= 1; }
       }

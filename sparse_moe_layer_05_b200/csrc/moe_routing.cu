@@ -16,73 +16,111 @@ namespace moe {
 namespace {
 
 // ------------------------------------------------------------ K1 logits ----
-// Block tile: 32 tokens x 64 experts, contraction in chunks of 32; each of the
-// 128 threads owns 4 tokens x 4 experts. Every logit is one fp32 accumulator
-// updated by fma in increasing contraction index, then the bias is added:
-// identical router rows therefore give bit-identical logits.
-constexpr int RT_T = 32, RT_E = 64, RT_K = 32;
+// Block tile: 32 tokens x BE experts (BE = 32 or 64). Four groups of threads
+// split the contraction: group q accumulates the 32-wide chunks q, q+4, q+8,
+// ... of d in increasing order, each thread holding 4 tokens x 4 experts in
+// fp32 (fma). At the end the four partial sums are added in the fixed order
+// ((g0 + g1) + g2) + g3, then the bias. Every logit of every expert follows
+// the same sequence of operations, so identical router rows give
+// bit-identical logits.
+constexpr int RT_T = 32, RT_K = 32, RT_G = 4;
 
-__global__ void __launch_bounds__(128) router_logits_kernel(const uint16_t* __restrict__ x,
-                                                            const float* __restrict__ W_r,
-                                                            const float* __restrict__ b_r,
-                                                            float* __restrict__ logits, int T,
-                                                            int E, int d, int* status) {
-  __shared__ __align__(16) float xs[RT_K][RT_T + 4];
-  __shared__ __align__(16) float ws[RT_K][RT_E + 4];
+template <int BE>
+struct RouterCfg {
+  static constexpr int TX = BE / 4;                 // expert groups of 4
+  static constexpr int TY = RT_T / 4;               // token groups of 4
+  static constexpr int GT = TX * TY;                // threads per k-group
+  static constexpr int THREADS = RT_G * GT;         // 128 (BE=32) or 256 (BE=64)
+  static constexpr int XS = RT_K * (RT_T + 4);      // floats per x chunk tile
+  static constexpr int WS = RT_K * (BE + 4);        // floats per W chunk tile
+  static constexpr int SMEM = RT_G * (XS + WS) * 4;
+};
+
+template <int BE>
+__global__ void __launch_bounds__(RouterCfg<BE>::THREADS)
+    router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W_r,
+                         const float* __restrict__ b_r, float* __restrict__ logits, int T, int E,
+                         int d, int* status) {
+  using C = RouterCfg<BE>;
+  extern __shared__ __align__(16) float rsm[];
   const int tid = threadIdx.x;
   if (status && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *status = 0;
-  const int t0 = blockIdx.x * RT_T, e0 = blockIdx.y * RT_E;
-  const int ty = tid >> 4, tx = tid & 15;
+  const int t0 = blockIdx.x * RT_T, e0 = blockIdx.y * BE;
+  const int grp = tid / C::GT, lt = tid % C::GT;
+  const int ty = lt / C::TX, tx = lt % C::TX;
+  float* xs = rsm + grp * (C::XS + C::WS);        // [RT_K][RT_T + 4]
+  float* ws = xs + C::XS;                          // [RT_K][BE + 4]
   float acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 
-  for (int k0 = 0; k0 < d; k0 += RT_K) {
-    {  // activations: 32 tokens x 32 bf16, 16 bytes per thread
-      const int tt = tid >> 2, kk = (tid & 3) * 8, t = t0 + tt;
+  const int nch = d / RT_K;
+  for (int c0 = 0; c0 < nch; c0 += RT_G) {
+    // all threads stage the (up to) four chunks c0..c0+3, one per group
+    for (int i = tid; i < RT_G * RT_T * 4; i += C::THREADS) {   // x: 16 bytes per item
+      const int g = i / (RT_T * 4), r = i % (RT_T * 4);
+      const int tt = r >> 2, kk = (r & 3) * 8, t = t0 + tt, c = c0 + g;
       uint4 v = make_uint4(0, 0, 0, 0);
-      if (t < T) v = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d + k0 + kk));
+      if (t < T && c < nch) v = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d + c * RT_K + kk));
+      float* xg = rsm + g * (C::XS + C::WS);
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        xs[kk + 2 * i][tt] = __uint_as_float(w[i] << 16);
-        xs[kk + 2 * i + 1][tt] = __uint_as_float(w[i] & 0xFFFF0000u);
+      for (int u = 0; u < 4; ++u) {
+        xg[(kk + 2 * u) * (RT_T + 4) + tt] = __uint_as_float(w[u] << 16);
+        xg[(kk + 2 * u + 1) * (RT_T + 4) + tt] = __uint_as_float(w[u] & 0xFFFF0000u);
       }
     }
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {  // router rows: 64 experts x 32 fp32
-      const int idx = tid + r * 128, ee = idx >> 3, kk = (idx & 7) * 4, e = e0 + ee;
+    for (int i = tid; i < RT_G * BE * 8; i += C::THREADS) {     // W: 16 bytes per item
+      const int g = i / (BE * 8), r = i % (BE * 8);
+      const int ee = r >> 3, kk = (r & 7) * 4, e = e0 + ee, c = c0 + g;
       float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e < E) v = __ldg(reinterpret_cast<const float4*>(W_r + (size_t)e * d + k0 + kk));
-      ws[kk + 0][ee] = v.x;
-      ws[kk + 1][ee] = v.y;
-      ws[kk + 2][ee] = v.z;
-      ws[kk + 3][ee] = v.w;
+      if (e < E && c < nch) v = __ldg(reinterpret_cast<const float4*>(W_r + (size_t)e * d + c * RT_K + kk));
+      float* wg = rsm + g * (C::XS + C::WS) + C::XS;
+      wg[(kk + 0) * (BE + 4) + ee] = v.x;
+      wg[(kk + 1) * (BE + 4) + ee] = v.y;
+      wg[(kk + 2) * (BE + 4) + ee] = v.z;
+      wg[(kk + 3) * (BE + 4) + ee] = v.w;
     }
     __syncthreads();
+    if (c0 + grp < nch) {
 #pragma unroll 8
-    for (int kk = 0; kk < RT_K; ++kk) {
-      const float4 a = *reinterpret_cast<const float4*>(&xs[kk][ty * 4]);
-      const float4 b = *reinterpret_cast<const float4*>(&ws[kk][tx * 4]);
-      const float av[4] = {a.x, a.y, a.z, a.w};
-      const float bv[4] = {b.x, b.y, b.z, b.w};
+      for (int kk = 0; kk < RT_K; ++kk) {
+        const float4 a = *reinterpret_cast<const float4*>(&xs[kk * (RT_T + 4) + ty * 4]);
+        const float4 b = *reinterpret_cast<const float4*>(&ws[kk * (BE + 4) + tx * 4]);
+        const float av[4] = {a.x, a.y, a.z, a.w};
+        const float bv[4] = {b.x, b.y, b.z, b.w};
 #pragma unroll
-      for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+      }
     }
     __syncthreads();
   }
+  // fixed-order combination of the four groups' partial sums
+  float* red = rsm;  // [RT_G - 1][RT_T][BE]
+  if (grp > 0) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int t = t0 + ty * 4 + i;
-    if (t >= T) continue;
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = e0 + tx * 4 + j;
-      if (e < E) logits[(size_t)t * E + e] = acc[i][j] + b_r[e];
+      for (int j = 0; j < 4; ++j)
+        red[((grp - 1) * RT_T + ty * 4 + i) * BE + tx * 4 + j] = acc[i][j];
+  }
+  __syncthreads();
+  if (grp == 0) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = t0 + ty * 4 + i;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int e = e0 + tx * 4 + j;
+        float v = acc[i][j];
+#pragma unroll
+        for (int g = 0; g < RT_G - 1; ++g) v += red[(g * RT_T + ty * 4 + i) * BE + tx * 4 + j];
+        if (t < T && e < E) logits[(size_t)t * E + e] = v + b_r[e];
+      }
     }
   }
 }
@@ -321,24 +359,41 @@ __global__ void __launch_bounds__(256) mxfp4_to_bf16_kernel(const uint8_t* __res
 }
 
 // -------------------------------------------------- scale transpose ----
-// [E][N][G] -> [E][G][N], through a 32 x 32 shared tile.
+// [E][N][G] -> [E][G][N]. A block takes 64 consecutive rows n (64*G
+// contiguous bytes), stages them in shared memory and writes, for every group
+// g, the 64 bytes out[g][n0 .. n0+63] as four 16-byte stores. N is a multiple
+// of 32, so full 64-row blocks store whole vectors; the last block of an
+// expert may hold 32 rows.
+constexpr int TR_ROWS = 64;
+
 __global__ void __launch_bounds__(256) transpose_scales_kernel(const uint8_t* __restrict__ in,
                                                                int N, int G,
                                                                uint8_t* __restrict__ out) {
-  __shared__ uint8_t tile[32][33];
-  const int e = blockIdx.z;
-  const int n0 = blockIdx.x * 32, g0 = blockIdx.y * 32;
-  const uint8_t* src = in + (size_t)e * N * G;
-  uint8_t* dst = out + (size_t)e * N * G;
-  const int tx = threadIdx.x & 31, ty = threadIdx.x >> 5;
-  for (int r = ty; r < 32; r += 8) {
-    const int n = n0 + r, g = g0 + tx;
-    if (n < N && g < G) tile[r][tx] = src[(size_t)n * G + g];
+  extern __shared__ __align__(16) uint8_t tsm[];  // [TR_ROWS][G]
+  const int e = blockIdx.y;
+  const int n0 = blockIdx.x * TR_ROWS;
+  const int rows = min(TR_ROWS, N - n0);
+  const uint8_t* src = in + ((size_t)e * N + n0) * G;
+  const int bytes = rows * G;
+  if ((reinterpret_cast<uintptr_t>(src) & 15) == 0 && (bytes & 15) == 0) {
+    for (int i = threadIdx.x; i < bytes / 16; i += blockDim.x)
+      reinterpret_cast<uint4*>(tsm)[i] = __ldg(reinterpret_cast<const uint4*>(src) + i);
+  } else {
+    for (int i = threadIdx.x; i < bytes; i += blockDim.x) tsm[i] = src[i];
   }
   __syncthreads();
-  for (int r = ty; r < 32; r += 8) {
-    const int g = g0 + r, n = n0 + tx;
-    if (n < N && g < G) dst[(size_t)g * N + n] = tile[tx][r];
+  uint8_t* dst = out + (size_t)e * N * G + n0;
+  const int vecs = rows / 16;
+  for (int i = threadIdx.x; i < G * vecs; i += blockDim.x) {
+    const int g = i / vecs, v = i % vecs;
+    uint32_t w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int r = v * 16 + q * 4;
+      w[q] = (uint32_t)tsm[(r + 0) * G + g] | ((uint32_t)tsm[(r + 1) * G + g] << 8) |
+             ((uint32_t)tsm[(r + 2) * G + g] << 16) | ((uint32_t)tsm[(r + 3) * G + g] << 24);
+    }
+    *reinterpret_cast<uint4*>(dst + (size_t)g * N + v * 16) = make_uint4(w[0], w[1], w[2], w[3]);
   }
 }
 
@@ -366,12 +421,29 @@ int grid_for(int64_t n, int per_block, int cap) {
 
 }  // namespace
 
+template <int BE>
+cudaError_t launch_router_be(const uint16_t* x, const float* W_r, const float* b_r, float* logits,
+                             int T, int E, int d, int* status, cudaStream_t st) {
+  using C = RouterCfg<BE>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(router_logits_kernel<BE>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  dim3 grid((T + RT_T - 1) / RT_T, (E + BE - 1) / BE);
+  router_logits_kernel<BE><<<grid, C::THREADS, C::SMEM, st>>>(x, W_r, b_r, logits, T, E, d, status);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, const float* b_r,
                                  float* logits, int T, int E, int d, int* status,
                                  cudaStream_t st) {
-  dim3 grid((T + RT_T - 1) / RT_T, (E + RT_E - 1) / RT_E);
-  router_logits_kernel<<<grid, 128, 0, st>>>(x, W_r, b_r, logits, T, E, d, status);
-  return cudaGetLastError();
+  if (E <= 32) return launch_router_be<32>(x, W_r, b_r, logits, T, E, d, status, st);
+  return launch_router_be<64>(x, W_r, b_r, logits, T, E, d, status, st);
 }
 
 cudaError_t launch_topk_softmax(const float* logits, int T, int E, int k, int32_t* topk_idx,
@@ -416,8 +488,9 @@ cudaError_t launch_combine(const float* yw, int T, int k, int d, uint16_t* out,
 
 cudaError_t launch_transpose_scales(const uint8_t* in, int E, int N, int G, uint8_t* out,
                                     cudaStream_t st) {
-  dim3 grid((N + 31) / 32, (G + 31) / 32, E);
-  transpose_scales_kernel<<<grid, 256, 0, st>>>(in, N, G, out);
+  const int smem = TR_ROWS * G;  // G <= 512 (K <= 16384): at most 32 KB
+  dim3 grid((N + TR_ROWS - 1) / TR_ROWS, E);
+  transpose_scales_kernel<<<grid, 256, smem, st>>>(in, N, G, out);
   return cudaGetLastError();
 }
 
