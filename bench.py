@@ -38,7 +38,7 @@ L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DOMINANT_STAGE = "gemm_gateup_swiglu"
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
-KERNEL_SOURCES = ["moe_grouped_gemm.cu", "moe_ptx.cuh"]
+KERNEL_SOURCES = ["moe_grouped_gemm.cu", "moe_ptx.cuh", "moe_abi.cu"]
 
 
 # ------------------------------------------------------------ host logic ----
@@ -93,14 +93,14 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
+def recorded_traffic(workload: str, T: int):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
     summary, if it was taken on the current kernel source; else None."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
         d = json.load(f)
-    ent = d.get(workload)
+    ent = d.get(f"{workload}:T={T}")
     if not ent or ent.get("source_hash") != kernel_source_hash():
         return None
     return ent.get("bytes_per_launch")
@@ -312,9 +312,24 @@ def run_ours(args, inp, name):
     dom_ms = sum(s[dom] for s in stage_ms) / len(stage_ms)
     dom_flops = 4.0 * inp.d * inp.I * T * inp.k
     peaks, kind = load_peaks()
-    peak = float(peaks["bf16_tflops"])
-    achieved = dom_flops / (dom_ms * 1e-3) / 1e12
     stage_avg = {n: sum(s[i] for s in stage_ms) / len(stage_ms) for i, n in enumerate(B.STAGES)}
+    counts = layer.intermediate("counts", T).cpu().numpy()
+    touched = int((counts > 0).sum())
+    # algorithmic bytes of one gate/up launch: the touched experts' MXFP4
+    # gate/up weights (codes + scales), the permuted activations read, H written
+    dom_bytes = (touched * (2 * inp.I * inp.d // 2 + 2 * inp.I * inp.d // 32)
+                 + T * inp.k * inp.d * 2 + T * inp.k * inp.I * 2)
+    decode = T * inp.k < 16 * inp.E       # few rows per expert: weight streaming
+    if decode:
+        peak = float(peaks["hbm_gbs"])
+        achieved = dom_bytes / (dom_ms * 1e-3) / 1e9
+        roof = {"bound": "hbm", "unit": "GB/s", "peak_source": f"hbm_gbs ({kind})",
+                "algorithmic_bytes_per_launch": dom_bytes}
+    else:
+        peak = float(peaks["bf16_tflops"])
+        achieved = dom_flops / (dom_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "unit": "TFLOP/s", "peak_source": f"bf16_tflops ({kind}, burst)",
+                "algorithmic_flops_per_launch": dom_flops}
 
     # end to end through the C ABI with host buffers: H2D + forward + D2H
     e2e_s = 0.0
@@ -341,14 +356,9 @@ def run_ours(args, inp, name):
         "config": workload_config(inp, name),
         "layer_tflops": layer_flops(inp.d, inp.I, inp.E, inp.k, T) * args.steps * world
         / step_s_max / 1e12,
-        "roofline": {
-            "bound": "tensor", "kernel": DOMINANT_STAGE, "achieved": achieved, "peak": peak,
-            "unit": "TFLOP/s", "frac": achieved / peak,
-            "peak_source": f"bf16_tflops ({kind}, burst)",
-            "traffic": recorded_traffic(name),
-            "algorithmic_flops_per_launch": dom_flops,
-            "avg_launch_ms": dom_ms,
-        },
+        "roofline": dict(roof, kernel=DOMINANT_STAGE, achieved=achieved, peak=peak,
+                         frac=achieved / peak, traffic=recorded_traffic(name, T),
+                         avg_launch_ms=dom_ms, touched_experts=touched),
         "stage_ms": stage_avg,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(T * inp.d * 2),
                 "d2h_bytes_per_step": int(T * inp.d * 2)},
