@@ -91,10 +91,14 @@ MOE_API int moe_version(void);
 
 /*
  * Tile policy of the grouped GEMMs, process-wide: 0 (default) picks by shape
- * -- CTA-pair tiles (a 2-CTA cluster computes 256 x 240 tiles with tcgen05
- * cta_group::2) when the experts average at least 192 routed rows, else
- * single-CTA tiles (256 x 128, the second 128-row half skipped for short
- * expert tails); 1 forces single-CTA tiles; 2 forces CTA-pair tiles. Both
+ * from the average number of routed rows per expert, P/E with P = T*k:
+ *   P/E < 32        swapped-operand tiles (128 weight rows x 64 tokens, the
+ *                   decoded weights as the UMMA A operand; decode batches),
+ *   32 <= P/E < 192 single-CTA tiles (256 x 128, the second 128-row half
+ *                   skipped for short expert tails),
+ *   P/E >= 192      CTA-pair tiles (a 2-CTA cluster computes 256 x 240 tiles
+ *                   with tcgen05 cta_group::2).
+ * 1, 2 and 3 force single-CTA, CTA-pair and swapped-operand tiles. All
  * compute the same function. Not thread-safe against concurrent forward
  * calls. MOE_ERR_INVALID_ARG for other values.
  */

@@ -13,16 +13,19 @@ constexpr int kVersion = 100;  // 0.1.0
 constexpr int kMaxDevices = 64;
 
 // Grouped-GEMM tile policy: 0 = choose by shape, 1 = single-CTA tiles,
-// 2 = CTA-pair tiles.
+// 2 = CTA-pair tiles, 3 = swapped-operand tiles.
 int g_tile_policy = 0;
 
-bool use_pair_tiles(int P, int E) {
-  if (g_tile_policy == 1) return false;
-  if (g_tile_policy == 2) return true;
-  // CTA-pair tiles (256 rows per tile, no half-tile skipping) measured faster
-  // down to 256 routed rows per expert on average; below ~192 the single-CTA
-  // tiles, which skip empty 128-row halves, are kept.
-  return static_cast<int64_t>(P) >= 192 * static_cast<int64_t>(E);
+int choose_tiles(int P, int E) {
+  if (g_tile_policy >= 1 && g_tile_policy <= 3) return g_tile_policy;
+  const int64_t p = P, e = E;
+  // Few routed rows per expert (decode): stream the weights with the
+  // swapped-operand kernel. From ~192 rows per expert the CTA-pair tiles were
+  // measured fastest; in between the single-CTA tiles, which skip empty
+  // 128-row halves.
+  if (p < 32 * e) return moe::TILES_SWAP;
+  if (p >= 192 * e) return moe::TILES_PAIR;
+  return moe::TILES_SINGLE;
 }
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
@@ -200,9 +203,9 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   E_.mark(5);
   MOE_CUDA(moe::launch_gather_rows(x, perm, P, k, d, xp, st));
   E_.mark(6);
-  MOE_CUDA(moe::launch_transpose_scales(gs, E, 2 * I, d / 32, gst, st));
+  MOE_CUDA(moe::launch_transpose_scales(gs, E, 2 * I, d / 32, counts, gst, st));
   E_.mark(7);
-  MOE_CUDA(moe::launch_transpose_scales(ds, E, d, I / 32, dst_, st));
+  MOE_CUDA(moe::launch_transpose_scales(ds, E, d, I / 32, counts, dst_, st));
   E_.mark(8);
 
   moe::GroupedGemmProblem g1;
@@ -221,7 +224,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   g1.topk_w = nullptr;
   g1.n_out = I;
   g1.status = status;
-  g1.use_pair = use_pair_tiles(P, E);
+  g1.tiles = choose_tiles(P, E);
   MOE_CUDA(moe::launch_gemm_gateup_swiglu(g1, num_sms, st));
   E_.mark(9);
 
@@ -263,7 +266,7 @@ const char* moe_status_string(moe_status s) {
 int moe_version(void) { return kVersion; }
 
 moe_status moe_set_tile_policy(int policy) {
-  if (policy < 0 || policy > 2) return MOE_ERR_INVALID_ARG;
+  if (policy < 0 || policy > 3) return MOE_ERR_INVALID_ARG;
   g_tile_policy = policy;
   return MOE_OK;
 }

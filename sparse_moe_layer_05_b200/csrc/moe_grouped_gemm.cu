@@ -726,6 +726,307 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::NUM_THREADS, 1
   }
 }
 
+// ================================================================= swap ====
+// Decode-sized variant (few routed rows per expert): the operands swap roles.
+// The decoded weight tile is the UMMA A operand (M = 128 weight rows) and the
+// expert's routed rows are B (N = 64 tokens), so the tensor work follows the
+// actual token count instead of a 128/256-row tile, and the kernel streams
+// weights. For gate/up a tile holds 64 gate rows and the matching 64 up rows
+// interleaved (gate j at row 2j, up j at row 2j+1), so the SwiGLU epilogue
+// pairs adjacent TMEM lanes with one shuffle. Each CTA builds its tile table
+// (expert, weight block, token block) from the device offsets; experts with
+// no tokens cost nothing.
+namespace swp {
+
+constexpr int MW = 128;               // weight rows per tile (UMMA M)
+constexpr int NT = 64;                // tokens per tile (UMMA N)
+constexpr int BK = 64;
+constexpr int NH = 64;                // weight rows per TMA box
+constexpr int ST = 4, SW = 4, SC = 12;
+constexpr int T_BYTES = NT * BK * 2;        // 8192
+constexpr int W_BYTES = MW * BK * 2;        // 16384
+constexpr int C_CODES = MW * BK / 2;        // 4096
+constexpr int S_OFF0 = C_CODES, S_OFF1 = C_CODES + 128;
+constexpr int C_TX = C_CODES + 2 * NH * 2;
+constexpr int C_BYTES = 4352;
+constexpr int NUM_THREADS = 512;
+constexpr int DEQ_THREADS = 256;
+constexpr int TMEM_COLS = 128;
+
+constexpr int OFF_W = 0;
+constexpr int OFF_T = OFF_W + SW * W_BYTES;
+constexpr int OFF_C = OFF_T + ST * T_BYTES;
+constexpr int OFF_BAR = OFF_C + SC * C_BYTES;
+constexpr int NUM_BARS = 2 * ST + 2 * SW + 2 * SC + 4;
+constexpr int OFF_MISC = (OFF_BAR + NUM_BARS * 8 + 15) & ~15;
+constexpr int OFF_TAB = OFF_MISC + 16;
+constexpr int SMEM_BYTES = OFF_TAB + 2 * (MAX_E + 1) * 4;
+constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
+static_assert(OFF_T % 1024 == 0 && OFF_C % 1024 == 0, "alignment");
+
+}  // namespace swp
+
+// position of element e (0..7) inside a chunk stored in kPerm8 order
+__device__ __forceinline__ int perm8_pos(int e) { return e < 4 ? 2 * e : 2 * (e - 4) + 1; }
+
+template <int EPI>
+__global__ void __launch_bounds__(swp::NUM_THREADS, 1)
+    grouped_mxfp4_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmA,
+                                   const __grid_constant__ CUtensorMap tmB,
+                                   const __grid_constant__ CUtensorMap tmS, const Args args) {
+  // local copies shadow the single-CTA kernel's constants of the same names
+  constexpr int MW = swp::MW, NT = swp::NT, BK = swp::BK, NH = swp::NH;
+  constexpr int ST = swp::ST, SW = swp::SW, SC = swp::SC;
+  constexpr int T_BYTES = swp::T_BYTES, W_BYTES = swp::W_BYTES, C_BYTES = swp::C_BYTES;
+  constexpr int C_TX = swp::C_TX, S_OFF0 = swp::S_OFF0, S_OFF1 = swp::S_OFF1;
+  constexpr int OFF_W = swp::OFF_W, OFF_T = swp::OFF_T, OFF_C = swp::OFF_C;
+  constexpr int OFF_BAR = swp::OFF_BAR, OFF_MISC = swp::OFF_MISC, OFF_TAB = swp::OFF_TAB;
+  constexpr int NUM_THREADS = swp::NUM_THREADS, DEQ_THREADS = swp::DEQ_THREADS;
+  constexpr int TMEM_COLS = swp::TMEM_COLS;
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const uint32_t bar0 = sbase + OFF_BAR;
+  auto bar_fullT = [&](int s) { return bar0 + 8u * s; };
+  auto bar_emptyT = [&](int s) { return bar0 + 8u * (ST + s); };
+  auto bar_fullW = [&](int s) { return bar0 + 8u * (2 * ST + s); };
+  auto bar_emptyW = [&](int s) { return bar0 + 8u * (2 * ST + SW + s); };
+  auto bar_fullC = [&](int s) { return bar0 + 8u * (2 * ST + 2 * SW + s); };
+  auto bar_emptyC = [&](int s) { return bar0 + 8u * (2 * ST + 2 * SW + SC + s); };
+  auto bar_accFull = [&](int s) { return bar0 + 8u * (2 * ST + 2 * SW + 2 * SC + s); };
+  auto bar_accEmpty = [&](int s) { return bar0 + 8u * (2 * ST + 2 * SW + 2 * SC + 2 + s); };
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  int* s_off = reinterpret_cast<int*>(smem + OFF_TAB);
+  int* s_tp = s_off + (MAX_E + 1);   // prefix of tiles per expert
+
+  const int E = args.E;
+  for (int i = threadIdx.x; i <= E; i += NUM_THREADS) s_off[i] = args.offsets[i];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    int acc = 0;
+    for (int e = 0; e < E; ++e) {
+      s_tp[e] = acc;
+      const int cnt = s_off[e + 1] - s_off[e];
+      acc += ((cnt + NT - 1) / NT) * args.n_tiles;
+    }
+    s_tp[E] = acc;
+    for (int s = 0; s < ST; ++s) {
+      mbar_init(bar_fullT(s), 1);
+      mbar_init(bar_emptyT(s), 1);
+    }
+    for (int s = 0; s < SW; ++s) {
+      mbar_init(bar_fullW(s), DEQ_THREADS);
+      mbar_init(bar_emptyW(s), 1);
+    }
+    for (int s = 0; s < SC; ++s) {
+      mbar_init(bar_fullC(s), 1);
+      mbar_init(bar_emptyC(s), DEQ_THREADS);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(bar_accFull(s), 1);
+      mbar_init(bar_accEmpty(s), 4 * 32);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmS);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(misc), TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = misc[0];
+
+  const int total = s_tp[E];
+  const int KB = (args.K + BK - 1) / BK;
+  // tile -> (expert, weight block, token block); tiles of an expert are
+  // weight-block major so that consecutive CTAs stream consecutive weights
+  auto decode = [&](int tile, int& e, int& wb, int& row0, int& rows) {
+    int lo = 0, hi = E;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_tp[mid] <= tile) lo = mid; else hi = mid;
+    }
+    e = lo;
+    const int cnt = s_off[e + 1] - s_off[e];
+    const int ntb = (cnt + NT - 1) / NT;
+    const int local = tile - s_tp[e];
+    wb = local / ntb;
+    const int tb = local % ntb;
+    row0 = s_off[e] + tb * NT;
+    rows = min(NT, cnt - tb * NT);
+  };
+  if (warp == 3) return;  // no role
+
+  if (warp == 0) {
+    // ------------------------------------------------ producer: tokens --
+    if (lane == 0) {
+      int st = 0, pt = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int e, wb, row0, rows;
+        decode(tile, e, wb, row0, rows);
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!(ok = mbar_wait(bar_emptyT(st), pt ^ 1, abort_flag, args.status))) break;
+          mbar_expect_tx(bar_fullT(st), T_BYTES);
+          tma_load_2d(sbase + OFF_T + st * T_BYTES, &tmA, kb * BK, row0, bar_fullT(st));
+          if (++st == ST) { st = 0; pt ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // --------------------------------------- producer: codes and scales --
+    if (lane == 0) {
+      int sc = 0, pc = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int e, wb, row0, rows;
+        decode(tile, e, wb, row0, rows);
+        const int rA = wb * args.row_step;
+        const int rB = rA + args.half_off;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!(ok = mbar_wait(bar_emptyC(sc), pc ^ 1, abort_flag, args.status))) break;
+          const uint32_t cdst = sbase + OFF_C + sc * C_BYTES;
+          mbar_expect_tx(bar_fullC(sc), C_TX);
+          tma_load_3d(cdst, &tmB, kb * (BK / 2), rA, e, bar_fullC(sc));
+          tma_load_3d(cdst + NH * (BK / 2), &tmB, kb * (BK / 2), rB, e, bar_fullC(sc));
+          tma_load_3d(cdst + S_OFF0, &tmS, rA, 2 * kb, e, bar_fullC(sc));
+          tma_load_3d(cdst + S_OFF1, &tmS, rB, 2 * kb, e, bar_fullC(sc));
+          if (++sc == SC) { sc = 0; pc ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------- UMMA issuer --
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(MW, NT);
+      int st = 0, pt = 0, sw = 0, pw = 0, it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+        const int ab = it & 1;
+        const uint32_t ap = (it >> 1) & 1;
+        if (!(ok = mbar_wait(bar_accEmpty(ab), ap ^ 1, abort_flag, args.status))) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + ab * NT;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!(ok = mbar_wait(bar_fullT(st), pt, abort_flag, args.status))) break;
+          if (!(ok = mbar_wait(bar_fullW(sw), pw, abort_flag, args.status))) break;
+          tc_fence_after();
+          const uint32_t w_addr = sbase + OFF_W + sw * W_BYTES;
+          const uint32_t t_addr = sbase + OFF_T + st * T_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / 16; ++kk)
+            umma_bf16(d, sdesc_k_sw128(w_addr + kk * 32), sdesc_k_sw128(t_addr + kk * 32), idesc,
+                      (kb | kk) != 0);
+          umma_commit(bar_emptyT(st));
+          umma_commit(bar_emptyW(sw));
+          if (++st == ST) { st = 0; pt ^= 1; }
+          if (++sw == SW) { sw = 0; pw ^= 1; }
+        }
+        if (ok) umma_commit(bar_accFull(ab));
+      }
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ----------------------------------------------------------- epilogue --
+    const int quad = warp & 3;
+    const int r = quad * 32 + lane;          // weight row of the tile = TMEM lane
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      int e, wb, row0, rows;
+      decode(tile, e, wb, row0, rows);
+      const int ab = it & 1;
+      const uint32_t ap = (it >> 1) & 1;
+      if (!mbar_wait(bar_accFull(ab), ap, abort_flag, args.status)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + ab * NT;
+#pragma unroll 1
+      for (int c = 0; c < NT && c < rows; c += 16) {
+        uint32_t y[16];
+        tmem_ld16_sync(taddr + c, y);
+        if (EPI == EPI_SWIGLU) {
+          // even lanes hold gate row j = r/2, odd lanes the up row j
+          const int j = wb * NH + (r >> 1);
+          const int col = (j & ~7) + perm8_pos(j & 7);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const float v = __uint_as_float(y[i]);
+            const float u = __shfl_xor_sync(0xFFFFFFFFu, v, 1);
+            if (!(lane & 1) && c + i < rows && j < args.n_out) {
+              const float h = silu_f(v) * u;
+              const __nv_bfloat16 hb = __float2bfloat16_rn(h);
+              args.out[static_cast<int64_t>(row0 + c + i) * args.n_out + col] =
+                  *reinterpret_cast<const uint16_t*>(&hb);
+            }
+          }
+        } else {
+          const int col = wb * MW + r;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if (c + i < rows) {
+              const int pr = args.perm[row0 + c + i];
+              const float w = args.topk_w[pr];
+              if (col < args.n_out)
+                args.out_f32[static_cast<int64_t>(pr) * args.n_out + col] =
+                    w * __uint_as_float(y[i]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_accEmpty(ab));
+    }
+  } else if (warp >= 8) {
+    // ----------------------------------------------------------- decoders --
+    const int t = threadIdx.x - 8 * 32;
+    const int n = t >> 1;            // box row: 0..63 first box, 64..127 second
+    const int g = t & 1;
+    const int soff = (n < NH ? S_OFF0 : S_OFF1) + g * NH + (n & (NH - 1));
+    // SwiGLU tiles interleave gate row j (first box) and up row j (second box)
+    const int orow = (EPI == EPI_SWIGLU) ? ((n < NH) ? 2 * n : 2 * (n - NH) + 1) : n;
+    const int swz = orow & 7;
+    int sc = 0, pc = 0, sw = 0, pw = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int kb = 0; kb < KB; ++kb) {
+        if (!(ok = mbar_wait(bar_fullC(sc), pc, abort_flag, args.status))) break;
+        const uint8_t* stage = smem + OFF_C + sc * C_BYTES;
+        const uint4 q = *reinterpret_cast<const uint4*>(stage + n * 32 + g * 16);
+        const uint32_t sv = stage[soff];
+        uint4 o[4];
+        mxfp4x32_to_bf16(q, sv, o);
+        if (!(ok = mbar_wait(bar_emptyW(sw), pw ^ 1, abort_flag, args.status))) break;
+        uint8_t* wrow = smem + OFF_W + sw * W_BYTES + orow * 128;
+#pragma unroll
+        for (int c = 0; c < 4; ++c)
+          *reinterpret_cast<uint4*>(wrow + (((4 * g + c) ^ swz) << 4)) = o[c];
+        // one proxy fence for the code-stage reads and the decoded-weight writes
+        fence_proxy_async_smem();
+        mbar_arrive(bar_emptyC(sc));
+        if (++sc == SC) { sc = 0; pc ^= 1; }
+        mbar_arrive(bar_fullW(sw));
+        if (++sw == SW) { sw = 0; pw ^= 1; }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
 // ----------------------------------------------------------- host side ----
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -797,6 +1098,60 @@ bool make_code_map_rows(CUtensorMap* m, const void* base, int E, int Nrows, int 
   const cuuint32_t box[3] = {BK / 2, static_cast<cuuint32_t>(rows), 1};
   return encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base, dims, strides, box,
                 CU_TENSOR_MAP_SWIZZLE_NONE);
+}
+
+// Activation rows [rows][K] bf16 as the swap kernel's B operand: box 64 x 64.
+bool make_tok_map(CUtensorMap* m, const void* base, int rows, int K) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K) * 2};
+  const cuuint32_t box[2] = {swp::BK, swp::NT};
+  return encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
+                CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+template <int EPI>
+cudaError_t launch_swap_impl(const GroupedGemmProblem& p, int num_sms, cudaStream_t st) {
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_mxfp4_gemm_swap_kernel<EPI>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         swp::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  CUtensorMap tmA, tmB, tmS;
+  if (!make_tok_map(&tmA, p.A, p.P, p.K)) return cudaErrorInvalidValue;
+  if (!make_code_map_rows(&tmB, p.codes, p.E, p.Nrows, p.K, swp::NH)) return cudaErrorInvalidValue;
+  if (!make_scale_map(&tmS, p.scales_t, p.E, p.Nrows, p.K, swp::NH)) return cudaErrorInvalidValue;
+  Args a;
+  a.offsets = p.offsets;
+  a.mprefix = p.mprefix;
+  a.E = p.E;
+  a.K = p.K;
+  a.Nrows = p.Nrows;
+  a.n_out = p.n_out;
+  a.out = p.out;
+  a.out_f32 = p.out_f32;
+  a.perm = p.perm;
+  a.topk_w = p.topk_w;
+  a.status = p.status;
+  if (EPI == EPI_SWIGLU) {
+    a.n_tiles = (p.n_out + swp::NH - 1) / swp::NH;   // weight blocks of 64 gate + 64 up rows
+    a.row_step = swp::NH;
+    a.half_off = p.n_out;
+  } else {
+    a.n_tiles = (p.n_out + swp::MW - 1) / swp::MW;   // weight blocks of 128 output rows
+    a.row_step = swp::MW;
+    a.half_off = swp::NH;
+  }
+  const int64_t tiles_bound =
+      ((static_cast<int64_t>(p.P) + swp::NT - 1) / swp::NT + p.E) * a.n_tiles;
+  const int grid = static_cast<int>(tiles_bound < num_sms ? tiles_bound : num_sms);
+  grouped_mxfp4_gemm_swap_kernel<EPI><<<grid, swp::NUM_THREADS, swp::SMEM_ALLOC, st>>>(tmA, tmB,
+                                                                                      tmS, a);
+  return cudaGetLastError();
 }
 
 template <int EPI>
@@ -894,12 +1249,14 @@ cudaError_t launch_impl(const GroupedGemmProblem& p, int num_sms, cudaStream_t s
 }  // namespace
 
 cudaError_t launch_gemm_gateup_swiglu(const GroupedGemmProblem& p, int num_sms, cudaStream_t st) {
-  if (p.use_pair) return launch_pair_impl<EPI_SWIGLU>(p, num_sms, st);
+  if (p.tiles == TILES_SWAP) return launch_swap_impl<EPI_SWIGLU>(p, num_sms, st);
+  if (p.tiles == TILES_PAIR) return launch_pair_impl<EPI_SWIGLU>(p, num_sms, st);
   return launch_impl<EPI_SWIGLU>(p, num_sms, st);
 }
 
 cudaError_t launch_gemm_down_combine(const GroupedGemmProblem& p, int num_sms, cudaStream_t st) {
-  if (p.use_pair) return launch_pair_impl<EPI_DOWN>(p, num_sms, st);
+  if (p.tiles == TILES_SWAP) return launch_swap_impl<EPI_DOWN>(p, num_sms, st);
+  if (p.tiles == TILES_PAIR) return launch_pair_impl<EPI_DOWN>(p, num_sms, st);
   return launch_impl<EPI_DOWN>(p, num_sms, st);
 }
 

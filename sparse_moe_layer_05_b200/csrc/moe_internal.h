@@ -39,9 +39,10 @@ cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* perm, int P, in
 // Per-token sum of the k weighted expert rows, rounded to bf16.
 cudaError_t launch_combine(const float* yw, int T, int k, int d, uint16_t* out,
                            cudaStream_t st);
-// E8M0 scales [E][N][G] -> [E][G][N] (the GEMMs load them with TMA per k-block).
-cudaError_t launch_transpose_scales(const uint8_t* in, int E, int N, int G, uint8_t* out,
-                                    cudaStream_t st);
+// E8M0 scales [E][N][G] -> [E][G][N] (the GEMMs load them with TMA per k-block);
+// experts with counts[e] == 0 are skipped (counts may be null: all experts).
+cudaError_t launch_transpose_scales(const uint8_t* in, int E, int N, int G, const int32_t* counts,
+                                    uint8_t* out, cudaStream_t st);
 // MXFP4 rows -> bf16 rows (same decoder as the GEMMs).
 cudaError_t launch_mxfp4_to_bf16(const uint8_t* codes, const uint8_t* scales, int rows, int K,
                                  uint16_t* out, cudaStream_t st);
@@ -60,8 +61,13 @@ struct GroupedGemmProblem {
   const float* topk_w;      // down: weight of each pair
   int n_out;                // output columns (I for SwiGLU, d for down)
   int* status;
-  bool use_pair;            // CTA-pair (2-SM) tiles instead of single-CTA tiles
+  int tiles;                // TILES_SINGLE, TILES_PAIR or TILES_SWAP
 };
+
+// Grouped-GEMM tile shapes.
+constexpr int TILES_SINGLE = 1;   // 256 activation rows x 128 weight rows, one CTA
+constexpr int TILES_PAIR = 2;     // 256 x 240 on a 2-CTA cluster (cta_group::2)
+constexpr int TILES_SWAP = 3;     // 128 weight rows x 64 tokens, weights as UMMA A
 cudaError_t launch_gemm_gateup_swiglu(const GroupedGemmProblem& p, int num_sms, cudaStream_t st);
 cudaError_t launch_gemm_down_combine(const GroupedGemmProblem& p, int num_sms, cudaStream_t st);
 

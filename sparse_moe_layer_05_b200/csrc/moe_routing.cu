@@ -57,33 +57,63 @@ __global__ void __launch_bounds__(RouterCfg<BE>::THREADS)
     for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 
   const int nch = d / RT_K;
-  for (int c0 = 0; c0 < nch; c0 += RT_G) {
-    // all threads stage the (up to) four chunks c0..c0+3, one per group
-    for (int i = tid; i < RT_G * RT_T * 4; i += C::THREADS) {   // x: 16 bytes per item
+  // items each thread stages per chunk group (x: 16-byte bf16 vectors, W: float4)
+  constexpr int XI = RT_G * RT_T * 4 / C::THREADS;
+  constexpr int WI = RT_G * BE * 8 / C::THREADS;
+  static_assert(XI * C::THREADS == RT_G * RT_T * 4 && WI * C::THREADS == RT_G * BE * 8, "split");
+  uint4 xr[XI];
+  float4 wr[WI];
+  auto fetch = [&](int c0) {  // global -> registers for chunks c0..c0+3
+#pragma unroll
+    for (int u = 0; u < XI; ++u) {
+      const int i = tid + u * C::THREADS;
       const int g = i / (RT_T * 4), r = i % (RT_T * 4);
       const int tt = r >> 2, kk = (r & 3) * 8, t = t0 + tt, c = c0 + g;
-      uint4 v = make_uint4(0, 0, 0, 0);
-      if (t < T && c < nch) v = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d + c * RT_K + kk));
-      float* xg = rsm + g * (C::XS + C::WS);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        xg[(kk + 2 * u) * (RT_T + 4) + tt] = __uint_as_float(w[u] << 16);
-        xg[(kk + 2 * u + 1) * (RT_T + 4) + tt] = __uint_as_float(w[u] & 0xFFFF0000u);
-      }
+      xr[u] = make_uint4(0, 0, 0, 0);
+      if (t < T && c < nch)
+        xr[u] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d + c * RT_K + kk));
     }
-    for (int i = tid; i < RT_G * BE * 8; i += C::THREADS) {     // W: 16 bytes per item
+#pragma unroll
+    for (int u = 0; u < WI; ++u) {
+      const int i = tid + u * C::THREADS;
       const int g = i / (BE * 8), r = i % (BE * 8);
       const int ee = r >> 3, kk = (r & 7) * 4, e = e0 + ee, c = c0 + g;
-      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e < E && c < nch) v = __ldg(reinterpret_cast<const float4*>(W_r + (size_t)e * d + c * RT_K + kk));
-      float* wg = rsm + g * (C::XS + C::WS) + C::XS;
-      wg[(kk + 0) * (BE + 4) + ee] = v.x;
-      wg[(kk + 1) * (BE + 4) + ee] = v.y;
-      wg[(kk + 2) * (BE + 4) + ee] = v.z;
-      wg[(kk + 3) * (BE + 4) + ee] = v.w;
+      wr[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (e < E && c < nch)
+        wr[u] = __ldg(reinterpret_cast<const float4*>(W_r + (size_t)e * d + c * RT_K + kk));
     }
+  };
+  auto stage = [&]() {  // registers -> shared (transposed to [k][token], [k][expert])
+#pragma unroll
+    for (int u = 0; u < XI; ++u) {
+      const int i = tid + u * C::THREADS;
+      const int g = i / (RT_T * 4), r = i % (RT_T * 4);
+      const int tt = r >> 2, kk = (r & 3) * 8;
+      float* xg = rsm + g * (C::XS + C::WS);
+      const uint32_t w[4] = {xr[u].x, xr[u].y, xr[u].z, xr[u].w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        xg[(kk + 2 * q) * (RT_T + 4) + tt] = __uint_as_float(w[q] << 16);
+        xg[(kk + 2 * q + 1) * (RT_T + 4) + tt] = __uint_as_float(w[q] & 0xFFFF0000u);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < WI; ++u) {
+      const int i = tid + u * C::THREADS;
+      const int g = i / (BE * 8), r = i % (BE * 8);
+      const int ee = r >> 3, kk = (r & 7) * 4;
+      float* wg = rsm + g * (C::XS + C::WS) + C::XS;
+      wg[(kk + 0) * (BE + 4) + ee] = wr[u].x;
+      wg[(kk + 1) * (BE + 4) + ee] = wr[u].y;
+      wg[(kk + 2) * (BE + 4) + ee] = wr[u].z;
+      wg[(kk + 3) * (BE + 4) + ee] = wr[u].w;
+    }
+  };
+  fetch(0);
+  for (int c0 = 0; c0 < nch; c0 += RT_G) {
+    stage();
     __syncthreads();
+    if (c0 + RT_G < nch) fetch(c0 + RT_G);  // in flight while this group computes
     if (c0 + grp < nch) {
 #pragma unroll 8
       for (int kk = 0; kk < RT_K; ++kk) {
@@ -368,9 +398,11 @@ constexpr int TR_ROWS = 64;
 
 __global__ void __launch_bounds__(256) transpose_scales_kernel(const uint8_t* __restrict__ in,
                                                                int N, int G,
+                                                               const int32_t* __restrict__ counts,
                                                                uint8_t* __restrict__ out) {
   extern __shared__ __align__(16) uint8_t tsm[];  // [TR_ROWS][G]
   const int e = blockIdx.y;
+  if (counts && counts[e] == 0) return;  // no GEMM tile reads this expert's scales
   const int n0 = blockIdx.x * TR_ROWS;
   const int rows = min(TR_ROWS, N - n0);
   const uint8_t* src = in + ((size_t)e * N + n0) * G;
@@ -486,11 +518,11 @@ cudaError_t launch_combine(const float* yw, int T, int k, int d, uint16_t* out,
   return cudaGetLastError();
 }
 
-cudaError_t launch_transpose_scales(const uint8_t* in, int E, int N, int G, uint8_t* out,
-                                    cudaStream_t st) {
+cudaError_t launch_transpose_scales(const uint8_t* in, int E, int N, int G, const int32_t* counts,
+                                    uint8_t* out, cudaStream_t st) {
   const int smem = TR_ROWS * G;  // G <= 512 (K <= 16384): at most 32 KB
   dim3 grid((N + TR_ROWS - 1) / TR_ROWS, E);
-  transpose_scales_kernel<<<grid, 256, smem, st>>>(in, N, G, out);
+  transpose_scales_kernel<<<grid, 256, smem, st>>>(in, N, G, counts, out);
   return cudaGetLastError();
 }
 

@@ -158,14 +158,17 @@ def test_forward_matches_oracle(case):
 
 
 PAIR_CASES = [
-    # name, d, I, E, k, T, seed -- experts with hundreds of rows, ragged tails
+    # name, d, I, E, k, T, seed -- ragged M/N/K tails, many and few rows per expert
     ("pair_ragged", 352, 224, 4, 2, 1500, 31),
     ("pair_wide", 2880, 2880, 8, 2, 1100, 32),
     ("pair_short_tail", 128, 256, 6, 3, 700, 33),
+    ("decode_wide", 2880, 2880, 64, 8, 64, 34),
+    ("decode_ragged", 352, 224, 16, 2, 40, 35),
+    ("decode_overflow", 256, 192, 4, 2, 150, 36),   # > 64 rows per expert: two token blocks
 ]
 
 
-@pytest.mark.parametrize("policy", [1, 2], ids=["single", "pair"])
+@pytest.mark.parametrize("policy", [1, 2, 3], ids=["single", "pair", "swap"])
 @pytest.mark.parametrize("case", PAIR_CASES, ids=[c[0] for c in PAIR_CASES])
 def test_forward_both_tile_policies(case, policy):
     from sparse_moe_layer_05_b200 import binding as B
