@@ -731,30 +731,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::NUM_THREADS, 1
 // The decoded weight tile is the UMMA A operand (M = 128 weight rows) and the
 // expert's routed rows are B (N = 64 tokens), so the tensor work follows the
 // actual token count instead of a 128/256-row tile, and the kernel streams
-// weights. For gate/up a tile holds 64 gate rows and the matching 64 up rows
-// interleaved (gate j at row 2j, up j at row 2j+1), so the SwiGLU epilogue
-// pairs adjacent TMEM lanes with one shuffle. Each CTA builds its tile table
-// (expert, weight block, token block) from the device offsets; experts with
-// no tokens cost nothing.
+// weights. The decoders store the decoded rows straight into tensor memory
+// (tcgen05.st, one TMEM lane per weight row) and the UMMA reads A from there:
+// decoded weights never pass through shared memory, whose bandwidth would
+// otherwise bound the weight stream. For gate/up a tile holds 64 gate rows
+// and the matching 64 up rows interleaved (gate j in lane 2j, up j in lane
+// 2j+1), so the SwiGLU epilogue pairs adjacent lanes with one shuffle. Each
+// CTA builds its tile table (expert, weight block, token block) from the
+// device offsets; experts with no tokens cost nothing.
 namespace swp {
 
-constexpr int MW = 128;               // weight rows per tile (UMMA M)
+constexpr int MW = 128;               // weight rows per tile (UMMA M = TMEM lanes)
 constexpr int NT = 64;                // tokens per tile (UMMA N)
 constexpr int BK = 64;
 constexpr int NH = 64;                // weight rows per TMA box
-constexpr int ST = 4, SW = 4, SC = 12;
+constexpr int ST = 6, SW = 8, SC = 12;
 constexpr int T_BYTES = NT * BK * 2;        // 8192
-constexpr int W_BYTES = MW * BK * 2;        // 16384
 constexpr int C_CODES = MW * BK / 2;        // 4096
 constexpr int S_OFF0 = C_CODES, S_OFF1 = C_CODES + 128;
 constexpr int C_TX = C_CODES + 2 * NH * 2;
 constexpr int C_BYTES = 4352;
 constexpr int NUM_THREADS = 512;
 constexpr int DEQ_THREADS = 256;
-constexpr int TMEM_COLS = 128;
+constexpr int TMEM_COLS = 512;
+constexpr int A_COL0 = 2 * NT;              // decoded weight stages after the accumulators
+constexpr int A_COLS = BK / 2;              // 32 columns (64 bf16 of K) per stage
+static_assert(A_COL0 + SW * A_COLS <= TMEM_COLS, "TMEM budget");
 
-constexpr int OFF_W = 0;
-constexpr int OFF_T = OFF_W + SW * W_BYTES;
+constexpr int OFF_T = 0;
 constexpr int OFF_C = OFF_T + ST * T_BYTES;
 constexpr int OFF_BAR = OFF_C + SC * C_BYTES;
 constexpr int NUM_BARS = 2 * ST + 2 * SW + 2 * SC + 4;
@@ -763,7 +767,7 @@ constexpr int OFF_TAB = OFF_MISC + 16;
 constexpr int SMEM_BYTES = OFF_TAB + 2 * (MAX_E + 1) * 4;
 constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
 static_assert(SMEM_ALLOC <= 232448, "shared memory budget");
-static_assert(OFF_T % 1024 == 0 && OFF_C % 1024 == 0, "alignment");
+static_assert(OFF_C % 1024 == 0, "alignment");
 
 }  // namespace swp
 
@@ -778,9 +782,10 @@ __global__ void __launch_bounds__(swp::NUM_THREADS, 1)
   // local copies shadow the single-CTA kernel's constants of the same names
   constexpr int MW = swp::MW, NT = swp::NT, BK = swp::BK, NH = swp::NH;
   constexpr int ST = swp::ST, SW = swp::SW, SC = swp::SC;
-  constexpr int T_BYTES = swp::T_BYTES, W_BYTES = swp::W_BYTES, C_BYTES = swp::C_BYTES;
+  constexpr int T_BYTES = swp::T_BYTES, C_BYTES = swp::C_BYTES;
   constexpr int C_TX = swp::C_TX, S_OFF0 = swp::S_OFF0, S_OFF1 = swp::S_OFF1;
-  constexpr int OFF_W = swp::OFF_W, OFF_T = swp::OFF_T, OFF_C = swp::OFF_C;
+  constexpr int A_COL0 = swp::A_COL0, A_COLS = swp::A_COLS;
+  constexpr int OFF_T = swp::OFF_T, OFF_C = swp::OFF_C;
   constexpr int OFF_BAR = swp::OFF_BAR, OFF_MISC = swp::OFF_MISC, OFF_TAB = swp::OFF_TAB;
   constexpr int NUM_THREADS = swp::NUM_THREADS, DEQ_THREADS = swp::DEQ_THREADS;
   constexpr int TMEM_COLS = swp::TMEM_COLS;
@@ -922,12 +927,12 @@ __global__ void __launch_bounds__(swp::NUM_THREADS, 1)
           if (!(ok = mbar_wait(bar_fullT(st), pt, abort_flag, args.status))) break;
           if (!(ok = mbar_wait(bar_fullW(sw), pw, abort_flag, args.status))) break;
           tc_fence_after();
-          const uint32_t w_addr = sbase + OFF_W + sw * W_BYTES;
+          const uint32_t a_tmem = tmem_base + A_COL0 + sw * A_COLS;
           const uint32_t t_addr = sbase + OFF_T + st * T_BYTES;
 #pragma unroll
           for (int kk = 0; kk < BK / 16; ++kk)
-            umma_bf16(d, sdesc_k_sw128(w_addr + kk * 32), sdesc_k_sw128(t_addr + kk * 32), idesc,
-                      (kb | kk) != 0);
+            umma_bf16_tmem_a(d, a_tmem + kk * 8, sdesc_k_sw128(t_addr + kk * 32), idesc,
+                             (kb | kk) != 0);
           umma_commit(bar_emptyT(st));
           umma_commit(bar_emptyW(sw));
           if (++st == ST) { st = 0; pt ^= 1; }
@@ -987,13 +992,18 @@ __global__ void __launch_bounds__(swp::NUM_THREADS, 1)
     }
   } else if (warp >= 8) {
     // ----------------------------------------------------------- decoders --
-    const int t = threadIdx.x - 8 * 32;
-    const int n = t >> 1;            // box row: 0..63 first box, 64..127 second
-    const int g = t & 1;
+    // Warp 8+q and warp 12+q both serve TMEM lanes 32q..32q+31 (one weight
+    // row per lane); the first decodes scale group 0 of the k-block (columns
+    // 0..15 of the stage), the second group 1 (columns 16..31).
+    const int wl = warp - 8;
+    const int quad = wl & 3, g = wl >> 2;
+    const int r = quad * 32 + lane;  // TMEM lane = weight row of the tile
+    // source row in the code stage: SwiGLU lanes interleave gate row r/2
+    // (first box) and up row r/2 (second box)
+    const int n = (EPI == EPI_SWIGLU) ? ((r & 1) ? NH + (r >> 1) : (r >> 1)) : r;
     const int soff = (n < NH ? S_OFF0 : S_OFF1) + g * NH + (n & (NH - 1));
-    // SwiGLU tiles interleave gate row j (first box) and up row j (second box)
-    const int orow = (EPI == EPI_SWIGLU) ? ((n < NH) ? 2 * n : 2 * (n - NH) + 1) : n;
-    const int swz = orow & 7;
+    const uint32_t lane_addr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + A_COL0 +
+                               g * (A_COLS / 2);
     int sc = 0, pc = 0, sw = 0, pw = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
@@ -1002,17 +1012,16 @@ __global__ void __launch_bounds__(swp::NUM_THREADS, 1)
         const uint8_t* stage = smem + OFF_C + sc * C_BYTES;
         const uint4 q = *reinterpret_cast<const uint4*>(stage + n * 32 + g * 16);
         const uint32_t sv = stage[soff];
-        uint4 o[4];
-        mxfp4x32_to_bf16(q, sv, o);
-        if (!(ok = mbar_wait(bar_emptyW(sw), pw ^ 1, abort_flag, args.status))) break;
-        uint8_t* wrow = smem + OFF_W + sw * W_BYTES + orow * 128;
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          *reinterpret_cast<uint4*>(wrow + (((4 * g + c) ^ swz) << 4)) = o[c];
-        // one proxy fence for the code-stage reads and the decoded-weight writes
+        // the next TMA write into this code stage must not overtake these reads
         fence_proxy_async_smem();
         mbar_arrive(bar_emptyC(sc));
         if (++sc == SC) { sc = 0; pc ^= 1; }
+        uint4 o[4];
+        mxfp4x32_to_bf16(q, sv, o);
+        if (!(ok = mbar_wait(bar_emptyW(sw), pw ^ 1, abort_flag, args.status))) break;
+        tc_fence_after();
+        tmem_st16_sync(lane_addr + sw * A_COLS, o);
+        tc_fence_before();
         mbar_arrive(bar_fullW(sw));
         if (++sw == SW) { sw = 0; pw ^= 1; }
       }

@@ -15,6 +15,9 @@ constexpr int kTileM = 256;
 
 inline int perm_chunks(int T) { return (T + kPermChunk - 1) / kPermChunk; }
 
+// Batches of at most this many tokens use the warp-per-token router kernel.
+constexpr int kRouterSmallT = 256;
+
 // K1: router logits s[t][e] = W_r[e] . x[t] + b_r[e] in fp32.
 cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, const float* b_r,
                                  float* logits, int T, int E, int d, int* status_to_clear,

@@ -155,6 +155,51 @@ __global__ void __launch_bounds__(RouterCfg<BE>::THREADS)
   }
 }
 
+// ----------------------------------------------- K1 logits, small batches ----
+// For a few tokens the tiled kernel has too few blocks to hide its chunk
+// latency; here one warp computes 4 experts' logits for one token. Lane l
+// accumulates the elements l*4 .. l*4+3 of every 128-element chunk in
+// increasing order (fma, fp32), then a fixed butterfly of shuffles adds the
+// 32 lane sums and the bias follows: every expert's logit sees the same
+// operation sequence, so identical router rows give bit-identical logits.
+constexpr int RS_EXPERTS = 32;  // experts per block (8 warps x 4)
+
+__global__ void __launch_bounds__(256) router_logits_small_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ W_r, const float* __restrict__ b_r,
+    float* __restrict__ logits, int T, int E, int d, int* status) {
+  const int t = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (status && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status = 0;
+  const int e0 = blockIdx.y * RS_EXPERTS + warp * 4;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  const uint16_t* xr = x + (size_t)t * d;
+  for (int k = lane * 4; k < d; k += 128) {
+    const uint2 xv = __ldg(reinterpret_cast<const uint2*>(xr + k));
+    const float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xFFFF0000u);
+    const float x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xFFFF0000u);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int e = e0 + j;
+      if (e < E) {
+        const float4 w = __ldg(reinterpret_cast<const float4*>(W_r + (size_t)e * d + k));
+        acc[j] = fmaf(x0, w.x, acc[j]);
+        acc[j] = fmaf(x1, w.y, acc[j]);
+        acc[j] = fmaf(x2, w.z, acc[j]);
+        acc[j] = fmaf(x3, w.w, acc[j]);
+      }
+    }
+  }
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xFFFFFFFFu, acc[j], off);
+  if (lane < 4) {
+    const int e = e0 + lane;
+    const float v = lane == 0 ? acc[0] : lane == 1 ? acc[1] : lane == 2 ? acc[2] : acc[3];
+    if (e < E) logits[(size_t)t * E + e] = v + b_r[e];
+  }
+}
+
 // ------------------------------------------------------ K1 top-k/softmax ----
 // One warp per token. Lane l holds the logits of experts l, l+32, ...; k rounds
 // of a warp arg-max on (logit descending, index ascending). Lane j keeps the
@@ -474,6 +519,11 @@ cudaError_t launch_router_be(const uint16_t* x, const float* W_r, const float* b
 cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, const float* b_r,
                                  float* logits, int T, int E, int d, int* status,
                                  cudaStream_t st) {
+  if (T <= kRouterSmallT) {
+    dim3 grid(T, (E + RS_EXPERTS - 1) / RS_EXPERTS);
+    router_logits_small_kernel<<<grid, 256, 0, st>>>(x, W_r, b_r, logits, T, E, d, status);
+    return cudaGetLastError();
+  }
   if (E <= 32) return launch_router_be<32>(x, W_r, b_r, logits, T, E, d, status, st);
   return launch_router_be<64>(x, W_r, b_r, logits, T, E, d, status, st);
 }
