@@ -273,6 +273,7 @@ def run_ours(args, inp, name):
     order = rank_token_order(T, rank)
     x_host = torch.from_numpy(np.ascontiguousarray(inp.x[order])).pin_memory()
     x = x_host.to(dev)
+    B.moe_set_tile_policy(args.tile_policy)
     layer = B.MoELayer(inp, device=dev, hostio=True)
     out = torch.empty((T, inp.d), dtype=torch.uint16, device=dev)
     out_host = torch.empty((T, inp.d), dtype=torch.uint16).pin_memory()
@@ -353,7 +354,7 @@ def run_ours(args, inp, name):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": workload_config(inp, name),
+        "config": dict(workload_config(inp, name), tile_policy=args.tile_policy),
         "layer_tflops": layer_flops(inp.d, inp.I, inp.E, inp.k, T) * args.steps * world
         / step_s_max / 1e12,
         "roofline": dict(roof, kernel=DOMINANT_STAGE, achieved=achieved, peak=peak,
@@ -377,6 +378,8 @@ def main(argv=None):
     ap.add_argument("--workload", default="20b", choices=list(W.SHAPES))
     ap.add_argument("--T", type=int, default=None, help="tokens per GPU (default: prefill T)")
     ap.add_argument("--ref-tokens", type=int, default=2, help="oracle tokens per reference step")
+    ap.add_argument("--tile-policy", type=int, default=0, choices=[0, 1, 2, 3, 4],
+                    help="grouped-GEMM tiles: 0 by shape, 1 single, 2 pair, 3 swap, 4 block-scaled")
     ap.add_argument("--cpu-sample", type=int, default=256,
                     help="tokens of the batch the oracle runs for cpu_baseline (0 = skip)")
     args = ap.parse_args(argv)

@@ -98,9 +98,20 @@ MOE_API int moe_version(void);
  *                   skipped for short expert tails),
  *   P/E >= 192      CTA-pair tiles (a 2-CTA cluster computes 256 x 240 tiles
  *                   with tcgen05 cta_group::2).
- * 1, 2 and 3 force single-CTA, CTA-pair and swapped-operand tiles. All
- * compute the same function. Not thread-safe against concurrent forward
- * calls. MOE_ERR_INVALID_ARG for other values.
+ * 1, 2 and 3 force single-CTA, CTA-pair and swapped-operand tiles; these
+ * decode the MXFP4 weights to bf16 in shared memory or TMEM and run bf16
+ * UMMAs on bf16 activations.
+ * 4 selects the block-scaled tiles: tcgen05.mma .kind::mxf8f6f4 with the E2M1
+ * codes widened to 8-bit containers by TMA, the E8M0 weight scales applied by
+ * the tensor core, and each bf16 activation (and H) row split per 32 elements
+ * into two E4M3 terms (hi and lo) with E8M0 scales; the split is exact for
+ * elements of at least 2^-13 of their group's max |x|, smaller ones keep an
+ * error below 2^-21 of it. 128 weight rows x 32 tokens per tile, two CTAs
+ * per SM. It needs d and I multiples of 64 of at least 128 and 32-byte
+ * aligned code arrays; otherwise policy 4 picks as policy 0 does.
+ * All policies compute the same function within the output tolerance. Not
+ * thread-safe against concurrent forward calls. MOE_ERR_INVALID_ARG for other
+ * values.
  */
 MOE_API moe_status moe_set_tile_policy(int policy);
 
@@ -221,6 +232,20 @@ typedef struct {
 MOE_API moe_status moe_workspace_layout(int E, int k, int T, int d, int I, moe_ws_layout* layout);
 
 /*
+ * The activation split of the block-scaled tiles (tile policy 4), on plain
+ * rows: x_dev [rows][K] bf16 -> hi_dev, lo_dev [rows][K] E4M3 bytes and
+ * scales_dev [rows][K/32][2] E8M0 bytes (hi, lo) such that, per group of 32,
+ * x = 2^(s_hi-127) e4m3(hi) + 2^(s_lo-127) e4m3(lo), exactly for every
+ * element of at least 2^-13 of the group's max |x| and within 2^-21 of that
+ * max otherwise (for groups whose max |x| is at least 2^-116). The pages have no counterpart: the split only lets bf16
+ * activations enter the tensor core's block-scaled MMA kind next to E2M1
+ * weights ("Four-bit expert weights"). K a multiple of 32; x_dev, hi_dev and
+ * lo_dev 16-byte aligned. All buffers are the caller's.
+ */
+MOE_API moe_status moe_mx_split_e4m3(const void* x_dev, int rows, int K, uint8_t* hi_dev,
+                                     uint8_t* lo_dev, uint8_t* scales_dev, void* stream);
+
+/*
  * Decode MXFP4 rows to bf16 on the device with the same decoder the grouped
  * GEMMs use ("Four-bit expert weights"). codes_dev [rows][K/2], scales_dev
  * [rows][K/32] -> out_dev [rows][K] bf16. K must be a multiple of 32.
@@ -245,7 +270,8 @@ MOE_API moe_status moe_selftest_wait_timeout(void* workspace_dev, void* stream);
 
 /*
  * Number of kernel launches one moe_forward call enqueues for this shape
- * (0 for T = 0). Used to count device work per step.
+ * under the current tile policy (0 for T = 0), assuming 32-byte aligned code
+ * arrays. Used to count device work per step.
  */
 MOE_API int moe_forward_launch_count(int E, int k, int T, int d, int I);
 

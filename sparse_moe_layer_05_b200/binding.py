@@ -27,7 +27,7 @@ STATUS = {
 EXPORTS = [
     "moe_status_string", "moe_version", "moe_workspace_size", "moe_forward",
     "moe_workspace_size_hostio", "moe_forward_hostio", "moe_route_workspace_size",
-    "moe_route", "moe_workspace_layout", "moe_mxfp4_to_bf16", "moe_sync_status",
+    "moe_route", "moe_workspace_layout", "moe_mxfp4_to_bf16", "moe_mx_split_e4m3", "moe_sync_status",
     "moe_selftest_wait_timeout", "moe_forward_launch_count", "moe_forward_timed",
     "moe_set_tile_policy", "moe_route_noalloc",
 ]
@@ -87,6 +87,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_workspace_layout.argtypes = [i32] * 5 + [ctypes.POINTER(WsLayout)]
     lib.moe_mxfp4_to_bf16.restype = i32
     lib.moe_mxfp4_to_bf16.argtypes = [u8p, u8p, i32, i32, vp, vp]
+    lib.moe_mx_split_e4m3.restype = i32
+    lib.moe_mx_split_e4m3.argtypes = [vp, i32, i32, u8p, u8p, u8p, vp]
     lib.moe_sync_status.restype = i32
     lib.moe_sync_status.argtypes = [vp, sz, vp]
     lib.moe_selftest_wait_timeout.restype = i32
@@ -205,17 +207,24 @@ def moe_route_noalloc(x, W_r, b_r, E, k, T, d, topk_idx, topk_w, counts, offsets
         _ptr(offsets), _ptr(perm), _stream(stream)))
 
 
+def moe_mx_split_e4m3(x, rows: int, K: int, hi, lo, scales, stream=None) -> None:
+    _require_cuda(x, hi, lo, scales)
+    _check("moe_mx_split_e4m3", load().moe_mx_split_e4m3(
+        _ptr(x), rows, K, _ptr(hi), _ptr(lo), _ptr(scales), _stream(stream)))
+
+
 def moe_mxfp4_to_bf16(codes, scales, rows: int, K: int, out, stream=None) -> None:
     _require_cuda(codes, scales, out)
     _check("moe_mxfp4_to_bf16", load().moe_mxfp4_to_bf16(
         _ptr(codes), _ptr(scales), rows, K, _ptr(out), _stream(stream)))
 
 
-TILE_AUTO, TILE_SINGLE, TILE_PAIR = 0, 1, 2
+TILE_AUTO, TILE_SINGLE, TILE_PAIR, TILE_SWAP, TILE_MX = 0, 1, 2, 3, 4
 
 
 def moe_set_tile_policy(policy: int) -> None:
-    """0 = by shape, 1 = single-CTA tiles, 2 = CTA-pair tiles (process-wide)."""
+    """0 = by shape, 1 = single-CTA, 2 = CTA-pair, 3 = swapped-operand,
+    4 = block-scaled tiles (process-wide)."""
     _check("moe_set_tile_policy", load().moe_set_tile_policy(policy))
 
 

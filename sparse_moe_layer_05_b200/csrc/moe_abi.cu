@@ -13,10 +13,16 @@ constexpr int kVersion = 100;  // 0.1.0
 constexpr int kMaxDevices = 64;
 
 // Grouped-GEMM tile policy: 0 = choose by shape, 1 = single-CTA tiles,
-// 2 = CTA-pair tiles, 3 = swapped-operand tiles.
+// 2 = CTA-pair tiles, 3 = swapped-operand tiles, 4 = block-scaled tiles.
 int g_tile_policy = 0;
 
-int choose_tiles(int P, int E) {
+// The block-scaled path reads the codes through 4-bit tensor maps: rows of a
+// multiple of 64 elements (at least 128) and 32-byte aligned code arrays.
+bool mx_shape_ok(int d, int I) { return d % 64 == 0 && I % 64 == 0 && d >= 128 && I >= 128; }
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31) == 0; }
+
+int choose_tiles(int P, int E, bool mx_ok) {
+  if (g_tile_policy == 4 && mx_ok) return moe::TILES_MX;
   if (g_tile_policy >= 1 && g_tile_policy <= 3) return g_tile_policy;
   const int64_t p = P, e = E;
   // Few routed rows per expert (decode): stream the weights with the
@@ -30,9 +36,14 @@ int choose_tiles(int P, int E) {
 
 size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
+// The block-scaled path's buffers share regions with the bf16 path's (one
+// forward call uses one path): the hi/lo token rows live in the xp region,
+// the hi/lo H rows in the h region, the B-scale blocks in the two regions of
+// transposed weight scales; each region is sized for the larger use.
 struct Layout {
   moe_ws_layout pub;
   size_t mprefix, chunk_hist, chunk_base, x_in, out_buf, gu_scales_t, d_scales_t;
+  size_t mx_tok_rows;
 };
 
 bool shape_ok(int E, int k, int T, int d) {
@@ -68,11 +79,16 @@ void make_layout(int E, int k, int T, int d, int I, bool hostio, Layout* L) {
   L->chunk_hist = take(NB * E * 4);
   L->chunk_base = take(NB * E * 4);
   L->pub.perm = take(P * 4);
-  L->pub.xp = take(P * d * 2);
-  L->pub.h = take(P * static_cast<size_t>(I) * 2);
+  const size_t tr = moe::mx_tok_rows(static_cast<int>(P), E);
+  L->mx_tok_rows = tr;
+  auto larger = [](size_t a, size_t b) { return a > b ? a : b; };
+  L->pub.xp = take(larger(P * d * 2, 2 * tr * d));
+  L->pub.h = take(larger(P * static_cast<size_t>(I) * 2, 2 * tr * I));
   L->pub.yw = take(P * d * 4);
-  L->gu_scales_t = take(static_cast<size_t>(E) * 2 * I * (d / 32));
-  L->d_scales_t = take(static_cast<size_t>(E) * d * (I / 32));
+  L->gu_scales_t = take(larger(static_cast<size_t>(E) * 2 * I * (d / 32),
+                               moe::mx_sfb_bytes(static_cast<int>(P), E, d)));
+  L->d_scales_t = take(larger(static_cast<size_t>(E) * d * (I / 32),
+                              moe::mx_sfb_bytes(static_cast<int>(P), E, I)));
   if (hostio) {
     L->x_in = take(static_cast<size_t>(T) * d * 2);
     L->out_buf = take(static_cast<size_t>(T) * d * 2);
@@ -201,6 +217,58 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   E_.mark(4);
   MOE_CUDA(moe::launch_perm_scatter(topk_idx, T, k, E, chunk_base, perm, nullptr, st));
   E_.mark(5);
+  const int tiles = choose_tiles(P, E, mx_shape_ok(d, I) && aligned32(gc) && aligned32(dc));
+  if (tiles == moe::TILES_MX) {
+    // block-scaled path: hi/lo token rows, no scale transposes
+    const size_t tr = L.mx_tok_rows;
+    uint8_t* qx = at<uint8_t>(ws, L.pub.xp);
+    uint8_t* qh = at<uint8_t>(ws, L.pub.h);
+    uint8_t* sfbx = at<uint8_t>(ws, L.gu_scales_t);
+    uint8_t* sfbh = at<uint8_t>(ws, L.d_scales_t);
+    MOE_CUDA(moe::launch_mx_quant_gather(x, perm, offsets, E, P, k, d, qx, qx + tr * d, sfbx, st));
+    E_.mark(6);
+    E_.mark(7);
+    E_.mark(8);
+    moe::MxGemmProblem m1;
+    memset(&m1, 0, sizeof(m1));
+    m1.codes = gc;
+    m1.scales = gs;
+    m1.b_hi = qx;
+    m1.b_lo = qx + tr * d;
+    m1.b_sfb = sfbx;
+    m1.offsets = offsets;
+    m1.P = P;
+    m1.E = E;
+    m1.K = d;
+    m1.I = I;
+    m1.tok_rows = static_cast<int>(tr);
+    m1.h_hi = qh;
+    m1.h_lo = qh + tr * I;
+    m1.h_sfb = sfbh;
+    m1.n_out = I;
+    m1.status = status;
+    MOE_CUDA(moe::launch_mx_gemm_gateup_swiglu(m1, num_sms, st));
+    E_.mark(9);
+    moe::MxGemmProblem m2 = m1;
+    m2.codes = dc;
+    m2.scales = ds;
+    m2.b_hi = qh;
+    m2.b_lo = qh + tr * I;
+    m2.b_sfb = sfbh;
+    m2.K = I;
+    m2.h_hi = nullptr;
+    m2.h_lo = nullptr;
+    m2.h_sfb = nullptr;
+    m2.out_f32 = yw;
+    m2.perm = perm;
+    m2.topk_w = topk_w;
+    m2.n_out = d;
+    MOE_CUDA(moe::launch_mx_gemm_down(m2, num_sms, st));
+    E_.mark(10);
+    MOE_CUDA(moe::launch_combine(yw, T, k, d, out, st));
+    E_.mark(11);
+    return MOE_OK;
+  }
   MOE_CUDA(moe::launch_gather_rows(x, perm, P, k, d, xp, st));
   E_.mark(6);
   MOE_CUDA(moe::launch_transpose_scales(gs, E, 2 * I, d / 32, counts, gst, st));
@@ -224,7 +292,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   g1.topk_w = nullptr;
   g1.n_out = I;
   g1.status = status;
-  g1.tiles = choose_tiles(P, E);
+  g1.tiles = tiles;
   MOE_CUDA(moe::launch_gemm_gateup_swiglu(g1, num_sms, st));
   E_.mark(9);
 
@@ -266,7 +334,7 @@ const char* moe_status_string(moe_status s) {
 int moe_version(void) { return kVersion; }
 
 moe_status moe_set_tile_policy(int policy) {
-  if (policy < 0 || policy > 3) return MOE_ERR_INVALID_ARG;
+  if (policy < 0 || policy > 4) return MOE_ERR_INVALID_ARG;
   g_tile_policy = policy;
   return MOE_OK;
 }
@@ -295,7 +363,8 @@ moe_status moe_workspace_layout(int E, int k, int T, int d, int I, moe_ws_layout
 
 int moe_forward_launch_count(int E, int k, int T, int d, int I) {
   if (!full_shape_ok(E, k, T, d, I) || T == 0) return 0;
-  return 11;
+  // the block-scaled path launches no scale transposes
+  return choose_tiles(T * k, E, mx_shape_ok(d, I)) == moe::TILES_MX ? 9 : 11;
 }
 
 moe_status moe_forward(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
@@ -449,6 +518,20 @@ moe_status moe_mxfp4_to_bf16(const uint8_t* codes_dev, const uint8_t* scales_dev
   MOE_CUDA(moe::launch_mxfp4_to_bf16(codes_dev, scales_dev, rows, K,
                                      static_cast<uint16_t*>(out_dev),
                                      static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_mx_split_e4m3(const void* x_dev, int rows, int K, uint8_t* hi_dev,
+                             uint8_t* lo_dev, uint8_t* scales_dev, void* stream) {
+  if (!x_dev || !hi_dev || !lo_dev || !scales_dev || rows < 0 || K < 32 || K % 32)
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_dev) || !aligned16(hi_dev) || !aligned16(lo_dev)) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
+  int num_sms = 0;
+  moe_status s = device_info(&num_sms);
+  if (s != MOE_OK) return s;
+  MOE_CUDA(moe::launch_mx_split_rows(static_cast<const uint16_t*>(x_dev), rows, K, hi_dev, lo_dev,
+                                     scales_dev, static_cast<cudaStream_t>(stream)));
   return MOE_OK;
 }
 

@@ -74,6 +74,48 @@ constexpr int TILES_SWAP = 3;     // 128 weight rows x 64 tokens, weights as UMM
 cudaError_t launch_gemm_gateup_swiglu(const GroupedGemmProblem& p, int num_sms, cudaStream_t st);
 cudaError_t launch_gemm_down_combine(const GroupedGemmProblem& p, int num_sms, cudaStream_t st);
 
+// ---------------------------------------------- block-scaled (MX) path ----
+// Tokens per tile of the block-scaled GEMMs; token rows are stored per expert
+// padded to a multiple of this.
+constexpr int kMxNT = 32;
+constexpr int TILES_MX = 4;       // block-scaled tcgen05 GEMMs (E2M1 x hi/lo E4M3)
+
+// Rows of the padded token layout and bytes of its B-scale blocks.
+size_t mx_tok_rows(int P, int E);
+size_t mx_sfb_bytes(int P, int E, int K);
+
+// K2: gather x rows into the padded token layout as hi/lo E4M3 rows plus the
+// B-scale blocks the GEMM loads per (token tile, k-block).
+cudaError_t launch_mx_quant_gather(const uint16_t* x, const int32_t* perm, const int32_t* offsets,
+                                   int E, int P, int k, int K, uint8_t* qhi, uint8_t* qlo,
+                                   uint8_t* sfb, cudaStream_t st);
+// The same split on plain rows, scales as [R][K/32][2] (hi byte, lo byte).
+cudaError_t launch_mx_split_rows(const uint16_t* x, int R, int K, uint8_t* qhi, uint8_t* qlo,
+                                 uint8_t* scales, cudaStream_t st);
+
+struct MxGemmProblem {
+  const uint8_t* codes;     // [E][rows][K/2] E2M1 codes
+  const uint8_t* scales;    // [E][rows][K/32] E8M0 scales (row-major, as given)
+  const uint8_t* b_hi;      // [tok_rows][K] E4M3 (padded token layout)
+  const uint8_t* b_lo;
+  const uint8_t* b_sfb;     // B-scale blocks
+  const int32_t* offsets;   // [E+1]
+  int P, E, K, I;
+  int tok_rows;
+  // SwiGLU: quantized H (padded layout) and its B-scale blocks
+  uint8_t* h_hi;
+  uint8_t* h_lo;
+  uint8_t* h_sfb;
+  // down: weighted rows
+  float* out_f32;
+  const int32_t* perm;
+  const float* topk_w;
+  int n_out;                // I for SwiGLU, d for down
+  int* status;
+};
+cudaError_t launch_mx_gemm_gateup_swiglu(const MxGemmProblem& p, int num_sms, cudaStream_t st);
+cudaError_t launch_mx_gemm_down(const MxGemmProblem& p, int num_sms, cudaStream_t st);
+
 // Debug/self-test: one bounded wait on an mbarrier that nothing completes.
 cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t st);
 

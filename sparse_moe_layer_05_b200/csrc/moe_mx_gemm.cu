@@ -1,0 +1,772 @@
+// moe_mx_gemm.cu -- expert-grouped MXFP4 GEMMs on the block-scaled tensor-core
+// path (tcgen05.mma .kind::mxf8f6f4): the E2M1 weight codes go from HBM to
+// shared memory by TMA (which widens them to 8-bit containers) and the E8M0
+// weight scales are applied by the tensor core, so no CUDA core decodes a
+// weight.
+//
+//   gate/up:  H[r, j] = silu(x_r . Wgate[e][j]) * (x_r . Wup[e][j])
+//   down:     Yw[pair(r), m] = p(pair(r)) * (H[r] . Wdown[e][m])
+//
+// Field guide "gpt-oss 20B", "03 Sparse Mixture of Experts" (SwiGLU experts,
+// weighted sum); "gpt-oss-20b and gpt-oss-120b", "Four-bit expert weights"
+// (E2M1 codes, one power-of-two scale per 32 weights).
+//
+// Activations. The tensor core's block-scaled kinds take no bf16 operand, so
+// each bf16 activation row is split, per group of 32 along K, into two E4M3
+// terms with E8M0 scales: hi = e4m3(x / 2^Eh) and lo = e4m3((x / 2^Eh - hi) *
+// 2^4), Eh = floor(log2 max|x|) - 7, scale bytes Eh + 127 and Eh + 123. For
+// every element with |x| >= 2^-13 max|x| of its group the split is exact
+// (x = 2^Eh hi + 2^(Eh-4) lo: x has 8 significant bits, hi keeps 4, the
+// remainder fits lo's 4 bits, |x/2^Eh - hi| <= 8); smaller elements keep an
+// error below 2^-21 max|x|. (Both hold for groups with max|x| >= 2^-116,
+// where Eh needs no clamping.) hi and lo enter one UMMA as separate columns of B
+// (tokens 0..NT-1 hi, NT..2NT-1 lo) and the epilogue adds the two results.
+//
+// Tiles. 128 weight rows (UMMA M) x NT tokens (UMMA N = 2 NT), 128 K per
+// shared-memory stage. Token rows live in a per-expert padded layout (each
+// expert's segment rounded up to a multiple of NT rows), so a token tile is
+// NT consecutive rows and its B scales one contiguous block. Two CTAs share an
+// SM; each has one MMA-issuing thread, which keeps the tensor pipe busy when
+// each UMMA is short (few tokens per expert).
+//
+// Warp roles (256 threads per CTA):
+//   warp 0      TMA producer: weight codes (E2M1 -> 8-bit containers), the hi
+//               and lo token rows, the tile's B scale block
+//   warp 1      TMEM allocator and UMMA issuer (one thread)
+//   warp 2      A-scale builder: gathers the k-block's E8M0 weight scales
+//               from global memory (four k-blocks ahead) into the layout
+//               tcgen05.cp reads
+//   warps 4-7   epilogue (TMEM lane quarters 0..3)
+//
+// K tail. The 4-bit tensor maps need row lengths in multiples of 128, so a K
+// that is 64 mod 128 is covered by the (K/128) full k-blocks of a main map and
+// one last k-block [K-128, K) from a second map based (K-128)/2 bytes into each
+// row; of that block only the K steps past the last full k-block are issued.
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "moe_internal.h"
+#include "moe_ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kMaxE = 256;
+
+// --------------------------------------------------- hi/lo E4M3 split ----
+
+// Groups of 32 along K: G = K/32 groups, KB = ceil(K/128) k-blocks; the last
+// k-block of a K that is not a multiple of 128 covers [K-128, K).
+__host__ __device__ __forceinline__ void group_to_kblock(int g, int G, int KB, int& kb, int& kk) {
+  const bool tail = (G % 4) != 0;
+  if (!tail || g < 4 * (KB - 1)) {
+    kb = g >> 2;
+    kk = g & 3;
+  } else {
+    kb = KB - 1;
+    kk = g - (G - 4);
+  }
+}
+
+// Byte offset of the B scale of token n (0..NT-1), term h (0 hi, 1 lo), K
+// step kk inside the block of one (token tile, k-block): TMEM column n/32 of
+// term h is word w = h*NT/32 + n/32, four words per 512-byte tcgen05.cp atom,
+// lane n%32 holding 16 bytes.
+__device__ __forceinline__ int sfb_offset(int NT, int n, int h, int kk) {
+  const int w = h * (NT / 32) + (n >> 5);
+  return (w >> 2) * 512 + (n & 31) * 16 + (w & 3) * 4 + kk;
+}
+
+__host__ __device__ constexpr int sfb_block_bytes(int NT) { return 512 * ((NT + 63) / 64); }
+
+// Splits 32 fp32 values (already bf16-exact) into hi / lo E4M3 bytes given the
+// group's max |v|; returns the hi scale byte (lo's is 4 less).
+__device__ __forceinline__ uint32_t split_group32(const float (&v)[32], float amax,
+                                                  uint32_t (&hi)[8], uint32_t (&lo)[8]) {
+  int eh;
+  if (amax == 0.f) {
+    eh = 0;
+  } else {
+    // floor(log2 amax) from the exponent field, minus 7 so that max|v|/2^eh
+    // lies in [128, 256); eh >= -123 keeps the lo scale byte (eh + 123) >= 0
+    // (groups with max|v| below 2^-116 lose the exactness bound below).
+    const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+    eh = max(e - 7, -123);
+  }
+  const float inv = __uint_as_float(static_cast<uint32_t>(127 - eh) << 23);   // 2^-eh
+#pragma unroll
+  for (int q = 0; q < 8; ++q) {
+    uint32_t hw = 0, lw = 0;
+#pragma unroll
+    for (int u = 0; u < 4; u += 2) {
+      const float a = v[4 * q + u] * inv, b = v[4 * q + u + 1] * inv;
+      const uint32_t h2 = f32x2_to_e4m3x2(a, b);
+      const float2 hb = e4m3x2_to_f32x2(h2);
+      const uint32_t l2 = f32x2_to_e4m3x2((a - hb.x) * 16.f, (b - hb.y) * 16.f);
+      hw |= h2 << (8 * u);
+      lw |= l2 << (8 * u);
+    }
+    hi[q] = hw;
+    lo[q] = lw;
+  }
+  return static_cast<uint32_t>(eh + 127);
+}
+
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+// One thread per (permuted row, group of 32): gathers x[token] into the padded
+// token layout as hi / lo E4M3 rows and writes the B scale blocks.
+template <int NT>
+__global__ void __launch_bounds__(256) mx_quant_gather_kernel(
+    const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
+    const int32_t* __restrict__ offsets, int E, int P, int k, int K, uint8_t* __restrict__ qhi,
+    uint8_t* __restrict__ qlo, uint8_t* __restrict__ sfb) {
+  __shared__ int s_off[kMaxE + 1], s_tb[kMaxE + 1];
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) s_off[i] = offsets[i];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int a = 0;
+    for (int e = 0; e < E; ++e) {
+      s_tb[e] = a;
+      a += (s_off[e + 1] - s_off[e] + NT - 1) / NT;
+    }
+    s_tb[E] = a;
+  }
+  __syncthreads();
+  const int G = K / 32, KB = (K + 127) / 128;
+  constexpr int SFB = sfb_block_bytes(NT);
+  const int64_t n = static_cast<int64_t>(P) * G;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int p = static_cast<int>(i / G), g = static_cast<int>(i % G);
+    int lo_e = 0, hi_e = E;   // largest e with s_off[e] <= p
+    while (hi_e - lo_e > 1) {
+      const int mid = (lo_e + hi_e) >> 1;
+      if (s_off[mid] <= p) lo_e = mid; else hi_e = mid;
+    }
+    const int e = lo_e;
+    const int pr = s_tb[e] * NT + (p - s_off[e]);
+    const int t = perm[p] / k;
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * K + 32 * g);
+    float v[32];
+    float amax = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 w = __ldg(src + c);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        v[8 * c + 2 * u] = bf16_bits_to_f32(ww[u] & 0xFFFFu);
+        v[8 * c + 2 * u + 1] = bf16_bits_to_f32(ww[u] >> 16);
+        amax = fmaxf(amax, fmaxf(fabsf(v[8 * c + 2 * u]), fabsf(v[8 * c + 2 * u + 1])));
+      }
+    }
+    uint32_t hw[8], lw[8];
+    const uint32_t sh = split_group32(v, amax, hw, lw);
+    uint4* dh = reinterpret_cast<uint4*>(qhi + static_cast<size_t>(pr) * K + 32 * g);
+    uint4* dl = reinterpret_cast<uint4*>(qlo + static_cast<size_t>(pr) * K + 32 * g);
+    dh[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    dh[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+    dl[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    dl[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+    int kb, kk;
+    group_to_kblock(g, G, KB, kb, kk);
+    uint8_t* blk = sfb + (static_cast<size_t>(pr / NT) * KB + kb) * SFB;
+    blk[sfb_offset(NT, pr % NT, 0, kk)] = static_cast<uint8_t>(sh);
+    blk[sfb_offset(NT, pr % NT, 1, kk)] = static_cast<uint8_t>(sh - 4);
+  }
+}
+
+// Plain row split (no gather): rows [R][K] bf16 -> hi, lo [R][K] E4M3 and
+// scales [R][K/32][2] (hi byte, lo byte).
+__global__ void __launch_bounds__(256) mx_split_rows_kernel(const uint16_t* __restrict__ x, int R,
+                                                            int K, uint8_t* __restrict__ qhi,
+                                                            uint8_t* __restrict__ qlo,
+                                                            uint8_t* __restrict__ scales) {
+  const int G = K / 32;
+  const int64_t n = static_cast<int64_t>(R) * G;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = i / G;
+    const int g = static_cast<int>(i % G);
+    const uint4* src = reinterpret_cast<const uint4*>(x + r * K + 32 * g);
+    float v[32];
+    float amax = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 w = __ldg(src + c);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        v[8 * c + 2 * u] = bf16_bits_to_f32(ww[u] & 0xFFFFu);
+        v[8 * c + 2 * u + 1] = bf16_bits_to_f32(ww[u] >> 16);
+        amax = fmaxf(amax, fmaxf(fabsf(v[8 * c + 2 * u]), fabsf(v[8 * c + 2 * u + 1])));
+      }
+    }
+    uint32_t hw[8], lw[8];
+    const uint32_t sh = split_group32(v, amax, hw, lw);
+    uint4* dh = reinterpret_cast<uint4*>(qhi + r * K + 32 * g);
+    uint4* dl = reinterpret_cast<uint4*>(qlo + r * K + 32 * g);
+    dh[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+    dh[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+    dl[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    dl[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+    scales[(r * G + g) * 2] = static_cast<uint8_t>(sh);
+    scales[(r * G + g) * 2 + 1] = static_cast<uint8_t>(sh - 4);
+  }
+}
+
+// ------------------------------------------------------------ the GEMM ----
+
+enum Epi { EPI_SWIGLU = 0, EPI_DOWN = 1 };
+
+template <int NT>
+struct MxCfg {
+  static constexpr int MW = 128;                    // weight rows per tile
+  static constexpr int N = 2 * NT;                  // UMMA N: hi and lo token columns
+  static constexpr int STAGES = 4;
+  static constexpr int A_BYTES = 128 * 128;         // E2M1 in 8-bit containers
+  static constexpr int A_TX = 128 * 64;             // packed bytes the TMA counts
+  static constexpr int B_BYTES = N * 128;
+  static constexpr int SFB_BYTES = sfb_block_bytes(NT);
+  static constexpr int OFF_B = A_BYTES;
+  static constexpr int OFF_SFA = OFF_B + B_BYTES;
+  static constexpr int OFF_SFB = OFF_SFA + 512;
+  static constexpr int STAGE_BYTES = ((OFF_SFB + SFB_BYTES) + 1023) / 1024 * 1024;
+  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
+  static constexpr int NUM_BARS = 2 * STAGES + 4;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_TAB = OFF_MISC + 16;
+  static constexpr int OFF_XCH = OFF_TAB + 3 * (kMaxE + 1) * 4;
+  static constexpr int SMEM_BYTES = OFF_XCH + 2 * 4 * NT * 4;
+  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+  static constexpr int NUM_THREADS = 256;
+  static constexpr int TMEM_COLS = 256;
+  static constexpr int SFA_COL = 2 * N;             // after the two accumulator buffers
+  static constexpr int SFB_COL = SFA_COL + 4;
+  static constexpr int TX_BYTES = A_TX + B_BYTES + SFB_BYTES;
+  static_assert(SFB_COL + 4 * ((SFB_BYTES + 511) / 512) <= TMEM_COLS, "TMEM budget");
+  static_assert(2 * SMEM_ALLOC + 2048 <= 233472, "two CTAs per SM");
+  static_assert(OFF_B % 1024 == 0 && (NT * 128) % 1024 == 0, "swizzle atom alignment");
+};
+
+struct MxArgs {
+  const int32_t* offsets;
+  int E, K, I;              // K: contraction length; I: intermediate size (SwiGLU tiles)
+  int n_wb;                 // weight blocks per expert
+  int rows_per_expert;      // weight rows of one expert in the scale array
+  const uint8_t* scales;    // [E][rows_per_expert][K/32] E8M0
+  const uint8_t* sfb;       // B scale blocks [token tile][KB][SFB_BYTES]
+  // SwiGLU: quantized H for the down GEMM
+  uint8_t* h_hi;
+  uint8_t* h_lo;
+  uint8_t* h_sfb;
+  int h_kb;                 // k-blocks of the down GEMM (ceil(I/128))
+  // down: weighted rows
+  float* out_f32;
+  int n_out;
+  const int32_t* perm;
+  const float* topk_w;
+  int* status;
+};
+
+__device__ __forceinline__ float silu_mx(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
+__device__ __forceinline__ uint16_t ldg_u16(const uint8_t* p) {
+  return __ldg(reinterpret_cast<const unsigned short*>(p));
+}
+
+template <int EPI, int NT>
+__global__ void __launch_bounds__(256, 2)
+    grouped_mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                           const __grid_constant__ CUtensorMap tmAt,
+                           const __grid_constant__ CUtensorMap tmBh,
+                           const __grid_constant__ CUtensorMap tmBl, const MxArgs args) {
+  using C = MxCfg<NT>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  auto bar_full = [&](int s) { return bar0 + 8u * s; };
+  auto bar_empty = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
+  auto bar_accFull = [&](int b) { return bar0 + 8u * (2 * C::STAGES + b); };
+  auto bar_accEmpty = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 2 + b); };
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  int* s_off = reinterpret_cast<int*>(smem + C::OFF_TAB);
+  int* s_tp = s_off + (kMaxE + 1);   // prefix of tiles per expert
+  int* s_tb = s_tp + (kMaxE + 1);    // prefix of token tiles per expert
+  float* s_xch = reinterpret_cast<float*>(smem + C::OFF_XCH);
+
+  const int E = args.E;
+  for (int i = threadIdx.x; i <= E; i += C::NUM_THREADS) s_off[i] = args.offsets[i];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    int acc = 0, tb = 0;
+    for (int e = 0; e < E; ++e) {
+      s_tp[e] = acc;
+      s_tb[e] = tb;
+      const int ntb = (s_off[e + 1] - s_off[e] + NT - 1) / NT;
+      acc += ntb * args.n_wb;
+      tb += ntb;
+    }
+    s_tp[E] = acc;
+    s_tb[E] = tb;
+    for (int s = 0; s < C::STAGES; ++s) {
+      mbar_init(bar_full(s), 2);    // producer (with the TMA bytes) + A-scale builder
+      mbar_init(bar_empty(s), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accFull(b), 1);
+      mbar_init(bar_accEmpty(b), 4 * 32);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmAt);
+    tma_prefetch_desc(&tmBh);
+    tma_prefetch_desc(&tmBl);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(misc), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = misc[0];
+
+  const int total = s_tp[E];
+  const int K = args.K;
+  const int G = K / 32;
+  const int KB = (K + 127) / 128;
+  const bool tail = (K % 128) != 0;
+  const int tail_k0 = 4 - (K % 128) / 32;   // first K step issued in the tail k-block
+  // tile -> (expert, weight block, token block), weight-block major inside an
+  // expert so that neighbouring CTAs stream neighbouring weights
+  auto decode = [&](int tile, int& e, int& wb, int& tb, int& rows) {
+    int lo = 0, hi = E;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_tp[mid] <= tile) lo = mid; else hi = mid;
+    }
+    e = lo;
+    const int cnt = s_off[e + 1] - s_off[e];
+    const int ntb = (cnt + NT - 1) / NT;
+    const int local = tile - s_tp[e];
+    wb = local / ntb;
+    tb = local % ntb;
+    rows = min(NT, cnt - tb * NT);
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer --
+    if (lane == 0) {
+      int s = 0, ph = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        int e, wb, tb, rows;
+        decode(tile, e, wb, tb, rows);
+        const int tok_tile = s_tb[e] + tb;
+        const int row_b = tok_tile * NT;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!(ok = mbar_wait(bar_empty(s), ph ^ 1, abort_flag, args.status))) break;
+          const uint32_t st = sbase + s * C::STAGE_BYTES;
+          const uint32_t fb = bar_full(s);
+          mbar_expect_tx(fb, C::TX_BYTES);
+          const bool last_tail = tail && kb == KB - 1;
+          const CUtensorMap* am = last_tail ? &tmAt : &tmA;
+          const int ax = last_tail ? 0 : kb * 128;
+          if (EPI == EPI_SWIGLU) {
+            // four boxes of 16 gate rows + the same 16 up rows (TMEM lanes
+            // 32q..32q+15 gate, 32q+16..32q+31 up)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              tma_load_3d(st + q * 4096, am, ax, wb * 64 + 16 * q, 2 * e, fb);
+          } else {
+            tma_load_3d(st, am, ax, wb * 128, e, fb);
+          }
+          const int bx = last_tail ? K - 128 : kb * 128;
+          tma_load_2d(st + C::OFF_B, &tmBh, bx, row_b, fb);
+          tma_load_2d(st + C::OFF_B + NT * 128, &tmBl, bx, row_b, fb);
+          bulk_load(st + C::OFF_SFB,
+                    args.sfb + (static_cast<size_t>(tok_tile) * KB + kb) * C::SFB_BYTES,
+                    C::SFB_BYTES, fb);
+          if (++s == C::STAGES) { s = 0; ph ^= 1; }
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // -------------------------------------------------- A-scale builder --
+    // Lane l owns shared-memory rows l, l+32, l+64, l+96 of the A tile; for
+    // each it loads the 4 scale bytes of the k-block (2-byte aligned: two
+    // 16-bit loads) four k-blocks ahead of their use.
+    constexpr int PD = 4;
+    const uint8_t* scales = args.scales;
+    const int rpe = args.rows_per_expert;
+    auto load_words = [&](int tile, int kb, uint32_t (&w)[4]) {
+      int e, wb, tb, rows;
+      decode(tile, e, wb, tb, rows);
+      const int gs = (tail && kb == KB - 1) ? G - 4 : 4 * kb;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        int r;
+        bool valid;
+        if (EPI == EPI_SWIGLU) {
+          const int jj = wb * 64 + 16 * j + (lane & 15);
+          valid = jj < args.I;
+          r = (lane < 16) ? jj : args.I + jj;
+        } else {
+          r = wb * 128 + 32 * j + lane;
+          valid = r < rpe;
+        }
+        if (valid) {
+          const uint8_t* p = scales + (static_cast<size_t>(e) * rpe + r) * G + gs;
+          w[j] = static_cast<uint32_t>(ldg_u16(p)) | (static_cast<uint32_t>(ldg_u16(p + 2)) << 16);
+        } else {
+          w[j] = 0x7F7F7F7Fu;
+        }
+      }
+    };
+    // (tile, kb) iterators: `c` consumes, `f` fetches PD steps ahead
+    int c_tile = blockIdx.x, c_kb = 0;
+    int f_tile = blockIdx.x, f_kb = 0;
+    auto advance = [&](int& tile, int& kb) {
+      if (++kb == KB) { kb = 0; tile += gridDim.x; }
+    };
+    uint32_t buf[PD][4];
+#pragma unroll
+    for (int u = 0; u < PD; ++u) {
+      if (f_tile < total) {
+        load_words(f_tile, f_kb, buf[u]);
+        advance(f_tile, f_kb);
+      }
+    }
+    int s = 0, ph = 0;
+    bool ok = true;
+    while (ok && c_tile < total) {
+#pragma unroll
+      for (int u = 0; u < PD; ++u) {
+        if (!ok || c_tile >= total) break;
+        if (!(ok = mbar_wait(bar_empty(s), ph ^ 1, abort_flag, args.status))) break;
+        *reinterpret_cast<uint4*>(smem + s * C::STAGE_BYTES + C::OFF_SFA + lane * 16) =
+            make_uint4(buf[u][0], buf[u][1], buf[u][2], buf[u][3]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_full(s));
+        if (++s == C::STAGES) { s = 0; ph ^= 1; }
+        advance(c_tile, c_kb);
+        if (f_tile < total) {
+          load_words(f_tile, f_kb, buf[u]);
+          advance(f_tile, f_kb);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // -------------------------------------------------------- UMMA issuer --
+    if (lane == 0) {
+      const uint32_t idesc0 = idesc_mx_e2m1_e4m3(C::MW, C::N, 0, 0);
+      const uint32_t sfa_t = tmem_base + C::SFA_COL, sfb_t = tmem_base + C::SFB_COL;
+      int s = 0, ph = 0, it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+        const int ab = it & 1;
+        const uint32_t ap = (it >> 1) & 1;
+        if (!(ok = mbar_wait(bar_accEmpty(ab), ap ^ 1, abort_flag, args.status))) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + ab * C::N;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!(ok = mbar_wait(bar_full(s), ph, abort_flag, args.status))) break;
+          tc_fence_after();
+          const uint32_t st = sbase + s * C::STAGE_BYTES;
+          tmem_cp_32x128b_x4(sfa_t, sdesc_k_noswizzle(st + C::OFF_SFA, 128));
+#pragma unroll
+          for (int a = 0; a < C::SFB_BYTES / 512; ++a)
+            tmem_cp_32x128b_x4(sfb_t + 4 * a, sdesc_k_noswizzle(st + C::OFF_SFB + 512 * a, 128));
+          const int k0 = (tail && kb == KB - 1) ? tail_k0 : 0;
+          for (int kk = k0; kk < 4; ++kk) {
+            const uint32_t id = idesc0 | (static_cast<uint32_t>(kk) << 4) |
+                                (static_cast<uint32_t>(kk) << 29);
+            umma_mxf8f6f4(d, sdesc_k_sw128(st + kk * 32), sdesc_k_sw128(st + C::OFF_B + kk * 32),
+                          id, sfa_t | (static_cast<uint32_t>(kk) << 30),
+                          sfb_t | (static_cast<uint32_t>(kk) << 30), (kb > 0 || kk > k0) ? 1u : 0u);
+          }
+          umma_commit(bar_empty(s));
+          if (++s == C::STAGES) { s = 0; ph ^= 1; }
+        }
+        if (ok) umma_commit(bar_accFull(ab));
+      }
+    }
+  } else if (warp >= 4) {
+    // ----------------------------------------------------------- epilogue --
+    // Every epilogue warp passes the SwiGLU exchange barrier once per tile,
+    // also after a failed wait, so that no warp is left at it alone.
+    const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31
+    const int m = quad * 32 + lane;            // weight row of the tile
+    bool ok = true;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      int e, wb, tb, rows;
+      decode(tile, e, wb, tb, rows);
+      const int ab = it & 1;
+      const uint32_t ap = (it >> 1) & 1;
+      if (ok) ok = mbar_wait(bar_accFull(ab), ap, abort_flag, args.status);
+      if (!ok && EPI != EPI_SWIGLU) break;
+      float y[NT];
+      if (ok) {
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + ab * C::N;
+#pragma unroll
+        for (int c = 0; c < NT; c += 16) {
+          uint32_t a[16], b[16];
+          tmem_ld16_sync(taddr + c, a);
+          tmem_ld16_sync(taddr + NT + c, b);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) y[c + i] = __uint_as_float(a[i]) + __uint_as_float(b[i]);
+        }
+        tc_fence_before();
+        mbar_arrive(bar_accEmpty(ab));     // accumulators are in registers now
+      } else {
+#pragma unroll
+        for (int t = 0; t < NT; ++t) y[t] = 0.f;
+      }
+
+      const int tok_tile = s_tb[e] + tb;
+      if (EPI == EPI_SWIGLU) {
+        // lanes 0-15: gate row j, lanes 16-31: up row j (j = wb*64 + 16*quad + lane%16);
+        // y[t] becomes h for the gate lanes and 0 elsewhere
+        const int j = wb * 64 + 16 * quad + (lane & 15);
+        const bool jv = ok && j < args.I && lane < 16;
+        float* xch = s_xch + (it & 1) * 4 * NT;
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const float u = __shfl_xor_sync(0xFFFFFFFFu, y[t], 16);
+          float hv = 0.f;
+          if (jv && t < rows) hv = __bfloat162float(__float2bfloat16_rn(silu_mx(y[t]) * u));
+          y[t] = hv;
+          float pm = fabsf(hv);
+#pragma unroll
+          for (int o = 1; o < 16; o <<= 1) pm = fmaxf(pm, __shfl_xor_sync(0xFFFFFFFFu, pm, o));
+          if (lane == 0) xch[quad * NT + t] = pm;
+        }
+        // max |h| over the 32 j of a group: quarters 0+1 and 2+3
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (ok) {
+          const int gj = 2 * wb + (quad >> 1);
+          int kb4, kk4;
+          group_to_kblock(gj, args.I / 32, args.h_kb, kb4, kk4);
+          uint8_t* hsfb = args.h_sfb + (static_cast<size_t>(tok_tile) * args.h_kb + kb4) *
+                                           sfb_block_bytes(NT);
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            if (t < rows) {
+              const float amax = fmaxf(xch[quad * NT + t], xch[(quad ^ 1) * NT + t]);
+              int eh = 0;
+              if (amax != 0.f) {
+                const int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+                eh = max(ex - 7, -123);
+              }
+              const float inv = __uint_as_float(static_cast<uint32_t>(127 - eh) << 23);
+              const float a = y[t] * inv;
+              const uint32_t h2 = f32x2_to_e4m3x2(a, 0.f);
+              const float2 hb = e4m3x2_to_f32x2(h2);
+              const uint32_t l2 = f32x2_to_e4m3x2((a - hb.x) * 16.f, 0.f);
+              if (jv) {
+                const size_t o = static_cast<size_t>(tok_tile * NT + t) * args.I + j;
+                args.h_hi[o] = static_cast<uint8_t>(h2 & 0xFF);
+                args.h_lo[o] = static_cast<uint8_t>(l2 & 0xFF);
+              }
+              if (lane == 0 && !(quad & 1)) {
+                hsfb[sfb_offset(NT, t, 0, kk4)] = static_cast<uint8_t>(eh + 127);
+                hsfb[sfb_offset(NT, t, 1, kk4)] = static_cast<uint8_t>(eh + 123);
+              }
+            }
+          }
+        }
+      } else {
+        const int col = wb * 128 + m;
+        if (col < args.n_out) {
+          const int p0 = s_off[e] + tb * NT;
+#pragma unroll
+          for (int t = 0; t < NT; ++t) {
+            if (t < rows) {
+              const int pr = args.perm[p0 + t];
+              args.out_f32[static_cast<int64_t>(pr) * args.n_out + col] = args.topk_w[pr] * y[t];
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ----------------------------------------------------------- host side ----
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+bool encode_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base,
+                const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, dt, rank, const_cast<void*>(base), dims, strides, box, es,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// E2M1 codes as 3D (K elements, rows, planes): the main map covers the first
+// 128*floor(K/128) elements of each row, the tail map the last 128 (based
+// (K-128)/2 bytes into the row); both widen to 8-bit containers.
+bool make_code_maps(CUtensorMap* main_map, CUtensorMap* tail_map, const uint8_t* codes, int K,
+                    int rows, int planes, int box_rows, int box_planes) {
+  const cuuint64_t rb = static_cast<cuuint64_t>(K / 2);
+  const cuuint64_t strides[2] = {rb, rb * static_cast<cuuint64_t>(rows)};
+  const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows),
+                             static_cast<cuuint32_t>(box_planes)};
+  const int kmain = (K / 128) * 128;
+  bool ok = true;
+  if (kmain > 0) {
+    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kmain), static_cast<cuuint64_t>(rows),
+                                static_cast<cuuint64_t>(planes)};
+    ok = encode_map(main_map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, codes, dims, strides, box);
+  }
+  if (ok && (K % 128) != 0) {
+    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(rows),
+                                static_cast<cuuint64_t>(planes)};
+    ok = encode_map(tail_map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, codes + (K - 128) / 2,
+                    dims, strides, box);
+  } else if (ok) {
+    *tail_map = *main_map;
+  }
+  if (ok && kmain == 0) *main_map = *tail_map;
+  return ok;
+}
+
+// E4M3 token rows [rows][K], box 128 x NT.
+bool make_tok8_map(CUtensorMap* m, const uint8_t* base, int rows, int K, int nt) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+  const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(nt)};
+  return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box);
+}
+
+template <int EPI, int NT>
+cudaError_t launch_mx_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st) {
+  using C = MxCfg<NT>;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_mx_gemm_kernel<EPI, NT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         C::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  CUtensorMap tmA, tmAt, tmBh, tmBl;
+  bool ok;
+  if (EPI == EPI_SWIGLU)
+    ok = make_code_maps(&tmA, &tmAt, p.codes, p.K, p.I, 2 * p.E, 16, 2);
+  else
+    ok = make_code_maps(&tmA, &tmAt, p.codes, p.K, p.n_out, p.E, 128, 1);
+  ok = ok && make_tok8_map(&tmBh, p.b_hi, p.tok_rows, p.K, NT) &&
+       make_tok8_map(&tmBl, p.b_lo, p.tok_rows, p.K, NT);
+  if (!ok) return cudaErrorInvalidValue;
+  MxArgs a;
+  a.offsets = p.offsets;
+  a.E = p.E;
+  a.K = p.K;
+  a.I = p.I;
+  a.scales = p.scales;
+  a.sfb = p.b_sfb;
+  a.h_hi = p.h_hi;
+  a.h_lo = p.h_lo;
+  a.h_sfb = p.h_sfb;
+  a.h_kb = (p.I + 127) / 128;
+  a.out_f32 = p.out_f32;
+  a.n_out = p.n_out;
+  a.perm = p.perm;
+  a.topk_w = p.topk_w;
+  a.status = p.status;
+  if (EPI == EPI_SWIGLU) {
+    a.n_wb = (p.I + 63) / 64;
+    a.rows_per_expert = 2 * p.I;
+  } else {
+    a.n_wb = (p.n_out + 127) / 128;
+    a.rows_per_expert = p.n_out;
+  }
+  const int64_t tiles_bound = (static_cast<int64_t>(p.P) / NT + p.E) * a.n_wb;
+  int64_t grid = 2 * static_cast<int64_t>(num_sms);
+  if (tiles_bound < grid) grid = tiles_bound;
+  if (grid < 1) grid = 1;
+  grouped_mx_gemm_kernel<EPI, NT><<<static_cast<int>(grid), C::NUM_THREADS, C::SMEM_ALLOC, st>>>(
+      tmA, tmAt, tmBh, tmBl, a);
+  return cudaGetLastError();
+}
+
+int grid_for_n(int64_t n, int per_thread_block, int cap) {
+  int64_t b = (n + per_thread_block - 1) / per_thread_block;
+  if (b < 1) b = 1;
+  if (b > cap) b = cap;
+  return static_cast<int>(b);
+}
+
+}  // namespace
+
+size_t mx_tok_rows(int P, int E) { return static_cast<size_t>(P) + static_cast<size_t>(E) * (kMxNT - 1); }
+size_t mx_sfb_bytes(int P, int E, int K) {
+  const size_t tiles = (static_cast<size_t>(P) + kMxNT - 1) / kMxNT + E;
+  return tiles * ((K + 127) / 128) * sfb_block_bytes(kMxNT);
+}
+
+cudaError_t launch_mx_quant_gather(const uint16_t* x, const int32_t* perm, const int32_t* offsets,
+                                   int E, int P, int k, int K, uint8_t* qhi, uint8_t* qlo,
+                                   uint8_t* sfb, cudaStream_t st) {
+  const int64_t n = static_cast<int64_t>(P) * (K / 32);
+  mx_quant_gather_kernel<kMxNT><<<grid_for_n(n, 256, 148 * 8), 256, 0, st>>>(
+      x, perm, offsets, E, P, k, K, qhi, qlo, sfb);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mx_split_rows(const uint16_t* x, int R, int K, uint8_t* qhi, uint8_t* qlo,
+                                 uint8_t* scales, cudaStream_t st) {
+  const int64_t n = static_cast<int64_t>(R) * (K / 32);
+  mx_split_rows_kernel<<<grid_for_n(n, 256, 148 * 8), 256, 0, st>>>(x, R, K, qhi, qlo, scales);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mx_gemm_gateup_swiglu(const MxGemmProblem& p, int num_sms, cudaStream_t st) {
+  return launch_mx_impl<EPI_SWIGLU, kMxNT>(p, num_sms, st);
+}
+
+cudaError_t launch_mx_gemm_down(const MxGemmProblem& p, int num_sms, cudaStream_t st) {
+  return launch_mx_impl<EPI_DOWN, kMxNT>(p, num_sms, st);
+}
+
+}  // namespace moe

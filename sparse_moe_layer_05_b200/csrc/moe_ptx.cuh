@@ -326,6 +326,83 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
          (static_cast<uint32_t>(M >> 4) << 24);
 }
 
+// ------------------------------------------- block-scaled (MX) tcgen05 ----
+
+// D[tmem] (+)= sum_k (a_mk 2^(sa_m - 127)) (b_nk 2^(sb_n - 127)) over one
+// K = 32 step with .kind::mxf8f6f4: A holds E2M1 values in 8-bit containers
+// (the layout the 16U4_ALIGN16B tensor maps write), B holds E4M3 values, both
+// K-major in 128-byte swizzled tiles. sa / sb are E8M0 scales read from TMEM:
+// lane m (A) or n (B) of column sf + m/32 (n/32) within each 32-lane quarter,
+// byte given by bits 30-31 of the scale address (and the matching sf-id field
+// of the instruction descriptor).
+__device__ __forceinline__ void umma_mxf8f6f4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                              uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                              uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Instruction descriptor for umma_mxf8f6f4: A E2M1, B E4M3, E8M0 scales, both
+// operands K-major, fp32 accumulator; sfa_id / sfb_id select the scale byte.
+__host__ __device__ constexpr uint32_t idesc_mx_e2m1_e4m3(int M, int N, uint32_t sfa_id,
+                                                         uint32_t sfb_id) {
+  return (sfb_id << 4) | (5u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24) | (sfa_id << 29);
+}
+
+// Shared memory -> TMEM: 32 lanes x 128 bits, replicated into all four 32-lane
+// quarters of the columns [taddr, taddr + 4).
+__device__ __forceinline__ void tmem_cp_32x128b_x4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+// Descriptor of an unswizzled K-major shared-memory tile: rows of 16 bytes,
+// 8-row core matrices `sbo` bytes apart (the tcgen05.cp source format).
+__device__ __forceinline__ uint64_t sdesc_k_noswizzle(uint32_t saddr, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(16 >> 4) << 16;
+  d |= static_cast<uint64_t>(sbo >> 4) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;
+}
+
+// Contiguous global -> shared copy of `bytes` (multiple of 16, both addresses
+// 16-byte aligned), completing on an mbarrier.
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+// Two fp32 -> two E4M3 (round to nearest even, saturating to +-448): the
+// result holds e4m3(a) in bits 0-7 and e4m3(b) in bits 8-15.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float a, float b) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
+  return r;
+}
+
+// Two E4M3 (bits 0-7, 8-15) -> two fp32 (exact).
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t v) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(v)));
+  uint16_t lo = static_cast<uint16_t>(h2 & 0xFFFFu), hi = static_cast<uint16_t>(h2 >> 16);
+  float fa, fb;
+  asm("cvt.f32.f16 %0, %1;" : "=f"(fa) : "h"(lo));
+  asm("cvt.f32.f16 %0, %1;" : "=f"(fb) : "h"(hi));
+  return make_float2(fa, fb);
+}
+
 // ------------------------------------------------------------ MXFP4 ----
 
 // bf16x2 product; exact whenever the product is representable.

@@ -165,10 +165,12 @@ PAIR_CASES = [
     ("decode_wide", 2880, 2880, 64, 8, 64, 34),
     ("decode_ragged", 352, 224, 16, 2, 40, 35),
     ("decode_overflow", 256, 192, 4, 2, 150, 36),   # > 64 rows per expert: two token blocks
+    ("mx_tails", 448, 320, 6, 2, 500, 37),           # K = 64 mod 128 in both GEMMs
+    ("mx_decode_many", 2880, 2880, 128, 4, 32, 38),  # many experts with 0-3 rows
 ]
 
 
-@pytest.mark.parametrize("policy", [1, 2, 3], ids=["single", "pair", "swap"])
+@pytest.mark.parametrize("policy", [1, 2, 3, 4], ids=["single", "pair", "swap", "mx"])
 @pytest.mark.parametrize("case", PAIR_CASES, ids=[c[0] for c in PAIR_CASES])
 def test_forward_both_tile_policies(case, policy):
     from sparse_moe_layer_05_b200 import binding as B
@@ -184,12 +186,56 @@ def test_forward_both_tile_policies(case, policy):
                                     inp.Wd_codes, inp.Wd_scales, k=k, return_hidden=True)
     G.assert_out_close(out, want)
     idx = layer.intermediate("topk_idx", T).cpu().numpy()
-    if np.array_equal(idx, r.idx):
+    # the block-scaled tiles keep H as hi/lo E4M3 rows, not bf16
+    mx = policy == 4 and d % 64 == 0 and I % 64 == 0 and min(d, I) >= 128
+    if np.array_equal(idx, r.idx) and not mx:
         c, o, p, _ = O.routing_tables(idx, E)
         H = O.bf16_to_f64(G.unpermute_chunks(layer.intermediate("h", T).cpu().numpy()))
         for e, (toks, h) in hidden.items():
             rms = np.sqrt(np.mean(h ** 2))
             assert np.all(np.abs(H[o[e]:o[e + 1]] - h) <= 2.0 ** -8 * np.abs(h) + 1e-3 * rms), e
+
+
+def _e4m3_to_f64(b):
+    b = b.astype(np.int64)
+    e, m = (b >> 3) & 15, b & 7
+    v = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1 + m / 8.0) * np.exp2(e - 7.0))
+    v = np.where((b & 0x7F) == 0x7F, np.nan, v)
+    return np.where(b >> 7, -v, v)
+
+
+def test_mx_split_is_exact_above_the_group_floor():
+    """hi/lo E4M3 split of bf16 rows: x = 2^(s_hi-127) hi + 2^(s_lo-127) lo, exact for
+    every element of at least 2^-13 of its group's max |x|, within 2^-21 of that max
+    otherwise (groups with max |x| >= 2^-116). Groups cover N(0,1), wide exponent
+    spreads, zeros and scales near both ends of that range."""
+    from sparse_moe_layer_05_b200 import binding as B
+    rng = np.random.default_rng(5)
+    R, K = 64, 2880
+    x = rng.standard_normal((R, K))
+    x *= np.exp2(rng.integers(-40, 40, size=(R, K // 32, 1)).astype(float)).repeat(32, 2).reshape(R, K)
+    x[1] = rng.standard_normal(K) * np.exp2(rng.uniform(-30, 0, size=K))  # far below the max
+    x[2] = 0.0
+    x[3, :32] = 0.0
+    x[4] = rng.standard_normal(K) * 2.0 ** 100
+    x[5] = rng.standard_normal(K) * 2.0 ** -105
+    xb = W.f32_to_bf16_bits(x.astype(np.float32))
+    hi = torch.empty((R, K), dtype=torch.uint8, device="cuda")
+    lo = torch.empty_like(hi)
+    sc = torch.empty((R, K // 32, 2), dtype=torch.uint8, device="cuda")
+    B.moe_mx_split_e4m3(_t(xb), R, K, hi, lo, sc)
+    torch.cuda.synchronize()
+    sc = sc.cpu().numpy().astype(np.int64)
+    s_hi = np.exp2(sc[..., 0] - 127.0).repeat(32, 1)
+    s_lo = np.exp2(sc[..., 1] - 127.0).repeat(32, 1)
+    rec = _e4m3_to_f64(hi.cpu().numpy()) * s_hi + _e4m3_to_f64(lo.cpu().numpy()) * s_lo
+    xv = O.bf16_to_f64(xb)
+    gmax = np.abs(xv).reshape(R, K // 32, 32).max(axis=2).repeat(32, 1)
+    big = np.abs(xv) >= 2.0 ** -13 * gmax
+    assert np.all(np.isfinite(rec))
+    assert np.array_equal(rec[big], xv[big])
+    assert np.all(np.abs(rec - xv)[~big] <= 2.0 ** -21 * gmax[~big])
+    assert np.all(sc[..., 1] == sc[..., 0] - 4)
 
 
 def test_forward_deterministic_and_hostio_equal():
