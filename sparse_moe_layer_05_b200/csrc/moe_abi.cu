@@ -18,7 +18,10 @@ int g_tile_policy = 0;
 
 // The block-scaled path reads the codes through 4-bit tensor maps: rows of a
 // multiple of 64 elements (at least 128) and 32-byte aligned code arrays.
-bool mx_shape_ok(int d, int I) { return d % 64 == 0 && I % 64 == 0 && d >= 128 && I >= 128; }
+bool mx_shape_ok(int d, int I) {
+  return d % 64 == 0 && I % 64 == 0 && d >= 128 && I >= 128 && d <= moe::kMxMaxK &&
+         I <= moe::kMxMaxK;
+}
 bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31) == 0; }
 
 int choose_tiles(int P, int E, bool mx_ok) {

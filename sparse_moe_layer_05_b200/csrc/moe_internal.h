@@ -78,6 +78,9 @@ cudaError_t launch_gemm_down_combine(const GroupedGemmProblem& p, int num_sms, c
 // Tokens per tile of the block-scaled GEMMs; token rows are stored per expert
 // padded to a multiple of this.
 constexpr int kMxNT = 32;
+// Largest d or I of the block-scaled path (a tile's weight scales, 128 rows of
+// K/32 bytes, are staged in shared memory).
+constexpr int kMxMaxK = 3072;
 constexpr int TILES_MX = 4;       // block-scaled tcgen05 GEMMs (E2M1 x hi/lo E4M3)
 
 // Rows of the padded token layout and bytes of its B-scale blocks.

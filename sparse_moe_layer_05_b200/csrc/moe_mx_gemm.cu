@@ -33,9 +33,9 @@
 //   warp 0      TMA producer: weight codes (E2M1 -> 8-bit containers), the hi
 //               and lo token rows, the tile's B scale block
 //   warp 1      TMEM allocator and UMMA issuer (one thread)
-//   warp 2      A-scale builder: gathers the k-block's E8M0 weight scales
-//               from global memory (four k-blocks ahead) into the layout
-//               tcgen05.cp reads
+//   warp 2      A-scale builder: turns the tile's E8M0 weight scales (one
+//               bulk copy per tile into shared memory, double-buffered) into
+//               the per-k-block layout tcgen05.cp reads
 //   warps 4-7   epilogue (TMEM lane quarters 0..3)
 //
 // K tail. The 4-bit tensor maps need row lengths in multiples of 128, so a K
@@ -224,7 +224,7 @@ template <int NT>
 struct MxCfg {
   static constexpr int MW = 128;                    // weight rows per tile
   static constexpr int N = 2 * NT;                  // UMMA N: hi and lo token columns
-  static constexpr int STAGES = 4;
+  static constexpr int STAGES = 3;
   static constexpr int A_BYTES = 128 * 128;         // E2M1 in 8-bit containers
   static constexpr int A_TX = 128 * 64;             // packed bytes the TMA counts
   static constexpr int B_BYTES = N * 128;
@@ -233,8 +233,10 @@ struct MxCfg {
   static constexpr int OFF_SFA = OFF_B + B_BYTES;
   static constexpr int OFF_SFB = OFF_SFA + 512;
   static constexpr int STAGE_BYTES = ((OFF_SFB + SFB_BYTES) + 1023) / 1024 * 1024;
-  static constexpr int OFF_BAR = STAGES * STAGE_BYTES;
-  static constexpr int NUM_BARS = 2 * STAGES + 4;
+  static constexpr int OFF_TS = STAGES * STAGE_BYTES;   // two tile-scale buffers
+  static constexpr int TS_BYTES = 128 * (kMxMaxK / 32);
+  static constexpr int OFF_BAR = OFF_TS + 2 * TS_BYTES;
+  static constexpr int NUM_BARS = 2 * STAGES + 8;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TAB = OFF_MISC + 16;
   static constexpr int OFF_XCH = OFF_TAB + 3 * (kMaxE + 1) * 4;
@@ -272,10 +274,6 @@ struct MxArgs {
 
 __device__ __forceinline__ float silu_mx(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-__device__ __forceinline__ uint16_t ldg_u16(const uint8_t* p) {
-  return __ldg(reinterpret_cast<const unsigned short*>(p));
-}
-
 template <int EPI, int NT>
 __global__ void __launch_bounds__(256, 2)
     grouped_mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -294,6 +292,8 @@ __global__ void __launch_bounds__(256, 2)
   auto bar_empty = [&](int s) { return bar0 + 8u * (C::STAGES + s); };
   auto bar_accFull = [&](int b) { return bar0 + 8u * (2 * C::STAGES + b); };
   auto bar_accEmpty = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 2 + b); };
+  auto bar_tsFull = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 4 + b); };
+  auto bar_tsEmpty = [&](int b) { return bar0 + 8u * (2 * C::STAGES + 6 + b); };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   int* s_off = reinterpret_cast<int*>(smem + C::OFF_TAB);
@@ -323,6 +323,8 @@ __global__ void __launch_bounds__(256, 2)
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_accFull(b), 1);
       mbar_init(bar_accEmpty(b), 4 * 32);
+      mbar_init(bar_tsFull(b), 1);
+      mbar_init(bar_tsEmpty(b), 1);
     }
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -365,13 +367,31 @@ __global__ void __launch_bounds__(256, 2)
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer --
     if (lane == 0) {
-      int s = 0, ph = 0;
+      int s = 0, ph = 0, it = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
         int e, wb, tb, rows;
         decode(tile, e, wb, tb, rows);
         const int tok_tile = s_tb[e] + tb;
         const int row_b = tok_tile * NT;
+        // the tile's weight scales: rows of G bytes, contiguous per block
+        const int b = it & 1;
+        if (!(ok = mbar_wait(bar_tsEmpty(b), ((it >> 1) & 1) ^ 1, abort_flag, args.status))) break;
+        const uint32_t ts = sbase + C::OFF_TS + b * C::TS_BYTES;
+        if (EPI == EPI_SWIGLU) {
+          const uint32_t half = 64u * G;
+          mbar_expect_tx(bar_tsFull(b), 2 * half);
+          bulk_load(ts, args.scales + (static_cast<size_t>(e) * 2 * args.I + wb * 64) * G, half,
+                    bar_tsFull(b));
+          bulk_load(ts + half,
+                    args.scales + (static_cast<size_t>(e) * 2 * args.I + args.I + wb * 64) * G,
+                    half, bar_tsFull(b));
+        } else {
+          const uint32_t bytes = static_cast<uint32_t>(min(128, args.rows_per_expert - wb * 128)) * G;
+          mbar_expect_tx(bar_tsFull(b), bytes);
+          bulk_load(ts, args.scales + (static_cast<size_t>(e) * args.rows_per_expert + wb * 128) * G,
+                    bytes, bar_tsFull(b));
+        }
         for (int kb = 0; kb < KB; ++kb) {
           if (!(ok = mbar_wait(bar_empty(s), ph ^ 1, abort_flag, args.status))) break;
           const uint32_t st = sbase + s * C::STAGE_BYTES;
@@ -401,69 +421,44 @@ __global__ void __launch_bounds__(256, 2)
     }
   } else if (warp == 2) {
     // -------------------------------------------------- A-scale builder --
-    // Lane l owns shared-memory rows l, l+32, l+64, l+96 of the A tile; for
-    // each it loads the 4 scale bytes of the k-block (2-byte aligned: two
-    // 16-bit loads) four k-blocks ahead of their use.
-    constexpr int PD = 4;
-    const uint8_t* scales = args.scales;
-    const int rpe = args.rows_per_expert;
-    auto load_words = [&](int tile, int kb, uint32_t (&w)[4]) {
-      int e, wb, tb, rows;
-      decode(tile, e, wb, tb, rows);
-      const int gs = (tail && kb == KB - 1) ? G - 4 : 4 * kb;
+    // Lane l fills bytes 16l..16l+15 of the k-block's 512-byte atom: the 4
+    // scale bytes of A-tile rows l, l+32, l+64, l+96, read from the tile's
+    // scale block (2-byte aligned rows of G bytes).
+    int srow[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        int r;
-        bool valid;
-        if (EPI == EPI_SWIGLU) {
-          const int jj = wb * 64 + 16 * j + (lane & 15);
-          valid = jj < args.I;
-          r = (lane < 16) ? jj : args.I + jj;
-        } else {
-          r = wb * 128 + 32 * j + lane;
-          valid = r < rpe;
-        }
-        if (valid) {
-          const uint8_t* p = scales + (static_cast<size_t>(e) * rpe + r) * G + gs;
-          w[j] = static_cast<uint32_t>(ldg_u16(p)) | (static_cast<uint32_t>(ldg_u16(p + 2)) << 16);
-        } else {
-          w[j] = 0x7F7F7F7Fu;
-        }
-      }
-    };
-    // (tile, kb) iterators: `c` consumes, `f` fetches PD steps ahead
-    int c_tile = blockIdx.x, c_kb = 0;
-    int f_tile = blockIdx.x, f_kb = 0;
-    auto advance = [&](int& tile, int& kb) {
-      if (++kb == KB) { kb = 0; tile += gridDim.x; }
-    };
-    uint32_t buf[PD][4];
-#pragma unroll
-    for (int u = 0; u < PD; ++u) {
-      if (f_tile < total) {
-        load_words(f_tile, f_kb, buf[u]);
-        advance(f_tile, f_kb);
-      }
+    for (int j = 0; j < 4; ++j) {
+      if (EPI == EPI_SWIGLU)   // gate rows first, then up rows, 64 each
+        srow[j] = (lane < 16) ? 16 * j + lane : 64 + 16 * j + (lane - 16);
+      else
+        srow[j] = 32 * j + lane;
     }
-    int s = 0, ph = 0;
+    int s = 0, ph = 0, it = 0;
     bool ok = true;
-    while (ok && c_tile < total) {
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+      const int b = it & 1;
+      if (!(ok = mbar_wait(bar_tsFull(b), (it >> 1) & 1, abort_flag, args.status))) break;
+      const uint8_t* ts = smem + C::OFF_TS + b * C::TS_BYTES;
+      for (int kb = 0; kb < KB; ++kb) {
+        const int gs = (tail && kb == KB - 1) ? G - 4 : 4 * kb;
+        uint32_t w[4];
 #pragma unroll
-      for (int u = 0; u < PD; ++u) {
-        if (!ok || c_tile >= total) break;
+        for (int j = 0; j < 4; ++j) {
+          const uint16_t* p = reinterpret_cast<const uint16_t*>(ts + srow[j] * G + gs);
+          w[j] = static_cast<uint32_t>(p[0]) | (static_cast<uint32_t>(p[1]) << 16);
+        }
         if (!(ok = mbar_wait(bar_empty(s), ph ^ 1, abort_flag, args.status))) break;
         *reinterpret_cast<uint4*>(smem + s * C::STAGE_BYTES + C::OFF_SFA + lane * 16) =
-            make_uint4(buf[u][0], buf[u][1], buf[u][2], buf[u][3]);
+            make_uint4(w[0], w[1], w[2], w[3]);
+        // orders this k-block's shared-memory reads and writes before the
+        // async-proxy accesses that follow (tcgen05.cp of the atom; the next
+        // bulk copy into the tile-scale buffer)
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_full(s));
         if (++s == C::STAGES) { s = 0; ph ^= 1; }
-        advance(c_tile, c_kb);
-        if (f_tile < total) {
-          load_words(f_tile, f_kb, buf[u]);
-          advance(f_tile, f_kb);
-        }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_tsEmpty(b));
     }
   } else if (warp == 1) {
     // -------------------------------------------------------- UMMA issuer --
