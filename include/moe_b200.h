@@ -106,8 +106,8 @@ MOE_API int moe_version(void);
  * the tensor core, and each bf16 activation (and H) row split per 32 elements
  * into two E4M3 terms (hi and lo) with E8M0 scales; the split is exact for
  * elements of at least 2^-13 of their group's max |x|, smaller ones keep an
- * error below 2^-21 of it. 128 weight rows x 32 tokens per tile, two CTAs
- * per SM. It needs d and I multiples of 64 in [128, 3072] and 32-byte
+ * error below 2^-21 of it. 128 weight rows x 16 tokens per tile, two CTAs
+ * per SM with two UMMA-issuing threads each. It needs d and I multiples of 64 in [128, 3072] and 32-byte
  * aligned code arrays; otherwise policy 4 picks as policy 0 does.
  * All policies compute the same function within the output tolerance. Not
  * thread-safe against concurrent forward calls. MOE_ERR_INVALID_ARG for other

@@ -77,7 +77,7 @@ cudaError_t launch_gemm_down_combine(const GroupedGemmProblem& p, int num_sms, c
 // ---------------------------------------------- block-scaled (MX) path ----
 // Tokens per tile of the block-scaled GEMMs; token rows are stored per expert
 // padded to a multiple of this.
-constexpr int kMxNT = 32;
+constexpr int kMxNT = 16;
 // Largest d or I of the block-scaled path (a tile's weight scales, 128 rows of
 // K/32 bytes, are staged in shared memory).
 constexpr int kMxMaxK = 3072;

@@ -25,14 +25,25 @@
 // Tiles. 128 weight rows (UMMA M) x NT tokens (UMMA N = 2 NT), 128 K per
 // shared-memory stage. Token rows live in a per-expert padded layout (each
 // expert's segment rounded up to a multiple of NT rows), so a token tile is
-// NT consecutive rows and its B scales one contiguous block. Two CTAs share an
-// SM; each has one MMA-issuing thread, which keeps the tensor pipe busy when
-// each UMMA is short (few tokens per expert).
+// NT consecutive rows and its B scales one contiguous block.
+//
+// Issue rate. With few tokens per expert each UMMA is short, and one thread
+// issuing the UMMAs, scale copies and commits of a k-block bounds the rate
+// (the issue latency of these tcgen05 operations, not the tensor pipe, is the
+// limit; it scales with the number of issuing threads per SM). So two CTAs
+// share an SM and each has two issuing threads: the CTA's k-blocks, numbered
+// q = 0, 1, 2, ... across its tiles, go to issuer q % 2, each accumulating
+// into its own TMEM buffer; the epilogue adds the two in a fixed order. With
+// an even number of stages, stage q % STAGES is always served by the same
+// issuer, so every waiter of a stage's barrier waits for its phases in
+// order (a parity wait cannot tell phase k done from phase k-1 pending).
 //
 // Warp roles (256 threads per CTA):
-//   warp 0      TMA producer: weight codes (E2M1 -> 8-bit containers), the hi
-//               and lo token rows, the tile's B scale block
-//   warp 1      TMEM allocator and UMMA issuer (one thread)
+//   warp 0      TMA producer, three copies per k-block: the weight codes
+//               (E2M1 -> 8-bit containers, one box), the hi and lo token rows
+//               (one box over both), the B scale block
+//   warp 1      TMEM allocator and UMMA issuer 0 (even q)
+//   warp 3      UMMA issuer 1 (odd q)
 //   warp 2      A-scale builder: turns the tile's E8M0 weight scales (one
 //               bulk copy per tile into shared memory, double-buffered) into
 //               the per-k-block layout tcgen05.cp reads
@@ -69,15 +80,17 @@ __host__ __device__ __forceinline__ void group_to_kblock(int g, int G, int KB, i
 }
 
 // Byte offset of the B scale of token n (0..NT-1), term h (0 hi, 1 lo), K
-// step kk inside the block of one (token tile, k-block): TMEM column n/32 of
-// term h is word w = h*NT/32 + n/32, four words per 512-byte tcgen05.cp atom,
-// lane n%32 holding 16 bytes.
+// step kk inside the block of one (token tile, k-block). B column c = h*NT + n
+// of the UMMA takes its scale from TMEM lane c%32 of column c/32: word w =
+// c/32 of lane c%32, four words (16 bytes) per lane in a 512-byte tcgen05.cp
+// atom.
 __device__ __forceinline__ int sfb_offset(int NT, int n, int h, int kk) {
-  const int w = h * (NT / 32) + (n >> 5);
-  return (w >> 2) * 512 + (n & 31) * 16 + (w & 3) * 4 + kk;
+  const int c = h * NT + n;
+  const int w = c >> 5;
+  return (w >> 2) * 512 + (c & 31) * 16 + (w & 3) * 4 + kk;
 }
 
-__host__ __device__ constexpr int sfb_block_bytes(int NT) { return 512 * ((NT + 63) / 64); }
+__host__ __device__ constexpr int sfb_block_bytes(int NT) { return 512 * ((2 * NT + 127) / 128); }
 
 // Splits 32 fp32 values (already bf16-exact) into hi / lo E4M3 bytes given the
 // group's max |v|; returns the hi scale byte (lo's is 4 less).
@@ -224,7 +237,7 @@ template <int NT>
 struct MxCfg {
   static constexpr int MW = 128;                    // weight rows per tile
   static constexpr int N = 2 * NT;                  // UMMA N: hi and lo token columns
-  static constexpr int STAGES = 3;
+  static constexpr int STAGES = 4;   // even: stage s is always consumed by issuer s % 2
   static constexpr int A_BYTES = 128 * 128;         // E2M1 in 8-bit containers
   static constexpr int A_TX = 128 * 64;             // packed bytes the TMA counts
   static constexpr int B_BYTES = N * 128;
@@ -244,10 +257,12 @@ struct MxCfg {
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
   static constexpr int NUM_THREADS = 256;
   static constexpr int TMEM_COLS = 256;
-  static constexpr int SFA_COL = 2 * N;             // after the two accumulator buffers
-  static constexpr int SFB_COL = SFA_COL + 4;
+  // accumulators: issuer u, tile buffer b at column (2u + b) N; then each
+  // issuer's scale columns (A: 4, B: 4 per 512-byte atom)
+  static constexpr int SF_COL0 = 4 * N;
+  static constexpr int SF_COLS = 4 + 4 * (SFB_BYTES / 512);
   static constexpr int TX_BYTES = A_TX + B_BYTES + SFB_BYTES;
-  static_assert(SFB_COL + 4 * ((SFB_BYTES + 511) / 512) <= TMEM_COLS, "TMEM budget");
+  static_assert(SF_COL0 + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(2 * SMEM_ALLOC + 2048 <= 233472, "two CTAs per SM");
   static_assert(OFF_B % 1024 == 0 && (NT * 128) % 1024 == 0, "swizzle atom alignment");
 };
@@ -278,8 +293,7 @@ template <int EPI, int NT>
 __global__ void __launch_bounds__(256, 2)
     grouped_mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmAt,
-                           const __grid_constant__ CUtensorMap tmBh,
-                           const __grid_constant__ CUtensorMap tmBl, const MxArgs args) {
+                           const __grid_constant__ CUtensorMap tmB, const MxArgs args) {
   using C = MxCfg<NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -321,7 +335,7 @@ __global__ void __launch_bounds__(256, 2)
       mbar_init(bar_empty(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_accFull(b), 1);
+      mbar_init(bar_accFull(b), 2);     // one commit per issuer
       mbar_init(bar_accEmpty(b), 4 * 32);
       mbar_init(bar_tsFull(b), 1);
       mbar_init(bar_tsEmpty(b), 1);
@@ -329,8 +343,7 @@ __global__ void __launch_bounds__(256, 2)
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmAt);
-    tma_prefetch_desc(&tmBh);
-    tma_prefetch_desc(&tmBl);
+    tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(misc), C::TMEM_COLS);
@@ -345,8 +358,7 @@ __global__ void __launch_bounds__(256, 2)
   const int K = args.K;
   const int G = K / 32;
   const int KB = (K + 127) / 128;
-  const bool tail = (K % 128) != 0;
-  const int tail_k0 = 4 - (K % 128) / 32;   // first K step issued in the tail k-block
+  const bool tail = (K % 128) != 0;         // K % 64 == 0: the tail k-block has 2 K steps
   // tile -> (expert, weight block, token block), weight-block major inside an
   // expert so that neighbouring CTAs stream neighbouring weights
   auto decode = [&](int tile, int& e, int& wb, int& tb, int& rows) {
@@ -367,16 +379,14 @@ __global__ void __launch_bounds__(256, 2)
   if (warp == 0) {
     // ------------------------------------------------------- TMA producer --
     if (lane == 0) {
-      int s = 0, ph = 0, it = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+      // The tile's weight scales (rows of G bytes, contiguous per block) go to
+      // tile-scale buffer it&1; the next tile's are requested a few k-blocks
+      // into the current tile, once the builder has released that buffer.
+      auto load_tile_scales = [&](int tile, int itx) -> bool {
         int e, wb, tb, rows;
         decode(tile, e, wb, tb, rows);
-        const int tok_tile = s_tb[e] + tb;
-        const int row_b = tok_tile * NT;
-        // the tile's weight scales: rows of G bytes, contiguous per block
-        const int b = it & 1;
-        if (!(ok = mbar_wait(bar_tsEmpty(b), ((it >> 1) & 1) ^ 1, abort_flag, args.status))) break;
+        const int b = itx & 1;
+        if (!mbar_wait(bar_tsEmpty(b), ((itx >> 1) & 1) ^ 1, abort_flag, args.status)) return false;
         const uint32_t ts = sbase + C::OFF_TS + b * C::TS_BYTES;
         if (EPI == EPI_SWIGLU) {
           const uint32_t half = 64u * G;
@@ -387,11 +397,22 @@ __global__ void __launch_bounds__(256, 2)
                     args.scales + (static_cast<size_t>(e) * 2 * args.I + args.I + wb * 64) * G,
                     half, bar_tsFull(b));
         } else {
-          const uint32_t bytes = static_cast<uint32_t>(min(128, args.rows_per_expert - wb * 128)) * G;
+          const uint32_t bytes =
+              static_cast<uint32_t>(min(128, args.rows_per_expert - wb * 128)) * G;
           mbar_expect_tx(bar_tsFull(b), bytes);
           bulk_load(ts, args.scales + (static_cast<size_t>(e) * args.rows_per_expert + wb * 128) * G,
                     bytes, bar_tsFull(b));
         }
+        return true;
+      };
+      int s = 0, ph = 0, it = 0;
+      bool ok = blockIdx.x >= total || load_tile_scales(blockIdx.x, 0);
+      const int kb_next = min(3, KB - 1);
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+        int e, wb, tb, rows;
+        decode(tile, e, wb, tb, rows);
+        const int tok_tile = s_tb[e] + tb;
+        const int row_b = tok_tile * NT;
         for (int kb = 0; kb < KB; ++kb) {
           if (!(ok = mbar_wait(bar_empty(s), ph ^ 1, abort_flag, args.status))) break;
           const uint32_t st = sbase + s * C::STAGE_BYTES;
@@ -401,21 +422,21 @@ __global__ void __launch_bounds__(256, 2)
           const CUtensorMap* am = last_tail ? &tmAt : &tmA;
           const int ax = last_tail ? 0 : kb * 128;
           if (EPI == EPI_SWIGLU) {
-            // four boxes of 16 gate rows + the same 16 up rows (TMEM lanes
-            // 32q..32q+15 gate, 32q+16..32q+31 up)
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-              tma_load_3d(st + q * 4096, am, ax, wb * 64 + 16 * q, 2 * e, fb);
+            // row blocks q = 0..3 of 16 gate rows then the same 16 up rows
+            // (TMEM lanes 32q..32q+15 gate, 32q+16..32q+31 up)
+            tma_load_4d(st, am, ax, 0, 2 * e, 4 * wb, fb);
           } else {
             tma_load_3d(st, am, ax, wb * 128, e, fb);
           }
           const int bx = last_tail ? K - 128 : kb * 128;
-          tma_load_2d(st + C::OFF_B, &tmBh, bx, row_b, fb);
-          tma_load_2d(st + C::OFF_B + NT * 128, &tmBl, bx, row_b, fb);
+          tma_load_3d(st + C::OFF_B, &tmB, bx, row_b, 0, fb);   // hi rows, then lo rows
           bulk_load(st + C::OFF_SFB,
                     args.sfb + (static_cast<size_t>(tok_tile) * KB + kb) * C::SFB_BYTES,
                     C::SFB_BYTES, fb);
           if (++s == C::STAGES) { s = 0; ph ^= 1; }
+          if (kb == kb_next && tile + static_cast<int>(gridDim.x) < total &&
+              !(ok = load_tile_scales(tile + gridDim.x, it + 1)))
+            break;
         }
       }
     }
@@ -460,36 +481,55 @@ __global__ void __launch_bounds__(256, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_tsEmpty(b));
     }
-  } else if (warp == 1) {
-    // -------------------------------------------------------- UMMA issuer --
+  } else if (warp == 1 || warp == 3) {
+    // ------------------------------------------------------- UMMA issuers --
+    // Issuer u takes the k-blocks with q % 2 == u (q counts this CTA's
+    // k-blocks across tiles), i.e. the stages s with s % 2 == u; the other
+    // issuer's k-blocks are stepped over without touching their barriers.
+    const int u = warp == 1 ? 0 : 1;
     if (lane == 0) {
       const uint32_t idesc0 = idesc_mx_e2m1_e4m3(C::MW, C::N, 0, 0);
-      const uint32_t sfa_t = tmem_base + C::SFA_COL, sfb_t = tmem_base + C::SFB_COL;
-      int s = 0, ph = 0, it = 0;
+      const uint32_t sfa_t = tmem_base + C::SF_COL0 + u * C::SF_COLS, sfb_t = sfa_t + 4;
+      int s = 0, ph = 0, it = 0, q = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
         const int ab = it & 1;
         const uint32_t ap = (it >> 1) & 1;
         if (!(ok = mbar_wait(bar_accEmpty(ab), ap ^ 1, abort_flag, args.status))) break;
         tc_fence_after();
-        const uint32_t d = tmem_base + ab * C::N;
-        for (int kb = 0; kb < KB; ++kb) {
-          if (!(ok = mbar_wait(bar_full(s), ph, abort_flag, args.status))) break;
-          tc_fence_after();
-          const uint32_t st = sbase + s * C::STAGE_BYTES;
-          tmem_cp_32x128b_x4(sfa_t, sdesc_k_noswizzle(st + C::OFF_SFA, 128));
+        const uint32_t d = tmem_base + (2 * u + ab) * C::N;
+        uint32_t accum = 0;   // the issuer's first k-block of the tile overwrites its buffer
+        for (int kb = 0; kb < KB; ++kb, ++q) {
+          if ((q & 1) == u) {
+            if (!(ok = mbar_wait(bar_full(s), ph, abort_flag, args.status))) break;
+            tc_fence_after();
+            const uint32_t st = sbase + s * C::STAGE_BYTES;
+            tmem_cp_32x128b_x4(sfa_t, sdesc_k_noswizzle(st + C::OFF_SFA, 128));
 #pragma unroll
-          for (int a = 0; a < C::SFB_BYTES / 512; ++a)
-            tmem_cp_32x128b_x4(sfb_t + 4 * a, sdesc_k_noswizzle(st + C::OFF_SFB + 512 * a, 128));
-          const int k0 = (tail && kb == KB - 1) ? tail_k0 : 0;
-          for (int kk = k0; kk < 4; ++kk) {
-            const uint32_t id = idesc0 | (static_cast<uint32_t>(kk) << 4) |
-                                (static_cast<uint32_t>(kk) << 29);
-            umma_mxf8f6f4(d, sdesc_k_sw128(st + kk * 32), sdesc_k_sw128(st + C::OFF_B + kk * 32),
-                          id, sfa_t | (static_cast<uint32_t>(kk) << 30),
-                          sfb_t | (static_cast<uint32_t>(kk) << 30), (kb > 0 || kk > k0) ? 1u : 0u);
+            for (int a = 0; a < C::SFB_BYTES / 512; ++a)
+              tmem_cp_32x128b_x4(sfb_t + 4 * a, sdesc_k_noswizzle(st + C::OFF_SFB + 512 * a, 128));
+            // K steps with compile-time indices (a data-dependent trip count
+            // here measurably slows the issue of each UMMA); the tail k-block
+            // of a K that is 64 mod 128 issues its last two steps only
+            auto step = [&](const int kk, const uint32_t acc) {
+              umma_mxf8f6f4(d, sdesc_k_sw128(st + kk * 32), sdesc_k_sw128(st + C::OFF_B + kk * 32),
+                            idesc0 | (static_cast<uint32_t>(kk) << 4) |
+                                (static_cast<uint32_t>(kk) << 29),
+                            sfa_t | (static_cast<uint32_t>(kk) << 30),
+                            sfb_t | (static_cast<uint32_t>(kk) << 30), acc);
+            };
+            if (!(tail && kb == KB - 1)) {
+              step(0, accum);
+              step(1, 1u);
+              step(2, 1u);
+              step(3, 1u);
+            } else {
+              step(2, accum);
+              step(3, 1u);
+            }
+            accum = 1;
+            umma_commit(bar_empty(s));
           }
-          umma_commit(bar_empty(s));
           if (++s == C::STAGES) { s = 0; ph ^= 1; }
         }
         if (ok) umma_commit(bar_accFull(ab));
@@ -513,14 +553,31 @@ __global__ void __launch_bounds__(256, 2)
       float y[NT];
       if (ok) {
         tc_fence_after();
-        const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + ab * C::N;
+        // y = (issuer 0: hi + lo) + (issuer 1: hi + lo); with a single
+        // k-block per tile only issuer (it*KB) % 2 wrote its buffer
+        const uint32_t lanes = static_cast<uint32_t>(quad * 32) << 16;
+        const bool use0 = KB > 1 || ((it * KB) & 1) == 0;
+        const bool use1 = KB > 1 || ((it * KB) & 1) == 1;
+        const uint32_t t0 = tmem_base + lanes + ab * C::N;
+        const uint32_t t1 = tmem_base + lanes + (2 + ab) * C::N;
 #pragma unroll
         for (int c = 0; c < NT; c += 16) {
           uint32_t a[16], b[16];
-          tmem_ld16_sync(taddr + c, a);
-          tmem_ld16_sync(taddr + NT + c, b);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) y[c + i] = __uint_as_float(a[i]) + __uint_as_float(b[i]);
+          for (int i = 0; i < 16; ++i) y[c + i] = 0.f;
+          if (use0) {
+            tmem_ld16_sync(t0 + c, a);
+            tmem_ld16_sync(t0 + NT + c, b);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) y[c + i] = __uint_as_float(a[i]) + __uint_as_float(b[i]);
+          }
+          if (use1) {
+            tmem_ld16_sync(t1 + c, a);
+            tmem_ld16_sync(t1 + NT + c, b);
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              y[c + i] += __uint_as_float(a[i]) + __uint_as_float(b[i]);
+          }
         }
         tc_fence_before();
         mbar_arrive(bar_accEmpty(ab));     // accumulators are in registers now
@@ -629,32 +686,37 @@ bool encode_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* ba
                 const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
-  const cuuint32_t es[3] = {1, 1, 1};
+  const cuuint32_t es[5] = {1, 1, 1, 1, 1};   // element strides, one per dimension (rank <= 5)
+  if (rank < 1 || rank > 5) return false;
   return enc(m, dt, rank, const_cast<void*>(base), dims, strides, box, es,
              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// E2M1 codes as 3D (K elements, rows, planes): the main map covers the first
+// E2M1 code maps (K elements first, then `rank`-1 row dimensions given by
+// dims_rest / strides / box_rest): the main map covers the first
 // 128*floor(K/128) elements of each row, the tail map the last 128 (based
 // (K-128)/2 bytes into the row); both widen to 8-bit containers.
 bool make_code_maps(CUtensorMap* main_map, CUtensorMap* tail_map, const uint8_t* codes, int K,
-                    int rows, int planes, int box_rows, int box_planes) {
-  const cuuint64_t rb = static_cast<cuuint64_t>(K / 2);
-  const cuuint64_t strides[2] = {rb, rb * static_cast<cuuint64_t>(rows)};
-  const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(box_rows),
-                             static_cast<cuuint32_t>(box_planes)};
+                    int rank, const cuuint64_t* dims_rest, const cuuint64_t* strides,
+                    const cuuint32_t* box_rest) {
+  cuuint64_t dims[5];
+  cuuint32_t box[5];
+  for (int i = 1; i < rank; ++i) {
+    dims[i] = dims_rest[i - 1];
+    box[i] = box_rest[i - 1];
+  }
+  box[0] = 128;
   const int kmain = (K / 128) * 128;
   bool ok = true;
   if (kmain > 0) {
-    const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kmain), static_cast<cuuint64_t>(rows),
-                                static_cast<cuuint64_t>(planes)};
-    ok = encode_map(main_map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, codes, dims, strides, box);
+    dims[0] = static_cast<cuuint64_t>(kmain);
+    ok = encode_map(main_map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, rank, codes, dims, strides,
+                    box);
   }
   if (ok && (K % 128) != 0) {
-    const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(rows),
-                                static_cast<cuuint64_t>(planes)};
-    ok = encode_map(tail_map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, codes + (K - 128) / 2,
+    dims[0] = 128;
+    ok = encode_map(tail_map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, rank, codes + (K - 128) / 2,
                     dims, strides, box);
   } else if (ok) {
     *tail_map = *main_map;
@@ -663,17 +725,21 @@ bool make_code_maps(CUtensorMap* main_map, CUtensorMap* tail_map, const uint8_t*
   return ok;
 }
 
-// E4M3 token rows [rows][K], box 128 x NT.
-bool make_tok8_map(CUtensorMap* m, const uint8_t* base, int rows, int K, int nt) {
-  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
-  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
-  const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(nt)};
-  return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base, dims, strides, box);
+// E4M3 token rows: hi rows [rows][K] followed by lo rows [rows][K], as one
+// (K, rows, 2) tensor; box 128 x NT x 2 (hi tile, then lo tile).
+bool make_tok8_map(CUtensorMap* m, const uint8_t* hi, int rows, int K, int nt) {
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows), 2};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(K),
+                                 static_cast<cuuint64_t>(K) * static_cast<cuuint64_t>(rows)};
+  const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(nt), 2};
+  return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, hi, dims, strides, box);
 }
 
 template <int EPI, int NT>
 cudaError_t launch_mx_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st) {
   using C = MxCfg<NT>;
+  // the kernel assumes K % 64 == 0 (tail k-blocks of 2 steps) and K <= kMxMaxK
+  if (p.K % 64 != 0 || p.K < 128 || p.K > kMxMaxK) return cudaErrorInvalidValue;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
@@ -684,14 +750,27 @@ cudaError_t launch_mx_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st)
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
-  CUtensorMap tmA, tmAt, tmBh, tmBl;
+  // the hi and lo token rows are read as the two planes of one tensor
+  if (p.b_lo != p.b_hi + static_cast<size_t>(p.tok_rows) * p.K) return cudaErrorInvalidValue;
+  CUtensorMap tmA, tmAt, tmB;
+  const cuuint64_t rb = static_cast<cuuint64_t>(p.K / 2);
   bool ok;
-  if (EPI == EPI_SWIGLU)
-    ok = make_code_maps(&tmA, &tmAt, p.codes, p.K, p.I, 2 * p.E, 16, 2);
-  else
-    ok = make_code_maps(&tmA, &tmAt, p.codes, p.K, p.n_out, p.E, 128, 1);
-  ok = ok && make_tok8_map(&tmBh, p.b_hi, p.tok_rows, p.K, NT) &&
-       make_tok8_map(&tmBl, p.b_lo, p.tok_rows, p.K, NT);
+  if (EPI == EPI_SWIGLU) {
+    // codes [E][2][I][K/2] as (K, 16 rows, 2E planes, I/16 row blocks): one
+    // box = 4 row blocks x (16 gate rows, 16 up rows)
+    const cuuint64_t dims[3] = {16, static_cast<cuuint64_t>(2 * p.E),
+                                static_cast<cuuint64_t>(p.I / 16)};
+    const cuuint64_t strides[3] = {rb, rb * static_cast<cuuint64_t>(p.I), rb * 16};
+    const cuuint32_t box[3] = {16, 2, 4};
+    ok = make_code_maps(&tmA, &tmAt, p.codes, p.K, 4, dims, strides, box);
+  } else {
+    // codes [E][d][K/2] as (K, d rows, E): one box = 128 rows
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(p.n_out), static_cast<cuuint64_t>(p.E)};
+    const cuuint64_t strides[2] = {rb, rb * static_cast<cuuint64_t>(p.n_out)};
+    const cuuint32_t box[2] = {128, 1};
+    ok = make_code_maps(&tmA, &tmAt, p.codes, p.K, 3, dims, strides, box);
+  }
+  ok = ok && make_tok8_map(&tmB, p.b_hi, p.tok_rows, p.K, NT);
   if (!ok) return cudaErrorInvalidValue;
   MxArgs a;
   a.offsets = p.offsets;
@@ -721,7 +800,7 @@ cudaError_t launch_mx_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st)
   if (tiles_bound < grid) grid = tiles_bound;
   if (grid < 1) grid = 1;
   grouped_mx_gemm_kernel<EPI, NT><<<static_cast<int>(grid), C::NUM_THREADS, C::SMEM_ALLOC, st>>>(
-      tmA, tmAt, tmBh, tmBl, a);
+      tmA, tmAt, tmB, a);
   return cudaGetLastError();
 }
 
