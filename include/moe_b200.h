@@ -92,8 +92,9 @@ MOE_API int moe_version(void);
 /*
  * Tile policy of the grouped GEMMs, process-wide: 0 (default) picks by shape
  * from the average number of routed rows per expert, P/E with P = T*k:
- *   P/E < 32        swapped-operand tiles (128 weight rows x 64 tokens, the
- *                   decoded weights as the UMMA A operand; decode batches),
+ *   P/E < 32        block-scaled tiles (policy 4 below) where the shape allows
+ *                   them, else swapped-operand tiles (128 weight rows x 64
+ *                   tokens, the decoded weights as the UMMA A operand),
  *   32 <= P/E < 192 single-CTA tiles (256 x 128, the second 128-row half
  *                   skipped for short expert tails),
  *   P/E >= 192      CTA-pair tiles (a 2-CTA cluster computes 256 x 240 tiles

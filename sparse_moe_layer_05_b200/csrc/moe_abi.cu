@@ -28,11 +28,12 @@ int choose_tiles(int P, int E, bool mx_ok) {
   if (g_tile_policy == 4 && mx_ok) return moe::TILES_MX;
   if (g_tile_policy >= 1 && g_tile_policy <= 3) return g_tile_policy;
   const int64_t p = P, e = E;
-  // Few routed rows per expert (decode): stream the weights with the
-  // swapped-operand kernel. From ~192 rows per expert the CTA-pair tiles were
-  // measured fastest; in between the single-CTA tiles, which skip empty
-  // 128-row halves.
-  if (p < 32 * e) return moe::TILES_SWAP;
+  // Few routed rows per expert (decode): stream the weights, with the
+  // block-scaled tiles where the shape allows (no CUDA-core weight decode),
+  // else the swapped-operand kernel. From ~192 rows per expert the CTA-pair
+  // tiles were measured fastest; in between the single-CTA tiles, which skip
+  // empty 128-row halves.
+  if (p < 32 * e) return mx_ok ? moe::TILES_MX : moe::TILES_SWAP;
   if (p >= 192 * e) return moe::TILES_PAIR;
   return moe::TILES_SINGLE;
 }

@@ -127,6 +127,7 @@ FORWARD_CASES = [
 
 @pytest.mark.parametrize("case", FORWARD_CASES, ids=[c[0] for c in FORWARD_CASES])
 def test_forward_matches_oracle(case):
+    from sparse_moe_layer_05_b200 import binding as B
     name, d, I, E, k, T, seed = case
     if name == "fixture":
         inp = W.make_inputs("fixture")
@@ -143,7 +144,10 @@ def test_forward_matches_oracle(case):
     perm = layer.intermediate("perm", T).cpu().numpy()
     c, o, p, _ = O.routing_tables(idx, E)
     assert np.array_equal(perm, p)
-    if np.array_equal(idx, r.idx):
+    # the block-scaled path (9 launches: no scale transposes) keeps x and H as
+    # hi/lo E4M3 rows, so the bf16 intermediates exist only on the other paths
+    bf16_path = B.moe_forward_launch_count(E, k, T, d, I) == len(B.STAGES)
+    if np.array_equal(idx, r.idx) and bf16_path:
         H = O.bf16_to_f64(G.unpermute_chunks(layer.intermediate("h", T).cpu().numpy()))
         xp = G.unpermute_chunks(layer.intermediate("xp", T).cpu().numpy())
         assert np.array_equal(xp, inp.x[perm // k])
