@@ -229,7 +229,10 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     uint8_t* qh = at<uint8_t>(ws, L.pub.h);
     uint8_t* sfbx = at<uint8_t>(ws, L.gu_scales_t);
     uint8_t* sfbh = at<uint8_t>(ws, L.d_scales_t);
-    MOE_CUDA(moe::launch_mx_quant_gather(x, perm, offsets, E, P, k, d, qx, qx + tr * d, sfbx, st));
+    // 16-token tiles while experts average under 64 rows, else 120-token tiles
+    const int variant = P < 64 * E ? moe::kMxSmall : moe::kMxLarge;
+    MOE_CUDA(moe::launch_mx_quant_gather(variant, x, perm, offsets, E, P, k, d, qx, qx + tr * d,
+                                         sfbx, st));
     E_.mark(6);
     E_.mark(7);
     E_.mark(8);
@@ -251,7 +254,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     m1.h_sfb = sfbh;
     m1.n_out = I;
     m1.status = status;
-    MOE_CUDA(moe::launch_mx_gemm_gateup_swiglu(m1, num_sms, st));
+    MOE_CUDA(moe::launch_mx_gemm_gateup_swiglu(variant, m1, num_sms, st));
     E_.mark(9);
     moe::MxGemmProblem m2 = m1;
     m2.codes = dc;
@@ -267,7 +270,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     m2.perm = perm;
     m2.topk_w = topk_w;
     m2.n_out = d;
-    MOE_CUDA(moe::launch_mx_gemm_down(m2, num_sms, st));
+    MOE_CUDA(moe::launch_mx_gemm_down(variant, m2, num_sms, st));
     E_.mark(10);
     MOE_CUDA(moe::launch_combine(yw, T, k, d, out, st));
     E_.mark(11);

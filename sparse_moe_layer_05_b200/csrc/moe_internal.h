@@ -75,23 +75,27 @@ cudaError_t launch_gemm_gateup_swiglu(const GroupedGemmProblem& p, int num_sms, 
 cudaError_t launch_gemm_down_combine(const GroupedGemmProblem& p, int num_sms, cudaStream_t st);
 
 // ---------------------------------------------- block-scaled (MX) path ----
-// Tokens per tile of the block-scaled GEMMs; token rows are stored per expert
-// padded to a multiple of this.
-constexpr int kMxNT = 16;
 // Largest d or I of the block-scaled path (a tile's weight scales, 128 rows of
 // K/32 bytes, are staged in shared memory).
 constexpr int kMxMaxK = 3072;
 constexpr int TILES_MX = 4;       // block-scaled tcgen05 GEMMs (E2M1 x hi/lo E4M3)
+// Tile variants: small (16-token tiles, two CTAs per SM, two UMMA issuers
+// each; few rows per expert) and large (120-token tiles, one CTA per SM).
+constexpr int kMxSmall = 0;
+constexpr int kMxLarge = 1;
+int mx_tile_tokens(int variant);
 
-// Rows of the padded token layout and bytes of its B-scale blocks.
+// Rows of the padded token layout (each expert's rows rounded up to a
+// multiple of the tile's tokens) and bytes of its B-scale blocks, for either
+// variant.
 size_t mx_tok_rows(int P, int E);
 size_t mx_sfb_bytes(int P, int E, int K);
 
 // K2: gather x rows into the padded token layout as hi/lo E4M3 rows plus the
 // B-scale blocks the GEMM loads per (token tile, k-block).
-cudaError_t launch_mx_quant_gather(const uint16_t* x, const int32_t* perm, const int32_t* offsets,
-                                   int E, int P, int k, int K, uint8_t* qhi, uint8_t* qlo,
-                                   uint8_t* sfb, cudaStream_t st);
+cudaError_t launch_mx_quant_gather(int variant, const uint16_t* x, const int32_t* perm,
+                                   const int32_t* offsets, int E, int P, int k, int K, uint8_t* qhi,
+                                   uint8_t* qlo, uint8_t* sfb, cudaStream_t st);
 // The same split on plain rows, scales as [R][K/32][2] (hi byte, lo byte).
 cudaError_t launch_mx_split_rows(const uint16_t* x, int R, int K, uint8_t* qhi, uint8_t* qlo,
                                  uint8_t* scales, cudaStream_t st);
@@ -116,8 +120,9 @@ struct MxGemmProblem {
   int n_out;                // I for SwiGLU, d for down
   int* status;
 };
-cudaError_t launch_mx_gemm_gateup_swiglu(const MxGemmProblem& p, int num_sms, cudaStream_t st);
-cudaError_t launch_mx_gemm_down(const MxGemmProblem& p, int num_sms, cudaStream_t st);
+cudaError_t launch_mx_gemm_gateup_swiglu(int variant, const MxGemmProblem& p, int num_sms,
+                                         cudaStream_t st);
+cudaError_t launch_mx_gemm_down(int variant, const MxGemmProblem& p, int num_sms, cudaStream_t st);
 
 // Debug/self-test: one bounded wait on an mbarrier that nothing completes.
 cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t st);

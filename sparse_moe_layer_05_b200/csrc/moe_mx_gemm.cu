@@ -47,7 +47,7 @@
 //   warp 2      A-scale builder: turns the tile's E8M0 weight scales (one
 //               bulk copy per tile into shared memory, double-buffered) into
 //               the per-k-block layout tcgen05.cp reads
-//   warps 4-7   epilogue (TMEM lane quarters 0..3)
+//   warps 4..    epilogue, in groups of four (TMEM lane quarters 0..3)
 //
 // K tail. The 4-bit tensor maps need row lengths in multiples of 128, so a K
 // that is 64 mod 128 is covered by the (K/128) full k-blocks of a main map and
@@ -233,11 +233,18 @@ __global__ void __launch_bounds__(256) mx_split_rows_kernel(const uint16_t* __re
 
 enum Epi { EPI_SWIGLU = 0, EPI_DOWN = 1 };
 
-template <int NT>
+// NT tokens per tile, ISSUERS UMMA-issuing threads per CTA, CTAS CTAs per SM,
+// EPI_WARPS epilogue warps (groups of four, one per TMEM lane quarter; group
+// g takes every (EPI_WARPS/4)-th chunk of token columns).
+template <int NT_, int ISSUERS_, int CTAS_, int EPI_WARPS_>
 struct MxCfg {
+  static constexpr int NT = NT_;
+  static constexpr int ISSUERS = ISSUERS_;
+  static constexpr int CTAS = CTAS_;
+  static constexpr int EPI_WARPS = EPI_WARPS_;
+  static constexpr int EPI_GROUPS = EPI_WARPS / 4;
   static constexpr int MW = 128;                    // weight rows per tile
   static constexpr int N = 2 * NT;                  // UMMA N: hi and lo token columns
-  static constexpr int STAGES = 4;   // even: stage s is always consumed by issuer s % 2
   static constexpr int A_BYTES = 128 * 128;         // E2M1 in 8-bit containers
   static constexpr int A_TX = 128 * 64;             // packed bytes the TMA counts
   static constexpr int B_BYTES = N * 128;
@@ -246,6 +253,8 @@ struct MxCfg {
   static constexpr int OFF_SFA = OFF_B + B_BYTES;
   static constexpr int OFF_SFB = OFF_SFA + 512;
   static constexpr int STAGE_BYTES = ((OFF_SFB + SFB_BYTES) + 1023) / 1024 * 1024;
+  // even, so that with two issuers stage s is always consumed by issuer s % 2
+  static constexpr int STAGES = 4;
   static constexpr int OFF_TS = STAGES * STAGE_BYTES;   // two tile-scale buffers
   static constexpr int TS_BYTES = 128 * (kMxMaxK / 32);
   static constexpr int OFF_BAR = OFF_TS + 2 * TS_BYTES;
@@ -253,19 +262,29 @@ struct MxCfg {
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TAB = OFF_MISC + 16;
   static constexpr int OFF_XCH = OFF_TAB + 3 * (kMaxE + 1) * 4;
-  static constexpr int SMEM_BYTES = OFF_XCH + 2 * 4 * NT * 4;
+  static constexpr int CH = 8;                      // epilogue token chunk (TMEM columns)
+  static constexpr int SMEM_BYTES = OFF_XCH + EPI_GROUPS * 2 * 4 * CH * 4;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
-  static constexpr int NUM_THREADS = 256;
-  static constexpr int TMEM_COLS = 256;
+  static constexpr int NUM_THREADS = 128 + 32 * EPI_WARPS;
+  static constexpr int TMEM_COLS = CTAS == 2 ? 256 : 512;
   // accumulators: issuer u, tile buffer b at column (2u + b) N; then each
   // issuer's scale columns (A: 4, B: 4 per 512-byte atom)
-  static constexpr int SF_COL0 = 4 * N;
+  static constexpr int SF_COL0 = 2 * ISSUERS * N;
   static constexpr int SF_COLS = 4 + 4 * (SFB_BYTES / 512);
   static constexpr int TX_BYTES = A_TX + B_BYTES + SFB_BYTES;
-  static_assert(SF_COL0 + 2 * SF_COLS <= TMEM_COLS, "TMEM budget");
-  static_assert(2 * SMEM_ALLOC + 2048 <= 233472, "two CTAs per SM");
+  static_assert(NT % CH == 0 && N <= 256, "tile width");
+  static_assert(EPI_WARPS % 4 == 0 && EPI_GROUPS <= 4, "epilogue warps");
+  static_assert(SF_COL0 + ISSUERS * SF_COLS <= TMEM_COLS, "TMEM budget");
+  static_assert(CTAS * (SMEM_ALLOC + 1024) <= 233472 && SMEM_ALLOC <= 232448, "shared memory");
   static_assert(OFF_B % 1024 == 0 && (NT * 128) % 1024 == 0, "swizzle atom alignment");
 };
+
+// Decode: 16-token tiles, two issuers, two CTAs per SM. Prefill: 120-token
+// tiles (UMMA N = 240, long enough per instruction for one issuer to keep the
+// tensor pipe busy), one CTA per SM, and 12 epilogue warps so that draining a
+// tile's 15 column chunks keeps pace with its UMMAs.
+using MxSmall = MxCfg<16, 2, 2, 4>;
+using MxLarge = MxCfg<120, 1, 1, 12>;
 
 struct MxArgs {
   const int32_t* offsets;
@@ -289,12 +308,12 @@ struct MxArgs {
 
 __device__ __forceinline__ float silu_mx(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-template <int EPI, int NT>
-__global__ void __launch_bounds__(256, 2)
+template <int EPI, class C>
+__global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
     grouped_mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmAt,
                            const __grid_constant__ CUtensorMap tmB, const MxArgs args) {
-  using C = MxCfg<NT>;
+  constexpr int NT = C::NT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -335,8 +354,8 @@ __global__ void __launch_bounds__(256, 2)
       mbar_init(bar_empty(s), 1);
     }
     for (int b = 0; b < 2; ++b) {
-      mbar_init(bar_accFull(b), 2);     // one commit per issuer
-      mbar_init(bar_accEmpty(b), 4 * 32);
+      mbar_init(bar_accFull(b), C::ISSUERS);     // one commit per issuer
+      mbar_init(bar_accEmpty(b), C::EPI_WARPS * 32);
       mbar_init(bar_tsFull(b), 1);
       mbar_init(bar_tsEmpty(b), 1);
     }
@@ -481,7 +500,7 @@ __global__ void __launch_bounds__(256, 2)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_tsEmpty(b));
     }
-  } else if (warp == 1 || warp == 3) {
+  } else if (warp == 1 || (C::ISSUERS == 2 && warp == 3)) {
     // ------------------------------------------------------- UMMA issuers --
     // Issuer u takes the k-blocks with q % 2 == u (q counts this CTA's
     // k-blocks across tiles), i.e. the stages s with s % 2 == u; the other
@@ -500,7 +519,7 @@ __global__ void __launch_bounds__(256, 2)
         const uint32_t d = tmem_base + (2 * u + ab) * C::N;
         uint32_t accum = 0;   // the issuer's first k-block of the tile overwrites its buffer
         for (int kb = 0; kb < KB; ++kb, ++q) {
-          if ((q & 1) == u) {
+          if ((q % C::ISSUERS) == u) {
             if (!(ok = mbar_wait(bar_full(s), ph, abort_flag, args.status))) break;
             tc_fence_after();
             const uint32_t st = sbase + s * C::STAGE_BYTES;
@@ -537,119 +556,121 @@ __global__ void __launch_bounds__(256, 2)
     }
   } else if (warp >= 4) {
     // ----------------------------------------------------------- epilogue --
-    // Every epilogue warp passes the SwiGLU exchange barrier once per tile,
-    // also after a failed wait, so that no warp is left at it alone.
+    // Chunks of CH token columns: hi and lo of every issuer's buffer are
+    // loaded and added, then SwiGLU + the hi/lo split of H (gate/up) or the
+    // weighted store (down). Every epilogue warp passes the SwiGLU exchange
+    // barrier once per chunk, also after a failed wait, so that no warp is
+    // left at it alone.
+    constexpr int CH = C::CH;
     const int quad = warp & 3;                 // TMEM lanes 32*quad .. +31
+    const int grp = (warp - 4) >> 2;           // epilogue group: chunks grp, grp + G, ...
     const int m = quad * 32 + lane;            // weight row of the tile
+    const uint32_t lanes = static_cast<uint32_t>(quad * 32) << 16;
     bool ok = true;
-    int it = 0;
+    int it = 0, xc = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       int e, wb, tb, rows;
       decode(tile, e, wb, tb, rows);
       const int ab = it & 1;
       const uint32_t ap = (it >> 1) & 1;
       if (ok) ok = mbar_wait(bar_accFull(ab), ap, abort_flag, args.status);
+      ok = __all_sync(0xFFFFFFFFu, ok);        // the TMEM loads below are warp-collective
       if (!ok && EPI != EPI_SWIGLU) break;
-      float y[NT];
-      if (ok) {
-        tc_fence_after();
-        // y = (issuer 0: hi + lo) + (issuer 1: hi + lo); with a single
-        // k-block per tile only issuer (it*KB) % 2 wrote its buffer
-        const uint32_t lanes = static_cast<uint32_t>(quad * 32) << 16;
-        const bool use0 = KB > 1 || ((it * KB) & 1) == 0;
-        const bool use1 = KB > 1 || ((it * KB) & 1) == 1;
-        const uint32_t t0 = tmem_base + lanes + ab * C::N;
-        const uint32_t t1 = tmem_base + lanes + (2 + ab) * C::N;
+      if (ok) tc_fence_after();
+      // with two issuers and a single k-block per tile only issuer
+      // (it*KB) % 2 wrote its buffer
+      const bool use0 = C::ISSUERS == 1 || KB > 1 || ((it * KB) & 1) == 0;
+      const bool use1 = C::ISSUERS == 2 && (KB > 1 || ((it * KB) & 1) == 1);
+      const uint32_t t0 = tmem_base + lanes + ab * C::N;
+      const uint32_t t1 = tmem_base + lanes + (2 + ab) * C::N;
+      const int tok_tile = s_tb[e] + tb;
+      const int j = wb * 64 + 16 * quad + (lane & 15);      // SwiGLU: H column of this lane
+      const bool jv = j < args.I && lane < 16;
+      const int col = wb * 128 + m;                          // down: output column
+#pragma unroll 1
+      for (int c = grp * CH; c < NT; c += C::EPI_GROUPS * CH, ++xc) {
+        float y[CH];
 #pragma unroll
-        for (int c = 0; c < NT; c += 16) {
-          uint32_t a[16], b[16];
-#pragma unroll
-          for (int i = 0; i < 16; ++i) y[c + i] = 0.f;
+        for (int i = 0; i < CH; ++i) y[i] = 0.f;
+        if (ok && c < rows) {
+          uint32_t a[8], b[8];
           if (use0) {
-            tmem_ld16_sync(t0 + c, a);
-            tmem_ld16_sync(t0 + NT + c, b);
+            tmem_ld8x2_sync(t0 + c, t0 + NT + c, a, b);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) y[c + i] = __uint_as_float(a[i]) + __uint_as_float(b[i]);
+            for (int i = 0; i < CH; ++i) y[i] = __uint_as_float(a[i]) + __uint_as_float(b[i]);
           }
           if (use1) {
-            tmem_ld16_sync(t1 + c, a);
-            tmem_ld16_sync(t1 + NT + c, b);
+            tmem_ld8x2_sync(t1 + c, t1 + NT + c, a, b);
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              y[c + i] += __uint_as_float(a[i]) + __uint_as_float(b[i]);
+            for (int i = 0; i < CH; ++i) y[i] += __uint_as_float(a[i]) + __uint_as_float(b[i]);
           }
         }
-        tc_fence_before();
-        mbar_arrive(bar_accEmpty(ab));     // accumulators are in registers now
-      } else {
+        if (EPI == EPI_SWIGLU) {
+          // lanes 0-15: gate row j, lanes 16-31: up row j; y becomes h for the
+          // gate lanes and 0 elsewhere
+          float* xch = s_xch + (grp * 2 + (xc & 1)) * 4 * CH;
 #pragma unroll
-        for (int t = 0; t < NT; ++t) y[t] = 0.f;
-      }
-
-      const int tok_tile = s_tb[e] + tb;
-      if (EPI == EPI_SWIGLU) {
-        // lanes 0-15: gate row j, lanes 16-31: up row j (j = wb*64 + 16*quad + lane%16);
-        // y[t] becomes h for the gate lanes and 0 elsewhere
-        const int j = wb * 64 + 16 * quad + (lane & 15);
-        const bool jv = ok && j < args.I && lane < 16;
-        float* xch = s_xch + (it & 1) * 4 * NT;
+          for (int i = 0; i < CH; ++i) {
+            const float u = __shfl_xor_sync(0xFFFFFFFFu, y[i], 16);
+            float hv = 0.f;
+            if (ok && jv && c + i < rows)
+              hv = __bfloat162float(__float2bfloat16_rn(silu_mx(y[i]) * u));
+            y[i] = hv;
+            float pm = fabsf(hv);
 #pragma unroll
-        for (int t = 0; t < NT; ++t) {
-          const float u = __shfl_xor_sync(0xFFFFFFFFu, y[t], 16);
-          float hv = 0.f;
-          if (jv && t < rows) hv = __bfloat162float(__float2bfloat16_rn(silu_mx(y[t]) * u));
-          y[t] = hv;
-          float pm = fabsf(hv);
+            for (int o = 1; o < 16; o <<= 1) pm = fmaxf(pm, __shfl_xor_sync(0xFFFFFFFFu, pm, o));
+            if (lane == 0) xch[quad * CH + i] = pm;
+          }
+          // max |h| over the 32 j of a group: quarters 0+1 and 2+3 (named
+          // barrier 1 + grp over the group's four warps)
+          asm volatile("bar.sync %0, 128;" ::"r"(1 + grp) : "memory");
+          if (ok) {
+            const int gj = 2 * wb + (quad >> 1);
+            int kb4, kk4;
+            group_to_kblock(gj, args.I / 32, args.h_kb, kb4, kk4);
+            uint8_t* hsfb = args.h_sfb + (static_cast<size_t>(tok_tile) * args.h_kb + kb4) *
+                                             sfb_block_bytes(NT);
 #pragma unroll
-          for (int o = 1; o < 16; o <<= 1) pm = fmaxf(pm, __shfl_xor_sync(0xFFFFFFFFu, pm, o));
-          if (lane == 0) xch[quad * NT + t] = pm;
-        }
-        // max |h| over the 32 j of a group: quarters 0+1 and 2+3
-        asm volatile("bar.sync 1, 128;" ::: "memory");
-        if (ok) {
-          const int gj = 2 * wb + (quad >> 1);
-          int kb4, kk4;
-          group_to_kblock(gj, args.I / 32, args.h_kb, kb4, kk4);
-          uint8_t* hsfb = args.h_sfb + (static_cast<size_t>(tok_tile) * args.h_kb + kb4) *
-                                           sfb_block_bytes(NT);
-#pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            if (t < rows) {
-              const float amax = fmaxf(xch[quad * NT + t], xch[(quad ^ 1) * NT + t]);
-              int eh = 0;
-              if (amax != 0.f) {
-                const int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127;
-                eh = max(ex - 7, -123);
-              }
-              const float inv = __uint_as_float(static_cast<uint32_t>(127 - eh) << 23);
-              const float a = y[t] * inv;
-              const uint32_t h2 = f32x2_to_e4m3x2(a, 0.f);
-              const float2 hb = e4m3x2_to_f32x2(h2);
-              const uint32_t l2 = f32x2_to_e4m3x2((a - hb.x) * 16.f, 0.f);
-              if (jv) {
-                const size_t o = static_cast<size_t>(tok_tile * NT + t) * args.I + j;
-                args.h_hi[o] = static_cast<uint8_t>(h2 & 0xFF);
-                args.h_lo[o] = static_cast<uint8_t>(l2 & 0xFF);
-              }
-              if (lane == 0 && !(quad & 1)) {
-                hsfb[sfb_offset(NT, t, 0, kk4)] = static_cast<uint8_t>(eh + 127);
-                hsfb[sfb_offset(NT, t, 1, kk4)] = static_cast<uint8_t>(eh + 123);
+            for (int i = 0; i < CH; ++i) {
+              const int t = c + i;
+              if (t < rows) {
+                const float amax = fmaxf(xch[quad * CH + i], xch[(quad ^ 1) * CH + i]);
+                int eh = 0;
+                if (amax != 0.f) {
+                  const int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+                  eh = max(ex - 7, -123);
+                }
+                const float inv = __uint_as_float(static_cast<uint32_t>(127 - eh) << 23);
+                const float a = y[i] * inv;
+                const uint32_t h2 = f32x2_to_e4m3x2(a, 0.f);
+                const float2 hb = e4m3x2_to_f32x2(h2);
+                const uint32_t l2 = f32x2_to_e4m3x2((a - hb.x) * 16.f, 0.f);
+                if (jv) {
+                  const size_t o = static_cast<size_t>(tok_tile * NT + t) * args.I + j;
+                  args.h_hi[o] = static_cast<uint8_t>(h2 & 0xFF);
+                  args.h_lo[o] = static_cast<uint8_t>(l2 & 0xFF);
+                }
+                if (lane == 0 && !(quad & 1)) {
+                  hsfb[sfb_offset(NT, t, 0, kk4)] = static_cast<uint8_t>(eh + 127);
+                  hsfb[sfb_offset(NT, t, 1, kk4)] = static_cast<uint8_t>(eh + 123);
+                }
               }
             }
           }
-        }
-      } else {
-        const int col = wb * 128 + m;
-        if (col < args.n_out) {
+        } else if (ok && col < args.n_out) {
           const int p0 = s_off[e] + tb * NT;
 #pragma unroll
-          for (int t = 0; t < NT; ++t) {
-            if (t < rows) {
-              const int pr = args.perm[p0 + t];
-              args.out_f32[static_cast<int64_t>(pr) * args.n_out + col] = args.topk_w[pr] * y[t];
+          for (int i = 0; i < CH; ++i) {
+            if (c + i < rows) {
+              const int pr = args.perm[p0 + c + i];
+              args.out_f32[static_cast<int64_t>(pr) * args.n_out + col] = args.topk_w[pr] * y[i];
             }
           }
         }
+      }
+      if (ok) {
+        tc_fence_before();
+        mbar_arrive(bar_accEmpty(ab));     // this tile's accumulators are read
       }
     }
   }
@@ -735,16 +756,16 @@ bool make_tok8_map(CUtensorMap* m, const uint8_t* hi, int rows, int K, int nt) {
   return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, hi, dims, strides, box);
 }
 
-template <int EPI, int NT>
+template <int EPI, class C>
 cudaError_t launch_mx_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st) {
-  using C = MxCfg<NT>;
+  constexpr int NT = C::NT;
   // the kernel assumes K % 64 == 0 (tail k-blocks of 2 steps) and K <= kMxMaxK
   if (p.K % 64 != 0 || p.K < 128 || p.K > kMxMaxK) return cudaErrorInvalidValue;
   static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(grouped_mx_gemm_kernel<EPI, NT>,
+    cudaError_t e = cudaFuncSetAttribute(grouped_mx_gemm_kernel<EPI, C>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          C::SMEM_ALLOC);
     if (e != cudaSuccess) return e;
@@ -796,13 +817,14 @@ cudaError_t launch_mx_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st)
     a.rows_per_expert = p.n_out;
   }
   const int64_t tiles_bound = (static_cast<int64_t>(p.P) / NT + p.E) * a.n_wb;
-  int64_t grid = 2 * static_cast<int64_t>(num_sms);
+  int64_t grid = C::CTAS * static_cast<int64_t>(num_sms);
   if (tiles_bound < grid) grid = tiles_bound;
   if (grid < 1) grid = 1;
-  grouped_mx_gemm_kernel<EPI, NT><<<static_cast<int>(grid), C::NUM_THREADS, C::SMEM_ALLOC, st>>>(
+  grouped_mx_gemm_kernel<EPI, C><<<static_cast<int>(grid), C::NUM_THREADS, C::SMEM_ALLOC, st>>>(
       tmA, tmAt, tmB, a);
   return cudaGetLastError();
 }
+
 
 int grid_for_n(int64_t n, int per_thread_block, int cap) {
   int64_t b = (n + per_thread_block - 1) / per_thread_block;
@@ -813,18 +835,34 @@ int grid_for_n(int64_t n, int per_thread_block, int cap) {
 
 }  // namespace
 
-size_t mx_tok_rows(int P, int E) { return static_cast<size_t>(P) + static_cast<size_t>(E) * (kMxNT - 1); }
-size_t mx_sfb_bytes(int P, int E, int K) {
-  const size_t tiles = (static_cast<size_t>(P) + kMxNT - 1) / kMxNT + E;
-  return tiles * ((K + 127) / 128) * sfb_block_bytes(kMxNT);
+int mx_tile_tokens(int variant) { return variant == kMxLarge ? MxLarge::NT : MxSmall::NT; }
+
+size_t mx_tok_rows(int P, int E) {
+  const int nt = MxSmall::NT > MxLarge::NT ? MxSmall::NT : MxLarge::NT;
+  return static_cast<size_t>(P) + static_cast<size_t>(E) * (nt - 1);
 }
 
-cudaError_t launch_mx_quant_gather(const uint16_t* x, const int32_t* perm, const int32_t* offsets,
-                                   int E, int P, int k, int K, uint8_t* qhi, uint8_t* qlo,
-                                   uint8_t* sfb, cudaStream_t st) {
+size_t mx_sfb_bytes(int P, int E, int K) {
+  size_t best = 0;
+  for (int nt : {MxSmall::NT, MxLarge::NT}) {
+    const size_t tiles = (static_cast<size_t>(P) + nt - 1) / nt + E;
+    const size_t b = tiles * ((K + 127) / 128) * sfb_block_bytes(nt);
+    if (b > best) best = b;
+  }
+  return best;
+}
+
+cudaError_t launch_mx_quant_gather(int variant, const uint16_t* x, const int32_t* perm,
+                                   const int32_t* offsets, int E, int P, int k, int K, uint8_t* qhi,
+                                   uint8_t* qlo, uint8_t* sfb, cudaStream_t st) {
   const int64_t n = static_cast<int64_t>(P) * (K / 32);
-  mx_quant_gather_kernel<kMxNT><<<grid_for_n(n, 256, 148 * 8), 256, 0, st>>>(
-      x, perm, offsets, E, P, k, K, qhi, qlo, sfb);
+  const int grid = grid_for_n(n, 256, 148 * 8);
+  if (variant == kMxLarge)
+    mx_quant_gather_kernel<MxLarge::NT><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, qhi,
+                                                               qlo, sfb);
+  else
+    mx_quant_gather_kernel<MxSmall::NT><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, qhi,
+                                                               qlo, sfb);
   return cudaGetLastError();
 }
 
@@ -835,12 +873,16 @@ cudaError_t launch_mx_split_rows(const uint16_t* x, int R, int K, uint8_t* qhi, 
   return cudaGetLastError();
 }
 
-cudaError_t launch_mx_gemm_gateup_swiglu(const MxGemmProblem& p, int num_sms, cudaStream_t st) {
-  return launch_mx_impl<EPI_SWIGLU, kMxNT>(p, num_sms, st);
+cudaError_t launch_mx_gemm_gateup_swiglu(int variant, const MxGemmProblem& p, int num_sms,
+                                         cudaStream_t st) {
+  return variant == kMxLarge ? launch_mx_impl<EPI_SWIGLU, MxLarge>(p, num_sms, st)
+                             : launch_mx_impl<EPI_SWIGLU, MxSmall>(p, num_sms, st);
 }
 
-cudaError_t launch_mx_gemm_down(const MxGemmProblem& p, int num_sms, cudaStream_t st) {
-  return launch_mx_impl<EPI_DOWN, kMxNT>(p, num_sms, st);
+cudaError_t launch_mx_gemm_down(int variant, const MxGemmProblem& p, int num_sms,
+                                cudaStream_t st) {
+  return variant == kMxLarge ? launch_mx_impl<EPI_DOWN, MxLarge>(p, num_sms, st)
+                             : launch_mx_impl<EPI_DOWN, MxSmall>(p, num_sms, st);
 }
 
 }  // namespace moe
