@@ -85,9 +85,10 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def kernel_source_hash() -> str:
+def kernel_source_hash(sources=None) -> str:
+    """Hash of the kernel sources a recorded ncu figure depends on."""
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
+    for f in sources or KERNEL_SOURCES:
         with open(os.path.join(ROOT, "sparse_moe_layer_05_b200", "csrc", f), "rb") as fh:
             h.update(fh.read())
     return h.hexdigest()[:16]
@@ -101,7 +102,7 @@ def recorded_traffic(workload: str, T: int):
     with open(TRAFFIC_FILE) as f:
         d = json.load(f)
     ent = d.get(f"{workload}:T={T}")
-    if not ent or ent.get("source_hash") != kernel_source_hash():
+    if not ent or ent.get("source_hash") != kernel_source_hash(ent.get("sources")):
         return None
     return ent.get("bytes_per_launch")
 
