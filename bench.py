@@ -370,6 +370,29 @@ def run_ours(args, inp, name):
     return line
 
 
+def probe_tensor():
+    """Measured UMMA rates on this device: MACs per SM clock for bf16 (kind::f16,
+    K = 16) and the block-scaled E2M1 x E4M3 kind (K = 32), M = 128, several N and
+    UMMAs per commit; TFLOP/s at the SM count and the maximum SM clock."""
+    import torch
+    from sparse_moe_layer_05_b200 import binding as B
+    torch.cuda.init()
+    props = torch.cuda.get_device_properties(0)
+    peaks, _ = load_peaks()
+    mhz = float(peaks.get("sm_max_mhz", 1965.0))
+    rows = []
+    for kind, kname in ((0, "bf16"), (1, "e2m1_x_e4m3_block_scaled")):
+        for n in (32, 64, 128, 240, 256):
+            for per_commit in (4, 16):
+                r = B.moe_probe_tensor_rate(kind, n, per_commit)
+                rows.append({"kind": kname, "N": n, "umma_per_commit": per_commit,
+                             "mac_per_clk_sm": round(r, 1),
+                             "tflops_at_max_clock": round(2 * r * props.multi_processor_count
+                                                          * mhz * 1e6 / 1e12, 1)})
+    print(json.dumps({"probe": "tensor_rate", "sms": props.multi_processor_count,
+                      "sm_max_mhz": mhz, "M": 128, "rows": rows}))
+
+
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -379,11 +402,16 @@ def main(argv=None):
     ap.add_argument("--workload", default="20b", choices=list(W.SHAPES))
     ap.add_argument("--T", type=int, default=None, help="tokens per GPU (default: prefill T)")
     ap.add_argument("--ref-tokens", type=int, default=2, help="oracle tokens per reference step")
+    ap.add_argument("--probe-tensor", action="store_true",
+                    help="print the measured UMMA rates (MAC per SM clock) and exit")
     ap.add_argument("--tile-policy", type=int, default=0, choices=[0, 1, 2, 3, 4],
                     help="grouped-GEMM tiles: 0 by shape, 1 single, 2 pair, 3 swap, 4 block-scaled")
     ap.add_argument("--cpu-sample", type=int, default=256,
                     help="tokens of the batch the oracle runs for cpu_baseline (0 = skip)")
     args = ap.parse_args(argv)
+    if args.probe_tensor:
+        probe_tensor()
+        return
     if args.warmup < 3:
         ap.error("--warmup must be at least 3")
     rank, world, local = dist_env()

@@ -270,6 +270,20 @@ MOE_API moe_status moe_sync_status(void* workspace_dev, size_t workspace_bytes, 
 MOE_API moe_status moe_selftest_wait_timeout(void* workspace_dev, void* stream);
 
 /*
+ * Tensor-core rate probe (diagnostic; the pages have no counterpart): on every
+ * SM one thread issues back-to-back UMMAs of M = 128 and N columns from
+ * shared-memory tiles, per_commit per tcgen05.commit, and *mac_per_clk_sm
+ * receives the multiply-accumulates per SM clock of the slowest SM. kind 0 is
+ * bf16 (kind::f16, K = 16 per UMMA), kind 1 the block-scaled E2M1 x E4M3 kind
+ * the block-scaled tiles use (kind::mxf8f6f4, K = 32). N in [16, 256], a
+ * multiple of 16; per_commit in [4, 64], a multiple of 4. Multiply by 2 x the
+ * SM count x the SM clock for FLOP/s. Allocates and frees a small device
+ * buffer and synchronises `stream`. MOE_ERR_TIMEOUT if a bounded wait gave up.
+ */
+MOE_API moe_status moe_probe_tensor_rate(int kind, int N, int per_commit, double* mac_per_clk_sm,
+                                         void* stream);
+
+/*
  * Number of kernel launches one moe_forward call enqueues for this shape
  * under the current tile policy (0 for T = 0), assuming 32-byte aligned code
  * arrays. Used to count device work per step.

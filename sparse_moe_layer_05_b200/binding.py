@@ -29,7 +29,7 @@ EXPORTS = [
     "moe_workspace_size_hostio", "moe_forward_hostio", "moe_route_workspace_size",
     "moe_route", "moe_workspace_layout", "moe_mxfp4_to_bf16", "moe_mx_split_e4m3", "moe_sync_status",
     "moe_selftest_wait_timeout", "moe_forward_launch_count", "moe_forward_timed",
-    "moe_set_tile_policy", "moe_route_noalloc",
+    "moe_set_tile_policy", "moe_route_noalloc", "moe_probe_tensor_rate",
 ]
 
 STAGES = ["router_logits", "topk_softmax", "perm_hist", "perm_scan", "perm_scatter",
@@ -87,6 +87,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_workspace_layout.argtypes = [i32] * 5 + [ctypes.POINTER(WsLayout)]
     lib.moe_mxfp4_to_bf16.restype = i32
     lib.moe_mxfp4_to_bf16.argtypes = [u8p, u8p, i32, i32, vp, vp]
+    lib.moe_probe_tensor_rate.restype = i32
+    lib.moe_probe_tensor_rate.argtypes = [i32, i32, i32, ctypes.POINTER(ctypes.c_double), vp]
     lib.moe_mx_split_e4m3.restype = i32
     lib.moe_mx_split_e4m3.argtypes = [vp, i32, i32, u8p, u8p, u8p, vp]
     lib.moe_sync_status.restype = i32
@@ -205,6 +207,14 @@ def moe_route_noalloc(x, W_r, b_r, E, k, T, d, topk_idx, topk_w, counts, offsets
     _check("moe_route_noalloc", load().moe_route_noalloc(
         _ptr(x), _ptr(W_r), _ptr(b_r), E, k, T, d, _ptr(topk_idx), _ptr(topk_w), _ptr(counts),
         _ptr(offsets), _ptr(perm), _stream(stream)))
+
+
+def moe_probe_tensor_rate(kind: int, N: int, per_commit: int, stream=None) -> float:
+    """MACs per SM clock of back-to-back UMMAs (kind 0 bf16, 1 block-scaled E2M1 x E4M3)."""
+    out = ctypes.c_double(0.0)
+    _check("moe_probe_tensor_rate", load().moe_probe_tensor_rate(kind, N, per_commit,
+                                                                 ctypes.byref(out), _stream(stream)))
+    return out.value
 
 
 def moe_mx_split_e4m3(x, rows: int, K: int, hi, lo, scales, stream=None) -> None:

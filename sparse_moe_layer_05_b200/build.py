@@ -15,7 +15,8 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmoe_b200.so")
-SOURCES = ["moe_abi.cu", "moe_routing.cu", "moe_grouped_gemm.cu", "moe_mx_gemm.cu", "moe_noalloc.cu"]
+SOURCES = ["moe_abi.cu", "moe_routing.cu", "moe_grouped_gemm.cu", "moe_mx_gemm.cu", "moe_noalloc.cu",
+           "moe_probe.cu"]
 HEADERS = ["moe_ptx.cuh", "moe_internal.h"]
 
 NVCC_FLAGS = [

@@ -185,6 +185,38 @@ struct StageEvents {
   }
 };
 
+// Launches of the router (logits, top-k, softmax) and, when perm is given, the
+// permutation (counts, offsets, M-tile prefix, perm). Batches of at most
+// kPermChunk tokens take one fused launch for the permutation (identical
+// results). ev marks launches 0..5 of moe_forward_timed.
+moe_status launch_routing(const uint16_t* x, const float* W_r, const float* b_r, int E, int k,
+                          int T, int d, float* logits, int32_t* topk_idx, float* topk_w,
+                          int32_t* counts, int32_t* offsets, int32_t* mprefix,
+                          int32_t* chunk_hist, int32_t* chunk_base, int32_t* perm, int* status,
+                          cudaStream_t st, const StageEvents& ev) {
+  const bool small = T <= moe::kPermChunk;
+  ev.mark(0);
+  MOE_CUDA(moe::launch_router_logits(x, W_r, b_r, logits, T, E, d, status, st));
+  ev.mark(1);
+  MOE_CUDA(moe::launch_topk_softmax(logits, T, E, k, topk_idx, topk_w, st));
+  ev.mark(2);
+  if (!perm) return MOE_OK;
+  if (small) {
+    MOE_CUDA(moe::launch_perm_small(topk_idx, T, k, E, counts, offsets, mprefix, perm, st));
+    ev.mark(3);
+    ev.mark(4);
+  } else {
+    MOE_CUDA(moe::launch_perm_hist(topk_idx, T, k, E, chunk_hist, st));
+    ev.mark(3);
+    MOE_CUDA(moe::launch_perm_scan(chunk_hist, moe::perm_chunks(T), E, counts, offsets, chunk_base,
+                                   mprefix, st));
+    ev.mark(4);
+    MOE_CUDA(moe::launch_perm_scatter(topk_idx, T, k, E, chunk_base, perm, nullptr, st));
+  }
+  ev.mark(5);
+  return MOE_OK;
+}
+
 moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, const uint8_t* gc,
                        const uint8_t* gs, const uint8_t* dc, const uint8_t* ds, int E, int k,
                        int T, int d, int I, uint16_t* out, void* ws, const Layout& L,
@@ -193,7 +225,6 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   memset(&none, 0, sizeof(none));
   const StageEvents& E_ = tev ? *tev : none;
   const int P = T * k;
-  const int NB = moe::perm_chunks(T);
   int* status = at<int>(ws, L.pub.status);
   float* logits = at<float>(ws, L.pub.logits);
   int32_t* topk_idx = at<int32_t>(ws, L.pub.topk_idx);
@@ -210,17 +241,9 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   uint8_t* gst = at<uint8_t>(ws, L.gu_scales_t);
   uint8_t* dst_ = at<uint8_t>(ws, L.d_scales_t);
 
-  E_.mark(0);
-  MOE_CUDA(moe::launch_router_logits(x, W_r, b_r, logits, T, E, d, status, st));
-  E_.mark(1);
-  MOE_CUDA(moe::launch_topk_softmax(logits, T, E, k, topk_idx, topk_w, st));
-  E_.mark(2);
-  MOE_CUDA(moe::launch_perm_hist(topk_idx, T, k, E, chunk_hist, st));
-  E_.mark(3);
-  MOE_CUDA(moe::launch_perm_scan(chunk_hist, NB, E, counts, offsets, chunk_base, mprefix, st));
-  E_.mark(4);
-  MOE_CUDA(moe::launch_perm_scatter(topk_idx, T, k, E, chunk_base, perm, nullptr, st));
-  E_.mark(5);
+  moe_status rs = launch_routing(x, W_r, b_r, E, k, T, d, logits, topk_idx, topk_w, counts,
+                                 offsets, mprefix, chunk_hist, chunk_base, perm, status, st, E_);
+  if (rs != MOE_OK) return rs;
   const int tiles = choose_tiles(P, E, mx_shape_ok(d, I) && aligned32(gc) && aligned32(dc));
   if (tiles == moe::TILES_MX) {
     // block-scaled path: hi/lo token rows, no scale transposes
@@ -370,8 +393,12 @@ moe_status moe_workspace_layout(int E, int k, int T, int d, int I, moe_ws_layout
 
 int moe_forward_launch_count(int E, int k, int T, int d, int I) {
   if (!full_shape_ok(E, k, T, d, I) || T == 0) return 0;
+  int n = 11;
+  // small batches: the permutation in one launch instead of three
+  if (T <= moe::kPermChunk) n -= 2;
   // the block-scaled path launches no scale transposes
-  return choose_tiles(T * k, E, mx_shape_ok(d, I)) == moe::TILES_MX ? 9 : 11;
+  if (choose_tiles(T * k, E, mx_shape_ok(d, I)) == moe::TILES_MX) n -= 2;
+  return n;
 }
 
 moe_status moe_forward(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
@@ -495,22 +522,14 @@ moe_status moe_route(const void* x_dev, const float* W_r_dev, const float* b_r_d
   moe_status s = device_info(&num_sms);
   if (s != MOE_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int NB = moe::perm_chunks(T);
-  float* logits = at<float>(workspace_dev, L.pub.logits);
-  int* status = at<int>(workspace_dev, L.pub.status);
-  MOE_CUDA(moe::launch_router_logits(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, logits,
-                                     T, E, d, status, st));
-  MOE_CUDA(moe::launch_topk_softmax(logits, T, E, k, topk_idx_dev, topk_w_dev, st));
-  if (nperm == 3) {
-    int32_t* chunk_hist = at<int32_t>(workspace_dev, L.chunk_hist);
-    int32_t* chunk_base = at<int32_t>(workspace_dev, L.chunk_base);
-    int32_t* mprefix = at<int32_t>(workspace_dev, L.mprefix);
-    MOE_CUDA(moe::launch_perm_hist(topk_idx_dev, T, k, E, chunk_hist, st));
-    MOE_CUDA(moe::launch_perm_scan(chunk_hist, NB, E, counts_dev, offsets_dev, chunk_base,
-                                   mprefix, st));
-    MOE_CUDA(moe::launch_perm_scatter(topk_idx_dev, T, k, E, chunk_base, perm_dev, nullptr, st));
-  }
-  return MOE_OK;
+  StageEvents none;
+  memset(&none, 0, sizeof(none));
+  return launch_routing(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, E, k, T, d,
+                        at<float>(workspace_dev, L.pub.logits), topk_idx_dev, topk_w_dev,
+                        counts_dev, offsets_dev, at<int32_t>(workspace_dev, L.mprefix),
+                        at<int32_t>(workspace_dev, L.chunk_hist),
+                        at<int32_t>(workspace_dev, L.chunk_base), nperm == 3 ? perm_dev : nullptr,
+                        at<int>(workspace_dev, L.pub.status), st, none);
 }
 
 moe_status moe_mxfp4_to_bf16(const uint8_t* codes_dev, const uint8_t* scales_dev, int rows, int K,
@@ -540,6 +559,49 @@ moe_status moe_mx_split_e4m3(const void* x_dev, int rows, int K, uint8_t* hi_dev
   MOE_CUDA(moe::launch_mx_split_rows(static_cast<const uint16_t*>(x_dev), rows, K, hi_dev, lo_dev,
                                      scales_dev, static_cast<cudaStream_t>(stream)));
   return MOE_OK;
+}
+
+moe_status moe_probe_tensor_rate(int kind, int N, int per_commit, double* mac_per_clk_sm,
+                                 void* stream) {
+  if (!mac_per_clk_sm || (kind != 0 && kind != 1) || N < 16 || N > 256 || N % 16 ||
+      per_commit < 4 || per_commit > 64 || per_commit % 4)
+    return MOE_ERR_INVALID_ARG;
+  int num_sms = 0;
+  moe_status s = device_info(&num_sms);
+  if (s != MOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned long long* d_cycles = nullptr;
+  const size_t bytes = static_cast<size_t>(num_sms) * 8 + 16;
+  MOE_CUDA(cudaMalloc(&d_cycles, bytes));
+  int* d_status = reinterpret_cast<int*>(d_cycles + num_sms);
+  moe_status r = MOE_OK;
+  if (cudaMemsetAsync(d_cycles, 0, bytes, st) != cudaSuccess ||
+      moe::launch_tensor_rate_probe(kind, N, per_commit, num_sms, d_cycles, d_status, st) !=
+          cudaSuccess ||
+      cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    r = MOE_ERR_CUDA;
+  }
+  unsigned long long* h = new unsigned long long[num_sms + 2];
+  if (r == MOE_OK && cudaMemcpy(h, d_cycles, bytes, cudaMemcpyDeviceToHost) != cudaSuccess) {
+    cudaGetLastError();
+    r = MOE_ERR_CUDA;
+  }
+  if (r == MOE_OK) {
+    const int status = *reinterpret_cast<int*>(h + num_sms);
+    unsigned long long worst = 0;
+    for (int i = 0; i < num_sms; ++i) worst = h[i] > worst ? h[i] : worst;
+    if (status || worst == 0) {
+      r = status ? static_cast<moe_status>(status) : MOE_ERR_CUDA;
+    } else {
+      const double k = kind == 1 ? 32.0 : 16.0;
+      const double macs = static_cast<double>(moe::tensor_rate_probe_iters()) * per_commit * 128.0 * N * k;
+      *mac_per_clk_sm = macs / static_cast<double>(worst);
+    }
+  }
+  delete[] h;
+  cudaFree(d_cycles);
+  return r;
 }
 
 moe_status moe_sync_status(void* workspace_dev, size_t workspace_bytes, void* stream) {

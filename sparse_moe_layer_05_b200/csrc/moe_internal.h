@@ -22,6 +22,11 @@ constexpr int kRouterSmallT = 256;
 cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, const float* b_r,
                                  float* logits, int T, int E, int d, int* status_to_clear,
                                  cudaStream_t st);
+// K2 for T <= kPermChunk in one launch: counts, offsets, M-tile prefix and
+// perm, identical to launch_perm_hist + launch_perm_scan + launch_perm_scatter.
+cudaError_t launch_perm_small(const int32_t* topk_idx, int T, int k, int E, int32_t* counts,
+                              int32_t* offsets, int32_t* mtile_prefix, int32_t* perm,
+                              cudaStream_t st);
 // K1: top-k (lower index wins ties) and the selected-set softmax.
 cudaError_t launch_topk_softmax(const float* logits, int T, int E, int k, int32_t* topk_idx,
                                 float* topk_w, cudaStream_t st);
@@ -123,6 +128,13 @@ struct MxGemmProblem {
 cudaError_t launch_mx_gemm_gateup_swiglu(int variant, const MxGemmProblem& p, int num_sms,
                                          cudaStream_t st);
 cudaError_t launch_mx_gemm_down(int variant, const MxGemmProblem& p, int num_sms, cudaStream_t st);
+
+// Tensor-core rate probe (moe_probe.cu): one CTA per SM issues UMMAs of the
+// given kind (0: bf16 kind::f16, K = 16; 1: block-scaled E2M1 x E4M3, K = 32)
+// with M = 128 and N columns, per_commit per commit; cycles[sm] = clock64 span.
+cudaError_t launch_tensor_rate_probe(int kind, int N, int per_commit, int num_sms,
+                                     unsigned long long* cycles, int* status, cudaStream_t st);
+int tensor_rate_probe_iters();
 
 // Debug/self-test: one bounded wait on an mbarrier that nothing completes.
 cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t st);

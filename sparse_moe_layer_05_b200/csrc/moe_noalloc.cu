@@ -107,7 +107,19 @@ moe_status moe_route_noalloc(const void* x_dev, const float* W_r_dev, const floa
   int32_t* chunk_hist = reinterpret_cast<int32_t*>(sb + L.chunk_hist);
   int32_t* chunk_base = reinterpret_cast<int32_t*>(sb + L.chunk_base);
   // Every buffer below is fully written before it is read; the status word
-  // is cleared by the first kernel.
+  // is cleared by the first kernel. Batches of at most kPermChunk tokens take
+  // the fused permutation launch (identical results).
+  if (T <= moe::kPermChunk) {
+    if (moe::launch_router_logits(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, logits, T,
+                                  E, d, status, st) != cudaSuccess ||
+        moe::launch_topk_softmax(logits, T, E, k, topk_idx_dev, topk_w_dev, st) != cudaSuccess ||
+        moe::launch_perm_small(topk_idx_dev, T, k, E, counts_dev, offsets_dev, mprefix, perm_dev,
+                               st) != cudaSuccess) {
+      cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+    return MOE_OK;
+  }
   if (moe::launch_router_logits(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, logits, T,
                                 E, d, status, st) != cudaSuccess ||
       moe::launch_topk_softmax(logits, T, E, k, topk_idx_dev, topk_w_dev, st) != cudaSuccess ||

@@ -164,15 +164,15 @@ __global__ void __launch_bounds__(RouterCfg<BE>::THREADS)
 // operation sequence, so identical router rows give bit-identical logits.
 constexpr int RS_EXPERTS = 32;  // experts per block (8 warps x 4)
 
-__global__ void __launch_bounds__(256) router_logits_small_kernel(
-    const uint16_t* __restrict__ x, const float* __restrict__ W_r, const float* __restrict__ b_r,
-    float* __restrict__ logits, int T, int E, int d, int* status) {
-  const int t = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (status && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status = 0;
-  const int e0 = blockIdx.y * RS_EXPERTS + warp * 4;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
-  const uint16_t* xr = x + (size_t)t * d;
+// Logits of experts e0..e0+3 for one token row xr (one warp): after the
+// butterfly every lane holds the four sums (bias not added).
+__device__ __forceinline__ void router_dot4(const uint16_t* __restrict__ xr,
+                                            const float* __restrict__ W_r, int e0, int E, int d,
+                                            int lane, float (&acc)[4]) {
+  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+  // unrolled so that several iterations' loads are in flight; the fma order
+  // per expert is unchanged (increasing k)
+#pragma unroll 4
   for (int k = lane * 4; k < d; k += 128) {
     const uint2 xv = __ldg(reinterpret_cast<const uint2*>(xr + k));
     const float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xFFFF0000u);
@@ -193,6 +193,17 @@ __global__ void __launch_bounds__(256) router_logits_small_kernel(
   for (int j = 0; j < 4; ++j)
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xFFFFFFFFu, acc[j], off);
+}
+
+__global__ void __launch_bounds__(256) router_logits_small_kernel(
+    const uint16_t* __restrict__ x, const float* __restrict__ W_r, const float* __restrict__ b_r,
+    float* __restrict__ logits, int T, int E, int d, int* status) {
+  const int t = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (status && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status = 0;
+  const int e0 = blockIdx.y * RS_EXPERTS + warp * 4;
+  float acc[4];
+  router_dot4(x + (size_t)t * d, W_r, e0, E, d, lane, acc);
   if (lane < 4) {
     const int e = e0 + lane;
     const float v = lane == 0 ? acc[0] : lane == 1 ? acc[1] : lane == 2 ? acc[2] : acc[3];
@@ -204,14 +215,9 @@ __global__ void __launch_bounds__(256) router_logits_small_kernel(
 // One warp per token. Lane l holds the logits of experts l, l+32, ...; k rounds
 // of a warp arg-max on (logit descending, index ascending). Lane j keeps the
 // j-th winner; the softmax runs over the k winners only.
-__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits,
-                                                           int T, int E, int k,
-                                                           int32_t* __restrict__ topk_idx,
-                                                           float* __restrict__ topk_w) {
-  const int lane = threadIdx.x & 31;
-  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (t >= T) return;
-  const float* s = logits + (size_t)t * E;
+__device__ __forceinline__ void topk_softmax_warp(const float* s, int E, int k, int lane,
+                                                  int32_t* __restrict__ idx_out,
+                                                  float* __restrict__ w_out) {
   float v[8];
   uint32_t taken = 0;
 #pragma unroll
@@ -257,9 +263,20 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
   if (lane < k) {
-    topk_idx[(size_t)t * k + lane] = my_idx;
-    topk_w[(size_t)t * k + lane] = ex / sum;
+    idx_out[lane] = my_idx;
+    w_out[lane] = ex / sum;
   }
+}
+
+__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits,
+                                                           int T, int E, int k,
+                                                           int32_t* __restrict__ topk_idx,
+                                                           float* __restrict__ topk_w) {
+  const int lane = threadIdx.x & 31;
+  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (t >= T) return;
+  topk_softmax_warp(logits + (size_t)t * E, E, k, lane, topk_idx + (size_t)t * k,
+                    topk_w + (size_t)t * k);
 }
 
 // --------------------------------------------------------- K2 histogram ----
@@ -365,6 +382,75 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(const int32_t* __rest
       perm[pos] = (int32_t)q;
       if (inv) inv[q] = pos;
     }
+  }
+}
+
+// ------------------------------------------------------ K2, small batches ----
+// For T <= kPermChunk (one chunk): histogram, scan and stable scatter in one
+// block, with the per-warp segments and ranks of perm_scatter_kernel; writes
+// counts, offsets, the M-tile prefix and perm exactly as the three kernels do.
+__global__ void __launch_bounds__(256) perm_small_kernel(const int32_t* __restrict__ topk_idx,
+                                                         int T, int k, int E,
+                                                         int32_t* __restrict__ counts,
+                                                         int32_t* __restrict__ offsets,
+                                                         int32_t* __restrict__ mtile_prefix,
+                                                         int32_t* __restrict__ perm) {
+  __shared__ int wbase[8][256];
+  __shared__ int s_cnt[256], s_mt[256];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < 8 * 256; i += blockDim.x) (&wbase[0][0])[i] = 0;
+  __syncthreads();
+  const int64_t qc1 = (int64_t)min(T, kPermChunk) * k;
+  const int64_t seg = (int64_t)(kPermChunk / 8) * k;
+  const int64_t q0 = warp * seg;
+  const int64_t q1 = min(qc1, q0 + seg);
+  for (int64_t q = q0 + lane; q < q1; q += 32) atomicAdd(&wbase[warp][topk_idx[q]], 1);
+  __syncthreads();
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < E)
+    for (int w = 0; w < 8; ++w) total += wbase[w][e];
+  s_cnt[e] = (e < E) ? total : 0;
+  s_mt[e] = (e < E) ? (total + kTileM - 1) / kTileM : 0;
+  __syncthreads();
+  if (e == 0) {  // E <= 256: a serial scan is cheap and plainly ordered
+    int a = 0, m = 0;
+    for (int i = 0; i < E; ++i) {
+      const int c = s_cnt[i], mt = s_mt[i];
+      s_cnt[i] = a;
+      s_mt[i] = m;
+      a += c;
+      m += mt;
+    }
+    offsets[E] = a;
+    mtile_prefix[E] = m;
+  }
+  __syncthreads();
+  if (e < E) {
+    offsets[e] = s_cnt[e];
+    mtile_prefix[e] = s_mt[e];
+    if (counts) counts[e] = total;
+    int run = s_cnt[e];
+    for (int w = 0; w < 8; ++w) {
+      const int c = wbase[w][e];
+      wbase[w][e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  const uint32_t lt = (1u << lane) - 1u;
+  for (int64_t qb = q0; qb < q1; qb += 32) {
+    const int64_t q = qb + lane;
+    const bool valid = q < q1;
+    const int ex = valid ? topk_idx[q] : -1 - lane;
+    const uint32_t m = __match_any_sync(0xFFFFFFFFu, ex);
+    const int rank = __popc(m & lt);
+    int pos = 0;
+    if (valid) pos = wbase[warp][ex] + rank;
+    __syncwarp();
+    if (valid && lane == __ffs(m) - 1) wbase[warp][ex] += __popc(m);
+    __syncwarp();
+    if (valid) perm[pos] = (int32_t)q;
   }
 }
 
@@ -526,6 +612,14 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, const floa
   }
   if (E <= 32) return launch_router_be<32>(x, W_r, b_r, logits, T, E, d, status, st);
   return launch_router_be<64>(x, W_r, b_r, logits, T, E, d, status, st);
+}
+
+cudaError_t launch_perm_small(const int32_t* topk_idx, int T, int k, int E, int32_t* counts,
+                              int32_t* offsets, int32_t* mtile_prefix, int32_t* perm,
+                              cudaStream_t st) {
+  if (T < 1 || T > kPermChunk) return cudaErrorInvalidValue;
+  perm_small_kernel<<<1, 256, 0, st>>>(topk_idx, T, k, E, counts, offsets, mtile_prefix, perm);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_topk_softmax(const float* logits, int T, int E, int k, int32_t* topk_idx,
