@@ -18,6 +18,8 @@ matmul as the only library primitive. Sources (page title, section):
 * "shrink/gpt_oss-mic", "Preserved properties": hidden_act is silu.
 * "gpt-oss-20b and gpt-oss-120b", "Four-bit expert weights": MXFP4, 4.25 bits
   per parameter counting the shared scales, to be decoded exactly.
+* field guide "gpt-oss 20B", "04 One decoder block": RMSNorm before the MoE,
+  the sublayer added back to the residual stream (``rms_norm``, ``moe_block``).
 
 Readings where the pages are silent (each also listed in the design notes):
 
@@ -27,7 +29,9 @@ Readings where the pages are silent (each also listed in the design notes):
 * MX groups run along the contraction dimension, 32 elements per E8M0 scale
   (bias 127, 0xFF is NaN); byte b holds element 2b in its low nibble;
 * E2M1 is 1 sign bit, 2 exponent bits with bias 1, 1 mantissa bit, with a
-  subnormal at exponent 0 (OCP Microscaling definition).
+  subnormal at exponent 0 (OCP Microscaling definition);
+* RMSNorm is g * h / sqrt(mean(h^2) + eps) with a caller-chosen eps, and its
+  output enters the layer rounded to bf16; the residual add is unrounded.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (closed forms, brute force, the silent-init identity, and the pages' printed
@@ -286,6 +290,54 @@ def moe_forward(x_bits, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales,
     if return_hidden:
         return out, r, hidden
     return out
+
+
+# --------------------------------------------------------------------------
+# Around the layer: the pre-MoE RMSNorm and the residual add
+# --------------------------------------------------------------------------
+
+
+def f64_to_bf16_bits(a: np.ndarray) -> np.ndarray:
+    """Round fp64 values to bf16 (nearest, ties to even), returned as bf16 bit
+    patterns. A bf16 value has 8 significant bits; below 2^-126 the quantum
+    stays 2^-133 (bf16 subnormals). Finite inputs within the bf16 range."""
+    a = np.asarray(a, dtype=np.float64)
+    _, e = np.frexp(a)                                  # a = m 2^e, 0.5 <= |m| < 1
+    q = np.exp2(np.maximum(e - 8, -133).astype(np.float64))
+    r = np.rint(a / q) * q                              # rint rounds halves to even
+    return (r.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
+def rms_norm(h: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
+    """RMSNorm(h)_i = g_i h_i / sqrt(mean_j h_j^2 + eps), row by row, fp64.
+
+    Field guide "gpt-oss 20B", "04 One decoder block": RMSNorm is applied
+    before the MoE. The pages give no formula or epsilon; the standard form
+    with a per-channel gain g and a caller-chosen eps is the reading taken.
+    """
+    h = np.asarray(h, dtype=np.float64)
+    ms = np.mean(h * h, axis=1, keepdims=True)
+    return h / np.sqrt(ms + eps) * np.asarray(g, dtype=np.float64)[None, :]
+
+
+def moe_block(h_bits, g, eps, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, k: int,
+              x_bits: Optional[np.ndarray] = None, tokens: Optional[Iterable[int]] = None):
+    """h + FFN(RMSNorm(h)) per token, in fp64: the MoE sublayer with its
+    pre-norm and residual add (field guide "gpt-oss 20B", "04 One decoder
+    block": each sublayer is added back to the residual stream).
+
+    The normalised rows enter the layer in its activation format, bf16:
+    x = bf16(RMSNorm(h)), unless ``x_bits`` supplies them. The layer output is
+    added to h before any rounding. Returns [T', d] float64.
+    """
+    h_all = np.asarray(h_bits)
+    tok = np.arange(h_all.shape[0]) if tokens is None else np.asarray(list(tokens), dtype=np.int64)
+    hf = bf16_to_f64(h_all[tok])
+    if x_bits is None:
+        xb = f64_to_bf16_bits(rms_norm(hf, g, eps))
+    else:
+        xb = np.asarray(x_bits)[tok]
+    return hf + moe_forward(xb, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, k=k)
 
 
 # --------------------------------------------------------------------------

@@ -293,14 +293,16 @@ def test_zero_tokens_is_a_no_op():
 
 
 def test_silent_init_identity_on_gpu():
-    """64a8 (x2 silent init) reproduces 32a4 at T = 64 (decode) and T = 512."""
+    """64a8 (x2 silent init) and 96a12 (x3) reproduce 32a4 at T = 64 (decode,
+    block-scaled tiles) and T = 512 (bf16 tiles)."""
     for T in (64, 512):
         base = W.make_inputs("20b", T=T)
-        exp = W.make_inputs("64a8", T=T)
         o2, _ = G.run_forward(base)
-        o8, _ = G.run_forward(exp)
         want = O.bf16_to_f64(o2)
-        G.assert_out_close(o8, want, what=f"64a8 vs 20b at T={T}")
+        for name in ("64a8", "96a12"):
+            exp = W.make_inputs(name, T=T)
+            o8, _ = G.run_forward(exp)
+            G.assert_out_close(o8, want, what=f"{name} vs 20b at T={T}")
 
 
 def test_timeout_path_reports_status_and_device_survives():

@@ -19,6 +19,9 @@ PIN_TESTS = [
     (P.test_selected_softmax_properties, {}),
     (P.test_routing_tables_match_stable_sort, {}),
     (P.test_k_equals_E_is_dense_mixture, {}),
+    (P.test_f64_to_bf16_rounding, {}),
+    (P.test_rms_norm_closed_forms, {}),
+    (P.test_moe_block_residual_and_norm, {}),
 ]
 
 
@@ -81,7 +84,23 @@ def _mut_unstable_tables(idx, E):
     return c, o, perm, inv
 
 
+def _mut_norm_sum_not_mean(h, g, eps):
+    h = np.asarray(h, dtype=np.float64)
+    ss = np.sum(h * h, axis=1, keepdims=True)
+    return h / np.sqrt(ss + eps) * np.asarray(g, dtype=np.float64)[None, :]
+
+
+def _mut_no_residual(h_bits, g, eps, *args, **kw):
+    return _orig_block(h_bits, g, eps, *args, **kw) - O.bf16_to_f64(np.asarray(h_bits))
+
+
+def _mut_round_toward_zero(a):
+    a = np.asarray(a, dtype=np.float64)
+    return (a.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+
+
 _orig_router = O.router_logits
+_orig_block = O.moe_block
 _orig_decode = O.mxfp4_decode
 _orig_e8m0 = O.e8m0_value
 _orig_tables = O.routing_tables
@@ -96,6 +115,9 @@ MUTATIONS = {
     "down projection transposed": ("expert_out", _mut_down_transposed),
     "ties to the higher index": ("topk_select", _mut_topk_high_index_ties),
     "unstable grouping": ("routing_tables", _mut_unstable_tables),
+    "norm by the sum of squares": ("rms_norm", _mut_norm_sum_not_mean),
+    "residual add dropped": ("moe_block", _mut_no_residual),
+    "bf16 truncation": ("f64_to_bf16_bits", _mut_round_toward_zero),
 }
 
 

@@ -375,3 +375,64 @@ def test_near_tie_detector():
     s = np.array([[3.0, 1.0, 1.0 + 5e-6, 0.0], [3.0, 2.0, 1.0, 0.0]])
     r = O.Routing(s, O.topk_select(s, 2), None)
     assert r.near_tie().tolist() == [True, False]
+
+
+# --------------------------------------------- pre-norm and residual add ----
+
+def test_f64_to_bf16_rounding():
+    """Nearest-even rounding to 8 significant bits, checked on hand-made values."""
+    one = 1.0
+    cases = {
+        one: 0x3F80,
+        one + 2.0 ** -7: 0x3F81,            # exactly representable
+        one + 2.0 ** -8: 0x3F80,            # halfway: ties to the even mantissa
+        one + 3 * 2.0 ** -8: 0x3F82,        # halfway: ties up to the even mantissa
+        one + 2.0 ** -8 + 2.0 ** -20: 0x3F81,
+        -3.0: 0xC040,
+        2.0 ** -130: 0x0008,                # bf16 subnormal
+    }
+    got = O.f64_to_bf16_bits(np.array(list(cases)))
+    assert [int(v) for v in got] == list(cases.values())
+    x = np.random.default_rng(1).standard_normal(1000)
+    b = O.f64_to_bf16_bits(x)
+    back = O.bf16_to_f64(b)
+    assert np.all(np.abs(back - x) <= 2.0 ** -8 * np.abs(x))   # half a quantum of 8 bits
+
+
+def test_rms_norm_closed_forms():
+    rng = np.random.default_rng(2)
+    h = rng.standard_normal((5, 48)) * rng.uniform(0.1, 10, size=(5, 1))
+    one = np.ones(48)
+    y = O.rms_norm(h, one, 0.0)
+    assert np.allclose(np.mean(y * y, axis=1), 1.0, rtol=1e-13)      # unit mean square
+    assert np.allclose(O.rms_norm(7.5 * h, one, 0.0), y, rtol=1e-13)  # scale invariant
+    c = np.full((1, 48), -2.0)
+    g = rng.uniform(0.5, 2.0, size=48)
+    assert np.allclose(O.rms_norm(c, g, 0.25), -2.0 / math.sqrt(4.25) * g[None, :], rtol=1e-14)
+    assert np.all(O.rms_norm(np.zeros((1, 48)), g, 1e-5) == 0.0)
+
+
+def test_moe_block_residual_and_norm():
+    """Zero expert weights leave exactly h; the sublayer sees the normalised rows
+    (a positive rescale of h changes only the residual term)."""
+    d, I, E, k, T = 64, 96, 4, 2, 6
+    inp = W.make_custom(d, I, E, k, T, seed=9)
+    g = np.random.default_rng(3).uniform(0.5, 1.5, size=d)
+    zero_gu = np.zeros_like(inp.Wgu_codes)
+    zero_d = np.zeros_like(inp.Wd_codes)
+    out0 = O.moe_block(inp.x, g, 1e-5, inp.W_r, inp.b_r, zero_gu, inp.Wgu_scales, zero_d,
+                       inp.Wd_scales, k=k)
+    assert np.array_equal(out0, O.bf16_to_f64(inp.x))
+    # h and 4h (exact in bf16) normalise to the same x when eps = 0
+    h4 = O.f64_to_bf16_bits(4.0 * O.bf16_to_f64(inp.x))
+    a = O.moe_block(inp.x, g, 0.0, inp.W_r, inp.b_r, inp.Wgu_codes, inp.Wgu_scales,
+                    inp.Wd_codes, inp.Wd_scales, k=k)
+    b = O.moe_block(h4, g, 0.0, inp.W_r, inp.b_r, inp.Wgu_codes, inp.Wgu_scales,
+                    inp.Wd_codes, inp.Wd_scales, k=k)
+    hx = O.bf16_to_f64(inp.x)
+    assert np.allclose(b - 4.0 * hx, a - hx, rtol=1e-12, atol=1e-12)
+    # and the sublayer term is the layer applied to bf16(RMSNorm(h))
+    xb = O.f64_to_bf16_bits(O.rms_norm(hx, g, 0.0))
+    ff = O.moe_forward(xb, inp.W_r, inp.b_r, inp.Wgu_codes, inp.Wgu_scales, inp.Wd_codes,
+                       inp.Wd_scales, k=k)
+    assert np.array_equal(a - hx, ff) or np.allclose(a - hx, ff, rtol=1e-13, atol=1e-13)
