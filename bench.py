@@ -304,6 +304,38 @@ def run_ours(args, inp, name):
     if status != 0:
         raise RuntimeError(f"device status {B.STATUS.get(status, status)} in the timed region")
     step_s = sum(s[-1] for s in stage_ms) / 1e3
+    block = None
+    if args.block:
+        # the same steps through moe_forward_block (RMSNorm, the layer, the residual
+        # add); the layer's stage times above explain it
+        g = torch.from_numpy(np.random.default_rng(7).uniform(0.5, 1.5, inp.d)
+                             .astype(np.float32)).to(dev)
+        bws = torch.empty(B.moe_workspace_size_block(inp.E, inp.k, T, inp.d, inp.I),
+                          dtype=torch.uint8, device=dev)
+        for _ in range(args.warmup):
+            flush.zero_()
+            B.moe_forward_block(x, g, 1e-5, layer.W_r, layer.b_r, layer.Wgu_codes,
+                                layer.Wgu_scales, layer.Wd_codes, layer.Wd_scales, inp.E, inp.k,
+                                T, inp.d, inp.I, out, bws)
+        barrier(world)
+        torch.cuda.synchronize()
+        bsum = 0.0
+        for _ in range(args.steps):
+            flush.zero_()
+            ev0 = torch.cuda.Event(enable_timing=True)
+            ev1 = torch.cuda.Event(enable_timing=True)
+            ev0.record(stream)
+            B.moe_forward_block(x, g, 1e-5, layer.W_r, layer.b_r, layer.Wgu_codes,
+                                layer.Wgu_scales, layer.Wd_codes, layer.Wd_scales, inp.E, inp.k,
+                                T, inp.d, inp.I, out, bws)
+            ev1.record(stream)
+            ev1.synchronize()
+            bsum += ev0.elapsed_time(ev1) / 1e3
+        if B.moe_sync_status(bws) != 0:
+            raise RuntimeError("device status after the block steps")
+        block = {"layer_ms_per_step": 1e3 * step_s / args.steps,
+                 "norm_and_residual_ms_per_step": 1e3 * (bsum - step_s) / args.steps}
+        step_s = bsum
     step_s_max = reduce_max(step_s, world)
     tokens_all = T * args.steps * world
     value = tokens_all / step_s_max
@@ -355,7 +387,8 @@ def run_ours(args, inp, name):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
-        "config": dict(workload_config(inp, name), tile_policy=args.tile_policy),
+        "config": dict(workload_config(inp, name), tile_policy=args.tile_policy,
+                       **({"block": "out = h + MoE(RMSNorm(h)), eps 1e-5"} if args.block else {})),
         "layer_tflops": layer_flops(inp.d, inp.I, inp.E, inp.k, T) * args.steps * world
         / step_s_max / 1e12,
         "roofline": dict(roof, kernel=DOMINANT_STAGE, achieved=achieved, peak=peak,
@@ -364,9 +397,12 @@ def run_ours(args, inp, name):
         "stage_ms": stage_avg,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(T * inp.d * 2),
                 "d2h_bytes_per_step": int(T * inp.d * 2)},
-        "gpu_launches": B.moe_forward_launch_count(inp.E, inp.k, T, inp.d, inp.I) * args.steps,
+        "gpu_launches": (B.moe_forward_launch_count(inp.E, inp.k, T, inp.d, inp.I)
+                         + (1 if args.block else 0)) * args.steps,
         "clocks": clk.summary(),
     }
+    if block:
+        line["block"] = block
     return line
 
 
@@ -402,6 +438,9 @@ def main(argv=None):
     ap.add_argument("--workload", default="20b", choices=list(W.SHAPES))
     ap.add_argument("--T", type=int, default=None, help="tokens per GPU (default: prefill T)")
     ap.add_argument("--ref-tokens", type=int, default=2, help="oracle tokens per reference step")
+    ap.add_argument("--block", action="store_true",
+                    help="time the MoE sublayer with its pre-norm and residual add "
+                         "(moe_forward_block: out = h + MoE(RMSNorm(h)))")
     ap.add_argument("--probe-tensor", action="store_true",
                     help="print the measured UMMA rates (MAC per SM clock) and exit")
     ap.add_argument("--tile-policy", type=int, default=0, choices=[0, 1, 2, 3, 4],

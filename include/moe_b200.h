@@ -270,6 +270,36 @@ MOE_API moe_status moe_sync_status(void* workspace_dev, size_t workspace_bytes, 
 MOE_API moe_status moe_selftest_wait_timeout(void* workspace_dev, void* stream);
 
 /*
+ * The MoE sublayer of a decoder block with its pre-norm and residual add
+ * (field guide "gpt-oss 20B", "04 One decoder block": RMSNorm is applied
+ * before the MoE and the sublayer is added back to the residual stream):
+ *   x   = bf16((h / sqrt(mean(h^2) + eps)) * g)   per row (moe_rms_norm)
+ *   out = bf16(h + sum_j p_j E_j(x))              (one rounding, after the add)
+ * h_dev [T][d] bf16 (the residual stream), g_dev [d] f32 (the norm's gain),
+ * eps >= 0 (the pages give no value; gpt-oss configurations commonly use
+ * 1e-5). All other arguments, the result, the errors and the stream semantics
+ * are those of moe_forward; the workspace must hold
+ * moe_workspace_size_block(...) bytes (moe_forward's, plus the x rows).
+ * moe_forward_launch_count(...) + 1 launches.
+ */
+MOE_API size_t moe_workspace_size_block(int E, int k, int T, int d, int I);
+MOE_API moe_status moe_forward_block(const void* h_dev, const float* g_dev, float eps,
+                                     const float* W_r_dev, const float* b_r_dev,
+                                     const uint8_t* Wgu_codes_dev, const uint8_t* Wgu_scales_dev,
+                                     const uint8_t* Wd_codes_dev, const uint8_t* Wd_scales_dev,
+                                     int E, int k, int T, int d, int I, void* out_dev,
+                                     void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/*
+ * The pre-MoE RMSNorm alone: x_dev[t] = bf16((h[t] / sqrt(mean(h[t]^2) + eps)) * g),
+ * h_dev and x_dev [T][d] bf16, g_dev [d] f32; d a multiple of 32; all three
+ * 16-byte aligned and the caller's. Per row: fp32 sum of squares (a fixed
+ * lane-strided order), IEEE sqrt and division, one rounding to bf16.
+ */
+MOE_API moe_status moe_rms_norm(const void* h_dev, const float* g_dev, float eps, int T, int d,
+                                void* x_dev, void* stream);
+
+/*
  * Tensor-core rate probe (diagnostic; the pages have no counterpart): on every
  * SM one thread issues back-to-back UMMAs of M = 128 and N columns from
  * shared-memory tiles, per_commit per tcgen05.commit, and *mac_per_clk_sm

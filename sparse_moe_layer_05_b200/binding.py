@@ -30,6 +30,7 @@ EXPORTS = [
     "moe_route", "moe_workspace_layout", "moe_mxfp4_to_bf16", "moe_mx_split_e4m3", "moe_sync_status",
     "moe_selftest_wait_timeout", "moe_forward_launch_count", "moe_forward_timed",
     "moe_set_tile_policy", "moe_route_noalloc", "moe_probe_tensor_rate",
+    "moe_workspace_size_block", "moe_forward_block", "moe_rms_norm",
 ]
 
 STAGES = ["router_logits", "topk_softmax", "perm_hist", "perm_scan", "perm_scatter",
@@ -87,6 +88,12 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_workspace_layout.argtypes = [i32] * 5 + [ctypes.POINTER(WsLayout)]
     lib.moe_mxfp4_to_bf16.restype = i32
     lib.moe_mxfp4_to_bf16.argtypes = [u8p, u8p, i32, i32, vp, vp]
+    lib.moe_workspace_size_block.restype = sz
+    lib.moe_workspace_size_block.argtypes = [i32] * 5
+    lib.moe_forward_block.restype = i32
+    lib.moe_forward_block.argtypes = [vp, fp, ctypes.c_float] + fwd[1:]
+    lib.moe_rms_norm.restype = i32
+    lib.moe_rms_norm.argtypes = [vp, fp, ctypes.c_float, i32, i32, vp, vp]
     lib.moe_probe_tensor_rate.restype = i32
     lib.moe_probe_tensor_rate.argtypes = [i32, i32, i32, ctypes.POINTER(ctypes.c_double), vp]
     lib.moe_mx_split_e4m3.restype = i32
@@ -207,6 +214,25 @@ def moe_route_noalloc(x, W_r, b_r, E, k, T, d, topk_idx, topk_w, counts, offsets
     _check("moe_route_noalloc", load().moe_route_noalloc(
         _ptr(x), _ptr(W_r), _ptr(b_r), E, k, T, d, _ptr(topk_idx), _ptr(topk_w), _ptr(counts),
         _ptr(offsets), _ptr(perm), _stream(stream)))
+
+
+def moe_workspace_size_block(E: int, k: int, T: int, d: int, I: int) -> int:
+    return int(load().moe_workspace_size_block(E, k, T, d, I))
+
+
+def moe_rms_norm(h, g, eps: float, T: int, d: int, x, stream=None) -> None:
+    _require_cuda(h, g, x)
+    _check("moe_rms_norm", load().moe_rms_norm(_ptr(h), _ptr(g), eps, T, d, _ptr(x), _stream(stream)))
+
+
+def moe_forward_block(h, g, eps: float, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales,
+                      E: int, k: int, T: int, d: int, I: int, out, workspace, stream=None) -> None:
+    """out = h + MoE(RMSNorm(h)) (bf16 rows; g f32 gain)."""
+    _require_cuda(h, g, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, out, workspace)
+    _check("moe_forward_block", load().moe_forward_block(
+        _ptr(h), _ptr(g), eps, _ptr(W_r), _ptr(b_r), _ptr(Wgu_codes), _ptr(Wgu_scales),
+        _ptr(Wd_codes), _ptr(Wd_scales), E, k, T, d, I, _ptr(out), _ptr(workspace),
+        workspace.numel(), _stream(stream)))
 
 
 def moe_probe_tensor_rate(kind: int, N: int, per_commit: int, stream=None) -> float:

@@ -48,6 +48,7 @@ struct Layout {
   moe_ws_layout pub;
   size_t mprefix, chunk_hist, chunk_base, x_in, out_buf, gu_scales_t, d_scales_t;
   size_t mx_tok_rows;
+  size_t x_norm;   // moe_forward_block: the normalised rows [T][d] bf16
 };
 
 bool shape_ok(int E, int k, int T, int d) {
@@ -63,7 +64,7 @@ bool full_shape_ok(int E, int k, int T, int d, int I) {
   return shape_ok(E, k, T, d) && I >= 32 && I <= 16384 && I % 32 == 0;
 }
 
-void make_layout(int E, int k, int T, int d, int I, bool hostio, Layout* L) {
+void make_layout(int E, int k, int T, int d, int I, bool hostio, Layout* L, bool block = false) {
   const size_t P = static_cast<size_t>(T) * k;
   const size_t NB = static_cast<size_t>(moe::perm_chunks(T));
   size_t off = 0;
@@ -97,6 +98,7 @@ void make_layout(int E, int k, int T, int d, int I, bool hostio, Layout* L) {
     L->x_in = take(static_cast<size_t>(T) * d * 2);
     L->out_buf = take(static_cast<size_t>(T) * d * 2);
   }
+  if (block) L->x_norm = take(static_cast<size_t>(T) * d * 2);
   L->pub.total = off;
 }
 
@@ -217,10 +219,13 @@ moe_status launch_routing(const uint16_t* x, const float* W_r, const float* b_r,
   return MOE_OK;
 }
 
+// The forward pass on the caller's stream. resid (optional, [T][d] bf16) is
+// added to the layer output before its rounding to bf16.
 moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, const uint8_t* gc,
                        const uint8_t* gs, const uint8_t* dc, const uint8_t* ds, int E, int k,
                        int T, int d, int I, uint16_t* out, void* ws, const Layout& L,
-                       cudaStream_t st, int num_sms, const StageEvents* tev = nullptr) {
+                       cudaStream_t st, int num_sms, const StageEvents* tev = nullptr,
+                       const uint16_t* resid = nullptr) {
   StageEvents none;
   memset(&none, 0, sizeof(none));
   const StageEvents& E_ = tev ? *tev : none;
@@ -295,7 +300,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     m2.n_out = d;
     MOE_CUDA(moe::launch_mx_gemm_down(variant, m2, num_sms, st));
     E_.mark(10);
-    MOE_CUDA(moe::launch_combine(yw, T, k, d, out, st));
+    MOE_CUDA(moe::launch_combine(yw, T, k, d, resid, out, st));
     E_.mark(11);
     return MOE_OK;
   }
@@ -339,7 +344,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   g2.n_out = d;
   MOE_CUDA(moe::launch_gemm_down_combine(g2, num_sms, st));
   E_.mark(10);
-  MOE_CUDA(moe::launch_combine(yw, T, k, d, out, st));
+  MOE_CUDA(moe::launch_combine(yw, T, k, d, resid, out, st));
   E_.mark(11);
   return MOE_OK;
 }
@@ -420,6 +425,53 @@ moe_status moe_forward(const void* x_dev, const float* W_r_dev, const float* b_r
                      Wgu_scales_dev, Wd_codes_dev, Wd_scales_dev, E, k, T, d, I,
                      static_cast<uint16_t*>(out_dev), workspace_dev, L,
                      static_cast<cudaStream_t>(stream), num_sms);
+}
+
+size_t moe_workspace_size_block(int E, int k, int T, int d, int I) {
+  if (!full_shape_ok(E, k, T, d, I)) return 0;
+  Layout L;
+  make_layout(E, k, T, d, I, false, &L, true);
+  return L.pub.total;
+}
+
+moe_status moe_rms_norm(const void* h_dev, const float* g_dev, float eps, int T, int d,
+                        void* x_dev, void* stream) {
+  if (!h_dev || !g_dev || !x_dev || T < 0 || d < 32 || d % 32 || !(eps >= 0.f))
+    return MOE_ERR_INVALID_ARG;
+  if (!aligned16(h_dev) || !aligned16(g_dev) || !aligned16(x_dev)) return MOE_ERR_INVALID_ARG;
+  if (T == 0) return MOE_OK;
+  int num_sms = 0;
+  moe_status s = device_info(&num_sms);
+  if (s != MOE_OK) return s;
+  MOE_CUDA(moe::launch_rms_norm(static_cast<const uint16_t*>(h_dev), g_dev, eps, T, d,
+                                static_cast<uint16_t*>(x_dev), static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
+}
+
+moe_status moe_forward_block(const void* h_dev, const float* g_dev, float eps, const float* W_r_dev,
+                             const float* b_r_dev, const uint8_t* Wgu_codes_dev,
+                             const uint8_t* Wgu_scales_dev, const uint8_t* Wd_codes_dev,
+                             const uint8_t* Wd_scales_dev, int E, int k, int T, int d, int I,
+                             void* out_dev, void* workspace_dev, size_t workspace_bytes,
+                             void* stream) {
+  moe_status s = check_forward_args(h_dev, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev,
+                                    Wd_codes_dev, Wd_scales_dev, E, k, T, d, I, out_dev,
+                                    workspace_dev);
+  if (s != MOE_OK) return s;
+  if (!g_dev || !aligned16(g_dev) || !(eps >= 0.f)) return MOE_ERR_INVALID_ARG;
+  Layout L;
+  make_layout(E, k, T, d, I, false, &L, true);
+  if (workspace_bytes < L.pub.total) return MOE_ERR_WORKSPACE;
+  if (T == 0) return MOE_OK;
+  int num_sms = 0;
+  if ((s = device_info(&num_sms)) != MOE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const uint16_t* h = static_cast<const uint16_t*>(h_dev);
+  uint16_t* x = at<uint16_t>(workspace_dev, L.x_norm);
+  MOE_CUDA(moe::launch_rms_norm(h, g_dev, eps, T, d, x, st));
+  return run_forward(x, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev, Wd_codes_dev,
+                     Wd_scales_dev, E, k, T, d, I, static_cast<uint16_t*>(out_dev), workspace_dev,
+                     L, st, num_sms, nullptr, h);
 }
 
 moe_status moe_forward_hostio(const void* x_host, const float* W_r_dev, const float* b_r_dev,

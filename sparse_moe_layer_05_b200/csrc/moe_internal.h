@@ -44,9 +44,13 @@ cudaError_t launch_perm_scatter(const int32_t* topk_idx, int T, int k, int E,
 // K2: gather activation rows into permuted order.
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* perm, int P, int k, int d,
                                uint16_t* xp, cudaStream_t st);
-// Per-token sum of the k weighted expert rows, rounded to bf16.
-cudaError_t launch_combine(const float* yw, int T, int k, int d, uint16_t* out,
-                           cudaStream_t st);
+// Per-token sum of the k weighted expert rows (plus the residual row, when
+// resid is not null), rounded once to bf16.
+cudaError_t launch_combine(const float* yw, int T, int k, int d, const uint16_t* resid,
+                           uint16_t* out, cudaStream_t st);
+// Pre-MoE RMSNorm: x = bf16((h / sqrt(mean(h^2) + eps)) * g), rows of d.
+cudaError_t launch_rms_norm(const uint16_t* h, const float* g, float eps, int T, int d,
+                            uint16_t* x, cudaStream_t st);
 // E8M0 scales [E][N][G] -> [E][G][N] (the GEMMs load them with TMA per k-block);
 // experts with counts[e] == 0 are skipped (counts may be null: all experts).
 cudaError_t launch_transpose_scales(const uint8_t* in, int E, int N, int G, const int32_t* counts,

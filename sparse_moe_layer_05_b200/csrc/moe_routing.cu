@@ -475,7 +475,8 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
 // ------------------------------------------------------------- combine ----
 // out[t] = sum_j yw[t*k + j], j ascending, fp32, rounded once to bf16.
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ yw, int T, int k,
-                                                      int d, uint16_t* __restrict__ out) {
+                                                      int d, const uint16_t* __restrict__ resid,
+                                                      uint16_t* __restrict__ out) {
   const int vec = d / 8;
   const int64_t n = (int64_t)T * vec;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
@@ -491,6 +492,15 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
       acc[0] += a.x; acc[1] += a.y; acc[2] += a.z; acc[3] += a.w;
       acc[4] += b.x; acc[5] += b.y; acc[6] += b.z; acc[7] += b.w;
     }
+    if (resid) {  // residual add (fp32), before the single rounding to bf16
+      const uint4 r = __ldg(reinterpret_cast<const uint4*>(resid + (size_t)t * d) + c);
+      const uint32_t rw[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        acc[2 * u] += __uint_as_float(rw[u] << 16);
+        acc[2 * u + 1] += __uint_as_float(rw[u] & 0xFFFF0000u);
+      }
+    }
     uint32_t o[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -498,6 +508,46 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
       o[u] = *reinterpret_cast<const uint32_t*>(&h);
     }
     reinterpret_cast<uint4*>(out + (size_t)t * d)[c] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+}
+
+// ----------------------------------------------------- pre-MoE RMSNorm ----
+// x = bf16((h / sqrt(mean(h^2) + eps)) * g), one warp per row: lane l sums the
+// squares of elements 4l + 128i .. +3 in increasing i (fp32 fma), a butterfly
+// adds the 32 partial sums, then every element is divided by the root and
+// multiplied by its gain, rounded once.
+// Field guide "gpt-oss 20B", "04 One decoder block" (RMSNorm before the MoE).
+__global__ void __launch_bounds__(256) rms_norm_kernel(const uint16_t* __restrict__ h,
+                                                       const float* __restrict__ g, float eps,
+                                                       int T, int d, uint16_t* __restrict__ x) {
+  const int lane = threadIdx.x & 31;
+  const int nwarps = (gridDim.x * blockDim.x) >> 5;
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
+    const uint16_t* hr = h + (size_t)t * d;
+    float ss = 0.f;
+    for (int k = lane * 4; k < d; k += 128) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(hr + k));
+      const float a = __uint_as_float(v.x << 16), b = __uint_as_float(v.x & 0xFFFF0000u);
+      const float c = __uint_as_float(v.y << 16), e = __uint_as_float(v.y & 0xFFFF0000u);
+      ss = fmaf(a, a, ss);
+      ss = fmaf(b, b, ss);
+      ss = fmaf(c, c, ss);
+      ss = fmaf(e, e, ss);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, off);
+    const float root = sqrtf(ss / (float)d + eps);
+    uint16_t* xr = x + (size_t)t * d;
+    for (int k = lane * 4; k < d; k += 128) {
+      const uint2 v = __ldg(reinterpret_cast<const uint2*>(hr + k));
+      const float4 gv = __ldg(reinterpret_cast<const float4*>(g + k));
+      const __nv_bfloat162 lo = __floats2bfloat162_rn((__uint_as_float(v.x << 16) / root) * gv.x,
+                                                      (__uint_as_float(v.x & 0xFFFF0000u) / root) * gv.y);
+      const __nv_bfloat162 hi = __floats2bfloat162_rn((__uint_as_float(v.y << 16) / root) * gv.z,
+                                                      (__uint_as_float(v.y & 0xFFFF0000u) / root) * gv.w);
+      reinterpret_cast<uint2*>(xr + k)[0] =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&lo), *reinterpret_cast<const uint32_t*>(&hi));
+    }
   }
 }
 
@@ -655,10 +705,16 @@ cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* perm, int P, in
   return cudaGetLastError();
 }
 
-cudaError_t launch_combine(const float* yw, int T, int k, int d, uint16_t* out,
-                           cudaStream_t st) {
+cudaError_t launch_combine(const float* yw, int T, int k, int d, const uint16_t* resid,
+                           uint16_t* out, cudaStream_t st) {
   const int64_t n = (int64_t)T * (d / 8);
-  combine_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(yw, T, k, d, out);
+  combine_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(yw, T, k, d, resid, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rms_norm(const uint16_t* h, const float* g, float eps, int T, int d,
+                            uint16_t* x, cudaStream_t st) {
+  rms_norm_kernel<<<grid_for(T, 8, 148 * 8), 256, 0, st>>>(h, g, eps, T, d, x);
   return cudaGetLastError();
 }
 

@@ -14,6 +14,8 @@ Workloads follow the shapes the pages give:
   32 experts, top-4), field guide "gpt-oss 20B", "03 Sparse Mixture of Experts".
 * ``64a8``     -- silent-init x2 expansion of ``20b`` (64 experts, top-8),
   "llm-surgery-dark-arts-gpt-oss-40b-64a8-init", section 2 "Silent Init".
+* ``96a12``    -- silent-init x3 expansion of ``20b`` (96 experts, top-12),
+  the same page's 96a12 variant (copies at e+32 and e+64).
 * ``128a4``    -- gpt-oss-120b routing (128 experts, top-4), "gpt-oss-20b and
   gpt-oss-120b" overview; with 8 router biases raised by 2.0 (skewed load).
 * ``248a20``   -- "gpt-oss-220a20b" model card: 128 base + 120 added expert
@@ -75,6 +77,8 @@ SHAPES: Dict[str, Shape] = {
                  "uniform in [-8,-4]"),
     "64a8": Shape("64a8", 2880, 2880, 64, 8, 8192, 64, 119, 123,
                   "silent-init x2 expansion of 20b (copies at e+32)"),
+    "96a12": Shape("96a12", 2880, 2880, 96, 12, 8192, 64, 119, 123,
+                   "silent-init x3 expansion of 20b (copies at e+32, e+64)"),
     "128a4": Shape("128a4", 2880, 2880, 128, 4, 16384, 32, 119, 123,
                    "gpt-oss-120b routing with +2.0 bias on experts 0..7"),
     "248a20": Shape("248a20", 2880, 2880, 248, 20, 4096, 16, 119, 123,
@@ -192,10 +196,10 @@ def make_inputs(name: str, T: Optional[int] = None, seed: int = 0) -> MoEInputs:
         return make_custom(s.d, s.I, s.E, s.k, T, seed=seed,
                            scale_lo=s.scale_lo, scale_hi=s.scale_hi,
                            name=name, T_draw=T_full)
-    if name == "64a8":
+    if name in ("64a8", "96a12"):
         base = make_inputs("20b", T=T, seed=seed)
-        out = _expand_silent(base, 2)
-        out.name = "64a8"
+        out = _expand_silent(base, 2 if name == "64a8" else 3)
+        out.name = name
         return out
     if name == "128a4":
         inp = make_custom(s.d, s.I, s.E, s.k, T, seed=seed + 1,

@@ -254,6 +254,40 @@ def test_tensor_rate_probe_near_the_nominal_dense_rates():
     assert 0.6 * 8192 <= mx <= 1.05 * 8192, mx
 
 
+@pytest.mark.parametrize("d,I,E,k,T", [(2880, 2880, 32, 4, 64), (352, 224, 8, 2, 500)],
+                         ids=["block_scaled_decode", "bf16_tiles"])
+def test_forward_block_rms_norm_and_residual(d, I, E, k, T):
+    """out = h + MoE(RMSNorm(h)): the norm against the oracle within one bf16 ulp, then
+    the block against h + MoE(x) computed by the oracle from the same normalised rows,
+    with the layer's tolerance on the sublayer term plus the output's bf16 rounding."""
+    from sparse_moe_layer_05_b200 import binding as B
+    inp = W.make_custom(d, I, E, k, T, seed=41)
+    rng = np.random.default_rng(42)
+    h = W.f32_to_bf16_bits((O.bf16_to_f64(inp.x) * 3.0 + 0.5).astype(np.float32))
+    g = rng.uniform(0.5, 1.5, size=d).astype(np.float32)
+    eps = 1e-5
+    layer = B.MoELayer(inp)
+    ht, gt = _t(h), torch.from_numpy(g).cuda()
+    xt = torch.empty_like(ht)
+    B.moe_rms_norm(ht, gt, eps, T, d, xt)
+    torch.cuda.synchronize()
+    x_gpu = xt.cpu().numpy()
+    x_or = O.f64_to_bf16_bits(O.rms_norm(O.bf16_to_f64(h), g.astype(np.float64), eps))
+    a, b = O.bf16_to_f64(x_gpu), O.bf16_to_f64(x_or)
+    assert np.all(np.abs(a - b) <= 2.0 ** -7 * np.maximum(np.abs(a), np.abs(b)))
+    ws = torch.empty(B.moe_workspace_size_block(E, k, T, d, I), dtype=torch.uint8, device="cuda")
+    out = torch.empty((T, d), dtype=torch.uint16, device="cuda")
+    B.moe_forward_block(ht, gt, eps, layer.W_r, layer.b_r, layer.Wgu_codes, layer.Wgu_scales,
+                        layer.Wd_codes, layer.Wd_scales, E, k, T, d, I, out, ws)
+    assert B.moe_sync_status(ws) == 0
+    got = O.bf16_to_f64(out.cpu().numpy())
+    want = O.moe_block(h, g, eps, inp.W_r, inp.b_r, inp.Wgu_codes, inp.Wgu_scales, inp.Wd_codes,
+                       inp.Wd_scales, k=k, x_bits=x_gpu)
+    ff = want - O.bf16_to_f64(h)
+    bound = 2e-2 * np.sqrt(np.mean(ff ** 2)) + 2.0 ** -8 * np.abs(want)
+    assert np.all(np.abs(got - want) <= bound), np.max(np.abs(got - want) / bound)
+
+
 def test_forward_deterministic_and_hostio_equal():
     from sparse_moe_layer_05_b200.binding import MoELayer
     inp = W.make_custom(352, 224, 8, 2, 600, seed=12)
