@@ -162,6 +162,13 @@ MOE_API moe_status moe_forward_timed(const void* x_dev, const float* W_r_dev, co
  * runs the forward pass and copies the result to out_host, then synchronises
  * `stream`. Expert and router weights stay on the device (the layer's
  * resident parameters). moe_workspace_size_hostio() gives the workspace size.
+ * Batches of at least 2048 tokens are processed as 4 chunks of tokens (each
+ * token's output depends on that token alone, so the result is the same):
+ * the copy in, the forward and the copy out of neighbouring chunks overlap on
+ * two copy streams the library creates once per device, ordered after the
+ * caller's earlier work on `stream`. Not thread-safe against concurrent
+ * host-buffer calls on one device. moe_workspace_size_hostio() is at least
+ * moe_workspace_size(), so one workspace serves both calls.
  */
 MOE_API size_t moe_workspace_size_hostio(int E, int k, int T, int d, int I);
 MOE_API moe_status moe_forward_hostio(const void* x_host, const float* W_r_dev, const float* b_r_dev,

@@ -122,6 +122,45 @@ void make_route_layout(int E, int k, int T, int d, Layout* L) {
   L->pub.total = off;
 }
 
+// Host-buffer calls on batches of at least kHostioChunkMin tokens split the
+// tokens into kHostioChunks chunks (each token's output depends on that token
+// alone, so the result is the same): the copy in of one chunk, the forward of
+// another and the copy out of a third overlap. Two chunk workspaces alternate;
+// the input and output rows of the whole batch are staged in the workspace.
+constexpr int kHostioChunks = 4;
+constexpr int kHostioChunkMin = 2048;
+
+struct HostioPlan {
+  int chunks, Tc;
+  Layout sub;          // layout of one chunk workspace (Tc tokens)
+  size_t sub_stride;   // bytes between the two chunk workspaces
+  size_t x_in, out_buf, total;
+};
+
+void make_hostio_plan(int E, int k, int T, int d, int I, HostioPlan* hp) {
+  memset(hp, 0, sizeof(*hp));
+  hp->chunks = T >= kHostioChunkMin ? kHostioChunks : 1;
+  if (hp->chunks == 1) {
+    make_layout(E, k, T, d, I, true, &hp->sub);
+    hp->Tc = T;
+    hp->x_in = hp->sub.x_in;
+    hp->out_buf = hp->sub.out_buf;
+    hp->total = hp->sub.pub.total;
+    return;
+  }
+  hp->Tc = (T + hp->chunks - 1) / hp->chunks;
+  make_layout(E, k, hp->Tc, d, I, false, &hp->sub);
+  hp->sub_stride = align256(hp->sub.pub.total);
+  const size_t rows = static_cast<size_t>(T) * d * 2;
+  hp->x_in = 2 * hp->sub_stride;
+  hp->out_buf = align256(hp->x_in + rows);
+  hp->total = align256(hp->out_buf + rows);
+  // a workspace sized for host-buffer calls also serves moe_forward
+  Layout full;
+  make_layout(E, k, T, d, I, false, &full);
+  if (hp->total < full.pub.total) hp->total = full.pub.total;
+}
+
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
 // Device capability and SM count, cached per device.
@@ -383,9 +422,9 @@ size_t moe_workspace_size(int E, int k, int T, int d, int I) {
 
 size_t moe_workspace_size_hostio(int E, int k, int T, int d, int I) {
   if (!full_shape_ok(E, k, T, d, I)) return 0;
-  Layout L;
-  make_layout(E, k, T, d, I, true, &L);
-  return L.pub.total;
+  HostioPlan hp;
+  make_hostio_plan(E, k, T, d, I, &hp);
+  return hp.total;
 }
 
 moe_status moe_workspace_layout(int E, int k, int T, int d, int I, moe_ws_layout* layout) {
@@ -483,26 +522,81 @@ moe_status moe_forward_hostio(const void* x_host, const float* W_r_dev, const fl
                                     Wd_codes_dev, Wd_scales_dev, E, k, T, d, I, out_host,
                                     workspace_dev);
   if (s != MOE_OK) return s;
-  Layout L;
-  make_layout(E, k, T, d, I, true, &L);
-  if (workspace_bytes < L.pub.total) return MOE_ERR_WORKSPACE;
+  HostioPlan hp;
+  make_hostio_plan(E, k, T, d, I, &hp);
+  if (workspace_bytes < hp.total) return MOE_ERR_WORKSPACE;
   if (T == 0) return MOE_OK;
   int num_sms = 0;
   if ((s = device_info(&num_sms)) != MOE_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t bytes = static_cast<size_t>(T) * d * 2;
-  uint16_t* x_in = at<uint16_t>(workspace_dev, L.x_in);
-  uint16_t* out_buf = at<uint16_t>(workspace_dev, L.out_buf);
-  MOE_CUDA(cudaMemcpyAsync(x_in, x_host, bytes, cudaMemcpyHostToDevice, st));
-  s = run_forward(x_in, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev, Wd_codes_dev,
-                  Wd_scales_dev, E, k, T, d, I, out_buf, workspace_dev, L, st, num_sms);
-  if (s != MOE_OK) return s;
-  MOE_CUDA(cudaMemcpyAsync(out_host, out_buf, bytes, cudaMemcpyDeviceToHost, st));
+  uint16_t* x_in = at<uint16_t>(workspace_dev, hp.x_in);
+  uint16_t* out_buf = at<uint16_t>(workspace_dev, hp.out_buf);
+  const uint16_t* xh = static_cast<const uint16_t*>(x_host);
+  uint16_t* oh = static_cast<uint16_t*>(out_host);
+  if (hp.chunks == 1) {
+    const size_t bytes = static_cast<size_t>(T) * d * 2;
+    MOE_CUDA(cudaMemcpyAsync(x_in, xh, bytes, cudaMemcpyHostToDevice, st));
+    s = run_forward(x_in, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev, Wd_codes_dev,
+                    Wd_scales_dev, E, k, T, d, I, out_buf, workspace_dev, hp.sub, st, num_sms);
+    if (s != MOE_OK) return s;
+    MOE_CUDA(cudaMemcpyAsync(oh, out_buf, bytes, cudaMemcpyDeviceToHost, st));
+  } else {
+    // copy streams and events, created once per device
+    struct CopyRes {
+      cudaStream_t h2d, d2h;
+      cudaEvent_t start, in[kHostioChunks], fwd[kHostioChunks], done;
+    };
+    static CopyRes res[kMaxDevices];
+    static bool have[kMaxDevices] = {false};
+    int dev = 0;
+    MOE_CUDA(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_NO_DEVICE;
+    CopyRes& r = res[dev];
+    if (!have[dev]) {
+      MOE_CUDA(cudaStreamCreateWithFlags(&r.h2d, cudaStreamNonBlocking));
+      MOE_CUDA(cudaStreamCreateWithFlags(&r.d2h, cudaStreamNonBlocking));
+      MOE_CUDA(cudaEventCreateWithFlags(&r.start, cudaEventDisableTiming));
+      MOE_CUDA(cudaEventCreateWithFlags(&r.done, cudaEventDisableTiming));
+      for (int c = 0; c < kHostioChunks; ++c) {
+        MOE_CUDA(cudaEventCreateWithFlags(&r.in[c], cudaEventDisableTiming));
+        MOE_CUDA(cudaEventCreateWithFlags(&r.fwd[c], cudaEventDisableTiming));
+      }
+      have[dev] = true;
+    }
+    // nothing of this call touches the workspace before the caller's earlier work on st
+    MOE_CUDA(cudaEventRecord(r.start, st));
+    MOE_CUDA(cudaStreamWaitEvent(r.h2d, r.start, 0));
+    for (int c = 0; c < hp.chunks; ++c) {
+      const int t0 = c * hp.Tc;
+      const int tn = T - t0 < hp.Tc ? T - t0 : hp.Tc;
+      if (tn <= 0) break;
+      const size_t off = static_cast<size_t>(t0) * d;
+      const size_t bytes = static_cast<size_t>(tn) * d * 2;
+      MOE_CUDA(cudaMemcpyAsync(x_in + off, xh + off, bytes, cudaMemcpyHostToDevice, r.h2d));
+      MOE_CUDA(cudaEventRecord(r.in[c], r.h2d));
+      MOE_CUDA(cudaStreamWaitEvent(st, r.in[c], 0));
+      // chunks c and c+2 share a workspace; both run in order on st
+      void* ws = static_cast<uint8_t*>(workspace_dev) + (c & 1) * hp.sub_stride;
+      s = run_forward(x_in + off, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev, Wd_codes_dev,
+                      Wd_scales_dev, E, k, tn, d, I, out_buf + off, ws, hp.sub, st, num_sms);
+      if (s != MOE_OK) return s;
+      MOE_CUDA(cudaEventRecord(r.fwd[c], st));
+      MOE_CUDA(cudaStreamWaitEvent(r.d2h, r.fwd[c], 0));
+      MOE_CUDA(cudaMemcpyAsync(oh + off, out_buf + off, bytes, cudaMemcpyDeviceToHost, r.d2h));
+    }
+    MOE_CUDA(cudaEventRecord(r.done, r.d2h));
+    MOE_CUDA(cudaStreamWaitEvent(st, r.done, 0));
+  }
   MOE_CUDA(cudaStreamSynchronize(st));
-  int dev_status = 0;
-  MOE_CUDA(cudaMemcpy(&dev_status, at<int>(workspace_dev, L.pub.status), sizeof(int),
-                      cudaMemcpyDeviceToHost));
-  return dev_status ? static_cast<moe_status>(dev_status) : MOE_OK;
+  // status words: one per (chunk) workspace
+  for (int w = 0; w < (hp.chunks > 1 ? 2 : 1); ++w) {
+    int dev_status = 0;
+    MOE_CUDA(cudaMemcpy(&dev_status,
+                        static_cast<uint8_t*>(workspace_dev) + w * hp.sub_stride + hp.sub.pub.status,
+                        sizeof(int), cudaMemcpyDeviceToHost));
+    if (dev_status) return static_cast<moe_status>(dev_status);
+  }
+  return MOE_OK;
 }
 
 moe_status moe_forward_timed(const void* x_dev, const float* W_r_dev, const float* b_r_dev,

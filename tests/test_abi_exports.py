@@ -52,6 +52,9 @@ def test_workspace_sizes():
     assert B.moe_workspace_size(4, 2, 8, 48, 64) == 0        # d % 32
     assert B.moe_workspace_size(4, 2, 8, 64, 40) == 0        # I % 32
     assert B.moe_workspace_size_hostio(4, 2, 8, 64, 64) > B.moe_workspace_size(4, 2, 8, 64, 64)
+    # chunked host-buffer calls (T >= 2048) still fit a device-buffer call
+    assert (B.moe_workspace_size_hostio(32, 4, 8192, 2880, 2880)
+            >= B.moe_workspace_size(32, 4, 8192, 2880, 2880))
     L = B.moe_workspace_layout(32, 4, 100, 2880, 2880)
     offs = sorted((v, k) for k, v in L.items() if k != "total")
     assert all(v % 256 == 0 for v, _ in offs)
