@@ -213,16 +213,25 @@ def silu(z: np.ndarray) -> np.ndarray:
         return z / (1.0 + np.exp(-z))
 
 
-def expert_hidden(xe: np.ndarray, Wgu: np.ndarray, I: int) -> np.ndarray:
-    """H = silu(xe Wgate^T) * (xe Wup^T); Wgu is the decoded [2I, d] matrix."""
+def expert_hidden(xe: np.ndarray, Wgu: np.ndarray, I: int,
+                  bias: Optional[np.ndarray] = None) -> np.ndarray:
+    """H = silu(xe Wgate^T + b_gate) * (xe Wup^T + b_up); Wgu is the decoded
+    [2I, d] matrix, bias (optional) the [2I] gate-then-up bias row."""
     g = xe @ Wgu[:I].T
     u = xe @ Wgu[I:].T
+    if bias is not None:
+        b = np.asarray(bias, dtype=np.float64)
+        g = g + b[None, :I]
+        u = u + b[None, I:]
     return silu(g) * u
 
 
-def expert_out(h: np.ndarray, Wd: np.ndarray) -> np.ndarray:
-    """y = H Wdown^T; Wd is the decoded [d, I] matrix."""
-    return h @ Wd.T
+def expert_out(h: np.ndarray, Wd: np.ndarray, bias: Optional[np.ndarray] = None) -> np.ndarray:
+    """y = H Wdown^T + b_down; Wd is the decoded [d, I] matrix, bias (optional) [d]."""
+    y = h @ Wd.T
+    if bias is not None:
+        y = y + np.asarray(bias, dtype=np.float64)[None, :]
+    return y
 
 
 # --------------------------------------------------------------------------
@@ -255,8 +264,13 @@ def route(x_bits: np.ndarray, W_r: np.ndarray, b_r: np.ndarray, k: int) -> Routi
 
 def moe_forward(x_bits, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales,
                 k: int, tokens: Optional[Iterable[int]] = None,
-                return_hidden: bool = False):
+                return_hidden: bool = False, Bgu: Optional[np.ndarray] = None,
+                Bd: Optional[np.ndarray] = None):
     """FFN(h) = sum_{i in top-k(s)} p_i(h) E_i(h) for each token, in fp64.
+
+    ``Bgu`` [E, 2I] and ``Bd`` [E, d] (optional) are per-expert biases of the
+    gate/up and down projections (the parameter totals of "gpt-oss-20b and
+    gpt-oss-120b" and the fixture page count them).
 
     ``tokens`` restricts the computation to a subset of rows (each token's
     output depends on that token alone). Returns out [T', d] float64, and with
@@ -280,8 +294,8 @@ def moe_forward(x_bits, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales,
             continue
         Wgu = mxfp4_decode(Wgu_codes[e], Wgu_scales[e])
         Wd = mxfp4_decode(Wd_codes[e], Wd_scales[e])
-        h = expert_hidden(xf[rows], Wgu, I)
-        y = expert_out(h, Wd)
+        h = expert_hidden(xf[rows], Wgu, I, None if Bgu is None else Bgu[e])
+        y = expert_out(h, Wd, None if Bd is None else Bd[e])
         contrib[rows, slots] = r.p[rows, slots][:, None] * y
         if return_hidden:
             hidden[e] = (tok[rows], h)
@@ -321,7 +335,8 @@ def rms_norm(h: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
 
 
 def moe_block(h_bits, g, eps, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, k: int,
-              x_bits: Optional[np.ndarray] = None, tokens: Optional[Iterable[int]] = None):
+              x_bits: Optional[np.ndarray] = None, tokens: Optional[Iterable[int]] = None,
+              Bgu: Optional[np.ndarray] = None, Bd: Optional[np.ndarray] = None):
     """h + FFN(RMSNorm(h)) per token, in fp64: the MoE sublayer with its
     pre-norm and residual add (field guide "gpt-oss 20B", "04 One decoder
     block": each sublayer is added back to the residual stream).
@@ -337,7 +352,8 @@ def moe_block(h_bits, g, eps, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scal
         xb = f64_to_bf16_bits(rms_norm(hf, g, eps))
     else:
         xb = np.asarray(x_bits)[tok]
-    return hf + moe_forward(xb, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, k=k)
+    return hf + moe_forward(xb, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, k=k,
+                            Bgu=Bgu, Bd=Bd)
 
 
 # --------------------------------------------------------------------------

@@ -22,6 +22,7 @@ PIN_TESTS = [
     (P.test_f64_to_bf16_rounding, {}),
     (P.test_rms_norm_closed_forms, {}),
     (P.test_moe_block_residual_and_norm, {}),
+    (P.test_expert_biases_closed_form, {}),
 ]
 
 
@@ -99,8 +100,21 @@ def _mut_round_toward_zero(a):
     return (a.astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
 
 
+def _mut_bias_after_silu(xe, Wgu, I, bias=None):
+    h = _orig_hidden(xe, Wgu, I)
+    if bias is None:
+        return h
+    b = np.asarray(bias, dtype=np.float64)
+    return (O.silu(xe @ Wgu[:I].T) + b[None, :I]) * (xe @ Wgu[I:].T + b[None, I:])
+
+
+def _mut_drop_down_bias(h, Wd, bias=None):
+    return h @ Wd.T
+
+
 _orig_router = O.router_logits
 _orig_block = O.moe_block
+_orig_hidden = O.expert_hidden
 _orig_decode = O.mxfp4_decode
 _orig_e8m0 = O.e8m0_value
 _orig_tables = O.routing_tables
@@ -118,6 +132,8 @@ MUTATIONS = {
     "norm by the sum of squares": ("rms_norm", _mut_norm_sum_not_mean),
     "residual add dropped": ("moe_block", _mut_no_residual),
     "bf16 truncation": ("f64_to_bf16_bits", _mut_round_toward_zero),
+    "gate bias after the silu": ("expert_hidden", _mut_bias_after_silu),
+    "down bias dropped": ("expert_out", _mut_drop_down_bias),
 }
 
 

@@ -436,3 +436,29 @@ def test_moe_block_residual_and_norm():
     ff = O.moe_forward(xb, inp.W_r, inp.b_r, inp.Wgu_codes, inp.Wgu_scales, inp.Wd_codes,
                        inp.Wd_scales, k=k)
     assert np.array_equal(a - hx, ff) or np.allclose(a - hx, ff, rtol=1e-13, atol=1e-13)
+
+
+# ---------------------------------------------------------- expert biases ----
+
+def test_expert_biases_closed_form():
+    """All-zero weights with biases: H = silu(b_gate) b_up and y = b_down + H Wd^T = b_down,
+    so the output is sum_j p_j b_down[e_j]; gate/up biases enter before the silu."""
+    d, I, E, k, T = 64, 96, 3, 2, 5
+    inp = W.make_custom(d, I, E, k, T, seed=21)
+    rng = np.random.default_rng(22)
+    Bgu = rng.standard_normal((E, 2 * I))
+    Bd = rng.standard_normal((E, d))
+    zgu, zd = np.zeros_like(inp.Wgu_codes), np.zeros_like(inp.Wd_codes)
+    out, r, hidden = O.moe_forward(inp.x, inp.W_r, inp.b_r, zgu, inp.Wgu_scales, zd,
+                                   inp.Wd_scales, k=k, return_hidden=True, Bgu=Bgu, Bd=Bd)
+    want = np.einsum("tj,tjd->td", r.p, Bd[r.idx])
+    assert np.allclose(out, want, rtol=1e-13, atol=1e-13)
+    for e, (toks, h) in hidden.items():
+        g, u = Bgu[e, :I], Bgu[e, I:]
+        assert np.allclose(h, np.broadcast_to(g / (1 + np.exp(-g)) * u, h.shape), rtol=1e-13)
+    # with real weights the gate bias shifts the silu argument, not its output
+    full = O.moe_forward(inp.x, inp.W_r, inp.b_r, inp.Wgu_codes, inp.Wgu_scales, inp.Wd_codes,
+                         inp.Wd_scales, k=k, Bgu=Bgu, Bd=np.zeros((E, d)))
+    plain = O.moe_forward(inp.x, inp.W_r, inp.b_r, inp.Wgu_codes, inp.Wgu_scales, inp.Wd_codes,
+                          inp.Wd_scales, k=k)
+    assert not np.allclose(full, plain)
