@@ -139,6 +139,26 @@ MOE_API moe_status moe_forward(const void* x_dev, const float* W_r_dev, const fl
                        void* workspace_dev, size_t workspace_bytes, void* stream);
 
 /*
+ * moe_forward with per-expert projection biases, as a gpt-oss expert carries
+ * them (the parameter totals of "gpt-oss-20b and gpt-oss-120b" count 2I + d
+ * bias values per expert):
+ *   H = silu(x Wgate^T + b_gate) * (x Wup^T + b_up),  y = H Wdown^T + b_down,
+ * and the layer output sum_j p_j y_j as in moe_forward.
+ * gu_bias_dev [E][2I] f32: row e holds expert e's gate biases (0..I-1), then
+ * its up biases (I..2I-1). down_bias_dev [E][d] f32. Either may be NULL (no
+ * bias on that projection; with both NULL this is moe_forward); each given
+ * one is 16-byte aligned device memory, read-only and the caller's. The
+ * biases are added to the fp32 accumulators in the GEMM epilogues (no extra
+ * launches). Errors, workspace and stream semantics are those of moe_forward.
+ */
+MOE_API moe_status moe_forward_biased(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
+                                      const uint8_t* Wgu_codes_dev, const uint8_t* Wgu_scales_dev,
+                                      const float* gu_bias_dev, const uint8_t* Wd_codes_dev,
+                                      const uint8_t* Wd_scales_dev, const float* down_bias_dev,
+                                      int E, int k, int T, int d, int I, void* out_dev,
+                                      void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/*
  * Same as moe_forward, instrumented: records a CUDA event on `stream` before
  * every kernel the pass launches and one after the last, waits for the last
  * event, and writes to stage_ms_host[0..11] (host memory, 12 floats) the
@@ -284,8 +304,9 @@ MOE_API moe_status moe_selftest_wait_timeout(void* workspace_dev, void* stream);
  *   out = bf16(h + sum_j p_j E_j(x))              (one rounding, after the add)
  * h_dev [T][d] bf16 (the residual stream), g_dev [d] f32 (the norm's gain),
  * eps >= 0 (the pages give no value; gpt-oss configurations commonly use
- * 1e-5). All other arguments, the result, the errors and the stream semantics
- * are those of moe_forward; the workspace must hold
+ * 1e-5); gu_bias_dev and down_bias_dev (each may be NULL) are the experts'
+ * biases as in moe_forward_biased. All other arguments, the result, the errors
+ * and the stream semantics are those of moe_forward; the workspace must hold
  * moe_workspace_size_block(...) bytes (moe_forward's, plus the x rows).
  * moe_forward_launch_count(...) + 1 launches.
  */
@@ -293,7 +314,8 @@ MOE_API size_t moe_workspace_size_block(int E, int k, int T, int d, int I);
 MOE_API moe_status moe_forward_block(const void* h_dev, const float* g_dev, float eps,
                                      const float* W_r_dev, const float* b_r_dev,
                                      const uint8_t* Wgu_codes_dev, const uint8_t* Wgu_scales_dev,
-                                     const uint8_t* Wd_codes_dev, const uint8_t* Wd_scales_dev,
+                                     const float* gu_bias_dev, const uint8_t* Wd_codes_dev,
+                                     const uint8_t* Wd_scales_dev, const float* down_bias_dev,
                                      int E, int k, int T, int d, int I, void* out_dev,
                                      void* workspace_dev, size_t workspace_bytes, void* stream);
 

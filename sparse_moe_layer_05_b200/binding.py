@@ -30,7 +30,7 @@ EXPORTS = [
     "moe_route", "moe_workspace_layout", "moe_mxfp4_to_bf16", "moe_mx_split_e4m3", "moe_sync_status",
     "moe_selftest_wait_timeout", "moe_forward_launch_count", "moe_forward_timed",
     "moe_set_tile_policy", "moe_route_noalloc", "moe_probe_tensor_rate",
-    "moe_workspace_size_block", "moe_forward_block", "moe_rms_norm",
+    "moe_workspace_size_block", "moe_forward_block", "moe_rms_norm", "moe_forward_biased",
 ]
 
 STAGES = ["router_logits", "topk_softmax", "perm_hist", "perm_scan", "perm_scatter",
@@ -91,7 +91,11 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_workspace_size_block.restype = sz
     lib.moe_workspace_size_block.argtypes = [i32] * 5
     lib.moe_forward_block.restype = i32
-    lib.moe_forward_block.argtypes = [vp, fp, ctypes.c_float] + fwd[1:]
+    # the biased forms: gate/up bias after the gate/up weights, down bias after the down ones
+    fwd_b = fwd[:5] + [fp] + fwd[5:7] + [fp] + fwd[7:]
+    lib.moe_forward_biased.restype = i32
+    lib.moe_forward_biased.argtypes = fwd_b
+    lib.moe_forward_block.argtypes = [vp, fp, ctypes.c_float] + fwd_b[1:]
     lib.moe_rms_norm.restype = i32
     lib.moe_rms_norm.argtypes = [vp, fp, ctypes.c_float, i32, i32, vp, vp]
     lib.moe_probe_tensor_rate.restype = i32
@@ -172,6 +176,18 @@ def moe_forward(x, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, E, k, T
         _stream(stream)))
 
 
+def moe_forward_biased(x, W_r, b_r, Wgu_codes, Wgu_scales, gu_bias, Wd_codes, Wd_scales, down_bias,
+                       E, k, T, d, I, out, workspace, stream=None) -> None:
+    """moe_forward with per-expert biases: gu_bias f32 [E, 2I] (gate then up),
+    down_bias f32 [E, d]; either may be None."""
+    _require_cuda(x, W_r, b_r, Wgu_codes, Wgu_scales, gu_bias, Wd_codes, Wd_scales, down_bias, out,
+                  workspace)
+    _check("moe_forward_biased", load().moe_forward_biased(
+        _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(Wgu_codes), _ptr(Wgu_scales), _ptr(gu_bias),
+        _ptr(Wd_codes), _ptr(Wd_scales), _ptr(down_bias), E, k, T, d, I, _ptr(out),
+        _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
 def moe_forward_timed(x, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, E, k, T, d, I,
                       out, workspace, stream=None) -> list:
     """Forward pass with per-launch CUDA-event timing; returns len(STAGES)+1
@@ -226,13 +242,15 @@ def moe_rms_norm(h, g, eps: float, T: int, d: int, x, stream=None) -> None:
 
 
 def moe_forward_block(h, g, eps: float, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales,
-                      E: int, k: int, T: int, d: int, I: int, out, workspace, stream=None) -> None:
-    """out = h + MoE(RMSNorm(h)) (bf16 rows; g f32 gain)."""
-    _require_cuda(h, g, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, out, workspace)
+                      E: int, k: int, T: int, d: int, I: int, out, workspace, stream=None,
+                      gu_bias=None, down_bias=None) -> None:
+    """out = h + MoE(RMSNorm(h)) (bf16 rows; g f32 gain; optional expert biases)."""
+    _require_cuda(h, g, W_r, b_r, Wgu_codes, Wgu_scales, gu_bias, Wd_codes, Wd_scales, down_bias,
+                  out, workspace)
     _check("moe_forward_block", load().moe_forward_block(
         _ptr(h), _ptr(g), eps, _ptr(W_r), _ptr(b_r), _ptr(Wgu_codes), _ptr(Wgu_scales),
-        _ptr(Wd_codes), _ptr(Wd_scales), E, k, T, d, I, _ptr(out), _ptr(workspace),
-        workspace.numel(), _stream(stream)))
+        _ptr(gu_bias), _ptr(Wd_codes), _ptr(Wd_scales), _ptr(down_bias), E, k, T, d, I,
+        _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)))
 
 
 def moe_probe_tensor_rate(kind: int, N: int, per_commit: int, stream=None) -> float:

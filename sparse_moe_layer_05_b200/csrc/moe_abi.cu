@@ -259,12 +259,14 @@ moe_status launch_routing(const uint16_t* x, const float* W_r, const float* b_r,
 }
 
 // The forward pass on the caller's stream. resid (optional, [T][d] bf16) is
-// added to the layer output before its rounding to bf16.
+// added to the layer output before its rounding to bf16; gu_bias ([E][2I]) and
+// dn_bias ([E][d]), each optional, are the experts' projection biases.
 moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, const uint8_t* gc,
                        const uint8_t* gs, const uint8_t* dc, const uint8_t* ds, int E, int k,
                        int T, int d, int I, uint16_t* out, void* ws, const Layout& L,
                        cudaStream_t st, int num_sms, const StageEvents* tev = nullptr,
-                       const uint16_t* resid = nullptr) {
+                       const uint16_t* resid = nullptr, const float* gu_bias = nullptr,
+                       const float* dn_bias = nullptr) {
   StageEvents none;
   memset(&none, 0, sizeof(none));
   const StageEvents& E_ = tev ? *tev : none;
@@ -321,6 +323,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     m1.h_sfb = sfbh;
     m1.n_out = I;
     m1.status = status;
+    m1.bias = gu_bias;
     MOE_CUDA(moe::launch_mx_gemm_gateup_swiglu(variant, m1, num_sms, st));
     E_.mark(9);
     moe::MxGemmProblem m2 = m1;
@@ -337,6 +340,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     m2.perm = perm;
     m2.topk_w = topk_w;
     m2.n_out = d;
+    m2.bias = dn_bias;
     MOE_CUDA(moe::launch_mx_gemm_down(variant, m2, num_sms, st));
     E_.mark(10);
     MOE_CUDA(moe::launch_combine(yw, T, k, d, resid, out, st));
@@ -367,6 +371,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   g1.n_out = I;
   g1.status = status;
   g1.tiles = tiles;
+  g1.bias = gu_bias;
   MOE_CUDA(moe::launch_gemm_gateup_swiglu(g1, num_sms, st));
   E_.mark(9);
 
@@ -381,6 +386,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   g2.perm = perm;
   g2.topk_w = topk_w;
   g2.n_out = d;
+  g2.bias = dn_bias;
   MOE_CUDA(moe::launch_gemm_down_combine(g2, num_sms, st));
   E_.mark(10);
   MOE_CUDA(moe::launch_combine(yw, T, k, d, resid, out, st));
@@ -450,10 +456,22 @@ moe_status moe_forward(const void* x_dev, const float* W_r_dev, const float* b_r
                        const uint8_t* Wd_codes_dev, const uint8_t* Wd_scales_dev, int E, int k,
                        int T, int d, int I, void* out_dev, void* workspace_dev,
                        size_t workspace_bytes, void* stream) {
+  return moe_forward_biased(x_dev, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev, nullptr,
+                            Wd_codes_dev, Wd_scales_dev, nullptr, E, k, T, d, I, out_dev,
+                            workspace_dev, workspace_bytes, stream);
+}
+
+moe_status moe_forward_biased(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
+                              const uint8_t* Wgu_codes_dev, const uint8_t* Wgu_scales_dev,
+                              const float* gu_bias_dev, const uint8_t* Wd_codes_dev,
+                              const uint8_t* Wd_scales_dev, const float* down_bias_dev, int E,
+                              int k, int T, int d, int I, void* out_dev, void* workspace_dev,
+                              size_t workspace_bytes, void* stream) {
   moe_status s = check_forward_args(x_dev, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev,
                                     Wd_codes_dev, Wd_scales_dev, E, k, T, d, I, out_dev,
                                     workspace_dev);
   if (s != MOE_OK) return s;
+  if (!aligned16(gu_bias_dev) || !aligned16(down_bias_dev)) return MOE_ERR_INVALID_ARG;
   Layout L;
   make_layout(E, k, T, d, I, false, &L);
   if (workspace_bytes < L.pub.total) return MOE_ERR_WORKSPACE;
@@ -463,7 +481,8 @@ moe_status moe_forward(const void* x_dev, const float* W_r_dev, const float* b_r
   return run_forward(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, Wgu_codes_dev,
                      Wgu_scales_dev, Wd_codes_dev, Wd_scales_dev, E, k, T, d, I,
                      static_cast<uint16_t*>(out_dev), workspace_dev, L,
-                     static_cast<cudaStream_t>(stream), num_sms);
+                     static_cast<cudaStream_t>(stream), num_sms, nullptr, nullptr, gu_bias_dev,
+                     down_bias_dev);
 }
 
 size_t moe_workspace_size_block(int E, int k, int T, int d, int I) {
@@ -489,8 +508,9 @@ moe_status moe_rms_norm(const void* h_dev, const float* g_dev, float eps, int T,
 
 moe_status moe_forward_block(const void* h_dev, const float* g_dev, float eps, const float* W_r_dev,
                              const float* b_r_dev, const uint8_t* Wgu_codes_dev,
-                             const uint8_t* Wgu_scales_dev, const uint8_t* Wd_codes_dev,
-                             const uint8_t* Wd_scales_dev, int E, int k, int T, int d, int I,
+                             const uint8_t* Wgu_scales_dev, const float* gu_bias_dev,
+                             const uint8_t* Wd_codes_dev, const uint8_t* Wd_scales_dev,
+                             const float* down_bias_dev, int E, int k, int T, int d, int I,
                              void* out_dev, void* workspace_dev, size_t workspace_bytes,
                              void* stream) {
   moe_status s = check_forward_args(h_dev, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev,
@@ -498,6 +518,7 @@ moe_status moe_forward_block(const void* h_dev, const float* g_dev, float eps, c
                                     workspace_dev);
   if (s != MOE_OK) return s;
   if (!g_dev || !aligned16(g_dev) || !(eps >= 0.f)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(gu_bias_dev) || !aligned16(down_bias_dev)) return MOE_ERR_INVALID_ARG;
   Layout L;
   make_layout(E, k, T, d, I, false, &L, true);
   if (workspace_bytes < L.pub.total) return MOE_ERR_WORKSPACE;
@@ -510,7 +531,7 @@ moe_status moe_forward_block(const void* h_dev, const float* g_dev, float eps, c
   MOE_CUDA(moe::launch_rms_norm(h, g_dev, eps, T, d, x, st));
   return run_forward(x, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev, Wd_codes_dev,
                      Wd_scales_dev, E, k, T, d, I, static_cast<uint16_t*>(out_dev), workspace_dev,
-                     L, st, num_sms, nullptr, h);
+                     L, st, num_sms, nullptr, h, gu_bias_dev, down_bias_dev);
 }
 
 moe_status moe_forward_hostio(const void* x_host, const float* W_r_dev, const float* b_r_dev,

@@ -91,6 +91,7 @@ struct Args {
   const int32_t* perm;
   const float* topk_w;
   int* status;
+  const float* bias;  // [E][2I] (SwiGLU) or [E][d] (down), or nullptr
 };
 
 struct TileInfo {
@@ -117,6 +118,40 @@ __device__ __forceinline__ void decode_tile(int tile, int n_tiles, int E, const 
 }
 
 __device__ __forceinline__ float silu_f(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
+// Bias of 8 gate columns col.. and the matching up columns (row layout
+// [gate 0..n-1 | up 0..n-1]); zeros without a bias row. n is a multiple of 8
+// and col < n, so both 32-byte reads stay inside the row.
+__device__ __forceinline__ void load_bias8x2(const float* brow, int col, int n, float* bg,
+                                             float* bu) {
+  if (brow && col < n) {
+    const float4* pg = reinterpret_cast<const float4*>(brow + col);
+    const float4* pu = reinterpret_cast<const float4*>(brow + n + col);
+    const float4 g0 = __ldg(pg), g1 = __ldg(pg + 1), u0 = __ldg(pu), u1 = __ldg(pu + 1);
+    bg[0] = g0.x; bg[1] = g0.y; bg[2] = g0.z; bg[3] = g0.w;
+    bg[4] = g1.x; bg[5] = g1.y; bg[6] = g1.z; bg[7] = g1.w;
+    bu[0] = u0.x; bu[1] = u0.y; bu[2] = u0.z; bu[3] = u0.w;
+    bu[4] = u1.x; bu[5] = u1.y; bu[6] = u1.z; bu[7] = u1.w;
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) bg[i] = bu[i] = 0.f;
+  }
+}
+
+// Bias of 16 output columns col.. (col + 16 <= the row length), or zeros.
+__device__ __forceinline__ void load_bias16(const float* brow, int col, float* b) {
+  if (brow) {
+    const float4* p = reinterpret_cast<const float4*>(brow + col);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 v = __ldg(p + i);
+      b[4 * i] = v.x; b[4 * i + 1] = v.y; b[4 * i + 2] = v.z; b[4 * i + 3] = v.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) b[i] = 0.f;
+  }
+}
 
 __device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
   const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
@@ -291,15 +326,19 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
           // columns 0..63 gate, 64..127 up; H stored in kPerm8 chunk order
           const int col0 = ti.nt * NH;
           uint16_t* orow = args.out + grow * args.n_out;
+          const float* brow = args.bias ? args.bias + static_cast<int64_t>(ti.e) * 2 * args.n_out
+                                        : nullptr;
 #pragma unroll 1
           for (int c = 0; c < NH; c += 8) {
             uint32_t g[8], u[8];
             tmem_ld8x2_sync(taddr + c, taddr + NH + c, g, u);
+            const int col = col0 + c;
+            float bg[8], bu[8];
+            load_bias8x2(brow, col, args.n_out, bg, bu);
             float h[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i)
-              h[i] = silu_f(__uint_as_float(g[i])) * __uint_as_float(u[i]);
-            const int col = col0 + c;
+              h[i] = silu_f(__uint_as_float(g[i]) + bg[i]) * (__uint_as_float(u[i]) + bu[i]);
             if (valid && col < args.n_out) {
               *reinterpret_cast<uint4*>(orow + col) =
                   make_uint4(pack_bf16x2(h[0], h[4]), pack_bf16x2(h[1], h[5]),
@@ -316,18 +355,23 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
             w = args.topk_w[pair];
           }
           float* orow = args.out_f32 + static_cast<int64_t>(pair) * args.n_out;
+          const float* brow = args.bias ? args.bias + static_cast<int64_t>(ti.e) * args.n_out
+                                        : nullptr;
 #pragma unroll 1
           for (int c = 0; c < BN; c += 16) {
             uint32_t y[16];
             tmem_ld16_sync(taddr + c, y);
             const int col = col0 + c;
             if (valid && col < args.n_out) {
+              float b[16];
+              load_bias16(brow, col, b);
               float4* dst = reinterpret_cast<float4*>(orow + col);
 #pragma unroll
               for (int i = 0; i < 4; ++i)
-                dst[i] = make_float4(w * __uint_as_float(y[4 * i]), w * __uint_as_float(y[4 * i + 1]),
-                                     w * __uint_as_float(y[4 * i + 2]),
-                                     w * __uint_as_float(y[4 * i + 3]));
+                dst[i] = make_float4(w * (__uint_as_float(y[4 * i]) + b[4 * i]),
+                                     w * (__uint_as_float(y[4 * i + 1]) + b[4 * i + 1]),
+                                     w * (__uint_as_float(y[4 * i + 2]) + b[4 * i + 2]),
+                                     w * (__uint_as_float(y[4 * i + 3]) + b[4 * i + 3]));
             }
           }
         }
@@ -440,7 +484,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::NUM_THREADS, 1
   constexpr int SC = pair::SC;
   constexpr int A_BYTES = pair::A_BYTES;
   constexpr int B_BYTES = pair::B_BYTES;
-  constexpr int C_CODES = pair::C_CODES;
   constexpr int S_ROWS = pair::S_ROWS;
   constexpr int S_OFF = pair::S_OFF;
   constexpr int C_TX = pair::C_TX;
@@ -626,15 +669,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::NUM_THREADS, 1
         // columns 0..119 gate (even CTA's rows), 120..239 up (odd CTA's rows)
         const int col0 = ti.nt * NH;
         uint16_t* orow = args.out + grow * args.n_out;
+        const float* brow = args.bias ? args.bias + static_cast<int64_t>(ti.e) * 2 * args.n_out
+                                      : nullptr;
 #pragma unroll 1
         for (int c = 0; c < NH; c += 8) {
           uint32_t g[8], u[8];
           tmem_ld8x2_sync(taddr + c, taddr + NH + c, g, u);
+          const int col = col0 + c;
+          float bg[8], bu[8];
+          load_bias8x2(brow, col, args.n_out, bg, bu);
           float h[8];
 #pragma unroll
           for (int i = 0; i < 8; ++i)
-            h[i] = silu_f(__uint_as_float(g[i])) * __uint_as_float(u[i]);
-          const int col = col0 + c;
+            h[i] = silu_f(__uint_as_float(g[i]) + bg[i]) * (__uint_as_float(u[i]) + bu[i]);
           if (valid && col < args.n_out) {
             *reinterpret_cast<uint4*>(orow + col) =
                 make_uint4(pack_bf16x2(h[0], h[4]), pack_bf16x2(h[1], h[5]),
@@ -650,18 +697,23 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::NUM_THREADS, 1
           w = args.topk_w[pr];
         }
         float* orow = args.out_f32 + static_cast<int64_t>(pr) * args.n_out;
+        const float* brow = args.bias ? args.bias + static_cast<int64_t>(ti.e) * args.n_out
+                                      : nullptr;
 #pragma unroll 1
         for (int c = 0; c < BN; c += 16) {
           uint32_t y[16];
           tmem_ld16_sync(taddr + c, y);
           const int col = col0 + c;
           if (valid && col < args.n_out) {
+            float b[16];
+            load_bias16(brow, col, b);
             float4* dst = reinterpret_cast<float4*>(orow + col);
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              dst[i] = make_float4(w * __uint_as_float(y[4 * i]), w * __uint_as_float(y[4 * i + 1]),
-                                   w * __uint_as_float(y[4 * i + 2]),
-                                   w * __uint_as_float(y[4 * i + 3]));
+              dst[i] = make_float4(w * (__uint_as_float(y[4 * i]) + b[4 * i]),
+                                   w * (__uint_as_float(y[4 * i + 1]) + b[4 * i + 1]),
+                                   w * (__uint_as_float(y[4 * i + 2]) + b[4 * i + 2]),
+                                   w * (__uint_as_float(y[4 * i + 3]) + b[4 * i + 3]));
           }
         }
       }
@@ -954,6 +1006,17 @@ __global__ void __launch_bounds__(swp::NUM_THREADS, 1)
       if (!mbar_wait(bar_accFull(ab), ap, abort_flag, args.status)) break;
       tc_fence_after();
       const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + ab * NT;
+      // this lane's weight row carries one bias value for the whole tile
+      float bl = 0.f;
+      if (args.bias) {
+        if (EPI == EPI_SWIGLU) {
+          const int jb = wb * NH + (r >> 1);
+          if (jb < args.n_out)
+            bl = args.bias[static_cast<int64_t>(e) * 2 * args.n_out + (r & 1) * args.n_out + jb];
+        } else if (wb * MW + r < args.n_out) {
+          bl = args.bias[static_cast<int64_t>(e) * args.n_out + wb * MW + r];
+        }
+      }
 #pragma unroll 1
       for (int c = 0; c < NT && c < rows; c += 16) {
         uint32_t y[16];
@@ -964,7 +1027,7 @@ __global__ void __launch_bounds__(swp::NUM_THREADS, 1)
           const int col = (j & ~7) + perm8_pos(j & 7);
 #pragma unroll
           for (int i = 0; i < 16; ++i) {
-            const float v = __uint_as_float(y[i]);
+            const float v = __uint_as_float(y[i]) + bl;
             const float u = __shfl_xor_sync(0xFFFFFFFFu, v, 1);
             if (!(lane & 1) && c + i < rows && j < args.n_out) {
               const float h = silu_f(v) * u;
@@ -982,7 +1045,7 @@ __global__ void __launch_bounds__(swp::NUM_THREADS, 1)
               const float w = args.topk_w[pr];
               if (col < args.n_out)
                 args.out_f32[static_cast<int64_t>(pr) * args.n_out + col] =
-                    w * __uint_as_float(y[i]);
+                    w * (__uint_as_float(y[i]) + bl);
             }
           }
         }
@@ -1145,6 +1208,7 @@ cudaError_t launch_swap_impl(const GroupedGemmProblem& p, int num_sms, cudaStrea
   a.out_f32 = p.out_f32;
   a.perm = p.perm;
   a.topk_w = p.topk_w;
+  a.bias = p.bias;
   a.status = p.status;
   if (EPI == EPI_SWIGLU) {
     a.n_tiles = (p.n_out + swp::NH - 1) / swp::NH;   // weight blocks of 64 gate + 64 up rows
@@ -1191,6 +1255,7 @@ cudaError_t launch_pair_impl(const GroupedGemmProblem& p, int num_sms, cudaStrea
   a.out_f32 = p.out_f32;
   a.perm = p.perm;
   a.topk_w = p.topk_w;
+  a.bias = p.bias;
   a.status = p.status;
   if (EPI == EPI_SWIGLU) {
     a.n_tiles = (p.n_out + pair::NH - 1) / pair::NH;
@@ -1237,6 +1302,7 @@ cudaError_t launch_impl(const GroupedGemmProblem& p, int num_sms, cudaStream_t s
   a.out_f32 = p.out_f32;
   a.perm = p.perm;
   a.topk_w = p.topk_w;
+  a.bias = p.bias;
   a.status = p.status;
   if (EPI == EPI_SWIGLU) {
     a.n_tiles = (p.n_out + NH - 1) / NH;

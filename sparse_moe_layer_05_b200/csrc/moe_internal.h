@@ -74,6 +74,10 @@ struct GroupedGemmProblem {
   int n_out;                // output columns (I for SwiGLU, d for down)
   int* status;
   int tiles;                // TILES_SINGLE, TILES_PAIR or TILES_SWAP
+  // optional per-expert bias (nullptr: none), added to the fp32 accumulator:
+  // SwiGLU [E][2I] (gate 0..I-1, up I..2I-1, before the silu); down [E][d]
+  // (before the routing weight)
+  const float* bias;
 };
 
 // Grouped-GEMM tile shapes.
@@ -128,6 +132,7 @@ struct MxGemmProblem {
   const float* topk_w;
   int n_out;                // I for SwiGLU, d for down
   int* status;
+  const float* bias;        // optional, as in GroupedGemmProblem
 };
 cudaError_t launch_mx_gemm_gateup_swiglu(int variant, const MxGemmProblem& p, int num_sms,
                                          cudaStream_t st);

@@ -304,6 +304,7 @@ struct MxArgs {
   const int32_t* perm;
   const float* topk_w;
   int* status;
+  const float* bias;        // [E][2I] (SwiGLU) or [E][d] (down), or nullptr
 };
 
 __device__ __forceinline__ float silu_mx(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
@@ -587,6 +588,16 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
       const int j = wb * 64 + 16 * quad + (lane & 15);      // SwiGLU: H column of this lane
       const bool jv = j < args.I && lane < 16;
       const int col = wb * 128 + m;                          // down: output column
+      // the bias of this lane's weight row (gate or up row j, or output column)
+      float bl = 0.f;
+      if (args.bias) {
+        if (EPI == EPI_SWIGLU) {
+          if (j < args.I)
+            bl = args.bias[static_cast<int64_t>(e) * 2 * args.I + (lane >> 4) * args.I + j];
+        } else if (col < args.n_out) {
+          bl = args.bias[static_cast<int64_t>(e) * args.n_out + col];
+        }
+      }
 #pragma unroll 1
       for (int c = grp * CH; c < NT; c += C::EPI_GROUPS * CH, ++xc) {
         float y[CH];
@@ -611,6 +622,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
           float* xch = s_xch + (grp * 2 + (xc & 1)) * 4 * CH;
 #pragma unroll
           for (int i = 0; i < CH; ++i) {
+            y[i] += bl;
             const float u = __shfl_xor_sync(0xFFFFFFFFu, y[i], 16);
             float hv = 0.f;
             if (ok && jv && c + i < rows)
@@ -663,7 +675,8 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
           for (int i = 0; i < CH; ++i) {
             if (c + i < rows) {
               const int pr = args.perm[p0 + c + i];
-              args.out_f32[static_cast<int64_t>(pr) * args.n_out + col] = args.topk_w[pr] * y[i];
+              args.out_f32[static_cast<int64_t>(pr) * args.n_out + col] =
+                  args.topk_w[pr] * (y[i] + bl);
             }
           }
         }
@@ -808,6 +821,7 @@ cudaError_t launch_mx_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st)
   a.n_out = p.n_out;
   a.perm = p.perm;
   a.topk_w = p.topk_w;
+  a.bias = p.bias;
   a.status = p.status;
   if (EPI == EPI_SWIGLU) {
     a.n_wb = (p.I + 63) / 64;

@@ -201,6 +201,93 @@ def test_forward_both_tile_policies(case, policy):
             assert np.all(np.abs(H[o[e]:o[e + 1]] - h) <= 2.0 ** -8 * np.abs(h) + 1e-3 * rms), e
 
 
+BIAS_CASES = [
+    # name, d, I, E, k, T, seed
+    ("bias_ragged", 352, 224, 8, 2, 1000, 51),
+    ("bias_decode", 2880, 2880, 32, 4, 64, 52),
+    ("bias_mx_tails", 448, 320, 6, 2, 500, 53),
+]
+
+
+def _expert_biases(inp, seed, gu=True, down=True):
+    """Per-expert biases on the scale of the terms they join: the gate/up
+    pre-activations and the expert outputs (RMS estimated from expert 0)."""
+    rng = np.random.default_rng(seed)
+    xf = O.bf16_to_f64(inp.x[:64])
+    pre = xf @ O.mxfp4_decode(inp.Wgu_codes[0], inp.Wgu_scales[0]).T
+    y = O.expert_out(O.expert_hidden(xf, O.mxfp4_decode(inp.Wgu_codes[0], inp.Wgu_scales[0]),
+                                     inp.I), O.mxfp4_decode(inp.Wd_codes[0], inp.Wd_scales[0]))
+    rms = lambda a: float(np.sqrt(np.mean(a ** 2)))
+    Bgu = (rng.standard_normal((inp.E, 2 * inp.I)) * rms(pre)).astype(np.float32) if gu else None
+    Bd = (rng.standard_normal((inp.E, inp.d)) * rms(y)).astype(np.float32) if down else None
+    return Bgu, Bd
+
+
+@pytest.mark.parametrize("policy", [1, 2, 3, 4], ids=["single", "pair", "swap", "mx"])
+@pytest.mark.parametrize("case", BIAS_CASES, ids=[c[0] for c in BIAS_CASES])
+def test_forward_expert_biases(case, policy):
+    """Gate/up biases before the silu and down biases before the routing weight,
+    in every tile family's epilogue; the output must also move away from the
+    unbiased layer by far more than the tolerance."""
+    from sparse_moe_layer_05_b200 import binding as B
+    name, d, I, E, k, T, seed = case
+    inp = W.make_custom(d, I, E, k, T, seed=seed)
+    Bgu, Bd = _expert_biases(inp, seed + 100)
+    layer = B.MoELayer(inp)
+    out = torch.empty((T, d), dtype=torch.uint16, device="cuda")
+    B.moe_set_tile_policy(policy)
+    try:
+        B.moe_forward_biased(_t(inp.x), layer.W_r, layer.b_r, layer.Wgu_codes, layer.Wgu_scales,
+                             _t(Bgu), layer.Wd_codes, layer.Wd_scales, _t(Bd), E, k, T, d, I, out,
+                             layer.workspace)
+        assert B.moe_sync_status(layer.workspace) == 0
+    finally:
+        B.moe_set_tile_policy(0)
+    got = out.cpu().numpy()
+    args = (inp.x, inp.W_r, inp.b_r, inp.Wgu_codes, inp.Wgu_scales, inp.Wd_codes, inp.Wd_scales)
+    want = O.moe_forward(*args, k=k, Bgu=Bgu.astype(np.float64), Bd=Bd.astype(np.float64))
+    G.assert_out_close(got, want)
+    plain = O.moe_forward(*args, k=k)
+    assert G.rel_rms_err(O.bf16_to_f64(got), plain)[0] > 10 * G.TOL_REL_RMS
+
+
+@pytest.mark.parametrize("which", ["gate_up_only", "down_only"])
+def test_forward_one_bias_and_block_with_biases(which):
+    """Either bias alone (the other NULL), through moe_forward_biased and through
+    moe_forward_block (norm, layer with biases, residual)."""
+    from sparse_moe_layer_05_b200 import binding as B
+    d, I, E, k, T = 2880, 2880, 16, 4, 96
+    inp = W.make_custom(d, I, E, k, T, seed=61)
+    Bgu, Bd = _expert_biases(inp, 62, gu=which == "gate_up_only", down=which == "down_only")
+    tb = lambda a: None if a is None else _t(a)
+    f64 = lambda a: None if a is None else a.astype(np.float64)
+    layer = B.MoELayer(inp)
+    out = torch.empty((T, d), dtype=torch.uint16, device="cuda")
+    B.moe_forward_biased(_t(inp.x), layer.W_r, layer.b_r, layer.Wgu_codes, layer.Wgu_scales,
+                         tb(Bgu), layer.Wd_codes, layer.Wd_scales, tb(Bd), E, k, T, d, I, out,
+                         layer.workspace)
+    assert B.moe_sync_status(layer.workspace) == 0
+    args = (inp.W_r, inp.b_r, inp.Wgu_codes, inp.Wgu_scales, inp.Wd_codes, inp.Wd_scales)
+    G.assert_out_close(out.cpu().numpy(), O.moe_forward(inp.x, *args, k=k, Bgu=f64(Bgu),
+                                                        Bd=f64(Bd)))
+    rng = np.random.default_rng(63)
+    h = W.f32_to_bf16_bits((O.bf16_to_f64(inp.x) * 2.0 - 0.25).astype(np.float32))
+    g = rng.uniform(0.5, 1.5, size=d).astype(np.float32)
+    ht, gt = _t(h), torch.from_numpy(g).cuda()
+    xt = torch.empty_like(ht)
+    B.moe_rms_norm(ht, gt, 1e-5, T, d, xt)
+    ws = torch.empty(B.moe_workspace_size_block(E, k, T, d, I), dtype=torch.uint8, device="cuda")
+    B.moe_forward_block(ht, gt, 1e-5, layer.W_r, layer.b_r, layer.Wgu_codes, layer.Wgu_scales,
+                        layer.Wd_codes, layer.Wd_scales, E, k, T, d, I, out, ws,
+                        gu_bias=tb(Bgu), down_bias=tb(Bd))
+    assert B.moe_sync_status(ws) == 0
+    got = O.bf16_to_f64(out.cpu().numpy())
+    want = O.moe_block(h, g, 1e-5, *args, k=k, x_bits=xt.cpu().numpy(), Bgu=f64(Bgu), Bd=f64(Bd))
+    ff = want - O.bf16_to_f64(h)
+    bound = 2e-2 * np.sqrt(np.mean(ff ** 2)) + 2.0 ** -8 * np.abs(want)
+    assert np.all(np.abs(got - want) <= bound), np.max(np.abs(got - want) / bound)
+
+
 def _e4m3_to_f64(b):
     b = b.astype(np.int64)
     e, m = (b >> 3) & 15, b & 7
