@@ -85,12 +85,38 @@ def load_peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
+def strip_c_comments(src: str) -> str:
+    """C/C++ source without its comments and blank lines (string and character
+    literals kept intact), so that a comment edit leaves the hash unchanged."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            while i < n and src[i] != "\n":
+                i += 1
+        elif src.startswith("/*", i):
+            e = src.find("*/", i + 2)
+            i = n if e < 0 else e + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (ln.rstrip() for ln in "".join(out).split("\n"))
+    return "\n".join(ln for ln in lines if ln)
+
+
 def kernel_source_hash(sources=None) -> str:
-    """Hash of the kernel sources a recorded ncu figure depends on."""
+    """Hash of the code (comments stripped) of the kernel sources a recorded
+    ncu figure depends on."""
     h = hashlib.sha256()
     for f in sources or KERNEL_SOURCES:
-        with open(os.path.join(ROOT, "sparse_moe_layer_05_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "sparse_moe_layer_05_b200", "csrc", f), encoding="utf-8") as fh:
+            h.update(strip_c_comments(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
@@ -305,18 +331,36 @@ def run_ours(args, inp, name):
         raise RuntimeError(f"device status {B.STATUS.get(status, status)} in the timed region")
     step_s = sum(s[-1] for s in stage_ms) / 1e3
     block = None
-    if args.block:
+    if args.block or args.bias:
         # the same steps through moe_forward_block (RMSNorm, the layer, the residual
-        # add); the layer's stage times above explain it
-        g = torch.from_numpy(np.random.default_rng(7).uniform(0.5, 1.5, inp.d)
-                             .astype(np.float32)).to(dev)
-        bws = torch.empty(B.moe_workspace_size_block(inp.E, inp.k, T, inp.d, inp.I),
-                          dtype=torch.uint8, device=dev)
+        # add) and/or with per-expert biases (moe_forward_biased); the layer's stage
+        # times above explain them
+        rng = np.random.default_rng(7)
+        gub = dnb = None
+        if args.bias:
+            gub = torch.from_numpy((rng.standard_normal((inp.E, 2 * inp.I)) * 0.1)
+                                   .astype(np.float32)).to(dev)
+            dnb = torch.from_numpy((rng.standard_normal((inp.E, inp.d)) * 0.1)
+                                   .astype(np.float32)).to(dev)
+        if args.block:
+            g = torch.from_numpy(rng.uniform(0.5, 1.5, inp.d).astype(np.float32)).to(dev)
+            bws = torch.empty(B.moe_workspace_size_block(inp.E, inp.k, T, inp.d, inp.I),
+                              dtype=torch.uint8, device=dev)
+
+            def variant_step():
+                B.moe_forward_block(x, g, 1e-5, layer.W_r, layer.b_r, layer.Wgu_codes,
+                                    layer.Wgu_scales, layer.Wd_codes, layer.Wd_scales, inp.E,
+                                    inp.k, T, inp.d, inp.I, out, bws, gu_bias=gub, down_bias=dnb)
+        else:
+            bws = layer.workspace
+
+            def variant_step():
+                B.moe_forward_biased(x, layer.W_r, layer.b_r, layer.Wgu_codes, layer.Wgu_scales,
+                                     gub, layer.Wd_codes, layer.Wd_scales, dnb, inp.E, inp.k, T,
+                                     inp.d, inp.I, out, bws)
         for _ in range(args.warmup):
             flush.zero_()
-            B.moe_forward_block(x, g, 1e-5, layer.W_r, layer.b_r, layer.Wgu_codes,
-                                layer.Wgu_scales, layer.Wd_codes, layer.Wd_scales, inp.E, inp.k,
-                                T, inp.d, inp.I, out, bws)
+            variant_step()
         barrier(world)
         torch.cuda.synchronize()
         bsum = 0.0
@@ -325,16 +369,16 @@ def run_ours(args, inp, name):
             ev0 = torch.cuda.Event(enable_timing=True)
             ev1 = torch.cuda.Event(enable_timing=True)
             ev0.record(stream)
-            B.moe_forward_block(x, g, 1e-5, layer.W_r, layer.b_r, layer.Wgu_codes,
-                                layer.Wgu_scales, layer.Wd_codes, layer.Wd_scales, inp.E, inp.k,
-                                T, inp.d, inp.I, out, bws)
+            variant_step()
             ev1.record(stream)
             ev1.synchronize()
             bsum += ev0.elapsed_time(ev1) / 1e3
         if B.moe_sync_status(bws) != 0:
-            raise RuntimeError("device status after the block steps")
+            raise RuntimeError("device status after the block / biased steps")
+        extra = ("norm_and_residual" if args.block else "bias") + (
+            "_and_bias" if args.block and args.bias else "")
         block = {"layer_ms_per_step": 1e3 * step_s / args.steps,
-                 "norm_and_residual_ms_per_step": 1e3 * (bsum - step_s) / args.steps}
+                 f"{extra}_ms_per_step": 1e3 * (bsum - step_s) / args.steps}
         step_s = bsum
     step_s_max = reduce_max(step_s, world)
     tokens_all = T * args.steps * world
@@ -388,7 +432,9 @@ def run_ours(args, inp, name):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "bf16", "data": "synthetic",
         "config": dict(workload_config(inp, name), tile_policy=args.tile_policy,
-                       **({"block": "out = h + MoE(RMSNorm(h)), eps 1e-5"} if args.block else {})),
+                       **({"block": "out = h + MoE(RMSNorm(h)), eps 1e-5"} if args.block else {}),
+                       **({"expert_biases": "gate/up [E, 2I] and down [E, d], f32"}
+                          if args.bias else {})),
         "layer_tflops": layer_flops(inp.d, inp.I, inp.E, inp.k, T) * args.steps * world
         / step_s_max / 1e12,
         "roofline": dict(roof, kernel=DOMINANT_STAGE, achieved=achieved, peak=peak,
@@ -402,7 +448,7 @@ def run_ours(args, inp, name):
         "clocks": clk.summary(),
     }
     if block:
-        line["block"] = block
+        line["block" if args.block else "bias"] = block
     return line
 
 
@@ -441,6 +487,9 @@ def main(argv=None):
     ap.add_argument("--block", action="store_true",
                     help="time the MoE sublayer with its pre-norm and residual add "
                          "(moe_forward_block: out = h + MoE(RMSNorm(h)))")
+    ap.add_argument("--bias", action="store_true",
+                    help="time the layer with per-expert gate/up and down biases "
+                         "(moe_forward_biased; with --block, the sublayer with biases)")
     ap.add_argument("--probe-tensor", action="store_true",
                     help="print the measured UMMA rates (MAC per SM clock) and exit")
     ap.add_argument("--tile-policy", type=int, default=0, choices=[0, 1, 2, 3, 4],

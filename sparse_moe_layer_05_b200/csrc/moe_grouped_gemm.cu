@@ -2,8 +2,9 @@
 // cores (tcgen05, TMEM accumulators, TMA-fed shared memory).
 //
 //   gate/up:  for the rows r of expert e (permuted order),
-//             H[r, n] = silu(x_r . Wgate[e][n]) * (x_r . Wup[e][n])
-//   down:     Yw[pair(r), m] = p(pair(r)) * (H[r] . Wdown[e][m])
+//             H[r, n] = silu(x_r . Wgate[e][n] + bg[e][n]) * (x_r . Wup[e][n] + bu[e][n])
+//   down:     Yw[pair(r), m] = p(pair(r)) * (H[r] . Wdown[e][m] + bd[e][m])
+// (the biases are optional; without them those terms are zero).
 //
 // Field guide "gpt-oss 20B", "03 Sparse Mixture of Experts" (SwiGLU experts,
 // weighted sum); "shrink/gpt_oss-mic", "Preserved properties" (silu);

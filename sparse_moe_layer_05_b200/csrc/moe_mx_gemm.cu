@@ -4,8 +4,9 @@
 // weight scales are applied by the tensor core, so no CUDA core decodes a
 // weight.
 //
-//   gate/up:  H[r, j] = silu(x_r . Wgate[e][j]) * (x_r . Wup[e][j])
-//   down:     Yw[pair(r), m] = p(pair(r)) * (H[r] . Wdown[e][m])
+//   gate/up:  H[r, j] = silu(x_r . Wgate[e][j] + bg[e][j]) * (x_r . Wup[e][j] + bu[e][j])
+//   down:     Yw[pair(r), m] = p(pair(r)) * (H[r] . Wdown[e][m] + bd[e][m])
+// (the biases are optional; without them those terms are zero).
 //
 // Field guide "gpt-oss 20B", "03 Sparse Mixture of Experts" (SwiGLU experts,
 // weighted sum); "gpt-oss-20b and gpt-oss-120b", "Four-bit expert weights"

@@ -16,6 +16,10 @@ Workloads follow the shapes the pages give:
   "llm-surgery-dark-arts-gpt-oss-40b-64a8-init", section 2 "Silent Init".
 * ``96a12``    -- silent-init x3 expansion of ``20b`` (96 experts, top-12),
   the same page's 96a12 variant (copies at e+32 and e+64).
+* ``64a4``, ``96a4`` -- the same two layers with the active count reduced to
+  4 (the page's "64a8 to 64a4, 96a12 to 96a4"); the page reaches it by router
+  bias adjustment after training, which is not specified, so at silent init
+  these are the expanded layers run at k = 4.
 * ``128a4``    -- gpt-oss-120b routing (128 experts, top-4), "gpt-oss-20b and
   gpt-oss-120b" overview; with 8 router biases raised by 2.0 (skewed load).
 * ``248a20``   -- "gpt-oss-220a20b" model card: 128 base + 120 added expert
@@ -79,6 +83,10 @@ SHAPES: Dict[str, Shape] = {
                   "silent-init x2 expansion of 20b (copies at e+32)"),
     "96a12": Shape("96a12", 2880, 2880, 96, 12, 8192, 64, 119, 123,
                    "silent-init x3 expansion of 20b (copies at e+32, e+64)"),
+    "64a4": Shape("64a4", 2880, 2880, 64, 4, 8192, 64, 119, 123,
+                  "64a8 layer run with the active count reduced to 4"),
+    "96a4": Shape("96a4", 2880, 2880, 96, 4, 8192, 64, 119, 123,
+                  "96a12 layer run with the active count reduced to 4"),
     "128a4": Shape("128a4", 2880, 2880, 128, 4, 16384, 32, 119, 123,
                    "gpt-oss-120b routing with +2.0 bias on experts 0..7"),
     "248a20": Shape("248a20", 2880, 2880, 248, 20, 4096, 16, 119, 123,
@@ -196,9 +204,10 @@ def make_inputs(name: str, T: Optional[int] = None, seed: int = 0) -> MoEInputs:
         return make_custom(s.d, s.I, s.E, s.k, T, seed=seed,
                            scale_lo=s.scale_lo, scale_hi=s.scale_hi,
                            name=name, T_draw=T_full)
-    if name in ("64a8", "96a12"):
+    if name in ("64a8", "96a12", "64a4", "96a4"):
         base = make_inputs("20b", T=T, seed=seed)
-        out = _expand_silent(base, 2 if name == "64a8" else 3)
+        out = _expand_silent(base, 2 if name.startswith("64") else 3)
+        out.k = s.k
         out.name = name
         return out
     if name == "128a4":

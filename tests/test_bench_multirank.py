@@ -83,3 +83,15 @@ def test_bench_rejects_multi_gpu_without_launcher():
                          timeout=300)
     assert out.returncode != 0
     assert "torch.distributed.run" in out.stderr
+
+
+def test_traffic_hash_ignores_comments_only():
+    """A recorded ncu traffic figure stays valid across comment edits of the
+    kernel sources and is dropped by any code edit."""
+    sys.path.insert(0, ROOT)
+    import bench
+    src = 'int a = 1; // one\n/* block\n comment */ const char* s = "x//y /*z*/";\n\nint b;\n'
+    assert bench.strip_c_comments(src) == 'int a = 1;\n const char* s = "x//y /*z*/";\nint b;'
+    assert bench.strip_c_comments(src.replace("// one", "// two")) == bench.strip_c_comments(src)
+    assert bench.strip_c_comments(src.replace("b;", "c;")) != bench.strip_c_comments(src)
+    assert bench.strip_c_comments("char q = '\"'; // x") == "char q = '\"';"

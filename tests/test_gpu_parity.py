@@ -431,6 +431,24 @@ def test_silent_init_identity_on_gpu():
             G.assert_out_close(o8, want, what=f"{name} vs 20b at T={T}")
 
 
+def test_reduced_active_count_on_gpu():
+    """64a4 (the x2 layer at k = 4) reproduces the 20b layer at k = 2; 96a4 (the x3
+    layer at k = 4: three copies of the best expert, one of the second) matches the
+    oracle on sampled tokens. T = 64 (block-scaled tiles) and 512 (bf16 tiles)."""
+    for T in (64, 512):
+        base = W.make_inputs("20b", T=T)
+        base.k = 2
+        o2, _ = G.run_forward(base)
+        o4, _ = G.run_forward(W.make_inputs("64a4", T=T))
+        G.assert_out_close(o4, O.bf16_to_f64(o2), what=f"64a4 vs 20b at k=2, T={T}")
+        inp = W.make_inputs("96a4", T=T)
+        o3, _ = G.run_forward(inp)
+        toks = np.sort(np.random.default_rng(T).choice(T, size=12, replace=False))
+        want = O.moe_forward(inp.x, inp.W_r, inp.b_r, inp.Wgu_codes, inp.Wgu_scales,
+                             inp.Wd_codes, inp.Wd_scales, k=4, tokens=toks)
+        G.assert_out_close(o3[toks], want, what=f"96a4 T={T} sampled")
+
+
 def test_timeout_path_reports_status_and_device_survives():
     from sparse_moe_layer_05_b200 import binding as B
     ws = torch.zeros(256, dtype=torch.uint8, device="cuda")

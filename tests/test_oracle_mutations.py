@@ -23,6 +23,7 @@ PIN_TESTS = [
     (P.test_rms_norm_closed_forms, {}),
     (P.test_moe_block_residual_and_norm, {}),
     (P.test_expert_biases_closed_form, {}),
+    (P.test_silent_init_reduced_active_count, {"M": 3, "k2": 4}),
 ]
 
 

@@ -322,6 +322,35 @@ def test_silent_init_identity(M):
         assert all(sum(1 for e in r.idx[t] if e % base.E == o) == M for o in ra.idx[t])
 
 
+@pytest.mark.parametrize("M,k2", [(2, 4), (3, 4), (2, 3), (3, 5)])
+def test_silent_init_reduced_active_count(M, k2):
+    """An x M silent-init layer run at k' = q M + r (r < M) routes each token to all
+    M copies of its q best original experts and to r copies of the next one (the
+    copies tie exactly), so with c_o = M or r its output is
+    sum_o c_o e^{s_o} E_o(x) / sum_o c_o e^{s_o} over those originals. The page's
+    "64a8 to 64a4, 96a12 to 96a4" is k' = 4 with M = 2 (the original layer at k = 2)
+    and M = 3 (three copies of the best expert, one of the second)."""
+    base = W.make_custom(64, 128, 6, 2, 40, seed=17, scale_lo=121, scale_hi=124)
+    exp = W.expand_silent(base, M)
+    got = O.moe_forward(exp.x, exp.W_r, exp.b_r, exp.Wgu_codes, exp.Wgu_scales, exp.Wd_codes,
+                        exp.Wd_scales, k=k2)
+    xf = O.bf16_to_f64(base.x)
+    s = xf @ base.W_r.astype(np.float64).T + base.b_r.astype(np.float64)
+    outs = np.stack([O.expert_out(O.expert_hidden(xf, O.mxfp4_decode(base.Wgu_codes[e],
+                                                                      base.Wgu_scales[e]), 128),
+                                  O.mxfp4_decode(base.Wd_codes[e], base.Wd_scales[e]))
+                     for e in range(base.E)], axis=1)             # [T, E, d]
+    q, r = divmod(k2, M)
+    want = np.zeros_like(got)
+    for t in range(base.T):
+        order = np.argsort(-s[t], kind="stable")
+        c = [M] * q + ([r] if r else [])
+        chosen = order[:len(c)]
+        w = np.array(c) * np.exp(s[t, chosen] - s[t, chosen].max())
+        want[t] = (w / w.sum()) @ outs[t, chosen]
+    assert np.max(np.abs(got - want)) <= 1e-12 * np.sqrt(np.mean(want ** 2))
+
+
 def test_fixture_workload_recipe():
     inp = W.make_inputs("fixture")
     assert (inp.d, inp.I, inp.E, inp.k, inp.T) == (64, 128, 4, 2, 256)
