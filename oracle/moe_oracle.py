@@ -24,7 +24,9 @@ matmul as the only library primitive. Sources (page title, section):
 Readings where the pages are silent (each also listed in the design notes):
 
 * ties in top-k go to the lower expert index;
-* SwiGLU is silu(gate) * up with no clamp, no extra constants, no bias;
+* SwiGLU is silu(gate) * up with no clamp and no extra constants; per-expert
+  gate/up and down biases are optional (the pages' parameter totals count
+  them; their formulas omit them);
 * gate and up rows are stacked [gate; up] in one packed tensor;
 * MX groups run along the contraction dimension, 32 elements per E8M0 scale
   (bias 127, 0xFF is NaN); byte b holds element 2b in its low nibble;
@@ -32,6 +34,11 @@ Readings where the pages are silent (each also listed in the design notes):
   subnormal at exponent 0 (OCP Microscaling definition);
 * RMSNorm is g * h / sqrt(mean(h^2) + eps) with a caller-chosen eps, and its
   output enters the layer rounded to bf16; the residual add is unrounded.
+
+The activation-quantised modes (``mx_quantize``, ``act_quant`` of
+``moe_forward``) are not the pages' method: they simulate what rounding the
+expert inputs to MXFP8 (E4M3) or MXFP4 (E2M1) blocks would cost, following the
+conversion of the OCP Microscaling Formats specification (v1.0, section 6.3).
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (closed forms, brute force, the silent-init identity, and the pages' printed
@@ -265,12 +272,16 @@ def route(x_bits: np.ndarray, W_r: np.ndarray, b_r: np.ndarray, k: int) -> Routi
 def moe_forward(x_bits, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales,
                 k: int, tokens: Optional[Iterable[int]] = None,
                 return_hidden: bool = False, Bgu: Optional[np.ndarray] = None,
-                Bd: Optional[np.ndarray] = None):
+                Bd: Optional[np.ndarray] = None, act_quant: Optional[str] = None):
     """FFN(h) = sum_{i in top-k(s)} p_i(h) E_i(h) for each token, in fp64.
 
     ``Bgu`` [E, 2I] and ``Bd`` [E, d] (optional) are per-expert biases of the
     gate/up and down projections (the parameter totals of "gpt-oss-20b and
     gpt-oss-120b" and the fixture page count them).
+
+    ``act_quant`` ("e4m3" or "e2m1", default None) simulates an activation-
+    quantised mode: each expert's input rows and its H rows pass through
+    ``mx_quantize`` (groups of 32 along the contraction) before the matmuls.
 
     ``tokens`` restricts the computation to a subset of rows (each token's
     output depends on that token alone). Returns out [T', d] float64, and with
@@ -294,8 +305,10 @@ def moe_forward(x_bits, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales,
             continue
         Wgu = mxfp4_decode(Wgu_codes[e], Wgu_scales[e])
         Wd = mxfp4_decode(Wd_codes[e], Wd_scales[e])
-        h = expert_hidden(xf[rows], Wgu, I, None if Bgu is None else Bgu[e])
-        y = expert_out(h, Wd, None if Bd is None else Bd[e])
+        xe = xf[rows] if act_quant is None else mx_quantize(xf[rows], act_quant)
+        h = expert_hidden(xe, Wgu, I, None if Bgu is None else Bgu[e])
+        he = h if act_quant is None else mx_quantize(h, act_quant)
+        y = expert_out(he, Wd, None if Bd is None else Bd[e])
         contrib[rows, slots] = r.p[rows, slots][:, None] * y
         if return_hidden:
             hidden[e] = (tok[rows], h)
@@ -354,6 +367,55 @@ def moe_block(h_bits, g, eps, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scal
         xb = np.asarray(x_bits)[tok]
     return hf + moe_forward(xb, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, k=k,
                             Bgu=Bgu, Bd=Bd)
+
+
+# --------------------------------------------------------------------------
+# Activation quantisation (a simulated mode, not the pages' method)
+# --------------------------------------------------------------------------
+
+# element formats: (exponent bits, mantissa bits, exponent bias, largest normal,
+# emax = exponent of the largest normal)
+MX_ELEMENTS = {
+    "e4m3": (4, 3, 7, 448.0, 8),   # OCP FP8 E4M3 (no infinities; S.1111.111 is NaN)
+    "e2m1": (2, 1, 1, 6.0, 2),     # OCP FP4 E2M1
+}
+
+
+def minifloat_round(v: np.ndarray, ebits: int, mbits: int, bias: int,
+                    max_normal: float) -> np.ndarray:
+    """Round v to the nearest value of a sign/exponent/mantissa format with
+    subnormals (ties to the even mantissa), clamping magnitudes above the
+    largest normal to it. fp64 in and out."""
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    emin = 1 - bias
+    with np.errstate(divide="ignore"):
+        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    e = np.maximum(e, emin)
+    quantum = np.exp2(e - mbits)
+    r = np.round(a / quantum) * quantum          # numpy rounds halves to even
+    r = np.minimum(r, max_normal)
+    return np.copysign(np.where(a > 0, r, 0.0), v)
+
+
+def mx_quantize(x: np.ndarray, elem: str, group: int = 32) -> np.ndarray:
+    """One MX block conversion along the last axis, returned dequantised.
+
+    Per group of ``group`` values: shared scale X = 2^(floor(log2 max|x|) - emax)
+    (a power of two, as an E8M0 byte holds), elements = minifloat_round(x / X);
+    the result is X * element. An all-zero group stays zero.
+    """
+    ebits, mbits, bias, max_normal, emax = MX_ELEMENTS[elem]
+    x = np.asarray(x, dtype=np.float64)
+    K = x.shape[-1]
+    if K % group:
+        raise ValueError("the last axis must hold whole groups")
+    g = x.reshape(*x.shape[:-1], K // group, group)
+    amax = np.abs(g).max(axis=-1, keepdims=True)
+    with np.errstate(divide="ignore"):
+        X = np.exp2(np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - emax)
+    q = minifloat_round(g / X, ebits, mbits, bias, max_normal) * X
+    return np.where(amax > 0, q, 0.0).reshape(x.shape)
 
 
 # --------------------------------------------------------------------------

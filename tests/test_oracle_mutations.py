@@ -24,6 +24,10 @@ PIN_TESTS = [
     (P.test_moe_block_residual_and_norm, {}),
     (P.test_expert_biases_closed_form, {}),
     (P.test_silent_init_reduced_active_count, {"M": 3, "k2": 4}),
+    (P.test_minifloat_round_on_its_grid, {"fmt": "e4m3", "ebits": 4, "mbits": 3, "bias": 7,
+                                          "ncodes": 127}),
+    (P.test_mx_quantize_shared_scale, {"fmt": "e4m3", "emax": 8}),
+    (P.test_act_quant_applies_to_expert_inputs_and_hidden_rows, {"fmt": "e4m3"}),
 ]
 
 
@@ -113,6 +117,30 @@ def _mut_drop_down_bias(h, Wd, bias=None):
     return h @ Wd.T
 
 
+def _mut_round_half_up(v, ebits, mbits, bias, max_normal):
+    v = np.asarray(v, dtype=np.float64)
+    a = np.abs(v)
+    e = np.maximum(np.floor(np.log2(np.where(a > 0, a, 1.0))), 1 - bias)
+    q = np.exp2(e - mbits)
+    r = np.minimum(np.floor(a / q + 0.5) * q, max_normal)
+    return np.copysign(np.where(a > 0, r, 0.0), v)
+
+
+def _mut_scale_from_ceil(x, elem, group=32):
+    # shared scale from ceil(log2 max|x|): one binade too coarse for most groups
+    x = np.asarray(x, dtype=np.float64)
+    g = x.reshape(*x.shape[:-1], x.shape[-1] // group, group)
+    amax = np.abs(g).max(axis=-1, keepdims=True)
+    ebits, mbits, bias, mx, emax = O.MX_ELEMENTS[elem]
+    X = np.exp2(np.ceil(np.log2(np.where(amax > 0, amax, 1.0))) - emax)
+    return (O.minifloat_round(g / X, ebits, mbits, bias, mx) * X).reshape(x.shape)
+
+
+def _mut_act_quant_ignored(*args, act_quant=None, **kw):
+    return _orig_forward(*args, **kw)
+
+
+_orig_forward = O.moe_forward
 _orig_router = O.router_logits
 _orig_block = O.moe_block
 _orig_hidden = O.expert_hidden
@@ -135,6 +163,9 @@ MUTATIONS = {
     "bf16 truncation": ("f64_to_bf16_bits", _mut_round_toward_zero),
     "gate bias after the silu": ("expert_hidden", _mut_bias_after_silu),
     "down bias dropped": ("expert_out", _mut_drop_down_bias),
+    "minifloat ties rounded up": ("minifloat_round", _mut_round_half_up),
+    "MX scale from the ceiling": ("mx_quantize", _mut_scale_from_ceil),
+    "activation quantisation ignored": ("moe_forward", _mut_act_quant_ignored),
 }
 
 

@@ -491,3 +491,83 @@ def test_expert_biases_closed_form():
     plain = O.moe_forward(inp.x, inp.W_r, inp.b_r, inp.Wgu_codes, inp.Wgu_scales, inp.Wd_codes,
                           inp.Wd_scales, k=k)
     assert not np.allclose(full, plain)
+
+
+# ------------------------------------- simulated activation quantisation ----
+
+@pytest.mark.parametrize("fmt,ebits,mbits,bias,ncodes", [("e4m3", 4, 3, 7, 127),
+                                                        ("e2m1", 2, 1, 1, 8)])
+def test_minifloat_round_on_its_grid(fmt, ebits, mbits, bias, ncodes):
+    """Every finite non-negative code (textbook decoding; E4M3's code 127 is NaN) is a
+    fixed point; a midpoint between neighbours goes to the even code (even mantissa);
+    a quarter of the way goes to the nearer one; magnitudes above the largest normal
+    clamp to it; signs are symmetric."""
+    max_normal = O.MX_ELEMENTS[fmt][3]
+    codes = np.arange(ncodes)
+    grid = np.array([_generic_minifloat(int(c), ebits, mbits, bias) for c in codes])
+    assert np.all(np.diff(grid) > 0) and grid[-1] == max_normal
+
+    def r(v):
+        return O.minifloat_round(np.asarray(v, dtype=np.float64), ebits, mbits, bias, max_normal)
+
+    assert np.array_equal(r(grid), grid) and np.array_equal(r(-grid), -grid)
+    lo, hi = grid[:-1], grid[1:]
+    assert np.array_equal(r((lo + hi) / 2), np.where(codes[:-1] % 2 == 0, lo, hi))
+    assert np.array_equal(r(lo + (hi - lo) / 4), lo)
+    assert np.array_equal(r(hi - (hi - lo) / 4), hi)
+    assert np.array_equal(r([max_normal * 1.01, max_normal * 1e6, -max_normal * 3]),
+                          [max_normal, max_normal, -max_normal])
+
+
+@pytest.mark.parametrize("fmt,emax", [("e4m3", 8), ("e2m1", 2)])
+def test_mx_quantize_shared_scale(fmt, emax):
+    """Shared scale 2^(floor(log2 max|x|) - emax) per group of 32: grid values times
+    that scale pass exactly; the group max lands in [2^emax, 2^(emax+1)) before
+    rounding (so 1.9 clamps to max_normal * 2^-emax); all-zero groups stay zero;
+    groups are independent; scaling by 2^m commutes."""
+    ebits, mbits, bias, max_normal, _ = O.MX_ELEMENTS[fmt]
+    rng = np.random.default_rng(11)
+    grid = np.array([_generic_minifloat(c, ebits, mbits, bias) for c in range(1 << (ebits + mbits))
+                     if _generic_minifloat(c, ebits, mbits, bias) <= max_normal])
+    x = rng.choice(grid, size=(3, 64)) * rng.choice([-1.0, 1.0], size=(3, 64))
+    x[:, 0] = 2.0 ** emax                              # group max = 2^emax: scale 1
+    x[:, 32] = 2.0 ** emax
+    for m in (-20, 0, 9):
+        xs = x * 2.0 ** m
+        assert np.array_equal(O.mx_quantize(xs, fmt), xs)
+    g = np.zeros((1, 32))
+    g[0, 0], g[0, 1] = 1.9, 1.0
+    q = O.mx_quantize(g, fmt)
+    assert q[0, 0] == max_normal * 2.0 ** -emax and q[0, 1] == 1.0
+    assert np.array_equal(O.mx_quantize(np.zeros((2, 32)), fmt), np.zeros((2, 32)))
+    y = rng.standard_normal((4, 96))
+    qy = O.mx_quantize(y, fmt)
+    y2 = y.copy()
+    y2[:, 64:] *= 1000.0
+    assert np.array_equal(O.mx_quantize(y2, fmt)[:, :64], qy[:, :64])
+    assert np.array_equal(O.mx_quantize(y * 2.0 ** 7, fmt), qy * 2.0 ** 7)
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e2m1"])
+def test_act_quant_applies_to_expert_inputs_and_hidden_rows(fmt):
+    """All-ones expert, constant input rows: the quantised input is a constant c_q,
+    H is the constant a = silu(d c_q) d c_q, its quantised value a_q follows from the
+    shared-scale rule on one binade, and out = I a_q."""
+    d, I = 64, 96
+    ebits, mbits, bias, max_normal, emax = O.MX_ELEMENTS[fmt]
+
+    def q_const(v):          # MX quantisation of a group whose 32 values all equal v > 0
+        X = 2.0 ** (math.floor(math.log2(v)) - emax)
+        step = 2.0 ** (emax - mbits)  # element spacing on the binade [2^emax, 2^(emax+1))
+        return X * min(step * round(v / X / step), max_normal)
+
+    x = _bf16(np.array([np.full(d, 0.05), np.full(d, 0.0071)]))
+    gu, gus, dc, ds = _const_layer(1, d, I, 2, 2, 2)            # every weight = 1.0
+    args = (x, np.zeros((1, d), np.float32), np.zeros(1, np.float32), gu, gus, dc, ds)
+    out = O.moe_forward(*args, k=1, act_quant=fmt)
+    for t, c in enumerate(O.bf16_to_f64(x)[:, 0]):
+        s = d * q_const(c)
+        a = s / (1 + math.exp(-s)) * s
+        assert np.allclose(out[t], I * q_const(a), rtol=1e-13, atol=0)
+    exact = O.moe_forward(*args, k=1)
+    assert not np.allclose(out, exact, rtol=1e-4)
