@@ -133,6 +133,58 @@ def recorded_traffic(workload: str, T: int):
     return ent.get("bytes_per_launch")
 
 
+def parse_cpulist(text: str) -> set:
+    """CPU ids of a sysfs cpulist such as "0-3,8,10-11"."""
+    cpus = set()
+    for part in text.strip().split(","):
+        if not part:
+            continue
+        lo, _, hi = part.partition("-")
+        cpus.update(range(int(lo), int(hi or lo) + 1))
+    return cpus
+
+
+def gpu_local_cpus(dev_index: int):
+    """The CPUs of the NUMA node the GPU hangs off (its PCI device's
+    local_cpulist) that this process may run on, or None if unknown."""
+    import torch
+    try:
+        p = torch.cuda.get_device_properties(dev_index)
+        bdf = f"{p.pci_domain_id:04x}:{p.pci_bus_id:02x}:{p.pci_device_id:02x}.0"
+        with open(f"/sys/bus/pci/devices/{bdf}/local_cpulist") as f:
+            cpus = parse_cpulist(f.read()) & os.sched_getaffinity(0)
+    except (OSError, AttributeError, ValueError):
+        return None
+    return cpus or None
+
+
+class NearGpuHostMemory:
+    """Run the enclosed host allocations on the GPU's NUMA node, so that
+    pinned buffers (placed where first touched) do not cross the socket link
+    on every copy; the process's CPU affinity is restored on exit."""
+
+    def __init__(self, dev_index: int):
+        self.cpus = gpu_local_cpus(dev_index)
+        self.saved = None
+
+    def __enter__(self):
+        if self.cpus:
+            self.saved = os.sched_getaffinity(0)
+            os.sched_setaffinity(0, self.cpus)
+        return self
+
+    def __exit__(self, *exc):
+        if self.saved is not None:
+            os.sched_setaffinity(0, self.saved)
+        return False
+
+    def describe(self) -> str:
+        if not self.cpus:
+            return "pinned (GPU's NUMA node unknown)"
+        c = sorted(self.cpus)
+        return f"pinned, first touched on the GPU's NUMA node ({len(c)} CPUs, {c[0]}..{c[-1]})"
+
+
 def layer_flops(d, I, E, k, T) -> float:
     return 6.0 * d * I * T * k + 2.0 * d * E * T
 
@@ -298,12 +350,15 @@ def run_ours(args, inp, name):
     dev = torch.device("cuda", local)
     T = inp.T
     order = rank_token_order(T, rank)
-    x_host = torch.from_numpy(np.ascontiguousarray(inp.x[order])).pin_memory()
+    near = NearGpuHostMemory(local)
+    with near:
+        x_host = torch.from_numpy(np.ascontiguousarray(inp.x[order])).pin_memory()
+        out_host = torch.empty((T, inp.d), dtype=torch.uint16).pin_memory()
+        out_host.zero_()
     x = x_host.to(dev)
     B.moe_set_tile_policy(args.tile_policy)
     layer = B.MoELayer(inp, device=dev, hostio=True)
     out = torch.empty((T, inp.d), dtype=torch.uint16, device=dev)
-    out_host = torch.empty((T, inp.d), dtype=torch.uint16).pin_memory()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
@@ -358,27 +413,36 @@ def run_ours(args, inp, name):
                 B.moe_forward_biased(x, layer.W_r, layer.b_r, layer.Wgu_codes, layer.Wgu_scales,
                                      gub, layer.Wd_codes, layer.Wd_scales, dnb, inp.E, inp.k, T,
                                      inp.d, inp.I, out, bws)
-        for _ in range(args.warmup):
-            flush.zero_()
-            variant_step()
-        barrier(world)
-        torch.cuda.synchronize()
-        bsum = 0.0
-        for _ in range(args.steps):
+        def plain_step():
+            layer.forward(x, out)
+
+        def timed(fn) -> float:
             flush.zero_()
             ev0 = torch.cuda.Event(enable_timing=True)
             ev1 = torch.cuda.Event(enable_timing=True)
             ev0.record(stream)
-            variant_step()
+            fn()
             ev1.record(stream)
             ev1.synchronize()
-            bsum += ev0.elapsed_time(ev1) / 1e3
-        if B.moe_sync_status(bws) != 0:
+            return ev0.elapsed_time(ev1) / 1e3
+
+        for _ in range(args.warmup):
+            timed(variant_step)
+            timed(plain_step)
+        barrier(world)
+        torch.cuda.synchronize()
+        # the plain layer timed the same way (two events, no per-stage events),
+        # alternating with the variant so that both see the same conditions
+        bsum = psum = 0.0
+        for _ in range(args.steps):
+            bsum += timed(variant_step)
+            psum += timed(plain_step)
+        if B.moe_sync_status(bws) != 0 or B.moe_sync_status(layer.workspace) != 0:
             raise RuntimeError("device status after the block / biased steps")
         extra = ("norm_and_residual" if args.block else "bias") + (
             "_and_bias" if args.block and args.bias else "")
-        block = {"layer_ms_per_step": 1e3 * step_s / args.steps,
-                 f"{extra}_ms_per_step": 1e3 * (bsum - step_s) / args.steps}
+        block = {"layer_ms_per_step": 1e3 * psum / args.steps,
+                 f"{extra}_ms_per_step": 1e3 * (bsum - psum) / args.steps}
         step_s = bsum
     step_s_max = reduce_max(step_s, world)
     tokens_all = T * args.steps * world
@@ -442,7 +506,7 @@ def run_ours(args, inp, name):
                          avg_launch_ms=dom_ms, touched_experts=touched),
         "stage_ms": stage_avg,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(T * inp.d * 2),
-                "d2h_bytes_per_step": int(T * inp.d * 2)},
+                "d2h_bytes_per_step": int(T * inp.d * 2), "host_buffers": near.describe()},
         "gpu_launches": (B.moe_forward_launch_count(inp.E, inp.k, T, inp.d, inp.I)
                          + (1 if args.block else 0)) * args.steps,
         "clocks": clk.summary(),

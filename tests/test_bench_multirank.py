@@ -95,3 +95,22 @@ def test_traffic_hash_ignores_comments_only():
     assert bench.strip_c_comments(src.replace("// one", "// two")) == bench.strip_c_comments(src)
     assert bench.strip_c_comments(src.replace("b;", "c;")) != bench.strip_c_comments(src)
     assert bench.strip_c_comments("char q = '\"'; // x") == "char q = '\"';"
+
+
+def test_cpulist_parsing_and_affinity_restore():
+    """sysfs cpulists ("0-3,8,10-11"); the near-GPU allocation scope restores the
+    process's CPU affinity, and does nothing when the GPU's node is unknown."""
+    sys.path.insert(0, ROOT)
+    import bench
+    assert bench.parse_cpulist("0-3,8,10-11\n") == {0, 1, 2, 3, 8, 10, 11}
+    assert bench.parse_cpulist("5") == {5}
+    before = os.sched_getaffinity(0)
+    near = bench.NearGpuHostMemory.__new__(bench.NearGpuHostMemory)
+    near.cpus, near.saved = {min(before)}, None
+    with near:
+        assert os.sched_getaffinity(0) == {min(before)}
+    assert os.sched_getaffinity(0) == before
+    near.cpus, near.saved = None, None
+    with near:
+        assert os.sched_getaffinity(0) == before
+    assert "unknown" in near.describe()
