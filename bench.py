@@ -37,6 +37,9 @@ UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 DOMINANT_STAGE = "gemm_gateup_swiglu"
+# launch boundaries recorded in the timed steps: the pass's start and end and
+# the two around the dominant kernel (each recorded event delays the next
+# launch by a few microseconds, so the per-stage breakdown is taken separately)
 TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
 KERNEL_SOURCES = ["moe_grouped_gemm.cu", "moe_ptx.cuh", "moe_abi.cu"]
 
@@ -362,9 +365,12 @@ def run_ours(args, inp, name):
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream()
 
+    dom = B.STAGES.index(DOMINANT_STAGE)
+    nb = len(B.STAGES)
+    timed_mask = (1 << 0) | (1 << dom) | (1 << (dom + 1)) | (1 << nb)
     for _ in range(args.warmup):
         flush.zero_()
-        layer.forward_timed(x, out)
+        layer.forward_timed_events(x, out, timed_mask)
     torch.cuda.synchronize()
     status = B.moe_sync_status(layer.workspace)
     if status != 0:
@@ -372,19 +378,26 @@ def run_ours(args, inp, name):
 
     clocks_path = os.path.join(ROOT, "gpurun_out", "bench_clocks.csv") if os.path.isdir(
         os.path.join(ROOT, "gpurun_out")) else None
-    stage_ms = []
+    step_ms = []
     barrier(world)
     torch.cuda.synchronize()
     with ClockSampler(local, clocks_path) as clk:
         for _ in range(args.steps):
             flush.zero_()
-            stage_ms.append(layer.forward_timed(x, out))
+            step_ms.append(layer.forward_timed_events(x, out, timed_mask))
         torch.cuda.synchronize()
     barrier(world)
     status = B.moe_sync_status(layer.workspace)
     if status != 0:
         raise RuntimeError(f"device status {B.STATUS.get(status, status)} in the timed region")
-    step_s = sum(s[-1] for s in stage_ms) / 1e3
+    step_s = sum(s[-1] for s in step_ms) / 1e3
+    # per-launch breakdown, after the timed region: every boundary recorded
+    stage_ms = []
+    for _ in range(min(args.steps, 5)):
+        flush.zero_()
+        stage_ms.append(layer.forward_timed(x, out))
+    if B.moe_sync_status(layer.workspace) != 0:
+        raise RuntimeError("device status after the per-stage steps")
     block = None
     if args.block or args.bias:
         # the same steps through moe_forward_block (RMSNorm, the layer, the residual
@@ -450,8 +463,8 @@ def run_ours(args, inp, name):
     ms_per_step = 1e3 * step_s_max / args.steps
 
     # dominant kernel: live CUDA-event durations of the gate/up GEMM launches
-    dom = B.STAGES.index(DOMINANT_STAGE)
-    dom_ms = sum(s[dom] for s in stage_ms) / len(stage_ms)
+    # in the timed steps
+    dom_ms = sum(s[dom] for s in step_ms) / len(step_ms)
     dom_flops = 4.0 * inp.d * inp.I * T * inp.k
     peaks, kind = load_peaks()
     stage_avg = {n: sum(s[i] for s in stage_ms) / len(stage_ms) for i, n in enumerate(B.STAGES)}

@@ -177,6 +177,27 @@ MOE_API moe_status moe_forward_timed(const void* x_dev, const float* W_r_dev, co
                                      float* stage_ms_host);
 
 /*
+ * moe_forward_timed with only some launch boundaries recorded, for timing
+ * with less interference: each event recorded between two launches delays
+ * the second by a few microseconds, which is visible on decode-sized steps.
+ * Bit i of event_mask (i = 0..11) records boundary i, the event before launch
+ * i in the order of moe_forward_timed (bit 11: after the last launch); bits 0
+ * and 11 are always recorded, bits above 11 are an error (MOE_ERR_INVALID_ARG).
+ * stage_ms_host[i] for a recorded boundary i < 11 is the device time to the
+ * next recorded boundary, 0 for the others; stage_ms_host[11] is the whole
+ * span. Example: bits 0, 8, 9, 11 give the gate/up GEMM alone in [8] and the
+ * whole pass in [11]. Blocks the calling thread until the pass has finished.
+ */
+MOE_API moe_status moe_forward_timed_events(const void* x_dev, const float* W_r_dev,
+                                            const float* b_r_dev, const uint8_t* Wgu_codes_dev,
+                                            const uint8_t* Wgu_scales_dev,
+                                            const uint8_t* Wd_codes_dev,
+                                            const uint8_t* Wd_scales_dev, int E, int k, int T,
+                                            int d, int I, void* out_dev, void* workspace_dev,
+                                            size_t workspace_bytes, void* stream,
+                                            unsigned int event_mask, float* stage_ms_host);
+
+/*
  * Same as moe_forward with the activations in host memory: copies x_host
  * (T*d*2 bytes; pinned memory gives asynchronous copies) to the workspace,
  * runs the forward pass and copies the result to out_host, then synchronises

@@ -31,6 +31,7 @@ EXPORTS = [
     "moe_selftest_wait_timeout", "moe_forward_launch_count", "moe_forward_timed",
     "moe_set_tile_policy", "moe_route_noalloc", "moe_probe_tensor_rate",
     "moe_workspace_size_block", "moe_forward_block", "moe_rms_norm", "moe_forward_biased",
+    "moe_forward_timed_events",
 ]
 
 STAGES = ["router_logits", "topk_softmax", "perm_hist", "perm_scan", "perm_scatter",
@@ -80,6 +81,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_forward_hostio.argtypes = fwd
     lib.moe_forward_timed.restype = i32
     lib.moe_forward_timed.argtypes = fwd + [ctypes.POINTER(ctypes.c_float)]
+    lib.moe_forward_timed_events.restype = i32
+    lib.moe_forward_timed_events.argtypes = fwd + [ctypes.c_uint, ctypes.POINTER(ctypes.c_float)]
     lib.moe_route.restype = i32
     lib.moe_route.argtypes = [vp, fp, fp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     lib.moe_route_noalloc.restype = i32
@@ -199,6 +202,20 @@ def moe_forward_timed(x, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, E
         _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(Wgu_codes), _ptr(Wgu_scales), _ptr(Wd_codes),
         _ptr(Wd_scales), E, k, T, d, I, _ptr(out), _ptr(workspace), workspace.numel(),
         _stream(stream), ms))
+    return list(ms)
+
+
+def moe_forward_timed_events(x, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, E, k, T, d,
+                             I, out, workspace, event_mask: int, stream=None) -> list:
+    """moe_forward_timed recording only the boundaries in event_mask (bit i:
+    before launch i, bit len(STAGES): after the last); entries of unrecorded
+    boundaries are 0, each recorded one spans to the next recorded. Blocks."""
+    _require_cuda(x, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, out, workspace)
+    ms = (ctypes.c_float * (len(STAGES) + 1))()
+    _check("moe_forward_timed_events", load().moe_forward_timed_events(
+        _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(Wgu_codes), _ptr(Wgu_scales), _ptr(Wd_codes),
+        _ptr(Wd_scales), E, k, T, d, I, _ptr(out), _ptr(workspace), workspace.numel(),
+        _stream(stream), event_mask, ms))
     return list(ms)
 
 
@@ -330,6 +347,12 @@ class MoELayer:
         return moe_forward_timed(x, self.W_r, self.b_r, self.Wgu_codes, self.Wgu_scales,
                                  self.Wd_codes, self.Wd_scales, self.E, self.k, T, self.d,
                                  self.I, out, self.workspace, stream)
+
+    def forward_timed_events(self, x, out, event_mask: int, stream=None):
+        T = x.shape[0]
+        return moe_forward_timed_events(x, self.W_r, self.b_r, self.Wgu_codes, self.Wgu_scales,
+                                        self.Wd_codes, self.Wd_scales, self.E, self.k, T, self.d,
+                                        self.I, out, self.workspace, event_mask, stream)
 
     def forward_hostio(self, x_host, out_host, stream=None):
         T = x_host.shape[0]

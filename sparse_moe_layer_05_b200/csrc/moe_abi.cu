@@ -215,14 +215,14 @@ moe_status check_forward_args(const void* x, const float* W_r, const float* b_r,
 }
 
 // Optional per-launch event recording (moe_forward_timed): ev[i] is recorded
-// before launch i, ev[kStages] after the last one.
+// before launch i, ev[kStages] after the last one; a null ev[i] is skipped.
 constexpr int kStages = 11;
 
 struct StageEvents {
   cudaEvent_t ev[kStages + 1];
   cudaStream_t st;
   void mark(int i) const {
-    if (ev[0]) cudaEventRecord(ev[i], st);
+    if (ev[i]) cudaEventRecord(ev[i], st);
   }
 };
 
@@ -625,7 +625,20 @@ moe_status moe_forward_timed(const void* x_dev, const float* W_r_dev, const floa
                              const uint8_t* Wd_codes_dev, const uint8_t* Wd_scales_dev, int E,
                              int k, int T, int d, int I, void* out_dev, void* workspace_dev,
                              size_t workspace_bytes, void* stream, float* stage_ms_host) {
+  return moe_forward_timed_events(x_dev, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev,
+                                  Wd_codes_dev, Wd_scales_dev, E, k, T, d, I, out_dev,
+                                  workspace_dev, workspace_bytes, stream,
+                                  (1u << (kStages + 1)) - 1u, stage_ms_host);
+}
+
+moe_status moe_forward_timed_events(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
+                                    const uint8_t* Wgu_codes_dev, const uint8_t* Wgu_scales_dev,
+                                    const uint8_t* Wd_codes_dev, const uint8_t* Wd_scales_dev,
+                                    int E, int k, int T, int d, int I, void* out_dev,
+                                    void* workspace_dev, size_t workspace_bytes, void* stream,
+                                    unsigned int event_mask, float* stage_ms_host) {
   if (!stage_ms_host) return MOE_ERR_INVALID_ARG;
+  if (event_mask >> (kStages + 1)) return MOE_ERR_INVALID_ARG;
   moe_status s = check_forward_args(x_dev, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev,
                                     Wd_codes_dev, Wd_scales_dev, E, k, T, d, I, out_dev,
                                     workspace_dev);
@@ -637,12 +650,16 @@ moe_status moe_forward_timed(const void* x_dev, const float* W_r_dev, const floa
   if (T == 0) return MOE_OK;
   int num_sms = 0;
   if ((s = device_info(&num_sms)) != MOE_OK) return s;
+  // the first and the last boundary are always recorded (the whole span)
+  event_mask |= 1u | (1u << kStages);
   StageEvents tev;
   tev.st = static_cast<cudaStream_t>(stream);
   for (int i = 0; i <= kStages; ++i) tev.ev[i] = nullptr;
   for (int i = 0; i <= kStages; ++i) {
+    if (!((event_mask >> i) & 1u)) continue;
     if (cudaEventCreate(&tev.ev[i]) != cudaSuccess) {
-      for (int j = 0; j < i; ++j) cudaEventDestroy(tev.ev[j]);
+      for (int j = 0; j < i; ++j)
+        if (tev.ev[j]) cudaEventDestroy(tev.ev[j]);
       cudaGetLastError();
       return MOE_ERR_CUDA;
     }
@@ -651,12 +668,19 @@ moe_status moe_forward_timed(const void* x_dev, const float* W_r_dev, const floa
                   Wgu_scales_dev, Wd_codes_dev, Wd_scales_dev, E, k, T, d, I,
                   static_cast<uint16_t*>(out_dev), workspace_dev, L, tev.st, num_sms, &tev);
   if (s == MOE_OK && cudaEventSynchronize(tev.ev[kStages]) == cudaSuccess) {
-    for (int i = 0; i < kStages; ++i) cudaEventElapsedTime(&stage_ms_host[i], tev.ev[i], tev.ev[i + 1]);
+    // a recorded boundary's entry spans to the next recorded boundary
+    for (int i = 0; i < kStages; ++i) {
+      if (!tev.ev[i]) continue;
+      int j = i + 1;
+      while (!tev.ev[j]) ++j;
+      cudaEventElapsedTime(&stage_ms_host[i], tev.ev[i], tev.ev[j]);
+    }
     cudaEventElapsedTime(&stage_ms_host[kStages], tev.ev[0], tev.ev[kStages]);
   } else if (s == MOE_OK) {
     s = MOE_ERR_CUDA;
   }
-  for (int i = 0; i <= kStages; ++i) cudaEventDestroy(tev.ev[i]);
+  for (int i = 0; i <= kStages; ++i)
+    if (tev.ev[i]) cudaEventDestroy(tev.ev[i]);
   cudaGetLastError();
   return s;
 }

@@ -393,6 +393,29 @@ def test_forward_deterministic_and_hostio_equal(T):
         assert np.array_equal(oh.numpy(), out1)
 
 
+def test_timed_events_sparse_mask():
+    """Only the masked boundaries are timed (others read 0; a recorded one spans to
+    the next recorded), the output is moe_forward's bit for bit, and mask bits above
+    the last boundary are rejected."""
+    from sparse_moe_layer_05_b200 import binding as B
+    for T in (64, 600):                        # block-scaled and bf16 tiles
+        inp = W.make_custom(448, 320, 8, 2, T, seed=17)
+        want, layer = G.run_forward(inp)
+        x = _t(inp.x)
+        out = torch.empty((T, inp.d), dtype=torch.uint16, device="cuda")
+        nb = len(B.STAGES)
+        dom = B.STAGES.index("gemm_gateup_swiglu")
+        ms = layer.forward_timed_events(x, out, (1 << dom) | (1 << (dom + 1)))
+        assert np.array_equal(out.cpu().numpy(), want)
+        assert all(ms[i] == 0.0 for i in range(nb) if i not in (0, dom, dom + 1))
+        assert ms[dom] > 0 and ms[dom + 1] > 0 and ms[0] > 0
+        assert abs(ms[0] + ms[dom] + ms[dom + 1] - ms[nb]) <= 1e-3 + 1e-3 * ms[nb]
+        full = layer.forward_timed(x, out)
+        assert all(v >= 0 for v in full) and full[nb] > 0
+        with pytest.raises(B.MoEError):
+            layer.forward_timed_events(x, out, 1 << (nb + 1))
+
+
 def test_skewed_routing_and_empty_experts():
     inp = W.make_custom(128, 128, 16, 2, 700, seed=13)
     inp.b_r[3] += 50.0            # every token picks expert 3
