@@ -207,8 +207,10 @@ MOE_API moe_status moe_forward_timed_events(const void* x_dev, const float* W_r_
  * token's output depends on that token alone, so the result is the same):
  * the copy in, the forward and the copy out of neighbouring chunks overlap on
  * two copy streams the library creates once per device, ordered after the
- * caller's earlier work on `stream`. Not thread-safe against concurrent
- * host-buffer calls on one device. moe_workspace_size_hostio() is at least
+ * caller's earlier work on `stream`. Host threads may call it concurrently on
+ * one device (with separate workspaces): they take turns at enqueueing and
+ * share the copy streams. If a launch fails, the call waits for the copies it
+ * had enqueued before it returns the error. moe_workspace_size_hostio() is at least
  * moe_workspace_size(), so one workspace serves both calls.
  */
 MOE_API size_t moe_workspace_size_hostio(int E, int k, int T, int d, int I);

@@ -4,6 +4,8 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <mutex>
+
 #include "../../include/moe_b200.h"
 #include "moe_internal.h"
 
@@ -562,16 +564,21 @@ moe_status moe_forward_hostio(const void* x_host, const float* W_r_dev, const fl
     if (s != MOE_OK) return s;
     MOE_CUDA(cudaMemcpyAsync(oh, out_buf, bytes, cudaMemcpyDeviceToHost, st));
   } else {
-    // copy streams and events, created once per device
+    // copy streams and events, created once per device. Calls from several
+    // host threads take turns at enqueueing (the events are shared: a wait
+    // must see the record of its own call); their copies then share the two
+    // copy streams in that order.
     struct CopyRes {
       cudaStream_t h2d, d2h;
       cudaEvent_t start, in[kHostioChunks], fwd[kHostioChunks], done;
     };
     static CopyRes res[kMaxDevices];
     static bool have[kMaxDevices] = {false};
+    static std::mutex lock[kMaxDevices];
     int dev = 0;
     MOE_CUDA(cudaGetDevice(&dev));
     if (dev < 0 || dev >= kMaxDevices) return MOE_ERR_NO_DEVICE;
+    std::lock_guard<std::mutex> guard(lock[dev]);
     CopyRes& r = res[dev];
     if (!have[dev]) {
       MOE_CUDA(cudaStreamCreateWithFlags(&r.h2d, cudaStreamNonBlocking));
@@ -600,7 +607,12 @@ moe_status moe_forward_hostio(const void* x_host, const float* W_r_dev, const fl
       void* ws = static_cast<uint8_t*>(workspace_dev) + (c & 1) * hp.sub_stride;
       s = run_forward(x_in + off, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev, Wd_codes_dev,
                       Wd_scales_dev, E, k, tn, d, I, out_buf + off, ws, hp.sub, st, num_sms);
-      if (s != MOE_OK) return s;
+      if (s != MOE_OK) {
+        // no copy of an earlier chunk may land after the call has returned
+        cudaStreamSynchronize(r.h2d);
+        cudaStreamSynchronize(r.d2h);
+        return s;
+      }
       MOE_CUDA(cudaEventRecord(r.fwd[c], st));
       MOE_CUDA(cudaStreamWaitEvent(r.d2h, r.fwd[c], 0));
       MOE_CUDA(cudaMemcpyAsync(oh + off, out_buf + off, bytes, cudaMemcpyDeviceToHost, r.d2h));

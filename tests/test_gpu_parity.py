@@ -393,6 +393,40 @@ def test_forward_deterministic_and_hostio_equal(T):
         assert np.array_equal(oh.numpy(), out1)
 
 
+def test_hostio_concurrent_threads():
+    """Two host threads run chunked host-buffer forwards on one device at once
+    (separate layers and workspaces, shared copy streams): every result equals the
+    device-buffer forward."""
+    import threading
+    from sparse_moe_layer_05_b200.binding import MoELayer
+    T = 4099
+    inp = W.make_custom(352, 224, 8, 2, T, seed=12)
+    want, _ = G.run_forward(inp)
+    layers = [MoELayer(inp, hostio=True) for _ in range(2)]
+    xh = torch.from_numpy(inp.x).pin_memory()
+    outs = [torch.empty((T, inp.d), dtype=torch.uint16).pin_memory() for _ in range(2)]
+    errors = []
+
+    def work(i):
+        try:
+            torch.cuda.set_device(0)
+            with torch.cuda.stream(torch.cuda.Stream()):
+                for _ in range(4):
+                    outs[i].zero_()
+                    layers[i].forward_hostio(xh, outs[i])
+                    if not np.array_equal(outs[i].numpy(), want):
+                        errors.append(i)
+        except Exception as e:          # reported below, on the main thread
+            errors.append(repr(e))
+
+    threads = [threading.Thread(target=work, args=(i,)) for i in range(2)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join()
+    assert not errors, errors
+
+
 def test_timed_events_sparse_mask():
     """Only the masked boundaries are timed (others read 0; a recorded one spans to
     the next recorded), the output is moe_forward's bit for bit, and mask bits above
