@@ -376,8 +376,7 @@ def run_ours(args, inp, name):
     if status != 0:
         raise RuntimeError(f"device status {B.STATUS.get(status, status)} after warm-up")
 
-    clocks_path = os.path.join(ROOT, "gpurun_out", "bench_clocks.csv") if os.path.isdir(
-        os.path.join(ROOT, "gpurun_out")) else None
+    clocks_path = args.clocks_csv
     step_ms = []
     barrier(world)
     torch.cuda.synchronize()
@@ -564,6 +563,8 @@ def main(argv=None):
     ap.add_argument("--block", action="store_true",
                     help="time the MoE sublayer with its pre-norm and residual add "
                          "(moe_forward_block: out = h + MoE(RMSNorm(h)))")
+    ap.add_argument("--clocks-csv", default=None,
+                    help="also write every clock sample of the timed region to this CSV file")
     ap.add_argument("--bias", action="store_true",
                     help="time the layer with per-expert gate/up and down biases "
                          "(moe_forward_biased; with --block, the sublayer with biases)")
