@@ -95,3 +95,58 @@ def test_argument_errors_before_any_launch(lib):
     r = lib.moe_route
     assert r(good, good, good, 4, 2, 8, 64, good, good, good, None, None, good, 1 << 20, None) == 1
     assert lib.moe_mxfp4_to_bf16(good, good, 4, 40, good, None) == 1
+
+
+def test_biased_block_and_timed_entries_check_arguments(lib):
+    """The entries added for expert biases, the sublayer and sparse timing reject
+    bad arguments before any launch; NULL biases are allowed."""
+    good = 0x10000
+    fwd = [good] * 7 + [4, 2, 8, 64, 128, good, good, 1 << 30, None]
+    biased = fwd[:5] + [good] + fwd[5:7] + [good] + fwd[7:]
+    f = lib.moe_forward_biased
+    a = list(biased)
+    a[5] = good + 4
+    assert f(*a) == 1                                   # misaligned gate/up bias
+    a = list(biased)
+    a[8] = good + 8
+    assert f(*a) == 1                                   # misaligned down bias
+    a = list(biased)
+    a[5], a[8], a[11] = None, None, 0
+    assert f(*a) == 0                                   # no biases, T = 0
+    a = list(biased)
+    a[10] = 5
+    assert f(*a) == 2                                   # k > E
+    blk = [good, good, ctypes.c_float(1e-5)] + biased[1:]
+    a = list(blk)
+    a[7] = good + 4
+    assert lib.moe_forward_block(*a) == 1               # misaligned gate/up bias
+    a = list(blk)
+    a[2] = ctypes.c_float(-1.0)
+    assert lib.moe_forward_block(*a) == 1               # eps < 0
+    ms = (ctypes.c_float * 12)()
+    t = lib.moe_forward_timed_events
+    assert t(*(fwd + [1 << 12, ms])) == 1               # a boundary past the last
+    assert t(*(fwd + [0x301, None])) == 1               # no output array
+    a = fwd + [0x301, ms]
+    a[9] = 0
+    assert t(*a) == 0 and list(ms) == [0.0] * 12        # T = 0: zeros, nothing launched
+
+
+@pytest.mark.parametrize("E,k,T,d,I", [(4, 2, 256, 64, 128), (32, 4, 8192, 2880, 2880),
+                                       (128, 4, 32, 2880, 2880), (248, 20, 16, 2880, 2880),
+                                       (8, 2, 1000, 352, 224), (1, 1, 1, 32, 32)])
+def test_workspace_regions_hold_their_arrays(E, k, T, d, I):
+    """Every public workspace region is 256-byte aligned and has room, up to the
+    next region, for the array the header says it holds."""
+    L = B.moe_workspace_layout(E, k, T, d, I)
+    P = T * k
+    need = {"status": 4, "logits": T * E * 4, "topk_idx": P * 4, "topk_w": P * 4,
+            "counts": E * 4, "offsets": (E + 1) * 4, "perm": P * 4, "xp": P * d * 2,
+            "h": P * I * 2, "yw": P * d * 4}
+    order = sorted((L[n], n) for n in need)
+    ends = [off for off, _ in order[1:]] + [L["total"]]
+    for (off, n), end in zip(order, ends):
+        assert off % 256 == 0, n
+        assert end - off >= need[n], (n, end - off, need[n])
+    assert B.moe_workspace_size(E, k, T, d, I) == L["total"]
+    assert B.moe_workspace_size_block(E, k, T, d, I) >= L["total"] + T * d * 2
