@@ -389,8 +389,8 @@ def minifloat_round(v: np.ndarray, ebits: int, mbits: int, bias: int,
     v = np.asarray(v, dtype=np.float64)
     a = np.abs(v)
     emin = 1 - bias
-    with np.errstate(divide="ignore"):
-        e = np.floor(np.log2(np.where(a > 0, a, 1.0)))
+    # floor(log2 a), exactly: a = m 2^x with m in [0.5, 1)
+    e = np.frexp(np.where(a > 0, a, 1.0))[1] - 1
     e = np.maximum(e, emin)
     quantum = np.exp2(e - mbits)
     r = np.round(a / quantum) * quantum          # numpy rounds halves to even
@@ -412,8 +412,7 @@ def mx_quantize(x: np.ndarray, elem: str, group: int = 32) -> np.ndarray:
         raise ValueError("the last axis must hold whole groups")
     g = x.reshape(*x.shape[:-1], K // group, group)
     amax = np.abs(g).max(axis=-1, keepdims=True)
-    with np.errstate(divide="ignore"):
-        X = np.exp2(np.floor(np.log2(np.where(amax > 0, amax, 1.0))) - emax)
+    X = np.exp2((np.frexp(np.where(amax > 0, amax, 1.0))[1] - 1) - emax)
     q = minifloat_round(g / X, ebits, mbits, bias, max_normal) * X
     return np.where(amax > 0, q, 0.0).reshape(x.shape)
 
