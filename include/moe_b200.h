@@ -108,13 +108,56 @@ MOE_API int moe_version(void);
  * into two E4M3 terms (hi and lo) with E8M0 scales; the split is exact for
  * elements of at least 2^-13 of their group's max |x|, smaller ones keep an
  * error below 2^-21 of it. 128 weight rows x 16 tokens per tile, two CTAs
- * per SM with two UMMA-issuing threads each. It needs d and I multiples of 64 in [128, 3072] and 32-byte
- * aligned code arrays; otherwise policy 4 picks as policy 0 does.
- * All policies compute the same function within the output tolerance. Not
- * thread-safe against concurrent forward calls. MOE_ERR_INVALID_ARG for other
+ * per SM with two UMMA-issuing threads each (120-token tiles, one CTA per SM,
+ * when experts average 64 rows or more).
+ * 5 selects the block-scaled tiles on a CTA pair: a 2-CTA cluster computes
+ * 256-token tiles with tcgen05.mma.cta_group::2 (M = 256 token rows, the two
+ * E4M3 terms issued as two UMMAs into one accumulator; N = 192 weight rows for
+ * gate/up, 240 for down).
+ * 4 and 5 need d and I multiples of 64 in [128, 3072] and 32-byte aligned
+ * code arrays; otherwise they pick as policy 0 does.
+ * All policies compute the same function within the output tolerance.
+ * This sets the process default that the entry points without an options
+ * argument use; a change takes effect for calls made after it, from any
+ * thread. Callers that share a process and want a policy of their own pass
+ * it per call through moe_forward_ex instead. MOE_ERR_INVALID_ARG for other
  * values.
  */
 MOE_API moe_status moe_set_tile_policy(int policy);
+
+/*
+ * Precision of the activations that enter the expert GEMMs (the expert inputs
+ * x and the SwiGLU rows H), per call through moe_forward_opts.act_quant.
+ *   MOE_ACT_BF16   the layer as the pages define it: bf16 activations used at
+ *                  full precision (the block-scaled tiles split each value
+ *                  exactly into two E4M3 terms); output within 2e-2 x RMS.
+ * The two others change the function ("gpt-oss-20b and gpt-oss-120b",
+ * "Four-bit expert weights" puts only the expert weights in MXFP4; field
+ * guide "gpt-oss 20B": MXFP4 is "not every path"): the activations are
+ * rounded to an MX block format, per group of 32 along the contraction, with
+ * the OCP Microscaling conversion (shared scale 2^(floor(log2 max|v|) - emax),
+ * elements rounded to nearest even, magnitudes above the largest normal
+ * clamped to it):
+ *   MOE_ACT_MXFP8  E4M3 elements (emax 8): the w4a8 layer;
+ *   MOE_ACT_MXFP4  E2M1 elements (emax 2): the w4a4 layer.
+ */
+typedef enum { MOE_ACT_BF16 = 0, MOE_ACT_MXFP8 = 1, MOE_ACT_MXFP4 = 2 } moe_act_quant;
+
+/*
+ * Per-call options of moe_forward_ex. Zero-initialise and set what you need.
+ *   tile_policy    -1: the process default (moe_set_tile_policy); 0: pick by
+ *                  shape; 1..5: force a tile family (as moe_set_tile_policy).
+ *                  0 is what a zeroed struct asks for.
+ *   act_quant      a moe_act_quant value (0 = MOE_ACT_BF16).
+ *   gu_bias_dev, down_bias_dev   the experts' biases as in
+ *                  moe_forward_biased; NULL for none.
+ */
+typedef struct {
+  int tile_policy;
+  int act_quant;
+  const float* gu_bias_dev;
+  const float* down_bias_dev;
+} moe_forward_opts;
 
 /*
  * Bytes of device workspace moe_forward needs for this shape (0 for invalid
@@ -157,6 +200,28 @@ MOE_API moe_status moe_forward_biased(const void* x_dev, const float* W_r_dev, c
                                       const uint8_t* Wd_scales_dev, const float* down_bias_dev,
                                       int E, int k, int T, int d, int I, void* out_dev,
                                       void* workspace_dev, size_t workspace_bytes, void* stream);
+
+/*
+ * moe_forward with per-call options (opts may be NULL: the process default
+ * tile policy, bf16 activations, no biases). Everything else -- arguments,
+ * workspace size (moe_workspace_size), errors, stream semantics -- is as in
+ * moe_forward. MOE_ERR_INVALID_ARG for a tile_policy outside -1..5 or an
+ * unknown act_quant; MOE_ERR_UNSUPPORTED for an act_quant the shape cannot
+ * run (the quantised modes need the block-scaled tiles' shapes: d and I
+ * multiples of 64 in [128, 3072], 32-byte aligned code arrays).
+ * The quantised modes always run the block-scaled tiles (E2M1 weights x E4M3
+ * or E2M1 activations, kind::mxf8f6f4, one term): 16-token tiles when experts
+ * average under 64 rows, else 128-token tiles, on a CTA pair with tile_policy 5.
+ * Their intermediates in the workspace: the converted x rows in the xp region
+ * and the converted H rows in the h region, in the padded token layout the
+ * block-scaled tiles read, their scales at x_scales and h_scales.
+ */
+MOE_API moe_status moe_forward_ex(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
+                                  const uint8_t* Wgu_codes_dev, const uint8_t* Wgu_scales_dev,
+                                  const uint8_t* Wd_codes_dev, const uint8_t* Wd_scales_dev,
+                                  int E, int k, int T, int d, int I, void* out_dev,
+                                  void* workspace_dev, size_t workspace_bytes,
+                                  const moe_forward_opts* opts, void* stream);
 
 /*
  * Same as moe_forward, instrumented: records a CUDA event on `stream` before
@@ -209,9 +274,12 @@ MOE_API moe_status moe_forward_timed_events(const void* x_dev, const float* W_r_
  * two copy streams the library creates once per device, ordered after the
  * caller's earlier work on `stream`. Host threads may call it concurrently on
  * one device (with separate workspaces): they take turns at enqueueing and
- * share the copy streams. If a launch fails, the call waits for the copies it
- * had enqueued before it returns the error. moe_workspace_size_hostio() is at least
- * moe_workspace_size(), so one workspace serves both calls.
+ * share the copy streams. If a launch or a copy fails, the call waits for the
+ * copies it had enqueued before it returns the error. The call returns the
+ * device status of the pass itself: each chunk keeps its own status word
+ * (chunk c uses 32-bit word c of the 16-byte status block at the workspace's
+ * start), so a timeout in any chunk is returned. moe_workspace_size_hostio()
+ * is at least moe_workspace_size(), so one workspace serves both calls.
  */
 MOE_API size_t moe_workspace_size_hostio(int E, int k, int T, int d, int I);
 MOE_API moe_status moe_forward_hostio(const void* x_host, const float* W_r_dev, const float* b_r_dev,
@@ -254,9 +322,11 @@ MOE_API moe_status moe_route(const void* x_dev, const float* W_r_dev, const floa
  * about 4.1 MiB that every GPU which loads the library holds until the
  * process exits. Limit: T * E <= 1,048,576 (e.g. T = 8192 tokens at E = 128,
  * or T = 4096 at E = 248); larger calls return MOE_ERR_UNSUPPORTED and
- * launch nothing. The first call on a device looks up the array's device
- * address (cudaGetSymbolAddress, with that device current); make that first
- * call before any stream capture. All calls on a device share the array and
+ * launch nothing. Every call looks up the array's device address on the
+ * current device (cudaGetSymbolAddress; no address is cached, so a new
+ * primary context or a device reset needs nothing from the caller); the
+ * first call on a device also loads the library's device code there, so
+ * make that first call before any stream capture. All calls on a device share the array and
  * it keeps the last call's contents (each call rewrites what it reads), so
  * calls whose device work overlaps -- concurrent streams, or several host
  * threads -- race on it; serialise them.
@@ -279,6 +349,9 @@ MOE_API moe_status moe_route_noalloc(const void* x_dev, const float* W_r_dev, co
  */
 typedef struct {
   size_t logits, topk_idx, topk_w, counts, offsets, perm, xp, h, yw, status, total;
+  /* the block-scaled tiles' B-scale blocks of the x rows and of the H rows
+   * (E8M0 bytes in the layout the GEMMs copy into tensor memory) */
+  size_t x_scales, h_scales;
 } moe_ws_layout;
 MOE_API moe_status moe_workspace_layout(int E, int k, int T, int d, int I, moe_ws_layout* layout);
 
@@ -295,6 +368,23 @@ MOE_API moe_status moe_workspace_layout(int E, int k, int T, int d, int I, moe_w
  */
 MOE_API moe_status moe_mx_split_e4m3(const void* x_dev, int rows, int K, uint8_t* hi_dev,
                                      uint8_t* lo_dev, uint8_t* scales_dev, void* stream);
+
+/*
+ * The activation conversion of the quantised modes (moe_forward_opts.act_quant)
+ * on plain rows, with the kernels the layer uses: x_dev [rows][K] bf16 ->
+ * q_dev [rows][K] E4M3 bytes (MOE_ACT_MXFP8) or [rows][K/2] packed E2M1 codes
+ * (MOE_ACT_MXFP4; byte b holds element 2b in its low nibble, as the weights),
+ * and scales_dev [rows][K/32] E8M0 bytes, per group of 32: the OCP
+ * Microscaling conversion (v1.0, section 6.3) with shared scale
+ * 2^(floor(log2 max|x|) - emax), emax 8 (E4M3) or 2 (E2M1), elements rounded
+ * to nearest even and clamped to the largest normal. A group whose max|x| is
+ * below 2^(emax - 127) keeps the smallest scale byte, 0; an all-zero group
+ * gets byte 127 and zero codes. The pages have no counterpart: they put only
+ * the expert weights in MXFP4 ("Four-bit expert weights"). K a multiple of 32;
+ * x_dev and q_dev 16-byte aligned; all buffers the caller's.
+ */
+MOE_API moe_status moe_mx_quantize(const void* x_dev, int rows, int K, int act_quant,
+                                   uint8_t* q_dev, uint8_t* scales_dev, void* stream);
 
 /*
  * Decode MXFP4 rows to bf16 on the device with the same decoder the grouped
@@ -350,20 +440,6 @@ MOE_API moe_status moe_forward_block(const void* h_dev, const float* g_dev, floa
  */
 MOE_API moe_status moe_rms_norm(const void* h_dev, const float* g_dev, float eps, int T, int d,
                                 void* x_dev, void* stream);
-
-/*
- * Tensor-core rate probe (diagnostic; the pages have no counterpart): on every
- * SM one thread issues back-to-back UMMAs of M = 128 and N columns from
- * shared-memory tiles, per_commit per tcgen05.commit, and *mac_per_clk_sm
- * receives the multiply-accumulates per SM clock of the slowest SM. kind 0 is
- * bf16 (kind::f16, K = 16 per UMMA), kind 1 the block-scaled E2M1 x E4M3 kind
- * the block-scaled tiles use (kind::mxf8f6f4, K = 32). N in [16, 256], a
- * multiple of 16; per_commit in [4, 64], a multiple of 4. Multiply by 2 x the
- * SM count x the SM clock for FLOP/s. Allocates and frees a small device
- * buffer and synchronises `stream`. MOE_ERR_TIMEOUT if a bounded wait gave up.
- */
-MOE_API moe_status moe_probe_tensor_rate(int kind, int N, int per_commit, double* mac_per_clk_sm,
-                                         void* stream);
 
 /*
  * Number of kernel launches one moe_forward call enqueues for this shape

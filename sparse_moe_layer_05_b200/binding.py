@@ -29,10 +29,17 @@ EXPORTS = [
     "moe_workspace_size_hostio", "moe_forward_hostio", "moe_route_workspace_size",
     "moe_route", "moe_workspace_layout", "moe_mxfp4_to_bf16", "moe_mx_split_e4m3", "moe_sync_status",
     "moe_selftest_wait_timeout", "moe_forward_launch_count", "moe_forward_timed",
-    "moe_set_tile_policy", "moe_route_noalloc", "moe_probe_tensor_rate",
+    "moe_set_tile_policy", "moe_route_noalloc",
     "moe_workspace_size_block", "moe_forward_block", "moe_rms_norm", "moe_forward_biased",
-    "moe_forward_timed_events",
+    "moe_forward_timed_events", "moe_forward_ex", "moe_mx_quantize",
 ]
+# the measurement library (libmoe_b200_probe.so, include/moe_b200_probe.h)
+PROBE_EXPORTS = ["moe_probe_tensor_rate", "moe_probe_error_string", "moe_probe_error_site"]
+PROBE_LIB_PATH = os.path.join(PKG, "libmoe_b200_probe.so")
+
+# moe_forward_opts.act_quant
+ACT_BF16, ACT_MXFP8, ACT_MXFP4 = 0, 1, 2
+ACT_MODES = {"bf16": ACT_BF16, "mxfp8": ACT_MXFP8, "mxfp4": ACT_MXFP4}
 
 STAGES = ["router_logits", "topk_softmax", "perm_hist", "perm_scan", "perm_scatter",
           "gather_rows", "transpose_scales_gu", "transpose_scales_d", "gemm_gateup_swiglu",
@@ -45,10 +52,16 @@ class MoEError(RuntimeError):
         self.code = code
 
 
+class ForwardOpts(ctypes.Structure):
+    """moe_forward_opts (include/moe_b200.h)."""
+    _fields_ = [("tile_policy", ctypes.c_int), ("act_quant", ctypes.c_int),
+                ("gu_bias_dev", ctypes.c_void_p), ("down_bias_dev", ctypes.c_void_p)]
+
+
 class WsLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in
                 ("logits", "topk_idx", "topk_w", "counts", "offsets", "perm", "xp", "h", "yw",
-                 "status", "total")]
+                 "status", "total", "x_scales", "h_scales")]
 
 
 _lib = None
@@ -101,8 +114,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_forward_block.argtypes = [vp, fp, ctypes.c_float] + fwd_b[1:]
     lib.moe_rms_norm.restype = i32
     lib.moe_rms_norm.argtypes = [vp, fp, ctypes.c_float, i32, i32, vp, vp]
-    lib.moe_probe_tensor_rate.restype = i32
-    lib.moe_probe_tensor_rate.argtypes = [i32, i32, i32, ctypes.POINTER(ctypes.c_double), vp]
+    lib.moe_forward_ex.restype = i32
+    lib.moe_forward_ex.argtypes = fwd[:15] + [ctypes.POINTER(ForwardOpts), vp]
+    lib.moe_mx_quantize.restype = i32
+    lib.moe_mx_quantize.argtypes = [vp, i32, i32, i32, u8p, u8p, vp]
     lib.moe_mx_split_e4m3.restype = i32
     lib.moe_mx_split_e4m3.argtypes = [vp, i32, i32, u8p, u8p, u8p, vp]
     lib.moe_sync_status.restype = i32
@@ -114,6 +129,27 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_forward_launch_count.restype = i32
     lib.moe_forward_launch_count.argtypes = [i32] * 5
     _lib = lib
+    return lib
+
+
+_probe_lib = None
+
+
+def load_probe(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load the tensor-core rate probe library (measurement tooling)."""
+    global _probe_lib
+    if _probe_lib is not None:
+        return _probe_lib
+    p = path or PROBE_LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError(f"{p} is missing: build it with `python -m sparse_moe_layer_05_b200.build`")
+    lib = ctypes.CDLL(p)
+    lib.moe_probe_tensor_rate.restype = ctypes.c_int
+    lib.moe_probe_tensor_rate.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                          ctypes.POINTER(ctypes.c_double), ctypes.c_void_p]
+    lib.moe_probe_error_string.restype = ctypes.c_char_p
+    lib.moe_probe_error_site.restype = ctypes.c_char_p
+    _probe_lib = lib
     return lib
 
 
@@ -189,6 +225,23 @@ def moe_forward_biased(x, W_r, b_r, Wgu_codes, Wgu_scales, gu_bias, Wd_codes, Wd
         _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(Wgu_codes), _ptr(Wgu_scales), _ptr(gu_bias),
         _ptr(Wd_codes), _ptr(Wd_scales), _ptr(down_bias), E, k, T, d, I, _ptr(out),
         _ptr(workspace), workspace.numel(), _stream(stream)))
+
+
+def moe_forward_ex(x, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, E, k, T, d, I,
+                   out, workspace, tile_policy: int = 0, act_quant=ACT_BF16, gu_bias=None,
+                   down_bias=None, stream=None) -> None:
+    """moe_forward with per-call options: tile_policy (-1 process default, 0 by
+    shape, 1..4 forced), act_quant (ACT_BF16, ACT_MXFP8, ACT_MXFP4 or their
+    names), optional expert biases."""
+    _require_cuda(x, W_r, b_r, Wgu_codes, Wgu_scales, gu_bias, Wd_codes, Wd_scales, down_bias, out,
+                  workspace)
+    if isinstance(act_quant, str):
+        act_quant = ACT_MODES[act_quant]
+    o = ForwardOpts(tile_policy, act_quant, _ptr(gu_bias) or None, _ptr(down_bias) or None)
+    _check("moe_forward_ex", load().moe_forward_ex(
+        _ptr(x), _ptr(W_r), _ptr(b_r), _ptr(Wgu_codes), _ptr(Wgu_scales), _ptr(Wd_codes),
+        _ptr(Wd_scales), E, k, T, d, I, _ptr(out), _ptr(workspace), workspace.numel(),
+        ctypes.byref(o), _stream(stream)))
 
 
 def moe_forward_timed(x, W_r, b_r, Wgu_codes, Wgu_scales, Wd_codes, Wd_scales, E, k, T, d, I,
@@ -271,11 +324,26 @@ def moe_forward_block(h, g, eps: float, W_r, b_r, Wgu_codes, Wgu_scales, Wd_code
 
 
 def moe_probe_tensor_rate(kind: int, N: int, per_commit: int, stream=None) -> float:
-    """MACs per SM clock of back-to-back UMMAs (kind 0 bf16, 1 block-scaled E2M1 x E4M3)."""
+    """MACs per SM clock of back-to-back UMMAs (kind 0 bf16, 1 block-scaled
+    E2M1 x E4M3, 2 block-scaled E2M1 x E2M1), from the probe library."""
     out = ctypes.c_double(0.0)
-    _check("moe_probe_tensor_rate", load().moe_probe_tensor_rate(kind, N, per_commit,
-                                                                 ctypes.byref(out), _stream(stream)))
+    lib = load_probe()
+    code = lib.moe_probe_tensor_rate(kind, N, per_commit, ctypes.byref(out), _stream(stream))
+    if code == 4:        # MOE_ERR_CUDA: say which call failed and how
+        raise MoEError(f"moe_probe_tensor_rate ({lib.moe_probe_error_site().decode()}: "
+                       f"{lib.moe_probe_error_string().decode()})", code)
+    _check("moe_probe_tensor_rate", code)
     return out.value
+
+
+def moe_mx_quantize(x, rows: int, K: int, act_quant, q, scales, stream=None) -> None:
+    """The quantised modes' activation conversion on plain bf16 rows: q [rows, K]
+    E4M3 (ACT_MXFP8) or [rows, K/2] packed E2M1 (ACT_MXFP4), scales [rows, K/32]."""
+    _require_cuda(x, q, scales)
+    if isinstance(act_quant, str):
+        act_quant = ACT_MODES[act_quant]
+    _check("moe_mx_quantize", load().moe_mx_quantize(
+        _ptr(x), rows, K, act_quant, _ptr(q), _ptr(scales), _stream(stream)))
 
 
 def moe_mx_split_e4m3(x, rows: int, K: int, hi, lo, scales, stream=None) -> None:
@@ -290,12 +358,13 @@ def moe_mxfp4_to_bf16(codes, scales, rows: int, K: int, out, stream=None) -> Non
         _ptr(codes), _ptr(scales), rows, K, _ptr(out), _stream(stream)))
 
 
-TILE_AUTO, TILE_SINGLE, TILE_PAIR, TILE_SWAP, TILE_MX = 0, 1, 2, 3, 4
+TILE_AUTO, TILE_SINGLE, TILE_PAIR, TILE_SWAP, TILE_MX, TILE_MX_PAIR = 0, 1, 2, 3, 4, 5
 
 
 def moe_set_tile_policy(policy: int) -> None:
     """0 = by shape, 1 = single-CTA, 2 = CTA-pair, 3 = swapped-operand,
-    4 = block-scaled tiles (process-wide)."""
+    4 = block-scaled tiles, 5 = block-scaled tiles on a CTA pair: the process
+    default of the calls without options (moe_forward_ex takes one per call)."""
     _check("moe_set_tile_policy", load().moe_set_tile_policy(policy))
 
 

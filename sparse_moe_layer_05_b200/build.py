@@ -15,9 +15,12 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmoe_b200.so")
-SOURCES = ["moe_abi.cu", "moe_routing.cu", "moe_grouped_gemm.cu", "moe_mx_gemm.cu", "moe_noalloc.cu",
-           "moe_probe.cu"]
+SOURCES = ["moe_abi.cu", "moe_routing.cu", "moe_grouped_gemm.cu", "moe_mx_gemm.cu", "moe_mx_pair.cu",
+           "moe_noalloc.cu"]
 HEADERS = ["moe_ptx.cuh", "moe_internal.h"]
+# the tensor-core rate probe: measurement tooling, a library of its own
+PROBE_LIB = os.path.join(PKG, "libmoe_b200_probe.so")
+PROBE_SOURCES = ["moe_probe.cu"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -34,22 +37,20 @@ def nvcc_path() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str, sources, headers) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS]
-    deps.append(os.path.join(ROOT, "include", "moe_b200.h"))
+    t = os.path.getmtime(lib)
+    deps = [os.path.join(CSRC, f) for f in list(sources) + list(headers)]
+    deps += [os.path.join(ROOT, "include", h) for h in ("moe_b200.h", "moe_b200_probe.h")]
     deps.append(os.path.abspath(__file__))
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + ".tmp"
+def _nvcc(lib: str, sources, verbose: bool, extra) -> None:
+    tmp = lib + ".tmp"
     cmd = [nvcc_path(), *NVCC_FLAGS, *extra, "-I", os.path.join(ROOT, "include"),
-           "-o", tmp, *[os.path.join(CSRC, f) for f in SOURCES]]
+           "-o", tmp, *[os.path.join(CSRC, f) for f in sources]]
     if verbose:
         print(" ".join(cmd), flush=True)
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -57,7 +58,15 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         raise RuntimeError(f"nvcc failed ({res.returncode}):\n{res.stdout}\n{res.stderr}")
     if verbose and res.stderr:
         print(res.stderr, file=sys.stderr)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build(force: bool = False, verbose: bool = False, extra=()) -> str:
+    """Build the layer's library and the probe library (each only when stale)."""
+    if force or _stale(LIB, SOURCES, HEADERS):
+        _nvcc(LIB, SOURCES, verbose, extra)
+    if force or _stale(PROBE_LIB, PROBE_SOURCES, ["moe_ptx.cuh"]):
+        _nvcc(PROBE_LIB, PROBE_SOURCES, verbose, extra)
     return LIB
 
 

@@ -4,6 +4,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "../../include/moe_b200.h"
@@ -14,9 +15,11 @@ namespace {
 constexpr int kVersion = 100;  // 0.1.0
 constexpr int kMaxDevices = 64;
 
-// Grouped-GEMM tile policy: 0 = choose by shape, 1 = single-CTA tiles,
-// 2 = CTA-pair tiles, 3 = swapped-operand tiles, 4 = block-scaled tiles.
-int g_tile_policy = 0;
+// Process default of the grouped-GEMM tile policy (moe_set_tile_policy):
+// 0 = choose by shape, 1 = single-CTA tiles, 2 = CTA-pair tiles,
+// 3 = swapped-operand tiles, 4 = block-scaled tiles. Calls through
+// moe_forward_ex carry their own policy and never read it.
+std::atomic<int> g_tile_policy{0};
 
 // The block-scaled path reads the codes through 4-bit tensor maps: rows of a
 // multiple of 64 elements (at least 128) and 32-byte aligned code arrays.
@@ -26,9 +29,10 @@ bool mx_shape_ok(int d, int I) {
 }
 bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31) == 0; }
 
-int choose_tiles(int P, int E, bool mx_ok) {
-  if (g_tile_policy == 4 && mx_ok) return moe::TILES_MX;
-  if (g_tile_policy >= 1 && g_tile_policy <= 3) return g_tile_policy;
+int choose_tiles(int policy, int P, int E, bool mx_ok) {
+  if (policy == 4 && mx_ok) return moe::TILES_MX;
+  if (policy == 5 && mx_ok) return moe::TILES_MX_PAIR;
+  if (policy >= 1 && policy <= 3) return policy;
   const int64_t p = P, e = E;
   // Few routed rows per expert (decode): stream the weights, with the
   // block-scaled tiles where the shape allows (no CUDA-core weight decode),
@@ -102,6 +106,8 @@ void make_layout(int E, int k, int T, int d, int I, bool hostio, Layout* L, bool
   }
   if (block) L->x_norm = take(static_cast<size_t>(T) * d * 2);
   L->pub.total = off;
+  L->pub.x_scales = L->gu_scales_t;
+  L->pub.h_scales = L->d_scales_t;
 }
 
 void make_route_layout(int E, int k, int T, int d, Layout* L) {
@@ -161,6 +167,13 @@ void make_hostio_plan(int E, int k, int T, int d, int I, HostioPlan* hp) {
   Layout full;
   make_layout(E, k, T, d, I, false, &full);
   if (hp->total < full.pub.total) hp->total = full.pub.total;
+}
+
+// Status word of host-buffer chunk c: word c of the 16-byte status block at
+// the start of the workspace (chunk 0's workspace), one word per chunk.
+int* chunk_status(void* ws, const HostioPlan& hp, int c) {
+  static_assert(kHostioChunks * sizeof(int) <= 16, "chunk status words fit the status block");
+  return reinterpret_cast<int*>(static_cast<uint8_t*>(ws) + hp.sub.pub.status) + c;
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
@@ -263,17 +276,40 @@ moe_status launch_routing(const uint16_t* x, const float* W_r, const float* b_r,
 // The forward pass on the caller's stream. resid (optional, [T][d] bf16) is
 // added to the layer output before its rounding to bf16; gu_bias ([E][2I]) and
 // dn_bias ([E][d]), each optional, are the experts' projection biases.
+// What a forward call may choose besides its tensors: the tile policy (as
+// moe_set_tile_policy; the process default for the entry points without
+// options), the experts' optional biases, and where the status word lives
+// (null: the workspace's own).
+struct FwdOpts {
+  int policy;
+  int act;                 // moe::ACT_HILO (bf16 precision), ACT_E4M3 or ACT_E2M1
+  const float* gu_bias;
+  const float* dn_bias;
+  int* status;
+};
+
+FwdOpts default_opts() {
+  FwdOpts o;
+  o.policy = g_tile_policy.load(std::memory_order_relaxed);
+  o.act = moe::ACT_HILO;
+  o.gu_bias = nullptr;
+  o.dn_bias = nullptr;
+  o.status = nullptr;
+  return o;
+}
+
 moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, const uint8_t* gc,
                        const uint8_t* gs, const uint8_t* dc, const uint8_t* ds, int E, int k,
                        int T, int d, int I, uint16_t* out, void* ws, const Layout& L,
-                       cudaStream_t st, int num_sms, const StageEvents* tev = nullptr,
-                       const uint16_t* resid = nullptr, const float* gu_bias = nullptr,
-                       const float* dn_bias = nullptr) {
+                       cudaStream_t st, int num_sms, const FwdOpts& opt,
+                       const StageEvents* tev = nullptr, const uint16_t* resid = nullptr) {
   StageEvents none;
   memset(&none, 0, sizeof(none));
   const StageEvents& E_ = tev ? *tev : none;
+  const float* gu_bias = opt.gu_bias;
+  const float* dn_bias = opt.dn_bias;
   const int P = T * k;
-  int* status = at<int>(ws, L.pub.status);
+  int* status = opt.status ? opt.status : at<int>(ws, L.pub.status);
   float* logits = at<float>(ws, L.pub.logits);
   int32_t* topk_idx = at<int32_t>(ws, L.pub.topk_idx);
   float* topk_w = at<float>(ws, L.pub.topk_w);
@@ -292,16 +328,78 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   moe_status rs = launch_routing(x, W_r, b_r, E, k, T, d, logits, topk_idx, topk_w, counts,
                                  offsets, mprefix, chunk_hist, chunk_base, perm, status, st, E_);
   if (rs != MOE_OK) return rs;
-  const int tiles = choose_tiles(P, E, mx_shape_ok(d, I) && aligned32(gc) && aligned32(dc));
-  if (tiles == moe::TILES_MX) {
+  const int tiles = opt.act != moe::ACT_HILO
+                        ? moe::TILES_MX
+                        : choose_tiles(opt.policy, P, E,
+                                       mx_shape_ok(d, I) && aligned32(gc) && aligned32(dc));
+  if (opt.act != moe::ACT_HILO) {
+    // quantised activations (w4a8, w4a4): one MX-converted row per routed
+    // pair, the same block-scaled kernels with a one-term B operand
+    uint8_t* qx = at<uint8_t>(ws, L.pub.xp);
+    uint8_t* qh = at<uint8_t>(ws, L.pub.h);
+    uint8_t* sfbx = at<uint8_t>(ws, L.gu_scales_t);
+    uint8_t* sfbh = at<uint8_t>(ws, L.d_scales_t);
+    // few rows per expert: 16-token tiles; else 128-token tiles, on a CTA
+    // pair when the policy asks for it
+    const int variant = P < 64 * E ? moe::kMxSmall
+                                   : (opt.policy == 5 ? moe::kMxPair : moe::kMxLarge);
+    MOE_CUDA(moe::launch_mx_act_quant_gather(variant, opt.act, x, perm, offsets, E, P, k, d, qx,
+                                             sfbx, st));
+    E_.mark(6);
+    E_.mark(7);
+    E_.mark(8);
+    moe::MxGemmProblem m1;
+    memset(&m1, 0, sizeof(m1));
+    m1.codes = gc;
+    m1.scales = gs;
+    m1.b_hi = qx;
+    m1.b_sfb = sfbx;
+    m1.offsets = offsets;
+    m1.P = P;
+    m1.E = E;
+    m1.K = d;
+    m1.I = I;
+    m1.tok_rows = static_cast<int>(L.mx_tok_rows);
+    m1.h_hi = qh;
+    m1.h_sfb = sfbh;
+    m1.n_out = I;
+    m1.status = status;
+    m1.bias = gu_bias;
+    m1.act = opt.act;
+    MOE_CUDA(variant == moe::kMxPair ? moe::launch_mx_pair_gateup_swiglu(m1, num_sms, st)
+                                     : moe::launch_mx_gemm_gateup_swiglu(variant, m1, num_sms, st));
+    E_.mark(9);
+    moe::MxGemmProblem m2 = m1;
+    m2.codes = dc;
+    m2.scales = ds;
+    m2.b_hi = qh;
+    m2.b_sfb = sfbh;
+    m2.K = I;
+    m2.h_hi = nullptr;
+    m2.h_sfb = nullptr;
+    m2.out_f32 = yw;
+    m2.perm = perm;
+    m2.topk_w = topk_w;
+    m2.n_out = d;
+    m2.bias = dn_bias;
+    MOE_CUDA(variant == moe::kMxPair ? moe::launch_mx_pair_down(m2, num_sms, st)
+                                     : moe::launch_mx_gemm_down(variant, m2, num_sms, st));
+    E_.mark(10);
+    MOE_CUDA(moe::launch_combine(yw, T, k, d, resid, out, st));
+    E_.mark(11);
+    return MOE_OK;
+  }
+  if (tiles == moe::TILES_MX || tiles == moe::TILES_MX_PAIR) {
     // block-scaled path: hi/lo token rows, no scale transposes
     const size_t tr = L.mx_tok_rows;
     uint8_t* qx = at<uint8_t>(ws, L.pub.xp);
     uint8_t* qh = at<uint8_t>(ws, L.pub.h);
     uint8_t* sfbx = at<uint8_t>(ws, L.gu_scales_t);
     uint8_t* sfbh = at<uint8_t>(ws, L.d_scales_t);
-    // 16-token tiles while experts average under 64 rows, else 120-token tiles
-    const int variant = P < 64 * E ? moe::kMxSmall : moe::kMxLarge;
+    // 16-token tiles while experts average under 64 rows, else 120-token
+    // tiles, or 256-token tiles on a CTA pair
+    const int variant = tiles == moe::TILES_MX_PAIR ? moe::kMxPair
+                                                    : (P < 64 * E ? moe::kMxSmall : moe::kMxLarge);
     MOE_CUDA(moe::launch_mx_quant_gather(variant, x, perm, offsets, E, P, k, d, qx, qx + tr * d,
                                          sfbx, st));
     E_.mark(6);
@@ -326,7 +424,8 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     m1.n_out = I;
     m1.status = status;
     m1.bias = gu_bias;
-    MOE_CUDA(moe::launch_mx_gemm_gateup_swiglu(variant, m1, num_sms, st));
+    MOE_CUDA(variant == moe::kMxPair ? moe::launch_mx_pair_gateup_swiglu(m1, num_sms, st)
+                                     : moe::launch_mx_gemm_gateup_swiglu(variant, m1, num_sms, st));
     E_.mark(9);
     moe::MxGemmProblem m2 = m1;
     m2.codes = dc;
@@ -343,7 +442,8 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     m2.topk_w = topk_w;
     m2.n_out = d;
     m2.bias = dn_bias;
-    MOE_CUDA(moe::launch_mx_gemm_down(variant, m2, num_sms, st));
+    MOE_CUDA(variant == moe::kMxPair ? moe::launch_mx_pair_down(m2, num_sms, st)
+                                     : moe::launch_mx_gemm_down(variant, m2, num_sms, st));
     E_.mark(10);
     MOE_CUDA(moe::launch_combine(yw, T, k, d, resid, out, st));
     E_.mark(11);
@@ -416,8 +516,8 @@ const char* moe_status_string(moe_status s) {
 int moe_version(void) { return kVersion; }
 
 moe_status moe_set_tile_policy(int policy) {
-  if (policy < 0 || policy > 4) return MOE_ERR_INVALID_ARG;
-  g_tile_policy = policy;
+  if (policy < 0 || policy > 5) return MOE_ERR_INVALID_ARG;
+  g_tile_policy.store(policy, std::memory_order_relaxed);
   return MOE_OK;
 }
 
@@ -449,7 +549,9 @@ int moe_forward_launch_count(int E, int k, int T, int d, int I) {
   // small batches: the permutation in one launch instead of three
   if (T <= moe::kPermChunk) n -= 2;
   // the block-scaled path launches no scale transposes
-  if (choose_tiles(T * k, E, mx_shape_ok(d, I)) == moe::TILES_MX) n -= 2;
+  const int tiles =
+      choose_tiles(g_tile_policy.load(std::memory_order_relaxed), T * k, E, mx_shape_ok(d, I));
+  if (tiles == moe::TILES_MX || tiles == moe::TILES_MX_PAIR) n -= 2;
   return n;
 }
 
@@ -469,11 +571,41 @@ moe_status moe_forward_biased(const void* x_dev, const float* W_r_dev, const flo
                               const uint8_t* Wd_scales_dev, const float* down_bias_dev, int E,
                               int k, int T, int d, int I, void* out_dev, void* workspace_dev,
                               size_t workspace_bytes, void* stream) {
+  moe_forward_opts o;
+  memset(&o, 0, sizeof(o));
+  o.tile_policy = -1;
+  o.gu_bias_dev = gu_bias_dev;
+  o.down_bias_dev = down_bias_dev;
+  return moe_forward_ex(x_dev, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev, Wd_codes_dev,
+                        Wd_scales_dev, E, k, T, d, I, out_dev, workspace_dev, workspace_bytes, &o,
+                        stream);
+}
+
+moe_status moe_forward_ex(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
+                          const uint8_t* Wgu_codes_dev, const uint8_t* Wgu_scales_dev,
+                          const uint8_t* Wd_codes_dev, const uint8_t* Wd_scales_dev, int E, int k,
+                          int T, int d, int I, void* out_dev, void* workspace_dev,
+                          size_t workspace_bytes, const moe_forward_opts* opts, void* stream) {
   moe_status s = check_forward_args(x_dev, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev,
                                     Wd_codes_dev, Wd_scales_dev, E, k, T, d, I, out_dev,
                                     workspace_dev);
   if (s != MOE_OK) return s;
-  if (!aligned16(gu_bias_dev) || !aligned16(down_bias_dev)) return MOE_ERR_INVALID_ARG;
+  FwdOpts o = default_opts();
+  if (opts) {
+    if (opts->tile_policy < -1 || opts->tile_policy > 5) return MOE_ERR_INVALID_ARG;
+    if (opts->act_quant < MOE_ACT_BF16 || opts->act_quant > MOE_ACT_MXFP4)
+      return MOE_ERR_INVALID_ARG;
+    if (opts->act_quant != MOE_ACT_BF16) {
+      // the quantised modes run on the block-scaled tiles only
+      if (!mx_shape_ok(d, I) || !aligned32(Wgu_codes_dev) || !aligned32(Wd_codes_dev))
+        return MOE_ERR_UNSUPPORTED;
+      o.act = opts->act_quant == MOE_ACT_MXFP8 ? moe::ACT_E4M3 : moe::ACT_E2M1;
+    }
+    if (opts->tile_policy >= 0) o.policy = opts->tile_policy;
+    o.gu_bias = opts->gu_bias_dev;
+    o.dn_bias = opts->down_bias_dev;
+  }
+  if (!aligned16(o.gu_bias) || !aligned16(o.dn_bias)) return MOE_ERR_INVALID_ARG;
   Layout L;
   make_layout(E, k, T, d, I, false, &L);
   if (workspace_bytes < L.pub.total) return MOE_ERR_WORKSPACE;
@@ -483,8 +615,7 @@ moe_status moe_forward_biased(const void* x_dev, const float* W_r_dev, const flo
   return run_forward(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, Wgu_codes_dev,
                      Wgu_scales_dev, Wd_codes_dev, Wd_scales_dev, E, k, T, d, I,
                      static_cast<uint16_t*>(out_dev), workspace_dev, L,
-                     static_cast<cudaStream_t>(stream), num_sms, nullptr, nullptr, gu_bias_dev,
-                     down_bias_dev);
+                     static_cast<cudaStream_t>(stream), num_sms, o);
 }
 
 size_t moe_workspace_size_block(int E, int k, int T, int d, int I) {
@@ -531,9 +662,12 @@ moe_status moe_forward_block(const void* h_dev, const float* g_dev, float eps, c
   const uint16_t* h = static_cast<const uint16_t*>(h_dev);
   uint16_t* x = at<uint16_t>(workspace_dev, L.x_norm);
   MOE_CUDA(moe::launch_rms_norm(h, g_dev, eps, T, d, x, st));
+  FwdOpts o = default_opts();
+  o.gu_bias = gu_bias_dev;
+  o.dn_bias = down_bias_dev;
   return run_forward(x, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev, Wd_codes_dev,
                      Wd_scales_dev, E, k, T, d, I, static_cast<uint16_t*>(out_dev), workspace_dev,
-                     L, st, num_sms, nullptr, h, gu_bias_dev, down_bias_dev);
+                     L, st, num_sms, o, nullptr, h);
 }
 
 moe_status moe_forward_hostio(const void* x_host, const float* W_r_dev, const float* b_r_dev,
@@ -556,11 +690,12 @@ moe_status moe_forward_hostio(const void* x_host, const float* W_r_dev, const fl
   uint16_t* out_buf = at<uint16_t>(workspace_dev, hp.out_buf);
   const uint16_t* xh = static_cast<const uint16_t*>(x_host);
   uint16_t* oh = static_cast<uint16_t*>(out_host);
+  const FwdOpts o = default_opts();
   if (hp.chunks == 1) {
     const size_t bytes = static_cast<size_t>(T) * d * 2;
     MOE_CUDA(cudaMemcpyAsync(x_in, xh, bytes, cudaMemcpyHostToDevice, st));
     s = run_forward(x_in, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev, Wd_codes_dev,
-                    Wd_scales_dev, E, k, T, d, I, out_buf, workspace_dev, hp.sub, st, num_sms);
+                    Wd_scales_dev, E, k, T, d, I, out_buf, workspace_dev, hp.sub, st, num_sms, o);
     if (s != MOE_OK) return s;
     MOE_CUDA(cudaMemcpyAsync(oh, out_buf, bytes, cudaMemcpyDeviceToHost, st));
   } else {
@@ -591,44 +726,59 @@ moe_status moe_forward_hostio(const void* x_host, const float* W_r_dev, const fl
       }
       have[dev] = true;
     }
+    // Every error exit below first waits for the copies already enqueued on
+    // the copy streams, so that none lands in the caller's host buffers after
+    // the call has returned.
+    auto drained = [&](moe_status err) {
+      cudaGetLastError();
+      cudaStreamSynchronize(r.h2d);
+      cudaStreamSynchronize(r.d2h);
+      cudaGetLastError();
+      return err;
+    };
+#define MOE_CUDA_CHUNKED(call) \
+  do {                                          \
+    if ((call) != cudaSuccess) return drained(MOE_ERR_CUDA); \
+  } while (0)
     // nothing of this call touches the workspace before the caller's earlier work on st
-    MOE_CUDA(cudaEventRecord(r.start, st));
-    MOE_CUDA(cudaStreamWaitEvent(r.h2d, r.start, 0));
+    MOE_CUDA_CHUNKED(cudaEventRecord(r.start, st));
+    MOE_CUDA_CHUNKED(cudaStreamWaitEvent(r.h2d, r.start, 0));
     for (int c = 0; c < hp.chunks; ++c) {
       const int t0 = c * hp.Tc;
       const int tn = T - t0 < hp.Tc ? T - t0 : hp.Tc;
       if (tn <= 0) break;
       const size_t off = static_cast<size_t>(t0) * d;
       const size_t bytes = static_cast<size_t>(tn) * d * 2;
-      MOE_CUDA(cudaMemcpyAsync(x_in + off, xh + off, bytes, cudaMemcpyHostToDevice, r.h2d));
-      MOE_CUDA(cudaEventRecord(r.in[c], r.h2d));
-      MOE_CUDA(cudaStreamWaitEvent(st, r.in[c], 0));
-      // chunks c and c+2 share a workspace; both run in order on st
+      MOE_CUDA_CHUNKED(cudaMemcpyAsync(x_in + off, xh + off, bytes, cudaMemcpyHostToDevice, r.h2d));
+      MOE_CUDA_CHUNKED(cudaEventRecord(r.in[c], r.h2d));
+      MOE_CUDA_CHUNKED(cudaStreamWaitEvent(st, r.in[c], 0));
+      // chunks c and c+2 share a workspace (both run in order on st), but
+      // each chunk records its device status in a word of its own, so that a
+      // later chunk's router, which clears its word, cannot erase an earlier
+      // chunk's timeout before the host reads it
       void* ws = static_cast<uint8_t*>(workspace_dev) + (c & 1) * hp.sub_stride;
+      FwdOpts oc = o;
+      oc.status = chunk_status(workspace_dev, hp, c);
       s = run_forward(x_in + off, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev, Wd_codes_dev,
-                      Wd_scales_dev, E, k, tn, d, I, out_buf + off, ws, hp.sub, st, num_sms);
-      if (s != MOE_OK) {
-        // no copy of an earlier chunk may land after the call has returned
-        cudaStreamSynchronize(r.h2d);
-        cudaStreamSynchronize(r.d2h);
-        return s;
-      }
-      MOE_CUDA(cudaEventRecord(r.fwd[c], st));
-      MOE_CUDA(cudaStreamWaitEvent(r.d2h, r.fwd[c], 0));
-      MOE_CUDA(cudaMemcpyAsync(oh + off, out_buf + off, bytes, cudaMemcpyDeviceToHost, r.d2h));
+                      Wd_scales_dev, E, k, tn, d, I, out_buf + off, ws, hp.sub, st, num_sms, oc);
+      if (s != MOE_OK) return drained(s);
+      MOE_CUDA_CHUNKED(cudaEventRecord(r.fwd[c], st));
+      MOE_CUDA_CHUNKED(cudaStreamWaitEvent(r.d2h, r.fwd[c], 0));
+      MOE_CUDA_CHUNKED(
+          cudaMemcpyAsync(oh + off, out_buf + off, bytes, cudaMemcpyDeviceToHost, r.d2h));
     }
-    MOE_CUDA(cudaEventRecord(r.done, r.d2h));
-    MOE_CUDA(cudaStreamWaitEvent(st, r.done, 0));
+    MOE_CUDA_CHUNKED(cudaEventRecord(r.done, r.d2h));
+    MOE_CUDA_CHUNKED(cudaStreamWaitEvent(st, r.done, 0));
+#undef MOE_CUDA_CHUNKED
   }
   MOE_CUDA(cudaStreamSynchronize(st));
-  // status words: one per (chunk) workspace
-  for (int w = 0; w < (hp.chunks > 1 ? 2 : 1); ++w) {
-    int dev_status = 0;
-    MOE_CUDA(cudaMemcpy(&dev_status,
-                        static_cast<uint8_t*>(workspace_dev) + w * hp.sub_stride + hp.sub.pub.status,
-                        sizeof(int), cudaMemcpyDeviceToHost));
-    if (dev_status) return static_cast<moe_status>(dev_status);
-  }
+  // the status word of every chunk (one for an unchunked call); a timeout in
+  // any chunk is the call's result
+  int words[kHostioChunks] = {0, 0, 0, 0};
+  MOE_CUDA(cudaMemcpy(words, chunk_status(workspace_dev, hp, 0), sizeof(int) * hp.chunks,
+                      cudaMemcpyDeviceToHost));
+  for (int c = 0; c < hp.chunks; ++c)
+    if (words[c]) return static_cast<moe_status>(words[c]);
   return MOE_OK;
 }
 
@@ -678,7 +828,8 @@ moe_status moe_forward_timed_events(const void* x_dev, const float* W_r_dev, con
   }
   s = run_forward(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, Wgu_codes_dev,
                   Wgu_scales_dev, Wd_codes_dev, Wd_scales_dev, E, k, T, d, I,
-                  static_cast<uint16_t*>(out_dev), workspace_dev, L, tev.st, num_sms, &tev);
+                  static_cast<uint16_t*>(out_dev), workspace_dev, L, tev.st, num_sms,
+                  default_opts(), &tev);
   if (s == MOE_OK && cudaEventSynchronize(tev.ev[kStages]) == cudaSuccess) {
     // a recorded boundary's entry spans to the next recorded boundary
     for (int i = 0; i < kStages; ++i) {
@@ -764,47 +915,19 @@ moe_status moe_mx_split_e4m3(const void* x_dev, int rows, int K, uint8_t* hi_dev
   return MOE_OK;
 }
 
-moe_status moe_probe_tensor_rate(int kind, int N, int per_commit, double* mac_per_clk_sm,
-                                 void* stream) {
-  if (!mac_per_clk_sm || (kind != 0 && kind != 1) || N < 16 || N > 256 || N % 16 ||
-      per_commit < 4 || per_commit > 64 || per_commit % 4)
-    return MOE_ERR_INVALID_ARG;
+moe_status moe_mx_quantize(const void* x_dev, int rows, int K, int act_quant, uint8_t* q_dev,
+                           uint8_t* scales_dev, void* stream) {
+  if (!x_dev || !q_dev || !scales_dev || rows < 0 || K < 32 || K % 32) return MOE_ERR_INVALID_ARG;
+  if (act_quant != MOE_ACT_MXFP8 && act_quant != MOE_ACT_MXFP4) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_dev) || !aligned16(q_dev)) return MOE_ERR_INVALID_ARG;
+  if (rows == 0) return MOE_OK;
   int num_sms = 0;
   moe_status s = device_info(&num_sms);
   if (s != MOE_OK) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  unsigned long long* d_cycles = nullptr;
-  const size_t bytes = static_cast<size_t>(num_sms) * 8 + 16;
-  MOE_CUDA(cudaMalloc(&d_cycles, bytes));
-  int* d_status = reinterpret_cast<int*>(d_cycles + num_sms);
-  moe_status r = MOE_OK;
-  if (cudaMemsetAsync(d_cycles, 0, bytes, st) != cudaSuccess ||
-      moe::launch_tensor_rate_probe(kind, N, per_commit, num_sms, d_cycles, d_status, st) !=
-          cudaSuccess ||
-      cudaStreamSynchronize(st) != cudaSuccess) {
-    cudaGetLastError();
-    r = MOE_ERR_CUDA;
-  }
-  unsigned long long* h = new unsigned long long[num_sms + 2];
-  if (r == MOE_OK && cudaMemcpy(h, d_cycles, bytes, cudaMemcpyDeviceToHost) != cudaSuccess) {
-    cudaGetLastError();
-    r = MOE_ERR_CUDA;
-  }
-  if (r == MOE_OK) {
-    const int status = *reinterpret_cast<int*>(h + num_sms);
-    unsigned long long worst = 0;
-    for (int i = 0; i < num_sms; ++i) worst = h[i] > worst ? h[i] : worst;
-    if (status || worst == 0) {
-      r = status ? static_cast<moe_status>(status) : MOE_ERR_CUDA;
-    } else {
-      const double k = kind == 1 ? 32.0 : 16.0;
-      const double macs = static_cast<double>(moe::tensor_rate_probe_iters()) * per_commit * 128.0 * N * k;
-      *mac_per_clk_sm = macs / static_cast<double>(worst);
-    }
-  }
-  delete[] h;
-  cudaFree(d_cycles);
-  return r;
+  MOE_CUDA(moe::launch_mx_act_quant_rows(act_quant == MOE_ACT_MXFP8 ? moe::ACT_E4M3 : moe::ACT_E2M1,
+                                         static_cast<const uint16_t*>(x_dev), rows, K, q_dev,
+                                         scales_dev, static_cast<cudaStream_t>(stream)));
+  return MOE_OK;
 }
 
 moe_status moe_sync_status(void* workspace_dev, size_t workspace_bytes, void* stream) {

@@ -92,11 +92,25 @@ cudaError_t launch_gemm_down_combine(const GroupedGemmProblem& p, int num_sms, c
 // K/32 bytes, are staged in shared memory).
 constexpr int kMxMaxK = 3072;
 constexpr int TILES_MX = 4;       // block-scaled tcgen05 GEMMs (E2M1 x hi/lo E4M3)
+constexpr int TILES_MX_PAIR = 5;  // the same on a CTA pair (cta_group::2, 256-token tiles)
 // Tile variants: small (16-token tiles, two CTAs per SM, two UMMA issuers
 // each; few rows per expert) and large (120-token tiles, one CTA per SM).
 constexpr int kMxSmall = 0;
 constexpr int kMxLarge = 1;
-int mx_tile_tokens(int variant);
+// CTA-pair variant (moe_mx_pair.cu): 256-token tiles on a 2-CTA cluster,
+// tokens as the UMMA A operand (M = 256); token rows padded to 128.
+constexpr int kMxPair = 2;
+int mx_tile_tokens(int variant, int act);
+
+// Activation operand of the block-scaled GEMMs (the B operand: token rows of x
+// for gate/up, of H for down), per group of 32 along K:
+//   ACT_HILO  bf16 precision: two E4M3 terms (hi, lo) with E8M0 scales
+//   ACT_E4M3  the w4a8 layer: one E4M3 element, OCP MX scale (emax 8)
+//   ACT_E2M1  the w4a4 layer: one E2M1 element, OCP MX scale (emax 2), rows
+//             packed two elements per byte (low nibble first)
+constexpr int ACT_HILO = 0;
+constexpr int ACT_E4M3 = 1;
+constexpr int ACT_E2M1 = 2;
 
 // Rows of the padded token layout (each expert's rows rounded up to a
 // multiple of the tile's tokens) and bytes of its B-scale blocks, for either
@@ -109,6 +123,16 @@ size_t mx_sfb_bytes(int P, int E, int K);
 cudaError_t launch_mx_quant_gather(int variant, const uint16_t* x, const int32_t* perm,
                                    const int32_t* offsets, int E, int P, int k, int K, uint8_t* qhi,
                                    uint8_t* qlo, uint8_t* sfb, cudaStream_t st);
+// The same for the quantised activation modes (act ACT_E4M3 or ACT_E2M1): one
+// MX-converted row per routed pair (K bytes, or K/2 for E2M1) plus its
+// B-scale blocks.
+cudaError_t launch_mx_act_quant_gather(int variant, int act, const uint16_t* x,
+                                       const int32_t* perm, const int32_t* offsets, int E, int P,
+                                       int k, int K, uint8_t* q, uint8_t* sfb, cudaStream_t st);
+// The MX conversion on plain rows: q [R][K] (E4M3) or [R][K/2] (E2M1, packed),
+// scales [R][K/32] E8M0.
+cudaError_t launch_mx_act_quant_rows(int act, const uint16_t* x, int R, int K, uint8_t* q,
+                                     uint8_t* scales, cudaStream_t st);
 // The same split on plain rows, scales as [R][K/32][2] (hi byte, lo byte).
 cudaError_t launch_mx_split_rows(const uint16_t* x, int R, int K, uint8_t* qhi, uint8_t* qlo,
                                  uint8_t* scales, cudaStream_t st);
@@ -133,17 +157,24 @@ struct MxGemmProblem {
   int n_out;                // I for SwiGLU, d for down
   int* status;
   const float* bias;        // optional, as in GroupedGemmProblem
+  int act;                  // ACT_HILO, ACT_E4M3 or ACT_E2M1 (b_lo / h_lo unused but HILO)
 };
 cudaError_t launch_mx_gemm_gateup_swiglu(int variant, const MxGemmProblem& p, int num_sms,
                                          cudaStream_t st);
 cudaError_t launch_mx_gemm_down(int variant, const MxGemmProblem& p, int num_sms, cudaStream_t st);
+// The CTA-pair variant (moe_mx_pair.cu): same problem description; token rows
+// and their scale blocks in the 128-row padded layout.
+cudaError_t launch_mx_pair_gateup_swiglu(const MxGemmProblem& p, int num_sms, cudaStream_t st);
+cudaError_t launch_mx_pair_down(const MxGemmProblem& p, int num_sms, cudaStream_t st);
 
-// Tensor-core rate probe (moe_probe.cu): one CTA per SM issues UMMAs of the
-// given kind (0: bf16 kind::f16, K = 16; 1: block-scaled E2M1 x E4M3, K = 32)
-// with M = 128 and N columns, per_commit per commit; cycles[sm] = clock64 span.
-cudaError_t launch_tensor_rate_probe(int kind, int N, int per_commit, int num_sms,
-                                     unsigned long long* cycles, int* status, cudaStream_t st);
-int tensor_rate_probe_iters();
+// Tensor maps of the block-scaled path (moe_mx_gemm.cu): E2M1 code rows
+// (main map over whole 128-element k-blocks plus a tail map for [K-128, K)),
+// E4M3 token rows as two planes (hi, lo) or one.
+bool mx_make_code_maps(CUtensorMap* main_map, CUtensorMap* tail_map, const uint8_t* codes, int K,
+                       int rank, const cuuint64_t* dims_rest, const cuuint64_t* strides,
+                       const cuuint32_t* box_rest);
+bool mx_make_tok8_map(CUtensorMap* m, const uint8_t* hi, int rows, int K, int nt);
+bool mx_make_tok8_map1(CUtensorMap* m, const uint8_t* q, int rows, int K, int nt);
 
 // Debug/self-test: one bounded wait on an mbarrier that nothing completes.
 cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t st);

@@ -91,7 +91,11 @@ __device__ __forceinline__ int sfb_offset(int NT, int n, int h, int kk) {
   return (w >> 2) * 512 + (c & 31) * 16 + (w & 3) * 4 + kk;
 }
 
-__host__ __device__ constexpr int sfb_block_bytes(int NT) { return 512 * ((2 * NT + 127) / 128); }
+// Bytes of one B-scale block: one 512-byte tcgen05.cp atom per 128 UMMA B
+// columns (terms x NT: hi and lo columns of the bf16 split, one set otherwise).
+__host__ __device__ constexpr int sfb_block_bytes(int NT, int terms = 2) {
+  return 512 * ((terms * NT + 127) / 128);
+}
 
 // Splits 32 fp32 values (already bf16-exact) into hi / lo E4M3 bytes given the
 // group's max |v|; returns the hi scale byte (lo's is 4 less).
@@ -127,6 +131,75 @@ __device__ __forceinline__ uint32_t split_group32(const float (&v)[32], float am
 }
 
 __device__ __forceinline__ float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
+
+// ------------------------------------------- MX conversion (w4a8, w4a4) ----
+// The OCP Microscaling conversion of one group of 32 values: shared scale
+// X = 2^(floor(log2 max|v|) - emax), emax 8 for E4M3 and 2 for E2M1;
+// elements v / X rounded to the nearest element value (ties to even),
+// magnitudes above the largest normal (448, 6) clamped to it. X's exponent is
+// kept in the E8M0 range (at least -127: groups whose max|v| is below
+// 2^(emax - 127) keep that smallest scale); an all-zero group takes X = 1.
+template <int ACT>
+__device__ __forceinline__ int mx_scale_exp(float amax) {
+  constexpr int emax = ACT == ACT_E2M1 ? 2 : 8;
+  if (!(amax > 0.f)) return 0;
+  const int e = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127;  // floor(log2)
+  return max(e - emax, -127);
+}
+
+// 32 values -> element codes: E4M3 bytes in w[0..7] (element i in byte i),
+// or E2M1 codes packed two per byte in w[0..3] (element 2i in the low nibble
+// of byte i). Returns the E8M0 scale byte.
+template <int ACT>
+__device__ __forceinline__ uint32_t mx_quant_group32(const float (&v)[32], float amax,
+                                                     uint32_t (&w)[8]) {
+  const int x = mx_scale_exp<ACT>(amax);
+  const float inv = __uint_as_float(static_cast<uint32_t>(127 - x) << 23);   // 2^-x
+  if (ACT == ACT_E4M3) {
+#pragma unroll
+    for (int q = 0; q < 8; ++q)
+      w[q] = f32x2_to_e4m3x2(v[4 * q] * inv, v[4 * q + 1] * inv) |
+             (f32x2_to_e4m3x2(v[4 * q + 2] * inv, v[4 * q + 3] * inv) << 16);
+  } else {
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t a = 0;
+#pragma unroll
+      for (int b = 0; b < 4; ++b)
+        a |= f32x2_to_e2m1x2(v[8 * q + 2 * b] * inv, v[8 * q + 2 * b + 1] * inv) << (8 * b);
+      w[q] = a;
+    }
+#pragma unroll
+    for (int q = 4; q < 8; ++q) w[q] = 0;
+  }
+  return static_cast<uint32_t>(x + 127);
+}
+
+// 32 bf16 values at src (16-byte aligned) -> fp32 and their max |v|.
+__device__ __forceinline__ float load_group32(const uint16_t* src16, float (&v)[32]) {
+  const uint4* src = reinterpret_cast<const uint4*>(src16);
+  float amax = 0.f;
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 w = __ldg(src + c);
+    const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      v[8 * c + 2 * u] = bf16_bits_to_f32(ww[u] & 0xFFFFu);
+      v[8 * c + 2 * u + 1] = bf16_bits_to_f32(ww[u] >> 16);
+      amax = fmaxf(amax, fmaxf(fabsf(v[8 * c + 2 * u]), fabsf(v[8 * c + 2 * u + 1])));
+    }
+  }
+  return amax;
+}
+
+// Stores one converted group: 32 bytes (E4M3) or 16 bytes (E2M1) at dst.
+template <int ACT>
+__device__ __forceinline__ void store_group32(uint8_t* dst, const uint32_t (&w)[8]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+  if (ACT == ACT_E4M3) d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+}
 
 // One thread per (permuted row, group of 32): gathers x[token] into the padded
 // token layout as hi / lo E4M3 rows and writes the B scale blocks.
@@ -230,6 +303,73 @@ __global__ void __launch_bounds__(256) mx_split_rows_kernel(const uint16_t* __re
   }
 }
 
+// One thread per (permuted row, group of 32) for the quantised activation
+// modes: x[token] -> one MX-converted row in the padded token layout (K bytes,
+// or K/2 for E2M1) and its scale byte in the B-scale blocks.
+template <int NT, int ACT>
+__global__ void __launch_bounds__(256) mx_act_quant_gather_kernel(
+    const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
+    const int32_t* __restrict__ offsets, int E, int P, int k, int K, uint8_t* __restrict__ q,
+    uint8_t* __restrict__ sfb) {
+  __shared__ int s_off[kMaxE + 1], s_tb[kMaxE + 1];
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) s_off[i] = offsets[i];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int a = 0;
+    for (int e = 0; e < E; ++e) {
+      s_tb[e] = a;
+      a += (s_off[e + 1] - s_off[e] + NT - 1) / NT;
+    }
+    s_tb[E] = a;
+  }
+  __syncthreads();
+  const int G = K / 32, KB = (K + 127) / 128;
+  constexpr int SFB = sfb_block_bytes(NT, 1);
+  constexpr int GB = ACT == ACT_E2M1 ? 16 : 32;     // bytes of one converted group
+  const size_t row_bytes = static_cast<size_t>(G) * GB;
+  const int64_t n = static_cast<int64_t>(P) * G;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int p = static_cast<int>(i / G), g = static_cast<int>(i % G);
+    int lo_e = 0, hi_e = E;   // largest e with s_off[e] <= p
+    while (hi_e - lo_e > 1) {
+      const int mid = (lo_e + hi_e) >> 1;
+      if (s_off[mid] <= p) lo_e = mid; else hi_e = mid;
+    }
+    const int e = lo_e;
+    const int pr = s_tb[e] * NT + (p - s_off[e]);
+    const int t = perm[p] / k;
+    float v[32];
+    const float amax = load_group32(x + static_cast<size_t>(t) * K + 32 * g, v);
+    uint32_t w[8];
+    const uint32_t sx = mx_quant_group32<ACT>(v, amax, w);
+    store_group32<ACT>(q + static_cast<size_t>(pr) * row_bytes + static_cast<size_t>(g) * GB, w);
+    int kb, kk;
+    group_to_kblock(g, G, KB, kb, kk);
+    uint8_t* blk = sfb + (static_cast<size_t>(pr / NT) * KB + kb) * SFB;
+    blk[sfb_offset(NT, pr % NT, 0, kk)] = static_cast<uint8_t>(sx);
+  }
+}
+
+// The MX conversion on plain rows: [R][K] bf16 -> q rows and scales [R][K/32].
+template <int ACT>
+__global__ void __launch_bounds__(256) mx_act_quant_rows_kernel(const uint16_t* __restrict__ x,
+                                                                int R, int K,
+                                                                uint8_t* __restrict__ q,
+                                                                uint8_t* __restrict__ scales) {
+  const int G = K / 32;
+  constexpr int GB = ACT == ACT_E2M1 ? 16 : 32;
+  const int64_t n = static_cast<int64_t>(R) * G;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float v[32];
+    const float amax = load_group32(x + i * 32, v);
+    uint32_t w[8];
+    scales[i] = static_cast<uint8_t>(mx_quant_group32<ACT>(v, amax, w));
+    store_group32<ACT>(q + i * GB, w);
+  }
+}
+
 // ------------------------------------------------------------ the GEMM ----
 
 enum Epi { EPI_SWIGLU = 0, EPI_DOWN = 1 };
@@ -237,19 +377,23 @@ enum Epi { EPI_SWIGLU = 0, EPI_DOWN = 1 };
 // NT tokens per tile, ISSUERS UMMA-issuing threads per CTA, CTAS CTAs per SM,
 // EPI_WARPS epilogue warps (groups of four, one per TMEM lane quarter; group
 // g takes every (EPI_WARPS/4)-th chunk of token columns).
-template <int NT_, int ISSUERS_, int CTAS_, int EPI_WARPS_>
+template <int NT_, int ISSUERS_, int CTAS_, int EPI_WARPS_, int ACT_ = ACT_HILO>
 struct MxCfg {
   static constexpr int NT = NT_;
   static constexpr int ISSUERS = ISSUERS_;
   static constexpr int CTAS = CTAS_;
   static constexpr int EPI_WARPS = EPI_WARPS_;
   static constexpr int EPI_GROUPS = EPI_WARPS / 4;
+  static constexpr int ACT = ACT_;                  // activation operand (ACT_*)
+  static constexpr int TERMS = ACT == ACT_HILO ? 2 : 1;
   static constexpr int MW = 128;                    // weight rows per tile
-  static constexpr int N = 2 * NT;                  // UMMA N: hi and lo token columns
+  static constexpr int N = TERMS * NT;              // UMMA N: (hi and lo) token columns
   static constexpr int A_BYTES = 128 * 128;         // E2M1 in 8-bit containers
   static constexpr int A_TX = 128 * 64;             // packed bytes the TMA counts
-  static constexpr int B_BYTES = N * 128;
-  static constexpr int SFB_BYTES = sfb_block_bytes(NT);
+  static constexpr int B_BYTES = N * 128;           // 8-bit elements (E2M1 widened by TMA)
+  static constexpr int B_TX = ACT == ACT_E2M1 ? N * 64 : B_BYTES;
+  static constexpr uint32_t BTYPE = ACT == ACT_E2M1 ? 5u : 0u;   // instruction B type
+  static constexpr int SFB_BYTES = sfb_block_bytes(NT, TERMS);
   static constexpr int OFF_B = A_BYTES;
   static constexpr int OFF_SFA = OFF_B + B_BYTES;
   static constexpr int OFF_SFB = OFF_SFA + 512;
@@ -272,8 +416,8 @@ struct MxCfg {
   // issuer's scale columns (A: 4, B: 4 per 512-byte atom)
   static constexpr int SF_COL0 = 2 * ISSUERS * N;
   static constexpr int SF_COLS = 4 + 4 * (SFB_BYTES / 512);
-  static constexpr int TX_BYTES = A_TX + B_BYTES + SFB_BYTES;
-  static_assert(NT % CH == 0 && N <= 256, "tile width");
+  static constexpr int TX_BYTES = A_TX + B_TX + SFB_BYTES;
+  static_assert(NT % CH == 0 && N <= 256 && N % 16 == 0, "tile width");
   static_assert(EPI_WARPS % 4 == 0 && EPI_GROUPS <= 4, "epilogue warps");
   static_assert(SF_COL0 + ISSUERS * SF_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(CTAS * (SMEM_ALLOC + 1024) <= 233472 && SMEM_ALLOC <= 232448, "shared memory");
@@ -286,6 +430,12 @@ struct MxCfg {
 // tile's 15 column chunks keeps pace with its UMMAs.
 using MxSmall = MxCfg<16, 2, 2, 4>;
 using MxLarge = MxCfg<120, 1, 1, 12>;
+// The quantised activation modes: one term, so 128-token tiles fill UMMA N =
+// 128 in the large variant (N must be a multiple of 16: 120 is not).
+template <int ACT> using MxSmallQ = MxCfg<16, 2, 2, 4, ACT>;
+template <int ACT> using MxLargeQ = MxCfg<128, 1, 1, 12, ACT>;
+// the largest token tile of any variant (the padded token layout's granule)
+constexpr int kMxMaxNT = 128;
 
 struct MxArgs {
   const int32_t* offsets;
@@ -314,7 +464,8 @@ template <int EPI, class C>
 __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
     grouped_mx_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmAt,
-                           const __grid_constant__ CUtensorMap tmB, const MxArgs args) {
+                           const __grid_constant__ CUtensorMap tmB,
+                           const __grid_constant__ CUtensorMap tmBt, const MxArgs args) {
   constexpr int NT = C::NT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -365,6 +516,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmAt);
     tma_prefetch_desc(&tmB);
+    if (C::ACT == ACT_E2M1) tma_prefetch_desc(&tmBt);
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(misc), C::TMEM_COLS);
@@ -450,7 +602,12 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
             tma_load_3d(st, am, ax, wb * 128, e, fb);
           }
           const int bx = last_tail ? K - 128 : kb * 128;
-          tma_load_3d(st + C::OFF_B, &tmB, bx, row_b, 0, fb);   // hi rows, then lo rows
+          if (C::ACT == ACT_HILO)
+            tma_load_3d(st + C::OFF_B, &tmB, bx, row_b, 0, fb);   // hi rows, then lo rows
+          else if (C::ACT == ACT_E4M3)
+            tma_load_2d(st + C::OFF_B, &tmB, bx, row_b, fb);
+          else   // packed E2M1 rows, widened like the weight codes (tail map for [K-128, K))
+            tma_load_2d(st + C::OFF_B, last_tail ? &tmBt : &tmB, last_tail ? 0 : kb * 128, row_b, fb);
           bulk_load(st + C::OFF_SFB,
                     args.sfb + (static_cast<size_t>(tok_tile) * KB + kb) * C::SFB_BYTES,
                     C::SFB_BYTES, fb);
@@ -509,7 +666,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
     // issuer's k-blocks are stepped over without touching their barriers.
     const int u = warp == 1 ? 0 : 1;
     if (lane == 0) {
-      const uint32_t idesc0 = idesc_mx_e2m1_e4m3(C::MW, C::N, 0, 0);
+      const uint32_t idesc0 = idesc_mx_e2m1(C::MW, C::N, 0, 0, C::BTYPE);
       const uint32_t sfa_t = tmem_base + C::SF_COL0 + u * C::SF_COLS, sfb_t = sfa_t + 4;
       int s = 0, ph = 0, it = 0, q = 0;
       bool ok = true;
@@ -606,15 +763,28 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
         for (int i = 0; i < CH; ++i) y[i] = 0.f;
         if (ok && c < rows) {
           uint32_t a[8], b[8];
-          if (use0) {
-            tmem_ld8x2_sync(t0 + c, t0 + NT + c, a, b);
+          if (C::TERMS == 2) {   // hi and lo products of the bf16 split
+            if (use0) {
+              tmem_ld8x2_sync(t0 + c, t0 + NT + c, a, b);
 #pragma unroll
-            for (int i = 0; i < CH; ++i) y[i] = __uint_as_float(a[i]) + __uint_as_float(b[i]);
-          }
-          if (use1) {
-            tmem_ld8x2_sync(t1 + c, t1 + NT + c, a, b);
+              for (int i = 0; i < CH; ++i) y[i] = __uint_as_float(a[i]) + __uint_as_float(b[i]);
+            }
+            if (use1) {
+              tmem_ld8x2_sync(t1 + c, t1 + NT + c, a, b);
 #pragma unroll
-            for (int i = 0; i < CH; ++i) y[i] += __uint_as_float(a[i]) + __uint_as_float(b[i]);
+              for (int i = 0; i < CH; ++i) y[i] += __uint_as_float(a[i]) + __uint_as_float(b[i]);
+            }
+          } else {
+            if (use0) {
+              tmem_ld8_sync(t0 + c, a);
+#pragma unroll
+              for (int i = 0; i < CH; ++i) y[i] = __uint_as_float(a[i]);
+            }
+            if (use1) {
+              tmem_ld8_sync(t1 + c, a);
+#pragma unroll
+              for (int i = 0; i < CH; ++i) y[i] += __uint_as_float(a[i]);
+            }
           }
         }
         if (EPI == EPI_SWIGLU) {
@@ -626,8 +796,12 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
             y[i] += bl;
             const float u = __shfl_xor_sync(0xFFFFFFFFu, y[i], 16);
             float hv = 0.f;
-            if (ok && jv && c + i < rows)
-              hv = __bfloat162float(__float2bfloat16_rn(silu_mx(y[i]) * u));
+            if (ok && jv && c + i < rows) {
+              hv = silu_mx(y[i]) * u;
+              // bf16 precision: H is a bf16 row (split exactly below); the
+              // quantised modes convert the fp32 value itself
+              if (C::ACT == ACT_HILO) hv = __bfloat162float(__float2bfloat16_rn(hv));
+            }
             y[i] = hv;
             float pm = fabsf(hv);
 #pragma unroll
@@ -637,7 +811,35 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
           // max |h| over the 32 j of a group: quarters 0+1 and 2+3 (named
           // barrier 1 + grp over the group's four warps)
           asm volatile("bar.sync %0, 128;" ::"r"(1 + grp) : "memory");
-          if (ok) {
+          if (ok && C::ACT != ACT_HILO) {
+            // one MX-converted element per H value: E4M3 bytes, or E2M1 codes
+            // packed in pairs (the even H column in the low nibble: lanes j
+            // and j + 1 are neighbours, the even one stores the byte)
+            const int gj = 2 * wb + (quad >> 1);
+            int kb4, kk4;
+            group_to_kblock(gj, args.I / 32, args.h_kb, kb4, kk4);
+            uint8_t* hsfb = args.h_sfb + (static_cast<size_t>(tok_tile) * args.h_kb + kb4) *
+                                             sfb_block_bytes(NT, 1);
+#pragma unroll
+            for (int i = 0; i < CH; ++i) {
+              const int t = c + i;
+              const float amax = fmaxf(xch[quad * CH + i], xch[(quad ^ 1) * CH + i]);
+              const int ex = mx_scale_exp<C::ACT>(amax);
+              const float a = y[i] * __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
+              const size_t row = static_cast<size_t>(tok_tile * NT + t);
+              if (C::ACT == ACT_E4M3) {
+                if (jv && t < rows)
+                  args.h_hi[row * args.I + j] = static_cast<uint8_t>(f32x2_to_e4m3x2(a, 0.f) & 0xFF);
+              } else {
+                const uint32_t code = f32_to_e2m1(a);
+                const uint32_t odd = __shfl_xor_sync(0xFFFFFFFFu, code, 1);
+                if (jv && t < rows && !(j & 1))
+                  args.h_hi[row * (args.I / 2) + j / 2] = static_cast<uint8_t>(code | (odd << 4));
+              }
+              if (t < rows && lane == 0 && !(quad & 1))
+                hsfb[sfb_offset(NT, t, 0, kk4)] = static_cast<uint8_t>(ex + 127);
+            }
+          } else if (ok) {
             const int gj = 2 * wb + (quad >> 1);
             int kb4, kk4;
             group_to_kblock(gj, args.I / 32, args.h_kb, kb4, kk4);
@@ -770,6 +972,14 @@ bool make_tok8_map(CUtensorMap* m, const uint8_t* hi, int rows, int K, int nt) {
   return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, hi, dims, strides, box);
 }
 
+// One plane of E4M3 token rows [rows][K]; box 128 x NT.
+bool make_tok8_map1(CUtensorMap* m, const uint8_t* q, int rows, int K, int nt) {
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(rows)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K)};
+  const cuuint32_t box[2] = {128, static_cast<cuuint32_t>(nt)};
+  return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, q, dims, strides, box);
+}
+
 template <int EPI, class C>
 cudaError_t launch_mx_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st) {
   constexpr int NT = C::NT;
@@ -786,8 +996,10 @@ cudaError_t launch_mx_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st)
     attr_set[dev] = true;
   }
   // the hi and lo token rows are read as the two planes of one tensor
-  if (p.b_lo != p.b_hi + static_cast<size_t>(p.tok_rows) * p.K) return cudaErrorInvalidValue;
-  CUtensorMap tmA, tmAt, tmB;
+  if (C::ACT == ACT_HILO && p.b_lo != p.b_hi + static_cast<size_t>(p.tok_rows) * p.K)
+    return cudaErrorInvalidValue;
+  if (p.act != C::ACT) return cudaErrorInvalidValue;
+  CUtensorMap tmA, tmAt, tmB, tmBt;
   const cuuint64_t rb = static_cast<cuuint64_t>(p.K / 2);
   bool ok;
   if (EPI == EPI_SWIGLU) {
@@ -805,7 +1017,19 @@ cudaError_t launch_mx_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st)
     const cuuint32_t box[2] = {128, 1};
     ok = make_code_maps(&tmA, &tmAt, p.codes, p.K, 3, dims, strides, box);
   }
-  ok = ok && make_tok8_map(&tmB, p.b_hi, p.tok_rows, p.K, NT);
+  if (C::ACT == ACT_HILO) {
+    ok = ok && make_tok8_map(&tmB, p.b_hi, p.tok_rows, p.K, NT);
+    tmBt = tmB;
+  } else if (C::ACT == ACT_E4M3) {
+    ok = ok && make_tok8_map1(&tmB, p.b_hi, p.tok_rows, p.K, NT);
+    tmBt = tmB;
+  } else {
+    // packed E2M1 token rows [tok_rows][K/2], widened to 8-bit containers
+    const cuuint64_t dims[1] = {static_cast<cuuint64_t>(p.tok_rows)};
+    const cuuint64_t strides[1] = {rb};
+    const cuuint32_t box[1] = {static_cast<cuuint32_t>(NT)};
+    ok = ok && make_code_maps(&tmB, &tmBt, p.b_hi, p.K, 2, dims, strides, box);
+  }
   if (!ok) return cudaErrorInvalidValue;
   MxArgs a;
   a.offsets = p.offsets;
@@ -836,7 +1060,7 @@ cudaError_t launch_mx_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st)
   if (tiles_bound < grid) grid = tiles_bound;
   if (grid < 1) grid = 1;
   grouped_mx_gemm_kernel<EPI, C><<<static_cast<int>(grid), C::NUM_THREADS, C::SMEM_ALLOC, st>>>(
-      tmA, tmAt, tmB, a);
+      tmA, tmAt, tmB, tmBt, a);
   return cudaGetLastError();
 }
 
@@ -850,18 +1074,36 @@ int grid_for_n(int64_t n, int per_thread_block, int cap) {
 
 }  // namespace
 
-int mx_tile_tokens(int variant) { return variant == kMxLarge ? MxLarge::NT : MxSmall::NT; }
+bool mx_make_code_maps(CUtensorMap* main_map, CUtensorMap* tail_map, const uint8_t* codes, int K,
+                       int rank, const cuuint64_t* dims_rest, const cuuint64_t* strides,
+                       const cuuint32_t* box_rest) {
+  return make_code_maps(main_map, tail_map, codes, K, rank, dims_rest, strides, box_rest);
+}
+bool mx_make_tok8_map(CUtensorMap* m, const uint8_t* hi, int rows, int K, int nt) {
+  return make_tok8_map(m, hi, rows, K, nt);
+}
+bool mx_make_tok8_map1(CUtensorMap* m, const uint8_t* q, int rows, int K, int nt) {
+  return make_tok8_map1(m, q, rows, K, nt);
+}
+
+int mx_tile_tokens(int variant, int act) {
+  if (variant == kMxPair) return kMxMaxNT;
+  if (act == ACT_HILO) return variant == kMxLarge ? MxLarge::NT : MxSmall::NT;
+  return variant == kMxLarge ? MxLargeQ<ACT_E4M3>::NT : MxSmallQ<ACT_E4M3>::NT;
+}
 
 size_t mx_tok_rows(int P, int E) {
-  const int nt = MxSmall::NT > MxLarge::NT ? MxSmall::NT : MxLarge::NT;
-  return static_cast<size_t>(P) + static_cast<size_t>(E) * (nt - 1);
+  static_assert(MxLarge::NT <= kMxMaxNT && MxLargeQ<ACT_E4M3>::NT <= kMxMaxNT, "granule");
+  return static_cast<size_t>(P) + static_cast<size_t>(E) * (kMxMaxNT - 1);
 }
 
 size_t mx_sfb_bytes(int P, int E, int K) {
   size_t best = 0;
-  for (int nt : {MxSmall::NT, MxLarge::NT}) {
-    const size_t tiles = (static_cast<size_t>(P) + nt - 1) / nt + E;
-    const size_t b = tiles * ((K + 127) / 128) * sfb_block_bytes(nt);
+  const int variants[5][2] = {{MxSmall::NT, 2}, {MxLarge::NT, 2}, {MxSmallQ<ACT_E4M3>::NT, 1},
+                              {MxLargeQ<ACT_E4M3>::NT, 1}, {kMxMaxNT, 2}};
+  for (const auto& v : variants) {
+    const size_t tiles = (static_cast<size_t>(P) + v[0] - 1) / v[0] + E;
+    const size_t b = tiles * ((K + 127) / 128) * sfb_block_bytes(v[0], v[1]);
     if (b > best) best = b;
   }
   return best;
@@ -872,12 +1114,51 @@ cudaError_t launch_mx_quant_gather(int variant, const uint16_t* x, const int32_t
                                    uint8_t* qlo, uint8_t* sfb, cudaStream_t st) {
   const int64_t n = static_cast<int64_t>(P) * (K / 32);
   const int grid = grid_for_n(n, 256, 148 * 8);
-  if (variant == kMxLarge)
+  if (variant == kMxPair)
+    mx_quant_gather_kernel<kMxMaxNT><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, qhi, qlo,
+                                                            sfb);
+  else if (variant == kMxLarge)
     mx_quant_gather_kernel<MxLarge::NT><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, qhi,
                                                                qlo, sfb);
   else
     mx_quant_gather_kernel<MxSmall::NT><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, qhi,
                                                                qlo, sfb);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mx_act_quant_gather(int variant, int act, const uint16_t* x,
+                                       const int32_t* perm, const int32_t* offsets, int E, int P,
+                                       int k, int K, uint8_t* q, uint8_t* sfb, cudaStream_t st) {
+  const int64_t n = static_cast<int64_t>(P) * (K / 32);
+  const int grid = grid_for_n(n, 256, 148 * 8);
+  constexpr int NS = MxSmallQ<ACT_E4M3>::NT, NL = MxLargeQ<ACT_E4M3>::NT;
+  static_assert(NL == kMxMaxNT, "the large and pair variants share the 128-row layout");
+  if (act == ACT_E4M3) {
+    if (variant != kMxSmall)
+      mx_act_quant_gather_kernel<NL, ACT_E4M3><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, q, sfb);
+    else
+      mx_act_quant_gather_kernel<NS, ACT_E4M3><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, q, sfb);
+  } else if (act == ACT_E2M1) {
+    if (variant != kMxSmall)
+      mx_act_quant_gather_kernel<NL, ACT_E2M1><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, q, sfb);
+    else
+      mx_act_quant_gather_kernel<NS, ACT_E2M1><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, q, sfb);
+  } else {
+    return cudaErrorInvalidValue;
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mx_act_quant_rows(int act, const uint16_t* x, int R, int K, uint8_t* q,
+                                     uint8_t* scales, cudaStream_t st) {
+  const int64_t n = static_cast<int64_t>(R) * (K / 32);
+  const int grid = grid_for_n(n, 256, 148 * 8);
+  if (act == ACT_E4M3)
+    mx_act_quant_rows_kernel<ACT_E4M3><<<grid, 256, 0, st>>>(x, R, K, q, scales);
+  else if (act == ACT_E2M1)
+    mx_act_quant_rows_kernel<ACT_E2M1><<<grid, 256, 0, st>>>(x, R, K, q, scales);
+  else
+    return cudaErrorInvalidValue;
   return cudaGetLastError();
 }
 
@@ -888,16 +1169,31 @@ cudaError_t launch_mx_split_rows(const uint16_t* x, int R, int K, uint8_t* qhi, 
   return cudaGetLastError();
 }
 
+template <int EPI>
+cudaError_t launch_mx_dispatch(int variant, const MxGemmProblem& p, int num_sms, cudaStream_t st) {
+  const bool large = variant == kMxLarge;
+  switch (p.act) {
+    case ACT_HILO:
+      return large ? launch_mx_impl<EPI, MxLarge>(p, num_sms, st)
+                   : launch_mx_impl<EPI, MxSmall>(p, num_sms, st);
+    case ACT_E4M3:
+      return large ? launch_mx_impl<EPI, MxLargeQ<ACT_E4M3>>(p, num_sms, st)
+                   : launch_mx_impl<EPI, MxSmallQ<ACT_E4M3>>(p, num_sms, st);
+    case ACT_E2M1:
+      return large ? launch_mx_impl<EPI, MxLargeQ<ACT_E2M1>>(p, num_sms, st)
+                   : launch_mx_impl<EPI, MxSmallQ<ACT_E2M1>>(p, num_sms, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
 cudaError_t launch_mx_gemm_gateup_swiglu(int variant, const MxGemmProblem& p, int num_sms,
                                          cudaStream_t st) {
-  return variant == kMxLarge ? launch_mx_impl<EPI_SWIGLU, MxLarge>(p, num_sms, st)
-                             : launch_mx_impl<EPI_SWIGLU, MxSmall>(p, num_sms, st);
+  return launch_mx_dispatch<EPI_SWIGLU>(variant, p, num_sms, st);
 }
 
 cudaError_t launch_mx_gemm_down(int variant, const MxGemmProblem& p, int num_sms,
                                 cudaStream_t st) {
-  return variant == kMxLarge ? launch_mx_impl<EPI_DOWN, MxLarge>(p, num_sms, st)
-                             : launch_mx_impl<EPI_DOWN, MxSmall>(p, num_sms, st);
+  return launch_mx_dispatch<EPI_DOWN>(variant, p, num_sms, st);
 }
 
 }  // namespace moe

@@ -1,0 +1,701 @@
+// moe_mx_pair.cu -- CTA-pair block-scaled expert GEMMs for experts with many
+// routed rows (prefill): tcgen05.mma.cta_group::2.kind::mxf8f6f4 with M = 256.
+//
+//   gate/up:  H[r, j] = silu(x_r . Wgate[e][j] + bg[e][j]) * (x_r . Wup[e][j] + bu[e][j])
+//   down:     Yw[pair(r), m] = p(pair(r)) * (H[r] . Wdown[e][m] + bd[e][m])
+//
+// Field guide "gpt-oss 20B", "03 Sparse Mixture of Experts" (SwiGLU experts,
+// weighted sum); "gpt-oss-20b and gpt-oss-120b", "Four-bit expert weights"
+// (E2M1 codes with one power-of-two scale per 32 weights).
+//
+// Operands. A is the expert's routed token rows (UMMA M = 256: 128 rows in
+// each CTA of the pair), B the expert's weight rows (E2M1 codes that TMA widens
+// to 8-bit containers; N = 2 NH, NH rows in each CTA). The tensor core applies
+// both E8M0 scale sets. With bf16-precision activations each token row comes as
+// two E4M3 terms (hi, lo; the split is exact for every element of at least
+// 2^-13 of its group's max) and each K step issues two UMMAs into the same
+// accumulator, one per term, over the same weight tile: the accumulator holds
+// x . w itself. The quantised modes (one E4M3 or E2M1 term) issue one.
+//
+// Tiles. 256 token rows x N weight rows, 128 K per shared-memory stage.
+//   gate/up: NH = 96: the even CTA holds gate rows j0..j0+95, the odd CTA the
+//            matching up rows, so accumulator column c (gate) and 96 + c (up)
+//            of a token's TMEM lane meet in one thread, and a tile's 96 H
+//            columns are three whole MX groups of 32 (the epilogue converts H
+//            for the down GEMM per group).
+//   down:    NH = 120: output columns n0..n0+239.
+// Token rows live in a padded layout (each expert's rows start at a multiple
+// of 128), so each CTA's half tile is one contiguous block of rows and its
+// scale block one contiguous run of bytes. A tile covers 256 rows of one
+// expert; when the expert's rows end inside the even CTA's half, the odd CTA
+// loads no token rows (its accumulator rows are never stored).
+//
+// Scale factors in tensor memory. Each CTA holds the A scales of its own 128
+// rows (one 512-byte tcgen05.cp atom per term: lane m % 32 of column m / 32)
+// and the B scales of all N columns (two atoms), at the same TMEM columns in
+// both CTAs; the even CTA's issuing thread copies them with
+// tcgen05.cp.cta_group::2, which moves each CTA's atom into its own TMEM.
+//
+// Roles (256 threads per CTA):
+//   warp 0   TMA producer: token rows (A) and their scale block, weight codes
+//            (B); the tile's weight-scale rows into a double buffer
+//   warp 1   TMEM allocation; in the even CTA the UMMA issuer
+//   warp 2   B-scale builder: the tile's weight scales -> two atoms per stage
+//   warp 3   in the odd CTA: relays "stage full" to the even CTA's issuer
+//   warps 4-7 epilogue (TMEM lane quarters 0..3: one token row per thread)
+// Every wait is bounded (moe_ptx.cuh): a stuck pipeline records a timeout in
+// the status word and the kernel exits.
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "moe_internal.h"
+#include "moe_ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kMaxE = 256;
+enum PairEpi { PAIR_SWIGLU = 0, PAIR_DOWN = 1 };
+
+// Byte of the scale of row (or column) c, K step kk, in a block of 512-byte
+// atoms: word c / 32 of lane c % 32, four words per lane per atom.
+__host__ __device__ __forceinline__ int atom_offset(int c, int kk) {
+  const int w = c >> 5;
+  return (w >> 2) * 512 + (c & 31) * 16 + (w & 3) * 4 + kk;
+}
+
+// Groups of 32 along K -> (k-block, K step) with the tail rule of the
+// block-scaled path: the last k-block of a K that is 64 mod 128 is [K-128, K).
+__host__ __device__ __forceinline__ void pair_group_to_kblock(int g, int G, int KB, int& kb,
+                                                              int& kk) {
+  if ((G % 4) == 0 || g < 4 * (KB - 1)) {
+    kb = g >> 2;
+    kk = g & 3;
+  } else {
+    kb = KB - 1;
+    kk = g - (G - 4);
+  }
+}
+
+constexpr int kPairSmemBudget = 232448 - 1024;   // opt-in maximum less alignment slack
+
+template <int EPI, int ACT>
+struct PairCfg {
+  static constexpr int TERMS = ACT == ACT_HILO ? 2 : 1;
+  static constexpr int MT = 128;                          // token rows per CTA
+  static constexpr int NH = EPI == PAIR_SWIGLU ? 96 : 120;  // weight rows per CTA
+  static constexpr int N = 2 * NH;                        // UMMA N
+  static constexpr int A_PLANE = MT * 128;                // one term, 8-bit elements
+  static constexpr int A_BYTES = TERMS * A_PLANE;
+  static constexpr int A_TX = ACT == ACT_E2M1 ? MT * 64 : A_BYTES;
+  static constexpr int B_BYTES = NH * 128;
+  static constexpr int B_TX = NH * 64;                    // packed code bytes
+  static constexpr int SFA_BYTES = 512 * TERMS;
+  static constexpr int SFB_BYTES = 1024;                  // N <= 256: two atoms
+  static constexpr int OFF_B = A_BYTES;
+  static constexpr int OFF_SFA = OFF_B + B_BYTES;
+  static constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
+  static constexpr int STAGE_BYTES = (OFF_SFB + SFB_BYTES + 1023) / 1024 * 1024;
+  static constexpr int TS_BYTES = N * (kMxMaxK / 32);     // a tile's weight-scale rows
+  static constexpr int FIXED = 2 * TS_BYTES + 3 * (kMaxE + 1) * 4 + 512;
+  static constexpr int STAGES_FIT = (kPairSmemBudget - FIXED) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+  static constexpr int OFF_TS = STAGES * STAGE_BYTES;
+  static constexpr int OFF_BAR = OFF_TS + 2 * TS_BYTES;
+  static constexpr int NUM_BARS = 3 * STAGES + 10;
+  static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
+  static constexpr int OFF_TAB = OFF_MISC + 16;
+  static constexpr int SMEM_BYTES = OFF_TAB + 3 * (kMaxE + 1) * 4;
+  static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
+  static constexpr int NUM_THREADS = 256;
+  static constexpr int EPI_WARPS = 4;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int ACC_COLS = N;                      // per accumulator buffer
+  static constexpr int SF_COL0 = 2 * N;                   // A scales (TERMS atoms), then B
+  static constexpr int TX_FULL = A_TX + B_TX + SFA_BYTES; // a stage with token rows
+  static constexpr uint32_t ATYPE = ACT == ACT_E2M1 ? 5u : 0u;   // E2M1 or E4M3
+  static_assert(STAGES >= 3, "pipeline depth");
+  static_assert(SF_COL0 + 4 * TERMS + 8 <= TMEM_COLS, "TMEM budget");
+  static_assert(SMEM_ALLOC <= 232448, "shared memory");
+  static_assert(OFF_B % 1024 == 0 && B_BYTES % 1024 == 0 && STAGE_BYTES % 1024 == 0, "swizzle");
+  static_assert(N % 16 == 0 && N <= 256, "UMMA N");
+};
+
+// Instruction descriptor: block-scaled kind::mxf8f6f4, A type atype (tokens),
+// B E2M1 (weights), E8M0 scales, K-major operands, fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_pair(int M, int N, uint32_t atype, uint32_t sf_id) {
+  return (sf_id << 4) | (atype << 7) | (5u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24) | (sf_id << 29);
+}
+
+__device__ __forceinline__ void umma_mx_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                             uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Shared memory -> TMEM in both CTAs of the pair (each CTA's atom at the same
+// shared-memory offset into its own TMEM), 32 lanes x 128 bits replicated into
+// the four lane quarters.
+__device__ __forceinline__ void tmem_cp_32x128b_x4_pair(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::2.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc)
+               : "memory");
+}
+
+struct PairArgs {
+  const int32_t* offsets;
+  int E, K, I;                // K: contraction; I: intermediate size
+  int n_out;                  // I (gate/up) or d (down)
+  int n_tiles;                // weight tiles per expert
+  int rows_per_expert;        // weight rows of an expert in the scale array (2I or d)
+  int KB;                     // k-blocks
+  const uint8_t* scales;      // [E][rows_per_expert][K/32] E8M0 weight scales
+  const uint8_t* sfa;         // token scale blocks [128-row tile][KB][SFA_BYTES]
+  // gate/up: converted H rows (h_lo: the lo plane of the bf16 split) and
+  // their scale blocks (the down GEMM's A operand)
+  uint8_t* h_q;
+  uint8_t* h_lo;
+  uint8_t* h_sfa;
+  int h_kb;
+  // down: weighted rows
+  float* out_f32;
+  const int32_t* perm;
+  const float* topk_w;
+  int* status;
+  const float* bias;          // [E][2I] or [E][d], or nullptr
+};
+
+__device__ __forceinline__ float silu_p(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
+template <int EPI, int ACT>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
+    grouped_mx_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                           const __grid_constant__ CUtensorMap tmAt,
+                           const __grid_constant__ CUtensorMap tmB,
+                           const __grid_constant__ CUtensorMap tmBt, const PairArgs args) {
+  using C = PairCfg<EPI, ACT>;
+  constexpr int S = C::STAGES;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = static_cast<int>(cluster_ctarank());
+  const int pair_id = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+
+  const uint32_t bar0 = sbase + C::OFF_BAR;
+  auto bar_full = [&](int s) { return bar0 + 8u * s; };
+  auto bar_empty = [&](int s) { return bar0 + 8u * (S + s); };
+  auto bar_peerFull = [&](int s) { return bar0 + 8u * (2 * S + s); };
+  auto bar_accFull = [&](int b) { return bar0 + 8u * (3 * S + b); };
+  auto bar_accEmpty = [&](int b) { return bar0 + 8u * (3 * S + 2 + b); };
+  auto bar_peerAcc = [&](int b) { return bar0 + 8u * (3 * S + 4 + b); };
+  auto bar_tsFull = [&](int b) { return bar0 + 8u * (3 * S + 6 + b); };
+  auto bar_tsEmpty = [&](int b) { return bar0 + 8u * (3 * S + 8 + b); };
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  int* s_off = reinterpret_cast<int*>(smem + C::OFF_TAB);
+  int* s_tp = s_off + (kMaxE + 1);   // prefix of tiles per expert
+  int* s_tb = s_tp + (kMaxE + 1);    // prefix of 128-row token tiles per expert
+
+  const int E = args.E;
+  for (int i = threadIdx.x; i <= E; i += C::NUM_THREADS) s_off[i] = args.offsets[i];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    *abort_flag = 0;
+    int acc = 0, tb = 0;
+    for (int e = 0; e < E; ++e) {
+      s_tp[e] = acc;
+      s_tb[e] = tb;
+      const int cnt = s_off[e + 1] - s_off[e];
+      acc += (cnt + 255) / 256 * args.n_tiles;
+      tb += (cnt + 127) / 128;
+    }
+    s_tp[E] = acc;
+    s_tb[E] = tb;
+    for (int s = 0; s < S; ++s) {
+      mbar_init(bar_full(s), 2);     // producer (with the TMA bytes) + B-scale builder
+      mbar_init(bar_empty(s), 1);    // the issuer's commit, multicast to both CTAs
+      mbar_init(bar_peerFull(s), 1); // the odd CTA's relay
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(bar_accFull(b), 1);
+      mbar_init(bar_accEmpty(b), C::EPI_WARPS * 32);
+      mbar_init(bar_peerAcc(b), 1);
+      mbar_init(bar_tsFull(b), 1);
+      mbar_init(bar_tsEmpty(b), 1);
+    }
+    fence_mbar_init();
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    tma_prefetch_desc(&tmBt);
+    if (ACT == ACT_E2M1) tma_prefetch_desc(&tmAt);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(smem_u32(misc), C::TMEM_COLS);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  tc_fence_after();
+  const uint32_t tmem_base = misc[0];
+
+  const int total = s_tp[E];
+  const int K = args.K;
+  const int G = K / 32;
+  const int KB = args.KB;
+  const bool tail = (K % 128) != 0;   // K % 64 == 0: the tail k-block has 2 K steps
+  // tile -> expert, weight tile nt, token pair-tile mt (token tiles fastest, so
+  // that neighbouring pairs share a weight tile in L2), rows of this CTA's half
+  struct Tile {
+    int e, nt, mt, rows;   // rows: valid token rows of this CTA's half (0..128)
+    int arow;              // first padded token row of this CTA's half
+    int ttile;             // its 128-row token tile
+  };
+  auto decode = [&](int tile, Tile& t) {
+    int lo = 0, hi = E;
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (s_tp[mid] <= tile) lo = mid; else hi = mid;
+    }
+    t.e = lo;
+    const int cnt = s_off[t.e + 1] - s_off[t.e];
+    const int mpairs = (cnt + 255) / 256;
+    const int local = tile - s_tp[t.e];
+    t.nt = local / mpairs;
+    t.mt = local % mpairs;
+    t.rows = min(128, max(0, cnt - t.mt * 256 - rank * 128));
+    t.ttile = s_tb[t.e] + 2 * t.mt + rank;
+    t.arow = t.ttile * 128;
+  };
+
+  if (warp == 0) {
+    // ------------------------------------------------------- TMA producer --
+    if (lane == 0) {
+      // a tile's weight-scale rows (this CTA's B columns and the peer's: all N
+      // columns' scales are needed in each CTA) into tile-scale buffer it & 1
+      auto load_tile_scales = [&](int tile, int itx) -> bool {
+        Tile t;
+        decode(tile, t);
+        const int b = itx & 1;
+        if (!mbar_wait(bar_tsEmpty(b), ((itx >> 1) & 1) ^ 1, abort_flag, args.status)) return false;
+        const uint32_t ts = sbase + C::OFF_TS + b * C::TS_BYTES;
+        const size_t ebase = static_cast<size_t>(t.e) * args.rows_per_expert;
+        if (EPI == PAIR_SWIGLU) {
+          const int j0 = t.nt * C::NH;
+          const uint32_t half = static_cast<uint32_t>(min(C::NH, args.I - j0)) * G;
+          mbar_expect_tx(bar_tsFull(b), 2 * half);
+          bulk_load(ts, args.scales + (ebase + j0) * G, half, bar_tsFull(b));
+          bulk_load(ts + C::NH * G, args.scales + (ebase + args.I + j0) * G, half, bar_tsFull(b));
+        } else {
+          const int n0 = t.nt * C::N;
+          const uint32_t bytes = static_cast<uint32_t>(min(C::N, args.n_out - n0)) * G;
+          mbar_expect_tx(bar_tsFull(b), bytes);
+          bulk_load(ts, args.scales + (ebase + n0) * G, bytes, bar_tsFull(b));
+        }
+        return true;
+      };
+      int s = 0, ph = 0, it = 0;
+      bool ok = pair_id >= total || load_tile_scales(pair_id, 0);
+      const int kb_next = min(3, KB - 1);
+      for (int tile = pair_id; tile < total && ok; tile += npairs, ++it) {
+        Tile t;
+        decode(tile, t);
+        const bool has_a = t.rows > 0;
+        // weight rows of this CTA's B half
+        const int wrow = EPI == PAIR_SWIGLU ? rank * args.I + t.nt * C::NH
+                                            : t.nt * C::N + rank * C::NH;
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!(ok = mbar_wait(bar_empty(s), ph ^ 1, abort_flag, args.status))) break;
+          const uint32_t st = sbase + s * C::STAGE_BYTES;
+          const uint32_t fb = bar_full(s);
+          mbar_expect_tx(fb, has_a ? C::TX_FULL : C::B_TX);
+          const bool last_tail = tail && kb == KB - 1;
+          const int kx = last_tail ? K - 128 : kb * 128;
+          if (has_a) {
+            if (ACT == ACT_HILO)
+              tma_load_3d(st, &tmA, kx, t.arow, 0, fb);   // hi rows, then lo rows
+            else if (ACT == ACT_E4M3)
+              tma_load_2d(st, &tmA, kx, t.arow, fb);
+            else
+              tma_load_2d(st, last_tail ? &tmAt : &tmA, last_tail ? 0 : kb * 128, t.arow, fb);
+            bulk_load(st + C::OFF_SFA,
+                      args.sfa + (static_cast<size_t>(t.ttile) * KB + kb) * C::SFA_BYTES,
+                      C::SFA_BYTES, fb);
+          }
+          tma_load_3d(st + C::OFF_B, last_tail ? &tmBt : &tmB, last_tail ? 0 : kb * 128, wrow, t.e,
+                      fb);
+          if (++s == S) { s = 0; ph ^= 1; }
+          if (kb == kb_next && tile + npairs < total && !(ok = load_tile_scales(tile + npairs, it + 1)))
+            break;
+        }
+      }
+    }
+  } else if (warp == 2) {
+    // -------------------------------------------------- B-scale builder --
+    // Lane l fills bytes 16l..16l+15 of both atoms: the four scale bytes (K
+    // steps 0..3 of the k-block) of B columns 32w + l (atom 0) and
+    // 128 + 32w + l (atom 1), w = 0..3, read from the tile's scale rows
+    // (row c of the tile-scale buffer is B column c; 2-byte aligned rows).
+    int s = 0, ph = 0, it = 0;
+    bool ok = true;
+    for (int tile = pair_id; tile < total && ok; tile += npairs, ++it) {
+      const int b = it & 1;
+      if (!(ok = mbar_wait(bar_tsFull(b), (it >> 1) & 1, abort_flag, args.status))) break;
+      const uint8_t* ts = smem + C::OFF_TS + b * C::TS_BYTES;
+      for (int kb = 0; kb < KB; ++kb) {
+        const int gs = (tail && kb == KB - 1) ? G - 4 : 4 * kb;
+        uint32_t w[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int c = 32 * j + lane;
+          w[j] = 0;
+          if (c < C::N) {
+            const uint16_t* p = reinterpret_cast<const uint16_t*>(ts + c * G + gs);
+            w[j] = static_cast<uint32_t>(p[0]) | (static_cast<uint32_t>(p[1]) << 16);
+          }
+        }
+        if (!(ok = mbar_wait(bar_empty(s), ph ^ 1, abort_flag, args.status))) break;
+        uint8_t* sfb = smem + s * C::STAGE_BYTES + C::OFF_SFB;
+        *reinterpret_cast<uint4*>(sfb + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4*>(sfb + 512 + lane * 16) = make_uint4(w[4], w[5], w[6], w[7]);
+        // orders these shared-memory writes (and the tile-scale reads) before
+        // the async-proxy accesses that follow: tcgen05.cp of the atoms, the
+        // next bulk copy into the tile-scale buffer
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar_full(s));
+        if (++s == S) { s = 0; ph ^= 1; }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_tsEmpty(b));
+    }
+  } else if (warp == 1) {
+    // ----------------------------------------- UMMA issuer (even CTA) --
+    if (rank == 0 && lane == 0) {
+      const uint32_t sfa_t = tmem_base + C::SF_COL0;
+      const uint32_t sfb_t = sfa_t + 4 * C::TERMS;
+      int s = 0, ph = 0, it = 0;
+      bool ok = true;
+      for (int tile = pair_id; tile < total && ok; tile += npairs, ++it) {
+        const int ab = it & 1;
+        const uint32_t ap = (it >> 1) & 1;
+        if (!(ok = mbar_wait(bar_accEmpty(ab), ap ^ 1, abort_flag, args.status))) break;
+        if (!(ok = mbar_wait_cluster(bar_peerAcc(ab), ap ^ 1, abort_flag, args.status))) break;
+        tc_fence_after();
+        const uint32_t d = tmem_base + ab * C::ACC_COLS;
+        uint32_t accum = 0;   // the tile's first UMMA overwrites the buffer
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!(ok = mbar_wait(bar_full(s), ph, abort_flag, args.status))) break;
+          if (!(ok = mbar_wait_cluster(bar_peerFull(s), ph, abort_flag, args.status))) break;
+          tc_fence_after();
+          const uint32_t st = sbase + s * C::STAGE_BYTES;
+#pragma unroll
+          for (int h = 0; h < C::TERMS; ++h)
+            tmem_cp_32x128b_x4_pair(sfa_t + 4 * h, sdesc_k_noswizzle(st + C::OFF_SFA + 512 * h, 128));
+          tmem_cp_32x128b_x4_pair(sfb_t, sdesc_k_noswizzle(st + C::OFF_SFB, 128));
+          tmem_cp_32x128b_x4_pair(sfb_t + 4, sdesc_k_noswizzle(st + C::OFF_SFB + 512, 128));
+          // K steps with compile-time indices; the tail k-block of a K that is
+          // 64 mod 128 issues its last two steps only
+          auto step = [&](const int kk) {
+#pragma unroll
+            for (int h = 0; h < C::TERMS; ++h) {
+              umma_mx_pair(d, sdesc_k_sw128(st + h * C::A_PLANE + kk * 32),
+                           sdesc_k_sw128(st + C::OFF_B + kk * 32),
+                           idesc_pair(256, C::N, C::ATYPE, static_cast<uint32_t>(kk)),
+                           (sfa_t + 4 * h) | (static_cast<uint32_t>(kk) << 30),
+                           sfb_t | (static_cast<uint32_t>(kk) << 30), accum);
+              accum = 1;
+            }
+          };
+          if (!(tail && kb == KB - 1)) {
+            step(0);
+            step(1);
+            step(2);
+            step(3);
+          } else {
+            step(2);
+            step(3);
+          }
+          umma_commit_pair(bar_empty(s));
+          if (++s == S) { s = 0; ph ^= 1; }
+        }
+        if (ok) umma_commit_pair(bar_accFull(ab));
+      }
+    }
+  } else if (warp == 3) {
+    // ------------------------------------ stage relay (odd CTA) --
+    if (rank == 1 && lane == 0) {
+      int s = 0, ph = 0;
+      bool ok = true;
+      for (int tile = pair_id; tile < total && ok; tile += npairs) {
+        for (int kb = 0; kb < KB; ++kb) {
+          if (!(ok = mbar_wait(bar_full(s), ph, abort_flag, args.status))) break;
+          // the stage is complete in this CTA's shared memory (observed with
+          // acquire semantics above); forward that to the issuer
+          mbar_arrive_remote_relaxed(mapa_shared(bar_peerFull(s), 0));
+          if (++s == S) { s = 0; ph ^= 1; }
+        }
+      }
+    }
+  } else {
+    // ----------------------------------------------------------- epilogue --
+    const int quad = warp & 3;
+    const int m = quad * 32 + lane;   // token row of this CTA's half
+    int it = 0;
+    for (int tile = pair_id; tile < total; tile += npairs, ++it) {
+      Tile t;
+      decode(tile, t);
+      const int ab = it & 1;
+      const uint32_t ap = (it >> 1) & 1;
+      if (!mbar_wait_cluster(bar_accFull(ab), ap, abort_flag, args.status)) break;
+      tc_fence_after();
+      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16) + ab * C::ACC_COLS;
+      const bool valid = m < t.rows;
+      if (EPI == PAIR_SWIGLU) {
+        // columns c < 96: gate row j0 + c, 96 + c: the same up row; three
+        // groups of 32 H columns, each converted for the down GEMM
+        const int j0 = t.nt * C::NH;
+        const float* brow = args.bias ? args.bias + static_cast<int64_t>(t.e) * 2 * args.I : nullptr;
+        const size_t hrow = static_cast<size_t>(t.arow) + m;
+#pragma unroll 1
+        for (int g = 0; g < C::NH / 32; ++g) {
+          const int jg = j0 + 32 * g;
+          float h[32];
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            uint32_t gv[16], uv[16];
+            tmem_ld16_sync(taddr + 32 * g + 16 * q, gv);
+            tmem_ld16_sync(taddr + C::NH + 32 * g + 16 * q, uv);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const int j = jg + 16 * q + i;
+              float gg = __uint_as_float(gv[i]), uu = __uint_as_float(uv[i]);
+              if (brow && j < args.I) {
+                gg += __ldg(brow + j);
+                uu += __ldg(brow + args.I + j);
+              }
+              float hv = silu_p(gg) * uu;
+              // bf16 precision: H is a bf16 row, split exactly below; the
+              // quantised modes convert the fp32 value itself
+              if (ACT == ACT_HILO) hv = __bfloat162float(__float2bfloat16_rn(hv));
+              h[16 * q + i] = hv;
+            }
+          }
+          if (!valid || jg >= args.I) continue;
+          float amax = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(h[i]));
+          int kb4, kk4;
+          pair_group_to_kblock(jg / 32, args.I / 32, args.h_kb, kb4, kk4);
+          uint8_t* blk = args.h_sfa + (static_cast<size_t>(t.ttile) * args.h_kb + kb4) * C::SFA_BYTES;
+          if (ACT == ACT_HILO) {
+            int eh = 0;
+            if (amax != 0.f) {
+              const int ex = static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127;
+              eh = max(ex - 7, -123);
+            }
+            const float inv = __uint_as_float(static_cast<uint32_t>(127 - eh) << 23);
+            uint32_t hw[8], lw[8];
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+              uint32_t a = 0, b = 0;
+#pragma unroll
+              for (int u = 0; u < 4; u += 2) {
+                const float x0 = h[4 * q + u] * inv, x1 = h[4 * q + u + 1] * inv;
+                const uint32_t h2 = f32x2_to_e4m3x2(x0, x1);
+                const float2 hb = e4m3x2_to_f32x2(h2);
+                const uint32_t l2 = f32x2_to_e4m3x2((x0 - hb.x) * 16.f, (x1 - hb.y) * 16.f);
+                a |= h2 << (8 * u);
+                b |= l2 << (8 * u);
+              }
+              hw[q] = a;
+              lw[q] = b;
+            }
+            const size_t o = hrow * static_cast<size_t>(args.n_out) + jg;   // rows of I bytes
+            uint4* dh = reinterpret_cast<uint4*>(args.h_q + o);
+            dh[0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            dh[1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+            uint4* dl = reinterpret_cast<uint4*>(args.h_lo + o);
+            dl[0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+            dl[1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+            blk[atom_offset(m, kk4)] = static_cast<uint8_t>(eh + 127);
+            blk[512 + atom_offset(m, kk4)] = static_cast<uint8_t>(eh + 123);
+          } else {
+            constexpr int emax = ACT == ACT_E2M1 ? 2 : 8;
+            int ex = 0;
+            if (amax > 0.f)
+              ex = max(static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127 - emax, -127);
+            const float inv = __uint_as_float(static_cast<uint32_t>(127 - ex) << 23);
+            if (ACT == ACT_E4M3) {
+              uint32_t w[8];
+#pragma unroll
+              for (int q = 0; q < 8; ++q)
+                w[q] = f32x2_to_e4m3x2(h[4 * q] * inv, h[4 * q + 1] * inv) |
+                       (f32x2_to_e4m3x2(h[4 * q + 2] * inv, h[4 * q + 3] * inv) << 16);
+              uint4* dq = reinterpret_cast<uint4*>(args.h_q + hrow * args.n_out + jg);
+              dq[0] = make_uint4(w[0], w[1], w[2], w[3]);
+              dq[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            } else {
+              uint32_t w[4];
+#pragma unroll
+              for (int q = 0; q < 4; ++q) {
+                uint32_t a = 0;
+#pragma unroll
+                for (int b = 0; b < 4; ++b)
+                  a |= f32x2_to_e2m1x2(h[8 * q + 2 * b] * inv, h[8 * q + 2 * b + 1] * inv) << (8 * b);
+                w[q] = a;
+              }
+              *reinterpret_cast<uint4*>(args.h_q + hrow * (args.n_out / 2) + jg / 2) =
+                  make_uint4(w[0], w[1], w[2], w[3]);
+            }
+            blk[atom_offset(m, kk4)] = static_cast<uint8_t>(ex + 127);
+          }
+        }
+      } else {
+        // weighted un-permute: fp32 row p * (y + b) of pair perm[row] at yw[pair]
+        const int n0 = t.nt * C::N;
+        int pr = 0;
+        float w = 0.f;
+        if (valid) {
+          pr = args.perm[s_off[t.e] + t.mt * 256 + rank * 128 + m];
+          w = args.topk_w[pr];
+        }
+        float* orow = args.out_f32 + static_cast<int64_t>(pr) * args.n_out;
+        const float* brow = args.bias ? args.bias + static_cast<int64_t>(t.e) * args.n_out : nullptr;
+#pragma unroll 1
+        for (int c = 0; c < C::N; c += 16) {
+          uint32_t y[16];
+          tmem_ld16_sync(taddr + c, y);
+          const int col = n0 + c;
+          if (valid && col < args.n_out) {
+            float b[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) b[i] = brow ? __ldg(brow + col + i) : 0.f;
+            float4* dst = reinterpret_cast<float4*>(orow + col);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_float4(w * (__uint_as_float(y[4 * i]) + b[4 * i]),
+                                   w * (__uint_as_float(y[4 * i + 1]) + b[4 * i + 1]),
+                                   w * (__uint_as_float(y[4 * i + 2]) + b[4 * i + 2]),
+                                   w * (__uint_as_float(y[4 * i + 3]) + b[4 * i + 3]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar_accEmpty(ab));
+      if (rank == 1 && threadIdx.x == 4 * 32) {
+        // accumulator relay: once all epilogue threads of this CTA have
+        // released the buffer, tell the even CTA's issuer
+        if (!mbar_wait(bar_accEmpty(ab), ap, abort_flag, args.status)) break;
+        mbar_arrive_remote(mapa_shared(bar_peerAcc(ab), 0));
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem_base, C::TMEM_COLS);
+  }
+}
+
+// ----------------------------------------------------------- host side ----
+
+template <int EPI, int ACT>
+cudaError_t launch_pair_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st) {
+  using C = PairCfg<EPI, ACT>;
+  if (p.K % 64 != 0 || p.K < 128 || p.K > kMxMaxK || p.act != ACT) return cudaErrorInvalidValue;
+  if (ACT == ACT_HILO && p.b_lo != p.b_hi + static_cast<size_t>(p.tok_rows) * p.K)
+    return cudaErrorInvalidValue;
+  static bool attr_set[64] = {false};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
+    cudaError_t e = cudaFuncSetAttribute(grouped_mx_pair_kernel<EPI, ACT>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_ALLOC);
+    if (e != cudaSuccess) return e;
+    attr_set[dev] = true;
+  }
+  CUtensorMap tmA, tmAt, tmB, tmBt;
+  bool ok;
+  if (ACT == ACT_HILO) {
+    ok = mx_make_tok8_map(&tmA, p.b_hi, p.tok_rows, p.K, C::MT);
+    tmAt = tmA;
+  } else if (ACT == ACT_E4M3) {
+    ok = mx_make_tok8_map1(&tmA, p.b_hi, p.tok_rows, p.K, C::MT);
+    tmAt = tmA;
+  } else {
+    const cuuint64_t dims[1] = {static_cast<cuuint64_t>(p.tok_rows)};
+    const cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.K / 2)};
+    const cuuint32_t box[1] = {static_cast<cuuint32_t>(C::MT)};
+    ok = mx_make_code_maps(&tmA, &tmAt, p.b_hi, p.K, 2, dims, strides, box);
+  }
+  const int rows = EPI == PAIR_SWIGLU ? 2 * p.I : p.n_out;
+  {
+    const cuuint64_t rb = static_cast<cuuint64_t>(p.K / 2);
+    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(p.E)};
+    const cuuint64_t strides[2] = {rb, rb * static_cast<cuuint64_t>(rows)};
+    const cuuint32_t box[2] = {static_cast<cuuint32_t>(C::NH), 1};
+    ok = ok && mx_make_code_maps(&tmB, &tmBt, p.codes, p.K, 3, dims, strides, box);
+  }
+  if (!ok) return cudaErrorInvalidValue;
+  PairArgs a;
+  a.offsets = p.offsets;
+  a.E = p.E;
+  a.K = p.K;
+  a.I = p.I;
+  a.n_out = p.n_out;
+  a.n_tiles = EPI == PAIR_SWIGLU ? (p.I + C::NH - 1) / C::NH : (p.n_out + C::N - 1) / C::N;
+  a.rows_per_expert = rows;
+  a.KB = (p.K + 127) / 128;
+  a.scales = p.scales;
+  a.sfa = p.b_sfb;
+  a.h_q = p.h_hi;
+  a.h_lo = p.h_lo;
+  a.h_sfa = p.h_sfb;
+  a.h_kb = (p.I + 127) / 128;
+  a.out_f32 = p.out_f32;
+  a.perm = p.perm;
+  a.topk_w = p.topk_w;
+  a.status = p.status;
+  a.bias = p.bias;
+  const int64_t tiles_bound = (static_cast<int64_t>(p.P) / 256 + p.E) * a.n_tiles;
+  int64_t pairs = num_sms / 2;
+  if (tiles_bound < pairs) pairs = tiles_bound;
+  if (pairs < 1) pairs = 1;
+  grouped_mx_pair_kernel<EPI, ACT><<<static_cast<int>(2 * pairs), C::NUM_THREADS, C::SMEM_ALLOC, st>>>(
+      tmA, tmAt, tmB, tmBt, a);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_mx_pair_gateup_swiglu(const MxGemmProblem& p, int num_sms, cudaStream_t st) {
+  switch (p.act) {
+    case ACT_HILO: return launch_pair_impl<PAIR_SWIGLU, ACT_HILO>(p, num_sms, st);
+    case ACT_E4M3: return launch_pair_impl<PAIR_SWIGLU, ACT_E4M3>(p, num_sms, st);
+    case ACT_E2M1: return launch_pair_impl<PAIR_SWIGLU, ACT_E2M1>(p, num_sms, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+cudaError_t launch_mx_pair_down(const MxGemmProblem& p, int num_sms, cudaStream_t st) {
+  switch (p.act) {
+    case ACT_HILO: return launch_pair_impl<PAIR_DOWN, ACT_HILO>(p, num_sms, st);
+    case ACT_E4M3: return launch_pair_impl<PAIR_DOWN, ACT_E4M3>(p, num_sms, st);
+    case ACT_E2M1: return launch_pair_impl<PAIR_DOWN, ACT_E2M1>(p, num_sms, st);
+  }
+  return cudaErrorInvalidValue;
+}
+
+}  // namespace moe

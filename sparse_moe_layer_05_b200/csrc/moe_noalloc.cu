@@ -11,9 +11,13 @@
 //
 // The array is a file-scope __device__ variable: every GPU that loads this
 // library holds it, kNoAllocScratchBytes of device memory, until the process
-// exits. Host code cannot use the array's name as a device address, so the
-// first call on each device looks the address up once with
-// cudaGetSymbolAddress (with that device current) and caches it.
+// exits. Host code cannot use the array's name as a device address, so every
+// call looks the address up with cudaGetSymbolAddress on the device that is
+// current for the call. Nothing is cached on the host: an address stays
+// right after a new primary context or a cudaDeviceReset, and host threads
+// making their first calls at the same time share no state here. The lookup
+// is a cheap runtime query; the first one on a device also loads the
+// library's module there, so make a first call before any stream capture.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -26,11 +30,8 @@ namespace {
 // (token, expert); the rest of the scratch is small tables.
 constexpr size_t kNoAllocMaxTE = size_t(1) << 20;
 constexpr size_t kNoAllocScratchBytes = kNoAllocMaxTE * 4 + (size_t(64) << 10);
-constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBytes];
-
-void* g_scratch_addr[kMaxDevices] = {nullptr};
 
 size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
@@ -58,23 +59,20 @@ ScratchLayout scratch_layout(int E, int T) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-// Device address of the scratch array on the current device (looked up once
-// per device).
+// Device address of the scratch array on the current device, looked up on
+// every call (see the file comment).
 moe_status scratch_base(void** out) {
   int dev = -1;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0) {
     cudaGetLastError();
     return MOE_ERR_NO_DEVICE;
   }
-  if (!g_scratch_addr[dev]) {
-    void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) {
-      cudaGetLastError();
-      return MOE_ERR_CUDA;
-    }
-    g_scratch_addr[dev] = p;
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_route_scratch) != cudaSuccess || !p) {
+    cudaGetLastError();
+    return MOE_ERR_CUDA;
   }
-  *out = g_scratch_addr[dev];
+  *out = p;
   return MOE_OK;
 }
 

@@ -1,9 +1,12 @@
 // moe_probe.cu -- tensor-core rate probe: the UMMA throughput the grouped
-// GEMMs can count on, measured on the device the library runs on.
+// GEMMs can count on, measured on the device it runs on. Built as a library
+// of its own (libmoe_b200_probe.so, include/moe_b200_probe.h): it is
+// measurement tooling for the benchmark, not part of the layer's interface.
 //
 // Each CTA (one per SM) has one thread that issues back-to-back UMMAs from
-// shared-memory tiles (M = 128, K = 16 for bf16, K = 32 for the block-scaled
-// E2M1 x E4M3 kind) into one TMEM accumulator, `per_commit` UMMAs per
+// shared-memory tiles (M = 128; K = 16 for bf16, K = 32 for the block-scaled
+// E2M1 x E4M3 kind, K = 64 for the block-scaled E2M1 x E2M1 kind::mxf4) into
+// one TMEM accumulator, `per_commit` UMMAs per
 // tcgen05.commit, keeping at most eight commits in flight. The operands are
 // zero (timing only). The result is MACs per SM clock, from clock64 over the
 // issuing loop plus the drain of the last commits, slowest SM. Every wait is
@@ -12,7 +15,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include "moe_internal.h"
+#include "../../include/moe_b200_probe.h"
 #include "moe_ptx.cuh"
 
 namespace moe {
@@ -68,6 +71,18 @@ __global__ void __launch_bounds__(128, 1)
           for (uint32_t kk = 0; kk < 4; ++kk)
             umma_mxf8f6f4(tb, sdesc_k_sw128(A + kk * 32), sdesc_k_sw128(B + kk * 32),
                           idesc_mx_e2m1_e4m3(128, N, kk, kk), sfa | (kk << 30), sfb | (kk << 30), 1u);
+        } else if (KIND == 2) {
+          // four K = 64 steps: two scale bytes per row and step, two steps per
+          // 32-bit scale word, so two scale columns per operand
+          tmem_cp_32x128b_x4(sfa, sdesc_k_noswizzle(SF, 128));
+          tmem_cp_32x128b_x4(sfb, sdesc_k_noswizzle(SF + 512, 128));
+#pragma unroll
+          for (uint32_t kk = 0; kk < 4; ++kk) {
+            const uint32_t id = (kk & 1) * 2;
+            umma_mxf4(tb, sdesc_k_sw128(A + kk * 32), sdesc_k_sw128(B + kk * 32),
+                      idesc_mxf4(128, N, id, id), (sfa + (kk >> 1)) | (id << 30),
+                      (sfb + (kk >> 1)) | (id << 30), 1u);
+          }
         } else {
 #pragma unroll
           for (uint32_t kk = 0; kk < 4; ++kk)
@@ -89,29 +104,92 @@ __global__ void __launch_bounds__(128, 1)
   if (threadIdx.x < 32) tmem_dealloc(tb, 512);
 }
 
-}  // namespace
-
 cudaError_t launch_tensor_rate_probe(int kind, int N, int per_commit, int num_sms,
                                      unsigned long long* cycles, int* status, cudaStream_t st) {
-  static bool attr_set[2][64] = {{false}};
+  static bool attr_set[3][64] = {{false}};
   int dev = 0;
   cudaGetDevice(&dev);
-  const int kd = kind == 1 ? 1 : 0;
+  const int kd = kind;
+  void (*fn)(int, int, unsigned long long*, int*) =
+      kd == 2 ? tensor_rate_probe_kernel<2>
+              : (kd == 1 ? tensor_rate_probe_kernel<1> : tensor_rate_probe_kernel<0>);
   if (dev >= 0 && dev < 64 && !attr_set[kd][dev]) {
-    cudaError_t e = kd ? cudaFuncSetAttribute(tensor_rate_probe_kernel<1>,
-                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kProbeSmem)
-                       : cudaFuncSetAttribute(tensor_rate_probe_kernel<0>,
-                                              cudaFuncAttributeMaxDynamicSharedMemorySize, kProbeSmem);
+    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, kProbeSmem);
     if (e != cudaSuccess) return e;
     attr_set[kd][dev] = true;
   }
-  if (kd)
-    tensor_rate_probe_kernel<1><<<num_sms, 128, kProbeSmem, st>>>(N, per_commit, cycles, status);
-  else
-    tensor_rate_probe_kernel<0><<<num_sms, 128, kProbeSmem, st>>>(N, per_commit, cycles, status);
+  fn<<<num_sms, 128, kProbeSmem, st>>>(N, per_commit, cycles, status);
   return cudaGetLastError();
 }
 
-int tensor_rate_probe_iters() { return kProbeIters; }
-
+}  // namespace
 }  // namespace moe
+
+namespace {
+// what the last failing CUDA call of this thread returned (moe_probe_error_string)
+thread_local const char* g_probe_err = "no error";
+thread_local const char* g_probe_where = "";
+
+bool probe_cuda(cudaError_t e, const char* where) {
+  if (e == cudaSuccess) return true;
+  g_probe_err = cudaGetErrorString(e);
+  g_probe_where = where;
+  cudaGetLastError();
+  return false;
+}
+}  // namespace
+
+extern "C" {
+
+const char* moe_probe_error_string(void) { return g_probe_err; }
+const char* moe_probe_error_site(void) { return g_probe_where; }
+
+moe_status moe_probe_tensor_rate(int kind, int N, int per_commit, double* mac_per_clk_sm,
+                                 void* stream) {
+  if (!mac_per_clk_sm || kind < 0 || kind > 2 || N < 16 || N > 256 || N % 16 ||
+      per_commit < 4 || per_commit > 64 || per_commit % 4)
+    return MOE_ERR_INVALID_ARG;
+  int dev = -1, major = 0, minor = 0, num_sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&num_sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return MOE_ERR_NO_DEVICE;
+  }
+  if (major != 10 || minor != 0) return MOE_ERR_NO_DEVICE;
+  g_probe_err = "no error";
+  g_probe_where = "";
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned long long* d_cycles = nullptr;
+  const size_t bytes = static_cast<size_t>(num_sms) * 8 + 16;
+  if (!probe_cuda(cudaMalloc(&d_cycles, bytes), "cudaMalloc")) return MOE_ERR_CUDA;
+  int* d_status = reinterpret_cast<int*>(d_cycles + num_sms);
+  moe_status r = MOE_OK;
+  if (!probe_cuda(cudaMemsetAsync(d_cycles, 0, bytes, st), "cudaMemsetAsync") ||
+      !probe_cuda(moe::launch_tensor_rate_probe(kind, N, per_commit, num_sms, d_cycles, d_status,
+                                                st),
+                  "probe launch") ||
+      !probe_cuda(cudaStreamSynchronize(st), "cudaStreamSynchronize"))
+    r = MOE_ERR_CUDA;
+  unsigned long long* h = new unsigned long long[num_sms + 2];
+  if (r == MOE_OK && !probe_cuda(cudaMemcpy(h, d_cycles, bytes, cudaMemcpyDeviceToHost), "cudaMemcpy"))
+    r = MOE_ERR_CUDA;
+  if (r == MOE_OK) {
+    const int status = *reinterpret_cast<int*>(h + num_sms);
+    unsigned long long worst = 0;
+    for (int i = 0; i < num_sms; ++i) worst = h[i] > worst ? h[i] : worst;
+    if (status || worst == 0) {
+      r = status ? static_cast<moe_status>(status) : MOE_ERR_CUDA;
+    } else {
+      const double k = kind == 2 ? 64.0 : (kind == 1 ? 32.0 : 16.0);
+      const double macs = static_cast<double>(moe::kProbeIters) * per_commit * 128.0 * N * k;
+      *mac_per_clk_sm = macs / static_cast<double>(worst);
+    }
+  }
+  delete[] h;
+  cudaFree(d_cycles);
+  return r;
+}
+
+}  // extern "C"

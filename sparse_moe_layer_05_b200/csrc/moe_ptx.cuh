@@ -300,6 +300,17 @@ __device__ __forceinline__ void tmem_ld8x2_sync(uint32_t ta, uint32_t tb, uint32
       : "memory");
 }
 
+// One 32-lane x 8-column load, then wait.
+__device__ __forceinline__ void tmem_ld8_sync(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n\t"
+      "tcgen05.wait::ld.sync.aligned;"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr)
+      : "memory");
+}
+
 // One 32-lane x 16-column load, then wait.
 __device__ __forceinline__ void tmem_ld16_sync(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
@@ -355,11 +366,40 @@ __device__ __forceinline__ void umma_mxf8f6f4(uint32_t d_tmem, uint64_t adesc, u
       : "memory");
 }
 
-// Instruction descriptor for umma_mxf8f6f4: A E2M1, B E4M3, E8M0 scales, both
-// operands K-major, fp32 accumulator; sfa_id / sfb_id select the scale byte.
+// Instruction descriptor for umma_mxf8f6f4: A E2M1, B of type btype (0 E4M3,
+// 5 E2M1 in 8-bit containers), E8M0 scales, both operands K-major, fp32
+// accumulator; sfa_id / sfb_id select the scale byte.
+__host__ __device__ constexpr uint32_t idesc_mx_e2m1(int M, int N, uint32_t sfa_id,
+                                                    uint32_t sfb_id, uint32_t btype) {
+  return (sfb_id << 4) | (5u << 7) | (btype << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+         (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24) | (sfa_id << 29);
+}
 __host__ __device__ constexpr uint32_t idesc_mx_e2m1_e4m3(int M, int N, uint32_t sfa_id,
                                                          uint32_t sfb_id) {
-  return (sfb_id << 4) | (5u << 7) | (0u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
+  return idesc_mx_e2m1(M, N, sfa_id, sfb_id, 0u);
+}
+
+// D[tmem] (+)= A B^T over one K = 64 step with .kind::mxf4: A and B hold
+// packed E2M1 values (two per byte, 32 bytes of K per row and step), K-major in
+// 128-byte swizzled tiles; every 32 elements of K carry an E8M0 scale
+// (.scale_vec::2X: two scale bytes per row and step, bytes sf_id and
+// sf_id + 1 of the row's 32-bit TMEM scale word, sf_id 0 or 2).
+__device__ __forceinline__ void umma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                          uint32_t idesc, uint32_t sfa_tmem, uint32_t sfb_tmem,
+                                          uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Instruction descriptor for umma_mxf4: A and B E2M1 (the .kind::mxf4 type
+// code 1), E8M0 scales, both K-major, fp32 accumulator.
+__host__ __device__ constexpr uint32_t idesc_mxf4(int M, int N, uint32_t sfa_id, uint32_t sfb_id) {
+  return (sfb_id << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24) | (sfa_id << 29);
 }
 
@@ -398,6 +438,24 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float a, float b) {
   uint16_t r;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(b), "f"(a));
   return r;
+}
+
+// fp32 -> E2M1 code (round to nearest even, saturating to +-6), in bits 0-3.
+__device__ __forceinline__ uint32_t f32_to_e2m1(float a) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tmov.b16 %0, {t, 0};\n\t}"
+      : "=h"(r)
+      : "f"(0.f), "f"(a));
+  return static_cast<uint32_t>(r) & 0xFu;
+}
+
+// Two fp32 -> two E2M1 codes in one byte: e2m1(a) in bits 0-3, e2m1(b) in 4-7.
+__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float a, float b) {
+  uint16_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tmov.b16 %0, {t, 0};\n\t}"
+      : "=h"(r)
+      : "f"(b), "f"(a));
+  return static_cast<uint32_t>(r) & 0xFFu;
 }
 
 // Two E4M3 (bits 0-7, 8-15) -> two fp32 (exact).

@@ -19,21 +19,87 @@ def lib():
     return B.load()
 
 
-def declared_functions():
-    names = set()
-    for fn in os.listdir(os.path.join(ROOT, "include")):
-        if fn.endswith(".h"):
-            src = open(os.path.join(ROOT, "include", fn)).read()
-            names |= set(re.findall(r"^MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src, re.M))
-    return sorted(names)
+def declared_functions(header):
+    src = open(os.path.join(ROOT, "include", header)).read()
+    return sorted(set(re.findall(r"^MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", src, re.M)))
 
 
 def test_every_declared_symbol_is_exported(lib):
-    names = declared_functions()
+    assert sorted(f for f in os.listdir(os.path.join(ROOT, "include")) if f.endswith(".h")) == \
+        ["moe_b200.h", "moe_b200_probe.h"]
+    names = declared_functions("moe_b200.h")
     assert len(names) >= 13
     for n in names:
         assert hasattr(lib, n), n
     assert set(names) == set(B.EXPORTS)
+    # the measurement tool is a library of its own; the layer's library lacks it
+    probe = B.load_probe()
+    pnames = declared_functions("moe_b200_probe.h")
+    assert set(pnames) == set(B.PROBE_EXPORTS)
+    for n in pnames:
+        assert hasattr(probe, n), n
+        assert not hasattr(lib, n), n
+
+
+def test_probe_checks_arguments_without_a_device():
+    probe = B.load_probe()
+    out = ctypes.c_double(0.0)
+    assert probe.moe_probe_tensor_rate(3, 256, 16, ctypes.byref(out), None) == 1   # kind
+    assert probe.moe_probe_tensor_rate(2, 250, 16, ctypes.byref(out), None) == 1   # N % 16
+    assert probe.moe_probe_tensor_rate(0, 256, 6, ctypes.byref(out), None) == 1    # per_commit
+    assert probe.moe_probe_tensor_rate(0, 256, 16, None, None) == 1                # no output
+
+
+def test_forward_ex_checks_options(lib):
+    """Per-call options are checked before any launch: the tile policy range, the
+    activation mode, the bias alignment; NULL options mean the defaults."""
+    good = 0x10000
+    fwd = [good] * 7 + [4, 2, 8, 64, 128, good, good, 1 << 30]
+    f = lib.moe_forward_ex
+    z = fwd[:]
+    z[9] = 0                                            # T = 0
+
+    def opts(**kw):
+        o = B.ForwardOpts(0, 0, None, None)
+        for k_, v in kw.items():
+            setattr(o, k_, v)
+        return ctypes.byref(o)
+
+    assert f(*(z + [None, None])) == 0                  # NULL options
+    assert f(*(z + [opts(), None])) == 0
+    assert f(*(z + [opts(tile_policy=-1), None])) == 0
+    assert f(*(z + [opts(tile_policy=5), None])) == 0
+    assert f(*(fwd + [opts(tile_policy=6), None])) == 1
+    assert f(*(fwd + [opts(tile_policy=-2), None])) == 1
+    assert f(*(fwd + [opts(act_quant=3), None])) == 1
+    assert f(*(fwd + [opts(act_quant=-1), None])) == 1
+    assert f(*(fwd + [opts(gu_bias_dev=good + 4), None])) == 1
+    # the quantised modes need the block-scaled tiles' shapes (d = 64 is not one)
+    assert f(*(fwd + [opts(act_quant=1), None])) == 2
+    assert f(*(fwd + [opts(act_quant=2), None])) == 2
+    q = lib.moe_mx_quantize
+    assert q(good, 4, 40, 1, good, good, None) == 1     # K not a multiple of 32
+    assert q(good, 4, 64, 0, good, good, None) == 1     # not a quantised mode
+    assert q(good, 4, 64, 3, good, good, None) == 1
+    assert q(good + 8, 4, 64, 1, good, good, None) == 1  # misaligned rows
+    assert q(good, 0, 64, 2, good, good, None) == 0     # no rows: nothing to do
+    a = fwd[:]
+    a[14] = 16
+    assert f(*(a + [opts(), None])) == 3                # workspace too small
+
+
+def test_hostio_status_block_holds_a_word_per_chunk():
+    """Chunked host-buffer calls (T >= 2048, four chunks on two alternating chunk
+    workspaces) give every chunk its own status word inside the 16-byte status
+    block at the workspace's start, so no chunk can clear another's timeout."""
+    for shape in [(32, 4, 8192, 2880, 2880), (8, 2, 4099, 352, 224), (4, 2, 2048, 64, 128)]:
+        E, k, T, d, I = shape
+        Tc = (T + 3) // 4
+        sub = B.moe_workspace_layout(E, k, Tc, d, I)
+        assert sub["status"] == 0
+        nxt = min(v for n, v in sub.items() if n not in ("status", "total"))
+        assert nxt >= 16                                 # four 32-bit words
+        assert B.moe_workspace_size_hostio(E, k, T, d, I) >= 2 * sub["total"]
 
 
 def test_status_strings_and_version(lib):

@@ -56,8 +56,11 @@ def _route_noalloc(inp, x, W_r, b_r):
 def test_noalloc_route_matches_workspace_route_on_consecutive_calls():
     # two calls in a row with different shapes: the second must not see the
     # first call's leftovers in the shared scratch array
+    # (the last two take the two permutation paths: several 256-token chunks,
+    # and one fused launch for at most 256 tokens)
     cases = [W.make_inputs("248a20", T=4096),      # T * E = 1,015,808, near the limit
-             W.make_custom(256, 128, 32, 4, 700, seed=41)]
+             W.make_custom(256, 128, 32, 4, 700, seed=41),
+             W.make_custom(2880, 128, 128, 4, 200, seed=42)]
     for inp in cases:
         x = torch.from_numpy(inp.x).cuda()
         W_r = torch.from_numpy(inp.W_r).cuda()
