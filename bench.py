@@ -385,9 +385,16 @@ def run_ours(args, inp, name):
     dom = B.STAGES.index(DOMINANT_STAGE)
     nb = len(B.STAGES)
     timed_mask = (1 << 0) | (1 << dom) | (1 << (dom + 1)) | (1 << nb)
+    # the per-call options (tile policy, activation mode) travel with every call
+    act = None if args.act_quant == "bf16" else args.act_quant
+    pol = args.tile_policy
+
+    def timed_pass(mask):
+        return layer.forward_timed_events(x, out, mask, tile_policy=pol, act_quant=act)
+
     for _ in range(args.warmup):
         flush.zero_()
-        layer.forward_timed_events(x, out, timed_mask)
+        timed_pass(timed_mask)
     torch.cuda.synchronize()
     status = B.moe_sync_status(layer.workspace)
     if status != 0:
@@ -400,7 +407,7 @@ def run_ours(args, inp, name):
     with ClockSampler(local, clocks_path) as clk:
         for _ in range(args.steps):
             flush.zero_()
-            step_ms.append(layer.forward_timed_events(x, out, timed_mask))
+            step_ms.append(timed_pass(timed_mask))
         torch.cuda.synchronize()
     barrier(world)
     status = B.moe_sync_status(layer.workspace)
@@ -411,7 +418,7 @@ def run_ours(args, inp, name):
     stage_ms = []
     for _ in range(min(args.steps, 5)):
         flush.zero_()
-        stage_ms.append(layer.forward_timed(x, out))
+        stage_ms.append(timed_pass((1 << (nb + 1)) - 1))
     if B.moe_sync_status(layer.workspace) != 0:
         raise RuntimeError("device status after the per-stage steps")
     # the device's routing of the batch (rank 0 runs the batch in its own order),
@@ -489,6 +496,14 @@ def run_ours(args, inp, name):
     stage_avg = {n: sum(s[i] for s in stage_ms) / len(stage_ms) for i, n in enumerate(B.STAGES)}
     counts = layer.intermediate("counts", T).cpu().numpy()
     touched = int((counts > 0).sum())
+    # the load the routing puts on the experts (the skewed 128a4 workload
+    # concentrates it): routed rows per touched expert, and the 256-row tiles
+    # they make against the 74 CTA pairs of the prefill kernels
+    nz = counts[counts > 0]
+    tiles256 = int(np.sum((nz + 255) // 256))
+    routing_load = {"rows_per_touched_expert": {"min": int(nz.min()), "median": float(np.median(nz)),
+                                                "max": int(nz.max())},
+                    "touched_experts": touched, "row_tiles_256": tiles256}
     # algorithmic bytes of one gate/up launch: the touched experts' MXFP4
     # gate/up weights (codes + scales), the permuted activations read, H written
     dom_bytes = (touched * (2 * inp.I * inp.d // 2 + 2 * inp.I * inp.d // 32)
@@ -500,9 +515,20 @@ def run_ours(args, inp, name):
         roof = {"bound": "hbm", "unit": "GB/s", "peak_source": f"hbm_gbs ({kind})",
                 "algorithmic_bytes_per_launch": dom_bytes}
     else:
-        peak = float(peaks["bf16_tflops"])
+        # the peak of the MMA kind the kernel runs: bf16 precision runs at the
+        # bf16 rate (kind::f16, or two E4M3 terms on the FP8-rate kind); w4a8
+        # and w4a4 on one CTA at the FP8 rate (kind::mxf8f6f4); w4a4 on a CTA
+        # pair at the FP4 rate (kind::mxf4): the measured bf16 peak times the
+        # nominal dense ratios 2 and 4
+        ratio, kname = 1.0, "bf16 rate"
+        if args.act_quant == "mxfp8" or (args.act_quant == "mxfp4" and args.tile_policy != 5):
+            ratio, kname = 2.0, "kind::mxf8f6f4, x2 (nominal FP8:BF16)"
+        elif args.act_quant == "mxfp4":
+            ratio, kname = 4.0, "kind::mxf4, x4 (nominal FP4:BF16)"
+        peak = ratio * float(peaks["bf16_tflops"])
         achieved = dom_flops / (dom_ms * 1e-3) / 1e12
-        roof = {"bound": "tensor", "unit": "TFLOP/s", "peak_source": f"bf16_tflops ({kind}, burst)",
+        roof = {"bound": "tensor", "unit": "TFLOP/s",
+                "peak_source": f"bf16_tflops ({kind}, burst); {kname}",
                 "algorithmic_flops_per_launch": dom_flops}
         # the pages' MXFP4 target: the same achieved rate against the dense FP4
         # peak, taken as the measured bf16 peak times the nominal dense ratio
@@ -520,6 +546,8 @@ def run_ours(args, inp, name):
                         "frac": step_bytes / (ms_per_step * 1e-3) / 1e9 / float(peaks["hbm_gbs"])}
 
     # end to end through the C ABI with host buffers: H2D + forward + D2H
+    # (the quantised modes: pinned copies around moe_forward_ex, the calls a
+    # user makes, since the host-buffer entry has no options)
     e2e_s = 0.0
     barrier(world)
     torch.cuda.synchronize()
@@ -528,7 +556,14 @@ def run_ours(args, inp, name):
         ev0 = torch.cuda.Event(enable_timing=True)
         ev1 = torch.cuda.Event(enable_timing=True)
         ev0.record(stream)
-        layer.forward_hostio(x_host, out_host)
+        if act is None and pol == 0:
+            layer.forward_hostio(x_host, out_host)
+        else:
+            x.copy_(x_host, non_blocking=True)
+            B.moe_forward_ex(x, layer.W_r, layer.b_r, layer.Wgu_codes, layer.Wgu_scales,
+                             layer.Wd_codes, layer.Wd_scales, inp.E, inp.k, T, inp.d, inp.I, out,
+                             layer.workspace, tile_policy=pol, act_quant=act or "bf16")
+            out_host.copy_(out, non_blocking=True)
         ev1.record(stream)
         ev1.synchronize()
         e2e_s += ev0.elapsed_time(ev1) / 1e3
@@ -540,8 +575,12 @@ def run_ours(args, inp, name):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16", "data": "synthetic",
+        "dtype": {"bf16": "bf16", "mxfp8": "e4m3", "mxfp4": "e2m1"}[args.act_quant],
+        "data": "synthetic",
         "config": dict(workload_config(inp, name), tile_policy=args.tile_policy,
+                       activations={"bf16": "bf16 (the pages' layer)",
+                                    "mxfp8": "MXFP8 E4M3 (the w4a8 layer)",
+                                    "mxfp4": "MXFP4 E2M1 (the w4a4 layer)"}[args.act_quant],
                        **({"block": "out = h + MoE(RMSNorm(h)), eps 1e-5"} if args.block else {}),
                        **({"expert_biases": "gate/up [E, 2I] and down [E, d], f32"}
                           if args.bias else {})),
@@ -551,6 +590,7 @@ def run_ours(args, inp, name):
                          frac=achieved / peak, traffic=recorded_traffic(name, T),
                          avg_launch_ms=dom_ms, touched_experts=touched),
         "stage_ms": stage_avg,
+        "routing_load": routing_load,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(T * inp.d * 2),
                 "d2h_bytes_per_step": int(T * inp.d * 2), "host_buffers": near.describe()},
         "gpu_launches": (B.moe_forward_launch_count(inp.E, inp.k, T, inp.d, inp.I)
@@ -611,6 +651,9 @@ def main(argv=None):
     ap.add_argument("--tile-policy", type=int, default=0, choices=[0, 1, 2, 3, 4, 5],
                     help="grouped-GEMM tiles: 0 by shape, 1 single, 2 pair, 3 swap, "
                          "4 block-scaled, 5 block-scaled CTA pair")
+    ap.add_argument("--act-quant", default="bf16", choices=["bf16", "mxfp8", "mxfp4"],
+                    help="activation precision of the expert GEMMs: bf16 (the pages' layer), "
+                         "or the w4a8 / w4a4 layers (moe_forward_ex act_quant)")
     ap.add_argument("--cpu-sample", type=int, default=256,
                     help="tokens of the batch the oracle runs for cpu_baseline (0 = skip)")
     args = ap.parse_args(argv)

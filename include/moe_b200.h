@@ -263,6 +263,19 @@ MOE_API moe_status moe_forward_timed_events(const void* x_dev, const float* W_r_
                                             unsigned int event_mask, float* stage_ms_host);
 
 /*
+ * moe_forward_timed_events with per-call options (opts as in moe_forward_ex;
+ * NULL: the defaults). Same timing semantics, errors and blocking.
+ */
+MOE_API moe_status moe_forward_timed_ex(const void* x_dev, const float* W_r_dev,
+                                        const float* b_r_dev, const uint8_t* Wgu_codes_dev,
+                                        const uint8_t* Wgu_scales_dev, const uint8_t* Wd_codes_dev,
+                                        const uint8_t* Wd_scales_dev, int E, int k, int T, int d,
+                                        int I, void* out_dev, void* workspace_dev,
+                                        size_t workspace_bytes, const moe_forward_opts* opts,
+                                        void* stream, unsigned int event_mask,
+                                        float* stage_ms_host);
+
+/*
  * Same as moe_forward with the activations in host memory: copies x_host
  * (T*d*2 bytes; pinned memory gives asynchronous copies) to the workspace,
  * runs the forward pass and copies the result to out_host, then synchronises

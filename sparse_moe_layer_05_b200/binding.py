@@ -31,7 +31,7 @@ EXPORTS = [
     "moe_selftest_wait_timeout", "moe_forward_launch_count", "moe_forward_timed",
     "moe_set_tile_policy", "moe_route_noalloc",
     "moe_workspace_size_block", "moe_forward_block", "moe_rms_norm", "moe_forward_biased",
-    "moe_forward_timed_events", "moe_forward_ex", "moe_mx_quantize",
+    "moe_forward_timed_events", "moe_forward_ex", "moe_mx_quantize", "moe_forward_timed_ex",
 ]
 # the measurement library (libmoe_b200_probe.so, include/moe_b200_probe.h)
 PROBE_EXPORTS = ["moe_probe_tensor_rate", "moe_probe_error_string", "moe_probe_error_site"]
@@ -116,6 +116,9 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.moe_rms_norm.argtypes = [vp, fp, ctypes.c_float, i32, i32, vp, vp]
     lib.moe_forward_ex.restype = i32
     lib.moe_forward_ex.argtypes = fwd[:15] + [ctypes.POINTER(ForwardOpts), vp]
+    lib.moe_forward_timed_ex.restype = i32
+    lib.moe_forward_timed_ex.argtypes = fwd[:15] + [ctypes.POINTER(ForwardOpts), vp, ctypes.c_uint,
+                                                    ctypes.POINTER(ctypes.c_float)]
     lib.moe_mx_quantize.restype = i32
     lib.moe_mx_quantize.argtypes = [vp, i32, i32, i32, u8p, u8p, vp]
     lib.moe_mx_split_e4m3.restype = i32
@@ -417,11 +420,27 @@ class MoELayer:
                                  self.Wd_codes, self.Wd_scales, self.E, self.k, T, self.d,
                                  self.I, out, self.workspace, stream)
 
-    def forward_timed_events(self, x, out, event_mask: int, stream=None):
+    def forward_timed_events(self, x, out, event_mask: int, stream=None, tile_policy=None,
+                             act_quant=None):
+        """moe_forward_timed_events; with tile_policy or act_quant given, the
+        per-call options form (moe_forward_timed_ex)."""
         T = x.shape[0]
-        return moe_forward_timed_events(x, self.W_r, self.b_r, self.Wgu_codes, self.Wgu_scales,
-                                        self.Wd_codes, self.Wd_scales, self.E, self.k, T, self.d,
-                                        self.I, out, self.workspace, event_mask, stream)
+        if tile_policy is None and act_quant is None:
+            return moe_forward_timed_events(x, self.W_r, self.b_r, self.Wgu_codes,
+                                            self.Wgu_scales, self.Wd_codes, self.Wd_scales,
+                                            self.E, self.k, T, self.d, self.I, out,
+                                            self.workspace, event_mask, stream)
+        if isinstance(act_quant, str):
+            act_quant = ACT_MODES[act_quant]
+        o = ForwardOpts(-1 if tile_policy is None else tile_policy,
+                        ACT_BF16 if act_quant is None else act_quant, None, None)
+        ms = (ctypes.c_float * (len(STAGES) + 1))()
+        _check("moe_forward_timed_ex", load().moe_forward_timed_ex(
+            _ptr(x), _ptr(self.W_r), _ptr(self.b_r), _ptr(self.Wgu_codes), _ptr(self.Wgu_scales),
+            _ptr(self.Wd_codes), _ptr(self.Wd_scales), self.E, self.k, T, self.d, self.I, _ptr(out),
+            _ptr(self.workspace), self.workspace.numel(), ctypes.byref(o), _stream(stream),
+            event_mask, ms))
+        return list(ms)
 
     def forward_hostio(self, x_host, out_host, stream=None):
         T = x_host.shape[0]

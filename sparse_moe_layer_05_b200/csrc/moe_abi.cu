@@ -298,6 +298,28 @@ FwdOpts default_opts() {
   return o;
 }
 
+// Per-call options -> FwdOpts (NULL: the defaults), checked before any launch.
+moe_status parse_opts(const moe_forward_opts* opts, int d, int I, const uint8_t* gc,
+                      const uint8_t* dc, FwdOpts* out) {
+  FwdOpts o = default_opts();
+  if (opts) {
+    if (opts->tile_policy < -1 || opts->tile_policy > 5) return MOE_ERR_INVALID_ARG;
+    if (opts->act_quant < MOE_ACT_BF16 || opts->act_quant > MOE_ACT_MXFP4)
+      return MOE_ERR_INVALID_ARG;
+    if (opts->act_quant != MOE_ACT_BF16) {
+      // the quantised modes run on the block-scaled tiles only
+      if (!mx_shape_ok(d, I) || !aligned32(gc) || !aligned32(dc)) return MOE_ERR_UNSUPPORTED;
+      o.act = opts->act_quant == MOE_ACT_MXFP8 ? moe::ACT_E4M3 : moe::ACT_E2M1;
+    }
+    if (opts->tile_policy >= 0) o.policy = opts->tile_policy;
+    o.gu_bias = opts->gu_bias_dev;
+    o.dn_bias = opts->down_bias_dev;
+  }
+  if (!aligned16(o.gu_bias) || !aligned16(o.dn_bias)) return MOE_ERR_INVALID_ARG;
+  *out = o;
+  return MOE_OK;
+}
+
 moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, const uint8_t* gc,
                        const uint8_t* gs, const uint8_t* dc, const uint8_t* ds, int E, int k,
                        int T, int d, int I, uint16_t* out, void* ws, const Layout& L,
@@ -343,8 +365,13 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     // pair when the policy asks for it
     const int variant = P < 64 * E ? moe::kMxSmall
                                    : (opt.policy == 5 ? moe::kMxPair : moe::kMxLarge);
-    MOE_CUDA(moe::launch_mx_act_quant_gather(variant, opt.act, x, perm, offsets, E, P, k, d, qx,
-                                             sfbx, st));
+    // E2M1 activations on the CTA pair run the kind::mxf4 kernel (both
+    // operands packed, 256-wide k-blocks) where d and I allow it
+    const int act = (opt.act == moe::ACT_E2M1 && variant == moe::kMxPair && d >= 256 && I >= 256)
+                        ? moe::ACT_F4
+                        : opt.act;
+    MOE_CUDA(moe::launch_mx_act_quant_gather(variant, act, x, perm, offsets, E, P, k, d, qx, sfbx,
+                                             st));
     E_.mark(6);
     E_.mark(7);
     E_.mark(8);
@@ -365,7 +392,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     m1.n_out = I;
     m1.status = status;
     m1.bias = gu_bias;
-    m1.act = opt.act;
+    m1.act = act;
     MOE_CUDA(variant == moe::kMxPair ? moe::launch_mx_pair_gateup_swiglu(m1, num_sms, st)
                                      : moe::launch_mx_gemm_gateup_swiglu(variant, m1, num_sms, st));
     E_.mark(9);
@@ -590,22 +617,8 @@ moe_status moe_forward_ex(const void* x_dev, const float* W_r_dev, const float* 
                                     Wd_codes_dev, Wd_scales_dev, E, k, T, d, I, out_dev,
                                     workspace_dev);
   if (s != MOE_OK) return s;
-  FwdOpts o = default_opts();
-  if (opts) {
-    if (opts->tile_policy < -1 || opts->tile_policy > 5) return MOE_ERR_INVALID_ARG;
-    if (opts->act_quant < MOE_ACT_BF16 || opts->act_quant > MOE_ACT_MXFP4)
-      return MOE_ERR_INVALID_ARG;
-    if (opts->act_quant != MOE_ACT_BF16) {
-      // the quantised modes run on the block-scaled tiles only
-      if (!mx_shape_ok(d, I) || !aligned32(Wgu_codes_dev) || !aligned32(Wd_codes_dev))
-        return MOE_ERR_UNSUPPORTED;
-      o.act = opts->act_quant == MOE_ACT_MXFP8 ? moe::ACT_E4M3 : moe::ACT_E2M1;
-    }
-    if (opts->tile_policy >= 0) o.policy = opts->tile_policy;
-    o.gu_bias = opts->gu_bias_dev;
-    o.dn_bias = opts->down_bias_dev;
-  }
-  if (!aligned16(o.gu_bias) || !aligned16(o.dn_bias)) return MOE_ERR_INVALID_ARG;
+  FwdOpts o;
+  if ((s = parse_opts(opts, d, I, Wgu_codes_dev, Wd_codes_dev, &o)) != MOE_OK) return s;
   Layout L;
   make_layout(E, k, T, d, I, false, &L);
   if (workspace_bytes < L.pub.total) return MOE_ERR_WORKSPACE;
@@ -799,12 +812,25 @@ moe_status moe_forward_timed_events(const void* x_dev, const float* W_r_dev, con
                                     int E, int k, int T, int d, int I, void* out_dev,
                                     void* workspace_dev, size_t workspace_bytes, void* stream,
                                     unsigned int event_mask, float* stage_ms_host) {
+  return moe_forward_timed_ex(x_dev, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev, Wd_codes_dev,
+                              Wd_scales_dev, E, k, T, d, I, out_dev, workspace_dev,
+                              workspace_bytes, nullptr, stream, event_mask, stage_ms_host);
+}
+
+moe_status moe_forward_timed_ex(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
+                                const uint8_t* Wgu_codes_dev, const uint8_t* Wgu_scales_dev,
+                                const uint8_t* Wd_codes_dev, const uint8_t* Wd_scales_dev, int E,
+                                int k, int T, int d, int I, void* out_dev, void* workspace_dev,
+                                size_t workspace_bytes, const moe_forward_opts* opts, void* stream,
+                                unsigned int event_mask, float* stage_ms_host) {
   if (!stage_ms_host) return MOE_ERR_INVALID_ARG;
   if (event_mask >> (kStages + 1)) return MOE_ERR_INVALID_ARG;
   moe_status s = check_forward_args(x_dev, W_r_dev, b_r_dev, Wgu_codes_dev, Wgu_scales_dev,
                                     Wd_codes_dev, Wd_scales_dev, E, k, T, d, I, out_dev,
                                     workspace_dev);
   if (s != MOE_OK) return s;
+  FwdOpts o;
+  if ((s = parse_opts(opts, d, I, Wgu_codes_dev, Wd_codes_dev, &o)) != MOE_OK) return s;
   Layout L;
   make_layout(E, k, T, d, I, false, &L);
   if (workspace_bytes < L.pub.total) return MOE_ERR_WORKSPACE;
@@ -828,8 +854,7 @@ moe_status moe_forward_timed_events(const void* x_dev, const float* W_r_dev, con
   }
   s = run_forward(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, Wgu_codes_dev,
                   Wgu_scales_dev, Wd_codes_dev, Wd_scales_dev, E, k, T, d, I,
-                  static_cast<uint16_t*>(out_dev), workspace_dev, L, tev.st, num_sms,
-                  default_opts(), &tev);
+                  static_cast<uint16_t*>(out_dev), workspace_dev, L, tev.st, num_sms, o, &tev);
   if (s == MOE_OK && cudaEventSynchronize(tev.ev[kStages]) == cudaSuccess) {
     // a recorded boundary's entry spans to the next recorded boundary
     for (int i = 0; i < kStages; ++i) {

@@ -108,9 +108,13 @@ int mx_tile_tokens(int variant, int act);
 //   ACT_E4M3  the w4a8 layer: one E4M3 element, OCP MX scale (emax 8)
 //   ACT_E2M1  the w4a4 layer: one E2M1 element, OCP MX scale (emax 2), rows
 //             packed two elements per byte (low nibble first)
+//   ACT_F4    the w4a4 layer on the CTA-pair kernel with tcgen05 kind::mxf4:
+//             rows as ACT_E2M1, both operands read packed (no widening), and
+//             the token-side scale blocks laid out per 256-wide k-block
 constexpr int ACT_HILO = 0;
 constexpr int ACT_E4M3 = 1;
 constexpr int ACT_E2M1 = 2;
+constexpr int ACT_F4 = 3;
 
 // Rows of the padded token layout (each expert's rows rounded up to a
 // multiple of the tile's tokens) and bytes of its B-scale blocks, for either
@@ -175,6 +179,10 @@ bool mx_make_code_maps(CUtensorMap* main_map, CUtensorMap* tail_map, const uint8
                        const cuuint32_t* box_rest);
 bool mx_make_tok8_map(CUtensorMap* m, const uint8_t* hi, int rows, int K, int nt);
 bool mx_make_tok8_map1(CUtensorMap* m, const uint8_t* q, int rows, int K, int nt);
+// A byte tensor (rank 1..5, dims/strides/box as cuTensorMapEncodeTiled takes
+// them, 128-byte swizzle).
+bool mx_make_bytes_map(CUtensorMap* m, const uint8_t* base, int rank, const cuuint64_t* dims,
+                       const cuuint64_t* strides, const cuuint32_t* box);
 
 // Debug/self-test: one bounded wait on an mbarrier that nothing completes.
 cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t st);

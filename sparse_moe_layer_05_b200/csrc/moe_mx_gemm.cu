@@ -306,7 +306,10 @@ __global__ void __launch_bounds__(256) mx_split_rows_kernel(const uint16_t* __re
 // One thread per (permuted row, group of 32) for the quantised activation
 // modes: x[token] -> one MX-converted row in the padded token layout (K bytes,
 // or K/2 for E2M1) and its scale byte in the B-scale blocks.
-template <int NT, int ACT>
+// KB256: the scale blocks of the kind::mxf4 kernel, per 256-wide k-block:
+// 1024 bytes per (token tile, k-block), group byte b (0..7) of token n at
+// (b / 4) * 512 + the 32x128b atom byte of (n, b % 4).
+template <int NT, int ACT, bool KB256 = false>
 __global__ void __launch_bounds__(256) mx_act_quant_gather_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
     const int32_t* __restrict__ offsets, int E, int P, int k, int K, uint8_t* __restrict__ q,
@@ -323,8 +326,8 @@ __global__ void __launch_bounds__(256) mx_act_quant_gather_kernel(
     s_tb[E] = a;
   }
   __syncthreads();
-  const int G = K / 32, KB = (K + 127) / 128;
-  constexpr int SFB = sfb_block_bytes(NT, 1);
+  const int G = K / 32, KB = KB256 ? (K + 255) / 256 : (K + 127) / 128;
+  constexpr int SFB = KB256 ? 1024 : sfb_block_bytes(NT, 1);
   constexpr int GB = ACT == ACT_E2M1 ? 16 : 32;     // bytes of one converted group
   const size_t row_bytes = static_cast<size_t>(G) * GB;
   const int64_t n = static_cast<int64_t>(P) * G;
@@ -344,10 +347,25 @@ __global__ void __launch_bounds__(256) mx_act_quant_gather_kernel(
     uint32_t w[8];
     const uint32_t sx = mx_quant_group32<ACT>(v, amax, w);
     store_group32<ACT>(q + static_cast<size_t>(pr) * row_bytes + static_cast<size_t>(g) * GB, w);
-    int kb, kk;
-    group_to_kblock(g, G, KB, kb, kk);
-    uint8_t* blk = sfb + (static_cast<size_t>(pr / NT) * KB + kb) * SFB;
-    blk[sfb_offset(NT, pr % NT, 0, kk)] = static_cast<uint8_t>(sx);
+    if (KB256) {
+      // 8 groups per k-block; the last k-block of a K that is not a multiple
+      // of 256 covers [K-256, K)
+      int kb, b;
+      if ((G % 8) == 0 || g < 8 * (KB - 1)) {
+        kb = g >> 3;
+        b = g & 7;
+      } else {
+        kb = KB - 1;
+        b = g - (G - 8);
+      }
+      uint8_t* blk = sfb + (static_cast<size_t>(pr / NT) * KB + kb) * SFB;
+      blk[(b >> 2) * 512 + sfb_offset(NT, pr % NT, 0, b & 3)] = static_cast<uint8_t>(sx);
+    } else {
+      int kb, kk;
+      group_to_kblock(g, G, KB, kb, kk);
+      uint8_t* blk = sfb + (static_cast<size_t>(pr / NT) * KB + kb) * SFB;
+      blk[sfb_offset(NT, pr % NT, 0, kk)] = static_cast<uint8_t>(sx);
+    }
   }
 }
 
@@ -1085,6 +1103,10 @@ bool mx_make_tok8_map(CUtensorMap* m, const uint8_t* hi, int rows, int K, int nt
 bool mx_make_tok8_map1(CUtensorMap* m, const uint8_t* q, int rows, int K, int nt) {
   return make_tok8_map1(m, q, rows, K, nt);
 }
+bool mx_make_bytes_map(CUtensorMap* m, const uint8_t* base, int rank, const cuuint64_t* dims,
+                       const cuuint64_t* strides, const cuuint32_t* box) {
+  return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, base, dims, strides, box);
+}
 
 int mx_tile_tokens(int variant, int act) {
   if (variant == kMxPair) return kMxMaxNT;
@@ -1106,7 +1128,9 @@ size_t mx_sfb_bytes(int P, int E, int K) {
     const size_t b = tiles * ((K + 127) / 128) * sfb_block_bytes(v[0], v[1]);
     if (b > best) best = b;
   }
-  return best;
+  // the kind::mxf4 pair kernel's blocks: 1024 bytes per 256-wide k-block
+  const size_t f4 = ((static_cast<size_t>(P) + kMxMaxNT - 1) / kMxMaxNT + E) * ((K + 255) / 256) * 1024;
+  return f4 > best ? f4 : best;
 }
 
 cudaError_t launch_mx_quant_gather(int variant, const uint16_t* x, const int32_t* perm,
@@ -1138,6 +1162,10 @@ cudaError_t launch_mx_act_quant_gather(int variant, int act, const uint16_t* x,
       mx_act_quant_gather_kernel<NL, ACT_E4M3><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, q, sfb);
     else
       mx_act_quant_gather_kernel<NS, ACT_E4M3><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, q, sfb);
+  } else if (act == ACT_F4) {
+    if (variant != kMxPair) return cudaErrorInvalidValue;
+    mx_act_quant_gather_kernel<NL, ACT_E2M1, true><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k,
+                                                                        K, q, sfb);
   } else if (act == ACT_E2M1) {
     if (variant != kMxSmall)
       mx_act_quant_gather_kernel<NL, ACT_E2M1><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, q, sfb);

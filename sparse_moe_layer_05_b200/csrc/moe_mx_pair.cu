@@ -81,17 +81,22 @@ constexpr int kPairSmemBudget = 232448 - 1024;   // opt-in maximum less alignmen
 
 template <int EPI, int ACT>
 struct PairCfg {
+  // kind::mxf4 (ACT_F4): both operands stay packed (two E2M1 per byte) in
+  // shared memory, so a 128-byte row holds 256 elements of K, and each UMMA
+  // (K = 64) takes two scale bytes per row: two scale words per k-block
+  static constexpr bool F4 = ACT == ACT_F4;
+  static constexpr int KBK = F4 ? 256 : 128;              // K elements per stage
   static constexpr int TERMS = ACT == ACT_HILO ? 2 : 1;
   static constexpr int MT = 128;                          // token rows per CTA
   static constexpr int NH = EPI == PAIR_SWIGLU ? 96 : 120;  // weight rows per CTA
   static constexpr int N = 2 * NH;                        // UMMA N
-  static constexpr int A_PLANE = MT * 128;                // one term, 8-bit elements
+  static constexpr int A_PLANE = MT * 128;                // one term: 128-byte rows
   static constexpr int A_BYTES = TERMS * A_PLANE;
   static constexpr int A_TX = ACT == ACT_E2M1 ? MT * 64 : A_BYTES;
   static constexpr int B_BYTES = NH * 128;
-  static constexpr int B_TX = NH * 64;                    // packed code bytes
-  static constexpr int SFA_BYTES = 512 * TERMS;
-  static constexpr int SFB_BYTES = 1024;                  // N <= 256: two atoms
+  static constexpr int B_TX = F4 ? B_BYTES : NH * 64;     // packed code bytes
+  static constexpr int SFA_BYTES = F4 ? 1024 : 512 * TERMS;
+  static constexpr int SFB_BYTES = F4 ? 2048 : 1024;      // N <= 256: 2 atoms per word
   static constexpr int OFF_B = A_BYTES;
   static constexpr int OFF_SFA = OFF_B + B_BYTES;
   static constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
@@ -111,11 +116,13 @@ struct PairCfg {
   static constexpr int EPI_WARPS = 4;
   static constexpr int TMEM_COLS = 512;
   static constexpr int ACC_COLS = N;                      // per accumulator buffer
-  static constexpr int SF_COL0 = 2 * N;                   // A scales (TERMS atoms), then B
+  static constexpr int SF_COL0 = 2 * N;                   // A scales, then B scales
+  static constexpr int SFA_COLS = SFA_BYTES / 128;        // 4 TMEM columns per atom
+  static constexpr int SFB_COLS = SFB_BYTES / 128;
   static constexpr int TX_FULL = A_TX + B_TX + SFA_BYTES; // a stage with token rows
   static constexpr uint32_t ATYPE = ACT == ACT_E2M1 ? 5u : 0u;   // E2M1 or E4M3
   static_assert(STAGES >= 3, "pipeline depth");
-  static_assert(SF_COL0 + 4 * TERMS + 8 <= TMEM_COLS, "TMEM budget");
+  static_assert(SF_COL0 + SFA_COLS + SFB_COLS <= TMEM_COLS, "TMEM budget");
   static_assert(SMEM_ALLOC <= 232448, "shared memory");
   static_assert(OFF_B % 1024 == 0 && B_BYTES % 1024 == 0 && STAGE_BYTES % 1024 == 0, "swizzle");
   static_assert(N % 16 == 0 && N <= 256, "UMMA N");
@@ -136,6 +143,20 @@ __device__ __forceinline__ void umma_mx_pair(uint32_t d_tmem, uint64_t adesc, ui
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::2.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
           d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// kind::mxf4 on the pair: A and B packed E2M1 (K = 64 per UMMA), two E8M0
+// scale bytes per row (bytes sf_id, sf_id + 1 of the row's scale word).
+__device__ __forceinline__ void umma_mxf4_pair(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                               uint32_t idesc, uint32_t sfa_tmem,
+                                               uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.scale_vec::2X [%0], %1, %2, %3, [%5], [%6], "
+      "p;\n\t}" ::"r"(d_tmem),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
       : "memory");
 }
@@ -251,7 +272,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
   const int K = args.K;
   const int G = K / 32;
   const int KB = args.KB;
-  const bool tail = (K % 128) != 0;   // K % 64 == 0: the tail k-block has 2 K steps
+  // K % 64 == 0: a K that is not a multiple of the k-block ends with a block
+  // [K - KBK, K) of which only the steps past the previous block are issued
+  const bool tail = (K % C::KBK) != 0;
+  const int tail_steps = (K % C::KBK) / 64;   // F4: K = 64 steps in the tail block
   // tile -> expert, weight tile nt, token pair-tile mt (token tiles fastest, so
   // that neighbouring pairs share a weight tile in L2), rows of this CTA's half
   struct Tile {
@@ -319,19 +343,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
           mbar_expect_tx(fb, has_a ? C::TX_FULL : C::B_TX);
           const bool last_tail = tail && kb == KB - 1;
           const int kx = last_tail ? K - 128 : kb * 128;
+          // F4: byte coordinates in the packed rows (two elements per byte)
+          const int kxb = last_tail ? (K - 256) / 2 : kb * 128;
           if (has_a) {
             if (ACT == ACT_HILO)
               tma_load_3d(st, &tmA, kx, t.arow, 0, fb);   // hi rows, then lo rows
             else if (ACT == ACT_E4M3)
               tma_load_2d(st, &tmA, kx, t.arow, fb);
+            else if (ACT == ACT_F4)
+              tma_load_2d(st, &tmA, kxb, t.arow, fb);
             else
               tma_load_2d(st, last_tail ? &tmAt : &tmA, last_tail ? 0 : kb * 128, t.arow, fb);
             bulk_load(st + C::OFF_SFA,
                       args.sfa + (static_cast<size_t>(t.ttile) * KB + kb) * C::SFA_BYTES,
                       C::SFA_BYTES, fb);
           }
-          tma_load_3d(st + C::OFF_B, last_tail ? &tmBt : &tmB, last_tail ? 0 : kb * 128, wrow, t.e,
-                      fb);
+          if (ACT == ACT_F4)
+            tma_load_3d(st + C::OFF_B, &tmB, kxb, wrow, t.e, fb);
+          else
+            tma_load_3d(st + C::OFF_B, last_tail ? &tmBt : &tmB, last_tail ? 0 : kb * 128, wrow,
+                        t.e, fb);
           if (++s == S) { s = 0; ph ^= 1; }
           if (kb == kb_next && tile + npairs < total && !(ok = load_tile_scales(tile + npairs, it + 1)))
             break;
@@ -351,21 +382,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
       if (!(ok = mbar_wait(bar_tsFull(b), (it >> 1) & 1, abort_flag, args.status))) break;
       const uint8_t* ts = smem + C::OFF_TS + b * C::TS_BYTES;
       for (int kb = 0; kb < KB; ++kb) {
-        const int gs = (tail && kb == KB - 1) ? G - 4 : 4 * kb;
-        uint32_t w[8];
+        // groups of this k-block: 4 (8 for F4); the tail block is [K - KBK, K)
+        constexpr int GPB = C::KBK / 32;
+        const int gs = (tail && kb == KB - 1) ? G - GPB : GPB * kb;
+        uint32_t w[C::F4 ? 16 : 8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           const int c = 32 * j + lane;
-          w[j] = 0;
-          if (c < C::N) {
-            const uint16_t* p = reinterpret_cast<const uint16_t*>(ts + c * G + gs);
-            w[j] = static_cast<uint32_t>(p[0]) | (static_cast<uint32_t>(p[1]) << 16);
+#pragma unroll
+          for (int q = 0; q < GPB / 4; ++q) {
+            // word q of column c: the scale bytes of groups gs + 4q .. + 3
+            // (2-byte aligned pairs; a group before the row start, possible
+            // only in a tail block whose first steps are not issued, reads 0)
+            uint32_t v = 0;
+            if (c < C::N) {
+              const int g0 = gs + 4 * q;
+              const uint16_t* p = reinterpret_cast<const uint16_t*>(ts + c * G);
+              const uint32_t lo = g0 >= 0 ? p[g0 >> 1] : 0u;
+              const uint32_t hi = g0 + 2 >= 0 ? p[(g0 >> 1) + 1] : 0u;
+              v = lo | (hi << 16);
+            }
+            w[8 * q + j] = v;
           }
         }
         if (!(ok = mbar_wait(bar_empty(s), ph ^ 1, abort_flag, args.status))) break;
         uint8_t* sfb = smem + s * C::STAGE_BYTES + C::OFF_SFB;
-        *reinterpret_cast<uint4*>(sfb + lane * 16) = make_uint4(w[0], w[1], w[2], w[3]);
-        *reinterpret_cast<uint4*>(sfb + 512 + lane * 16) = make_uint4(w[4], w[5], w[6], w[7]);
+        // atoms: [word 0: columns 0-127, 128-255][word 1: ...] (F4 has two words)
+#pragma unroll
+        for (int q = 0; q < GPB / 4; ++q) {
+          *reinterpret_cast<uint4*>(sfb + 1024 * q + lane * 16) =
+              make_uint4(w[8 * q], w[8 * q + 1], w[8 * q + 2], w[8 * q + 3]);
+          *reinterpret_cast<uint4*>(sfb + 1024 * q + 512 + lane * 16) =
+              make_uint4(w[8 * q + 4], w[8 * q + 5], w[8 * q + 6], w[8 * q + 7]);
+        }
         // orders these shared-memory writes (and the tile-scale reads) before
         // the async-proxy accesses that follow: tcgen05.cp of the atoms, the
         // next bulk copy into the tile-scale buffer
@@ -381,7 +430,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
     // ----------------------------------------- UMMA issuer (even CTA) --
     if (rank == 0 && lane == 0) {
       const uint32_t sfa_t = tmem_base + C::SF_COL0;
-      const uint32_t sfb_t = sfa_t + 4 * C::TERMS;
+      const uint32_t sfb_t = sfa_t + C::SFA_COLS;
       int s = 0, ph = 0, it = 0;
       bool ok = true;
       for (int tile = pair_id; tile < total && ok; tile += npairs, ++it) {
@@ -397,22 +446,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
           if (!(ok = mbar_wait_cluster(bar_peerFull(s), ph, abort_flag, args.status))) break;
           tc_fence_after();
           const uint32_t st = sbase + s * C::STAGE_BYTES;
+          // scale atoms (each 4 TMEM columns): A's terms (or F4's two words),
+          // then B's (two per word)
 #pragma unroll
-          for (int h = 0; h < C::TERMS; ++h)
-            tmem_cp_32x128b_x4_pair(sfa_t + 4 * h, sdesc_k_noswizzle(st + C::OFF_SFA + 512 * h, 128));
-          tmem_cp_32x128b_x4_pair(sfb_t, sdesc_k_noswizzle(st + C::OFF_SFB, 128));
-          tmem_cp_32x128b_x4_pair(sfb_t + 4, sdesc_k_noswizzle(st + C::OFF_SFB + 512, 128));
-          // K steps with compile-time indices; the tail k-block of a K that is
-          // 64 mod 128 issues its last two steps only
+          for (int a = 0; a < C::SFA_BYTES / 512; ++a)
+            tmem_cp_32x128b_x4_pair(sfa_t + 4 * a, sdesc_k_noswizzle(st + C::OFF_SFA + 512 * a, 128));
+#pragma unroll
+          for (int a = 0; a < C::SFB_BYTES / 512; ++a)
+            tmem_cp_32x128b_x4_pair(sfb_t + 4 * a, sdesc_k_noswizzle(st + C::OFF_SFB + 512 * a, 128));
+          // K steps with compile-time indices; a tail k-block issues only its
+          // steps past the previous block
           auto step = [&](const int kk) {
-#pragma unroll
-            for (int h = 0; h < C::TERMS; ++h) {
-              umma_mx_pair(d, sdesc_k_sw128(st + h * C::A_PLANE + kk * 32),
-                           sdesc_k_sw128(st + C::OFF_B + kk * 32),
-                           idesc_pair(256, C::N, C::ATYPE, static_cast<uint32_t>(kk)),
-                           (sfa_t + 4 * h) | (static_cast<uint32_t>(kk) << 30),
-                           sfb_t | (static_cast<uint32_t>(kk) << 30), accum);
+            if (C::F4) {
+              const uint32_t id = static_cast<uint32_t>(kk & 1) * 2;
+              umma_mxf4_pair(d, sdesc_k_sw128(st + kk * 32), sdesc_k_sw128(st + C::OFF_B + kk * 32),
+                             idesc_mxf4(256, C::N, id, id), (sfa_t + 4 * (kk >> 1)) | (id << 30),
+                             (sfb_t + 8 * (kk >> 1)) | (id << 30), accum);
               accum = 1;
+            } else {
+#pragma unroll
+              for (int h = 0; h < C::TERMS; ++h) {
+                umma_mx_pair(d, sdesc_k_sw128(st + h * C::A_PLANE + kk * 32),
+                             sdesc_k_sw128(st + C::OFF_B + kk * 32),
+                             idesc_pair(256, C::N, C::ATYPE, static_cast<uint32_t>(kk)),
+                             (sfa_t + 4 * h) | (static_cast<uint32_t>(kk) << 30),
+                             sfb_t | (static_cast<uint32_t>(kk) << 30), accum);
+                accum = 1;
+              }
             }
           };
           if (!(tail && kb == KB - 1)) {
@@ -420,8 +480,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             step(1);
             step(2);
             step(3);
-          } else {
+          } else if (tail_steps == 3) {
+            step(1);
             step(2);
+            step(3);
+          } else if (tail_steps == 2) {
+            step(2);
+            step(3);
+          } else {
             step(3);
           }
           umma_commit_pair(bar_empty(s));
@@ -494,8 +560,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
 #pragma unroll
           for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(h[i]));
           int kb4, kk4;
-          pair_group_to_kblock(jg / 32, args.I / 32, args.h_kb, kb4, kk4);
-          uint8_t* blk = args.h_sfa + (static_cast<size_t>(t.ttile) * args.h_kb + kb4) * C::SFA_BYTES;
+          uint8_t* blk;
+          if (C::F4) {
+            // 256-wide k-blocks of the kind::mxf4 down GEMM: group byte b
+            // (0..7) of the block in atom b / 4
+            const int gI = args.I / 32, g = jg / 32;
+            int b;
+            if ((gI % 8) == 0 || g < 8 * (args.h_kb - 1)) {
+              kb4 = g >> 3;
+              b = g & 7;
+            } else {
+              kb4 = args.h_kb - 1;
+              b = g - (gI - 8);
+            }
+            kk4 = b & 3;
+            blk = args.h_sfa + (static_cast<size_t>(t.ttile) * args.h_kb + kb4) * C::SFA_BYTES +
+                  512 * (b >> 2);
+          } else {
+            pair_group_to_kblock(jg / 32, args.I / 32, args.h_kb, kb4, kk4);
+            blk = args.h_sfa + (static_cast<size_t>(t.ttile) * args.h_kb + kb4) * C::SFA_BYTES;
+          }
           if (ACT == ACT_HILO) {
             int eh = 0;
             if (amax != 0.f) {
@@ -529,7 +613,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
             blk[atom_offset(m, kk4)] = static_cast<uint8_t>(eh + 127);
             blk[512 + atom_offset(m, kk4)] = static_cast<uint8_t>(eh + 123);
           } else {
-            constexpr int emax = ACT == ACT_E2M1 ? 2 : 8;
+            constexpr int emax = (ACT == ACT_E2M1 || ACT == ACT_F4) ? 2 : 8;
             int ex = 0;
             if (amax > 0.f)
               ex = max(static_cast<int>((__float_as_uint(amax) >> 23) & 0xFF) - 127 - emax, -127);
@@ -615,6 +699,7 @@ template <int EPI, int ACT>
 cudaError_t launch_pair_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st) {
   using C = PairCfg<EPI, ACT>;
   if (p.K % 64 != 0 || p.K < 128 || p.K > kMxMaxK || p.act != ACT) return cudaErrorInvalidValue;
+  if (C::F4 && p.K < 256) return cudaErrorInvalidValue;   // a k-block is 256 elements
   if (ACT == ACT_HILO && p.b_lo != p.b_hi + static_cast<size_t>(p.tok_rows) * p.K)
     return cudaErrorInvalidValue;
   static bool attr_set[64] = {false};
@@ -634,6 +719,10 @@ cudaError_t launch_pair_impl(const MxGemmProblem& p, int num_sms, cudaStream_t s
   } else if (ACT == ACT_E4M3) {
     ok = mx_make_tok8_map1(&tmA, p.b_hi, p.tok_rows, p.K, C::MT);
     tmAt = tmA;
+  } else if (ACT == ACT_F4) {
+    // packed rows of K/2 bytes, read as bytes: 128 bytes = 256 elements
+    ok = mx_make_tok8_map1(&tmA, p.b_hi, p.tok_rows, p.K / 2, C::MT);
+    tmAt = tmA;
   } else {
     const cuuint64_t dims[1] = {static_cast<cuuint64_t>(p.tok_rows)};
     const cuuint64_t strides[1] = {static_cast<cuuint64_t>(p.K / 2)};
@@ -643,10 +732,18 @@ cudaError_t launch_pair_impl(const MxGemmProblem& p, int num_sms, cudaStream_t s
   const int rows = EPI == PAIR_SWIGLU ? 2 * p.I : p.n_out;
   {
     const cuuint64_t rb = static_cast<cuuint64_t>(p.K / 2);
-    const cuuint64_t dims[2] = {static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(p.E)};
-    const cuuint64_t strides[2] = {rb, rb * static_cast<cuuint64_t>(rows)};
-    const cuuint32_t box[2] = {static_cast<cuuint32_t>(C::NH), 1};
-    ok = ok && mx_make_code_maps(&tmB, &tmBt, p.codes, p.K, 3, dims, strides, box);
+    if (ACT == ACT_F4) {
+      const cuuint64_t dims[3] = {rb, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(p.E)};
+      const cuuint64_t strides[2] = {rb, rb * static_cast<cuuint64_t>(rows)};
+      const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(C::NH), 1};
+      ok = ok && mx_make_bytes_map(&tmB, p.codes, 3, dims, strides, box);
+      tmBt = tmB;
+    } else {
+      const cuuint64_t dims[2] = {static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(p.E)};
+      const cuuint64_t strides[2] = {rb, rb * static_cast<cuuint64_t>(rows)};
+      const cuuint32_t box[2] = {static_cast<cuuint32_t>(C::NH), 1};
+      ok = ok && mx_make_code_maps(&tmB, &tmBt, p.codes, p.K, 3, dims, strides, box);
+    }
   }
   if (!ok) return cudaErrorInvalidValue;
   PairArgs a;
@@ -657,13 +754,13 @@ cudaError_t launch_pair_impl(const MxGemmProblem& p, int num_sms, cudaStream_t s
   a.n_out = p.n_out;
   a.n_tiles = EPI == PAIR_SWIGLU ? (p.I + C::NH - 1) / C::NH : (p.n_out + C::N - 1) / C::N;
   a.rows_per_expert = rows;
-  a.KB = (p.K + 127) / 128;
+  a.KB = (p.K + C::KBK - 1) / C::KBK;
   a.scales = p.scales;
   a.sfa = p.b_sfb;
   a.h_q = p.h_hi;
   a.h_lo = p.h_lo;
   a.h_sfa = p.h_sfb;
-  a.h_kb = (p.I + 127) / 128;
+  a.h_kb = (p.I + C::KBK - 1) / C::KBK;   // the down GEMM's k-blocks
   a.out_f32 = p.out_f32;
   a.perm = p.perm;
   a.topk_w = p.topk_w;
@@ -685,6 +782,7 @@ cudaError_t launch_mx_pair_gateup_swiglu(const MxGemmProblem& p, int num_sms, cu
     case ACT_HILO: return launch_pair_impl<PAIR_SWIGLU, ACT_HILO>(p, num_sms, st);
     case ACT_E4M3: return launch_pair_impl<PAIR_SWIGLU, ACT_E4M3>(p, num_sms, st);
     case ACT_E2M1: return launch_pair_impl<PAIR_SWIGLU, ACT_E2M1>(p, num_sms, st);
+    case ACT_F4: return launch_pair_impl<PAIR_SWIGLU, ACT_F4>(p, num_sms, st);
   }
   return cudaErrorInvalidValue;
 }
@@ -694,6 +792,7 @@ cudaError_t launch_mx_pair_down(const MxGemmProblem& p, int num_sms, cudaStream_
     case ACT_HILO: return launch_pair_impl<PAIR_DOWN, ACT_HILO>(p, num_sms, st);
     case ACT_E4M3: return launch_pair_impl<PAIR_DOWN, ACT_E4M3>(p, num_sms, st);
     case ACT_E2M1: return launch_pair_impl<PAIR_DOWN, ACT_E2M1>(p, num_sms, st);
+    case ACT_F4: return launch_pair_impl<PAIR_DOWN, ACT_F4>(p, num_sms, st);
   }
   return cudaErrorInvalidValue;
 }

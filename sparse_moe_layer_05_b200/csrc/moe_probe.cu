@@ -73,15 +73,18 @@ __global__ void __launch_bounds__(128, 1)
                           idesc_mx_e2m1_e4m3(128, N, kk, kk), sfa | (kk << 30), sfb | (kk << 30), 1u);
         } else if (KIND == 2) {
           // four K = 64 steps: two scale bytes per row and step, two steps per
-          // 32-bit scale word, so two scale columns per operand
+          // 32-bit scale word, so two scale atoms (4 TMEM columns each) per
+          // operand for the 256 K of the four steps
           tmem_cp_32x128b_x4(sfa, sdesc_k_noswizzle(SF, 128));
+          tmem_cp_32x128b_x4(sfa + 4, sdesc_k_noswizzle(SF, 128));
           tmem_cp_32x128b_x4(sfb, sdesc_k_noswizzle(SF + 512, 128));
+          tmem_cp_32x128b_x4(sfb + 4, sdesc_k_noswizzle(SF + 512, 128));
 #pragma unroll
           for (uint32_t kk = 0; kk < 4; ++kk) {
             const uint32_t id = (kk & 1) * 2;
             umma_mxf4(tb, sdesc_k_sw128(A + kk * 32), sdesc_k_sw128(B + kk * 32),
-                      idesc_mxf4(128, N, id, id), (sfa + (kk >> 1)) | (id << 30),
-                      (sfb + (kk >> 1)) | (id << 30), 1u);
+                      idesc_mxf4(128, N, id, id), (sfa + 4 * (kk >> 1)) | (id << 30),
+                      (sfb + 4 * (kk >> 1)) | (id << 30), 1u);
           }
         } else {
 #pragma unroll

@@ -205,20 +205,32 @@ def mx_padded_rows(offsets, NT):
     return pr
 
 
-def mx_scale_bytes(sfb, pr, K, NT, terms=1):
-    """E8M0 scale bytes [len(pr)][K/32] of the rows at padded positions pr."""
-    G, KB = K // 32, (K + 127) // 128
-    blk = 512 * ((terms * NT + 127) // 128)
+def mx_scale_bytes(sfb, pr, K, NT, terms=1, kb256=False):
+    """E8M0 scale bytes [len(pr)][K/32] of the rows at padded positions pr.
+    kb256: the kind::mxf4 kernel's blocks, 1024 bytes per 256-wide k-block,
+    group byte b (0..7) of a block in atom b // 4."""
+    G = K // 32
+    n = pr % NT
+    w = n // 32
+    atom = (w // 4) * 512 + (n % 32) * 16 + (w % 4) * 4
     out = np.empty((len(pr), G), dtype=np.uint8)
+    if kb256:
+        KB = (K + 255) // 256
+        for g in range(G):
+            if G % 8 == 0 or g < 8 * (KB - 1):
+                kb, b = g // 8, g % 8
+            else:
+                kb, b = KB - 1, g - (G - 8)
+            out[:, g] = sfb[(pr // NT * KB + kb) * 1024 + (b // 4) * 512 + atom + b % 4]
+        return out
+    KB = (K + 127) // 128
+    blk = 512 * ((terms * NT + 127) // 128)
     for g in range(G):
         if G % 4 == 0 or g < 4 * (KB - 1):
             kb, kk = g // 4, g % 4
         else:
             kb, kk = KB - 1, g - (G - 4)
-        n = pr % NT
-        w = n // 32
-        off = (pr // NT * KB + kb) * blk + (w // 4) * 512 + (n % 32) * 16 + (w % 4) * 4 + kk
-        out[:, g] = sfb[off]
+        out[:, g] = sfb[(pr // NT * KB + kb) * blk + atom + kk]
     return out
 
 

@@ -140,9 +140,13 @@ def test_quantised_layer_against_the_simulation(case, mode, policy):
     ws = layer.workspace.cpu().numpy()
     qb = 1 if elem == "e4m3" else 2                   # elements per byte
 
+    # w4a4 on the CTA pair runs kind::mxf4 (d, I >= 256), whose scale blocks
+    # are laid out per 256-wide k-block
+    f4 = mode == "mxfp4" and policy == 5 and P >= 64 * E and min(d, I) >= 256
+
     def rows_of(region, scales, K):
         q = ws[L[region]:L[region] + (int(pr.max()) + 1) * K // qb].reshape(-1, K // qb)[pr]
-        s = G.mx_scale_bytes(ws[L[scales]:], pr, K, NT)
+        s = G.mx_scale_bytes(ws[L[scales]:], pr, K, NT, kb256=f4)
         return G.mx_dequant(q, s, elem)
 
     # (a) x: bit-exact conversion of each routed token's row
@@ -151,9 +155,11 @@ def test_quantised_layer_against_the_simulation(case, mode, policy):
     # (b) H: equal except at rounding midpoints of the fp64 value
     hq = rows_of("h", "h_scales", I)
     flips = total = 0
+    wq_of = {}
     for e, (toks, h) in hidden.items():
         got = hq[offsets[e]:offsets[e + 1]]
         wq = O.mx_quantize(h, elem)
+        wq_of[e] = wq
         total += got.size
         bad = got != wq
         if not bad.any():
@@ -168,19 +174,28 @@ def test_quantised_layer_against_the_simulation(case, mode, policy):
     # (c) the down projection of the GPU's own converted H, weighted and summed
     yw = layer.intermediate("yw", T).cpu().numpy().reshape(T, k, d)
     pre = G.slot_sum_f32(yw)
-    exp = np.zeros((T, d))
+    exp = np.zeros((T, d))       # the GPU's converted H through the fp64 down projection
+    flip = np.zeros((T, d))      # what the H midpoint flips alone contribute
     for e in range(E):
         a, b = offsets[e], offsets[e + 1]
         if a == b:
             continue
         wd = O.mxfp4_decode(inp.Wd_codes[e], inp.Wd_scales[e])
         pairs = perm[a:b]
-        y = hq[a:b] @ wd.T
-        np.add.at(exp, pairs // k, topk_w.reshape(-1)[pairs][:, None].astype(np.float64) * y)
+        pw = topk_w.reshape(-1)[pairs][:, None].astype(np.float64)
+        np.add.at(exp, pairs // k, pw * (hq[a:b] @ wd.T))
+        np.add.at(flip, pairs // k, pw * ((hq[a:b] - wq_of[e]) @ wd.T))
     rd, rms_d, _ = G.rel_rms_err(pre.astype(np.float64), exp)
     assert rd <= 2e-3, rd
     assert np.array_equal(out, G.f32_to_bf16_rne(pre))
-    # (d) the layer against the simulated layer
-    r_out = G.assert_out_close(out, want, what=f"{mode} {name}")
-    print(f"[act_quant] {mode} {name}: H midpoint flips {flips} of {total}; down GEMM on the "
+    # (d) the layer against the simulated layer: within the layer's tolerance
+    # plus the bf16 output's rounding, once the flips' own contribution (either
+    # rounding of a midpoint value is correct) is allowed for
+    got = O.bf16_to_f64(out)
+    r_out, rms, _ = G.rel_rms_err(got, want)
+    bound = G.TOL_REL_RMS * rms + G.BF16_REL * np.abs(want) + np.abs(flip)
+    excess = np.abs(got - want) / bound
+    assert np.all(excess <= 1.0), (mode, name, float(excess.max()), r_out)
+    print(f"[act_quant] {mode} {name} policy {policy}: H midpoint flips {flips} of {total} "
+          f"(moving the layer by up to {np.abs(flip).max() / rms:.2e} x RMS); down GEMM on the "
           f"GPU's H {rd:.2e} x RMS; layer vs simulation {r_out:.3e} x RMS")
