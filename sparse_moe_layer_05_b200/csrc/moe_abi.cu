@@ -245,6 +245,14 @@ struct StageEvents {
 // permutation (counts, offsets, M-tile prefix, perm). Batches of at most
 // kPermChunk tokens take one fused launch for the permutation (identical
 // results). ev marks launches 0..5 of moe_forward_timed.
+// The launches of one pass: the first is ordered after everything earlier on
+// the stream as usual; the rest use programmatic dependent launch (see
+// moe::launch_kernel). Cleared again when the pass's launches are done.
+struct PdlPass {
+  PdlPass() { moe::pdl_launches() = false; }
+  ~PdlPass() { moe::pdl_launches() = false; }
+};
+
 moe_status launch_routing(const uint16_t* x, const float* W_r, const float* b_r, int E, int k,
                           int T, int d, float* logits, int32_t* topk_idx, float* topk_w,
                           int32_t* counts, int32_t* offsets, int32_t* mprefix,
@@ -253,6 +261,7 @@ moe_status launch_routing(const uint16_t* x, const float* W_r, const float* b_r,
   const bool small = T <= moe::kPermChunk;
   ev.mark(0);
   MOE_CUDA(moe::launch_router_logits(x, W_r, b_r, logits, T, E, d, status, st));
+  moe::pdl_launches() = true;
   ev.mark(1);
   MOE_CUDA(moe::launch_topk_softmax(logits, T, E, k, topk_idx, topk_w, st));
   ev.mark(2);
@@ -328,6 +337,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   StageEvents none;
   memset(&none, 0, sizeof(none));
   const StageEvents& E_ = tev ? *tev : none;
+  PdlPass pdl_pass;
   const float* gu_bias = opt.gu_bias;
   const float* dn_bias = opt.dn_bias;
   const int P = T * k;
@@ -903,6 +913,7 @@ moe_status moe_route(const void* x_dev, const float* W_r_dev, const float* b_r_d
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   StageEvents none;
   memset(&none, 0, sizeof(none));
+  PdlPass pdl_pass;
   return launch_routing(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, E, k, T, d,
                         at<float>(workspace_dev, L.pub.logits), topk_idx_dev, topk_w_dev,
                         counts_dev, offsets_dev, at<int32_t>(workspace_dev, L.mprefix),

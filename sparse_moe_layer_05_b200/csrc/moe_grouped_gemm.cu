@@ -164,6 +164,7 @@ __global__ void __launch_bounds__(NUM_THREADS, 1)
     grouped_mxfp4_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                               const __grid_constant__ CUtensorMap tmB,
                               const __grid_constant__ CUtensorMap tmS, const Args args) {
+  pdl_wait_and_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
@@ -475,6 +476,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(pair::NUM_THREADS, 1
     grouped_mxfp4_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                                    const __grid_constant__ CUtensorMap tmB,
                                    const __grid_constant__ CUtensorMap tmS, const Args args) {
+  pdl_wait_and_trigger();
   // local copies shadow the single-CTA kernel's constants of the same names
   constexpr int BMH = pair::BMH;
   constexpr int BK = pair::BK;
@@ -832,6 +834,7 @@ __global__ void __launch_bounds__(swp::NUM_THREADS, 1)
     grouped_mxfp4_gemm_swap_kernel(const __grid_constant__ CUtensorMap tmA,
                                    const __grid_constant__ CUtensorMap tmB,
                                    const __grid_constant__ CUtensorMap tmS, const Args args) {
+  pdl_wait_and_trigger();
   // local copies shadow the single-CTA kernel's constants of the same names
   constexpr int MW = swp::MW, NT = swp::NT, BK = swp::BK, NH = swp::NH;
   constexpr int ST = swp::ST, SW = swp::SW, SC = swp::SC;
@@ -1223,7 +1226,7 @@ cudaError_t launch_swap_impl(const GroupedGemmProblem& p, int num_sms, cudaStrea
   const int64_t tiles_bound =
       ((static_cast<int64_t>(p.P) + swp::NT - 1) / swp::NT + p.E) * a.n_tiles;
   const int grid = static_cast<int>(tiles_bound < num_sms ? tiles_bound : num_sms);
-  grouped_mxfp4_gemm_swap_kernel<EPI><<<grid, swp::NUM_THREADS, swp::SMEM_ALLOC, st>>>(tmA, tmB,
+  launch_kernel(grouped_mxfp4_gemm_swap_kernel<EPI>, dim3(grid), dim3(swp::NUM_THREADS), swp::SMEM_ALLOC, st, tmA, tmB,
                                                                                       tmS, a);
   return cudaGetLastError();
 }
@@ -1272,7 +1275,7 @@ cudaError_t launch_pair_impl(const GroupedGemmProblem& p, int num_sms, cudaStrea
   int64_t pairs = num_sms / 2;
   if (tiles_bound < pairs) pairs = tiles_bound;
   const int grid = static_cast<int>(2 * pairs);
-  grouped_mxfp4_gemm_pair_kernel<EPI><<<grid, pair::NUM_THREADS, pair::SMEM_ALLOC, st>>>(tmA, tmB,
+  launch_kernel(grouped_mxfp4_gemm_pair_kernel<EPI>, dim3(grid), dim3(pair::NUM_THREADS), pair::SMEM_ALLOC, st, tmA, tmB,
                                                                                       tmS, a);
   return cudaGetLastError();
 }
@@ -1318,7 +1321,7 @@ cudaError_t launch_impl(const GroupedGemmProblem& p, int num_sms, cudaStream_t s
   const int64_t mt_bound = (static_cast<int64_t>(p.P) + BM - 1) / BM + p.E;
   const int64_t tiles_bound = mt_bound * a.n_tiles;
   const int grid = static_cast<int>(tiles_bound < num_sms ? tiles_bound : num_sms);
-  grouped_mxfp4_gemm_kernel<EPI><<<grid, NUM_THREADS, SMEM_ALLOC, st>>>(tmA, tmB, tmS, a);
+  launch_kernel(grouped_mxfp4_gemm_kernel<EPI>, dim3(grid), dim3(NUM_THREADS), SMEM_ALLOC, st, tmA, tmB, tmS, a);
   return cudaGetLastError();
 }
 

@@ -8,6 +8,29 @@
 
 namespace moe {
 
+// Launches of a forward pass after its first one are made with programmatic
+// stream serialization (each kernel's launch and prologue overlap its
+// predecessor's tail; every kernel waits for its predecessor before touching
+// global memory, moe_ptx.cuh). The flag is per host thread: the ABI sets it
+// once a pass has launched its first kernel and clears it at the pass's end.
+bool& pdl_launches();
+
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_launches() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Token chunk of the permutation kernels (tokens per block).
 constexpr int kPermChunk = 256;
 // Rows of one M tile of the grouped GEMMs.

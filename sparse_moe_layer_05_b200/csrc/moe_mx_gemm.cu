@@ -208,6 +208,7 @@ __global__ void __launch_bounds__(256) mx_quant_gather_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
     const int32_t* __restrict__ offsets, int E, int P, int k, int K, uint8_t* __restrict__ qhi,
     uint8_t* __restrict__ qlo, uint8_t* __restrict__ sfb) {
+  pdl_wait_and_trigger();
   __shared__ int s_off[kMaxE + 1], s_tb[kMaxE + 1];
   for (int i = threadIdx.x; i <= E; i += blockDim.x) s_off[i] = offsets[i];
   __syncthreads();
@@ -270,6 +271,7 @@ __global__ void __launch_bounds__(256) mx_split_rows_kernel(const uint16_t* __re
                                                             int K, uint8_t* __restrict__ qhi,
                                                             uint8_t* __restrict__ qlo,
                                                             uint8_t* __restrict__ scales) {
+  pdl_wait_and_trigger();
   const int G = K / 32;
   const int64_t n = static_cast<int64_t>(R) * G;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
@@ -314,6 +316,7 @@ __global__ void __launch_bounds__(256) mx_act_quant_gather_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ perm,
     const int32_t* __restrict__ offsets, int E, int P, int k, int K, uint8_t* __restrict__ q,
     uint8_t* __restrict__ sfb) {
+  pdl_wait_and_trigger();
   __shared__ int s_off[kMaxE + 1], s_tb[kMaxE + 1];
   for (int i = threadIdx.x; i <= E; i += blockDim.x) s_off[i] = offsets[i];
   __syncthreads();
@@ -375,6 +378,7 @@ __global__ void __launch_bounds__(256) mx_act_quant_rows_kernel(const uint16_t* 
                                                                 int R, int K,
                                                                 uint8_t* __restrict__ q,
                                                                 uint8_t* __restrict__ scales) {
+  pdl_wait_and_trigger();
   const int G = K / 32;
   constexpr int GB = ACT == ACT_E2M1 ? 16 : 32;
   const int64_t n = static_cast<int64_t>(R) * G;
@@ -484,6 +488,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
                            const __grid_constant__ CUtensorMap tmAt,
                            const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmBt, const MxArgs args) {
+  pdl_wait_and_trigger();
   constexpr int NT = C::NT;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -1077,7 +1082,7 @@ cudaError_t launch_mx_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st)
   int64_t grid = C::CTAS * static_cast<int64_t>(num_sms);
   if (tiles_bound < grid) grid = tiles_bound;
   if (grid < 1) grid = 1;
-  grouped_mx_gemm_kernel<EPI, C><<<static_cast<int>(grid), C::NUM_THREADS, C::SMEM_ALLOC, st>>>(
+  launch_kernel(grouped_mx_gemm_kernel<EPI, C>, dim3(static_cast<int>(grid)), dim3(C::NUM_THREADS), C::SMEM_ALLOC, st, 
       tmA, tmAt, tmB, tmBt, a);
   return cudaGetLastError();
 }
@@ -1139,13 +1144,13 @@ cudaError_t launch_mx_quant_gather(int variant, const uint16_t* x, const int32_t
   const int64_t n = static_cast<int64_t>(P) * (K / 32);
   const int grid = grid_for_n(n, 256, 148 * 8);
   if (variant == kMxPair)
-    mx_quant_gather_kernel<kMxMaxNT><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, qhi, qlo,
+    launch_kernel(mx_quant_gather_kernel<kMxMaxNT>, dim3(grid), dim3(256), 0, st, x, perm, offsets, E, P, k, K, qhi, qlo,
                                                             sfb);
   else if (variant == kMxLarge)
-    mx_quant_gather_kernel<MxLarge::NT><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, qhi,
+    launch_kernel(mx_quant_gather_kernel<MxLarge::NT>, dim3(grid), dim3(256), 0, st, x, perm, offsets, E, P, k, K, qhi,
                                                                qlo, sfb);
   else
-    mx_quant_gather_kernel<MxSmall::NT><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, qhi,
+    launch_kernel(mx_quant_gather_kernel<MxSmall::NT>, dim3(grid), dim3(256), 0, st, x, perm, offsets, E, P, k, K, qhi,
                                                                qlo, sfb);
   return cudaGetLastError();
 }
@@ -1159,18 +1164,18 @@ cudaError_t launch_mx_act_quant_gather(int variant, int act, const uint16_t* x,
   static_assert(NL == kMxMaxNT, "the large and pair variants share the 128-row layout");
   if (act == ACT_E4M3) {
     if (variant != kMxSmall)
-      mx_act_quant_gather_kernel<NL, ACT_E4M3><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, q, sfb);
+      launch_kernel(mx_act_quant_gather_kernel<NL, ACT_E4M3>, dim3(grid), dim3(256), 0, st, x, perm, offsets, E, P, k, K, q, sfb);
     else
-      mx_act_quant_gather_kernel<NS, ACT_E4M3><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, q, sfb);
+      launch_kernel(mx_act_quant_gather_kernel<NS, ACT_E4M3>, dim3(grid), dim3(256), 0, st, x, perm, offsets, E, P, k, K, q, sfb);
   } else if (act == ACT_F4) {
     if (variant != kMxPair) return cudaErrorInvalidValue;
-    mx_act_quant_gather_kernel<NL, ACT_E2M1, true><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k,
+    launch_kernel(mx_act_quant_gather_kernel<NL, ACT_E2M1, true>, dim3(grid), dim3(256), 0, st, x, perm, offsets, E, P, k,
                                                                         K, q, sfb);
   } else if (act == ACT_E2M1) {
     if (variant != kMxSmall)
-      mx_act_quant_gather_kernel<NL, ACT_E2M1><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, q, sfb);
+      launch_kernel(mx_act_quant_gather_kernel<NL, ACT_E2M1>, dim3(grid), dim3(256), 0, st, x, perm, offsets, E, P, k, K, q, sfb);
     else
-      mx_act_quant_gather_kernel<NS, ACT_E2M1><<<grid, 256, 0, st>>>(x, perm, offsets, E, P, k, K, q, sfb);
+      launch_kernel(mx_act_quant_gather_kernel<NS, ACT_E2M1>, dim3(grid), dim3(256), 0, st, x, perm, offsets, E, P, k, K, q, sfb);
   } else {
     return cudaErrorInvalidValue;
   }
@@ -1182,9 +1187,9 @@ cudaError_t launch_mx_act_quant_rows(int act, const uint16_t* x, int R, int K, u
   const int64_t n = static_cast<int64_t>(R) * (K / 32);
   const int grid = grid_for_n(n, 256, 148 * 8);
   if (act == ACT_E4M3)
-    mx_act_quant_rows_kernel<ACT_E4M3><<<grid, 256, 0, st>>>(x, R, K, q, scales);
+    launch_kernel(mx_act_quant_rows_kernel<ACT_E4M3>, dim3(grid), dim3(256), 0, st, x, R, K, q, scales);
   else if (act == ACT_E2M1)
-    mx_act_quant_rows_kernel<ACT_E2M1><<<grid, 256, 0, st>>>(x, R, K, q, scales);
+    launch_kernel(mx_act_quant_rows_kernel<ACT_E2M1>, dim3(grid), dim3(256), 0, st, x, R, K, q, scales);
   else
     return cudaErrorInvalidValue;
   return cudaGetLastError();
@@ -1193,7 +1198,8 @@ cudaError_t launch_mx_act_quant_rows(int act, const uint16_t* x, int R, int K, u
 cudaError_t launch_mx_split_rows(const uint16_t* x, int R, int K, uint8_t* qhi, uint8_t* qlo,
                                  uint8_t* scales, cudaStream_t st) {
   const int64_t n = static_cast<int64_t>(R) * (K / 32);
-  mx_split_rows_kernel<<<grid_for_n(n, 256, 148 * 8), 256, 0, st>>>(x, R, K, qhi, qlo, scales);
+  launch_kernel(mx_split_rows_kernel, dim3(grid_for_n(n, 256, 148 * 8)), dim3(256), 0, st, x, R, K, qhi, qlo,
+                scales);
   return cudaGetLastError();
 }
 

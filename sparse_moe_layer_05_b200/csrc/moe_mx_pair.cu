@@ -36,13 +36,14 @@
 // both CTAs; the even CTA's issuing thread copies them with
 // tcgen05.cp.cta_group::2, which moves each CTA's atom into its own TMEM.
 //
-// Roles (256 threads per CTA):
+// Roles (384 threads per CTA):
 //   warp 0   TMA producer: token rows (A) and their scale block, weight codes
 //            (B); the tile's weight-scale rows into a double buffer
 //   warp 1   TMEM allocation; in the even CTA the UMMA issuer
 //   warp 2   B-scale builder: the tile's weight scales -> two atoms per stage
 //   warp 3   in the odd CTA: relays "stage full" to the even CTA's issuer
-//   warps 4-7 epilogue (TMEM lane quarters 0..3: one token row per thread)
+//   warps 4-11 epilogue: warp w reads TMEM lane quarter w % 4 (one token row
+//            per thread); warps 4-7 and 8-11 take alternate column groups
 // Every wait is bounded (moe_ptx.cuh): a stuck pipeline records a timeout in
 // the status word and the kernel exits.
 #include <cuda_bf16.h>
@@ -112,8 +113,8 @@ struct PairCfg {
   static constexpr int OFF_TAB = OFF_MISC + 16;
   static constexpr int SMEM_BYTES = OFF_TAB + 3 * (kMaxE + 1) * 4;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
-  static constexpr int NUM_THREADS = 256;
-  static constexpr int EPI_WARPS = 4;
+  static constexpr int EPI_WARPS = 8;                     // two per TMEM lane quarter
+  static constexpr int NUM_THREADS = 128 + 32 * EPI_WARPS;
   static constexpr int TMEM_COLS = 512;
   static constexpr int ACC_COLS = N;                      // per accumulator buffer
   static constexpr int SF_COL0 = 2 * N;                   // A scales, then B scales
@@ -195,11 +196,12 @@ struct PairArgs {
 __device__ __forceinline__ float silu_p(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 template <int EPI, int ACT>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     grouped_mx_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmAt,
                            const __grid_constant__ CUtensorMap tmB,
                            const __grid_constant__ CUtensorMap tmBt, const PairArgs args) {
+  pdl_wait_and_trigger();
   using C = PairCfg<EPI, ACT>;
   constexpr int S = C::STAGES;
   extern __shared__ uint8_t smem_raw[];
@@ -275,7 +277,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
   // K % 64 == 0: a K that is not a multiple of the k-block ends with a block
   // [K - KBK, K) of which only the steps past the previous block are issued
   const bool tail = (K % C::KBK) != 0;
-  const int tail_steps = (K % C::KBK) / 64;   // F4: K = 64 steps in the tail block
+  // K steps in the tail block past the previous block (a step is 32 elements
+  // of K, 64 for F4): 2 for the 8-bit kinds, 1..3 for F4
+  const int tail_steps = (K % C::KBK) / (C::F4 ? 64 : 32);
   // tile -> expert, weight tile nt, token pair-tile mt (token tiles fastest, so
   // that neighbouring pairs share a weight tile in L2), rows of this CTA's half
   struct Tile {
@@ -514,7 +518,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
   } else {
     // ----------------------------------------------------------- epilogue --
     const int quad = warp & 3;
-    const int m = quad * 32 + lane;   // token row of this CTA's half
+    const int egrp = (warp - 4) >> 2;   // 0 or 1: alternate column groups
+    const int m = quad * 32 + lane;     // token row of this CTA's half
     int it = 0;
     for (int tile = pair_id; tile < total; tile += npairs, ++it) {
       Tile t;
@@ -532,7 +537,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         const float* brow = args.bias ? args.bias + static_cast<int64_t>(t.e) * 2 * args.I : nullptr;
         const size_t hrow = static_cast<size_t>(t.arow) + m;
 #pragma unroll 1
-        for (int g = 0; g < C::NH / 32; ++g) {
+        for (int g = egrp; g < C::NH / 32; g += 2) {
           const int jg = j0 + 32 * g;
           float h[32];
 #pragma unroll
@@ -655,7 +660,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(256, 1)
         float* orow = args.out_f32 + static_cast<int64_t>(pr) * args.n_out;
         const float* brow = args.bias ? args.bias + static_cast<int64_t>(t.e) * args.n_out : nullptr;
 #pragma unroll 1
-        for (int c = 0; c < C::N; c += 16) {
+        for (int c = 16 * egrp; c < C::N; c += 32) {
           uint32_t y[16];
           tmem_ld16_sync(taddr + c, y);
           const int col = n0 + c;
@@ -770,7 +775,7 @@ cudaError_t launch_pair_impl(const MxGemmProblem& p, int num_sms, cudaStream_t s
   int64_t pairs = num_sms / 2;
   if (tiles_bound < pairs) pairs = tiles_bound;
   if (pairs < 1) pairs = 1;
-  grouped_mx_pair_kernel<EPI, ACT><<<static_cast<int>(2 * pairs), C::NUM_THREADS, C::SMEM_ALLOC, st>>>(
+  launch_kernel(grouped_mx_pair_kernel<EPI, ACT>, dim3(static_cast<int>(2 * pairs)), dim3(C::NUM_THREADS), C::SMEM_ALLOC, st, 
       tmA, tmAt, tmB, tmBt, a);
   return cudaGetLastError();
 }

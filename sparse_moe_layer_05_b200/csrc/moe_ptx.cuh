@@ -16,6 +16,19 @@ constexpr int kStatusTimeout = 5;
 // Wall-clock budget of one bounded wait, in nanoseconds of %globaltimer.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 
+// Programmatic dependent launch. A kernel launched with programmatic stream
+// serialization may start while its predecessor on the stream is still
+// running; griddepcontrol.wait blocks until that predecessor has completed and
+// its memory is visible (a no-op for kernels launched without it). Every
+// kernel of the library executes it before its first global-memory access, so
+// by induction all earlier kernels of the stream have completed by then. The
+// trigger lets the stream's next kernel be scheduled once every CTA of this
+// one has started (its CTAs then wait in griddepcontrol.wait).
+__device__ __forceinline__ void pdl_wait_and_trigger() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -41,6 +41,7 @@ __global__ void __launch_bounds__(RouterCfg<BE>::THREADS)
     router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W_r,
                          const float* __restrict__ b_r, float* __restrict__ logits, int T, int E,
                          int d, int* status) {
+  pdl_wait_and_trigger();
   using C = RouterCfg<BE>;
   extern __shared__ __align__(16) float rsm[];
   const int tid = threadIdx.x;
@@ -198,6 +199,7 @@ __device__ __forceinline__ void router_dot4(const uint16_t* __restrict__ xr,
 __global__ void __launch_bounds__(256) router_logits_small_kernel(
     const uint16_t* __restrict__ x, const float* __restrict__ W_r, const float* __restrict__ b_r,
     float* __restrict__ logits, int T, int E, int d, int* status) {
+  pdl_wait_and_trigger();
   const int t = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (status && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status = 0;
@@ -291,6 +293,7 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
                                                            int T, int E, int k,
                                                            int32_t* __restrict__ topk_idx,
                                                            float* __restrict__ topk_w) {
+  pdl_wait_and_trigger();
   const int lane = threadIdx.x & 31;
   const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   if (t >= T) return;
@@ -302,6 +305,7 @@ __global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restri
 __global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t* __restrict__ topk_idx,
                                                         int T, int k, int E,
                                                         int32_t* __restrict__ chunk_hist) {
+  pdl_wait_and_trigger();
   __shared__ int h[256];
   for (int e = threadIdx.x; e < E; e += blockDim.x) h[e] = 0;
   __syncthreads();
@@ -321,6 +325,7 @@ __global__ void __launch_bounds__(256) perm_scan_kernel(const int32_t* __restric
                                                         int32_t* __restrict__ offsets,
                                                         int32_t* __restrict__ chunk_base,
                                                         int32_t* __restrict__ mtile_prefix) {
+  pdl_wait_and_trigger();
   __shared__ int s_cnt[256], s_mt[256];
   const int e = threadIdx.x;
   int run = 0;
@@ -365,6 +370,7 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(const int32_t* __rest
                                                            const int32_t* __restrict__ chunk_base,
                                                            int32_t* __restrict__ perm,
                                                            int32_t* __restrict__ inv) {
+  pdl_wait_and_trigger();
   __shared__ int wbase[8][256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   for (int i = threadIdx.x; i < 8 * 256; i += blockDim.x) (&wbase[0][0])[i] = 0;
@@ -414,6 +420,7 @@ __global__ void __launch_bounds__(256) perm_small_kernel(const int32_t* __restri
                                                          int32_t* __restrict__ offsets,
                                                          int32_t* __restrict__ mtile_prefix,
                                                          int32_t* __restrict__ perm) {
+  pdl_wait_and_trigger();
   __shared__ int wbase[8][256];
   __shared__ int s_cnt[256], s_mt[256];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -480,6 +487,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
                                                           const int32_t* __restrict__ perm, int P,
                                                           int k, int d,
                                                           uint16_t* __restrict__ xp) {
+  pdl_wait_and_trigger();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   const int vec = d / 8;  // 16-byte vectors per row
@@ -496,6 +504,7 @@ __global__ void __launch_bounds__(256) gather_rows_kernel(const uint16_t* __rest
 __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ yw, int T, int k,
                                                       int d, const uint16_t* __restrict__ resid,
                                                       uint16_t* __restrict__ out) {
+  pdl_wait_and_trigger();
   const int vec = d / 8;
   const int64_t n = (int64_t)T * vec;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
@@ -539,6 +548,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const float* __restrict__ 
 __global__ void __launch_bounds__(256) rms_norm_kernel(const uint16_t* __restrict__ h,
                                                        const float* __restrict__ g, float eps,
                                                        int T, int d, uint16_t* __restrict__ x) {
+  pdl_wait_and_trigger();
   const int lane = threadIdx.x & 31;
   const int nwarps = (gridDim.x * blockDim.x) >> 5;
   for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nwarps) {
@@ -575,6 +585,7 @@ __global__ void __launch_bounds__(256) mxfp4_to_bf16_kernel(const uint8_t* __res
                                                             const uint8_t* __restrict__ scales,
                                                             int rows, int K,
                                                             uint16_t* __restrict__ out) {
+  pdl_wait_and_trigger();
   const int groups = K / 32;
   const int64_t n = (int64_t)rows * groups;
   for (int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; g < n;
@@ -600,6 +611,7 @@ __global__ void __launch_bounds__(256) transpose_scales_kernel(const uint8_t* __
                                                                int N, int G,
                                                                const int32_t* __restrict__ counts,
                                                                uint8_t* __restrict__ out) {
+  pdl_wait_and_trigger();
   extern __shared__ __align__(16) uint8_t tsm[];  // [TR_ROWS][G]
   const int e = blockIdx.y;
   if (counts && counts[e] == 0) return;  // no GEMM tile reads this expert's scales
@@ -633,6 +645,7 @@ __global__ void __launch_bounds__(256) transpose_scales_kernel(const uint8_t* __
 // A bounded wait on a barrier whose phase never completes; the wait gives up
 // after kWaitLimitNs and records MOE_ERR_TIMEOUT in *status.
 __global__ void wait_timeout_selftest_kernel(int* status) {
+  pdl_wait_and_trigger();
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
   if (threadIdx.x == 0) {
@@ -653,6 +666,11 @@ int grid_for(int64_t n, int per_block, int cap) {
 
 }  // namespace
 
+bool& pdl_launches() {
+  static thread_local bool on = false;
+  return on;
+}
+
 template <int BE>
 cudaError_t launch_router_be(const uint16_t* x, const float* W_r, const float* b_r, float* logits,
                              int T, int E, int d, int* status, cudaStream_t st) {
@@ -667,7 +685,7 @@ cudaError_t launch_router_be(const uint16_t* x, const float* W_r, const float* b
     attr_set[dev] = true;
   }
   dim3 grid((T + RT_T - 1) / RT_T, (E + BE - 1) / BE);
-  router_logits_kernel<BE><<<grid, C::THREADS, C::SMEM, st>>>(x, W_r, b_r, logits, T, E, d, status);
+  launch_kernel(router_logits_kernel<BE>, dim3(grid), dim3(C::THREADS), C::SMEM, st, x, W_r, b_r, logits, T, E, d, status);
   return cudaGetLastError();
 }
 
@@ -676,7 +694,7 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, const floa
                                  cudaStream_t st) {
   if (T <= kRouterSmallT) {
     dim3 grid(T, (E + RS_EXPERTS - 1) / RS_EXPERTS);
-    router_logits_small_kernel<<<grid, 256, 0, st>>>(x, W_r, b_r, logits, T, E, d, status);
+    launch_kernel(router_logits_small_kernel, dim3(grid), dim3(256), 0, st, x, W_r, b_r, logits, T, E, d, status);
     return cudaGetLastError();
   }
   if (E <= 32) return launch_router_be<32>(x, W_r, b_r, logits, T, E, d, status, st);
@@ -687,26 +705,26 @@ cudaError_t launch_perm_small(const int32_t* topk_idx, int T, int k, int E, int3
                               int32_t* offsets, int32_t* mtile_prefix, int32_t* perm,
                               cudaStream_t st) {
   if (T < 1 || T > kPermChunk) return cudaErrorInvalidValue;
-  perm_small_kernel<<<1, 256, 0, st>>>(topk_idx, T, k, E, counts, offsets, mtile_prefix, perm);
+  launch_kernel(perm_small_kernel, dim3(1), dim3(256), 0, st, topk_idx, T, k, E, counts, offsets, mtile_prefix, perm);
   return cudaGetLastError();
 }
 
 cudaError_t launch_topk_softmax(const float* logits, int T, int E, int k, int32_t* topk_idx,
                                 float* topk_w, cudaStream_t st) {
-  topk_softmax_kernel<<<(T + 7) / 8, 256, 0, st>>>(logits, T, E, k, topk_idx, topk_w);
+  launch_kernel(topk_softmax_kernel, dim3((T + 7) / 8), dim3(256), 0, st, logits, T, E, k, topk_idx, topk_w);
   return cudaGetLastError();
 }
 
 cudaError_t launch_perm_hist(const int32_t* topk_idx, int T, int k, int E, int32_t* chunk_hist,
                              cudaStream_t st) {
-  perm_hist_kernel<<<perm_chunks(T), 256, 0, st>>>(topk_idx, T, k, E, chunk_hist);
+  launch_kernel(perm_hist_kernel, dim3(perm_chunks(T)), dim3(256), 0, st, topk_idx, T, k, E, chunk_hist);
   return cudaGetLastError();
 }
 
 cudaError_t launch_perm_scan(const int32_t* chunk_hist, int nchunks, int E, int32_t* counts,
                              int32_t* offsets, int32_t* chunk_base, int32_t* mtile_prefix,
                              cudaStream_t st) {
-  perm_scan_kernel<<<1, 256, 0, st>>>(chunk_hist, nchunks, E, counts, offsets, chunk_base,
+  launch_kernel(perm_scan_kernel, dim3(1), dim3(256), 0, st, chunk_hist, nchunks, E, counts, offsets, chunk_base,
                                       mtile_prefix);
   return cudaGetLastError();
 }
@@ -714,26 +732,28 @@ cudaError_t launch_perm_scan(const int32_t* chunk_hist, int nchunks, int E, int3
 cudaError_t launch_perm_scatter(const int32_t* topk_idx, int T, int k, int E,
                                 const int32_t* chunk_base, int32_t* perm, int32_t* inv,
                                 cudaStream_t st) {
-  perm_scatter_kernel<<<perm_chunks(T), 256, 0, st>>>(topk_idx, T, k, E, chunk_base, perm, inv);
+  launch_kernel(perm_scatter_kernel, dim3(perm_chunks(T)), dim3(256), 0, st, topk_idx, T, k, E, chunk_base, perm, inv);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gather_rows(const uint16_t* x, const int32_t* perm, int P, int k, int d,
                                uint16_t* xp, cudaStream_t st) {
-  gather_rows_kernel<<<grid_for(P, 8, 148 * 16), 256, 0, st>>>(x, perm, P, k, d, xp);
+  launch_kernel(gather_rows_kernel, dim3(grid_for(P, 8, 148 * 16)), dim3(256), 0, st, x, perm, P, k, d,
+                xp);
   return cudaGetLastError();
 }
 
 cudaError_t launch_combine(const float* yw, int T, int k, int d, const uint16_t* resid,
                            uint16_t* out, cudaStream_t st) {
   const int64_t n = (int64_t)T * (d / 8);
-  combine_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(yw, T, k, d, resid, out);
+  launch_kernel(combine_kernel, dim3(grid_for(n, 256, 148 * 16)), dim3(256), 0, st, yw, T, k, d, resid,
+                out);
   return cudaGetLastError();
 }
 
 cudaError_t launch_rms_norm(const uint16_t* h, const float* g, float eps, int T, int d,
                             uint16_t* x, cudaStream_t st) {
-  rms_norm_kernel<<<grid_for(T, 8, 148 * 8), 256, 0, st>>>(h, g, eps, T, d, x);
+  launch_kernel(rms_norm_kernel, dim3(grid_for(T, 8, 148 * 8)), dim3(256), 0, st, h, g, eps, T, d, x);
   return cudaGetLastError();
 }
 
@@ -741,19 +761,20 @@ cudaError_t launch_transpose_scales(const uint8_t* in, int E, int N, int G, cons
                                     uint8_t* out, cudaStream_t st) {
   const int smem = TR_ROWS * G;  // G <= 512 (K <= 16384): at most 32 KB
   dim3 grid((N + TR_ROWS - 1) / TR_ROWS, E);
-  transpose_scales_kernel<<<grid, 256, smem, st>>>(in, N, G, counts, out);
+  launch_kernel(transpose_scales_kernel, dim3(grid), dim3(256), smem, st, in, N, G, counts, out);
   return cudaGetLastError();
 }
 
 cudaError_t launch_mxfp4_to_bf16(const uint8_t* codes, const uint8_t* scales, int rows, int K,
                                  uint16_t* out, cudaStream_t st) {
   const int64_t n = (int64_t)rows * (K / 32);
-  mxfp4_to_bf16_kernel<<<grid_for(n, 256, 148 * 16), 256, 0, st>>>(codes, scales, rows, K, out);
+  launch_kernel(mxfp4_to_bf16_kernel, dim3(grid_for(n, 256, 148 * 16)), dim3(256), 0, st, codes, scales,
+                rows, K, out);
   return cudaGetLastError();
 }
 
 cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t st) {
-  wait_timeout_selftest_kernel<<<1, 32, 0, st>>>(status);
+  launch_kernel(wait_timeout_selftest_kernel, dim3(1), dim3(32), 0, st, status);
   return cudaGetLastError();
 }
 
