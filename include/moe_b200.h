@@ -97,8 +97,10 @@ MOE_API int moe_version(void);
  *                   tokens, the decoded weights as the UMMA A operand),
  *   32 <= P/E < 192 single-CTA tiles (256 x 128, the second 128-row half
  *                   skipped for short expert tails),
- *   P/E >= 192      CTA-pair tiles (a 2-CTA cluster computes 256 x 240 tiles
- *                   with tcgen05 cta_group::2).
+ *   P/E >= 192      CTA-pair tiles: the block-scaled ones (policy 5 below)
+ *                   where the shape allows them, else bf16 CTA-pair tiles (a
+ *                   2-CTA cluster computes 256 x 240 tiles with tcgen05
+ *                   cta_group::2).
  * 1, 2 and 3 force single-CTA, CTA-pair and swapped-operand tiles; these
  * decode the MXFP4 weights to bf16 in shared memory or TMEM and run bf16
  * UMMAs on bf16 activations.
@@ -210,8 +212,10 @@ MOE_API moe_status moe_forward_biased(const void* x_dev, const float* W_r_dev, c
  * run (the quantised modes need the block-scaled tiles' shapes: d and I
  * multiples of 64 in [128, 3072], 32-byte aligned code arrays).
  * The quantised modes always run the block-scaled tiles (E2M1 weights x E4M3
- * or E2M1 activations, kind::mxf8f6f4, one term): 16-token tiles when experts
- * average under 64 rows, else 128-token tiles, on a CTA pair with tile_policy 5.
+ * or E2M1 activations, one term): 16-token tiles when experts average under
+ * 64 rows; 256-token tiles on a CTA pair with tile_policy 5, or with 0 when
+ * experts average 192 rows or more (w4a4 there runs kind::mxf4 when d and I
+ * are at least 256); else 128-token tiles on one CTA.
  * Their intermediates in the workspace: the converted x rows in the xp region
  * and the converted H rows in the h region, in the padded token layout the
  * block-scaled tiles read, their scales at x_scales and h_scales.

@@ -15,9 +15,9 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmoe_b200.so")
-SOURCES = ["moe_abi.cu", "moe_routing.cu", "moe_grouped_gemm.cu", "moe_mx_gemm.cu", "moe_mx_pair.cu",
-           "moe_noalloc.cu"]
-HEADERS = ["moe_ptx.cuh", "moe_internal.h"]
+SOURCES = ["moe_abi.cu", "moe_routing.cu", "moe_router_tc.cu", "moe_grouped_gemm.cu",
+           "moe_mx_gemm.cu", "moe_mx_pair.cu", "moe_noalloc.cu"]
+HEADERS = ["moe_ptx.cuh", "moe_internal.h", "moe_topk.cuh"]
 # the tensor-core rate probe: measurement tooling, a library of its own
 PROBE_LIB = os.path.join(PKG, "libmoe_b200_probe.so")
 PROBE_SOURCES = ["moe_probe.cu"]

@@ -50,6 +50,14 @@ cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, const floa
 cudaError_t launch_perm_small(const int32_t* topk_idx, int T, int k, int E, int32_t* counts,
                               int32_t* offsets, int32_t* mtile_prefix, int32_t* perm,
                               cudaStream_t st);
+// K1 on the tensor cores for T > kRouterSmallT (moe_router_tc.cu): splits
+// W_r into three bf16 terms in `terms` (router_tc_terms_bytes), then one
+// kernel computes the logits, the top-k and the softmax. Its first launch
+// clears *status.
+size_t router_tc_terms_bytes(int E, int d);
+cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b_r, int T, int E,
+                             int k, int d, uint16_t* terms, int32_t* topk_idx, float* topk_w,
+                             int* status, cudaStream_t st);
 // K1: top-k (lower index wins ties) and the selected-set softmax.
 cudaError_t launch_topk_softmax(const float* logits, int T, int E, int k, int32_t* topk_idx,
                                 float* topk_w, cudaStream_t st);
@@ -206,6 +214,9 @@ bool mx_make_tok8_map1(CUtensorMap* m, const uint8_t* q, int rows, int K, int nt
 // them, 128-byte swizzle).
 bool mx_make_bytes_map(CUtensorMap* m, const uint8_t* base, int rank, const cuuint64_t* dims,
                        const cuuint64_t* strides, const cuuint32_t* box);
+// The same for a bf16 tensor.
+bool mx_encode_bf16_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                        const cuuint64_t* strides, const cuuint32_t* box);
 
 // Debug/self-test: one bounded wait on an mbarrier that nothing completes.
 cudaError_t launch_wait_timeout_selftest(int* status, cudaStream_t st);

@@ -1112,6 +1112,10 @@ bool mx_make_bytes_map(CUtensorMap* m, const uint8_t* base, int rank, const cuui
                        const cuuint64_t* strides, const cuuint32_t* box) {
   return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, rank, base, dims, strides, box);
 }
+bool mx_encode_bf16_map(CUtensorMap* m, const void* base, int rank, const cuuint64_t* dims,
+                        const cuuint64_t* strides, const cuuint32_t* box) {
+  return encode_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, rank, base, dims, strides, box);
+}
 
 int mx_tile_tokens(int variant, int act) {
   if (variant == kMxPair) return kMxMaxNT;

@@ -125,10 +125,11 @@ def test_workspace_sizes():
     offs = sorted((v, k) for k, v in L.items() if k != "total")
     assert all(v % 256 == 0 for v, _ in offs)
     assert L["status"] == 0 and L["total"] >= L["yw"] + 400 * 2880 * 2
-    # prefill shapes: 11 launches; batches of <= 256 tokens fuse the three
-    # permutation kernels (-2); decode shapes take the block-scaled path, which
-    # launches no scale transposes (-2)
-    assert B.moe_forward_launch_count(32, 4, 8192, 2880, 2880) == len(B.STAGES)
+    # 11 launches at most; batches of <= 256 tokens fuse the three permutation
+    # kernels (-2); the block-scaled paths (decode shapes, and prefill shapes
+    # on the CTA pair) launch no scale transposes (-2); the bf16 tiles do
+    assert B.moe_forward_launch_count(32, 4, 8192, 2880, 2880) == len(B.STAGES) - 2
+    assert B.moe_forward_launch_count(32, 4, 8192, 352, 224) == len(B.STAGES)
     assert B.moe_forward_launch_count(32, 4, 100, 2880, 2880) == len(B.STAGES) - 4
     assert B.moe_forward_launch_count(32, 4, 100, 352, 2880) == len(B.STAGES) - 2
     assert B.moe_forward_launch_count(128, 4, 300, 2880, 2880) == len(B.STAGES) - 2

@@ -103,6 +103,38 @@ def test_router_silent_init_copies_tie_exactly():
     G.compare_routing(i8, w8, O.route(exp.x, exp.W_r, exp.b_r, 8), copies_of=32)
 
 
+@pytest.mark.parametrize("d,E,k,T", [(64, 256, 32, 300), (2880, 248, 20, 512), (64, 4, 2, 1000),
+                                     (96, 40, 8, 400), (2880, 128, 4, 257)],
+                         ids=["E256_k32", "E248_k20", "E4", "d96", "T257"])
+def test_router_tensor_core_path(d, E, k, T):
+    """Batches over 256 tokens route on the tensor cores (fp32 router weights as
+    three bf16 terms, top-k and softmax in the same kernel): the choice on every
+    token against the oracle, the tables bit-exact. Cases: 256 expert columns (two
+    stages), 4 experts padded to 16, d = 32 mod 64 (a half-empty last k-block), a
+    ragged last 128-token tile."""
+    inp = W.make_custom(d, 64, E, k, T, seed=90 + E)
+    idx, w, counts, offsets, perm = _route_gpu(inp, T)
+    r = O.route(inp.x, inp.W_r, inp.b_r, k)
+    ties = G.compare_routing(idx, w, r)
+    G.check_tables_against_oracle(idx, counts, offsets, perm, r, E)
+    assert np.all(np.abs(w.sum(1) - 1) < 1e-6)
+    print(f"[router] tensor-core path d={d} E={E} k={k} T={T}: near-ties {ties}")
+
+
+def test_router_silent_init_copies_tie_exactly_tensor_cores():
+    """Above 256 tokens (the tensor-core router) duplicated router rows still give
+    bit-identical logits: each copy directly follows its original with an equal
+    weight."""
+    base = W.make_inputs("20b", T=512)
+    exp = W.make_inputs("64a8", T=512)
+    i2, w2, *_ = _route_gpu(base, 512)
+    i8, w8, *_ = _route_gpu(exp, 512)
+    for t in range(512):
+        assert sorted(set(e % 32 for e in i8[t])) == sorted(i2[t].tolist())
+        for j in range(0, 8, 2):
+            assert i8[t, j + 1] == i8[t, j] + 32 and w8[t, j] == w8[t, j + 1]
+
+
 def test_router_max_experts_and_k():
     inp = W.make_custom(64, 64, 256, 32, 100, seed=21)
     idx, w, counts, offsets, perm = _route_gpu(inp, 100)

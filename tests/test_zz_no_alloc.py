@@ -34,6 +34,17 @@ def _outputs(E, k, T):
             torch.empty(T * k, dtype=torch.int32, device=dev))
 
 
+def _tables(idx, E):
+    """counts, offsets and the stable permutation of a top-k choice (integer
+    bookkeeping, written out here so this file needs no oracle for it)."""
+    flat = idx.reshape(-1).astype(np.int64)
+    counts = np.bincount(flat, minlength=E).astype(np.int32)
+    offsets = np.zeros(E + 1, dtype=np.int32)
+    offsets[1:] = np.cumsum(counts)
+    perm = np.argsort(flat, kind="stable").astype(np.int32)
+    return counts, offsets, perm, None
+
+
 def _route_with_workspace(inp, x, W_r, b_r):
     from sparse_moe_layer_05_b200 import binding as B
     E, k, T, d = inp.E, inp.k, inp.T, inp.d
@@ -68,11 +79,23 @@ def test_noalloc_route_matches_workspace_route_on_consecutive_calls():
         want = _route_with_workspace(inp, x, W_r, b_r)
         got = _route_noalloc(inp, x, W_r, b_r)
         idx, w, counts, offsets, perm = got
-        assert np.array_equal(idx, want[0])
-        assert np.max(np.abs(w - want[1])) <= 1e-6        # same kernels: equal in practice
-        assert np.array_equal(counts, want[2])
-        assert np.array_equal(offsets, want[3])
-        assert np.array_equal(perm, want[4])
+        # Above 256 tokens the workspace entry computes the logits on the tensor
+        # cores and this one on the CUDA cores (both fp32 dot products, summed in
+        # different orders), so a token whose k-th and (k+1)-th logits nearly
+        # tie may choose differently: allowed only for the oracle's near-ties
+        # (gap below 1e-5), with the tables then checked for the choice made.
+        same = np.all(idx == want[0], axis=1)
+        if not same.all():
+            from oracle import moe_oracle as O
+            tie = O.route(inp.x, inp.W_r, inp.b_r, inp.k).near_tie(1e-5)
+            assert np.all(tie[~same]), np.nonzero(~same & ~tie)[0][:5]
+            assert (~same).sum() <= 2
+        assert np.max(np.abs(w[same] - want[1][same])) <= 1e-6
+        c, o, p, _ = _tables(idx, inp.E)
+        assert np.array_equal(counts, c) and np.array_equal(offsets, o)
+        assert np.array_equal(perm, p)
+        if same.all():
+            assert np.array_equal(counts, want[2]) and np.array_equal(perm, want[4])
 
 
 def test_noalloc_route_rejects_oversized_calls():
