@@ -311,6 +311,16 @@ MOE_API moe_status moe_forward_hostio(const void* x_host, const float* W_r_dev, 
  * ("Proof", s_i and p_i), then the stable grouping of the T*k (token, slot)
  * pairs by expert.
  *
+ * Precision of the choice: the logits are fp32 dot products on the tensor
+ * cores (the fp32 router weights as three bf16 terms, exactly). Where two
+ * neighbouring logits of a token's top-k list, or the k-th and a runner-up,
+ * lie within tau_t = 2^-17 ||x_t||_2 max_e ||W_r[e]||_2 of each other, their
+ * order is decided on fp64 dot products of the same inputs; so the experts
+ * and their order are those of the exact logits, equal exact logits going to
+ * the lower index. The softmax uses the fp32 logits (the fp64 ones where
+ * they were computed). moe_forward leaves the fp32 logits in its workspace
+ * (moe_workspace_layout's logits, [T][E]).
+ *
  *   topk_idx_dev [T][k] int32, topk_w_dev [T][k] float32
  *   counts_dev   [E]    int32  pairs routed to each expert
  *   offsets_dev  [E+1]  int32  exclusive prefix sum of counts
@@ -334,10 +344,11 @@ MOE_API moe_status moe_route(const void* x_dev, const float* W_r_dev, const floa
  * pages have no counterpart to this entry point; it is a deployment aid.
  *
  * Same arguments, outputs and results as moe_route (all five outputs are
- * required here), minus the workspace. The scratch it needs (router logits
- * and small routing tables) lives in one device array owned by the library:
- * about 4.1 MiB that every GPU which loads the library holds until the
- * process exits. Limit: T * E <= 1,048,576 (e.g. T = 8192 tokens at E = 128,
+ * required here), minus the workspace; it makes the same launches as
+ * moe_route, so its results are bit-identical to moe_route's. The scratch it
+ * needs (router logits, the router's split weights and small routing tables)
+ * lives in one device array owned by the library: 28.1 MiB that every GPU
+ * which loads the library holds until the process exits. Limit: T * E <= 1,048,576 (e.g. T = 8192 tokens at E = 128,
  * or T = 4096 at E = 248); larger calls return MOE_ERR_UNSUPPORTED and
  * launch nothing. Every call looks up the array's device address on the
  * current device (cudaGetSymbolAddress; no address is cached, so a new

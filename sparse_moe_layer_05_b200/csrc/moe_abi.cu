@@ -54,7 +54,7 @@ size_t align256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 struct Layout {
   moe_ws_layout pub;
   size_t mprefix, chunk_hist, chunk_base, x_in, out_buf, gu_scales_t, d_scales_t;
-  size_t router_terms;   // the tensor-core router's bf16 weight terms (T > 256)
+  size_t router_terms;   // the router's bf16 weight terms and row norms
   size_t mx_tok_rows;
   size_t x_norm;   // moe_forward_block: the normalised rows [T][d] bf16
 };
@@ -92,7 +92,7 @@ void make_layout(int E, int k, int T, int d, int I, bool hostio, Layout* L, bool
   L->chunk_hist = take(NB * E * 4);
   L->chunk_base = take(NB * E * 4);
   L->pub.perm = take(P * 4);
-  L->router_terms = take(T > moe::kRouterSmallT ? moe::router_tc_terms_bytes(E, d) : 0);
+  L->router_terms = take(moe::router_tc_scratch_bytes(E, d));
   const size_t tr = moe::mx_tok_rows(static_cast<int>(P), E);
   L->mx_tok_rows = tr;
   auto larger = [](size_t a, size_t b) { return a > b ? a : b; };
@@ -130,7 +130,7 @@ void make_route_layout(int E, int k, int T, int d, Layout* L) {
   L->chunk_hist = take(NB * E * 4);
   L->chunk_base = take(NB * E * 4);
   L->pub.offsets = take(static_cast<size_t>(E + 1) * 4);  // used when the caller passes none
-  L->router_terms = take(T > moe::kRouterSmallT ? moe::router_tc_terms_bytes(E, d) : 0);
+  L->router_terms = take(moe::router_tc_scratch_bytes(E, d));
   L->pub.total = off;
 }
 
@@ -258,26 +258,21 @@ struct PdlPass {
 };
 
 moe_status launch_routing(const uint16_t* x, const float* W_r, const float* b_r, int E, int k,
-                          int T, int d, float* logits, uint16_t* router_terms, int32_t* topk_idx,
+                          int T, int d, float* logits, void* router_terms, int32_t* topk_idx,
                           float* topk_w, int32_t* counts, int32_t* offsets, int32_t* mprefix,
                           int32_t* chunk_hist, int32_t* chunk_base, int32_t* perm, int* status,
                           cudaStream_t st, const StageEvents& ev) {
   const bool small = T <= moe::kPermChunk;
   ev.mark(0);
-  if (T > moe::kRouterSmallT) {
+  {
     // tensor-core logits with the top-k and softmax in the same kernel (its
     // stage time covers both; the top-k stage reads 0)
     moe::pdl_launches() = false;
-    cudaError_t e = moe::launch_router_tc(x, W_r, b_r, T, E, k, d, router_terms, topk_idx, topk_w,
-                                          status, st);
+    cudaError_t e = moe::launch_router_tc(x, W_r, b_r, T, E, k, d, router_terms, logits, topk_idx,
+                                          topk_w, status, st);
     moe::pdl_launches() = true;
     MOE_CUDA(e);
     ev.mark(1);
-  } else {
-    MOE_CUDA(moe::launch_router_logits(x, W_r, b_r, logits, T, E, d, status, st));
-    moe::pdl_launches() = true;
-    ev.mark(1);
-    MOE_CUDA(moe::launch_topk_softmax(logits, T, E, k, topk_idx, topk_w, st));
   }
   ev.mark(2);
   if (!perm) return MOE_OK;
@@ -372,7 +367,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
   uint8_t* gst = at<uint8_t>(ws, L.gu_scales_t);
   uint8_t* dst_ = at<uint8_t>(ws, L.d_scales_t);
 
-  moe_status rs = launch_routing(x, W_r, b_r, E, k, T, d, logits, at<uint16_t>(ws, L.router_terms),
+  moe_status rs = launch_routing(x, W_r, b_r, E, k, T, d, logits, at<void>(ws, L.router_terms),
                                  topk_idx, topk_w, counts, offsets, mprefix, chunk_hist,
                                  chunk_base, perm, status, st, E_);
   if (rs != MOE_OK) return rs;
@@ -934,7 +929,7 @@ moe_status moe_route(const void* x_dev, const float* W_r_dev, const float* b_r_d
   PdlPass pdl_pass;
   return launch_routing(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, E, k, T, d,
                         at<float>(workspace_dev, L.pub.logits),
-                        at<uint16_t>(workspace_dev, L.router_terms), topk_idx_dev, topk_w_dev,
+                        at<void>(workspace_dev, L.router_terms), topk_idx_dev, topk_w_dev,
                         counts_dev, offsets_dev, at<int32_t>(workspace_dev, L.mprefix),
                         at<int32_t>(workspace_dev, L.chunk_hist),
                         at<int32_t>(workspace_dev, L.chunk_base), nperm == 3 ? perm_dev : nullptr,

@@ -31,6 +31,27 @@ cudaError_t launch_kernel(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_
   return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
 }
 
+// Same, as clusters of `cluster` CTAs along x (grid.x a multiple of it).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_kernel_cluster(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                  int cluster, cudaStream_t st, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(cluster);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl_launches() ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 // Token chunk of the permutation kernels (tokens per block).
 constexpr int kPermChunk = 256;
 // Rows of one M tile of the grouped GEMMs.
@@ -38,29 +59,20 @@ constexpr int kTileM = 256;
 
 inline int perm_chunks(int T) { return (T + kPermChunk - 1) / kPermChunk; }
 
-// Batches of at most this many tokens use the warp-per-token router kernel.
-constexpr int kRouterSmallT = 256;
-
-// K1: router logits s[t][e] = W_r[e] . x[t] + b_r[e] in fp32.
-cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, const float* b_r,
-                                 float* logits, int T, int E, int d, int* status_to_clear,
-                                 cudaStream_t st);
 // K2 for T <= kPermChunk in one launch: counts, offsets, M-tile prefix and
 // perm, identical to launch_perm_hist + launch_perm_scan + launch_perm_scatter.
 cudaError_t launch_perm_small(const int32_t* topk_idx, int T, int k, int E, int32_t* counts,
                               int32_t* offsets, int32_t* mtile_prefix, int32_t* perm,
                               cudaStream_t st);
-// K1 on the tensor cores for T > kRouterSmallT (moe_router_tc.cu): splits
-// W_r into three bf16 terms in `terms` (router_tc_terms_bytes), then one
-// kernel computes the logits, the top-k and the softmax. Its first launch
-// clears *status.
-size_t router_tc_terms_bytes(int E, int d);
+// K1, the router (moe_router_tc.cu): splits W_r into three bf16 terms and
+// its row norms in `scratch` (router_tc_scratch_bytes), then one kernel
+// computes the logits (written to `logits`, [T][E] fp32), the top-k with
+// near ties settled in fp64, and the softmax. Its first launch clears
+// *status.
+size_t router_tc_scratch_bytes(int E, int d);
 cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b_r, int T, int E,
-                             int k, int d, uint16_t* terms, int32_t* topk_idx, float* topk_w,
-                             int* status, cudaStream_t st);
-// K1: top-k (lower index wins ties) and the selected-set softmax.
-cudaError_t launch_topk_softmax(const float* logits, int T, int E, int k, int32_t* topk_idx,
-                                float* topk_w, cudaStream_t st);
+                             int k, int d, void* scratch, float* logits, int32_t* topk_idx,
+                             float* topk_w, int* status, cudaStream_t st);
 // K2: per-chunk expert histograms.
 cudaError_t launch_perm_hist(const int32_t* topk_idx, int T, int k, int E, int32_t* chunk_hist,
                              cudaStream_t st);

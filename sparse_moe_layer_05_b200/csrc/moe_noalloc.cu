@@ -27,19 +27,23 @@
 namespace {
 
 // Largest T * E accepted: the fp32 router logits take 4 bytes per
-// (token, expert); the rest of the scratch is small tables.
+// (token, expert). The router's split weights (three bf16 terms per weight
+// and one norm per expert row) take at most 3 * 256 * 16384 * 2 + 1024
+// bytes; the rest of the scratch is small tables.
 constexpr size_t kNoAllocMaxTE = size_t(1) << 20;
-constexpr size_t kNoAllocScratchBytes = kNoAllocMaxTE * 4 + (size_t(64) << 10);
+constexpr size_t kNoAllocRouterBytes = size_t(3) * 256 * 16384 * 2 + 1024;
+constexpr size_t kNoAllocScratchBytes =
+    kNoAllocMaxTE * 4 + kNoAllocRouterBytes + (size_t(64) << 10);
 
 __device__ __align__(256) unsigned char g_route_scratch[kNoAllocScratchBytes];
 
 size_t round256(size_t v) { return (v + 255) & ~static_cast<size_t>(255); }
 
 struct ScratchLayout {
-  size_t status, logits, mprefix, chunk_hist, chunk_base, total;
+  size_t status, logits, router, mprefix, chunk_hist, chunk_base, total;
 };
 
-ScratchLayout scratch_layout(int E, int T) {
+ScratchLayout scratch_layout(int E, int T, int d) {
   const size_t nb = static_cast<size_t>(moe::perm_chunks(T));
   ScratchLayout L;
   size_t off = 0;
@@ -53,6 +57,8 @@ ScratchLayout scratch_layout(int E, int T) {
   off = round256(off + nb * E * 4);
   L.logits = off;
   off = round256(off + static_cast<size_t>(T) * E * 4);
+  L.router = off;
+  off = round256(off + moe::router_tc_scratch_bytes(E, d));
   L.total = off;
   return L;
 }
@@ -92,7 +98,7 @@ moe_status moe_route_noalloc(const void* x_dev, const float* W_r_dev, const floa
   if (static_cast<size_t>(T) * static_cast<size_t>(E) > kNoAllocMaxTE) return MOE_ERR_UNSUPPORTED;
   if (!aligned16(x_dev) || !aligned16(W_r_dev) || !aligned16(b_r_dev)) return MOE_ERR_INVALID_ARG;
   if (T == 0) return MOE_OK;
-  const ScratchLayout L = scratch_layout(E, T);
+  const ScratchLayout L = scratch_layout(E, T, d);
   if (L.total > kNoAllocScratchBytes) return MOE_ERR_UNSUPPORTED;
   void* base = nullptr;
   moe_status s = scratch_base(&base);
@@ -106,26 +112,25 @@ moe_status moe_route_noalloc(const void* x_dev, const float* W_r_dev, const floa
   int32_t* chunk_base = reinterpret_cast<int32_t*>(sb + L.chunk_base);
   // Every buffer below is fully written before it is read; the status word
   // is cleared by the first kernel. Batches of at most kPermChunk tokens take
-  // the fused permutation launch (identical results).
-  if (T <= moe::kPermChunk) {
-    if (moe::launch_router_logits(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, logits, T,
-                                  E, d, status, st) != cudaSuccess ||
-        moe::launch_topk_softmax(logits, T, E, k, topk_idx_dev, topk_w_dev, st) != cudaSuccess ||
-        moe::launch_perm_small(topk_idx_dev, T, k, E, counts_dev, offsets_dev, mprefix, perm_dev,
-                               st) != cudaSuccess) {
-      cudaGetLastError();
-      return MOE_ERR_CUDA;
-    }
-    return MOE_OK;
+  // the fused permutation launch (identical results). The launches are the
+  // ones moe_route makes, in the same order and configuration.
+  const uint16_t* x = static_cast<const uint16_t*>(x_dev);
+  moe::pdl_launches() = false;
+  bool launched = moe::launch_router_tc(x, W_r_dev, b_r_dev, T, E, k, d, sb + L.router, logits,
+                                        topk_idx_dev, topk_w_dev, status, st) == cudaSuccess;
+  if (launched && T <= moe::kPermChunk) {
+    launched = moe::launch_perm_small(topk_idx_dev, T, k, E, counts_dev, offsets_dev, mprefix,
+                                      perm_dev, st) == cudaSuccess;
+  } else if (launched) {
+    launched =
+        moe::launch_perm_hist(topk_idx_dev, T, k, E, chunk_hist, st) == cudaSuccess &&
+        moe::launch_perm_scan(chunk_hist, moe::perm_chunks(T), E, counts_dev, offsets_dev,
+                              chunk_base, mprefix, st) == cudaSuccess &&
+        moe::launch_perm_scatter(topk_idx_dev, T, k, E, chunk_base, perm_dev, nullptr, st) ==
+            cudaSuccess;
   }
-  if (moe::launch_router_logits(static_cast<const uint16_t*>(x_dev), W_r_dev, b_r_dev, logits, T,
-                                E, d, status, st) != cudaSuccess ||
-      moe::launch_topk_softmax(logits, T, E, k, topk_idx_dev, topk_w_dev, st) != cudaSuccess ||
-      moe::launch_perm_hist(topk_idx_dev, T, k, E, chunk_hist, st) != cudaSuccess ||
-      moe::launch_perm_scan(chunk_hist, moe::perm_chunks(T), E, counts_dev, offsets_dev,
-                            chunk_base, mprefix, st) != cudaSuccess ||
-      moe::launch_perm_scatter(topk_idx_dev, T, k, E, chunk_base, perm_dev, nullptr, st) !=
-          cudaSuccess) {
+  moe::pdl_launches() = false;
+  if (!launched) {
     cudaGetLastError();
     return MOE_ERR_CUDA;
   }

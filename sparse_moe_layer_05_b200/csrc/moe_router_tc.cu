@@ -1,5 +1,5 @@
-// moe_router_tc.cu -- the router on the tensor cores, for batches of more than
-// 256 tokens, with the top-k and the selected-set softmax in the same kernel.
+// moe_router_tc.cu -- the router on the tensor cores, with the top-k and the
+// selected-set softmax in the same kernel, for every batch size.
 //
 //   s[t][e] = sum_i x[t][i] W_r[e][i] + b_r[e]
 //   then top-k over e (lower index first on ties) and the softmax over the k
@@ -12,22 +12,45 @@
 // hi = bf16(W), mid = bf16(W - hi), lo = W - hi - mid (each rounding to nearest
 // even): an fp32 value has 24 significant bits and each term holds the next 8,
 // so hi + mid + lo = W exactly (for |W| >= 2^-101, where no term is subnormal).
-// Each product of x with a term is exact in fp32 and the tensor core
-// accumulates them in fp32: the logits are fp32 dot products as on the CUDA
-// cores, in a different summation order. Every expert's column goes through
-// the same operations, so identical router rows still give identical logits.
+// Each product of x with a term is exact in fp32. The x.hi products go to one
+// TMEM accumulator and the x.mid and x.lo products (2^-8 and 2^-16 of the
+// logit's size) to a second, so the accumulator that carries the logit's
+// magnitude sees d/16 accumulation steps, not 3d/16. The logit is
+// hi_acc + lo_acc (+ the partial sums of the other CTAs of the cluster, in
+// rank order) + b_r, in fp32. Every expert's column goes through the same
+// operations, so identical router rows give identical logits.
 //
-// Tiles. One CTA per 128 tokens (UMMA M = 128) and all experts at once (N = E
-// rounded up to 16, at most 256, one TMEM accumulator), 64 elements of d per
-// shared-memory stage: the x tile by one TMA box, the three weight terms by one
-// 3-D box. Twelve UMMAs per stage (4 K steps x 3 terms). The epilogue adds the
-// bias, stores the logits in shared memory (over the drained stages), and one
-// warp per token selects its k experts there.
+// Near ties. The tensor core's fp32 accumulation differs from exact
+// arithmetic by a small multiple of fp32 rounding of the running sums. For
+// token t the kernel takes tau_t = 2^-17 ||x_t||_2 max_e ||W_r[e]||_2 (by
+// Cauchy-Schwarz every partial sum of x_t . W_r[e] is at most
+// ||x_t|| ||W_r[e]|| in size, and 2^-17 of it is far above the error of
+// d/16 fp32 roundings of sums of that size for d <= 16384): where two
+// neighbouring logits of the top-k list (or the k-th and a runner-up) lie
+// within tau_t, their order is decided on fp64 dot products of the original
+// bf16 x and fp32 W_r (moe_topk.cuh), which equal the exact values to about
+// 1e-13 relative. Everywhere else the fp32 order is the exact order.
+//
+// Tiles. One cluster of C CTAs (C = 1, 2, 4 or 8) per 128 tokens (UMMA
+// M = 128): CTA r of the cluster contracts k-blocks [r KB / C, (r+1) KB / C)
+// of d (64 elements per block) for all experts at once (N = E rounded up to
+// 16, at most 256), up to eight shared-memory stages: the x tile by one TMA
+// box, the three weight terms by one 3-D box. Twelve UMMAs per stage (4 K
+// steps x 3 terms). C grows while the grid stays within one wave of the SMs,
+// so small batches (decode) spread d over eight SMs and large ones keep one
+// CTA per token tile. While the UMMAs run, the epilogue warps add up
+// ||x_t||^2 of their token rows from the same stages. At the end each CTA
+// writes its partial logits to shared memory; after a cluster barrier CTA r
+// finishes rows [r 128 / C, (r+1) 128 / C): it adds the C partials (through
+// distributed shared memory, in rank order) and the bias, writes the logits,
+// and one warp per token selects its k experts.
 //
 // Roles (256 threads): warp 0 TMA producer, warp 1 TMEM allocation and UMMA
-// issue, warps 4-7 TMEM -> shared memory; then all eight warps run the top-k.
-// Every wait is bounded (moe_ptx.cuh).
+// issue, warps 4-7 row norms, then TMEM -> shared memory; all eight warps run
+// the top-k. Every wait is bounded (moe_ptx.cuh); every CTA reaches both
+// cluster barriers on every path.
 #include <cuda_bf16.h>
+#include <float.h>
 #include <stdint.h>
 
 #include "moe_internal.h"
@@ -37,17 +60,23 @@
 namespace moe {
 namespace {
 
-constexpr int RT_M = 128;                 // tokens per CTA
+constexpr int RT_M = 128;                 // tokens per cluster
 constexpr int RT_BK = 64;                 // d elements per stage (128 bytes of bf16)
-constexpr int RT_MAX_STAGES = 4;
+constexpr int RT_MAX_STAGES = 8;
+constexpr int RT_MAX_CLUSTER = 8;
 constexpr int RT_THREADS = 256;
 constexpr int RT_SMEM_LIMIT = 232448 - 1024;
+constexpr int RT_FIXED = 1024;            // barriers, TMEM address, flags
+// the refinement margin tau_t relative to ||x_t|| max_e ||W_r[e]|| (2^-17)
+constexpr float kRefineRel = 7.62939453125e-06f;
 
 struct RouterTcShape {
   int npad;          // E rounded up to 16
   int stage_bytes;   // x tile + three weight-term tiles
   int stages;
-  int logits_ld;     // floats per logits row in shared memory
+  int ld;            // floats per partial-logits row in shared memory
+  int tmem_cols;
+  int body;          // stages, or the partial logits and row norms after them
   int smem_alloc;
 };
 
@@ -55,48 +84,96 @@ RouterTcShape router_tc_shape(int E) {
   RouterTcShape s;
   s.npad = (E + 15) / 16 * 16;
   s.stage_bytes = RT_M * 128 + 3 * s.npad * 128;
-  s.logits_ld = s.npad + 4;
-  const int logits_bytes = RT_M * s.logits_ld * 4;
-  const int fixed = 1024;   // barriers and the TMEM address
-  int st = (RT_SMEM_LIMIT - fixed) / s.stage_bytes;
+  s.ld = s.npad + 4;
+  const int partial_bytes = RT_M * s.ld * 4 + RT_M * 4;
+  int st = (RT_SMEM_LIMIT - RT_FIXED - 1024) / s.stage_bytes;
   if (st > RT_MAX_STAGES) st = RT_MAX_STAGES;
   s.stages = st;
-  int body = st * s.stage_bytes;
-  if (body < logits_bytes) body = logits_bytes;
-  s.smem_alloc = body + fixed + 1024;
+  s.body = st * s.stage_bytes;
+  if (s.body < partial_bytes) s.body = (partial_bytes + 1023) / 1024 * 1024;
+  int cols = 32;
+  while (cols < 2 * s.npad) cols *= 2;
+  s.tmem_cols = cols;
+  s.smem_alloc = s.body + RT_FIXED + 1024;
   return s;
 }
 
-// W_r [E][d] fp32 -> terms [3][npad][d] bf16 (rows E..npad-1 zero).
+// W_r [E][d] fp32 -> terms [3][npad][d] bf16 (rows E..npad-1 zero) and
+// norms[npad] = ||W_r[e]||_2 (fp32, in one fixed order; 0 for the padding
+// rows). One block per row.
 __global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ W_r, int E,
                                                            int npad, int d,
                                                            uint16_t* __restrict__ terms,
+                                                           float* __restrict__ norms,
                                                            int* status) {
   pdl_wait_and_trigger();
   // the first kernel of the pass clears the status word
   if (status && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
-  const int64_t n = static_cast<int64_t>(npad) * d;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = i / d;
-    const float w = row < E ? W_r[i] : 0.f;
-    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
-    const float r1 = w - __bfloat162float(hi);
-    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
-    const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
-    terms[i] = __bfloat16_as_ushort(hi);
-    terms[n + i] = __bfloat16_as_ushort(mid);
-    terms[2 * n + i] = __bfloat16_as_ushort(lo);
+  const int row = blockIdx.x;
+  const size_t n = static_cast<size_t>(npad) * d;
+  const size_t base = static_cast<size_t>(row) * d;
+  float ss = 0.f;
+  for (int i = threadIdx.x * 4; i < d; i += 256 * 4) {
+    float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (row < E) w = __ldg(reinterpret_cast<const float4*>(W_r + base + i));
+    const float wv[4] = {w.x, w.y, w.z, w.w};
+    uint16_t h[4], m[4], l[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(wv[j]);
+      const float r1 = wv[j] - __bfloat162float(hi);
+      const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+      const __nv_bfloat16 lo = __float2bfloat16_rn(r1 - __bfloat162float(mid));
+      h[j] = __bfloat16_as_ushort(hi);
+      m[j] = __bfloat16_as_ushort(mid);
+      l[j] = __bfloat16_as_ushort(lo);
+      ss = fmaf(wv[j], wv[j], ss);
+    }
+    *reinterpret_cast<uint2*>(terms + base + i) =
+        make_uint2(h[0] | (uint32_t(h[1]) << 16), h[2] | (uint32_t(h[3]) << 16));
+    *reinterpret_cast<uint2*>(terms + n + base + i) =
+        make_uint2(m[0] | (uint32_t(m[1]) << 16), m[2] | (uint32_t(m[3]) << 16));
+    *reinterpret_cast<uint2*>(terms + 2 * n + base + i) =
+        make_uint2(l[0] | (uint32_t(l[1]) << 16), l[2] | (uint32_t(l[3]) << 16));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, off);
+  __shared__ float red[8];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) s += red[w];
+    norms[row] = sqrtf(s);
   }
 }
 
 struct RouterTcArgs {
+  const uint16_t* x;
+  const float* W_r;
   const float* b_r;
-  int T, E, k, d, npad, stages, logits_ld, stage_bytes;
+  const float* norms;
+  int T, E, k, d, npad, stages, ld, stage_bytes, body, tmem_cols, KB;
+  float* logits;
   int32_t* topk_idx;
   float* topk_w;
   int* status;
 };
+
+// Wait for an mbarrier phase regardless of the abort flag, at most
+// kWaitLimitNs (used only on the way out after a wait gave up).
+__device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity))
+    if (globaltimer_ns() - t0 > kWaitLimitNs) return;
+}
+
+__device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
 
 __global__ void __launch_bounds__(RT_THREADS, 1)
     router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
@@ -108,18 +185,31 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
   const uint32_t sbase = smem_u32(smem);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int S = args.stages;
-  const int body = max(S * args.stage_bytes, RT_M * args.logits_ld * 4);
-  const uint32_t bar0 = sbase + body;
+  const uint32_t bar0 = sbase + args.body;
   auto bar_full = [&](int s) { return bar0 + 8u * s; };
   auto bar_empty = [&](int s) { return bar0 + 8u * (RT_MAX_STAGES + s); };
   const uint32_t bar_acc = bar0 + 8u * (2 * RT_MAX_STAGES);
-  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + body + 8 * (2 * RT_MAX_STAGES + 1));
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + args.body + 8 * (2 * RT_MAX_STAGES + 1));
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  // after the main loop: partial logits [128][ld] and ||x||^2 partials [128]
+  float* partial = reinterpret_cast<float*>(smem);
+  float* xsq_part = partial + RT_M * args.ld;
+
+  const uint32_t rank = cluster_ctarank();
+  uint32_t csize;
+  asm volatile("mov.u32 %0, %%cluster_nctarank;" : "=r"(csize));
+  const int tile = static_cast<int>(blockIdx.x / csize);
+  const int t0 = tile * RT_M;
+  const int kb0 = static_cast<int>(rank) * args.KB / static_cast<int>(csize);
+  const int kb1 = (static_cast<int>(rank) + 1) * args.KB / static_cast<int>(csize);
+  const int nkb = kb1 - kb0;
+
   if (threadIdx.x == 0) {
     *abort_flag = 0;
+    misc[2] = misc[3] = 0;
     for (int s = 0; s < S; ++s) {
       mbar_init(bar_full(s), 1);
-      mbar_init(bar_empty(s), 1);
+      mbar_init(bar_empty(s), 1 + 4);   // the UMMA commit and the four norm warps
     }
     mbar_init(bar_acc, 1);
     fence_mbar_init();
@@ -127,112 +217,249 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     tma_prefetch_desc(&tmW);
   }
   if (warp == 1) {
-    tmem_alloc(smem_u32(misc), 256);
+    tmem_alloc(smem_u32(misc), static_cast<uint32_t>(args.tmem_cols));
     tmem_relinquish();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = misc[0];
-  const int t0 = blockIdx.x * RT_M;
-  const int KB = (args.d + RT_BK - 1) / RT_BK;
+  const uint32_t tmem_lo = tmem_base + static_cast<uint32_t>(args.npad);
   bool ok = true;
 
   if (warp == 0) {
     if (lane == 0) {
-      int s = 0, ph = 0;
+      int s = 0, ph = 0, issued = 0;
       const uint32_t tx = static_cast<uint32_t>(args.stage_bytes);
-      for (int kb = 0; kb < KB; ++kb) {
+      for (int i = 0; i < nkb; ++i) {
         if (!(ok = mbar_wait(bar_empty(s), ph ^ 1, abort_flag, args.status))) break;
         const uint32_t st = sbase + s * args.stage_bytes;
+        const int kx = (kb0 + i) * RT_BK;
         mbar_expect_tx(bar_full(s), tx);
-        tma_load_2d(st, &tmX, kb * RT_BK, t0, bar_full(s));
-        tma_load_3d(st + RT_M * 128, &tmW, kb * RT_BK, 0, 0, bar_full(s));
+        tma_load_2d(st, &tmX, kx, t0, bar_full(s));
+        tma_load_3d(st + RT_M * 128, &tmW, kx, 0, 0, bar_full(s));
+        issued = i + 1;
         if (++s == S) { s = 0; ph ^= 1; }
       }
+      misc[2] = static_cast<uint32_t>(issued);
     }
   } else if (warp == 1) {
     if (lane == 0) {
       const uint32_t idesc = idesc_bf16_f32(RT_M, args.npad);
       const uint32_t term_bytes = static_cast<uint32_t>(args.npad) * 128;
-      int s = 0, ph = 0;
-      for (int kb = 0; kb < KB; ++kb) {
+      int s = 0, ph = 0, consumed = 0;
+      for (int i = 0; i < nkb; ++i) {
         if (!(ok = mbar_wait(bar_full(s), ph, abort_flag, args.status))) break;
+        consumed = i + 1;
         tc_fence_after();
         const uint32_t st = sbase + s * args.stage_bytes;
         const uint32_t wb = st + RT_M * 128;
 #pragma unroll
         for (int kk = 0; kk < RT_BK / 16; ++kk) {
-#pragma unroll
-          for (int h = 0; h < 3; ++h)
-            umma_bf16(tmem_base, sdesc_k_sw128(st + kk * 32),
-                      sdesc_k_sw128(wb + h * term_bytes + kk * 32), idesc,
-                      (kb | kk | h) != 0 ? 1u : 0u);
+          const uint32_t acc = (i | kk) != 0 ? 1u : 0u;
+          const uint64_t ad = sdesc_k_sw128(st + kk * 32);
+          umma_bf16(tmem_base, ad, sdesc_k_sw128(wb + kk * 32), idesc, acc);
+          umma_bf16(tmem_lo, ad, sdesc_k_sw128(wb + term_bytes + kk * 32), idesc, acc);
+          umma_bf16(tmem_lo, ad, sdesc_k_sw128(wb + 2 * term_bytes + kk * 32), idesc, 1u);
         }
         umma_commit(bar_empty(s));
         if (++s == S) { s = 0; ph ^= 1; }
       }
-      if (ok) umma_commit(bar_acc);
+      misc[3] = static_cast<uint32_t>(consumed);
+      // after the issued UMMAs (also when the loop gave up, so that the TMEM
+      // is released only once they are done)
+      umma_commit(bar_acc);
     }
   } else if (warp >= 4) {
-    // TMEM -> shared memory logits (bias added); the stages are drained once
-    // the last commit has arrived
+    // ||x_t||^2 over this CTA's k-blocks from the staged x tiles (row r of a
+    // tile is its 128 bytes at r * 128, chunks permuted by the swizzle), then
+    // the partial logits TMEM -> shared memory once the last commit arrived
     const int quad = warp & 3;
     const int r = quad * 32 + lane;
-    ok = mbar_wait(bar_acc, 0, abort_flag, args.status);
+    float xsq = 0.f;
+    int s = 0, ph = 0;
+    for (int i = 0; i < nkb; ++i) {
+      ok = __all_sync(0xFFFFFFFFu, mbar_wait(bar_full(s), ph, abort_flag, args.status));
+      if (!ok) break;
+      {
+        const uint4* row = reinterpret_cast<const uint4*>(smem + s * args.stage_bytes + r * 128);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 q = row[c];
+          const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            const float a = __uint_as_float(w[j] << 16), b = __uint_as_float(w[j] & 0xFFFF0000u);
+            xsq = fmaf(a, a, xsq);
+            xsq = fmaf(b, b, xsq);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar_empty(s));
+      if (++s == S) { s = 0; ph ^= 1; }
+    }
+    if (ok && nkb > 0) ok = mbar_wait(bar_acc, 0, abort_flag, args.status);
     ok = __all_sync(0xFFFFFFFFu, ok);
-    if (ok) {
-      tc_fence_after();
-      float* row = reinterpret_cast<float*>(smem) + static_cast<size_t>(r) * args.logits_ld;
-      const uint32_t taddr = tmem_base + (static_cast<uint32_t>(quad * 32) << 16);
+    tc_fence_after();
+    float* prow = partial + static_cast<size_t>(r) * args.ld;
+    if (ok && nkb > 0) {
+      const uint32_t lanes = static_cast<uint32_t>(quad * 32) << 16;
       for (int c = 0; c < args.npad; c += 16) {
-        uint32_t v[16];
-        tmem_ld16_sync(taddr + c, v);
+        uint32_t a[16], b[16];
+        tmem_ld16_sync(tmem_base + lanes + c, a);
+        tmem_ld16_sync(tmem_lo + lanes + c, b);
 #pragma unroll
         for (int i = 0; i < 16; i += 4) {
           float4 o;
-          o.x = __uint_as_float(v[i]) + (c + i < args.E ? __ldg(args.b_r + c + i) : 0.f);
-          o.y = __uint_as_float(v[i + 1]) + (c + i + 1 < args.E ? __ldg(args.b_r + c + i + 1) : 0.f);
-          o.z = __uint_as_float(v[i + 2]) + (c + i + 2 < args.E ? __ldg(args.b_r + c + i + 2) : 0.f);
-          o.w = __uint_as_float(v[i + 3]) + (c + i + 3 < args.E ? __ldg(args.b_r + c + i + 3) : 0.f);
-          *reinterpret_cast<float4*>(row + c + i) = o;
+          o.x = __uint_as_float(a[i]) + __uint_as_float(b[i]);
+          o.y = __uint_as_float(a[i + 1]) + __uint_as_float(b[i + 1]);
+          o.z = __uint_as_float(a[i + 2]) + __uint_as_float(b[i + 2]);
+          o.w = __uint_as_float(a[i + 3]) + __uint_as_float(b[i + 3]);
+          *reinterpret_cast<float4*>(prow + c + i) = o;
         }
       }
+    } else {
+      for (int c = 0; c < args.npad; c += 4)
+        *reinterpret_cast<float4*>(prow + c) = make_float4(0.f, 0.f, 0.f, 0.f);
     }
+    xsq_part[r] = xsq;
   }
   tc_fence_before();
   __syncthreads();
-  // top-k and softmax, one warp per token, over the logits in shared memory
-  if (!*abort_flag) {
-    for (int tt = warp; tt < RT_M; tt += RT_THREADS / 32) {
-      const int t = t0 + tt;
-      if (t >= args.T) break;
-      topk_softmax_warp(reinterpret_cast<const float*>(smem) + static_cast<size_t>(tt) * args.logits_ld,
-                        args.E, args.k, lane, args.topk_idx + static_cast<size_t>(t) * args.k,
-                        args.topk_w + static_cast<size_t>(t) * args.k);
-    }
+  if (*abort_flag && threadIdx.x == 0) {
+    // a wait gave up: let the loads still in flight land and the issued UMMAs
+    // finish before the shared and tensor memory are given back (bounded)
+    for (uint32_t i = misc[3]; i < misc[2]; ++i)
+      drain_wait(bar_full(static_cast<int>(i % S)), (i / S) & 1u);
+    drain_wait(bar_acc, 0);
   }
+  __syncthreads();
+  // every CTA's partials are complete and visible to the cluster
+  cluster_sync();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, 256);
+    tmem_dealloc(tmem_base, static_cast<uint32_t>(args.tmem_cols));
   }
+
+  // rows [rank 128 / C, (rank+1) 128 / C): sum of the partials in rank order,
+  // bias, logits out, top-k with near-tie refinement and softmax
+  if (!*abort_flag) {
+    const int E = args.E;
+    float wmax = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = lane + 32 * j;
+      if (e < E) wmax = fmaxf(wmax, __ldg(args.norms + e));
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1)
+      wmax = fmaxf(wmax, __shfl_xor_sync(0xFFFFFFFFu, wmax, off));
+    const int rpc = RT_M / static_cast<int>(csize);
+    const int rbeg = static_cast<int>(rank) * rpc;
+    const uint32_t pbase = smem_u32(partial);
+    const uint32_t xbase = smem_u32(xsq_part);
+    for (int rr = rbeg + warp; rr < rbeg + rpc; rr += RT_THREADS / 32) {
+      const int t = t0 + rr;
+      if (t >= args.T) break;
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int e = lane + 32 * j;
+        v[j] = -FLT_MAX;
+        if (e < E) {
+          const uint32_t a = pbase + static_cast<uint32_t>((rr * args.ld + e) * 4);
+          float s = 0.f;
+          for (uint32_t q = 0; q < csize; ++q) s += ld_shared_cluster_f32(mapa_shared(a, q));
+          v[j] = s + __ldg(args.b_r + e);
+          args.logits[static_cast<size_t>(t) * E + e] = v[j];
+        }
+      }
+      float xsq = 0.f;
+      for (uint32_t q = 0; q < csize; ++q)
+        xsq += ld_shared_cluster_f32(mapa_shared(xbase + static_cast<uint32_t>(rr * 4), q));
+      float tau = kRefineRel * sqrtf(xsq) * wmax;
+      if (!(tau <= FLT_MAX)) tau = 0.f;
+      topk_refine_softmax_warp(v, E, args.k, tau, args.x + static_cast<size_t>(t) * args.d,
+                               args.W_r, args.b_r, args.d, lane,
+                               args.topk_idx + static_cast<size_t>(t) * args.k,
+                               args.topk_w + static_cast<size_t>(t) * args.k);
+    }
+  }
+  // no CTA leaves while another may still read its shared memory
+  cluster_sync();
+}
+
+// Clusters of C CTAs of router_tc_kernel (the largest shared-memory shape)
+// that can be resident at once on the current device, cached per device.
+int max_active_clusters(int dev, int C, size_t smem) {
+  static int cache[64][4] = {};
+  int slot = C == 2 ? 1 : C == 4 ? 2 : C == 8 ? 3 : 0;
+  if (dev < 0 || dev >= 64) return 0;
+  if (!cache[dev][slot]) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(C) * 16);
+    cfg.blockDim = dim3(RT_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = static_cast<unsigned>(C);
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    if (cudaOccupancyMaxActiveClusters(&n, router_tc_kernel, &cfg) != cudaSuccess || n < 1) {
+      cudaGetLastError();
+      n = -1;   // not available: this size is not used
+    }
+    cache[dev][slot] = n;
+  }
+  return cache[dev][slot];
+}
+
+int num_sms_of(int dev) {
+  static int cache[64] = {};
+  if (dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+      n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// CTAs per cluster: doubled (up to 8) while every CTA keeps at least one
+// k-block and all clusters of the grid fit on the device at once.
+int cluster_size(int T, int d, int dev, size_t smem) {
+  const int tiles = (T + RT_M - 1) / RT_M;
+  const int KB = (d + RT_BK - 1) / RT_BK;
+  const int sms = num_sms_of(dev);
+  int C = 1;
+  while (C < RT_MAX_CLUSTER && 2 * C <= KB && tiles * 2 * C <= sms &&
+         tiles <= max_active_clusters(dev, 2 * C, smem))
+    C *= 2;
+  return C;
 }
 
 }  // namespace
 
-size_t router_tc_terms_bytes(int E, int d) {
-  return static_cast<size_t>(3) * ((E + 15) / 16 * 16) * d * 2;
+size_t router_tc_scratch_bytes(int E, int d) {
+  const size_t npad = static_cast<size_t>((E + 15) / 16 * 16);
+  return 3 * npad * static_cast<size_t>(d) * 2 + npad * 4;
 }
 
 cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b_r, int T, int E,
-                             int k, int d, uint16_t* terms, int32_t* topk_idx, float* topk_w,
-                             int* status, cudaStream_t st) {
-  if (E < 1 || E > 256 || d % 32 != 0 || T < 1) return cudaErrorInvalidValue;
+                             int k, int d, void* scratch, float* logits, int32_t* topk_idx,
+                             float* topk_w, int* status, cudaStream_t st) {
+  if (E < 1 || E > 256 || k < 1 || k > E || k > 32 || d % 32 != 0 || T < 1)
+    return cudaErrorInvalidValue;
   const RouterTcShape sh = router_tc_shape(E);
   if (sh.stages < 2) return cudaErrorInvalidValue;
-  static bool attr_set[64] = {false};
   int dev = 0;
   cudaGetDevice(&dev);
+  static bool attr_set[64] = {false};
   if (dev >= 0 && dev < 64 && !attr_set[dev]) {
     // the largest shape's requirement, set once per device
     const RouterTcShape big = router_tc_shape(256);
@@ -242,13 +469,13 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b
     if (e != cudaSuccess) return e;
     attr_set[dev] = true;
   }
+  uint16_t* terms = static_cast<uint16_t*>(scratch);
+  float* norms = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) +
+                                          3 * static_cast<size_t>(sh.npad) * d * 2);
   // the weight split: the first launch of the pass (it clears the status word)
   {
-    const int64_t n = static_cast<int64_t>(sh.npad) * d;
-    int64_t blocks = (n + 255) / 256;
-    if (blocks > 148 * 8) blocks = 148 * 8;
-    cudaError_t e = launch_kernel(router_split_kernel, dim3(static_cast<int>(blocks)), dim3(256), 0,
-                                  st, W_r, E, sh.npad, d, terms, status);
+    cudaError_t e = launch_kernel(router_split_kernel, dim3(sh.npad), dim3(256), 0, st, W_r, E,
+                                  sh.npad, d, terms, norms, status);
     if (e != cudaSuccess) return e;
     pdl_launches() = true;   // the router kernel may overlap the split's tail
   }
@@ -266,21 +493,30 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b
     const cuuint32_t box[3] = {RT_BK, static_cast<cuuint32_t>(sh.npad), 3};
     if (!mx_encode_bf16_map(&tmW, terms, 3, dims, strides, box)) return cudaErrorInvalidValue;
   }
+  const int C = cluster_size(T, d, dev, static_cast<size_t>(router_tc_shape(256).smem_alloc));
   RouterTcArgs a;
+  a.x = x;
+  a.W_r = W_r;
   a.b_r = b_r;
+  a.norms = norms;
   a.T = T;
   a.E = E;
   a.k = k;
   a.d = d;
   a.npad = sh.npad;
   a.stages = sh.stages;
-  a.logits_ld = sh.logits_ld;
+  a.ld = sh.ld;
   a.stage_bytes = sh.stage_bytes;
+  a.body = sh.body;
+  a.tmem_cols = sh.tmem_cols;
+  a.KB = (d + RT_BK - 1) / RT_BK;
+  a.logits = logits;
   a.topk_idx = topk_idx;
   a.topk_w = topk_w;
   a.status = status;
-  return launch_kernel(router_tc_kernel, dim3((T + RT_M - 1) / RT_M), dim3(RT_THREADS),
-                       static_cast<size_t>(sh.smem_alloc), st, tmX, tmW, a);
+  const int tiles = (T + RT_M - 1) / RT_M;
+  return launch_kernel_cluster(router_tc_kernel, dim3(tiles * C), dim3(RT_THREADS),
+                               static_cast<size_t>(sh.smem_alloc), C, st, tmX, tmW, a);
 }
 
 }  // namespace moe

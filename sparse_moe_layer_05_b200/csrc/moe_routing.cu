@@ -1,234 +1,18 @@
-// moe_routing.cu -- router (logits, top-k, selected-set softmax), the stable
-// expert permutation, the activation gather and the per-token combine.
+// moe_routing.cu -- the stable expert permutation, the activation gather and
+// the per-token combine (the router itself is moe_router_tc.cu).
 //
-// Router: "llm-surgery-dark-arts-gpt-oss-40b-64a8-init", section 2, "Proof":
-// s_i = W_r[i] . h + b_r[i]; p_i = exp(s_i) / sum over the selected set.
 // Field guide "gpt-oss 20B", "03 Sparse Mixture of Experts": score all
-// experts, keep the top k, normalise only those.
+// experts, keep the top k, normalise only those, and sum the weighted expert
+// outputs of each token.
 #include <cuda_bf16.h>
 #include <float.h>
 #include <stdint.h>
 
 #include "moe_internal.h"
 #include "moe_ptx.cuh"
-#include "moe_topk.cuh"
 
 namespace moe {
 namespace {
-
-// ------------------------------------------------------------ K1 logits ----
-// Block tile: 32 tokens x BE experts (BE = 32 or 64). Four groups of threads
-// split the contraction: group q accumulates the 32-wide chunks q, q+4, q+8,
-// ... of d in increasing order, each thread holding 4 tokens x 4 experts in
-// fp32 (fma). At the end the four partial sums are added in the fixed order
-// ((g0 + g1) + g2) + g3, then the bias. Every logit of every expert follows
-// the same sequence of operations, so identical router rows give
-// bit-identical logits.
-constexpr int RT_T = 32, RT_K = 32, RT_G = 4;
-
-template <int BE>
-struct RouterCfg {
-  static constexpr int TX = BE / 4;                 // expert groups of 4
-  static constexpr int TY = RT_T / 4;               // token groups of 4
-  static constexpr int GT = TX * TY;                // threads per k-group
-  static constexpr int THREADS = RT_G * GT;         // 128 (BE=32) or 256 (BE=64)
-  static constexpr int XS = RT_K * (RT_T + 4);      // floats per x chunk tile
-  static constexpr int WS = RT_K * (BE + 4);        // floats per W chunk tile
-  static constexpr int SMEM = RT_G * (XS + WS) * 4;
-};
-
-template <int BE>
-__global__ void __launch_bounds__(RouterCfg<BE>::THREADS)
-    router_logits_kernel(const uint16_t* __restrict__ x, const float* __restrict__ W_r,
-                         const float* __restrict__ b_r, float* __restrict__ logits, int T, int E,
-                         int d, int* status) {
-  pdl_wait_and_trigger();
-  using C = RouterCfg<BE>;
-  extern __shared__ __align__(16) float rsm[];
-  const int tid = threadIdx.x;
-  if (status && blockIdx.x == 0 && blockIdx.y == 0 && tid == 0) *status = 0;
-  const int t0 = blockIdx.x * RT_T, e0 = blockIdx.y * BE;
-  const int grp = tid / C::GT, lt = tid % C::GT;
-  const int ty = lt / C::TX, tx = lt % C::TX;
-  float* xs = rsm + grp * (C::XS + C::WS);        // [RT_K][RT_T + 4]
-  float* ws = xs + C::XS;                          // [RT_K][BE + 4]
-  float acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-
-  const int nch = d / RT_K;
-  // items each thread stages per chunk group (x: 16-byte bf16 vectors, W: float4)
-  constexpr int XI = RT_G * RT_T * 4 / C::THREADS;
-  constexpr int WI = RT_G * BE * 8 / C::THREADS;
-  static_assert(XI * C::THREADS == RT_G * RT_T * 4 && WI * C::THREADS == RT_G * BE * 8, "split");
-  uint4 xr[XI];
-  float4 wr[WI];
-  auto fetch = [&](int c0) {  // global -> registers for chunks c0..c0+3
-#pragma unroll
-    for (int u = 0; u < XI; ++u) {
-      const int i = tid + u * C::THREADS;
-      const int g = i / (RT_T * 4), r = i % (RT_T * 4);
-      const int tt = r >> 2, kk = (r & 3) * 8, t = t0 + tt, c = c0 + g;
-      xr[u] = make_uint4(0, 0, 0, 0);
-      if (t < T && c < nch)
-        xr[u] = __ldg(reinterpret_cast<const uint4*>(x + (size_t)t * d + c * RT_K + kk));
-    }
-#pragma unroll
-    for (int u = 0; u < WI; ++u) {
-      const int i = tid + u * C::THREADS;
-      const int g = i / (BE * 8), r = i % (BE * 8);
-      const int ee = r >> 3, kk = (r & 7) * 4, e = e0 + ee, c = c0 + g;
-      wr[u] = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (e < E && c < nch)
-        wr[u] = __ldg(reinterpret_cast<const float4*>(W_r + (size_t)e * d + c * RT_K + kk));
-    }
-  };
-  auto stage = [&]() {  // registers -> shared (transposed to [k][token], [k][expert])
-#pragma unroll
-    for (int u = 0; u < XI; ++u) {
-      const int i = tid + u * C::THREADS;
-      const int g = i / (RT_T * 4), r = i % (RT_T * 4);
-      const int tt = r >> 2, kk = (r & 3) * 8;
-      float* xg = rsm + g * (C::XS + C::WS);
-      const uint32_t w[4] = {xr[u].x, xr[u].y, xr[u].z, xr[u].w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        xg[(kk + 2 * q) * (RT_T + 4) + tt] = __uint_as_float(w[q] << 16);
-        xg[(kk + 2 * q + 1) * (RT_T + 4) + tt] = __uint_as_float(w[q] & 0xFFFF0000u);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < WI; ++u) {
-      const int i = tid + u * C::THREADS;
-      const int g = i / (BE * 8), r = i % (BE * 8);
-      const int ee = r >> 3, kk = (r & 7) * 4;
-      float* wg = rsm + g * (C::XS + C::WS) + C::XS;
-      wg[(kk + 0) * (BE + 4) + ee] = wr[u].x;
-      wg[(kk + 1) * (BE + 4) + ee] = wr[u].y;
-      wg[(kk + 2) * (BE + 4) + ee] = wr[u].z;
-      wg[(kk + 3) * (BE + 4) + ee] = wr[u].w;
-    }
-  };
-  fetch(0);
-  for (int c0 = 0; c0 < nch; c0 += RT_G) {
-    stage();
-    __syncthreads();
-    if (c0 + RT_G < nch) fetch(c0 + RT_G);  // in flight while this group computes
-    if (c0 + grp < nch) {
-#pragma unroll 8
-      for (int kk = 0; kk < RT_K; ++kk) {
-        const float4 a = *reinterpret_cast<const float4*>(&xs[kk * (RT_T + 4) + ty * 4]);
-        const float4 b = *reinterpret_cast<const float4*>(&ws[kk * (BE + 4) + tx * 4]);
-        const float av[4] = {a.x, a.y, a.z, a.w};
-        const float bv[4] = {b.x, b.y, b.z, b.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
-      }
-    }
-    __syncthreads();
-  }
-  // fixed-order combination of the four groups' partial sums
-  float* red = rsm;  // [RT_G - 1][RT_T][BE]
-  if (grp > 0) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j)
-        red[((grp - 1) * RT_T + ty * 4 + i) * BE + tx * 4 + j] = acc[i][j];
-  }
-  __syncthreads();
-  if (grp == 0) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int t = t0 + ty * 4 + i;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int e = e0 + tx * 4 + j;
-        float v = acc[i][j];
-#pragma unroll
-        for (int g = 0; g < RT_G - 1; ++g) v += red[(g * RT_T + ty * 4 + i) * BE + tx * 4 + j];
-        if (t < T && e < E) logits[(size_t)t * E + e] = v + b_r[e];
-      }
-    }
-  }
-}
-
-// ----------------------------------------------- K1 logits, small batches ----
-// For a few tokens the tiled kernel has too few blocks to hide its chunk
-// latency; here one warp computes 4 experts' logits for one token. Lane l
-// accumulates the elements l*4 .. l*4+3 of every 128-element chunk in
-// increasing order (fma, fp32), then a fixed butterfly of shuffles adds the
-// 32 lane sums and the bias follows: every expert's logit sees the same
-// operation sequence, so identical router rows give bit-identical logits.
-constexpr int RS_EXPERTS = 32;  // experts per block (8 warps x 4)
-
-// Logits of experts e0..e0+3 for one token row xr (one warp): after the
-// butterfly every lane holds the four sums (bias not added).
-__device__ __forceinline__ void router_dot4(const uint16_t* __restrict__ xr,
-                                            const float* __restrict__ W_r, int e0, int E, int d,
-                                            int lane, float (&acc)[4]) {
-  acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
-  // unrolled so that several iterations' loads are in flight; the fma order
-  // per expert is unchanged (increasing k)
-#pragma unroll 4
-  for (int k = lane * 4; k < d; k += 128) {
-    const uint2 xv = __ldg(reinterpret_cast<const uint2*>(xr + k));
-    const float x0 = __uint_as_float(xv.x << 16), x1 = __uint_as_float(xv.x & 0xFFFF0000u);
-    const float x2 = __uint_as_float(xv.y << 16), x3 = __uint_as_float(xv.y & 0xFFFF0000u);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int e = e0 + j;
-      if (e < E) {
-        const float4 w = __ldg(reinterpret_cast<const float4*>(W_r + (size_t)e * d + k));
-        acc[j] = fmaf(x0, w.x, acc[j]);
-        acc[j] = fmaf(x1, w.y, acc[j]);
-        acc[j] = fmaf(x2, w.z, acc[j]);
-        acc[j] = fmaf(x3, w.w, acc[j]);
-      }
-    }
-  }
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) acc[j] += __shfl_xor_sync(0xFFFFFFFFu, acc[j], off);
-}
-
-__global__ void __launch_bounds__(256) router_logits_small_kernel(
-    const uint16_t* __restrict__ x, const float* __restrict__ W_r, const float* __restrict__ b_r,
-    float* __restrict__ logits, int T, int E, int d, int* status) {
-  pdl_wait_and_trigger();
-  const int t = blockIdx.x;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (status && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *status = 0;
-  const int e0 = blockIdx.y * RS_EXPERTS + warp * 4;
-  float acc[4];
-  router_dot4(x + (size_t)t * d, W_r, e0, E, d, lane, acc);
-  if (lane < 4) {
-    const int e = e0 + lane;
-    const float v = lane == 0 ? acc[0] : lane == 1 ? acc[1] : lane == 2 ? acc[2] : acc[3];
-    if (e < E) logits[(size_t)t * E + e] = v + b_r[e];
-  }
-}
-
-// ------------------------------------------------------ K1 top-k/softmax ----
-// The warp top-k and softmax (topk_softmax_warp) live in moe_topk.cuh; the
-// tensor-core router uses them too.
-
-__global__ void __launch_bounds__(256) topk_softmax_kernel(const float* __restrict__ logits,
-                                                           int T, int E, int k,
-                                                           int32_t* __restrict__ topk_idx,
-                                                           float* __restrict__ topk_w) {
-  pdl_wait_and_trigger();
-  const int lane = threadIdx.x & 31;
-  const int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (t >= T) return;
-  topk_softmax_warp(logits + (size_t)t * E, E, k, lane, topk_idx + (size_t)t * k,
-                    topk_w + (size_t)t * k);
-}
 
 // --------------------------------------------------------- K2 histogram ----
 __global__ void __launch_bounds__(256) perm_hist_kernel(const int32_t* __restrict__ topk_idx,
@@ -600,47 +384,11 @@ bool& pdl_launches() {
   return on;
 }
 
-template <int BE>
-cudaError_t launch_router_be(const uint16_t* x, const float* W_r, const float* b_r, float* logits,
-                             int T, int E, int d, int* status, cudaStream_t st) {
-  using C = RouterCfg<BE>;
-  static bool attr_set[64] = {false};
-  int dev = 0;
-  cudaGetDevice(&dev);
-  if (dev >= 0 && dev < 64 && !attr_set[dev]) {
-    cudaError_t e = cudaFuncSetAttribute(router_logits_kernel<BE>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e != cudaSuccess) return e;
-    attr_set[dev] = true;
-  }
-  dim3 grid((T + RT_T - 1) / RT_T, (E + BE - 1) / BE);
-  launch_kernel(router_logits_kernel<BE>, dim3(grid), dim3(C::THREADS), C::SMEM, st, x, W_r, b_r, logits, T, E, d, status);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_router_logits(const uint16_t* x, const float* W_r, const float* b_r,
-                                 float* logits, int T, int E, int d, int* status,
-                                 cudaStream_t st) {
-  if (T <= kRouterSmallT) {
-    dim3 grid(T, (E + RS_EXPERTS - 1) / RS_EXPERTS);
-    launch_kernel(router_logits_small_kernel, dim3(grid), dim3(256), 0, st, x, W_r, b_r, logits, T, E, d, status);
-    return cudaGetLastError();
-  }
-  if (E <= 32) return launch_router_be<32>(x, W_r, b_r, logits, T, E, d, status, st);
-  return launch_router_be<64>(x, W_r, b_r, logits, T, E, d, status, st);
-}
-
 cudaError_t launch_perm_small(const int32_t* topk_idx, int T, int k, int E, int32_t* counts,
                               int32_t* offsets, int32_t* mtile_prefix, int32_t* perm,
                               cudaStream_t st) {
   if (T < 1 || T > kPermChunk) return cudaErrorInvalidValue;
   launch_kernel(perm_small_kernel, dim3(1), dim3(256), 0, st, topk_idx, T, k, E, counts, offsets, mtile_prefix, perm);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_topk_softmax(const float* logits, int T, int E, int k, int32_t* topk_idx,
-                                float* topk_w, cudaStream_t st) {
-  launch_kernel(topk_softmax_kernel, dim3((T + 7) / 8), dim3(256), 0, st, logits, T, E, k, topk_idx, topk_w);
   return cudaGetLastError();
 }
 

@@ -1,8 +1,7 @@
 // moe_topk.cuh -- top-k over one token's expert logits and the softmax over
 // the selected set, one warp per token ("llm-surgery-dark-arts-gpt-oss-40b-
 // 64a8-init", section 2, "Proof": i in top-k(s), p_i = exp(s_i) / sum over
-// the selected set). Used by the router kernels of moe_routing.cu and
-// moe_router_tc.cu.
+// the selected set). Used by the router kernel of moe_router_tc.cu.
 #pragma once
 
 #include <float.h>
@@ -10,11 +9,7 @@
 
 namespace moe {
 
-// One warp per token. Lane l holds the logits of experts l, l+32, ...; k rounds
-// of a warp arg-max on (logit descending, index ascending). Lane j keeps the
-// j-th winner; the softmax runs over the k winners only.
-//
-// The arg-max compares 32-bit keys that order the logits totally: a float's
+// The arg-max of the top-k compares 32-bit keys that order the logits totally: a float's
 // bits mapped to an unsigned integer that increases with the value, -0 taken
 // as +0 (equal logits tie, the lower index wins), and every NaN mapped below
 // -inf (key 0). A NaN logit therefore loses to every number, NaNs tie among
@@ -26,22 +21,56 @@ __device__ __forceinline__ uint32_t logit_order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-__device__ __forceinline__ void topk_softmax_warp(const float* s, int E, int k, int lane,
-                                                  int32_t* __restrict__ idx_out,
-                                                  float* __restrict__ w_out) {
-  float v[8];
+// Same 64-bit order for fp64 values (a float widened to double keeps its
+// place among the floats).
+__device__ __forceinline__ uint64_t value_order_key(double f) {
+  if (f != f) return 0ull;
+  uint64_t u = static_cast<uint64_t>(__double_as_longlong(f));
+  if (u == 0x8000000000000000ull) u = 0ull;
+  return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
+}
+
+// One warp per token: the top-k of the token's logits v (lane l holds experts
+// l, l+32, ..., -FLT_MAX past E), the order of near ties settled in fp64, and
+// the softmax over the k selected.
+//
+// 1. Rounds of a warp arg-max on (logit descending, index ascending) list the
+//    k largest logits, then go on while the next one lies within tau of the
+//    k-th (the candidates that might belong in the top k), at most 64
+//    entries. Position p of the list sits in lane p % 32, slot p / 32.
+// 2. An entry is refined when its gap to the entry before or after it is at
+//    most tau: its logit is recomputed as the fp64 dot product of the bf16 x
+//    row with the fp32 router row (every product exact in fp64), plus the
+//    bias. Entries of one chain of near gaps are all refined; entries whose
+//    gaps are all above tau keep their fp32 value, which lies within tau/2 of
+//    the exact one on either side, so no refined entry can pass them.
+// 3. With any entry refined, k rounds of the arg-max over the list (fp64
+//    values) give the final order; otherwise the list's first k entries are
+//    the result.
+// tau = 0 turns the refinement off (the list is then the plain top-k).
+__device__ __forceinline__ void topk_refine_softmax_warp(const float (&v)[8], int E, int k,
+                                                         float tau,
+                                                         const uint16_t* __restrict__ x_row,
+                                                         const float* __restrict__ W_r,
+                                                         const float* __restrict__ b_r, int d,
+                                                         int lane, int32_t* __restrict__ idx_out,
+                                                         float* __restrict__ w_out) {
+  const unsigned full = 0xFFFFFFFFu;
   uint32_t key[8];
   uint32_t taken = 0;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
     const int e = lane + 32 * j;
-    v[j] = (e < E) ? s[e] : -FLT_MAX;
     key[j] = logit_order_key(v[j]);
     if (e >= E) taken |= 1u << j;
   }
-  int my_idx = 0;
-  float my_val = 0.f, top = 0.f;
-  for (int r = 0; r < k; ++r) {
+  int cidx[2] = {0, 0};
+  float cval[2] = {0.f, 0.f};
+  int m = 0;
+  float kth = 0.f;
+  const int maxc = E < 64 ? E : 64;
+  const bool refine = tau > 0.f;
+  for (int r = 0; r < maxc; ++r) {
     uint32_t bk = 0;
     float bv = 0.f;
     int bi = 0x7FFFFFFF;
@@ -57,9 +86,9 @@ __device__ __forceinline__ void topk_softmax_warp(const float* s, int E, int k, 
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
-      const uint32_t ok = __shfl_xor_sync(0xFFFFFFFFu, bk, off);
-      const float ov = __shfl_xor_sync(0xFFFFFFFFu, bv, off);
-      const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, off);
+      const uint32_t ok = __shfl_xor_sync(full, bk, off);
+      const float ov = __shfl_xor_sync(full, bv, off);
+      const int oi = __shfl_xor_sync(full, bi, off);
       const bool better = (bi == 0x7FFFFFFF) ||
                           (oi != 0x7FFFFFFF && (ok > bk || (ok == bk && oi < bi)));
       if (better) {
@@ -68,17 +97,149 @@ __device__ __forceinline__ void topk_softmax_warp(const float* s, int E, int k, 
         bi = oi;
       }
     }
+    // past the k-th: only runners-up within tau of it
+    if (r >= k && !(refine && kth - bv <= tau)) break;
     if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    if (r == 0) top = bv;
-    if (lane == r) {
-      my_idx = bi;
-      my_val = bv;
+    if (r == k - 1) kth = bv;
+    if ((r & 31) == lane) {
+      cidx[r >> 5] = bi;
+      cval[r >> 5] = bv;
+    }
+    m = r + 1;
+  }
+
+  // near gaps: near_p = (p + 1 < m) && cval_p - cval_{p+1} <= tau
+  float nx0 = __shfl_down_sync(full, cval[0], 1);
+  const float head1 = __shfl_sync(full, cval[1], 0);
+  if (lane == 31) nx0 = head1;
+  const float nx1 = __shfl_down_sync(full, cval[1], 1);
+  const bool near0 = refine && lane + 1 < m && cval[0] - nx0 <= tau;
+  const bool near1 = refine && 33 + lane < m && cval[1] - nx1 <= tau;
+  bool pv0 = __shfl_up_sync(full, near0, 1);
+  bool pv1 = __shfl_up_sync(full, near1, 1);
+  const bool tail0 = __shfl_sync(full, near0, 31);
+  if (lane == 0) {
+    pv0 = false;
+    pv1 = tail0;
+  }
+  const uint32_t ref0 = __ballot_sync(full, lane < m && (near0 || pv0));
+  const uint32_t ref1 = __ballot_sync(full, 32 + lane < m && (near1 || pv1));
+
+  int my_idx;
+  double my_val, top;
+  if ((ref0 | ref1) == 0) {
+    my_idx = cidx[0];
+    my_val = static_cast<double>(cval[0]);
+    top = static_cast<double>(__shfl_sync(full, cval[0], 0));
+  } else {
+    double val[2] = {static_cast<double>(cval[0]), static_cast<double>(cval[1])};
+    uint64_t pending = static_cast<uint64_t>(ref0) | (static_cast<uint64_t>(ref1) << 32);
+    const int d128 = d & ~127;
+    while (pending) {
+      // up to four refined entries per pass over the x row
+      int pos[4], ex[4];
+      int ng = 0;
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        pos[g] = -1;
+        ex[g] = 0;
+        if (pending) {
+          const int p = __ffsll(static_cast<long long>(pending)) - 1;
+          pending &= pending - 1;
+          const int src = (p >> 5) ? cidx[1] : cidx[0];
+          pos[g] = p;
+          ex[g] = __shfl_sync(full, src, p & 31);
+          ng = g + 1;
+        }
+      }
+      double acc[4] = {0.0, 0.0, 0.0, 0.0};
+#pragma unroll 2
+      for (int i = 4 * lane; i < d128; i += 128) {
+        const uint2 xb = __ldg(reinterpret_cast<const uint2*>(x_row + i));
+        const double x0 = __uint_as_float(xb.x << 16), x1 = __uint_as_float(xb.x & 0xFFFF0000u);
+        const double x2 = __uint_as_float(xb.y << 16), x3 = __uint_as_float(xb.y & 0xFFFF0000u);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          if (g < ng) {
+            const float4 w =
+                __ldg(reinterpret_cast<const float4*>(W_r + static_cast<size_t>(ex[g]) * d + i));
+            acc[g] = fma(x0, static_cast<double>(w.x), acc[g]);
+            acc[g] = fma(x1, static_cast<double>(w.y), acc[g]);
+            acc[g] = fma(x2, static_cast<double>(w.z), acc[g]);
+            acc[g] = fma(x3, static_cast<double>(w.w), acc[g]);
+          }
+        }
+      }
+      for (int i = d128 + lane; i < d; i += 32) {
+        const double xv = __uint_as_float(static_cast<uint32_t>(__ldg(x_row + i)) << 16);
+#pragma unroll
+        for (int g = 0; g < 4; ++g)
+          if (g < ng)
+            acc[g] = fma(xv, static_cast<double>(__ldg(W_r + static_cast<size_t>(ex[g]) * d + i)),
+                         acc[g]);
+      }
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        if (g < ng) {
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) acc[g] += __shfl_xor_sync(full, acc[g], off);
+          const double s = acc[g] + static_cast<double>(__ldg(b_r + ex[g]));
+          if ((pos[g] & 31) == lane) val[pos[g] >> 5] = s;
+        }
+      }
+    }
+    // the final order over the m entries
+    uint32_t ctaken = 0;
+    if (lane >= m) ctaken |= 1u;
+    if (32 + lane >= m) ctaken |= 2u;
+    uint64_t vk[2] = {value_order_key(val[0]), value_order_key(val[1])};
+    my_idx = 0;
+    my_val = 0.0;
+    top = 0.0;
+    for (int r = 0; r < k; ++r) {
+      uint64_t bk = 0;
+      double bv = 0.0;
+      int bi = 0x7FFFFFFF, bs = -1;
+#pragma unroll
+      for (int s2 = 0; s2 < 2; ++s2) {
+        if (ctaken & (1u << s2)) continue;
+        if (bi == 0x7FFFFFFF || vk[s2] > bk || (vk[s2] == bk && cidx[s2] < bi)) {
+          bk = vk[s2];
+          bv = val[s2];
+          bi = cidx[s2];
+          bs = s2;
+        }
+      }
+      int bl = bs >= 0 ? lane : -1;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) {
+        const uint64_t ok = __shfl_xor_sync(full, bk, off);
+        const double ov = __shfl_xor_sync(full, bv, off);
+        const int oi = __shfl_xor_sync(full, bi, off);
+        const int ol = __shfl_xor_sync(full, bl, off);
+        const int os = __shfl_xor_sync(full, bs, off);
+        const bool better = (bi == 0x7FFFFFFF) ||
+                            (oi != 0x7FFFFFFF && (ok > bk || (ok == bk && oi < bi)));
+        if (better) {
+          bk = ok;
+          bv = ov;
+          bi = oi;
+          bl = ol;
+          bs = os;
+        }
+      }
+      if (bl == lane && bs >= 0) ctaken |= 1u << bs;
+      if (r == 0) top = bv;
+      if (lane == r) {
+        my_idx = bi;
+        my_val = bv;
+      }
     }
   }
-  const float ex = (lane < k) ? expf(my_val - top) : 0.f;
+  const float ex = (lane < k) ? expf(static_cast<float>(my_val - top)) : 0.f;
   float sum = ex;
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, off);
+  for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(full, sum, off);
   if (lane < k) {
     idx_out[lane] = my_idx;
     w_out[lane] = ex / sum;

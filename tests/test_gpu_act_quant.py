@@ -107,14 +107,14 @@ QUANT_CASES = [
 ]
 
 
-@pytest.mark.parametrize("policy", [0, 5], ids=["one_cta", "cta_pair"])
+@pytest.mark.parametrize("policy", [0, 4, 5], ids=["by_shape", "one_cta", "cta_pair"])
 @pytest.mark.parametrize("mode", list(MODES))
 @pytest.mark.parametrize("case", QUANT_CASES, ids=[c[0] for c in QUANT_CASES])
 def test_quantised_layer_against_the_simulation(case, mode, policy):
     from sparse_moe_layer_05_b200 import binding as B
     elem = MODES[mode]
     name, d, I, E, k, T, seed = case
-    if policy == 5 and T * k < 64 * E:
+    if policy != 0 and T * k < 64 * E:
         pytest.skip("few rows per expert: the 16-token tiles run either way")
     inp = W.make_custom(d, I, E, k, T, seed=seed)
     layer = B.MoELayer(inp)
@@ -140,9 +140,11 @@ def test_quantised_layer_against_the_simulation(case, mode, policy):
     ws = layer.workspace.cpu().numpy()
     qb = 1 if elem == "e4m3" else 2                   # elements per byte
 
-    # w4a4 on the CTA pair runs kind::mxf4 (d, I >= 256), whose scale blocks
-    # are laid out per 256-wide k-block
-    f4 = mode == "mxfp4" and policy == 5 and P >= 64 * E and min(d, I) >= 256
+    # the CTA-pair tiles run where forced (policy 5) and, picked by shape, from
+    # 192 rows per expert; w4a4 on them runs kind::mxf4 (d, I >= 256), whose
+    # scale blocks are laid out per 256-wide k-block
+    pair = P >= 64 * E and (policy == 5 or (policy == 0 and P >= 192 * E))
+    f4 = mode == "mxfp4" and pair and min(d, I) >= 256
 
     def rows_of(region, scales, K):
         q = ws[L[region]:L[region] + (int(pr.max()) + 1) * K // qb].reshape(-1, K // qb)[pr]

@@ -609,10 +609,11 @@ def _output_tokens(T, k, offsets, perm, seed):
 
 @pytest.mark.parametrize("name,T", FULL_CASES, ids=[f"{n}-T{t}" for n, t in FULL_CASES])
 def test_full_size_every_token_routed_and_sampled_outputs(name, T):
-    """At the full batch of every configuration: top-k indices, weights, counts,
-    offsets and the permutation against the oracle on every token (near-ties,
-    whose k-th and (k+1)-th oracle logits lie within 1e-5, are counted and
-    printed; their choice must still be valid); outputs of at least 256 tokens,
+    """At the full batch of every configuration: the router's fp32 logits within
+    their error bound on every token; top-k indices, weights, counts, offsets
+    and the permutation against the oracle on every token (exact ties below
+    NEAR_TIE are counted and printed; their choice must still be valid);
+    outputs of at least 256 tokens,
     among them every expert's first and last routed token, against the oracle,
     both as the bf16 output (tolerance plus the output's own rounding) and,
     strictly, as the fp32 sum before that rounding."""
@@ -627,6 +628,8 @@ def test_full_size_every_token_routed_and_sampled_outputs(name, T):
     offsets = layer.intermediate("offsets", T).cpu().numpy()
     perm = layer.intermediate("perm", T).cpu().numpy()
     r = O.route(inp.x, inp.W_r, inp.b_r, inp.k)
+    G.check_router_logits(layer.intermediate("logits", T).cpu().numpy(), r, inp.x, inp.W_r,
+                          what=f"{name} T={T}")
     copies = 32 if name == "64a8" else None
     ties = G.compare_routing(idx, w, r, copies_of=copies, max_exempt=max(2, T // 1000))
     same = G.check_tables_against_oracle(idx, counts, offsets, perm, r, inp.E)
