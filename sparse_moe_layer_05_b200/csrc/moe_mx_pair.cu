@@ -191,11 +191,6 @@ struct PairArgs {
   const float* topk_w;
   int* status;
   const float* bias;          // [E][2I] or [E][d], or nullptr
-  // for the L2 prefetch of the next tile's operands
-  const uint8_t* a_rows;      // token rows (hi plane; the lo plane a_plane bytes later)
-  size_t a_plane;             // bytes of one token-row plane (0: one plane)
-  int a_row_bytes;            // bytes of one token row
-  const uint8_t* codes;       // weight codes [E][rows_per_expert][K/2]
 };
 
 __device__ __forceinline__ float silu_p(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
@@ -338,31 +333,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
       int s = 0, ph = 0, it = 0;
       bool ok = pair_id >= total || load_tile_scales(pair_id, 0);
       const int kb_next = min(3, KB - 1);
-      // L2 prefetch of a tile's operands for this CTA: its weight rows and
-      // (when it has any) its 128 token rows, so that the stage loads of the
-      // next tile hit L2 instead of waiting on HBM
-      auto prefetch_tile = [&](int tile) {
-        Tile t;
-        decode(tile, t);
-        const int wr = EPI == PAIR_SWIGLU ? rank * args.I + t.nt * C::NH
-                                          : t.nt * C::N + rank * C::NH;
-        const int nrows = min(C::NH, args.rows_per_expert - wr);
-        if (nrows > 0)
-          prefetch_l2_bulk(args.codes + (static_cast<size_t>(t.e) * args.rows_per_expert + wr) *
-                                            (K / 2),
-                           static_cast<uint32_t>(nrows) * (K / 2));
-        if (t.rows > 0) {
-          const uint32_t bytes = static_cast<uint32_t>(t.rows) * args.a_row_bytes;
-          const uint8_t* a = args.a_rows + static_cast<size_t>(t.arow) * args.a_row_bytes;
-          prefetch_l2_bulk(a, (bytes + 15) & ~15u);
-          if (args.a_plane) prefetch_l2_bulk(a + args.a_plane, (bytes + 15) & ~15u);
-        }
-      };
       for (int tile = pair_id; tile < total && ok; tile += npairs, ++it) {
         Tile t;
         decode(tile, t);
         const bool has_a = t.rows > 0;
-        if (tile + npairs < total) prefetch_tile(tile + npairs);
         // weight rows of this CTA's B half
         const int wrow = EPI == PAIR_SWIGLU ? rank * args.I + t.nt * C::NH
                                             : t.nt * C::N + rank * C::NH;
@@ -797,10 +771,6 @@ cudaError_t launch_pair_impl(const MxGemmProblem& p, int num_sms, cudaStream_t s
   a.topk_w = p.topk_w;
   a.status = p.status;
   a.bias = p.bias;
-  a.a_rows = p.b_hi;
-  a.a_row_bytes = ACT == ACT_E2M1 || ACT == ACT_F4 ? p.K / 2 : p.K;
-  a.a_plane = ACT == ACT_HILO ? static_cast<size_t>(p.tok_rows) * p.K : 0;
-  a.codes = p.codes;
   const int64_t tiles_bound = (static_cast<int64_t>(p.P) / 256 + p.E) * a.n_tiles;
   int64_t pairs = num_sms / 2;
   if (tiles_bound < pairs) pairs = tiles_bound;

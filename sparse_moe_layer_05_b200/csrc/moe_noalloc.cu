@@ -27,11 +27,12 @@
 namespace {
 
 // Largest T * E accepted: the fp32 router logits take 4 bytes per
-// (token, expert). The router's split weights (three bf16 terms per weight
-// and one norm per expert row) take at most 3 * 256 * 16384 * 2 + 1024
-// bytes; the rest of the scratch is small tables.
+// (token, expert). The router's split weights (three bf16 terms per weight,
+// a norm and a fingerprint per expert row) take at most
+// 3 * 256 * 16384 * 2 + 256 * 12 bytes; the rest of the scratch is small
+// tables.
 constexpr size_t kNoAllocMaxTE = size_t(1) << 20;
-constexpr size_t kNoAllocRouterBytes = size_t(3) * 256 * 16384 * 2 + 1024;
+constexpr size_t kNoAllocRouterBytes = size_t(3) * 256 * 16384 * 2 + 4096;
 constexpr size_t kNoAllocScratchBytes =
     kNoAllocMaxTE * 4 + kNoAllocRouterBytes + (size_t(64) << 10);
 

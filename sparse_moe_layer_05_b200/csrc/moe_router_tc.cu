@@ -72,6 +72,8 @@ constexpr float kRefineRel = 7.62939453125e-06f;
 
 struct RouterTcShape {
   int npad;          // E rounded up to 16
+  int nacc;          // TMEM accumulators: 3 (hi, mid, lo) or 2 (hi, mid + lo)
+  int per;           // weight terms per UMMA (their B rows and accumulators are adjacent)
   int stage_bytes;   // x tile + three weight-term tiles
   int stages;
   int ld;            // floats per partial-logits row in shared memory
@@ -91,20 +93,27 @@ RouterTcShape router_tc_shape(int E) {
   s.stages = st;
   s.body = st * s.stage_bytes;
   if (s.body < partial_bytes) s.body = (partial_bytes + 1023) / 1024 * 1024;
+  s.nacc = 3 * s.npad <= 512 ? 3 : 2;
+  s.per = s.nacc == 3 ? (256 / s.npad < 3 ? 256 / s.npad : 3) : 1;
   int cols = 32;
-  while (cols < 2 * s.npad) cols *= 2;
+  while (cols < s.nacc * s.npad) cols *= 2;
   s.tmem_cols = cols;
   s.smem_alloc = s.body + RT_FIXED + 1024;
   return s;
 }
 
-// W_r [E][d] fp32 -> terms [3][npad][d] bf16 (rows E..npad-1 zero) and
+// W_r [E][d] fp32 -> terms [3][npad][d] bf16 (rows E..npad-1 zero),
 // norms[npad] = ||W_r[e]||_2 (fp32, in one fixed order; 0 for the padding
-// rows). One block per row.
-__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ W_r, int E,
+// rows) and fps[npad], a 64-bit fingerprint of each row and its bias (sum of
+// bits(w_i) (2i + 1) plus bits(b) times an odd constant, mod 2^64): rows with
+// equal weights and bias (the copies of a silent-init layer) get equal
+// fingerprints. One block per row.
+__global__ void __launch_bounds__(256) router_split_kernel(const float* __restrict__ W_r,
+                                                           const float* __restrict__ b_r, int E,
                                                            int npad, int d,
                                                            uint16_t* __restrict__ terms,
                                                            float* __restrict__ norms,
+                                                           unsigned long long* __restrict__ fps,
                                                            int* status) {
   pdl_wait_and_trigger();
   // the first kernel of the pass clears the status word
@@ -113,6 +122,7 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
   const size_t n = static_cast<size_t>(npad) * d;
   const size_t base = static_cast<size_t>(row) * d;
   float ss = 0.f;
+  unsigned long long fp = 0ull;
   for (int i = threadIdx.x * 4; i < d; i += 256 * 4) {
     float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
     if (row < E) w = __ldg(reinterpret_cast<const float4*>(W_r + base + i));
@@ -128,6 +138,8 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
       m[j] = __bfloat16_as_ushort(mid);
       l[j] = __bfloat16_as_ushort(lo);
       ss = fmaf(wv[j], wv[j], ss);
+      fp += static_cast<unsigned long long>(__float_as_uint(wv[j])) *
+            static_cast<unsigned long long>(2 * (i + j) + 1);
     }
     *reinterpret_cast<uint2*>(terms + base + i) =
         make_uint2(h[0] | (uint32_t(h[1]) << 16), h[2] | (uint32_t(h[3]) << 16));
@@ -137,15 +149,29 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
         make_uint2(l[0] | (uint32_t(l[1]) << 16), l[2] | (uint32_t(l[3]) << 16));
   }
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, off);
+  for (int off = 16; off > 0; off >>= 1) {
+    ss += __shfl_xor_sync(0xFFFFFFFFu, ss, off);
+    fp += __shfl_xor_sync(0xFFFFFFFFu, fp, off);
+  }
   __shared__ float red[8];
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __shared__ unsigned long long redf[8];
+  if ((threadIdx.x & 31) == 0) {
+    red[threadIdx.x >> 5] = ss;
+    redf[threadIdx.x >> 5] = fp;
+  }
   __syncthreads();
   if (threadIdx.x == 0) {
     float s = 0.f;
+    unsigned long long f = row < E ? static_cast<unsigned long long>(__float_as_uint(b_r[row])) *
+                                         0x9E3779B97F4A7C15ull
+                                   : 0ull;
 #pragma unroll
-    for (int w = 0; w < 8; ++w) s += red[w];
+    for (int w = 0; w < 8; ++w) {
+      s += red[w];
+      f += redf[w];
+    }
     norms[row] = sqrtf(s);
+    fps[row] = f;
   }
 }
 
@@ -154,7 +180,8 @@ struct RouterTcArgs {
   const float* W_r;
   const float* b_r;
   const float* norms;
-  int T, E, k, d, npad, stages, ld, stage_bytes, body, tmem_cols, KB;
+  const unsigned long long* fps;
+  int T, E, k, d, npad, nacc, per, stages, ld, stage_bytes, body, tmem_cols, KB;
   float* logits;
   int32_t* topk_idx;
   float* topk_w;
@@ -172,6 +199,15 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity) {
 __device__ __forceinline__ float ld_shared_cluster_f32(uint32_t addr) {
   float v;
   asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ float4 ld_shared_cluster_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
   return v;
 }
 
@@ -224,7 +260,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = misc[0];
-  const uint32_t tmem_lo = tmem_base + static_cast<uint32_t>(args.npad);
+  const uint32_t npad_u = static_cast<uint32_t>(args.npad);
   bool ok = true;
 
   if (warp == 0) {
@@ -245,8 +281,12 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(RT_M, args.npad);
-      const uint32_t term_bytes = static_cast<uint32_t>(args.npad) * 128;
+      // three accumulators: terms t .. t + per - 1 in one UMMA (their B rows
+      // and accumulator columns are adjacent); two: hi, then mid and lo into
+      // the second
+      const uint32_t idesc1 = idesc_bf16_f32(RT_M, args.npad);
+      const uint32_t idescp = idesc_bf16_f32(RT_M, args.per * args.npad);
+      const uint32_t term_bytes = npad_u * 128;
       int s = 0, ph = 0, consumed = 0;
       for (int i = 0; i < nkb; ++i) {
         if (!(ok = mbar_wait(bar_full(s), ph, abort_flag, args.status))) break;
@@ -258,9 +298,20 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         for (int kk = 0; kk < RT_BK / 16; ++kk) {
           const uint32_t acc = (i | kk) != 0 ? 1u : 0u;
           const uint64_t ad = sdesc_k_sw128(st + kk * 32);
-          umma_bf16(tmem_base, ad, sdesc_k_sw128(wb + kk * 32), idesc, acc);
-          umma_bf16(tmem_lo, ad, sdesc_k_sw128(wb + term_bytes + kk * 32), idesc, acc);
-          umma_bf16(tmem_lo, ad, sdesc_k_sw128(wb + 2 * term_bytes + kk * 32), idesc, 1u);
+          if (args.nacc == 3) {
+            for (int t = 0; t < 3; t += args.per) {
+              const bool whole = t + args.per <= 3;
+              umma_bf16(tmem_base + static_cast<uint32_t>(t) * npad_u, ad,
+                        sdesc_k_sw128(wb + t * term_bytes + kk * 32), whole ? idescp : idesc1, acc);
+              if (!whole) break;
+            }
+          } else {
+            umma_bf16(tmem_base, ad, sdesc_k_sw128(wb + kk * 32), idesc1, acc);
+            umma_bf16(tmem_base + npad_u, ad, sdesc_k_sw128(wb + term_bytes + kk * 32), idesc1,
+                      acc);
+            umma_bf16(tmem_base + npad_u, ad, sdesc_k_sw128(wb + 2 * term_bytes + kk * 32),
+                      idesc1, 1u);
+          }
         }
         umma_commit(bar_empty(s));
         if (++s == S) { s = 0; ph ^= 1; }
@@ -305,10 +356,17 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     float* prow = partial + static_cast<size_t>(r) * args.ld;
     if (ok && nkb > 0) {
       const uint32_t lanes = static_cast<uint32_t>(quad * 32) << 16;
+      // partial logit = hi + (mid + lo), or hi + (mid and lo accumulated together)
       for (int c = 0; c < args.npad; c += 16) {
-        uint32_t a[16], b[16];
+        uint32_t a[16], b[16], l[16];
         tmem_ld16_sync(tmem_base + lanes + c, a);
-        tmem_ld16_sync(tmem_lo + lanes + c, b);
+        tmem_ld16_sync(tmem_base + npad_u + lanes + c, b);
+        if (args.nacc == 3) {
+          tmem_ld16_sync(tmem_base + 2 * npad_u + lanes + c, l);
+#pragma unroll
+          for (int i = 0; i < 16; ++i)
+            b[i] = __float_as_uint(__uint_as_float(b[i]) + __uint_as_float(l[i]));
+        }
 #pragma unroll
         for (int i = 0; i < 16; i += 4) {
           float4 o;
@@ -362,17 +420,40 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     for (int rr = rbeg + warp; rr < rbeg + rpc; rr += RT_THREADS / 32) {
       const int t = t0 + rr;
       if (t >= args.T) break;
+      // lane l holds experts 128 h + 4 l + i (slot 4 h + i); the C partials
+      // of four experts come in one 16-byte load per CTA, all issued before
+      // the adds (rank order)
       float v[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int e = lane + 32 * j;
-        v[j] = -FLT_MAX;
-        if (e < E) {
-          const uint32_t a = pbase + static_cast<uint32_t>((rr * args.ld + e) * 4);
-          float s = 0.f;
-          for (uint32_t q = 0; q < csize; ++q) s += ld_shared_cluster_f32(mapa_shared(a, q));
-          v[j] = s + __ldg(args.b_r + e);
-          args.logits[static_cast<size_t>(t) * E + e] = v[j];
+      for (int h = 0; h < 2; ++h) {
+        const int e0 = 128 * h + 4 * lane;
+        float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (e0 < args.npad) {
+          const uint32_t a = pbase + static_cast<uint32_t>((rr * args.ld + e0) * 4);
+          float4 part[RT_MAX_CLUSTER];
+#pragma unroll
+          for (int q = 0; q < RT_MAX_CLUSTER; ++q)
+            if (q < static_cast<int>(csize))
+              part[q] = ld_shared_cluster_f32x4(mapa_shared(a, static_cast<uint32_t>(q)));
+#pragma unroll
+          for (int q = 0; q < RT_MAX_CLUSTER; ++q) {
+            if (q < static_cast<int>(csize)) {
+              acc4.x += part[q].x;
+              acc4.y += part[q].y;
+              acc4.z += part[q].z;
+              acc4.w += part[q].w;
+            }
+          }
+        }
+        const float av[4] = {acc4.x, acc4.y, acc4.z, acc4.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int e = e0 + i;
+          v[4 * h + i] = -FLT_MAX;
+          if (e < E) {
+            v[4 * h + i] = av[i] + __ldg(args.b_r + e);
+            args.logits[static_cast<size_t>(t) * E + e] = v[4 * h + i];
+          }
         }
       }
       float xsq = 0.f;
@@ -381,7 +462,7 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
       float tau = kRefineRel * sqrtf(xsq) * wmax;
       if (!(tau <= FLT_MAX)) tau = 0.f;
       topk_refine_softmax_warp(v, E, args.k, tau, args.x + static_cast<size_t>(t) * args.d,
-                               args.W_r, args.b_r, args.d, lane,
+                               args.W_r, args.b_r, args.fps, args.d, lane,
                                args.topk_idx + static_cast<size_t>(t) * args.k,
                                args.topk_w + static_cast<size_t>(t) * args.k);
     }
@@ -447,7 +528,7 @@ int cluster_size(int T, int d, int dev, size_t smem) {
 
 size_t router_tc_scratch_bytes(int E, int d) {
   const size_t npad = static_cast<size_t>((E + 15) / 16 * 16);
-  return 3 * npad * static_cast<size_t>(d) * 2 + npad * 4;
+  return 3 * npad * static_cast<size_t>(d) * 2 + npad * 4 + npad * 8;
 }
 
 cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b_r, int T, int E,
@@ -472,10 +553,11 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b
   uint16_t* terms = static_cast<uint16_t*>(scratch);
   float* norms = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) +
                                           3 * static_cast<size_t>(sh.npad) * d * 2);
+  unsigned long long* fps = reinterpret_cast<unsigned long long*>(norms + sh.npad);
   // the weight split: the first launch of the pass (it clears the status word)
   {
-    cudaError_t e = launch_kernel(router_split_kernel, dim3(sh.npad), dim3(256), 0, st, W_r, E,
-                                  sh.npad, d, terms, norms, status);
+    cudaError_t e = launch_kernel(router_split_kernel, dim3(sh.npad), dim3(256), 0, st, W_r, b_r,
+                                  E, sh.npad, d, terms, norms, fps, status);
     if (e != cudaSuccess) return e;
     pdl_launches() = true;   // the router kernel may overlap the split's tail
   }
@@ -499,11 +581,14 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b
   a.W_r = W_r;
   a.b_r = b_r;
   a.norms = norms;
+  a.fps = fps;
   a.T = T;
   a.E = E;
   a.k = k;
   a.d = d;
   a.npad = sh.npad;
+  a.nacc = sh.nacc;
+  a.per = sh.per;
   a.stages = sh.stages;
   a.ld = sh.ld;
   a.stage_bytes = sh.stage_bytes;

@@ -30,9 +30,15 @@ __device__ __forceinline__ uint64_t value_order_key(double f) {
   return (u & 0x8000000000000000ull) ? ~u : (u | 0x8000000000000000ull);
 }
 
-// One warp per token: the top-k of the token's logits v (lane l holds experts
-// l, l+32, ..., -FLT_MAX past E), the order of near ties settled in fp64, and
-// the softmax over the k selected.
+// Expert held in slot j of lane l: four consecutive experts per lane in each
+// half of 128 (so that a lane reads its logits with 16-byte loads).
+__device__ __forceinline__ int slot_expert(int lane, int j) {
+  return 128 * (j >> 2) + 4 * lane + (j & 3);
+}
+
+// One warp per token: the top-k of the token's logits v (slot j of lane l
+// holds expert slot_expert(l, j), -FLT_MAX past E), the order of near ties
+// settled in fp64, and the softmax over the k selected.
 //
 // 1. Rounds of a warp arg-max on (logit descending, index ascending) list the
 //    k largest logits, then go on while the next one lies within tau of the
@@ -43,7 +49,10 @@ __device__ __forceinline__ uint64_t value_order_key(double f) {
 //    row with the fp32 router row (every product exact in fp64), plus the
 //    bias. Entries of one chain of near gaps are all refined; entries whose
 //    gaps are all above tau keep their fp32 value, which lies within tau/2 of
-//    the exact one on either side, so no refined entry can pass them.
+//    the exact one on either side, so no refined entry can pass them. A gap
+//    of exactly zero between rows with equal fingerprints (fps: equal router
+//    rows and biases, e.g. copied experts) is not near: such logits are equal
+//    on every evaluation and already ordered by index.
 // 3. With any entry refined, k rounds of the arg-max over the list (fp64
 //    values) give the final order; otherwise the list's first k entries are
 //    the result.
@@ -52,7 +61,9 @@ __device__ __forceinline__ void topk_refine_softmax_warp(const float (&v)[8], in
                                                          float tau,
                                                          const uint16_t* __restrict__ x_row,
                                                          const float* __restrict__ W_r,
-                                                         const float* __restrict__ b_r, int d,
+                                                         const float* __restrict__ b_r,
+                                                         const unsigned long long* __restrict__ fps,
+                                                         int d,
                                                          int lane, int32_t* __restrict__ idx_out,
                                                          float* __restrict__ w_out) {
   const unsigned full = 0xFFFFFFFFu;
@@ -60,7 +71,7 @@ __device__ __forceinline__ void topk_refine_softmax_warp(const float (&v)[8], in
   uint32_t taken = 0;
 #pragma unroll
   for (int j = 0; j < 8; ++j) {
-    const int e = lane + 32 * j;
+    const int e = slot_expert(lane, j);
     key[j] = logit_order_key(v[j]);
     if (e >= E) taken |= 1u << j;
   }
@@ -77,7 +88,7 @@ __device__ __forceinline__ void topk_refine_softmax_warp(const float (&v)[8], in
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
       if (taken & (1u << j)) continue;
-      const int e = lane + 32 * j;
+      const int e = slot_expert(lane, j);
       if (bi == 0x7FFFFFFF || key[j] > bk || (key[j] == bk && e < bi)) {
         bk = key[j];
         bv = v[j];
@@ -99,7 +110,7 @@ __device__ __forceinline__ void topk_refine_softmax_warp(const float (&v)[8], in
     }
     // past the k-th: only runners-up within tau of it
     if (r >= k && !(refine && kth - bv <= tau)) break;
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (((bi & 127) >> 2) == lane) taken |= 1u << (((bi >> 7) << 2) | (bi & 3));
     if (r == k - 1) kth = bv;
     if ((r & 31) == lane) {
       cidx[r >> 5] = bi;
@@ -108,13 +119,22 @@ __device__ __forceinline__ void topk_refine_softmax_warp(const float (&v)[8], in
     m = r + 1;
   }
 
-  // near gaps: near_p = (p + 1 < m) && cval_p - cval_{p+1} <= tau
+  // near gaps: near_p = (p + 1 < m) && cval_p - cval_{p+1} <= tau, unless the
+  // two are copies (equal value and fingerprint)
   float nx0 = __shfl_down_sync(full, cval[0], 1);
   const float head1 = __shfl_sync(full, cval[1], 0);
   if (lane == 31) nx0 = head1;
   const float nx1 = __shfl_down_sync(full, cval[1], 1);
-  const bool near0 = refine && lane + 1 < m && cval[0] - nx0 <= tau;
-  const bool near1 = refine && 33 + lane < m && cval[1] - nx1 <= tau;
+  const unsigned long long f0 = (refine && lane < m) ? __ldg(fps + cidx[0]) : 0ull;
+  const unsigned long long f1 = (refine && 32 + lane < m) ? __ldg(fps + cidx[1]) : 1ull;
+  unsigned long long nf0 = __shfl_down_sync(full, f0, 1);
+  const unsigned long long fhead1 = __shfl_sync(full, f1, 0);
+  if (lane == 31) nf0 = fhead1;
+  const unsigned long long nf1 = __shfl_down_sync(full, f1, 1);
+  const bool copy0 = cval[0] == nx0 && f0 == nf0;
+  const bool copy1 = cval[1] == nx1 && f1 == nf1;
+  const bool near0 = refine && lane + 1 < m && cval[0] - nx0 <= tau && !copy0;
+  const bool near1 = refine && 33 + lane < m && cval[1] - nx1 <= tau && !copy1;
   bool pv0 = __shfl_up_sync(full, near0, 1);
   bool pv1 = __shfl_up_sync(full, near1, 1);
   const bool tail0 = __shfl_sync(full, near0, 31);
@@ -153,7 +173,7 @@ __device__ __forceinline__ void topk_refine_softmax_warp(const float (&v)[8], in
         }
       }
       double acc[4] = {0.0, 0.0, 0.0, 0.0};
-#pragma unroll 2
+#pragma unroll 4
       for (int i = 4 * lane; i < d128; i += 128) {
         const uint2 xb = __ldg(reinterpret_cast<const uint2*>(x_row + i));
         const double x0 = __uint_as_float(xb.x << 16), x1 = __uint_as_float(xb.x & 0xFFFF0000u);
