@@ -46,8 +46,9 @@
 // and one warp per token selects its k experts.
 //
 // Roles (256 threads): warp 0 TMA producer, warp 1 TMEM allocation and UMMA
-// issue, warps 4-7 row norms, then TMEM -> shared memory; all eight warps run
-// the top-k. Every wait is bounded (moe_ptx.cuh); every CTA reaches both
+// issue, warps 4-7 row norms, then TMEM -> shared memory; after the cluster
+// barrier all threads sum the partials of this CTA's rows (in place) and all
+// eight warps run the top-k. Every wait is bounded (moe_ptx.cuh); every CTA reaches both
 // cluster barriers on every path.
 #include <cuda_bf16.h>
 #include <float.h>
@@ -400,10 +401,55 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     tmem_dealloc(tmem_base, static_cast<uint32_t>(args.tmem_cols));
   }
 
-  // rows [rank 128 / C, (rank+1) 128 / C): sum of the partials in rank order,
-  // bias, logits out, top-k with near-tie refinement and softmax
+  // rows [rank 128 / C, (rank+1) 128 / C) are finished by this CTA; no other
+  // CTA reads them from this CTA's buffer, so their sums go back in place
   if (!*abort_flag) {
     const int E = args.E;
+    const int rpc = RT_M / static_cast<int>(csize);
+    const int rbeg = static_cast<int>(rank) * rpc;
+    const uint32_t pbase = smem_u32(partial);
+    const uint32_t xbase = smem_u32(xsq_part);
+    // 1. logits = the C partials in rank order + bias (four experts per item,
+    //    every CTA's 16 bytes loaded before the adds), written out; ||x_t||^2
+    const int nch = args.npad / 4;
+    for (int it = threadIdx.x; it < rpc * nch; it += RT_THREADS) {
+      const int rr = rbeg + it / nch;
+      const int e0 = (it % nch) * 4;
+      const uint32_t a = pbase + static_cast<uint32_t>((rr * args.ld + e0) * 4);
+      float4 part[RT_MAX_CLUSTER];
+#pragma unroll
+      for (int q = 0; q < RT_MAX_CLUSTER; ++q)
+        if (q < static_cast<int>(csize))
+          part[q] = ld_shared_cluster_f32x4(mapa_shared(a, static_cast<uint32_t>(q)));
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int q = 0; q < RT_MAX_CLUSTER; ++q) {
+        if (q < static_cast<int>(csize)) {
+          acc[0] += part[q].x;
+          acc[1] += part[q].y;
+          acc[2] += part[q].z;
+          acc[3] += part[q].w;
+        }
+      }
+      const int t = t0 + rr;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (e0 + i < E) {
+          acc[i] += __ldg(args.b_r + e0 + i);
+          if (t < args.T) args.logits[static_cast<size_t>(t) * E + e0 + i] = acc[i];
+        }
+      }
+      *reinterpret_cast<float4*>(partial + rr * args.ld + e0) =
+          make_float4(acc[0], acc[1], acc[2], acc[3]);
+    }
+    for (int rr = rbeg + static_cast<int>(threadIdx.x); rr < rbeg + rpc; rr += RT_THREADS) {
+      float xsq = 0.f;
+      for (uint32_t q = 0; q < csize; ++q)
+        xsq += ld_shared_cluster_f32(mapa_shared(xbase + static_cast<uint32_t>(rr * 4), q));
+      xsq_part[rr] = xsq;
+    }
+    __syncthreads();
+    // 2. one warp per token: top-k with near-tie refinement, softmax
     float wmax = 0.f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -413,53 +459,22 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1)
       wmax = fmaxf(wmax, __shfl_xor_sync(0xFFFFFFFFu, wmax, off));
-    const int rpc = RT_M / static_cast<int>(csize);
-    const int rbeg = static_cast<int>(rank) * rpc;
-    const uint32_t pbase = smem_u32(partial);
-    const uint32_t xbase = smem_u32(xsq_part);
     for (int rr = rbeg + warp; rr < rbeg + rpc; rr += RT_THREADS / 32) {
       const int t = t0 + rr;
       if (t >= args.T) break;
-      // lane l holds experts 128 h + 4 l + i (slot 4 h + i); the C partials
-      // of four experts come in one 16-byte load per CTA, all issued before
-      // the adds (rank order)
+      // lane l holds experts 128 h + 4 l + i (slot 4 h + i)
       float v[8];
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int e0 = 128 * h + 4 * lane;
-        float4 acc4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (e0 < args.npad) {
-          const uint32_t a = pbase + static_cast<uint32_t>((rr * args.ld + e0) * 4);
-          float4 part[RT_MAX_CLUSTER];
-#pragma unroll
-          for (int q = 0; q < RT_MAX_CLUSTER; ++q)
-            if (q < static_cast<int>(csize))
-              part[q] = ld_shared_cluster_f32x4(mapa_shared(a, static_cast<uint32_t>(q)));
-#pragma unroll
-          for (int q = 0; q < RT_MAX_CLUSTER; ++q) {
-            if (q < static_cast<int>(csize)) {
-              acc4.x += part[q].x;
-              acc4.y += part[q].y;
-              acc4.z += part[q].z;
-              acc4.w += part[q].w;
-            }
-          }
-        }
-        const float av[4] = {acc4.x, acc4.y, acc4.z, acc4.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int e = e0 + i;
-          v[4 * h + i] = -FLT_MAX;
-          if (e < E) {
-            v[4 * h + i] = av[i] + __ldg(args.b_r + e);
-            args.logits[static_cast<size_t>(t) * E + e] = v[4 * h + i];
-          }
-        }
+        float4 q4 = make_float4(-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX);
+        if (e0 < args.npad) q4 = *reinterpret_cast<const float4*>(partial + rr * args.ld + e0);
+        v[4 * h] = e0 < E ? q4.x : -FLT_MAX;
+        v[4 * h + 1] = e0 + 1 < E ? q4.y : -FLT_MAX;
+        v[4 * h + 2] = e0 + 2 < E ? q4.z : -FLT_MAX;
+        v[4 * h + 3] = e0 + 3 < E ? q4.w : -FLT_MAX;
       }
-      float xsq = 0.f;
-      for (uint32_t q = 0; q < csize; ++q)
-        xsq += ld_shared_cluster_f32(mapa_shared(xbase + static_cast<uint32_t>(rr * 4), q));
-      float tau = kRefineRel * sqrtf(xsq) * wmax;
+      float tau = kRefineRel * sqrtf(xsq_part[rr]) * wmax;
       if (!(tau <= FLT_MAX)) tau = 0.f;
       topk_refine_softmax_warp(v, E, args.k, tau, args.x + static_cast<size_t>(t) * args.d,
                                args.W_r, args.b_r, args.fps, args.d, lane,

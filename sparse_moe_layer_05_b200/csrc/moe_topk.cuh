@@ -49,10 +49,12 @@ __device__ __forceinline__ int slot_expert(int lane, int j) {
 //    row with the fp32 router row (every product exact in fp64), plus the
 //    bias. Entries of one chain of near gaps are all refined; entries whose
 //    gaps are all above tau keep their fp32 value, which lies within tau/2 of
-//    the exact one on either side, so no refined entry can pass them. A gap
-//    of exactly zero between rows with equal fingerprints (fps: equal router
-//    rows and biases, e.g. copied experts) is not near: such logits are equal
-//    on every evaluation and already ordered by index.
+//    the exact one on either side, so no refined entry can pass them. Rows
+//    with equal fingerprints (fps: equal router rows and biases, e.g. copied
+//    experts) and equal fp32 logits are copies: a gap of zero between copies
+//    needs no refinement (their logits are equal on every evaluation and
+//    already in index order); where one copy is refined, all copies of its
+//    group take the same fp64 value.
 // 3. With any entry refined, k rounds of the arg-max over the list (fp64
 //    values) give the final order; otherwise the list's first k entries are
 //    the result.
@@ -119,41 +121,50 @@ __device__ __forceinline__ void topk_refine_softmax_warp(const float (&v)[8], in
     m = r + 1;
   }
 
-  // near gaps: near_p = (p + 1 < m) && cval_p - cval_{p+1} <= tau, unless the
-  // two are copies (equal value and fingerprint)
+  // Links between list positions p and p + 1 (bit p of 64-bit masks):
+  // close (gap at most tau) and, among those, copies (equal value and equal
+  // fingerprint: the same router row and bias). Fingerprints are read only
+  // when some link is close.
   float nx0 = __shfl_down_sync(full, cval[0], 1);
   const float head1 = __shfl_sync(full, cval[1], 0);
   if (lane == 31) nx0 = head1;
   const float nx1 = __shfl_down_sync(full, cval[1], 1);
-  const unsigned long long f0 = (refine && lane < m) ? __ldg(fps + cidx[0]) : 0ull;
-  const unsigned long long f1 = (refine && 32 + lane < m) ? __ldg(fps + cidx[1]) : 1ull;
-  unsigned long long nf0 = __shfl_down_sync(full, f0, 1);
-  const unsigned long long fhead1 = __shfl_sync(full, f1, 0);
-  if (lane == 31) nf0 = fhead1;
-  const unsigned long long nf1 = __shfl_down_sync(full, f1, 1);
-  const bool copy0 = cval[0] == nx0 && f0 == nf0;
-  const bool copy1 = cval[1] == nx1 && f1 == nf1;
-  const bool near0 = refine && lane + 1 < m && cval[0] - nx0 <= tau && !copy0;
-  const bool near1 = refine && 33 + lane < m && cval[1] - nx1 <= tau && !copy1;
-  bool pv0 = __shfl_up_sync(full, near0, 1);
-  bool pv1 = __shfl_up_sync(full, near1, 1);
-  const bool tail0 = __shfl_sync(full, near0, 31);
-  if (lane == 0) {
-    pv0 = false;
-    pv1 = tail0;
+  const bool close0 = refine && lane + 1 < m && cval[0] - nx0 <= tau;
+  const bool close1 = refine && 33 + lane < m && cval[1] - nx1 <= tau;
+  const uint64_t close_m = static_cast<uint64_t>(__ballot_sync(full, close0)) |
+                           (static_cast<uint64_t>(__ballot_sync(full, close1)) << 32);
+  uint64_t refine_m = 0, copy_m = 0;
+  if (close_m) {
+    const unsigned long long f0 = lane < m ? __ldg(fps + cidx[0]) : 0ull;
+    const unsigned long long f1 = 32 + lane < m ? __ldg(fps + cidx[1]) : 0ull;
+    unsigned long long nf0 = __shfl_down_sync(full, f0, 1);
+    const unsigned long long fhead1 = __shfl_sync(full, f1, 0);
+    if (lane == 31) nf0 = fhead1;
+    const unsigned long long nf1 = __shfl_down_sync(full, f1, 1);
+    copy_m = static_cast<uint64_t>(__ballot_sync(full, close0 && cval[0] == nx0 && f0 == nf0)) |
+             (static_cast<uint64_t>(__ballot_sync(full, close1 && cval[1] == nx1 && f1 == nf1))
+              << 32);
+    // both ends of every close link that is not a copy, then whole groups of
+    // copies around them (a copy gets the value of the first of its group)
+    const uint64_t near_m = close_m & ~copy_m;
+    refine_m = near_m | (near_m << 1);
+    for (;;) {
+      const uint64_t g = refine_m | ((refine_m << 1) & (copy_m << 1)) | ((refine_m >> 1) & copy_m);
+      if (g == refine_m) break;
+      refine_m = g;
+    }
   }
-  const uint32_t ref0 = __ballot_sync(full, lane < m && (near0 || pv0));
-  const uint32_t ref1 = __ballot_sync(full, 32 + lane < m && (near1 || pv1));
 
   int my_idx;
   double my_val, top;
-  if ((ref0 | ref1) == 0) {
+  if (refine_m == 0) {
     my_idx = cidx[0];
     my_val = static_cast<double>(cval[0]);
     top = static_cast<double>(__shfl_sync(full, cval[0], 0));
   } else {
     double val[2] = {static_cast<double>(cval[0]), static_cast<double>(cval[1])};
-    uint64_t pending = static_cast<uint64_t>(ref0) | (static_cast<uint64_t>(ref1) << 32);
+    // computed: the first entry of each refined group of copies
+    uint64_t pending = refine_m & ~(copy_m << 1);
     const int d128 = d & ~127;
     while (pending) {
       // up to four refined entries per pass over the x row
@@ -204,7 +215,13 @@ __device__ __forceinline__ void topk_refine_softmax_warp(const float (&v)[8], in
 #pragma unroll
           for (int off = 16; off > 0; off >>= 1) acc[g] += __shfl_xor_sync(full, acc[g], off);
           const double s = acc[g] + static_cast<double>(__ldg(b_r + ex[g]));
-          if ((pos[g] & 31) == lane) val[pos[g] >> 5] = s;
+          // the entry and the copies that follow it
+          const int len = __ffsll(static_cast<long long>(~(copy_m >> pos[g])));
+#pragma unroll
+          for (int sl = 0; sl < 2; ++sl) {
+            const int q = 32 * sl + lane;
+            if (q >= pos[g] && q < pos[g] + len) val[sl] = s;
+          }
         }
       }
     }
