@@ -120,15 +120,18 @@ def kernel_source_hash(sources=None) -> str:
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str, T: int):
+def recorded_traffic(workload: str, T: int, tile_policy: int = 0, act_quant: str = "bf16"):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
-    summary, if it was taken on the current kernel source; else None."""
+    summary, if it was taken on the current kernel source and in the same
+    configuration (tile policy, activation mode); else None."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
     with open(TRAFFIC_FILE) as f:
         d = json.load(f)
     ent = d.get(f"{workload}:T={T}")
     if not ent or ent.get("source_hash") != kernel_source_hash(ent.get("sources")):
+        return None
+    if ent.get("tile_policy", 0) != tile_policy or ent.get("act_quant", "bf16") != act_quant:
         return None
     return ent.get("bytes_per_launch")
 
@@ -587,7 +590,8 @@ def run_ours(args, inp, name):
         "layer_tflops": layer_flops(inp.d, inp.I, inp.E, inp.k, T) * args.steps * world
         / step_s_max / 1e12,
         "roofline": dict(roof, kernel=DOMINANT_STAGE, achieved=achieved, peak=peak,
-                         frac=achieved / peak, traffic=recorded_traffic(name, T),
+                         frac=achieved / peak,
+                         traffic=recorded_traffic(name, T, args.tile_policy, args.act_quant),
                          avg_launch_ms=dom_ms, touched_experts=touched),
         "stage_ms": stage_avg,
         "routing_load": routing_load,

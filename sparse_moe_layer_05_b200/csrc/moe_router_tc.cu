@@ -71,6 +71,23 @@ constexpr int RT_FIXED = 1024;            // barriers, TMEM address, flags
 // the refinement margin tau_t relative to ||x_t|| max_e ||W_r[e]|| (2^-17)
 constexpr float kRefineRel = 7.62939453125e-06f;
 
+// Refinements are queued per warp in shared memory (above the partial
+// logits) and computed by the whole block together: each fp64 dot product is
+// split over all 256 threads, so a refinement costs one pass of loads
+// instead of a warp's chain of them. A warp whose queue is full refines
+// alone.
+constexpr int RQ_PER_WARP = 4;            // queued token lists per warp
+constexpr int RJ_PER_WARP = 64;           // queued dot products per warp
+struct RefineReq {
+  int row, m, pad0, pad1;
+  unsigned long long refine_m, copy_m;
+  double val[64];
+  int cidx[64];
+};
+constexpr int RT_WARPS = 8;
+constexpr int kQueueBytes = 64 + RT_WARPS * RQ_PER_WARP * static_cast<int>(sizeof(RefineReq)) +
+                            RT_WARPS * RJ_PER_WARP * 4 + 4 * RT_WARPS * 8;
+
 struct RouterTcShape {
   int npad;          // E rounded up to 16
   int nacc;          // TMEM accumulators: 3 (hi, mid, lo) or 2 (hi, mid + lo)
@@ -88,7 +105,7 @@ RouterTcShape router_tc_shape(int E) {
   s.npad = (E + 15) / 16 * 16;
   s.stage_bytes = RT_M * 128 + 3 * s.npad * 128;
   s.ld = s.npad + 4;
-  const int partial_bytes = RT_M * s.ld * 4 + RT_M * 4;
+  const int partial_bytes = RT_M * s.ld * 4 + RT_M * 4 + kQueueBytes + 16;
   int st = (RT_SMEM_LIMIT - RT_FIXED - 1024) / s.stage_bytes;
   if (st > RT_MAX_STAGES) st = RT_MAX_STAGES;
   s.stages = st;
@@ -347,12 +364,18 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
           }
         }
       }
+      // these generic-proxy reads must be ordered before the next TMA write
+      // into the stage (async proxy)
+      fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar_empty(s));
       if (++s == S) { s = 0; ph ^= 1; }
     }
     if (ok && nkb > 0) ok = mbar_wait(bar_acc, 0, abort_flag, args.status);
     ok = __all_sync(0xFFFFFFFFu, ok);
+    // the partial rows below overwrite the stages: no warp of the four may
+    // still be reading the last x tile for its norms
+    asm volatile("bar.sync 1, 128;" ::: "memory");
     tc_fence_after();
     float* prow = partial + static_cast<size_t>(r) * args.ld;
     if (ok && nkb > 0) {
@@ -459,6 +482,15 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1)
       wmax = fmaxf(wmax, __shfl_xor_sync(0xFFFFFFFFu, wmax, off));
+    // the queue (above the partial logits and row norms)
+    uint8_t* qb = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(xsq_part + RT_M) + 15) & ~static_cast<uintptr_t>(15));
+    int* q_nreq = reinterpret_cast<int*>(qb);                 // [8]
+    int* q_njob = q_nreq + RT_WARPS;                          // [8]
+    RefineReq* reqs = reinterpret_cast<RefineReq*>(qb + 64);  // [8][RQ_PER_WARP]
+    uint32_t* jobs = reinterpret_cast<uint32_t*>(reqs + RT_WARPS * RQ_PER_WARP);  // [8][RJ]
+    double* red = reinterpret_cast<double*>(jobs + RT_WARPS * RJ_PER_WARP);     // [4][8]
+    int nreq = 0, njob = 0;
     for (int rr = rbeg + warp; rr < rbeg + rpc; rr += RT_THREADS / 32) {
       const int t = t0 + rr;
       if (t >= args.T) break;
@@ -476,10 +508,121 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
       }
       float tau = kRefineRel * sqrtf(xsq_part[rr]) * wmax;
       if (!(tau <= FLT_MAX)) tau = 0.f;
-      topk_refine_softmax_warp(v, E, args.k, tau, args.x + static_cast<size_t>(t) * args.d,
-                               args.W_r, args.b_r, args.fps, args.d, lane,
-                               args.topk_idx + static_cast<size_t>(t) * args.k,
-                               args.topk_w + static_cast<size_t>(t) * args.k);
+      TopkList L;
+      topk_list(v, E, args.k, tau, args.fps, lane, L);
+      int32_t* idx_out = args.topk_idx + static_cast<size_t>(t) * args.k;
+      float* w_out = args.topk_w + static_cast<size_t>(t) * args.k;
+      double val[2] = {static_cast<double>(L.cval[0]), static_cast<double>(L.cval[1])};
+      if (L.refine_m == 0) {
+        topk_emit(L, val, args.k, lane, idx_out, w_out);
+        continue;
+      }
+      const uint64_t starts = topk_refine_starts(L);
+      const int nj = __popcll(starts);
+      if (nreq < RQ_PER_WARP && njob + nj <= RJ_PER_WARP) {
+        RefineReq& R = reqs[warp * RQ_PER_WARP + nreq];
+        if (lane == 0) {
+          R.row = rr;
+          R.m = L.m;
+          R.refine_m = L.refine_m;
+          R.copy_m = L.copy_m;
+        }
+        R.cidx[lane] = L.cidx[0];
+        R.cidx[32 + lane] = L.cidx[1];
+        R.val[lane] = val[0];
+        R.val[32 + lane] = val[1];
+#pragma unroll
+        for (int sl = 0; sl < 2; ++sl) {
+          const int q = 32 * sl + lane;
+          if ((starts >> q) & 1ull) {
+            const int j = njob + __popcll(starts & ((1ull << q) - 1ull));
+            jobs[warp * RJ_PER_WARP + j] = (static_cast<uint32_t>(nreq) << 8) | static_cast<uint32_t>(q);
+          }
+        }
+        ++nreq;
+        njob += nj;
+      } else {
+        topk_refine_warp(L, args.x + static_cast<size_t>(t) * args.d, args.W_r, args.b_r, args.d,
+                         lane, val);
+        topk_emit(L, val, args.k, lane, idx_out, w_out);
+      }
+    }
+    if (lane == 0) {
+      q_nreq[warp] = nreq;
+      q_njob[warp] = njob;
+    }
+    __syncthreads();
+    // the queued dot products, four at a time, each over all threads
+    int jbase[RT_WARPS + 1];
+    jbase[0] = 0;
+#pragma unroll
+    for (int w = 0; w < RT_WARPS; ++w) jbase[w + 1] = jbase[w] + q_njob[w];
+    const int total = jbase[RT_WARPS];
+    for (int base = 0; base < total; base += 4) {
+      double acc[4] = {0.0, 0.0, 0.0, 0.0};
+      int ex[4] = {0, 0, 0, 0}, rq[4] = {0, 0, 0, 0}, ps[4] = {0, 0, 0, 0};
+      const uint16_t* xr[4] = {args.x, args.x, args.x, args.x};
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const int J = base + g;
+        if (J < total) {
+          int w = 0;
+          while (J >= jbase[w + 1]) ++w;
+          const uint32_t jw = jobs[w * RJ_PER_WARP + (J - jbase[w])];
+          rq[g] = w * RQ_PER_WARP + static_cast<int>(jw >> 8);
+          ps[g] = static_cast<int>(jw & 255u);
+          ex[g] = reqs[rq[g]].cidx[ps[g]];
+          xr[g] = args.x + static_cast<size_t>(t0 + reqs[rq[g]].row) * args.d;
+        }
+      }
+      for (int i = 4 * static_cast<int>(threadIdx.x); i < args.d; i += 4 * RT_THREADS) {
+#pragma unroll
+        for (int g = 0; g < 4; ++g) {
+          if (base + g < total) {
+            const uint2 xb = __ldg(reinterpret_cast<const uint2*>(xr[g] + i));
+            const float4 wv = __ldg(
+                reinterpret_cast<const float4*>(args.W_r + static_cast<size_t>(ex[g]) * args.d + i));
+            acc[g] = fma(static_cast<double>(__uint_as_float(xb.x << 16)), static_cast<double>(wv.x), acc[g]);
+            acc[g] = fma(static_cast<double>(__uint_as_float(xb.x & 0xFFFF0000u)), static_cast<double>(wv.y), acc[g]);
+            acc[g] = fma(static_cast<double>(__uint_as_float(xb.y << 16)), static_cast<double>(wv.z), acc[g]);
+            acc[g] = fma(static_cast<double>(__uint_as_float(xb.y & 0xFFFF0000u)), static_cast<double>(wv.w), acc[g]);
+          }
+        }
+      }
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc[g] += __shfl_xor_sync(0xFFFFFFFFu, acc[g], off);
+        if (lane == 0) red[g * RT_WARPS + warp] = acc[g];
+      }
+      __syncthreads();
+      if (static_cast<int>(threadIdx.x) < 4 && base + static_cast<int>(threadIdx.x) < total) {
+        const int g = static_cast<int>(threadIdx.x);
+        double sum = 0.0;
+#pragma unroll
+        for (int w = 0; w < RT_WARPS; ++w) sum += red[g * RT_WARPS + w];
+        sum += static_cast<double>(__ldg(args.b_r + ex[g]));
+        RefineReq& R = reqs[rq[g]];
+        const int len = __ffsll(static_cast<long long>(~(R.copy_m >> ps[g])));
+        for (int q = ps[g]; q < ps[g] + len; ++q) R.val[q] = sum;
+      }
+      __syncthreads();
+    }
+    // the queued tokens' final order, softmax and stores
+    for (int i = 0; i < q_nreq[warp]; ++i) {
+      const RefineReq& R = reqs[warp * RQ_PER_WARP + i];
+      TopkList L;
+      L.cidx[0] = R.cidx[lane];
+      L.cidx[1] = R.cidx[32 + lane];
+      L.cval[0] = 0.f;
+      L.cval[1] = 0.f;
+      L.m = R.m;
+      L.refine_m = R.refine_m;
+      L.copy_m = R.copy_m;
+      const double val[2] = {R.val[lane], R.val[32 + lane]};
+      const int t = t0 + R.row;
+      topk_emit(L, val, args.k, lane, args.topk_idx + static_cast<size_t>(t) * args.k,
+                args.topk_w + static_cast<size_t>(t) * args.k);
     }
   }
   // no CTA leaves while another may still read its shared memory

@@ -21,6 +21,11 @@ __device__ __forceinline__ uint32_t logit_order_key(float f) {
   return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
+// The logit a key stands for (-0 comes back as +0, any NaN as a NaN).
+__device__ __forceinline__ float logit_of_key(uint32_t key) {
+  return __uint_as_float((key & 0x80000000u) ? (key & 0x7FFFFFFFu) : ~key);
+}
+
 // Same 64-bit order for fp64 values (a float widened to double keeps its
 // place among the floats).
 __device__ __forceinline__ uint64_t value_order_key(double f) {
@@ -38,36 +43,39 @@ __device__ __forceinline__ int slot_expert(int lane, int j) {
 
 // One warp per token: the top-k of the token's logits v (slot j of lane l
 // holds expert slot_expert(l, j), -FLT_MAX past E), the order of near ties
-// settled in fp64, and the softmax over the k selected.
+// settled in fp64, and the softmax over the k selected. Three steps, which a
+// kernel may run apart (all refinements of a block together, for instance):
 //
-// 1. Rounds of a warp arg-max on (logit descending, index ascending) list the
-//    k largest logits, then go on while the next one lies within tau of the
-//    k-th (the candidates that might belong in the top k), at most 64
-//    entries. Position p of the list sits in lane p % 32, slot p / 32.
-// 2. An entry is refined when its gap to the entry before or after it is at
-//    most tau: its logit is recomputed as the fp64 dot product of the bf16 x
-//    row with the fp32 router row (every product exact in fp64), plus the
-//    bias. Entries of one chain of near gaps are all refined; entries whose
-//    gaps are all above tau keep their fp32 value, which lies within tau/2 of
-//    the exact one on either side, so no refined entry can pass them. Rows
-//    with equal fingerprints (fps: equal router rows and biases, e.g. copied
-//    experts) and equal fp32 logits are copies: a gap of zero between copies
-//    needs no refinement (their logits are equal on every evaluation and
-//    already in index order); where one copy is refined, all copies of its
-//    group take the same fp64 value.
-// 3. With any entry refined, k rounds of the arg-max over the list (fp64
-//    values) give the final order; otherwise the list's first k entries are
-//    the result.
-// tau = 0 turns the refinement off (the list is then the plain top-k).
-__device__ __forceinline__ void topk_refine_softmax_warp(const float (&v)[8], int E, int k,
-                                                         float tau,
-                                                         const uint16_t* __restrict__ x_row,
-                                                         const float* __restrict__ W_r,
-                                                         const float* __restrict__ b_r,
-                                                         const unsigned long long* __restrict__ fps,
-                                                         int d,
-                                                         int lane, int32_t* __restrict__ idx_out,
-                                                         float* __restrict__ w_out) {
+// 1. topk_list: rounds of a warp arg-max on (logit descending, index
+//    ascending; two redux instructions per round) list the k largest logits,
+//    then go on while the next one lies within tau of the k-th (the
+//    candidates that might belong in the top k), at most 64 entries. Position
+//    p of the list sits in lane p % 32, slot p / 32. An entry is to be
+//    refined when its gap to the entry before or after it is at most tau.
+//    Rows with equal fingerprints (fps: equal router rows and biases, e.g.
+//    copied experts) and equal fp32 logits are copies: a gap of zero between
+//    copies needs no refinement (their logits are equal on every evaluation
+//    and already in index order); where one copy is refined, all copies of
+//    its group are, with one value. Entries whose gaps are all above tau keep
+//    their fp32 value, which lies within tau/2 of the exact one on either
+//    side, so no refined entry can pass them. tau = 0 turns refinement off.
+// 2. The refined entries' logits become fp64 dot products of the bf16 x row
+//    with the fp32 router row (every product exact in fp64), plus the bias:
+//    topk_refine_warp does it with the warp alone.
+// 3. topk_emit: with any entry refined, k rounds of the arg-max over the list
+//    (fp64 values) give the final order, else the list's first k entries are
+//    the result; then the softmax over the k and the stores.
+struct TopkList {
+  int cidx[2];       // expert at positions lane and 32 + lane
+  float cval[2];     // its fp32 logit
+  int m;             // entries in the list
+  uint64_t refine_m; // positions to refine (bit p)
+  uint64_t copy_m;   // bit p: the entry at p + 1 is a copy of the one at p
+};
+
+__device__ __forceinline__ void topk_list(const float (&v)[8], int E, int k, float tau,
+                                          const unsigned long long* __restrict__ fps, int lane,
+                                          TopkList& L) {
   const unsigned full = 0xFFFFFFFFu;
   uint32_t key[8];
   uint32_t taken = 0;
@@ -77,15 +85,17 @@ __device__ __forceinline__ void topk_refine_softmax_warp(const float (&v)[8], in
     key[j] = logit_order_key(v[j]);
     if (e >= E) taken |= 1u << j;
   }
-  int cidx[2] = {0, 0};
-  float cval[2] = {0.f, 0.f};
-  int m = 0;
+  L.cidx[0] = L.cidx[1] = 0;
+  L.cval[0] = L.cval[1] = 0.f;
+  L.m = 0;
+  L.refine_m = L.copy_m = 0;
   float kth = 0.f;
   const int maxc = E < 64 ? E : 64;
   const bool refine = tau > 0.f;
   for (int r = 0; r < maxc; ++r) {
+    // this lane's best untaken entry, then the warp's: the largest key
+    // (redux max), among the lanes holding it the lowest expert (redux min)
     uint32_t bk = 0;
-    float bv = 0.f;
     int bi = 0x7FFFFFFF;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
@@ -93,143 +103,163 @@ __device__ __forceinline__ void topk_refine_softmax_warp(const float (&v)[8], in
       const int e = slot_expert(lane, j);
       if (bi == 0x7FFFFFFF || key[j] > bk || (key[j] == bk && e < bi)) {
         bk = key[j];
-        bv = v[j];
         bi = e;
       }
     }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const uint32_t ok = __shfl_xor_sync(full, bk, off);
-      const float ov = __shfl_xor_sync(full, bv, off);
-      const int oi = __shfl_xor_sync(full, bi, off);
-      const bool better = (bi == 0x7FFFFFFF) ||
-                          (oi != 0x7FFFFFFF && (ok > bk || (ok == bk && oi < bi)));
-      if (better) {
-        bk = ok;
-        bv = ov;
-        bi = oi;
-      }
-    }
+    const uint32_t top_key = __reduce_max_sync(full, bk);
+    bi = static_cast<int>(__reduce_min_sync(
+        full, (bi != 0x7FFFFFFF && bk == top_key) ? static_cast<uint32_t>(bi) : 0xFFFFFFFFu));
+    const float bv = logit_of_key(top_key);
     // past the k-th: only runners-up within tau of it
     if (r >= k && !(refine && kth - bv <= tau)) break;
     if (((bi & 127) >> 2) == lane) taken |= 1u << (((bi >> 7) << 2) | (bi & 3));
     if (r == k - 1) kth = bv;
     if ((r & 31) == lane) {
-      cidx[r >> 5] = bi;
-      cval[r >> 5] = bv;
+      if (r < 32) {
+        L.cidx[0] = bi;
+        L.cval[0] = bv;
+      } else {
+        L.cidx[1] = bi;
+        L.cval[1] = bv;
+      }
     }
-    m = r + 1;
+    L.m = r + 1;
   }
-
-  // Links between list positions p and p + 1 (bit p of 64-bit masks):
-  // close (gap at most tau) and, among those, copies (equal value and equal
-  // fingerprint: the same router row and bias). Fingerprints are read only
-  // when some link is close.
-  float nx0 = __shfl_down_sync(full, cval[0], 1);
-  const float head1 = __shfl_sync(full, cval[1], 0);
+  const int m = L.m;
+  // links between positions p and p + 1: close (gap at most tau) and, among
+  // those, copies; fingerprints are read only when some link is close
+  float nx0 = __shfl_down_sync(full, L.cval[0], 1);
+  const float head1 = __shfl_sync(full, L.cval[1], 0);
   if (lane == 31) nx0 = head1;
-  const float nx1 = __shfl_down_sync(full, cval[1], 1);
-  const bool close0 = refine && lane + 1 < m && cval[0] - nx0 <= tau;
-  const bool close1 = refine && 33 + lane < m && cval[1] - nx1 <= tau;
+  const float nx1 = __shfl_down_sync(full, L.cval[1], 1);
+  const bool close0 = refine && lane + 1 < m && L.cval[0] - nx0 <= tau;
+  const bool close1 = refine && 33 + lane < m && L.cval[1] - nx1 <= tau;
   const uint64_t close_m = static_cast<uint64_t>(__ballot_sync(full, close0)) |
                            (static_cast<uint64_t>(__ballot_sync(full, close1)) << 32);
-  uint64_t refine_m = 0, copy_m = 0;
   if (close_m) {
-    const unsigned long long f0 = lane < m ? __ldg(fps + cidx[0]) : 0ull;
-    const unsigned long long f1 = 32 + lane < m ? __ldg(fps + cidx[1]) : 0ull;
+    const unsigned long long f0 = lane < m ? __ldg(fps + L.cidx[0]) : 0ull;
+    const unsigned long long f1 = 32 + lane < m ? __ldg(fps + L.cidx[1]) : 0ull;
     unsigned long long nf0 = __shfl_down_sync(full, f0, 1);
     const unsigned long long fhead1 = __shfl_sync(full, f1, 0);
     if (lane == 31) nf0 = fhead1;
     const unsigned long long nf1 = __shfl_down_sync(full, f1, 1);
-    copy_m = static_cast<uint64_t>(__ballot_sync(full, close0 && cval[0] == nx0 && f0 == nf0)) |
-             (static_cast<uint64_t>(__ballot_sync(full, close1 && cval[1] == nx1 && f1 == nf1))
-              << 32);
+    const uint64_t copy_m =
+        static_cast<uint64_t>(__ballot_sync(full, close0 && L.cval[0] == nx0 && f0 == nf0)) |
+        (static_cast<uint64_t>(__ballot_sync(full, close1 && L.cval[1] == nx1 && f1 == nf1))
+         << 32);
     // both ends of every close link that is not a copy, then whole groups of
-    // copies around them (a copy gets the value of the first of its group)
+    // copies around them
     const uint64_t near_m = close_m & ~copy_m;
-    refine_m = near_m | (near_m << 1);
+    uint64_t rm = near_m | (near_m << 1);
     for (;;) {
-      const uint64_t g = refine_m | ((refine_m << 1) & (copy_m << 1)) | ((refine_m >> 1) & copy_m);
-      if (g == refine_m) break;
-      refine_m = g;
+      const uint64_t g = rm | ((rm << 1) & (copy_m << 1)) | ((rm >> 1) & copy_m);
+      if (g == rm) break;
+      rm = g;
     }
+    L.refine_m = rm;
+    L.copy_m = copy_m;
   }
+}
 
-  int my_idx;
-  double my_val, top;
-  if (refine_m == 0) {
-    my_idx = cidx[0];
-    my_val = static_cast<double>(cval[0]);
-    top = static_cast<double>(__shfl_sync(full, cval[0], 0));
-  } else {
-    double val[2] = {static_cast<double>(cval[0]), static_cast<double>(cval[1])};
-    // computed: the first entry of each refined group of copies
-    uint64_t pending = refine_m & ~(copy_m << 1);
-    const int d128 = d & ~127;
-    while (pending) {
-      // up to four refined entries per pass over the x row
-      int pos[4], ex[4];
-      int ng = 0;
+// Entries computed for a refined list: the first entry of each refined group
+// of copies (the others take its value).
+__device__ __forceinline__ uint64_t topk_refine_starts(const TopkList& L) {
+  return L.refine_m & ~(L.copy_m << 1);
+}
+
+// Positions pos .. pos + len - 1 of the group that starts at pos.
+__device__ __forceinline__ int topk_group_len(const TopkList& L, int pos) {
+  return __ffsll(static_cast<long long>(~(L.copy_m >> pos)));
+}
+
+// Step 2 by the warp alone: val[slot] becomes the fp64 logit of each refined
+// entry (others keep their fp32 value).
+__device__ __forceinline__ void topk_refine_warp(const TopkList& L,
+                                                 const uint16_t* __restrict__ x_row,
+                                                 const float* __restrict__ W_r,
+                                                 const float* __restrict__ b_r, int d, int lane,
+                                                 double (&val)[2]) {
+  const unsigned full = 0xFFFFFFFFu;
+  uint64_t pending = topk_refine_starts(L);
+  const int d128 = d & ~127;
+  while (pending) {
+    // up to four refined entries per pass over the x row
+    int pos[4], ex[4];
+    int ng = 0;
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        pos[g] = -1;
-        ex[g] = 0;
-        if (pending) {
-          const int p = __ffsll(static_cast<long long>(pending)) - 1;
-          pending &= pending - 1;
-          const int src = (p >> 5) ? cidx[1] : cidx[0];
-          pos[g] = p;
-          ex[g] = __shfl_sync(full, src, p & 31);
-          ng = g + 1;
-        }
+    for (int g = 0; g < 4; ++g) {
+      pos[g] = -1;
+      ex[g] = 0;
+      if (pending) {
+        const int p = __ffsll(static_cast<long long>(pending)) - 1;
+        pending &= pending - 1;
+        const int src = (p >> 5) ? L.cidx[1] : L.cidx[0];
+        pos[g] = p;
+        ex[g] = __shfl_sync(full, src, p & 31);
+        ng = g + 1;
       }
-      double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    }
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
 #pragma unroll 4
-      for (int i = 4 * lane; i < d128; i += 128) {
-        const uint2 xb = __ldg(reinterpret_cast<const uint2*>(x_row + i));
-        const double x0 = __uint_as_float(xb.x << 16), x1 = __uint_as_float(xb.x & 0xFFFF0000u);
-        const double x2 = __uint_as_float(xb.y << 16), x3 = __uint_as_float(xb.y & 0xFFFF0000u);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          if (g < ng) {
-            const float4 w =
-                __ldg(reinterpret_cast<const float4*>(W_r + static_cast<size_t>(ex[g]) * d + i));
-            acc[g] = fma(x0, static_cast<double>(w.x), acc[g]);
-            acc[g] = fma(x1, static_cast<double>(w.y), acc[g]);
-            acc[g] = fma(x2, static_cast<double>(w.z), acc[g]);
-            acc[g] = fma(x3, static_cast<double>(w.w), acc[g]);
-          }
-        }
-      }
-      for (int i = d128 + lane; i < d; i += 32) {
-        const double xv = __uint_as_float(static_cast<uint32_t>(__ldg(x_row + i)) << 16);
-#pragma unroll
-        for (int g = 0; g < 4; ++g)
-          if (g < ng)
-            acc[g] = fma(xv, static_cast<double>(__ldg(W_r + static_cast<size_t>(ex[g]) * d + i)),
-                         acc[g]);
-      }
+    for (int i = 4 * lane; i < d128; i += 128) {
+      const uint2 xb = __ldg(reinterpret_cast<const uint2*>(x_row + i));
+      const double x0 = __uint_as_float(xb.x << 16), x1 = __uint_as_float(xb.x & 0xFFFF0000u);
+      const double x2 = __uint_as_float(xb.y << 16), x3 = __uint_as_float(xb.y & 0xFFFF0000u);
 #pragma unroll
       for (int g = 0; g < 4; ++g) {
         if (g < ng) {
-#pragma unroll
-          for (int off = 16; off > 0; off >>= 1) acc[g] += __shfl_xor_sync(full, acc[g], off);
-          const double s = acc[g] + static_cast<double>(__ldg(b_r + ex[g]));
-          // the entry and the copies that follow it
-          const int len = __ffsll(static_cast<long long>(~(copy_m >> pos[g])));
-#pragma unroll
-          for (int sl = 0; sl < 2; ++sl) {
-            const int q = 32 * sl + lane;
-            if (q >= pos[g] && q < pos[g] + len) val[sl] = s;
-          }
+          const float4 w =
+              __ldg(reinterpret_cast<const float4*>(W_r + static_cast<size_t>(ex[g]) * d + i));
+          acc[g] = fma(x0, static_cast<double>(w.x), acc[g]);
+          acc[g] = fma(x1, static_cast<double>(w.y), acc[g]);
+          acc[g] = fma(x2, static_cast<double>(w.z), acc[g]);
+          acc[g] = fma(x3, static_cast<double>(w.w), acc[g]);
         }
       }
     }
-    // the final order over the m entries
+    for (int i = d128 + lane; i < d; i += 32) {
+      const double xv = __uint_as_float(static_cast<uint32_t>(__ldg(x_row + i)) << 16);
+#pragma unroll
+      for (int g = 0; g < 4; ++g)
+        if (g < ng)
+          acc[g] = fma(xv, static_cast<double>(__ldg(W_r + static_cast<size_t>(ex[g]) * d + i)),
+                       acc[g]);
+    }
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      if (g < ng) {
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) acc[g] += __shfl_xor_sync(full, acc[g], off);
+        const double s = acc[g] + static_cast<double>(__ldg(b_r + ex[g]));
+        const int len = topk_group_len(L, pos[g]);
+#pragma unroll
+        for (int sl = 0; sl < 2; ++sl) {
+          const int q = 32 * sl + lane;
+          if (q >= pos[g] && q < pos[g] + len) val[sl] = s;
+        }
+      }
+    }
+  }
+}
+
+// Step 3: final order (fp64 values where refined), softmax over the k
+// winners, stores of their experts and weights.
+__device__ __forceinline__ void topk_emit(const TopkList& L, const double (&val)[2], int k,
+                                          int lane, int32_t* __restrict__ idx_out,
+                                          float* __restrict__ w_out) {
+  const unsigned full = 0xFFFFFFFFu;
+  const int m = L.m;
+  int my_idx;
+  double my_val, top;
+  if (L.refine_m == 0) {
+    my_idx = L.cidx[0];
+    my_val = static_cast<double>(L.cval[0]);
+    top = static_cast<double>(__shfl_sync(full, L.cval[0], 0));
+  } else {
     uint32_t ctaken = 0;
     if (lane >= m) ctaken |= 1u;
     if (32 + lane >= m) ctaken |= 2u;
-    uint64_t vk[2] = {value_order_key(val[0]), value_order_key(val[1])};
+    const uint64_t vk[2] = {value_order_key(val[0]), value_order_key(val[1])};
     my_idx = 0;
     my_val = 0.0;
     top = 0.0;
@@ -240,10 +270,10 @@ __device__ __forceinline__ void topk_refine_softmax_warp(const float (&v)[8], in
 #pragma unroll
       for (int s2 = 0; s2 < 2; ++s2) {
         if (ctaken & (1u << s2)) continue;
-        if (bi == 0x7FFFFFFF || vk[s2] > bk || (vk[s2] == bk && cidx[s2] < bi)) {
+        if (bi == 0x7FFFFFFF || vk[s2] > bk || (vk[s2] == bk && L.cidx[s2] < bi)) {
           bk = vk[s2];
           bv = val[s2];
-          bi = cidx[s2];
+          bi = L.cidx[s2];
           bs = s2;
         }
       }
