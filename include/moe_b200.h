@@ -347,7 +347,7 @@ MOE_API moe_status moe_route(const void* x_dev, const float* W_r_dev, const floa
  * required here), minus the workspace; it makes the same launches as
  * moe_route, so its results are bit-identical to moe_route's. The scratch it
  * needs (router logits, the router's split weights and small routing tables)
- * lives in one device array owned by the library: 28.1 MiB that every GPU
+ * lives in one device array owned by the library: 32.1 MiB that every GPU
  * which loads the library holds until the process exits. Limit: T * E <= 1,048,576 (e.g. T = 8192 tokens at E = 128,
  * or T = 4096 at E = 248); larger calls return MOE_ERR_UNSUPPORTED and
  * launch nothing. Every call looks up the array's device address on the

@@ -92,7 +92,7 @@ void make_layout(int E, int k, int T, int d, int I, bool hostio, Layout* L, bool
   L->chunk_hist = take(NB * E * 4);
   L->chunk_base = take(NB * E * 4);
   L->pub.perm = take(P * 4);
-  L->router_terms = take(moe::router_tc_scratch_bytes(E, d));
+  L->router_terms = take(moe::router_tc_scratch_bytes(E, d, T));
   const size_t tr = moe::mx_tok_rows(static_cast<int>(P), E);
   L->mx_tok_rows = tr;
   auto larger = [](size_t a, size_t b) { return a > b ? a : b; };
@@ -130,7 +130,7 @@ void make_route_layout(int E, int k, int T, int d, Layout* L) {
   L->chunk_hist = take(NB * E * 4);
   L->chunk_base = take(NB * E * 4);
   L->pub.offsets = take(static_cast<size_t>(E + 1) * 4);  // used when the caller passes none
-  L->router_terms = take(moe::router_tc_scratch_bytes(E, d));
+  L->router_terms = take(moe::router_tc_scratch_bytes(E, d, T));
   L->pub.total = off;
 }
 
@@ -595,7 +595,7 @@ moe_status moe_workspace_layout(int E, int k, int T, int d, int I, moe_ws_layout
 
 int moe_forward_launch_count(int E, int k, int T, int d, int I) {
   if (!full_shape_ok(E, k, T, d, I) || T == 0) return 0;
-  int n = 11;
+  int n = 12;
   // small batches: the permutation in one launch instead of three
   if (T <= moe::kPermChunk) n -= 2;
   // the block-scaled path launches no scale transposes

@@ -64,12 +64,12 @@ inline int perm_chunks(int T) { return (T + kPermChunk - 1) / kPermChunk; }
 cudaError_t launch_perm_small(const int32_t* topk_idx, int T, int k, int E, int32_t* counts,
                               int32_t* offsets, int32_t* mtile_prefix, int32_t* perm,
                               cudaStream_t st);
-// K1, the router (moe_router_tc.cu): splits W_r into three bf16 terms and
-// its row norms in `scratch` (router_tc_scratch_bytes), then one kernel
-// computes the logits (written to `logits`, [T][E] fp32), the top-k with
-// near ties settled in fp64, and the softmax. Its first launch clears
-// *status.
-size_t router_tc_scratch_bytes(int E, int d);
+// K1, the router (moe_router_tc.cu): splits W_r into three bf16 terms, its
+// row norms and fingerprints in `scratch` (router_tc_scratch_bytes, which
+// also holds ||x_t||^2 per token); then one kernel computes the logits
+// (written to `logits`, [T][E] fp32) and one the top-k with near ties settled
+// in fp64, and the softmax. Its first launch clears *status.
+size_t router_tc_scratch_bytes(int E, int d, int T);
 cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b_r, int T, int E,
                              int k, int d, void* scratch, float* logits, int32_t* topk_idx,
                              float* topk_w, int* status, cudaStream_t st);

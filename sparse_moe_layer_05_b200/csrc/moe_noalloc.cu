@@ -29,10 +29,10 @@ namespace {
 // Largest T * E accepted: the fp32 router logits take 4 bytes per
 // (token, expert). The router's split weights (three bf16 terms per weight,
 // a norm and a fingerprint per expert row) take at most
-// 3 * 256 * 16384 * 2 + 256 * 12 bytes; the rest of the scratch is small
-// tables.
+// 3 * 256 * 16384 * 2 + 256 * 12 bytes, its per-token ||x||^2 at most
+// 4 * 2^20 bytes; the rest of the scratch is small tables.
 constexpr size_t kNoAllocMaxTE = size_t(1) << 20;
-constexpr size_t kNoAllocRouterBytes = size_t(3) * 256 * 16384 * 2 + 4096;
+constexpr size_t kNoAllocRouterBytes = size_t(3) * 256 * 16384 * 2 + 4096 + kNoAllocMaxTE * 4;
 constexpr size_t kNoAllocScratchBytes =
     kNoAllocMaxTE * 4 + kNoAllocRouterBytes + (size_t(64) << 10);
 
@@ -59,7 +59,7 @@ ScratchLayout scratch_layout(int E, int T, int d) {
   L.logits = off;
   off = round256(off + static_cast<size_t>(T) * E * 4);
   L.router = off;
-  off = round256(off + moe::router_tc_scratch_bytes(E, d));
+  off = round256(off + moe::router_tc_scratch_bytes(E, d, T));
   L.total = off;
   return L;
 }

@@ -71,22 +71,19 @@ constexpr int RT_FIXED = 1024;            // barriers, TMEM address, flags
 // the refinement margin tau_t relative to ||x_t|| max_e ||W_r[e]|| (2^-17)
 constexpr float kRefineRel = 7.62939453125e-06f;
 
-// Refinements are queued per warp in shared memory (above the partial
-// logits) and computed by the whole block together: each fp64 dot product is
-// split over all 256 threads, so a refinement costs one pass of loads
-// instead of a warp's chain of them. A warp whose queue is full refines
+// The top-k kernel queues each token's refinements in shared memory and
+// computes them with the whole block: each fp64 dot product is split over
+// all 256 threads, so a refinement costs one pass of loads instead of a
+// warp's chain of them. A token with more than RJ_PER_WARP of them refines
 // alone.
-constexpr int RQ_PER_WARP = 4;            // queued token lists per warp
-constexpr int RJ_PER_WARP = 64;           // queued dot products per warp
+constexpr int RJ_PER_WARP = 64;           // queued dot products per token
 struct RefineReq {
   int row, m, pad0, pad1;
   unsigned long long refine_m, copy_m;
   double val[64];
   int cidx[64];
 };
-constexpr int RT_WARPS = 8;
-constexpr int kQueueBytes = 64 + RT_WARPS * RQ_PER_WARP * static_cast<int>(sizeof(RefineReq)) +
-                            RT_WARPS * RJ_PER_WARP * 4 + 4 * RT_WARPS * 8;
+constexpr int TK_WARPS = 8;               // tokens per block of the top-k kernel
 
 struct RouterTcShape {
   int npad;          // E rounded up to 16
@@ -105,7 +102,7 @@ RouterTcShape router_tc_shape(int E) {
   s.npad = (E + 15) / 16 * 16;
   s.stage_bytes = RT_M * 128 + 3 * s.npad * 128;
   s.ld = s.npad + 4;
-  const int partial_bytes = RT_M * s.ld * 4 + RT_M * 4 + kQueueBytes + 16;
+  const int partial_bytes = RT_M * s.ld * 4 + RT_M * 4;
   int st = (RT_SMEM_LIMIT - RT_FIXED - 1024) / s.stage_bytes;
   if (st > RT_MAX_STAGES) st = RT_MAX_STAGES;
   s.stages = st;
@@ -201,6 +198,7 @@ struct RouterTcArgs {
   const unsigned long long* fps;
   int T, E, k, d, npad, nacc, per, stages, ld, stage_bytes, body, tmem_cols, KB;
   float* logits;
+  float* xsq;
   int32_t* topk_idx;
   float* topk_w;
   int* status;
@@ -424,8 +422,8 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
     tmem_dealloc(tmem_base, static_cast<uint32_t>(args.tmem_cols));
   }
 
-  // rows [rank 128 / C, (rank+1) 128 / C) are finished by this CTA; no other
-  // CTA reads them from this CTA's buffer, so their sums go back in place
+  // rows [rank 128 / C, (rank+1) 128 / C) are finished by this CTA: logits
+  // and ||x_t||^2 to global memory for the top-k kernel
   if (!*abort_flag) {
     const int E = args.E;
     const int rpc = RT_M / static_cast<int>(csize);
@@ -455,178 +453,174 @@ __global__ void __launch_bounds__(RT_THREADS, 1)
         }
       }
       const int t = t0 + rr;
+      if (t < args.T) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (e0 + i < E) {
-          acc[i] += __ldg(args.b_r + e0 + i);
-          if (t < args.T) args.logits[static_cast<size_t>(t) * E + e0 + i] = acc[i];
-        }
+        for (int i = 0; i < 4; ++i)
+          if (e0 + i < E)
+            args.logits[static_cast<size_t>(t) * E + e0 + i] = acc[i] + __ldg(args.b_r + e0 + i);
       }
-      *reinterpret_cast<float4*>(partial + rr * args.ld + e0) =
-          make_float4(acc[0], acc[1], acc[2], acc[3]);
     }
     for (int rr = rbeg + static_cast<int>(threadIdx.x); rr < rbeg + rpc; rr += RT_THREADS) {
       float xsq = 0.f;
       for (uint32_t q = 0; q < csize; ++q)
         xsq += ld_shared_cluster_f32(mapa_shared(xbase + static_cast<uint32_t>(rr * 4), q));
-      xsq_part[rr] = xsq;
-    }
-    __syncthreads();
-    // 2. one warp per token: top-k with near-tie refinement, softmax
-    float wmax = 0.f;
-#pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      const int e = lane + 32 * j;
-      if (e < E) wmax = fmaxf(wmax, __ldg(args.norms + e));
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1)
-      wmax = fmaxf(wmax, __shfl_xor_sync(0xFFFFFFFFu, wmax, off));
-    // the queue (above the partial logits and row norms)
-    uint8_t* qb = reinterpret_cast<uint8_t*>(
-        (reinterpret_cast<uintptr_t>(xsq_part + RT_M) + 15) & ~static_cast<uintptr_t>(15));
-    int* q_nreq = reinterpret_cast<int*>(qb);                 // [8]
-    int* q_njob = q_nreq + RT_WARPS;                          // [8]
-    RefineReq* reqs = reinterpret_cast<RefineReq*>(qb + 64);  // [8][RQ_PER_WARP]
-    uint32_t* jobs = reinterpret_cast<uint32_t*>(reqs + RT_WARPS * RQ_PER_WARP);  // [8][RJ]
-    double* red = reinterpret_cast<double*>(jobs + RT_WARPS * RJ_PER_WARP);     // [4][8]
-    int nreq = 0, njob = 0;
-    for (int rr = rbeg + warp; rr < rbeg + rpc; rr += RT_THREADS / 32) {
-      const int t = t0 + rr;
-      if (t >= args.T) break;
-      // lane l holds experts 128 h + 4 l + i (slot 4 h + i)
-      float v[8];
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        const int e0 = 128 * h + 4 * lane;
-        float4 q4 = make_float4(-FLT_MAX, -FLT_MAX, -FLT_MAX, -FLT_MAX);
-        if (e0 < args.npad) q4 = *reinterpret_cast<const float4*>(partial + rr * args.ld + e0);
-        v[4 * h] = e0 < E ? q4.x : -FLT_MAX;
-        v[4 * h + 1] = e0 + 1 < E ? q4.y : -FLT_MAX;
-        v[4 * h + 2] = e0 + 2 < E ? q4.z : -FLT_MAX;
-        v[4 * h + 3] = e0 + 3 < E ? q4.w : -FLT_MAX;
-      }
-      float tau = kRefineRel * sqrtf(xsq_part[rr]) * wmax;
-      if (!(tau <= FLT_MAX)) tau = 0.f;
-      TopkList L;
-      topk_list(v, E, args.k, tau, args.fps, lane, L);
-      int32_t* idx_out = args.topk_idx + static_cast<size_t>(t) * args.k;
-      float* w_out = args.topk_w + static_cast<size_t>(t) * args.k;
-      double val[2] = {static_cast<double>(L.cval[0]), static_cast<double>(L.cval[1])};
-      if (L.refine_m == 0) {
-        topk_emit(L, val, args.k, lane, idx_out, w_out);
-        continue;
-      }
-      const uint64_t starts = topk_refine_starts(L);
-      const int nj = __popcll(starts);
-      if (nreq < RQ_PER_WARP && njob + nj <= RJ_PER_WARP) {
-        RefineReq& R = reqs[warp * RQ_PER_WARP + nreq];
-        if (lane == 0) {
-          R.row = rr;
-          R.m = L.m;
-          R.refine_m = L.refine_m;
-          R.copy_m = L.copy_m;
-        }
-        R.cidx[lane] = L.cidx[0];
-        R.cidx[32 + lane] = L.cidx[1];
-        R.val[lane] = val[0];
-        R.val[32 + lane] = val[1];
-#pragma unroll
-        for (int sl = 0; sl < 2; ++sl) {
-          const int q = 32 * sl + lane;
-          if ((starts >> q) & 1ull) {
-            const int j = njob + __popcll(starts & ((1ull << q) - 1ull));
-            jobs[warp * RJ_PER_WARP + j] = (static_cast<uint32_t>(nreq) << 8) | static_cast<uint32_t>(q);
-          }
-        }
-        ++nreq;
-        njob += nj;
-      } else {
-        topk_refine_warp(L, args.x + static_cast<size_t>(t) * args.d, args.W_r, args.b_r, args.d,
-                         lane, val);
-        topk_emit(L, val, args.k, lane, idx_out, w_out);
-      }
-    }
-    if (lane == 0) {
-      q_nreq[warp] = nreq;
-      q_njob[warp] = njob;
-    }
-    __syncthreads();
-    // the queued dot products, four at a time, each over all threads
-    int jbase[RT_WARPS + 1];
-    jbase[0] = 0;
-#pragma unroll
-    for (int w = 0; w < RT_WARPS; ++w) jbase[w + 1] = jbase[w] + q_njob[w];
-    const int total = jbase[RT_WARPS];
-    for (int base = 0; base < total; base += 4) {
-      double acc[4] = {0.0, 0.0, 0.0, 0.0};
-      int ex[4] = {0, 0, 0, 0}, rq[4] = {0, 0, 0, 0}, ps[4] = {0, 0, 0, 0};
-      const uint16_t* xr[4] = {args.x, args.x, args.x, args.x};
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const int J = base + g;
-        if (J < total) {
-          int w = 0;
-          while (J >= jbase[w + 1]) ++w;
-          const uint32_t jw = jobs[w * RJ_PER_WARP + (J - jbase[w])];
-          rq[g] = w * RQ_PER_WARP + static_cast<int>(jw >> 8);
-          ps[g] = static_cast<int>(jw & 255u);
-          ex[g] = reqs[rq[g]].cidx[ps[g]];
-          xr[g] = args.x + static_cast<size_t>(t0 + reqs[rq[g]].row) * args.d;
-        }
-      }
-      for (int i = 4 * static_cast<int>(threadIdx.x); i < args.d; i += 4 * RT_THREADS) {
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          if (base + g < total) {
-            const uint2 xb = __ldg(reinterpret_cast<const uint2*>(xr[g] + i));
-            const float4 wv = __ldg(
-                reinterpret_cast<const float4*>(args.W_r + static_cast<size_t>(ex[g]) * args.d + i));
-            acc[g] = fma(static_cast<double>(__uint_as_float(xb.x << 16)), static_cast<double>(wv.x), acc[g]);
-            acc[g] = fma(static_cast<double>(__uint_as_float(xb.x & 0xFFFF0000u)), static_cast<double>(wv.y), acc[g]);
-            acc[g] = fma(static_cast<double>(__uint_as_float(xb.y << 16)), static_cast<double>(wv.z), acc[g]);
-            acc[g] = fma(static_cast<double>(__uint_as_float(xb.y & 0xFFFF0000u)), static_cast<double>(wv.w), acc[g]);
-          }
-        }
-      }
-#pragma unroll
-      for (int g = 0; g < 4; ++g) {
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) acc[g] += __shfl_xor_sync(0xFFFFFFFFu, acc[g], off);
-        if (lane == 0) red[g * RT_WARPS + warp] = acc[g];
-      }
-      __syncthreads();
-      if (static_cast<int>(threadIdx.x) < 4 && base + static_cast<int>(threadIdx.x) < total) {
-        const int g = static_cast<int>(threadIdx.x);
-        double sum = 0.0;
-#pragma unroll
-        for (int w = 0; w < RT_WARPS; ++w) sum += red[g * RT_WARPS + w];
-        sum += static_cast<double>(__ldg(args.b_r + ex[g]));
-        RefineReq& R = reqs[rq[g]];
-        const int len = __ffsll(static_cast<long long>(~(R.copy_m >> ps[g])));
-        for (int q = ps[g]; q < ps[g] + len; ++q) R.val[q] = sum;
-      }
-      __syncthreads();
-    }
-    // the queued tokens' final order, softmax and stores
-    for (int i = 0; i < q_nreq[warp]; ++i) {
-      const RefineReq& R = reqs[warp * RQ_PER_WARP + i];
-      TopkList L;
-      L.cidx[0] = R.cidx[lane];
-      L.cidx[1] = R.cidx[32 + lane];
-      L.cval[0] = 0.f;
-      L.cval[1] = 0.f;
-      L.m = R.m;
-      L.refine_m = R.refine_m;
-      L.copy_m = R.copy_m;
-      const double val[2] = {R.val[lane], R.val[32 + lane]};
-      const int t = t0 + R.row;
-      topk_emit(L, val, args.k, lane, args.topk_idx + static_cast<size_t>(t) * args.k,
-                args.topk_w + static_cast<size_t>(t) * args.k);
+      if (t0 + rr < args.T) args.xsq[t0 + rr] = xsq;
     }
   }
   // no CTA leaves while another may still read its shared memory
   cluster_sync();
+}
+
+struct RouterTopkArgs {
+  const float* logits;
+  const float* xsq;
+  const float* norms;
+  const unsigned long long* fps;
+  const uint16_t* x;
+  const float* W_r;
+  const float* b_r;
+  int T, E, k, d;
+  int32_t* topk_idx;
+  float* topk_w;
+};
+
+// One warp per token: top-k of its fp32 logits, near ties settled in fp64
+// (the block's queued dot products computed by all its threads), softmax.
+__global__ void __launch_bounds__(TK_WARPS * 32) router_topk_kernel(const RouterTopkArgs args) {
+  pdl_wait_and_trigger();
+  __shared__ RefineReq reqs[TK_WARPS];
+  __shared__ uint32_t jobs[TK_WARPS * RJ_PER_WARP];
+  __shared__ int q_njob[TK_WARPS];
+  __shared__ double red[4 * TK_WARPS];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int E = args.E;
+  const int t = static_cast<int>(blockIdx.x) * TK_WARPS + warp;
+  float wmax = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    const int e = lane + 32 * j;
+    if (e < E) wmax = fmaxf(wmax, __ldg(args.norms + e));
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) wmax = fmaxf(wmax, __shfl_xor_sync(0xFFFFFFFFu, wmax, off));
+  int njob = 0;
+  if (t < args.T) {
+    // lane l holds experts 128 h + 4 l + i (slot 4 h + i)
+    const float* row = args.logits + static_cast<size_t>(t) * E;
+    float v[8];
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int e = slot_expert(lane, j);
+      v[j] = e < E ? __ldg(row + e) : -FLT_MAX;
+    }
+    float tau = kRefineRel * sqrtf(__ldg(args.xsq + t)) * wmax;
+    if (!(tau <= FLT_MAX)) tau = 0.f;
+    TopkList L;
+    topk_list(v, E, args.k, tau, args.fps, lane, L);
+    int32_t* idx_out = args.topk_idx + static_cast<size_t>(t) * args.k;
+    float* w_out = args.topk_w + static_cast<size_t>(t) * args.k;
+    double val[2] = {static_cast<double>(L.cval[0]), static_cast<double>(L.cval[1])};
+    const uint64_t starts = topk_refine_starts(L);
+    const int nj = __popcll(starts);
+    if (L.refine_m == 0) {
+      topk_emit(L, val, args.k, lane, idx_out, w_out);
+    } else if (nj <= RJ_PER_WARP) {
+      RefineReq& R = reqs[warp];
+      if (lane == 0) {
+        R.row = t;
+        R.m = L.m;
+        R.refine_m = L.refine_m;
+        R.copy_m = L.copy_m;
+      }
+      R.cidx[lane] = L.cidx[0];
+      R.cidx[32 + lane] = L.cidx[1];
+      R.val[lane] = val[0];
+      R.val[32 + lane] = val[1];
+#pragma unroll
+      for (int sl = 0; sl < 2; ++sl) {
+        const int q = 32 * sl + lane;
+        if ((starts >> q) & 1ull)
+          jobs[warp * RJ_PER_WARP + __popcll(starts & ((1ull << q) - 1ull))] =
+              static_cast<uint32_t>(q);
+      }
+      njob = nj;
+    } else {
+      topk_refine_warp(L, args.x + static_cast<size_t>(t) * args.d, args.W_r, args.b_r, args.d,
+                       lane, val);
+      topk_emit(L, val, args.k, lane, idx_out, w_out);
+    }
+  }
+  if (lane == 0) q_njob[warp] = njob;
+  __syncthreads();
+  // the queued dot products, four at a time, each over all threads
+  int jbase[TK_WARPS + 1];
+  jbase[0] = 0;
+#pragma unroll
+  for (int w = 0; w < TK_WARPS; ++w) jbase[w + 1] = jbase[w] + q_njob[w];
+  const int total = jbase[TK_WARPS];
+  for (int base = 0; base < total; base += 4) {
+    double acc[4] = {0.0, 0.0, 0.0, 0.0};
+    int ex[4] = {0, 0, 0, 0}, rw[4] = {0, 0, 0, 0}, ps[4] = {0, 0, 0, 0};
+    const uint16_t* xr[4] = {args.x, args.x, args.x, args.x};
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      const int J = base + g;
+      if (J < total) {
+        int w = 0;
+        while (J >= jbase[w + 1]) ++w;
+        rw[g] = w;
+        ps[g] = static_cast<int>(jobs[w * RJ_PER_WARP + (J - jbase[w])]);
+        ex[g] = reqs[w].cidx[ps[g]];
+        xr[g] = args.x + static_cast<size_t>(reqs[w].row) * args.d;
+      }
+    }
+    for (int i = 4 * static_cast<int>(threadIdx.x); i < args.d; i += 4 * TK_WARPS * 32) {
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        if (base + g < total) {
+          const uint2 xb = __ldg(reinterpret_cast<const uint2*>(xr[g] + i));
+          const float4 wv = __ldg(
+              reinterpret_cast<const float4*>(args.W_r + static_cast<size_t>(ex[g]) * args.d + i));
+          acc[g] = fma(static_cast<double>(__uint_as_float(xb.x << 16)), static_cast<double>(wv.x), acc[g]);
+          acc[g] = fma(static_cast<double>(__uint_as_float(xb.x & 0xFFFF0000u)), static_cast<double>(wv.y), acc[g]);
+          acc[g] = fma(static_cast<double>(__uint_as_float(xb.y << 16)), static_cast<double>(wv.z), acc[g]);
+          acc[g] = fma(static_cast<double>(__uint_as_float(xb.y & 0xFFFF0000u)), static_cast<double>(wv.w), acc[g]);
+        }
+      }
+    }
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) acc[g] += __shfl_xor_sync(0xFFFFFFFFu, acc[g], off);
+      if (lane == 0) red[g * TK_WARPS + warp] = acc[g];
+    }
+    __syncthreads();
+    if (static_cast<int>(threadIdx.x) < 4 && base + static_cast<int>(threadIdx.x) < total) {
+      const int g = static_cast<int>(threadIdx.x);
+      double sum = 0.0;
+#pragma unroll
+      for (int w = 0; w < TK_WARPS; ++w) sum += red[g * TK_WARPS + w];
+      sum += static_cast<double>(__ldg(args.b_r + ex[g]));
+      RefineReq& R = reqs[rw[g]];
+      const int len = __ffsll(static_cast<long long>(~(R.copy_m >> ps[g])));
+      for (int q = ps[g]; q < ps[g] + len; ++q) R.val[q] = sum;
+    }
+    __syncthreads();
+  }
+  if (njob > 0) {
+    const RefineReq& R = reqs[warp];
+    TopkList L;
+    L.cidx[0] = R.cidx[lane];
+    L.cidx[1] = R.cidx[32 + lane];
+    L.cval[0] = 0.f;
+    L.cval[1] = 0.f;
+    L.m = R.m;
+    L.refine_m = R.refine_m;
+    L.copy_m = R.copy_m;
+    const double val[2] = {R.val[lane], R.val[32 + lane]};
+    topk_emit(L, val, args.k, lane, args.topk_idx + static_cast<size_t>(t) * args.k,
+              args.topk_w + static_cast<size_t>(t) * args.k);
+  }
 }
 
 // Clusters of C CTAs of router_tc_kernel (the largest shared-memory shape)
@@ -684,9 +678,9 @@ int cluster_size(int T, int d, int dev, size_t smem) {
 
 }  // namespace
 
-size_t router_tc_scratch_bytes(int E, int d) {
+size_t router_tc_scratch_bytes(int E, int d, int T) {
   const size_t npad = static_cast<size_t>((E + 15) / 16 * 16);
-  return 3 * npad * static_cast<size_t>(d) * 2 + npad * 4 + npad * 8;
+  return 3 * npad * static_cast<size_t>(d) * 2 + npad * 4 + npad * 8 + static_cast<size_t>(T) * 4;
 }
 
 cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b_r, int T, int E,
@@ -712,6 +706,7 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b
   float* norms = reinterpret_cast<float*>(static_cast<uint8_t*>(scratch) +
                                           3 * static_cast<size_t>(sh.npad) * d * 2);
   unsigned long long* fps = reinterpret_cast<unsigned long long*>(norms + sh.npad);
+  float* xsq = reinterpret_cast<float*>(fps + sh.npad);
   // the weight split: the first launch of the pass (it clears the status word)
   {
     cudaError_t e = launch_kernel(router_split_kernel, dim3(sh.npad), dim3(256), 0, st, W_r, b_r,
@@ -754,12 +749,30 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b
   a.tmem_cols = sh.tmem_cols;
   a.KB = (d + RT_BK - 1) / RT_BK;
   a.logits = logits;
+  a.xsq = xsq;
   a.topk_idx = topk_idx;
   a.topk_w = topk_w;
   a.status = status;
   const int tiles = (T + RT_M - 1) / RT_M;
-  return launch_kernel_cluster(router_tc_kernel, dim3(tiles * C), dim3(RT_THREADS),
-                               static_cast<size_t>(sh.smem_alloc), C, st, tmX, tmW, a);
+  cudaError_t e = launch_kernel_cluster(router_tc_kernel, dim3(tiles * C), dim3(RT_THREADS),
+                                        static_cast<size_t>(sh.smem_alloc), C, st, tmX, tmW, a);
+  if (e != cudaSuccess) return e;
+  RouterTopkArgs ta;
+  ta.logits = logits;
+  ta.xsq = xsq;
+  ta.norms = norms;
+  ta.fps = fps;
+  ta.x = x;
+  ta.W_r = W_r;
+  ta.b_r = b_r;
+  ta.T = T;
+  ta.E = E;
+  ta.k = k;
+  ta.d = d;
+  ta.topk_idx = topk_idx;
+  ta.topk_w = topk_w;
+  return launch_kernel(router_topk_kernel, dim3((T + TK_WARPS - 1) / TK_WARPS),
+                       dim3(TK_WARPS * 32), 0, st, ta);
 }
 
 }  // namespace moe
