@@ -55,6 +55,7 @@ struct Layout {
   moe_ws_layout pub;
   size_t mprefix, chunk_hist, chunk_base, x_in, out_buf, gu_scales_t, d_scales_t;
   size_t router_terms;   // the router's bf16 weight terms and row norms
+  size_t inv;            // permuted row of each (token, slot) pair
   size_t mx_tok_rows;
   size_t x_norm;   // moe_forward_block: the normalised rows [T][d] bf16
 };
@@ -92,6 +93,7 @@ void make_layout(int E, int k, int T, int d, int I, bool hostio, Layout* L, bool
   L->chunk_hist = take(NB * E * 4);
   L->chunk_base = take(NB * E * 4);
   L->pub.perm = take(P * 4);
+  L->inv = take(P * 4);
   L->router_terms = take(moe::router_tc_scratch_bytes(E, d, T));
   const size_t tr = moe::mx_tok_rows(static_cast<int>(P), E);
   L->mx_tok_rows = tr;
@@ -261,7 +263,7 @@ moe_status launch_routing(const uint16_t* x, const float* W_r, const float* b_r,
                           int T, int d, float* logits, void* router_terms, int32_t* topk_idx,
                           float* topk_w, int32_t* counts, int32_t* offsets, int32_t* mprefix,
                           int32_t* chunk_hist, int32_t* chunk_base, int32_t* perm, int* status,
-                          cudaStream_t st, const StageEvents& ev) {
+                          cudaStream_t st, const StageEvents& ev, int32_t* inv = nullptr) {
   const bool small = T <= moe::kPermChunk;
   ev.mark(0);
   {
@@ -286,7 +288,7 @@ moe_status launch_routing(const uint16_t* x, const float* W_r, const float* b_r,
     MOE_CUDA(moe::launch_perm_scan(chunk_hist, moe::perm_chunks(T), E, counts, offsets, chunk_base,
                                    mprefix, st));
     ev.mark(4);
-    MOE_CUDA(moe::launch_perm_scatter(topk_idx, T, k, E, chunk_base, perm, nullptr, st));
+    MOE_CUDA(moe::launch_perm_scatter(topk_idx, T, k, E, chunk_base, perm, inv, st));
   }
   ev.mark(5);
   return MOE_OK;
@@ -369,7 +371,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
 
   moe_status rs = launch_routing(x, W_r, b_r, E, k, T, d, logits, at<void>(ws, L.router_terms),
                                  topk_idx, topk_w, counts, offsets, mprefix, chunk_hist,
-                                 chunk_base, perm, status, st, E_);
+                                 chunk_base, perm, status, st, E_, at<int32_t>(ws, L.inv));
   if (rs != MOE_OK) return rs;
   const int tiles = opt.act != moe::ACT_HILO
                         ? moe::TILES_MX
@@ -450,8 +452,12 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     // tiles, or 256-token tiles on a CTA pair
     const int variant = tiles == moe::TILES_MX_PAIR ? moe::kMxPair
                                                     : (P < 64 * E ? moe::kMxSmall : moe::kMxLarge);
+    // token-major when the three-launch permutation wrote the inverse (more
+    // than kPermChunk tokens), else row-major
+    const bool inv_ok = T > moe::kPermChunk;
     MOE_CUDA(moe::launch_mx_quant_gather(variant, x, perm, offsets, E, P, k, d, qx, qx + tr * d,
-                                         sfbx, st));
+                                         sfbx, inv_ok ? topk_idx : nullptr,
+                                         inv_ok ? at<int32_t>(ws, L.inv) : nullptr, T, st));
     E_.mark(6);
     E_.mark(7);
     E_.mark(8);

@@ -166,10 +166,13 @@ size_t mx_tok_rows(int P, int E);
 size_t mx_sfb_bytes(int P, int E, int K);
 
 // K2: gather x rows into the padded token layout as hi/lo E4M3 rows plus the
-// B-scale blocks the GEMM loads per (token tile, k-block).
+// B-scale blocks the GEMM loads per (token tile, k-block). With inv (pair id
+// -> permuted row) and topk_idx, token-major: each token's groups converted
+// once for its k rows (identical results).
 cudaError_t launch_mx_quant_gather(int variant, const uint16_t* x, const int32_t* perm,
                                    const int32_t* offsets, int E, int P, int k, int K, uint8_t* qhi,
-                                   uint8_t* qlo, uint8_t* sfb, cudaStream_t st);
+                                   uint8_t* qlo, uint8_t* sfb, const int32_t* topk_idx,
+                                   const int32_t* inv, int T, cudaStream_t st);
 // The same for the quantised activation modes (act ACT_E4M3 or ACT_E2M1): one
 // MX-converted row per routed pair (K bytes, or K/2 for E2M1) plus its
 // B-scale blocks.

@@ -265,6 +265,71 @@ __global__ void __launch_bounds__(256) mx_quant_gather_kernel(
   }
 }
 
+// The same rows, token-major: one thread per (token, group of 32) converts
+// the group once and writes it to each of the token's k permuted rows (inv:
+// pair id t*k + j -> permuted row), so the conversion work does not grow
+// with k. Results identical to mx_quant_gather_kernel.
+template <int NT>
+__global__ void __launch_bounds__(256) mx_quant_gather_tok_kernel(
+    const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_idx,
+    const int32_t* __restrict__ inv, const int32_t* __restrict__ offsets, int E, int T, int k,
+    int K, uint8_t* __restrict__ qhi, uint8_t* __restrict__ qlo, uint8_t* __restrict__ sfb) {
+  pdl_wait_and_trigger();
+  __shared__ int s_off[kMaxE + 1], s_tb[kMaxE + 1];
+  for (int i = threadIdx.x; i <= E; i += blockDim.x) s_off[i] = offsets[i];
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int a = 0;
+    for (int e = 0; e < E; ++e) {
+      s_tb[e] = a;
+      a += (s_off[e + 1] - s_off[e] + NT - 1) / NT;
+    }
+    s_tb[E] = a;
+  }
+  __syncthreads();
+  const int G = K / 32, KB = (K + 127) / 128;
+  constexpr int SFB = sfb_block_bytes(NT);
+  const int64_t n = static_cast<int64_t>(T) * G;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int t = static_cast<int>(i / G), g = static_cast<int>(i % G);
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * K + 32 * g);
+    float v[32];
+    float amax = 0.f;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const uint4 w = __ldg(src + c);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        v[8 * c + 2 * u] = bf16_bits_to_f32(ww[u] & 0xFFFFu);
+        v[8 * c + 2 * u + 1] = bf16_bits_to_f32(ww[u] >> 16);
+        amax = fmaxf(amax, fmaxf(fabsf(v[8 * c + 2 * u]), fabsf(v[8 * c + 2 * u + 1])));
+      }
+    }
+    uint32_t hw[8], lw[8];
+    const uint32_t sh = split_group32(v, amax, hw, lw);
+    const uint4 h0 = make_uint4(hw[0], hw[1], hw[2], hw[3]), h1 = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+    const uint4 l0 = make_uint4(lw[0], lw[1], lw[2], lw[3]), l1 = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+    int kb, kk;
+    group_to_kblock(g, G, KB, kb, kk);
+    for (int j = 0; j < k; ++j) {
+      const int q = t * k + j;
+      const int e = __ldg(topk_idx + q);
+      const int pr = s_tb[e] * NT + (__ldg(inv + q) - s_off[e]);
+      uint4* dh = reinterpret_cast<uint4*>(qhi + static_cast<size_t>(pr) * K + 32 * g);
+      uint4* dl = reinterpret_cast<uint4*>(qlo + static_cast<size_t>(pr) * K + 32 * g);
+      dh[0] = h0;
+      dh[1] = h1;
+      dl[0] = l0;
+      dl[1] = l1;
+      uint8_t* blk = sfb + (static_cast<size_t>(pr / NT) * KB + kb) * SFB;
+      blk[sfb_offset(NT, pr % NT, 0, kk)] = static_cast<uint8_t>(sh);
+      blk[sfb_offset(NT, pr % NT, 1, kk)] = static_cast<uint8_t>(sh - 4);
+    }
+  }
+}
+
 // Plain row split (no gather): rows [R][K] bf16 -> hi, lo [R][K] E4M3 and
 // scales [R][K/32][2] (hi byte, lo byte).
 __global__ void __launch_bounds__(256) mx_split_rows_kernel(const uint16_t* __restrict__ x, int R,
@@ -1144,7 +1209,21 @@ size_t mx_sfb_bytes(int P, int E, int K) {
 
 cudaError_t launch_mx_quant_gather(int variant, const uint16_t* x, const int32_t* perm,
                                    const int32_t* offsets, int E, int P, int k, int K, uint8_t* qhi,
-                                   uint8_t* qlo, uint8_t* sfb, cudaStream_t st) {
+                                   uint8_t* qlo, uint8_t* sfb, const int32_t* topk_idx,
+                                   const int32_t* inv, int T, cudaStream_t st) {
+  if (inv && topk_idx) {
+    const int grid = grid_for_n(static_cast<int64_t>(T) * (K / 32), 256, 148 * 8);
+    if (variant == kMxPair)
+      launch_kernel(mx_quant_gather_tok_kernel<kMxMaxNT>, dim3(grid), dim3(256), 0, st, x,
+                    topk_idx, inv, offsets, E, T, k, K, qhi, qlo, sfb);
+    else if (variant == kMxLarge)
+      launch_kernel(mx_quant_gather_tok_kernel<MxLarge::NT>, dim3(grid), dim3(256), 0, st, x,
+                    topk_idx, inv, offsets, E, T, k, K, qhi, qlo, sfb);
+    else
+      launch_kernel(mx_quant_gather_tok_kernel<MxSmall::NT>, dim3(grid), dim3(256), 0, st, x,
+                    topk_idx, inv, offsets, E, T, k, K, qhi, qlo, sfb);
+    return cudaGetLastError();
+  }
   const int64_t n = static_cast<int64_t>(P) * (K / 32);
   const int grid = grid_for_n(n, 256, 148 * 8);
   if (variant == kMxPair)
