@@ -17,7 +17,7 @@ CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libmoe_b200.so")
 SOURCES = ["moe_abi.cu", "moe_routing.cu", "moe_router_tc.cu", "moe_grouped_gemm.cu",
            "moe_mx_gemm.cu", "moe_mx_pair.cu", "moe_noalloc.cu"]
-HEADERS = ["moe_ptx.cuh", "moe_internal.h", "moe_topk.cuh"]
+HEADERS = ["moe_ptx.cuh", "moe_internal.h", "moe_topk.cuh", "moe_perm_small.cuh"]
 # the tensor-core rate probe: measurement tooling, a library of its own
 PROBE_LIB = os.path.join(PKG, "libmoe_b200_probe.so")
 PROBE_SOURCES = ["moe_probe.cu"]

@@ -267,11 +267,15 @@ moe_status launch_routing(const uint16_t* x, const float* W_r, const float* b_r,
   const bool small = T <= moe::kPermChunk;
   ev.mark(0);
   {
-    // tensor-core logits with the top-k and softmax in the same kernel (its
-    // stage time covers both; the top-k stage reads 0)
+    // the router: weight split, tensor-core logits, top-k and softmax (its
+    // stage time covers all three launches; the top-k stage reads 0); for
+    // at most kPermChunk tokens the top-k kernel's last block also builds the
+    // permutation
     moe::pdl_launches() = false;
     cudaError_t e = moe::launch_router_tc(x, W_r, b_r, T, E, k, d, router_terms, logits, topk_idx,
-                                          topk_w, status, st);
+                                          topk_w, status, st, small ? counts : nullptr,
+                                          small ? offsets : nullptr, small ? mprefix : nullptr,
+                                          small ? perm : nullptr);
     moe::pdl_launches() = true;
     MOE_CUDA(e);
     ev.mark(1);
@@ -279,7 +283,6 @@ moe_status launch_routing(const uint16_t* x, const float* W_r, const float* b_r,
   ev.mark(2);
   if (!perm) return MOE_OK;
   if (small) {
-    MOE_CUDA(moe::launch_perm_small(topk_idx, T, k, E, counts, offsets, mprefix, perm, st));
     ev.mark(3);
     ev.mark(4);
   } else {
@@ -602,8 +605,8 @@ moe_status moe_workspace_layout(int E, int k, int T, int d, int I, moe_ws_layout
 int moe_forward_launch_count(int E, int k, int T, int d, int I) {
   if (!full_shape_ok(E, k, T, d, I) || T == 0) return 0;
   int n = 12;
-  // small batches: the permutation in one launch instead of three
-  if (T <= moe::kPermChunk) n -= 2;
+  // small batches: the permutation inside the router's top-k launch
+  if (T <= moe::kPermChunk) n -= 3;
   // the block-scaled path launches no scale transposes
   const int tiles =
       choose_tiles(g_tile_policy.load(std::memory_order_relaxed), T * k, E, mx_shape_ok(d, I));

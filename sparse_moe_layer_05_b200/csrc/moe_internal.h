@@ -70,9 +70,13 @@ cudaError_t launch_perm_small(const int32_t* topk_idx, int T, int k, int E, int3
 // (written to `logits`, [T][E] fp32) and one the top-k with near ties settled
 // in fp64, and the softmax. Its first launch clears *status.
 size_t router_tc_scratch_bytes(int E, int d, int T);
+// With perm given and T <= kPermChunk, the top-k kernel's last block also
+// builds the permutation (counts may be null), as launch_perm_small would.
 cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b_r, int T, int E,
                              int k, int d, void* scratch, float* logits, int32_t* topk_idx,
-                             float* topk_w, int* status, cudaStream_t st);
+                             float* topk_w, int* status, cudaStream_t st,
+                             int32_t* counts = nullptr, int32_t* offsets = nullptr,
+                             int32_t* mtile_prefix = nullptr, int32_t* perm = nullptr);
 // K2: per-chunk expert histograms.
 cudaError_t launch_perm_hist(const int32_t* topk_idx, int T, int k, int E, int32_t* chunk_hist,
                              cudaStream_t st);

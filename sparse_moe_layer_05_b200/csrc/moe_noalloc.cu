@@ -112,17 +112,19 @@ moe_status moe_route_noalloc(const void* x_dev, const float* W_r_dev, const floa
   int32_t* chunk_hist = reinterpret_cast<int32_t*>(sb + L.chunk_hist);
   int32_t* chunk_base = reinterpret_cast<int32_t*>(sb + L.chunk_base);
   // Every buffer below is fully written before it is read; the status word
-  // is cleared by the first kernel. Batches of at most kPermChunk tokens take
-  // the fused permutation launch (identical results). The launches are the
-  // ones moe_route makes, in the same order and configuration.
+  // is cleared by the first kernel. Batches of at most kPermChunk tokens get
+  // their permutation from the router's top-k launch (identical results).
+  // The launches are the ones moe_route makes, in the same order and
+  // configuration.
   const uint16_t* x = static_cast<const uint16_t*>(x_dev);
   moe::pdl_launches() = false;
-  bool launched = moe::launch_router_tc(x, W_r_dev, b_r_dev, T, E, k, d, sb + L.router, logits,
-                                        topk_idx_dev, topk_w_dev, status, st) == cudaSuccess;
-  if (launched && T <= moe::kPermChunk) {
-    launched = moe::launch_perm_small(topk_idx_dev, T, k, E, counts_dev, offsets_dev, mprefix,
-                                      perm_dev, st) == cudaSuccess;
-  } else if (launched) {
+  const bool small = T <= moe::kPermChunk;
+  bool launched =
+      moe::launch_router_tc(x, W_r_dev, b_r_dev, T, E, k, d, sb + L.router, logits, topk_idx_dev,
+                            topk_w_dev, status, st, small ? counts_dev : nullptr,
+                            small ? offsets_dev : nullptr, small ? mprefix : nullptr,
+                            small ? perm_dev : nullptr) == cudaSuccess;
+  if (launched && !small) {
     launched =
         moe::launch_perm_hist(topk_idx_dev, T, k, E, chunk_hist, st) == cudaSuccess &&
         moe::launch_perm_scan(chunk_hist, moe::perm_chunks(T), E, counts_dev, offsets_dev,

@@ -56,6 +56,7 @@
 
 #include "moe_internal.h"
 #include "moe_ptx.cuh"
+#include "moe_perm_small.cuh"
 #include "moe_topk.cuh"
 
 namespace moe {
@@ -129,10 +130,14 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
                                                            uint16_t* __restrict__ terms,
                                                            float* __restrict__ norms,
                                                            unsigned long long* __restrict__ fps,
-                                                           int* status) {
+                                                           int* status, int* done_blocks) {
   pdl_wait_and_trigger();
-  // the first kernel of the pass clears the status word
-  if (status && blockIdx.x == 0 && threadIdx.x == 0) *status = 0;
+  // the first kernel of the pass clears the status word and the top-k
+  // kernel's count of finished blocks
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (status) *status = 0;
+    *done_blocks = 0;
+  }
   const int row = blockIdx.x;
   const size_t n = static_cast<size_t>(npad) * d;
   const size_t base = static_cast<size_t>(row) * d;
@@ -482,6 +487,10 @@ struct RouterTopkArgs {
   int T, E, k, d;
   int32_t* topk_idx;
   float* topk_w;
+  // T <= kPermChunk with the permutation requested: the last block to finish
+  // builds it (counts may be null)
+  int32_t *counts, *offsets, *mtile_prefix, *perm;
+  int* done_blocks;
 };
 
 // One warp per token: top-k of its fp32 logits, near ties settled in fp64
@@ -489,6 +498,8 @@ struct RouterTopkArgs {
 __global__ void __launch_bounds__(TK_WARPS * 32) router_topk_kernel(const RouterTopkArgs args) {
   pdl_wait_and_trigger();
   __shared__ RefineReq reqs[TK_WARPS];
+  __shared__ PermSmallSmem perm_sm;
+  __shared__ int last_block;
   __shared__ uint32_t jobs[TK_WARPS * RJ_PER_WARP];
   __shared__ int q_njob[TK_WARPS];
   __shared__ double red[4 * TK_WARPS];
@@ -621,6 +632,20 @@ __global__ void __launch_bounds__(TK_WARPS * 32) router_topk_kernel(const Router
     topk_emit(L, val, args.k, lane, args.topk_idx + static_cast<size_t>(t) * args.k,
               args.topk_w + static_cast<size_t>(t) * args.k);
   }
+  if (args.perm) {
+    // the last block to finish sees every block's top-k (each block's stores,
+    // then a device-scope fence, then its count) and builds the permutation
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0)
+      last_block = atomicAdd(args.done_blocks, 1) == static_cast<int>(gridDim.x) - 1;
+    __syncthreads();
+    if (last_block) {
+      __threadfence();
+      perm_small_block(args.topk_idx, args.T, args.k, args.E, args.counts, args.offsets,
+                       args.mtile_prefix, args.perm, perm_sm);
+    }
+  }
 }
 
 // Clusters of C CTAs of router_tc_kernel (the largest shared-memory shape)
@@ -680,12 +705,14 @@ int cluster_size(int T, int d, int dev, size_t smem) {
 
 size_t router_tc_scratch_bytes(int E, int d, int T) {
   const size_t npad = static_cast<size_t>((E + 15) / 16 * 16);
-  return 3 * npad * static_cast<size_t>(d) * 2 + npad * 4 + npad * 8 + static_cast<size_t>(T) * 4;
+  return 3 * npad * static_cast<size_t>(d) * 2 + npad * 4 + npad * 8 + static_cast<size_t>(T) * 4 +
+         16;
 }
 
 cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b_r, int T, int E,
                              int k, int d, void* scratch, float* logits, int32_t* topk_idx,
-                             float* topk_w, int* status, cudaStream_t st) {
+                             float* topk_w, int* status, cudaStream_t st, int32_t* counts,
+                             int32_t* offsets, int32_t* mtile_prefix, int32_t* perm) {
   if (E < 1 || E > 256 || k < 1 || k > E || k > 32 || d % 32 != 0 || T < 1)
     return cudaErrorInvalidValue;
   const RouterTcShape sh = router_tc_shape(E);
@@ -707,10 +734,11 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b
                                           3 * static_cast<size_t>(sh.npad) * d * 2);
   unsigned long long* fps = reinterpret_cast<unsigned long long*>(norms + sh.npad);
   float* xsq = reinterpret_cast<float*>(fps + sh.npad);
+  int* done_blocks = reinterpret_cast<int*>(xsq + T);
   // the weight split: the first launch of the pass (it clears the status word)
   {
     cudaError_t e = launch_kernel(router_split_kernel, dim3(sh.npad), dim3(256), 0, st, W_r, b_r,
-                                  E, sh.npad, d, terms, norms, fps, status);
+                                  E, sh.npad, d, terms, norms, fps, status, done_blocks);
     if (e != cudaSuccess) return e;
     pdl_launches() = true;   // the router kernel may overlap the split's tail
   }
@@ -771,6 +799,12 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b
   ta.d = d;
   ta.topk_idx = topk_idx;
   ta.topk_w = topk_w;
+  const bool fuse_perm = perm && T <= kPermChunk;
+  ta.counts = fuse_perm ? counts : nullptr;
+  ta.offsets = fuse_perm ? offsets : nullptr;
+  ta.mtile_prefix = fuse_perm ? mtile_prefix : nullptr;
+  ta.perm = fuse_perm ? perm : nullptr;
+  ta.done_blocks = done_blocks;
   return launch_kernel(router_topk_kernel, dim3((T + TK_WARPS - 1) / TK_WARPS),
                        dim3(TK_WARPS * 32), 0, st, ta);
 }

@@ -9,6 +9,7 @@
 #include <stdint.h>
 
 #include "moe_internal.h"
+#include "moe_perm_small.cuh"
 #include "moe_ptx.cuh"
 
 namespace moe {
@@ -125,8 +126,7 @@ __global__ void __launch_bounds__(256) perm_scatter_kernel(const int32_t* __rest
 
 // ------------------------------------------------------ K2, small batches ----
 // For T <= kPermChunk (one chunk): histogram, scan and stable scatter in one
-// block, with the per-warp segments and ranks of perm_scatter_kernel; writes
-// counts, offsets, the M-tile prefix and perm exactly as the three kernels do.
+// block (moe_perm_small.cuh).
 __global__ void __launch_bounds__(256) perm_small_kernel(const int32_t* __restrict__ topk_idx,
                                                          int T, int k, int E,
                                                          int32_t* __restrict__ counts,
@@ -134,63 +134,8 @@ __global__ void __launch_bounds__(256) perm_small_kernel(const int32_t* __restri
                                                          int32_t* __restrict__ mtile_prefix,
                                                          int32_t* __restrict__ perm) {
   pdl_wait_and_trigger();
-  __shared__ int wbase[8][256];
-  __shared__ int s_cnt[256], s_mt[256];
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < 8 * 256; i += blockDim.x) (&wbase[0][0])[i] = 0;
-  __syncthreads();
-  const int64_t qc1 = (int64_t)min(T, kPermChunk) * k;
-  const int64_t seg = (int64_t)(kPermChunk / 8) * k;
-  const int64_t q0 = warp * seg;
-  const int64_t q1 = min(qc1, q0 + seg);
-  for (int64_t q = q0 + lane; q < q1; q += 32) atomicAdd(&wbase[warp][topk_idx[q]], 1);
-  __syncthreads();
-  const int e = threadIdx.x;
-  int total = 0;
-  if (e < E)
-    for (int w = 0; w < 8; ++w) total += wbase[w][e];
-  s_cnt[e] = (e < E) ? total : 0;
-  s_mt[e] = (e < E) ? (total + kTileM - 1) / kTileM : 0;
-  __syncthreads();
-  if (e == 0) {  // E <= 256: a serial scan is cheap and plainly ordered
-    int a = 0, m = 0;
-    for (int i = 0; i < E; ++i) {
-      const int c = s_cnt[i], mt = s_mt[i];
-      s_cnt[i] = a;
-      s_mt[i] = m;
-      a += c;
-      m += mt;
-    }
-    offsets[E] = a;
-    mtile_prefix[E] = m;
-  }
-  __syncthreads();
-  if (e < E) {
-    offsets[e] = s_cnt[e];
-    mtile_prefix[e] = s_mt[e];
-    if (counts) counts[e] = total;
-    int run = s_cnt[e];
-    for (int w = 0; w < 8; ++w) {
-      const int c = wbase[w][e];
-      wbase[w][e] = run;
-      run += c;
-    }
-  }
-  __syncthreads();
-  const uint32_t lt = (1u << lane) - 1u;
-  for (int64_t qb = q0; qb < q1; qb += 32) {
-    const int64_t q = qb + lane;
-    const bool valid = q < q1;
-    const int ex = valid ? topk_idx[q] : -1 - lane;
-    const uint32_t m = __match_any_sync(0xFFFFFFFFu, ex);
-    const int rank = __popc(m & lt);
-    int pos = 0;
-    if (valid) pos = wbase[warp][ex] + rank;
-    __syncwarp();
-    if (valid && lane == __ffs(m) - 1) wbase[warp][ex] += __popc(m);
-    __syncwarp();
-    if (valid) perm[pos] = (int32_t)q;
-  }
+  __shared__ PermSmallSmem sm;
+  perm_small_block(topk_idx, T, k, E, counts, offsets, mtile_prefix, perm, sm);
 }
 
 // ----------------------------------------------------------- K2 gather ----

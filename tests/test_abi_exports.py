@@ -125,16 +125,16 @@ def test_workspace_sizes():
     offs = sorted((v, k) for k, v in L.items() if k != "total")
     assert all(v % 256 == 0 for v, _ in offs)
     assert L["status"] == 0 and L["total"] >= L["yw"] + 400 * 2880 * 2
-    # batches of <= 256 tokens fuse the three permutation kernels (-2); the
-    # block-scaled paths (decode shapes, and prefill shapes on the CTA pair)
-    # launch no scale transposes (-2); the bf16 tiles do
+    # the block-scaled paths (decode shapes, and prefill shapes on the CTA
+    # pair) launch no scale transposes (-2); the bf16 tiles do
     # 12 launches: the router's three (weight split, logits, top-k), three
-    # for the permutation (one for at most 256 tokens), the gather, two
-    # scale transposes (none on the block-scaled tiles), two GEMMs, combine
+    # for the permutation (none of its own for at most 256 tokens: the top-k
+    # launch builds it), the gather, two scale transposes (none on the
+    # block-scaled tiles), two GEMMs, combine
     assert B.moe_forward_launch_count(32, 4, 8192, 2880, 2880) == 10
     assert B.moe_forward_launch_count(32, 4, 8192, 352, 224) == 12
-    assert B.moe_forward_launch_count(32, 4, 100, 2880, 2880) == 8
-    assert B.moe_forward_launch_count(32, 4, 100, 352, 2880) == 10
+    assert B.moe_forward_launch_count(32, 4, 100, 2880, 2880) == 7
+    assert B.moe_forward_launch_count(32, 4, 100, 352, 2880) == 9
     assert B.moe_forward_launch_count(128, 4, 300, 2880, 2880) == 10
     assert B.moe_forward_launch_count(32, 4, 0, 2880, 2880) == 0
 
