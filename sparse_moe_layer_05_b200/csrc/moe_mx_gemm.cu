@@ -543,6 +543,12 @@ struct MxArgs {
   const float* topk_w;
   int* status;
   const float* bias;        // [E][2I] (SwiGLU) or [E][d] (down), or nullptr
+  // combine in the down epilogue (16-token tiles; MxGemmProblem)
+  uint16_t* out_bf16;
+  const uint16_t* resid;
+  int* tok_cnt;
+  int tok_cnt_n;
+  int k;
 };
 
 __device__ __forceinline__ float silu_mx(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
@@ -577,6 +583,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
 
   const int E = args.E;
   for (int i = threadIdx.x; i <= E; i += C::NUM_THREADS) s_off[i] = args.offsets[i];
+  if (EPI == EPI_SWIGLU && args.tok_cnt)   // for the down launch's combine
+    for (int i = blockIdx.x * C::NUM_THREADS + threadIdx.x; i < args.tok_cnt_n;
+         i += gridDim.x * C::NUM_THREADS)
+      args.tok_cnt[i] = 0;
   __syncthreads();
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -822,7 +832,10 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
       const uint32_t ap = (it >> 1) & 1;
       if (ok) ok = mbar_wait(bar_accFull(ab), ap, abort_flag, args.status);
       ok = __all_sync(0xFFFFFFFFu, ok);        // the TMEM loads below are warp-collective
-      if (!ok && EPI != EPI_SWIGLU) break;
+      // the fused combine's barriers, like the SwiGLU exchange, are passed by
+      // every epilogue warp in every tile, also after a failed wait
+      const bool fused_combine = EPI == EPI_DOWN && NT <= 16 && args.out_bf16 != nullptr;
+      if (!ok && EPI != EPI_SWIGLU && !fused_combine) break;
       if (ok) tc_fence_after();
       // with two issuers and a single k-block per tile only issuer
       // (it*KB) % 2 wrote its buffer
@@ -971,6 +984,40 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
             }
           }
         }
+      }
+      if (fused_combine) {
+        // combine: the tile whose rows complete a token's k rows of this
+        // 128-column block sums them in slot order, adds the residual and
+        // rounds once to bf16 (as combine_kernel does)
+        int* s_last = reinterpret_cast<int*>(s_xch);
+        __threadfence();
+        asm volatile("bar.sync 7, 128;" ::: "memory");
+        if (m < NT) {
+          int last = -1;
+          if (ok && m < rows) {
+            const int tok = args.perm[s_off[e] + tb * NT + m] / args.k;
+            const int old = atomicAdd(args.tok_cnt + static_cast<size_t>(tok) * args.n_wb + wb, 1);
+            if (old == args.k - 1) last = tok;
+          }
+          s_last[m] = last;
+        }
+        asm volatile("bar.sync 7, 128;" ::: "memory");
+        __threadfence();
+        if (ok && col < args.n_out) {
+          for (int i = 0; i < rows; ++i) {
+            const int tok = s_last[i];
+            if (tok < 0) continue;
+            float acc = 0.f;
+            for (int jj = 0; jj < args.k; ++jj)
+              acc += __ldcg(args.out_f32 + (static_cast<size_t>(tok) * args.k + jj) * args.n_out + col);
+            if (args.resid)
+              acc += __uint_as_float(
+                  static_cast<uint32_t>(args.resid[static_cast<size_t>(tok) * args.n_out + col]) << 16);
+            args.out_bf16[static_cast<size_t>(tok) * args.n_out + col] =
+                __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+          }
+        }
+        asm volatile("bar.sync 7, 128;" ::: "memory");
       }
       if (ok) {
         tc_fence_before();
@@ -1136,6 +1183,11 @@ cudaError_t launch_mx_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st)
   a.topk_w = p.topk_w;
   a.bias = p.bias;
   a.status = p.status;
+  a.out_bf16 = C::NT <= 16 ? p.out_bf16 : nullptr;
+  a.resid = p.resid;
+  a.tok_cnt = p.tok_cnt;
+  a.tok_cnt_n = p.tok_cnt_n;
+  a.k = p.k;
   if (EPI == EPI_SWIGLU) {
     a.n_wb = (p.I + 63) / 64;
     a.rows_per_expert = 2 * p.I;
