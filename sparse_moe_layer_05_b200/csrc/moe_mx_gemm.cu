@@ -265,10 +265,13 @@ __global__ void __launch_bounds__(256) mx_quant_gather_kernel(
   }
 }
 
-// The same rows, token-major: one thread per (token, group of 32) converts
-// the group once and writes it to each of the token's k permuted rows (inv:
-// pair id t*k + j -> permuted row), so the conversion work does not grow
-// with k. Results identical to mx_quant_gather_kernel.
+// The same rows, token-major: one thread per (token, 128-wide k-block)
+// converts the k-block's (up to) four groups once and writes them to each of
+// the token's k permuted rows (inv: pair id t*k + j -> permuted row), with
+// the four scale bytes of a row's k-block as one 32-bit word per term. The
+// conversion work does not grow with k and the scale stores are words, not
+// bytes. Results identical to mx_quant_gather_kernel (the tail k-block's
+// unused scale bytes 0 and 1 are written as zero).
 template <int NT>
 __global__ void __launch_bounds__(256) mx_quant_gather_tok_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_idx,
@@ -288,44 +291,64 @@ __global__ void __launch_bounds__(256) mx_quant_gather_tok_kernel(
   }
   __syncthreads();
   const int G = K / 32, KB = (K + 127) / 128;
+  const bool tail = (G % 4) != 0;
   constexpr int SFB = sfb_block_bytes(NT);
-  const int64_t n = static_cast<int64_t>(T) * G;
+  const int64_t n = static_cast<int64_t>(T) * KB;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int t = static_cast<int>(i / G), g = static_cast<int>(i % G);
-    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * K + 32 * g);
-    float v[32];
-    float amax = 0.f;
+    const int t = static_cast<int>(i / KB), kb = static_cast<int>(i % KB);
+    const int g0 = 4 * kb;
+    const int ng = min(4, G - g0);
+    // a tail k-block holds groups G-2, G-1 at scale positions 2 and 3
+    const int kk0 = (tail && kb == KB - 1) ? 4 - ng : 0;
+    uint4 h4[4][2], l4[4][2];
+    uint32_t shw = 0, slw = 0;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-      const uint4 w = __ldg(src + c);
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+    for (int q = 0; q < 4; ++q) {
+      if (q < ng) {
+        const uint4* src =
+            reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * K + 32 * (g0 + q));
+        float v[32];
+        float amax = 0.f;
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        v[8 * c + 2 * u] = bf16_bits_to_f32(ww[u] & 0xFFFFu);
-        v[8 * c + 2 * u + 1] = bf16_bits_to_f32(ww[u] >> 16);
-        amax = fmaxf(amax, fmaxf(fabsf(v[8 * c + 2 * u]), fabsf(v[8 * c + 2 * u + 1])));
+        for (int c = 0; c < 4; ++c) {
+          const uint4 w = __ldg(src + c);
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            v[8 * c + 2 * u] = bf16_bits_to_f32(ww[u] & 0xFFFFu);
+            v[8 * c + 2 * u + 1] = bf16_bits_to_f32(ww[u] >> 16);
+            amax = fmaxf(amax, fmaxf(fabsf(v[8 * c + 2 * u]), fabsf(v[8 * c + 2 * u + 1])));
+          }
+        }
+        uint32_t hw[8], lw[8];
+        const uint32_t sh = split_group32(v, amax, hw, lw);
+        h4[q][0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        h4[q][1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+        l4[q][0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        l4[q][1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+        shw |= (sh & 0xFFu) << (8 * (kk0 + q));
+        slw |= ((sh - 4) & 0xFFu) << (8 * (kk0 + q));
       }
     }
-    uint32_t hw[8], lw[8];
-    const uint32_t sh = split_group32(v, amax, hw, lw);
-    const uint4 h0 = make_uint4(hw[0], hw[1], hw[2], hw[3]), h1 = make_uint4(hw[4], hw[5], hw[6], hw[7]);
-    const uint4 l0 = make_uint4(lw[0], lw[1], lw[2], lw[3]), l1 = make_uint4(lw[4], lw[5], lw[6], lw[7]);
-    int kb, kk;
-    group_to_kblock(g, G, KB, kb, kk);
     for (int j = 0; j < k; ++j) {
-      const int q = t * k + j;
-      const int e = __ldg(topk_idx + q);
-      const int pr = s_tb[e] * NT + (__ldg(inv + q) - s_off[e]);
-      uint4* dh = reinterpret_cast<uint4*>(qhi + static_cast<size_t>(pr) * K + 32 * g);
-      uint4* dl = reinterpret_cast<uint4*>(qlo + static_cast<size_t>(pr) * K + 32 * g);
-      dh[0] = h0;
-      dh[1] = h1;
-      dl[0] = l0;
-      dl[1] = l1;
+      const int qp = t * k + j;
+      const int e = __ldg(topk_idx + qp);
+      const int pr = s_tb[e] * NT + (__ldg(inv + qp) - s_off[e]);
+      uint4* dh = reinterpret_cast<uint4*>(qhi + static_cast<size_t>(pr) * K + 32 * g0);
+      uint4* dl = reinterpret_cast<uint4*>(qlo + static_cast<size_t>(pr) * K + 32 * g0);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        if (q < ng) {
+          dh[2 * q] = h4[q][0];
+          dh[2 * q + 1] = h4[q][1];
+          dl[2 * q] = l4[q][0];
+          dl[2 * q + 1] = l4[q][1];
+        }
+      }
       uint8_t* blk = sfb + (static_cast<size_t>(pr / NT) * KB + kb) * SFB;
-      blk[sfb_offset(NT, pr % NT, 0, kk)] = static_cast<uint8_t>(sh);
-      blk[sfb_offset(NT, pr % NT, 1, kk)] = static_cast<uint8_t>(sh - 4);
+      *reinterpret_cast<uint32_t*>(blk + sfb_offset(NT, pr % NT, 0, 0)) = shw;
+      *reinterpret_cast<uint32_t*>(blk + sfb_offset(NT, pr % NT, 1, 0)) = slw;
     }
   }
 }
@@ -985,8 +1008,13 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
           }
         }
       }
+      if (ok) {
+        tc_fence_before();
+        mbar_arrive(bar_accEmpty(ab));     // this tile's accumulators are read
+      }
       if (fused_combine) {
-        // combine: the tile whose rows complete a token's k rows of this
+        // combine (after the accumulator buffer is released, so the next
+        // tile's UMMAs run meanwhile): the tile whose rows complete a token's k rows of this
         // 128-column block sums them in slot order, adds the residual and
         // rounds once to bf16 (as combine_kernel does)
         int* s_last = reinterpret_cast<int*>(s_xch);
@@ -1018,10 +1046,6 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
           }
         }
         asm volatile("bar.sync 7, 128;" ::: "memory");
-      }
-      if (ok) {
-        tc_fence_before();
-        mbar_arrive(bar_accEmpty(ab));     // this tile's accumulators are read
       }
     }
   }
@@ -1264,7 +1288,7 @@ cudaError_t launch_mx_quant_gather(int variant, const uint16_t* x, const int32_t
                                    uint8_t* qlo, uint8_t* sfb, const int32_t* topk_idx,
                                    const int32_t* inv, int T, cudaStream_t st) {
   if (inv && topk_idx) {
-    const int grid = grid_for_n(static_cast<int64_t>(T) * (K / 32), 256, 148 * 8);
+    const int grid = grid_for_n(static_cast<int64_t>(T) * ((K + 127) / 128), 256, 148 * 8);
     if (variant == kMxPair)
       launch_kernel(mx_quant_gather_tok_kernel<kMxMaxNT>, dim3(grid), dim3(256), 0, st, x,
                     topk_idx, inv, offsets, E, T, k, K, qhi, qlo, sfb);
