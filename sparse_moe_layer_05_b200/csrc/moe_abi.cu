@@ -56,7 +56,6 @@ struct Layout {
   size_t mprefix, chunk_hist, chunk_base, x_in, out_buf, gu_scales_t, d_scales_t;
   size_t router_terms;   // the router's bf16 weight terms and row norms
   size_t inv;            // permuted row of each (token, slot) pair
-  size_t tok_cnt;        // per (token, 128-column block) arrival counts of the fused combine
   size_t mx_tok_rows;
   size_t x_norm;   // moe_forward_block: the normalised rows [T][d] bf16
 };
@@ -95,7 +94,6 @@ void make_layout(int E, int k, int T, int d, int I, bool hostio, Layout* L, bool
   L->chunk_base = take(NB * E * 4);
   L->pub.perm = take(P * 4);
   L->inv = take(P * 4);
-  L->tok_cnt = take(static_cast<size_t>(T) * ((d + 127) / 128) * 4);
   L->router_terms = take(moe::router_tc_scratch_bytes(E, d, T));
   const size_t tr = moe::mx_tok_rows(static_cast<int>(P), E);
   L->mx_tok_rows = tr;
@@ -423,12 +421,6 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     m1.status = status;
     m1.bias = gu_bias;
     m1.act = act;
-    // 16-token tiles: the combine runs in the down GEMM's epilogue
-    const bool fuse = variant == moe::kMxSmall;
-    if (fuse) {
-      m1.tok_cnt = at<int>(ws, L.tok_cnt);
-      m1.tok_cnt_n = T * ((d + 127) / 128);
-    }
     MOE_CUDA(variant == moe::kMxPair ? moe::launch_mx_pair_gateup_swiglu(m1, num_sms, st)
                                      : moe::launch_mx_gemm_gateup_swiglu(variant, m1, num_sms, st));
     E_.mark(9);
@@ -445,15 +437,10 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     m2.topk_w = topk_w;
     m2.n_out = d;
     m2.bias = dn_bias;
-    if (fuse) {
-      m2.out_bf16 = static_cast<uint16_t*>(out);
-      m2.resid = resid;
-      m2.k = k;
-    }
     MOE_CUDA(variant == moe::kMxPair ? moe::launch_mx_pair_down(m2, num_sms, st)
                                      : moe::launch_mx_gemm_down(variant, m2, num_sms, st));
     E_.mark(10);
-    if (!fuse) MOE_CUDA(moe::launch_combine(yw, T, k, d, resid, out, st));
+    MOE_CUDA(moe::launch_combine(yw, T, k, d, resid, out, st));
     E_.mark(11);
     return MOE_OK;
   }
@@ -496,12 +483,6 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     m1.n_out = I;
     m1.status = status;
     m1.bias = gu_bias;
-    // 16-token tiles: the combine runs in the down GEMM's epilogue
-    const bool fuse = variant == moe::kMxSmall;
-    if (fuse) {
-      m1.tok_cnt = at<int>(ws, L.tok_cnt);
-      m1.tok_cnt_n = T * ((d + 127) / 128);
-    }
     MOE_CUDA(variant == moe::kMxPair ? moe::launch_mx_pair_gateup_swiglu(m1, num_sms, st)
                                      : moe::launch_mx_gemm_gateup_swiglu(variant, m1, num_sms, st));
     E_.mark(9);
@@ -520,15 +501,10 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     m2.topk_w = topk_w;
     m2.n_out = d;
     m2.bias = dn_bias;
-    if (fuse) {
-      m2.out_bf16 = static_cast<uint16_t*>(out);
-      m2.resid = resid;
-      m2.k = k;
-    }
     MOE_CUDA(variant == moe::kMxPair ? moe::launch_mx_pair_down(m2, num_sms, st)
                                      : moe::launch_mx_gemm_down(variant, m2, num_sms, st));
     E_.mark(10);
-    if (!fuse) MOE_CUDA(moe::launch_combine(yw, T, k, d, resid, out, st));
+    MOE_CUDA(moe::launch_combine(yw, T, k, d, resid, out, st));
     E_.mark(11);
     return MOE_OK;
   }
@@ -635,8 +611,6 @@ int moe_forward_launch_count(int E, int k, int T, int d, int I) {
   const int tiles =
       choose_tiles(g_tile_policy.load(std::memory_order_relaxed), T * k, E, mx_shape_ok(d, I));
   if (tiles == moe::TILES_MX || tiles == moe::TILES_MX_PAIR) n -= 2;
-  // 16-token block-scaled tiles: the combine inside the down GEMM
-  if (tiles == moe::TILES_MX && T * k < 64 * E) n -= 1;
   return n;
 }
 

@@ -212,16 +212,6 @@ struct MxGemmProblem {
   int* status;
   const float* bias;        // optional, as in GroupedGemmProblem
   int act;                  // ACT_HILO, ACT_E4M3 or ACT_E2M1 (b_lo / h_lo unused but HILO)
-  // Combine in the down GEMM's epilogue (16-token tiles only): with out_bf16
-  // set, the tile that completes a token's k rows of a 128-column block sums
-  // them in slot order (+ resid) into out_bf16, using tok_cnt [T][ceil(d/128)]
-  // arrival counts; the gate/up launch of the same pass zeroes tok_cnt
-  // (tok_cnt_n ints) before the down launch runs.
-  uint16_t* out_bf16;
-  const uint16_t* resid;
-  int* tok_cnt;
-  int tok_cnt_n;
-  int k;
 };
 cudaError_t launch_mx_gemm_gateup_swiglu(int variant, const MxGemmProblem& p, int num_sms,
                                          cudaStream_t st);

@@ -265,13 +265,10 @@ __global__ void __launch_bounds__(256) mx_quant_gather_kernel(
   }
 }
 
-// The same rows, token-major: one thread per (token, 128-wide k-block)
-// converts the k-block's (up to) four groups once and writes them to each of
-// the token's k permuted rows (inv: pair id t*k + j -> permuted row), with
-// the four scale bytes of a row's k-block as one 32-bit word per term. The
-// conversion work does not grow with k and the scale stores are words, not
-// bytes. Results identical to mx_quant_gather_kernel (the tail k-block's
-// unused scale bytes 0 and 1 are written as zero).
+// The same rows, token-major: one thread per (token, group of 32) converts
+// the group once and writes it to each of the token's k permuted rows (inv:
+// pair id t*k + j -> permuted row), so the conversion work does not grow
+// with k. Results identical to mx_quant_gather_kernel.
 template <int NT>
 __global__ void __launch_bounds__(256) mx_quant_gather_tok_kernel(
     const uint16_t* __restrict__ x, const int32_t* __restrict__ topk_idx,
@@ -291,64 +288,44 @@ __global__ void __launch_bounds__(256) mx_quant_gather_tok_kernel(
   }
   __syncthreads();
   const int G = K / 32, KB = (K + 127) / 128;
-  const bool tail = (G % 4) != 0;
   constexpr int SFB = sfb_block_bytes(NT);
-  const int64_t n = static_cast<int64_t>(T) * KB;
+  const int64_t n = static_cast<int64_t>(T) * G;
   for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
        i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int t = static_cast<int>(i / KB), kb = static_cast<int>(i % KB);
-    const int g0 = 4 * kb;
-    const int ng = min(4, G - g0);
-    // a tail k-block holds groups G-2, G-1 at scale positions 2 and 3
-    const int kk0 = (tail && kb == KB - 1) ? 4 - ng : 0;
-    uint4 h4[4][2], l4[4][2];
-    uint32_t shw = 0, slw = 0;
+    const int t = static_cast<int>(i / G), g = static_cast<int>(i % G);
+    const uint4* src = reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * K + 32 * g);
+    float v[32];
+    float amax = 0.f;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      if (q < ng) {
-        const uint4* src =
-            reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * K + 32 * (g0 + q));
-        float v[32];
-        float amax = 0.f;
+    for (int c = 0; c < 4; ++c) {
+      const uint4 w = __ldg(src + c);
+      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const uint4 w = __ldg(src + c);
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            v[8 * c + 2 * u] = bf16_bits_to_f32(ww[u] & 0xFFFFu);
-            v[8 * c + 2 * u + 1] = bf16_bits_to_f32(ww[u] >> 16);
-            amax = fmaxf(amax, fmaxf(fabsf(v[8 * c + 2 * u]), fabsf(v[8 * c + 2 * u + 1])));
-          }
-        }
-        uint32_t hw[8], lw[8];
-        const uint32_t sh = split_group32(v, amax, hw, lw);
-        h4[q][0] = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        h4[q][1] = make_uint4(hw[4], hw[5], hw[6], hw[7]);
-        l4[q][0] = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-        l4[q][1] = make_uint4(lw[4], lw[5], lw[6], lw[7]);
-        shw |= (sh & 0xFFu) << (8 * (kk0 + q));
-        slw |= ((sh - 4) & 0xFFu) << (8 * (kk0 + q));
+      for (int u = 0; u < 4; ++u) {
+        v[8 * c + 2 * u] = bf16_bits_to_f32(ww[u] & 0xFFFFu);
+        v[8 * c + 2 * u + 1] = bf16_bits_to_f32(ww[u] >> 16);
+        amax = fmaxf(amax, fmaxf(fabsf(v[8 * c + 2 * u]), fabsf(v[8 * c + 2 * u + 1])));
       }
     }
+    uint32_t hw[8], lw[8];
+    const uint32_t sh = split_group32(v, amax, hw, lw);
+    const uint4 h0 = make_uint4(hw[0], hw[1], hw[2], hw[3]), h1 = make_uint4(hw[4], hw[5], hw[6], hw[7]);
+    const uint4 l0 = make_uint4(lw[0], lw[1], lw[2], lw[3]), l1 = make_uint4(lw[4], lw[5], lw[6], lw[7]);
+    int kb, kk;
+    group_to_kblock(g, G, KB, kb, kk);
     for (int j = 0; j < k; ++j) {
-      const int qp = t * k + j;
-      const int e = __ldg(topk_idx + qp);
-      const int pr = s_tb[e] * NT + (__ldg(inv + qp) - s_off[e]);
-      uint4* dh = reinterpret_cast<uint4*>(qhi + static_cast<size_t>(pr) * K + 32 * g0);
-      uint4* dl = reinterpret_cast<uint4*>(qlo + static_cast<size_t>(pr) * K + 32 * g0);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        if (q < ng) {
-          dh[2 * q] = h4[q][0];
-          dh[2 * q + 1] = h4[q][1];
-          dl[2 * q] = l4[q][0];
-          dl[2 * q + 1] = l4[q][1];
-        }
-      }
+      const int q = t * k + j;
+      const int e = __ldg(topk_idx + q);
+      const int pr = s_tb[e] * NT + (__ldg(inv + q) - s_off[e]);
+      uint4* dh = reinterpret_cast<uint4*>(qhi + static_cast<size_t>(pr) * K + 32 * g);
+      uint4* dl = reinterpret_cast<uint4*>(qlo + static_cast<size_t>(pr) * K + 32 * g);
+      dh[0] = h0;
+      dh[1] = h1;
+      dl[0] = l0;
+      dl[1] = l1;
       uint8_t* blk = sfb + (static_cast<size_t>(pr / NT) * KB + kb) * SFB;
-      *reinterpret_cast<uint32_t*>(blk + sfb_offset(NT, pr % NT, 0, 0)) = shw;
-      *reinterpret_cast<uint32_t*>(blk + sfb_offset(NT, pr % NT, 1, 0)) = slw;
+      blk[sfb_offset(NT, pr % NT, 0, kk)] = static_cast<uint8_t>(sh);
+      blk[sfb_offset(NT, pr % NT, 1, kk)] = static_cast<uint8_t>(sh - 4);
     }
   }
 }
@@ -566,12 +543,6 @@ struct MxArgs {
   const float* topk_w;
   int* status;
   const float* bias;        // [E][2I] (SwiGLU) or [E][d] (down), or nullptr
-  // combine in the down epilogue (16-token tiles; MxGemmProblem)
-  uint16_t* out_bf16;
-  const uint16_t* resid;
-  int* tok_cnt;
-  int tok_cnt_n;
-  int k;
 };
 
 __device__ __forceinline__ float silu_mx(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
@@ -606,10 +577,6 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
 
   const int E = args.E;
   for (int i = threadIdx.x; i <= E; i += C::NUM_THREADS) s_off[i] = args.offsets[i];
-  if (EPI == EPI_SWIGLU && args.tok_cnt)   // for the down launch's combine
-    for (int i = blockIdx.x * C::NUM_THREADS + threadIdx.x; i < args.tok_cnt_n;
-         i += gridDim.x * C::NUM_THREADS)
-      args.tok_cnt[i] = 0;
   __syncthreads();
   if (threadIdx.x == 0) {
     *abort_flag = 0;
@@ -855,10 +822,7 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
       const uint32_t ap = (it >> 1) & 1;
       if (ok) ok = mbar_wait(bar_accFull(ab), ap, abort_flag, args.status);
       ok = __all_sync(0xFFFFFFFFu, ok);        // the TMEM loads below are warp-collective
-      // the fused combine's barriers, like the SwiGLU exchange, are passed by
-      // every epilogue warp in every tile, also after a failed wait
-      const bool fused_combine = EPI == EPI_DOWN && NT <= 16 && args.out_bf16 != nullptr;
-      if (!ok && EPI != EPI_SWIGLU && !fused_combine) break;
+      if (!ok && EPI != EPI_SWIGLU) break;
       if (ok) tc_fence_after();
       // with two issuers and a single k-block per tile only issuer
       // (it*KB) % 2 wrote its buffer
@@ -1011,41 +975,6 @@ __global__ void __launch_bounds__(C::NUM_THREADS, C::CTAS)
       if (ok) {
         tc_fence_before();
         mbar_arrive(bar_accEmpty(ab));     // this tile's accumulators are read
-      }
-      if (fused_combine) {
-        // combine (after the accumulator buffer is released, so the next
-        // tile's UMMAs run meanwhile): the tile whose rows complete a token's k rows of this
-        // 128-column block sums them in slot order, adds the residual and
-        // rounds once to bf16 (as combine_kernel does)
-        int* s_last = reinterpret_cast<int*>(s_xch);
-        __threadfence();
-        asm volatile("bar.sync 7, 128;" ::: "memory");
-        if (m < NT) {
-          int last = -1;
-          if (ok && m < rows) {
-            const int tok = args.perm[s_off[e] + tb * NT + m] / args.k;
-            const int old = atomicAdd(args.tok_cnt + static_cast<size_t>(tok) * args.n_wb + wb, 1);
-            if (old == args.k - 1) last = tok;
-          }
-          s_last[m] = last;
-        }
-        asm volatile("bar.sync 7, 128;" ::: "memory");
-        __threadfence();
-        if (ok && col < args.n_out) {
-          for (int i = 0; i < rows; ++i) {
-            const int tok = s_last[i];
-            if (tok < 0) continue;
-            float acc = 0.f;
-            for (int jj = 0; jj < args.k; ++jj)
-              acc += __ldcg(args.out_f32 + (static_cast<size_t>(tok) * args.k + jj) * args.n_out + col);
-            if (args.resid)
-              acc += __uint_as_float(
-                  static_cast<uint32_t>(args.resid[static_cast<size_t>(tok) * args.n_out + col]) << 16);
-            args.out_bf16[static_cast<size_t>(tok) * args.n_out + col] =
-                __bfloat16_as_ushort(__float2bfloat16_rn(acc));
-          }
-        }
-        asm volatile("bar.sync 7, 128;" ::: "memory");
       }
     }
   }
@@ -1207,11 +1136,6 @@ cudaError_t launch_mx_impl(const MxGemmProblem& p, int num_sms, cudaStream_t st)
   a.topk_w = p.topk_w;
   a.bias = p.bias;
   a.status = p.status;
-  a.out_bf16 = C::NT <= 16 ? p.out_bf16 : nullptr;
-  a.resid = p.resid;
-  a.tok_cnt = p.tok_cnt;
-  a.tok_cnt_n = p.tok_cnt_n;
-  a.k = p.k;
   if (EPI == EPI_SWIGLU) {
     a.n_wb = (p.I + 63) / 64;
     a.rows_per_expert = 2 * p.I;
@@ -1288,7 +1212,7 @@ cudaError_t launch_mx_quant_gather(int variant, const uint16_t* x, const int32_t
                                    uint8_t* qlo, uint8_t* sfb, const int32_t* topk_idx,
                                    const int32_t* inv, int T, cudaStream_t st) {
   if (inv && topk_idx) {
-    const int grid = grid_for_n(static_cast<int64_t>(T) * ((K + 127) / 128), 256, 148 * 8);
+    const int grid = grid_for_n(static_cast<int64_t>(T) * (K / 32), 256, 148 * 8);
     if (variant == kMxPair)
       launch_kernel(mx_quant_gather_tok_kernel<kMxMaxNT>, dim3(grid), dim3(256), 0, st, x,
                     topk_idx, inv, offsets, E, T, k, K, qhi, qlo, sfb);
