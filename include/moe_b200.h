@@ -228,14 +228,16 @@ MOE_API moe_status moe_forward_ex(const void* x_dev, const float* W_r_dev, const
                                   const moe_forward_opts* opts, void* stream);
 
 /*
- * Same as moe_forward, instrumented: records a CUDA event on `stream` before
- * every kernel the pass launches and one after the last, waits for the last
+ * Same as moe_forward, instrumented: records a CUDA event on `stream` at the
+ * boundaries of the pass's stages and one after the last, waits for the last
  * event, and writes to stage_ms_host[0..11] (host memory, 12 floats) the
- * device time in milliseconds of each launch, in order -- router logits,
- * top-k/softmax, expert histogram, scan, scatter, activation gather, the two
- * scale transposes (gate/up, down), gate/up GEMM + SwiGLU, down GEMM +
- * weighted un-permute, per-token sum -- and in stage_ms_host[11] the span
- * from the first launch to the end of the last.
+ * device time in milliseconds of each stage, in order -- router (its weight
+ * split, logits and top-k/softmax launches; for at most 256 tokens also the
+ * permutation), top-k/softmax (0: inside the router stage), expert histogram,
+ * scan, scatter, activation gather, the two scale transposes (gate/up, down),
+ * gate/up GEMM + SwiGLU, down GEMM + weighted un-permute, per-token sum --
+ * and in stage_ms_host[11] the span from the first launch to the end of the
+ * last. A stage the pass does not launch reads as the cost of its two events.
  * Blocks the calling thread until the pass has finished.
  */
 MOE_API moe_status moe_forward_timed(const void* x_dev, const float* W_r_dev, const float* b_r_dev,
