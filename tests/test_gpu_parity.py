@@ -143,6 +143,48 @@ def test_router_max_experts_and_k():
     assert np.array_equal(perm, p) and np.array_equal(offsets, o)
 
 
+@pytest.mark.parametrize("case", ["order_and_boundary", "chain_with_copies"])
+def test_router_near_ties_settled_exactly(case):
+    """Router rows that differ by ~1e-6 in their logits, far below the fp32
+    tensor-core error (~1e-5) but far above two fp64 evaluations' (~1e-13):
+    the choice and its order must be the exact ones on every token, which only
+    the fp64 refinement of near ties can give. order_and_boundary: experts 0/1
+    always selected (bias +6) with their order decided by the tiny gap, experts
+    2/3 competing for the last slot (bias +3). chain_with_copies: sixteen
+    near-identical rows (bias +6, k = 8 of them selected) and exact copies of
+    four of them (equal logits: lower index first)."""
+    d = 2880
+    rng = np.random.default_rng(5)
+    if case == "order_and_boundary":
+        inp = W.make_custom(d, 64, 8, 3, 512, seed=77)
+        for a, b, bias in [(0, 1, 6.0), (2, 3, 3.0)]:
+            u = rng.standard_normal(d) / np.sqrt(d)
+            inp.W_r[b] = (inp.W_r[a].astype(np.float64) + 1e-6 * u).astype(np.float32)
+            inp.b_r[a] = inp.b_r[b] = bias
+    else:
+        inp = W.make_custom(d, 64, 64, 8, 512, seed=78)
+        base = inp.W_r[0].astype(np.float64)
+        for j in range(16):
+            inp.W_r[j] = (base + 1e-6 * rng.standard_normal(d) / np.sqrt(d)).astype(np.float32)
+            inp.b_r[j] = 6.0
+        for j in range(4):
+            inp.W_r[16 + j] = inp.W_r[j]
+            inp.b_r[16 + j] = inp.b_r[j]
+    T = inp.T
+    idx, w, counts, offsets, perm = _route_gpu(inp, T)
+    r = O.route(inp.x, inp.W_r, inp.b_r, inp.k)
+    srt = -np.sort(-r.s, axis=1)
+    gaps = -np.diff(srt[:, :inp.k + 1], axis=1)
+    close = int(np.sum((gaps < 1e-4) & (gaps > 0)))
+    assert close > T // 2, close          # the case really is full of near ties
+    # copies at the k-th / (k+1)-th boundary tie exactly (an exempt token whose
+    # choice is still validated); everything else must be exact
+    ties = G.compare_routing(idx, w, r, max_exempt=T if case == "chain_with_copies" else None)
+    G.check_tables_against_oracle(idx, counts, offsets, perm, r, inp.E)
+    print(f"[router] near ties {case}: {close} gaps below 1e-4 among the top k+1, "
+          f"exempt {ties}; every other choice and order exact")
+
+
 def test_router_total_order_with_nan_and_inf_logits():
     """Logits that are NaN or infinite still give one selection that every lane of
     the warp agrees on, the oracle's: numbers in descending order, then -inf, then
