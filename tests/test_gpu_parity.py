@@ -107,11 +107,12 @@ def test_router_silent_init_copies_tie_exactly():
                                      (96, 40, 8, 400), (2880, 128, 4, 257)],
                          ids=["E256_k32", "E248_k20", "E4", "d96", "T257"])
 def test_router_tensor_core_path(d, E, k, T):
-    """Batches over 256 tokens route on the tensor cores (fp32 router weights as
-    three bf16 terms, top-k and softmax in the same kernel): the choice on every
-    token against the oracle, the tables bit-exact. Cases: 256 expert columns (two
-    stages), 4 experts padded to 16, d = 32 mod 64 (a half-empty last k-block), a
-    ragged last 128-token tile."""
+    """The tensor-core router (fp32 router weights as three bf16 terms, logits
+    split over a cluster, top-k with fp64 near-tie refinement) at shapes off the
+    workloads: the choice on every token against the oracle, the tables
+    bit-exact. Cases: 256 expert columns (two stages, two accumulators), 4
+    experts padded to 16, d = 32 mod 64 (a half-empty last k-block), a ragged last
+    128-token tile."""
     inp = W.make_custom(d, 64, E, k, T, seed=90 + E)
     idx, w, counts, offsets, perm = _route_gpu(inp, T)
     r = O.route(inp.x, inp.W_r, inp.b_r, k)
