@@ -196,16 +196,10 @@ __global__ void __launch_bounds__(256) router_split_kernel(const float* __restri
 }
 
 struct RouterTcArgs {
-  const uint16_t* x;
-  const float* W_r;
   const float* b_r;
-  const float* norms;
-  const unsigned long long* fps;
-  int T, E, k, d, npad, nacc, per, stages, ld, stage_bytes, body, tmem_cols, KB;
-  float* logits;
-  float* xsq;
-  int32_t* topk_idx;
-  float* topk_w;
+  int T, E, d, npad, nacc, per, stages, ld, stage_bytes, body, tmem_cols, KB;
+  float* logits;   // [T][E]
+  float* xsq;      // [T]: ||x_t||^2
   int* status;
 };
 
@@ -758,14 +752,9 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b
   }
   const int C = cluster_size(T, d, dev, static_cast<size_t>(router_tc_shape(256).smem_alloc));
   RouterTcArgs a;
-  a.x = x;
-  a.W_r = W_r;
   a.b_r = b_r;
-  a.norms = norms;
-  a.fps = fps;
   a.T = T;
   a.E = E;
-  a.k = k;
   a.d = d;
   a.npad = sh.npad;
   a.nacc = sh.nacc;
@@ -778,8 +767,6 @@ cudaError_t launch_router_tc(const uint16_t* x, const float* W_r, const float* b
   a.KB = (d + RT_BK - 1) / RT_BK;
   a.logits = logits;
   a.xsq = xsq;
-  a.topk_idx = topk_idx;
-  a.topk_w = topk_w;
   a.status = status;
   const int tiles = (T + RT_M - 1) / RT_M;
   cudaError_t e = launch_kernel_cluster(router_tc_kernel, dim3(tiles * C), dim3(RT_THREADS),
