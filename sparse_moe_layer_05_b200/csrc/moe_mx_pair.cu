@@ -23,7 +23,7 @@
 //            of a token's TMEM lane meet in one thread, and a tile's 96 H
 //            columns are three whole MX groups of 32 (the epilogue converts H
 //            for the down GEMM per group).
-//   down:    NH = 120: output columns n0..n0+239.
+//   down:    NH = 112 (120 for kind::mxf4): output columns n0..n0+N-1.
 // Token rows live in a padded layout (each expert's rows start at a multiple
 // of 128), so each CTA's half tile is one contiguous block of rows and its
 // scale block one contiguous run of bytes. A tile covers 256 rows of one
@@ -31,17 +31,26 @@
 // loads no token rows (its accumulator rows are never stored).
 //
 // Scale factors in tensor memory. Each CTA holds the A scales of its own 128
-// rows (one 512-byte tcgen05.cp atom per term: lane m % 32 of column m / 32)
-// and the B scales of all N columns (two atoms), at the same TMEM columns in
-// both CTAs; the even CTA's issuing thread copies them with
-// tcgen05.cp.cta_group::2, which moves each CTA's atom into its own TMEM.
+// rows (one 512-byte atom per term: row m's four K-step bytes in lane m % 32
+// of column m / 32, the same in all four lane quarters) and the B scales of
+// all N columns (two atoms), at the same TMEM columns in both CTAs. For the
+// 8-bit kinds each pipeline stage has its own slot of scale columns, which
+// four builder warps (one per TMEM lane quarter) fill with tcgen05.st while
+// the stage's operands arrive, so that the issuing thread issues only UMMAs
+// and commits (a tcgen05.cp costs that thread about as long as a UMMA). For
+// kind::mxf4 (six atoms per stage: the slots would not fit beside the two
+// accumulators) the atoms are staged in shared memory and the issuing thread
+// copies them with tcgen05.cp.cta_group::2 before each stage's UMMAs.
 //
-// Roles (384 threads per CTA):
+// Roles (448 threads per CTA; 384 for kind::mxf4):
 //   warp 0   TMA producer: token rows (A) and their scale block, weight codes
 //            (B); the tile's weight-scale rows into a double buffer
-//   warp 1   TMEM allocation; in the even CTA the UMMA issuer
-//   warp 2   B-scale builder: the tile's weight scales -> two atoms per stage
-//   warp 3   in the odd CTA: relays "stage full" to the even CTA's issuer
+//   warp 1   TMEM allocation; in the even CTA the UMMA issuer, in the odd CTA
+//            the relay of "stage full" to the even CTA's issuer
+//   warps 2, 3, 12, 13  scale builders, TMEM lane quarters 2, 3, 0, 1: the
+//            stage's token scale atoms and the tile's weight scales -> the
+//            stage's slot (kind::mxf4: warp 2 alone, B atoms into shared
+//            memory)
 //   warps 4-11 epilogue: warp w reads TMEM lane quarter w % 4 (one token row
 //            per thread); warps 4-7 and 8-11 take alternate column groups
 // Every wait is bounded (moe_ptx.cuh): a stuck pipeline records a timeout in
@@ -89,7 +98,12 @@ struct PairCfg {
   static constexpr int KBK = F4 ? 256 : 128;              // K elements per stage
   static constexpr int TERMS = ACT == ACT_HILO ? 2 : 1;
   static constexpr int MT = 128;                          // token rows per CTA
-  static constexpr int NH = EPI == PAIR_SWIGLU ? 96 : 120;  // weight rows per CTA
+  // scale atoms reach TMEM by tcgen05.st into per-stage slots (8-bit kinds)
+  // or by tcgen05.cp from shared memory (kind::mxf4)
+  static constexpr bool SFST = !F4;
+  // weight rows per CTA; down: two accumulators of N = 224 leave 64 TMEM
+  // columns for the scale slots
+  static constexpr int NH = EPI == PAIR_SWIGLU ? 96 : (SFST ? 112 : 120);
   static constexpr int N = 2 * NH;                        // UMMA N
   static constexpr int A_PLANE = MT * 128;                // one term: 128-byte rows
   static constexpr int A_BYTES = TERMS * A_PLANE;
@@ -101,29 +115,37 @@ struct PairCfg {
   static constexpr int OFF_B = A_BYTES;
   static constexpr int OFF_SFA = OFF_B + B_BYTES;
   static constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
-  static constexpr int STAGE_BYTES = (OFF_SFB + SFB_BYTES + 1023) / 1024 * 1024;
+  static constexpr int STAGE_BYTES = (OFF_SFB + (SFST ? 0 : SFB_BYTES) + 1023) / 1024 * 1024;
   static constexpr int TS_BYTES = N * (kMxMaxK / 32);     // a tile's weight-scale rows
   static constexpr int FIXED = 2 * TS_BYTES + 3 * (kMaxE + 1) * 4 + 512;
   static constexpr int STAGES_FIT = (kPairSmemBudget - FIXED) / STAGE_BYTES;
-  static constexpr int STAGES = STAGES_FIT > 6 ? 6 : STAGES_FIT;
+  static constexpr int A_ATOMS = SFA_BYTES / 512;
+  static constexpr int B_ATOMS = SFB_BYTES / 512;
+  static constexpr int SLOT_COLS = 4 * (A_ATOMS + B_ATOMS);   // one stage's scale columns
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int STAGES_TMEM = SFST ? (TMEM_COLS - 2 * N) / SLOT_COLS : 6;
+  static constexpr int STAGES_CAP = STAGES_TMEM < 6 ? STAGES_TMEM : 6;
+  static constexpr int STAGES = STAGES_FIT > STAGES_CAP ? STAGES_CAP : STAGES_FIT;
   static constexpr int OFF_TS = STAGES * STAGE_BYTES;
   static constexpr int OFF_BAR = OFF_TS + 2 * TS_BYTES;
-  static constexpr int NUM_BARS = 3 * STAGES + 10;
+  static constexpr int NUM_BARS = 4 * STAGES + 10;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TAB = OFF_MISC + 16;
   static constexpr int SMEM_BYTES = OFF_TAB + 3 * (kMaxE + 1) * 4;
   static constexpr int SMEM_ALLOC = SMEM_BYTES + 1024;
   static constexpr int EPI_WARPS = 8;                     // two per TMEM lane quarter
-  static constexpr int NUM_THREADS = 128 + 32 * EPI_WARPS;
-  static constexpr int TMEM_COLS = 512;
+  static constexpr int BUILDERS = SFST ? 4 : 1;           // scale-builder warps
+  static constexpr int NUM_THREADS = 128 + 32 * EPI_WARPS + (SFST ? 64 : 0);
   static constexpr int ACC_COLS = N;                      // per accumulator buffer
   static constexpr int SF_COL0 = 2 * N;                   // A scales, then B scales
   static constexpr int SFA_COLS = SFA_BYTES / 128;        // 4 TMEM columns per atom
   static constexpr int SFB_COLS = SFB_BYTES / 128;
-  static constexpr int TX_FULL = A_TX + B_TX + SFA_BYTES; // a stage with token rows
+  static constexpr int TX_FULL = A_TX + B_TX + (SFST ? 0 : SFA_BYTES);   // a stage with token rows
   static constexpr uint32_t ATYPE = ACT == ACT_E2M1 ? 5u : 0u;   // E2M1 or E4M3
   static_assert(STAGES >= 3, "pipeline depth");
-  static_assert(SF_COL0 + SFA_COLS + SFB_COLS <= TMEM_COLS, "TMEM budget");
+  static_assert(SF_COL0 + (SFST ? STAGES * SLOT_COLS : SFA_COLS + SFB_COLS) <= TMEM_COLS,
+                "TMEM budget");
+  static_assert(NUM_BARS * 8 + 16 <= 512, "barrier space");
   static_assert(SMEM_ALLOC <= 232448, "shared memory");
   static_assert(OFF_B % 1024 == 0 && B_BYTES % 1024 == 0 && STAGE_BYTES % 1024 == 0, "swizzle");
   static_assert(N % 16 == 0 && N <= 256, "UMMA N");
@@ -196,7 +218,7 @@ struct PairArgs {
 __device__ __forceinline__ float silu_p(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
 template <int EPI, int ACT>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI, ACT>::NUM_THREADS, 1)
     grouped_mx_pair_kernel(const __grid_constant__ CUtensorMap tmA,
                            const __grid_constant__ CUtensorMap tmAt,
                            const __grid_constant__ CUtensorMap tmB,
@@ -215,12 +237,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   const uint32_t bar0 = sbase + C::OFF_BAR;
   auto bar_full = [&](int s) { return bar0 + 8u * s; };
   auto bar_empty = [&](int s) { return bar0 + 8u * (S + s); };
-  auto bar_peerFull = [&](int s) { return bar0 + 8u * (2 * S + s); };
   auto bar_accFull = [&](int b) { return bar0 + 8u * (3 * S + b); };
   auto bar_accEmpty = [&](int b) { return bar0 + 8u * (3 * S + 2 + b); };
   auto bar_peerAcc = [&](int b) { return bar0 + 8u * (3 * S + 4 + b); };
   auto bar_tsFull = [&](int b) { return bar0 + 8u * (3 * S + 6 + b); };
   auto bar_tsEmpty = [&](int b) { return bar0 + 8u * (3 * S + 8 + b); };
+  auto bar_sfaFull = [&](int s) { return bar0 + 8u * (3 * S + 10 + s); };
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   int* s_off = reinterpret_cast<int*>(smem + C::OFF_TAB);
@@ -243,16 +265,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
     s_tp[E] = acc;
     s_tb[E] = tb;
     for (int s = 0; s < S; ++s) {
-      mbar_init(bar_full(s), 2);     // producer (with the TMA bytes) + B-scale builder
+      // producer (with the TMA bytes) + builders; in the even CTA also the
+      // odd CTA's relay, so that one wait covers both halves of the stage
+      mbar_init(bar_full(s), 1 + C::BUILDERS + (rank == 0 ? 1 : 0));
+      mbar_init(bar_sfaFull(s), 1);  // the stage's token scale block (8-bit kinds)
       mbar_init(bar_empty(s), 1);    // the issuer's commit, multicast to both CTAs
-      mbar_init(bar_peerFull(s), 1); // the odd CTA's relay
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(bar_accFull(b), 1);
       mbar_init(bar_accEmpty(b), C::EPI_WARPS * 32);
       mbar_init(bar_peerAcc(b), 1);
       mbar_init(bar_tsFull(b), 1);
-      mbar_init(bar_tsEmpty(b), 1);
+      mbar_init(bar_tsEmpty(b), C::BUILDERS);
     }
     fence_mbar_init();
     tma_prefetch_desc(&tmA);
@@ -345,6 +369,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
           const uint32_t st = sbase + s * C::STAGE_BYTES;
           const uint32_t fb = bar_full(s);
           mbar_expect_tx(fb, has_a ? C::TX_FULL : C::B_TX);
+          if (C::SFST) mbar_expect_tx(bar_sfaFull(s), has_a ? C::SFA_BYTES : 0u);
           const bool last_tail = tail && kb == KB - 1;
           const int kx = last_tail ? K - 128 : kb * 128;
           // F4: byte coordinates in the packed rows (two elements per byte)
@@ -360,7 +385,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
               tma_load_2d(st, last_tail ? &tmAt : &tmA, last_tail ? 0 : kb * 128, t.arow, fb);
             bulk_load(st + C::OFF_SFA,
                       args.sfa + (static_cast<size_t>(t.ttile) * KB + kb) * C::SFA_BYTES,
-                      C::SFA_BYTES, fb);
+                      C::SFA_BYTES, C::SFST ? bar_sfaFull(s) : fb);
           }
           if (ACT == ACT_F4)
             tma_load_3d(st + C::OFF_B, &tmB, kxb, wrow, t.e, fb);
@@ -373,12 +398,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         }
       }
     }
-  } else if (warp == 2) {
-    // -------------------------------------------------- B-scale builder --
-    // Lane l fills bytes 16l..16l+15 of both atoms: the four scale bytes (K
-    // steps 0..3 of the k-block) of B columns 32w + l (atom 0) and
-    // 128 + 32w + l (atom 1), w = 0..3, read from the tile's scale rows
-    // (row c of the tile-scale buffer is B column c; 2-byte aligned rows).
+  } else if (warp == 2 || (C::SFST && (warp == 3 || warp >= 12))) {
+    // ------------------------------------------------------ scale builders --
+    // Lane l forms row l of both B atoms: the four scale bytes (K steps 0..3
+    // of the k-block) of B columns 32w + l (atom 0) and 128 + 32w + l (atom
+    // 1), w = 0..3, read from the tile's scale rows (row c of the tile-scale
+    // buffer is B column c; 2-byte aligned rows). 8-bit kinds: each builder
+    // stores them, after row l of the stage's token scale atoms, into lane l
+    // of its TMEM lane quarter of the stage's slot.
     int s = 0, ph = 0, it = 0;
     bool ok = true;
     for (int tile = pair_id; tile < total && ok; tile += npairs, ++it) {
@@ -409,19 +436,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
             w[8 * q + j] = v;
           }
         }
-        if (!(ok = mbar_wait(bar_empty(s), ph ^ 1, abort_flag, args.status))) break;
-        uint8_t* sfb = smem + s * C::STAGE_BYTES + C::OFF_SFB;
-        // atoms: [word 0: columns 0-127, 128-255][word 1: ...] (F4 has two words)
+        if (C::SFST) {
+          // the stage's token scale block has landed; the producer loaded it
+          // after "stage empty", so the UMMAs that last read this slot are done
+          if (!(ok = mbar_wait(bar_sfaFull(s), ph, abort_flag, args.status))) break;
+          tc_fence_after();
+          const uint8_t* sfa = smem + s * C::STAGE_BYTES + C::OFF_SFA;
+          const uint32_t slot = tmem_base + (static_cast<uint32_t>((warp & 3) * 32) << 16) +
+                                static_cast<uint32_t>(C::SF_COL0 + s * C::SLOT_COLS);
 #pragma unroll
-        for (int q = 0; q < GPB / 4; ++q) {
-          *reinterpret_cast<uint4*>(sfb + 1024 * q + lane * 16) =
-              make_uint4(w[8 * q], w[8 * q + 1], w[8 * q + 2], w[8 * q + 3]);
-          *reinterpret_cast<uint4*>(sfb + 1024 * q + 512 + lane * 16) =
-              make_uint4(w[8 * q + 4], w[8 * q + 5], w[8 * q + 6], w[8 * q + 7]);
+          for (int a = 0; a < C::A_ATOMS; ++a)
+            tmem_st4(slot + 4 * a, *reinterpret_cast<const uint4*>(sfa + 512 * a + lane * 16));
+          tmem_st4(slot + 4 * C::A_ATOMS, make_uint4(w[0], w[1], w[2], w[3]));
+          tmem_st4(slot + 4 * C::A_ATOMS + 4, make_uint4(w[4], w[5], w[6], w[7]));
+          tmem_wait_st();
+          tc_fence_before();
+        } else {
+          if (!(ok = mbar_wait(bar_empty(s), ph ^ 1, abort_flag, args.status))) break;
+          uint8_t* sfb = smem + s * C::STAGE_BYTES + C::OFF_SFB;
+          // atoms: [word 0: columns 0-127, 128-255][word 1: ...] (F4 has two words)
+#pragma unroll
+          for (int q = 0; q < GPB / 4; ++q) {
+            *reinterpret_cast<uint4*>(sfb + 1024 * q + lane * 16) =
+                make_uint4(w[8 * q], w[8 * q + 1], w[8 * q + 2], w[8 * q + 3]);
+            *reinterpret_cast<uint4*>(sfb + 1024 * q + 512 + lane * 16) =
+                make_uint4(w[8 * q + 4], w[8 * q + 5], w[8 * q + 6], w[8 * q + 7]);
+          }
         }
-        // orders these shared-memory writes (and the tile-scale reads) before
-        // the async-proxy accesses that follow: tcgen05.cp of the atoms, the
-        // next bulk copy into the tile-scale buffer
+        // orders the shared-memory accesses above (tile-scale and scale-block
+        // reads, atoms written for tcgen05.cp) before the async-proxy accesses
+        // that follow: tcgen05.cp, the next bulk copies into these buffers
         fence_proxy_async_smem();
         __syncwarp();
         if (lane == 0) mbar_arrive(bar_full(s));
@@ -433,8 +477,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
   } else if (warp == 1) {
     // ----------------------------------------- UMMA issuer (even CTA) --
     if (rank == 0 && lane == 0) {
-      const uint32_t sfa_t = tmem_base + C::SF_COL0;
-      const uint32_t sfb_t = sfa_t + C::SFA_COLS;
       int s = 0, ph = 0, it = 0;
       bool ok = true;
       for (int tile = pair_id; tile < total && ok; tile += npairs, ++it) {
@@ -446,32 +488,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         const uint32_t d = tmem_base + ab * C::ACC_COLS;
         uint32_t accum = 0;   // the tile's first UMMA overwrites the buffer
         for (int kb = 0; kb < KB; ++kb) {
-          if (!(ok = mbar_wait(bar_full(s), ph, abort_flag, args.status))) break;
-          if (!(ok = mbar_wait_cluster(bar_peerFull(s), ph, abort_flag, args.status))) break;
+          if (!(ok = mbar_wait_cluster(bar_full(s), ph, abort_flag, args.status))) break;
           tc_fence_after();
           const uint32_t st = sbase + s * C::STAGE_BYTES;
           // scale atoms (each 4 TMEM columns): A's terms (or F4's two words),
-          // then B's (two per word)
+          // then B's (two per word); 8-bit kinds: the stage's slot, filled by
+          // the builders; F4: one slot, copied here
+          const uint32_t sfa_t =
+              tmem_base + static_cast<uint32_t>(C::SF_COL0 + (C::SFST ? s * C::SLOT_COLS : 0));
+          const uint32_t sfb_t = sfa_t + 4 * C::A_ATOMS;
+          // operand descriptors of the stage; each K step adds its byte
+          // offset to the start-address field (addresses stay below 2^18)
+          const uint64_t ad0 = sdesc_k_sw128(st), bd0 = sdesc_k_sw128(st + C::OFF_B);
+          if (!C::SFST) {
 #pragma unroll
-          for (int a = 0; a < C::SFA_BYTES / 512; ++a)
-            tmem_cp_32x128b_x4_pair(sfa_t + 4 * a, sdesc_k_noswizzle(st + C::OFF_SFA + 512 * a, 128));
+            for (int a = 0; a < C::A_ATOMS; ++a)
+              tmem_cp_32x128b_x4_pair(sfa_t + 4 * a,
+                                      sdesc_k_noswizzle(st + C::OFF_SFA + 512 * a, 128));
 #pragma unroll
-          for (int a = 0; a < C::SFB_BYTES / 512; ++a)
-            tmem_cp_32x128b_x4_pair(sfb_t + 4 * a, sdesc_k_noswizzle(st + C::OFF_SFB + 512 * a, 128));
+            for (int a = 0; a < C::B_ATOMS; ++a)
+              tmem_cp_32x128b_x4_pair(sfb_t + 4 * a,
+                                      sdesc_k_noswizzle(st + C::OFF_SFB + 512 * a, 128));
+          }
           // K steps with compile-time indices; a tail k-block issues only its
           // steps past the previous block
           auto step = [&](const int kk) {
             if (C::F4) {
               const uint32_t id = static_cast<uint32_t>(kk & 1) * 2;
-              umma_mxf4_pair(d, sdesc_k_sw128(st + kk * 32), sdesc_k_sw128(st + C::OFF_B + kk * 32),
+              umma_mxf4_pair(d, ad0 + static_cast<uint64_t>(kk * 2), bd0 + static_cast<uint64_t>(kk * 2),
                              idesc_mxf4(256, C::N, id, id), (sfa_t + 4 * (kk >> 1)) | (id << 30),
                              (sfb_t + 8 * (kk >> 1)) | (id << 30), accum);
               accum = 1;
             } else {
 #pragma unroll
               for (int h = 0; h < C::TERMS; ++h) {
-                umma_mx_pair(d, sdesc_k_sw128(st + h * C::A_PLANE + kk * 32),
-                             sdesc_k_sw128(st + C::OFF_B + kk * 32),
+                umma_mx_pair(d, ad0 + static_cast<uint64_t>((h * C::A_PLANE + kk * 32) >> 4),
+                             bd0 + static_cast<uint64_t>(kk * 2),
                              idesc_pair(256, C::N, C::ATYPE, static_cast<uint32_t>(kk)),
                              (sfa_t + 4 * h) | (static_cast<uint32_t>(kk) << 30),
                              sfb_t | (static_cast<uint32_t>(kk) << 30), accum);
@@ -499,23 +551,24 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(384, 1)
         }
         if (ok) umma_commit_pair(bar_accFull(ab));
       }
-    }
-  } else if (warp == 3) {
-    // ------------------------------------ stage relay (odd CTA) --
-    if (rank == 1 && lane == 0) {
+    } else if (rank == 1 && lane == 0) {
+      // ---------------------------------------- stage relay (odd CTA) --
       int s = 0, ph = 0;
       bool ok = true;
       for (int tile = pair_id; tile < total && ok; tile += npairs) {
         for (int kb = 0; kb < KB; ++kb) {
           if (!(ok = mbar_wait(bar_full(s), ph, abort_flag, args.status))) break;
-          // the stage is complete in this CTA's shared memory (observed with
-          // acquire semantics above); forward that to the issuer
-          mbar_arrive_remote_relaxed(mapa_shared(bar_peerFull(s), 0));
+          // the stage is complete in this CTA's shared memory and TMEM slot
+          // (observed with acquire semantics above: the builders waited for
+          // their tcgen05.st to complete before arriving); forward that to the
+          // issuer. A release at cluster scope here measured 0.35 us per stage
+          // on the issuer's critical path.
+          mbar_arrive_remote_relaxed(mapa_shared(bar_full(s), 0));
           if (++s == S) { s = 0; ph ^= 1; }
         }
       }
     }
-  } else {
+  } else if (warp >= 4 && warp < 4 + C::EPI_WARPS) {
     // ----------------------------------------------------------- epilogue --
     const int quad = warp & 3;
     const int egrp = (warp - 4) >> 2;   // 0 or 1: alternate column groups

@@ -261,6 +261,17 @@ __device__ __forceinline__ void tmem_st16_sync(uint32_t taddr, const uint4 (&v)[
       : "memory");
 }
 
+// Registers -> TMEM: 4 consecutive 32-bit columns of this thread's lane; no
+// wait (tmem_wait_st completes this warp's stores).
+__device__ __forceinline__ void tmem_st4(uint32_t taddr, uint4 v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr),
+               "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // CTA-pair UMMA (issued by the even CTA of a cluster pair): A rows 0..127 come
 // from this CTA's shared memory and rows 128..255 from the peer's at the same
 // offsets; B's N columns are split the same way; each CTA's TMEM receives its
