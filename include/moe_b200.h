@@ -235,7 +235,9 @@ MOE_API moe_status moe_forward_ex(const void* x_dev, const float* W_r_dev, const
  * split, logits and top-k/softmax launches; for at most 256 tokens also the
  * permutation), top-k/softmax (0: inside the router stage), expert histogram,
  * scan, scatter, activation gather, the two scale transposes (gate/up, down),
- * gate/up GEMM + SwiGLU, down GEMM + weighted un-permute, per-token sum --
+ * gate/up GEMM + SwiGLU, down GEMM + weighted un-permute (on the CTA-pair
+ * tiles with the launch before it that lays out the down weights' scale
+ * atoms), per-token sum --
  * and in stage_ms_host[11] the span from the first launch to the end of the
  * last. A stage the pass does not launch reads as the cost of its two events.
  * Blocks the calling thread until the pass has finished.

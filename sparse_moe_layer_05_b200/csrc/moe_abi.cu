@@ -57,6 +57,7 @@ struct Layout {
   size_t router_terms;   // the router's bf16 weight terms and row norms
   size_t inv;            // permuted row of each (token, slot) pair
   size_t mx_tok_rows;
+  size_t wsfb;     // the CTA-pair down GEMM's weight-scale atoms
   size_t x_norm;   // moe_forward_block: the normalised rows [T][d] bf16
 };
 
@@ -105,6 +106,7 @@ void make_layout(int E, int k, int T, int d, int I, bool hostio, Layout* L, bool
                                moe::mx_sfb_bytes(static_cast<int>(P), E, d)));
   L->d_scales_t = take(larger(static_cast<size_t>(E) * d * (I / 32),
                               moe::mx_sfb_bytes(static_cast<int>(P), E, I)));
+  L->wsfb = take(moe::mx_pair_down_atom_bytes(E, d, I));
   if (hostio) {
     L->x_in = take(static_cast<size_t>(T) * d * 2);
     L->out_buf = take(static_cast<size_t>(T) * d * 2);
@@ -433,6 +435,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     m2.h_hi = nullptr;
     m2.h_sfb = nullptr;
     m2.out_f32 = yw;
+    m2.wsfb = at<uint8_t>(ws, L.wsfb);   // CTA pair, 8-bit activations
     m2.perm = perm;
     m2.topk_w = topk_w;
     m2.n_out = d;
@@ -497,6 +500,7 @@ moe_status run_forward(const uint16_t* x, const float* W_r, const float* b_r, co
     m2.h_lo = nullptr;
     m2.h_sfb = nullptr;
     m2.out_f32 = yw;
+    m2.wsfb = at<uint8_t>(ws, L.wsfb);   // CTA pair, 8-bit activations
     m2.perm = perm;
     m2.topk_w = topk_w;
     m2.n_out = d;
@@ -611,6 +615,8 @@ int moe_forward_launch_count(int E, int k, int T, int d, int I) {
   const int tiles =
       choose_tiles(g_tile_policy.load(std::memory_order_relaxed), T * k, E, mx_shape_ok(d, I));
   if (tiles == moe::TILES_MX || tiles == moe::TILES_MX_PAIR) n -= 2;
+  // the CTA-pair down GEMM lays out its weight-scale atoms first
+  if (tiles == moe::TILES_MX_PAIR) n += 1;
   return n;
 }
 

@@ -212,6 +212,9 @@ struct MxGemmProblem {
   int* status;
   const float* bias;        // optional, as in GroupedGemmProblem
   int act;                  // ACT_HILO, ACT_E4M3 or ACT_E2M1 (b_lo / h_lo unused but HILO)
+  // CTA-pair down GEMM with 8-bit activations: room for its weight-scale atoms
+  // (mx_pair_down_atom_bytes), written by the launch before the GEMM
+  uint8_t* wsfb;
 };
 cudaError_t launch_mx_gemm_gateup_swiglu(int variant, const MxGemmProblem& p, int num_sms,
                                          cudaStream_t st);
@@ -220,6 +223,7 @@ cudaError_t launch_mx_gemm_down(int variant, const MxGemmProblem& p, int num_sms
 // and their scale blocks in the 128-row padded layout.
 cudaError_t launch_mx_pair_gateup_swiglu(const MxGemmProblem& p, int num_sms, cudaStream_t st);
 cudaError_t launch_mx_pair_down(const MxGemmProblem& p, int num_sms, cudaStream_t st);
+size_t mx_pair_down_atom_bytes(int E, int d, int I);
 
 // Tensor maps of the block-scaled path (moe_mx_gemm.cu): E2M1 code rows
 // (main map over whole 128-element k-blocks plus a tail map for [K-128, K)),

@@ -41,6 +41,11 @@
 // kind::mxf4 (six atoms per stage: the slots would not fit beside the two
 // accumulators) the atoms are staged in shared memory and the issuing thread
 // copies them with tcgen05.cp.cta_group::2 before each stage's UMMAs.
+// The gate/up builders form the weight atoms from the tile's scale rows,
+// staged in shared memory per tile; the down GEMM's weight atoms are laid
+// out in global memory beforehand (pair_weight_atoms_kernel, one 1 KB block
+// per tile and k-block) and arrive with the stage, which leaves the down
+// GEMM the shared memory for a fourth stage.
 //
 // Roles (448 threads per CTA; 384 for kind::mxf4):
 //   warp 0   TMA producer: token rows (A) and their scale block, weight codes
@@ -101,6 +106,9 @@ struct PairCfg {
   // scale atoms reach TMEM by tcgen05.st into per-stage slots (8-bit kinds)
   // or by tcgen05.cp from shared memory (kind::mxf4)
   static constexpr bool SFST = !F4;
+  // down GEMM, 8-bit kinds: weight atoms pre-built in global memory, loaded
+  // with each stage (no tile-scale buffers)
+  static constexpr bool SFBG = EPI == PAIR_DOWN && SFST;
   // weight rows per CTA; down: two accumulators of N = 224 leave 64 TMEM
   // columns for the scale slots
   static constexpr int NH = EPI == PAIR_SWIGLU ? 96 : (SFST ? 112 : 120);
@@ -115,9 +123,11 @@ struct PairCfg {
   static constexpr int OFF_B = A_BYTES;
   static constexpr int OFF_SFA = OFF_B + B_BYTES;
   static constexpr int OFF_SFB = OFF_SFA + SFA_BYTES;
-  static constexpr int STAGE_BYTES = (OFF_SFB + (SFST ? 0 : SFB_BYTES) + 1023) / 1024 * 1024;
+  static constexpr int STAGE_BYTES =
+      (OFF_SFB + ((SFST && !SFBG) ? 0 : SFB_BYTES) + 1023) / 1024 * 1024;
   static constexpr int TS_BYTES = N * (kMxMaxK / 32);     // a tile's weight-scale rows
-  static constexpr int FIXED = 2 * TS_BYTES + 3 * (kMaxE + 1) * 4 + 512;
+  static constexpr int TS_BUFS = SFBG ? 0 : 2;
+  static constexpr int FIXED = TS_BUFS * TS_BYTES + 3 * (kMaxE + 1) * 4 + 512;
   static constexpr int STAGES_FIT = (kPairSmemBudget - FIXED) / STAGE_BYTES;
   static constexpr int A_ATOMS = SFA_BYTES / 512;
   static constexpr int B_ATOMS = SFB_BYTES / 512;
@@ -127,7 +137,7 @@ struct PairCfg {
   static constexpr int STAGES_CAP = STAGES_TMEM < 6 ? STAGES_TMEM : 6;
   static constexpr int STAGES = STAGES_FIT > STAGES_CAP ? STAGES_CAP : STAGES_FIT;
   static constexpr int OFF_TS = STAGES * STAGE_BYTES;
-  static constexpr int OFF_BAR = OFF_TS + 2 * TS_BYTES;
+  static constexpr int OFF_BAR = OFF_TS + TS_BUFS * TS_BYTES;
   static constexpr int NUM_BARS = 4 * STAGES + 10;
   static constexpr int OFF_MISC = OFF_BAR + NUM_BARS * 8;
   static constexpr int OFF_TAB = OFF_MISC + 16;
@@ -201,6 +211,7 @@ struct PairArgs {
   int KB;                     // k-blocks
   const uint8_t* scales;      // [E][rows_per_expert][K/32] E8M0 weight scales
   const uint8_t* sfa;         // token scale blocks [128-row tile][KB][SFA_BYTES]
+  const uint8_t* wsfb;        // SFBG: weight atoms [E][n_tiles][KB][SFB_BYTES]
   // gate/up: converted H rows (h_lo: the lo plane of the bf16 split) and
   // their scale blocks (the down GEMM's A operand)
   uint8_t* h_q;
@@ -336,7 +347,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI, ACT>::N
       auto load_tile_scales = [&](int tile, int itx) -> bool {
         Tile t;
         decode(tile, t);
-        const int b = itx & 1;
+        const int b = itx & 1;   // (not reached with SFBG)
         if (!mbar_wait(bar_tsEmpty(b), ((itx >> 1) & 1) ^ 1, abort_flag, args.status)) return false;
         const uint32_t ts = sbase + C::OFF_TS + b * C::TS_BYTES;
         const size_t ebase = static_cast<size_t>(t.e) * args.rows_per_expert;
@@ -355,7 +366,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI, ACT>::N
         return true;
       };
       int s = 0, ph = 0, it = 0;
-      bool ok = pair_id >= total || load_tile_scales(pair_id, 0);
+      bool ok = pair_id >= total || C::SFBG || load_tile_scales(pair_id, 0);
       const int kb_next = min(3, KB - 1);
       for (int tile = pair_id; tile < total && ok; tile += npairs, ++it) {
         Tile t;
@@ -369,7 +380,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI, ACT>::N
           const uint32_t st = sbase + s * C::STAGE_BYTES;
           const uint32_t fb = bar_full(s);
           mbar_expect_tx(fb, has_a ? C::TX_FULL : C::B_TX);
-          if (C::SFST) mbar_expect_tx(bar_sfaFull(s), has_a ? C::SFA_BYTES : 0u);
+          if (C::SFST)
+            mbar_expect_tx(bar_sfaFull(s),
+                           (has_a ? C::SFA_BYTES : 0u) + (C::SFBG ? C::SFB_BYTES : 0u));
+          if (C::SFBG)
+            bulk_load(st + C::OFF_SFB,
+                      args.wsfb + ((static_cast<size_t>(t.e) * args.n_tiles + t.nt) * KB + kb) *
+                                      C::SFB_BYTES,
+                      C::SFB_BYTES, bar_sfaFull(s));
           const bool last_tail = tail && kb == KB - 1;
           const int kx = last_tail ? K - 128 : kb * 128;
           // F4: byte coordinates in the packed rows (two elements per byte)
@@ -393,7 +411,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI, ACT>::N
             tma_load_3d(st + C::OFF_B, last_tail ? &tmBt : &tmB, last_tail ? 0 : kb * 128, wrow,
                         t.e, fb);
           if (++s == S) { s = 0; ph ^= 1; }
-          if (kb == kb_next && tile + npairs < total && !(ok = load_tile_scales(tile + npairs, it + 1)))
+          if (!C::SFBG && kb == kb_next && tile + npairs < total &&
+              !(ok = load_tile_scales(tile + npairs, it + 1)))
             break;
         }
       }
@@ -410,7 +429,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI, ACT>::N
     bool ok = true;
     for (int tile = pair_id; tile < total && ok; tile += npairs, ++it) {
       const int b = it & 1;
-      if (!(ok = mbar_wait(bar_tsFull(b), (it >> 1) & 1, abort_flag, args.status))) break;
+      if (!C::SFBG && !(ok = mbar_wait(bar_tsFull(b), (it >> 1) & 1, abort_flag, args.status)))
+        break;
       const uint8_t* ts = smem + C::OFF_TS + b * C::TS_BYTES;
       for (int kb = 0; kb < KB; ++kb) {
         // groups of this k-block: 4 (8 for F4); the tail block is [K - KBK, K)
@@ -418,7 +438,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI, ACT>::N
         const int gs = (tail && kb == KB - 1) ? G - GPB : GPB * kb;
         uint32_t w[C::F4 ? 16 : 8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < (C::SFBG ? 0 : 8); ++j) {
           const int c = 32 * j + lane;
 #pragma unroll
           for (int q = 0; q < GPB / 4; ++q) {
@@ -447,8 +467,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI, ACT>::N
 #pragma unroll
           for (int a = 0; a < C::A_ATOMS; ++a)
             tmem_st4(slot + 4 * a, *reinterpret_cast<const uint4*>(sfa + 512 * a + lane * 16));
-          tmem_st4(slot + 4 * C::A_ATOMS, make_uint4(w[0], w[1], w[2], w[3]));
-          tmem_st4(slot + 4 * C::A_ATOMS + 4, make_uint4(w[4], w[5], w[6], w[7]));
+          if (C::SFBG) {
+            const uint8_t* sfb = smem + s * C::STAGE_BYTES + C::OFF_SFB;
+#pragma unroll
+            for (int a = 0; a < C::B_ATOMS; ++a)
+              tmem_st4(slot + 4 * (C::A_ATOMS + a),
+                       *reinterpret_cast<const uint4*>(sfb + 512 * a + lane * 16));
+          } else {
+            tmem_st4(slot + 4 * C::A_ATOMS, make_uint4(w[0], w[1], w[2], w[3]));
+            tmem_st4(slot + 4 * C::A_ATOMS + 4, make_uint4(w[4], w[5], w[6], w[7]));
+          }
           tmem_wait_st();
           tc_fence_before();
         } else {
@@ -472,7 +500,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI, ACT>::N
         if (++s == S) { s = 0; ph ^= 1; }
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar_tsEmpty(b));
+      if (!C::SFBG && lane == 0) mbar_arrive(bar_tsEmpty(b));
     }
   } else if (warp == 1) {
     // ----------------------------------------- UMMA issuer (even CTA) --
@@ -751,6 +779,50 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI, ACT>::N
   }
 }
 
+// Weight-scale atoms of the down GEMM's tiles: for expert e, weight tile nt
+// (B columns c = 0..N-1, output rows nt N + c) and k-block kb, the 1 KB block
+// of two 512-byte atoms the builders store into TMEM: word (c / 32) % 4 of
+// row c % 32 of atom c / 128 holds the scale bytes of the k-block's four
+// groups of 32 (the last block of a K that is not a multiple of 128 takes the
+// last four groups), zero for columns past N or past the output rows. One
+// CTA per (e, nt): the tile's scale rows (one contiguous run) are staged in
+// shared memory with coalesced loads, then each thread forms one word of
+// every k-block's block.
+constexpr int kAtomRowsMax = 224 * (kMxMaxK / 32);
+__global__ void __launch_bounds__(256) pair_weight_atoms_kernel(const uint8_t* __restrict__ scales,
+                                                                int rows, int G, int n_out, int N,
+                                                                int n_tiles, int KB,
+                                                                uint8_t* __restrict__ atoms) {
+  __shared__ __align__(16) uint8_t srows[kAtomRowsMax];
+  pdl_wait_and_trigger();
+  const int e = blockIdx.x / n_tiles, nt = blockIdx.x % n_tiles;
+  const int n0 = nt * N;
+  const int nrows = min(N, n_out - n0);
+  const int bytes = nrows * G;
+  const uint8_t* src = scales + (static_cast<size_t>(e) * rows + n0) * G;
+  if ((reinterpret_cast<uintptr_t>(src) & 15) == 0 && (bytes & 15) == 0) {
+    for (int o = 16 * threadIdx.x; o < bytes; o += 16 * 256)
+      *reinterpret_cast<uint4*>(srows + o) = __ldg(reinterpret_cast<const uint4*>(src + o));
+  } else {
+    for (int o = threadIdx.x; o < bytes; o += 256) srows[o] = src[o];
+  }
+  __syncthreads();
+  const int i = threadIdx.x;
+  const int c = 32 * (4 * (i >> 7) + (i & 3)) + ((i >> 2) & 31);
+  const bool valid = c < nrows;
+  const uint8_t* row = srows + (valid ? c : 0) * G;
+  uint32_t* dst = reinterpret_cast<uint32_t*>(atoms + static_cast<size_t>(blockIdx.x) * KB * 1024) + i;
+  const bool tail = (G % 4) != 0;
+  for (int kb = 0; kb < KB; ++kb) {
+    const int g0 = (tail && kb == KB - 1) ? G - 4 : 4 * kb;
+    uint32_t v = 0;
+    if (valid)
+      v = static_cast<uint32_t>(row[g0]) | (static_cast<uint32_t>(row[g0 + 1]) << 8) |
+          (static_cast<uint32_t>(row[g0 + 2]) << 16) | (static_cast<uint32_t>(row[g0 + 3]) << 24);
+    dst[kb * 256] = v;
+  }
+}
+
 // ----------------------------------------------------------- host side ----
 
 template <int EPI, int ACT>
@@ -824,6 +896,16 @@ cudaError_t launch_pair_impl(const MxGemmProblem& p, int num_sms, cudaStream_t s
   a.topk_w = p.topk_w;
   a.status = p.status;
   a.bias = p.bias;
+  a.wsfb = nullptr;
+  if (C::SFBG) {
+    static_assert(!C::SFBG || C::SFB_BYTES == 1024, "atom block");
+    if (p.wsfb == nullptr || C::N > 224) return cudaErrorInvalidValue;
+    launch_kernel(pair_weight_atoms_kernel, dim3(p.E * a.n_tiles), dim3(256), 0, st, p.scales,
+                  rows, p.K / 32, p.n_out, C::N, a.n_tiles, a.KB, p.wsfb);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    a.wsfb = p.wsfb;
+  }
   const int64_t tiles_bound = (static_cast<int64_t>(p.P) / 256 + p.E) * a.n_tiles;
   int64_t pairs = num_sms / 2;
   if (tiles_bound < pairs) pairs = tiles_bound;
@@ -843,6 +925,11 @@ cudaError_t launch_mx_pair_gateup_swiglu(const MxGemmProblem& p, int num_sms, cu
     case ACT_F4: return launch_pair_impl<PAIR_SWIGLU, ACT_F4>(p, num_sms, st);
   }
   return cudaErrorInvalidValue;
+}
+
+size_t mx_pair_down_atom_bytes(int E, int d, int I) {
+  // tiles of N = 224 output rows, k-blocks of 128 (the 8-bit kinds' down GEMM)
+  return static_cast<size_t>(E) * ((d + 223) / 224) * ((I + 127) / 128) * 1024;
 }
 
 cudaError_t launch_mx_pair_down(const MxGemmProblem& p, int num_sms, cudaStream_t st) {

@@ -130,8 +130,9 @@ def test_workspace_sizes():
     # 12 launches: the router's three (weight split, logits, top-k), three
     # for the permutation (none of its own for at most 256 tokens: the top-k
     # launch builds it), the gather, two scale transposes (none on the
-    # block-scaled tiles), two GEMMs, combine
-    assert B.moe_forward_launch_count(32, 4, 8192, 2880, 2880) == 10
+    # block-scaled tiles), two GEMMs, combine; the CTA-pair tiles add one
+    # (the down weights' scale atoms)
+    assert B.moe_forward_launch_count(32, 4, 8192, 2880, 2880) == 11
     assert B.moe_forward_launch_count(32, 4, 8192, 352, 224) == 12
     assert B.moe_forward_launch_count(32, 4, 100, 2880, 2880) == 7
     assert B.moe_forward_launch_count(32, 4, 100, 352, 2880) == 9
