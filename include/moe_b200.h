@@ -164,8 +164,10 @@ typedef struct {
 /*
  * Bytes of device workspace moe_forward needs for this shape (0 for invalid
  * shapes). The workspace holds the router's logits and top-k, the routing
- * tables, the permuted activations, the SwiGLU hidden rows H [T*k][I] bf16 and
- * the weighted per-slot expert outputs [T*k][d] fp32.
+ * tables, the permuted activations, the SwiGLU hidden rows H [T*k][I] bf16,
+ * the weighted per-slot expert outputs [T*k][d] fp32, and the down weights'
+ * scale factors re-laid out for the CTA-pair tiles (E * ceil(d/224) *
+ * ceil(I/128) KiB).
  */
 MOE_API size_t moe_workspace_size(int E, int k, int T, int d, int I);
 
