@@ -424,7 +424,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PairCfg<EPI, ACT>::N
     // 1), w = 0..3, read from the tile's scale rows (row c of the tile-scale
     // buffer is B column c; 2-byte aligned rows). 8-bit kinds: each builder
     // stores them, after row l of the stage's token scale atoms, into lane l
-    // of its TMEM lane quarter of the stage's slot.
+    // of its TMEM lane quarter of the stage's slot. Down GEMM (SFBG): the
+    // stage brings both weight atoms ready-made, and the builders store row l
+    // of each as it is.
     int s = 0, ph = 0, it = 0;
     bool ok = true;
     for (int tile = pair_id; tile < total && ok; tile += npairs, ++it) {
