@@ -120,6 +120,40 @@ def kernel_source_hash(sources=None) -> str:
     return h.hexdigest()[:16]
 
 
+def quant_tiles(args, inp, T: int):
+    """Tile family of a quantised-activation forward (w4a8, w4a4), as
+    moe_forward_ex picks it: 16-token tiles under 64 rows per expert; the CTA
+    pair when tile policy 5 forces it or, by shape, from 192 rows per expert;
+    else 128-token tiles on one CTA."""
+    P, E = T * inp.k, inp.E
+    if P < 64 * E:
+        return "small"
+    if args.tile_policy == 5 or (args.tile_policy == 0 and P >= 192 * E):
+        return "pair"
+    return "large"
+
+
+def quant_runs_mxf4(args, inp, T: int) -> bool:
+    """w4a4 on the CTA pair runs kind::mxf4 where d and I are at least 256."""
+    return (args.act_quant == "mxfp4" and quant_tiles(args, inp, T) == "pair"
+            and min(inp.d, inp.I) >= 256)
+
+
+def forward_launches(args, inp, T: int) -> int:
+    """Kernel launches of one forward: the library's count for the bf16 path;
+    for the quantised modes router (3), permutation (3; inside the router's
+    top-k launch for at most 256 tokens), the converting gather, the two
+    GEMMs and the combine, plus the down weights' atom pass on the CTA pair
+    with 8-bit activations."""
+    if args.act_quant == "bf16":
+        from sparse_moe_layer_05_b200 import binding as B
+        return B.moe_forward_launch_count(inp.E, inp.k, T, inp.d, inp.I)
+    n = 10 - (3 if T <= 256 else 0)
+    if quant_tiles(args, inp, T) == "pair" and not quant_runs_mxf4(args, inp, T):
+        n += 1
+    return n
+
+
 def recorded_traffic(workload: str, T: int, tile_policy: int = 0, act_quant: str = "bf16"):
     """DRAM bytes per launch of the dominant kernel from the committed ncu
     summary, if it was taken on the current kernel source and in the same
@@ -524,7 +558,7 @@ def run_ours(args, inp, name):
         # pair at the FP4 rate (kind::mxf4): the measured bf16 peak times the
         # nominal dense ratios 2 and 4
         ratio, kname = 1.0, "bf16 rate"
-        if args.act_quant == "mxfp8" or (args.act_quant == "mxfp4" and args.tile_policy != 5):
+        if args.act_quant != "bf16" and not quant_runs_mxf4(args, inp, T):
             ratio, kname = 2.0, "kind::mxf8f6f4, x2 (nominal FP8:BF16)"
         elif args.act_quant == "mxfp4":
             ratio, kname = 4.0, "kind::mxf4, x4 (nominal FP4:BF16)"
@@ -597,8 +631,7 @@ def run_ours(args, inp, name):
         "routing_load": routing_load,
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": int(T * inp.d * 2),
                 "d2h_bytes_per_step": int(T * inp.d * 2), "host_buffers": near.describe()},
-        "gpu_launches": (B.moe_forward_launch_count(inp.E, inp.k, T, inp.d, inp.I)
-                         + (1 if args.block else 0)) * args.steps,
+        "gpu_launches": (forward_launches(args, inp, T) + (1 if args.block else 0)) * args.steps,
         "clocks": clk.summary(),
     }
     line["_topk_idx"] = topk_idx
